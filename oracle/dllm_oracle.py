@@ -1,0 +1,403 @@
+"""Plain fp64 CPU oracle for one block-diffusion denoising step of the LLaDA2.0-Uni MoE dLLM backbone.
+
+TEST INFRASTRUCTURE. Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline / reference leg of
+``bench.py`` may import this module. The library (CUDA kernels behind the C ABI and its Python binding) never
+calls it and shares no code with it.
+
+Every step is its plain definition, in fp64 numpy, in the pages' order. Sources, by page title and section:
+
+  [R] "[논문 리뷰] LLaDA2.0-Uni: Unifying Multimodal Understanding and Generation with Diffusion Large Language
+      Model" (paper review, baba9811.github.io):
+        "Block Diffusion Language Model (BDLM)"  - blocks: bidirectional inside, left-to-right across, earlier
+                                                   blocks always clean context
+        "MoE 백본과 Block-wise Attention"          - MoE backbone, router picks top-k experts per token; block-wise
+                                                   attention pattern
+        "Positional Embedding & 임의 해상도"       - 1D RoPE over the flattened sequence
+        "SPRINT — 학습 없는 추론 가속"              - sparse prefix retention (mean-normalised key norm l~_i,
+                                                   alpha = 0.5, per-modality keep ratios); non-uniform unmasking
+                                                   (accept all c > tau ~ 0.93, at least ceil(m/(T-t)) per step;
+                                                   the standard schedule ceil(m/T)); c_i = max_v p(v | x_t)
+        "BDLM Loss (사전학습)"                     - conditioning on clean x_{0,<k} and noisy x_{t,k}
+        "Load Balancing — Auxiliary-loss-free MoE Bias" - a per-expert bias steers expert load
+  [M] "LLaDA2.0-Uni：基于扩散大型语言模型的多模态理解与生成统一框架" (HF-mirror README, ai.gitcode.com):
+        "SPRINT 加速技术"  - prefix KV computed once in a warm-up and reused; adaptive unmasking with
+                           k = ceil(remaining_masked / steps_left); batch acceptance of all p > threshold;
+                           keep_ratio / cache_warmup_steps knobs
+        usage examples     - block_length=32, steps=8, cfg_scale=2.0 (text-to-image); steps=32,
+                             threshold=0.93, keep_ratio=0.5 (understanding)
+
+Readings where the pages are silent (each also listed in the design notes):
+  * router: sigmoid scores; bias added for selection only; gates = unbiased scores of the chosen experts,
+    renormalised to sum 1; no extra routed scaling; ties -> lower expert id; slots ordered by biased score.
+  * shared expert: same SwiGLU MLP on every token, weight 1.
+  * SwiGLU: down(silu(gate x) * (up x)); fused gate|up weight stores gate rows then up rows.
+  * RMSNorm: x / sqrt(mean(x^2) + eps) * g.
+  * RoPE: rotate-half pairing (i, i + d/2), theta_i = base^(-2i/d), absolute positions.
+  * attention: scale 1/sqrt(d); kv head of q head h is floor(h * Hkv / Hq); key j visible to query i iff
+    floor(pos_j / L) <= floor(pos_i / L).
+  * SPRINT score (formula stripped on the page): key-norm term only, l_i = mean over kv heads of ||K[h, i]||_2,
+    divided by its mean over the prefix; keep ceil(r * P) largest, ties -> lower position; kept set in
+    position order.
+  * threshold rule (formula stripped on the page): k_t = min(m, max(ceil(m / (T_s - t)), min(k_max, #{c > tau}))).
+  * CFG: z = z_u + s (z_c - z_u) computed in float32 (the precision in which the argmax is decided).
+  * confidence c = max softmax at temperature 1 over the scored vocabulary; candidate = lowest argmax.
+  * storage rounding: wherever the library stores a tensor in its storage type (bf16 or fp32) the oracle rounds
+    its fp64 value to that type (round-to-nearest-even) at the same point; between those points it is fp64.
+"""
+import math
+import numpy as np
+
+# --------------------------------------------------------------------------------------------------------------
+# storage rounding
+
+
+def round_bf16(x):
+    """Round fp64 values to the nearest bf16 (8 significant bits, ties to even), returned as fp64."""
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)                       # x = m * 2**e, 0.5 <= |m| < 1
+    return np.ldexp(np.rint(np.ldexp(m, 8)), e - 8)
+
+
+def round_f32(x):
+    return np.asarray(x, dtype=np.float64).astype(np.float32).astype(np.float64)
+
+
+def store(x, dtype):
+    """Value of ``x`` after the library writes it in storage type ``dtype`` ("bf16" or "f32")."""
+    return round_bf16(x) if dtype == "bf16" else round_f32(x)
+
+
+def f64(a):
+    """Exact widening of a numpy array or torch tensor (bf16 / fp32 / int) to fp64 numpy."""
+    if hasattr(a, "detach"):                 # torch tensor: widen through torch (exact), then to numpy
+        import torch
+        return a.detach().to("cpu", torch.float64).numpy()
+    return np.asarray(a, dtype=np.float64)
+
+
+# --------------------------------------------------------------------------------------------------------------
+# per-layer building blocks
+
+
+def rmsnorm(x, g, eps):
+    """RMSNorm over the last axis: x * (mean(x^2) + eps)^(-1/2) * g."""
+    x = f64(x)
+    return x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps) * f64(g)
+
+
+def rope(x, pos, base):
+    """1D rotary embedding [R] "Positional Embedding": x [..., n, heads, d] at absolute positions pos [n].
+
+    Rotate-half pairing: element i pairs with i + d/2, angle pos * base^(-2i/d)."""
+    x = f64(x)
+    d = x.shape[-1]
+    half = d // 2
+    inv = base ** (-2.0 * np.arange(half, dtype=np.float64) / d)
+    ang = np.asarray(pos, dtype=np.float64)[:, None] * inv[None, :]      # [n, half]
+    cos = np.cos(ang)[:, None, :]
+    sin = np.sin(ang)[:, None, :]
+    x1, x2 = x[..., :half], x[..., half:]
+    return np.concatenate([x1 * cos - x2 * sin, x2 * cos + x1 * sin], axis=-1)
+
+
+def block_visible(q_pos, k_pos, blk_len):
+    """[R] "Block Diffusion Language Model (BDLM)": a query sees every key of its own block and of earlier
+    blocks, none of later blocks. Blocks are [j*L, (j+1)*L) from position 0."""
+    qb = np.asarray(q_pos, dtype=np.int64)[:, None] // blk_len
+    kb = np.asarray(k_pos, dtype=np.int64)[None, :] // blk_len
+    return kb <= qb
+
+
+def attention(q, k, v, q_pos, k_pos, blk_len, scale=None):
+    """Block-causal softmax attention for one batch row, two passes with an explicit mask.
+
+    q [Lq, Hq, d], k/v [Nk, Hkv, d], q_pos [Lq], k_pos [Nk] -> o [Lq, Hq, d]."""
+    q, k, v = f64(q), f64(k), f64(v)
+    Lq, Hq, d = q.shape
+    Hkv = k.shape[1]
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    vis = block_visible(q_pos, k_pos, blk_len)
+    o = np.zeros_like(q)
+    for h in range(Hq):
+        g = h * Hkv // Hq
+        s = (q[:, h, :] @ k[:, g, :].T) * scale
+        s = np.where(vis, s, -np.inf)
+        smax = s.max(axis=1, keepdims=True)
+        p = np.exp(s - smax)
+        p = p / p.sum(axis=1, keepdims=True)
+        o[:, h, :] = p @ v[:, g, :]
+    return o
+
+
+def prefix_scores(k_prefix):
+    """[R] "SPRINT" sparse prefix retention, key-norm term: l_i = mean over kv heads of ||K[h, i]||_2,
+    mean-normalised over the prefix. k_prefix [Hkv, P, d] -> l~ [P]."""
+    kk = f64(k_prefix)
+    l = np.sqrt((kk * kk).sum(axis=-1)).mean(axis=0)
+    return l / l.mean()
+
+
+def prefix_retain(k_prefix, ratio):
+    """Kept prefix positions, in position order: the ceil(ratio * P) largest l~_i, ties -> lower position.
+
+    Returns (keep_pos [n_keep] int64, scores [P], margin) where margin is the score gap between the last kept
+    and the first dropped position (inf when nothing is dropped)."""
+    sc = prefix_scores(k_prefix)
+    P = sc.shape[0]
+    n_keep = int(math.ceil(ratio * P))
+    order = sorted(range(P), key=lambda i: (-sc[i], i))
+    keep = np.array(sorted(order[:n_keep]), dtype=np.int64)
+    margin = sc[order[n_keep - 1]] - sc[order[n_keep]] if n_keep < P else np.inf
+    return keep, sc, margin
+
+
+def sigmoid(x):
+    return 1.0 / (1.0 + np.exp(-x))
+
+
+def route(h, w_router, bias, k):
+    """[R] "MoE 백본" top-k router with the aux-loss-free bias of [R] "Load Balancing" used for selection only.
+
+    h [T, H], w_router [E, H], bias [E] -> ids [T, k] (slots in biased-score order), gates [T, k],
+    scores [T, E], margin [T] (biased score of slot k-1 minus the best unchosen biased score)."""
+    s = sigmoid(f64(h) @ f64(w_router).T)
+    b = f64(bias)
+    T, E = s.shape
+    ids = np.zeros((T, k), dtype=np.int64)
+    gates = np.zeros((T, k))
+    margin = np.full(T, np.inf)
+    for t in range(T):
+        biased = s[t] + b
+        order = sorted(range(E), key=lambda e: (-biased[e], e))
+        ids[t] = order[:k]
+        sel = s[t, ids[t]]
+        gates[t] = sel / sel.sum()
+        if k < E:
+            margin[t] = biased[order[k - 1]] - biased[order[k]]
+    return ids, gates, s, margin
+
+
+def silu(x):
+    return x * sigmoid(x)
+
+
+def swiglu_mlp(x, w_gu, w_down, dtype):
+    """down(silu(gate x) * (up x)) for rows x [n, H]; w_gu [2I, H] = [gate; up], w_down [H, I].
+    The activation is stored in ``dtype`` before the down projection."""
+    x = f64(x)
+    w_gu = f64(w_gu)
+    I = w_gu.shape[0] // 2
+    g = x @ w_gu[:I].T
+    u = x @ w_gu[I:].T
+    a = store(silu(g) * u, dtype)
+    return a @ f64(w_down).T
+
+
+def moe_delta(h, ids, gates, w_gu, w_down, w_gu_shared, w_down_shared, dtype):
+    """MoE FFN output before the residual: shared(h_t) + sum_j gates[t, j] * expert_{ids[t, j]}(h_t).
+    A plain per-token loop over the chosen experts (no permutation)."""
+    h = f64(h)
+    T = h.shape[0]
+    out = np.zeros_like(h)
+    for t in range(T):
+        acc = np.zeros(h.shape[1])
+        if w_gu_shared is not None:
+            acc += swiglu_mlp(h[t:t + 1], w_gu_shared, w_down_shared, dtype)[0]
+        for j in range(ids.shape[1]):
+            e = int(ids[t, j])
+            acc += gates[t, j] * swiglu_mlp(h[t:t + 1], w_gu[e], w_down[e], dtype)[0]
+        out[t] = acc
+    return out
+
+
+# --------------------------------------------------------------------------------------------------------------
+# confidence and unmasking
+
+
+def cfg_combine_f32(zc, zu, scale):
+    """Classifier-free guidance z = z_u + s (z_c - z_u), each operation rounded to float32 in this order
+    (subtract, multiply, add)."""
+    zc = np.asarray(f64(zc), dtype=np.float32)
+    zu = np.asarray(f64(zu), dtype=np.float32)
+    diff = (zc - zu).astype(np.float32)
+    prod = (np.float32(scale) * diff).astype(np.float32)
+    return (zu + prod).astype(np.float32).astype(np.float64)
+
+
+def confidence(z):
+    """[R] "SPRINT": c = max_v softmax(z)_v, the candidate token is the lowest argmax.
+    z [n, V] -> (cand [n] int64, c [n], lse [n], zmax [n])."""
+    z = f64(z)
+    zmax = z.max(axis=1)
+    cand = z.argmax(axis=1)                  # numpy returns the first (lowest) index of the maximum
+    lse = zmax + np.log(np.exp(z - zmax[:, None]).sum(axis=1))
+    return cand.astype(np.int64), np.exp(zmax - lse), lse, zmax
+
+
+def unmask_count(m, t, T_s, mode, tau=None, k_max=None, conf_masked=None):
+    """Positions to unmask at step t (0-based) of T_s with m still masked.
+
+    fixed ([M] "SPRINT 加速技术", [R] standard schedule): ceil(m / (T_s - t)).
+    threshold ([R] "SPRINT" non-uniform unmasking, [M] batch acceptance): every c > tau, capped at k_max, and
+    never fewer than ceil(m / (T_s - t)); never more than m."""
+    if m == 0:
+        return 0
+    floor_k = -(-m // (T_s - t))
+    if mode == 0:
+        return min(m, floor_k)
+    above = int(np.sum(np.asarray(conf_masked) > tau))
+    return min(m, max(floor_k, min(k_max, above)))
+
+
+def select_positions(conf_row, masked_row, k):
+    """The k masked positions of one block row with the highest confidence, ties -> lower position.
+    Returns (chosen positions in rank order, margin between rank k-1 and rank k, or inf)."""
+    pos = [i for i in range(len(masked_row)) if masked_row[i]]
+    order = sorted(pos, key=lambda i: (-conf_row[i], i))
+    margin = conf_row[order[k - 1]] - conf_row[order[k]] if 0 < k < len(order) else np.inf
+    return order[:k], margin
+
+
+def unmask(z_rows, row_pos, tokens, mask, t, T_s, mode=0, tau=0.9, k_max=8, vocab_offset=0,
+           z_uncond=None, cfg_scale=1.0):
+    """One unmasking step over a batch of block rows.
+
+    z_rows [n, V]: logits of the still-masked positions, row r belongs to flat position row_pos[r] = b*L + i of
+    the conditional rows. With ``z_uncond`` given, the rows are combined by CFG first, and the selection is
+    written to both halves of the batch (rows b and b + B/2).
+    Returns dict(tokens, mask, sel [Bl, k], nsel [Bl], conf [Bl, L], cand [Bl, L], tie_rank [Bl],
+    tie_tau [Bl]) where Bl is the number of logical rows."""
+    tokens = np.array(tokens, dtype=np.int64, copy=True)
+    mask = np.array(mask, dtype=np.int64, copy=True)
+    B, L = mask.shape
+    Bl = B // 2 if z_uncond is not None else B
+    z = cfg_combine_f32(z_rows, z_uncond, cfg_scale) if z_uncond is not None else f64(z_rows)
+    cand_r, conf_r, _, _ = confidence(z)
+    conf = np.zeros((Bl, L))
+    cand = np.full((Bl, L), -1, dtype=np.int64)
+    for r, p in enumerate(row_pos):
+        b, i = divmod(int(p), L)
+        conf[b, i] = conf_r[r]
+        cand[b, i] = cand_r[r] + vocab_offset
+    sel, nsel = [], np.zeros(Bl, dtype=np.int64)
+    tie_rank = np.zeros(Bl, dtype=bool)
+    tie_tau = np.zeros(Bl, dtype=bool)
+    for b in range(Bl):
+        masked = mask[b].astype(bool)
+        m = int(masked.sum())
+        cm = conf[b][masked]
+        kt = unmask_count(m, t, T_s, mode, tau, k_max, cm)
+        chosen, margin = select_positions(conf[b], masked, kt)
+        tie_rank[b] = margin < 1e-6 * max(conf[b].max(), 1e-30)
+        if mode == 1 and m:
+            tie_tau[b] = bool(np.any(np.abs(cm - tau) < 1e-6))
+        for i in chosen:
+            tokens[b, i] = cand[b, i]
+            mask[b, i] = 0
+            if z_uncond is not None:
+                tokens[b + Bl, i] = cand[b, i]
+                mask[b + Bl, i] = 0
+        sel.append(chosen)
+        nsel[b] = kt
+    return dict(tokens=tokens, mask=mask, sel=sel, nsel=nsel, conf=conf, cand=cand,
+                tie_rank=tie_rank, tie_tau=tie_tau)
+
+
+# --------------------------------------------------------------------------------------------------------------
+# the denoising pass
+
+
+def _layer_kv(h_rows, lw, w, pos):
+    """q/k/v of rows h_rows [n, H] at positions pos: GEMM, RoPE on q and k, storage rounding."""
+    qkv = f64(h_rows) @ f64(lw["w_qkv"]).T
+    Hq, Hkv, d = w.Hq, w.Hkv, w.d
+    n = qkv.shape[0]
+    q = qkv[:, : Hq * d].reshape(n, Hq, d)
+    k = qkv[:, Hq * d: (Hq + Hkv) * d].reshape(n, Hkv, d)
+    v = qkv[:, (Hq + Hkv) * d:].reshape(n, Hkv, d)
+    q = store(rope(q, pos, w.rope_base), w.dtype)
+    k = store(rope(k, pos, w.rope_base), w.dtype)
+    v = store(v, w.dtype)
+    return q, k, v
+
+
+def forward_block(w, weights, caches, tokens, mask, keep=None, want_logits=True, skip_last_ffn=False):
+    """The backbone over one block for every batch row.
+
+    w: workload (dims, dtype, eps, rope_base, blk len L, prefix length P); weights: dict from the synthetic
+    generator (torch or numpy arrays); caches: per layer (K, V) [B, Hkv, >=P, d]; tokens/mask [B, L].
+    keep: per layer, per row, array of kept prefix positions (SPRINT) or None for the full prefix.
+    Returns dict(x [B, L, H] final hidden before the final norm, block_k / block_v per layer [B, L, Hkv, d],
+    route per layer (ids, gates, margin), logits [n_m, vlen] for the masked rows, row_pos [n_m])."""
+    B, L, P, H = w.B, w.L, w.P, w.H
+    dt = w.dtype
+    tok = np.where(np.asarray(mask).astype(bool), w.mask_id, np.asarray(tokens))
+    emb = weights["embed"]
+    x = np.stack([f64(emb[int(i)]) for i in tok.reshape(-1)]).reshape(B * L, H)     # exact copy of the rows
+    pos = np.arange(P, P + L)
+    out = dict(block_k=[], block_v=[], route=[])
+    n_layers = len(weights["layers"])
+    for li, lw in enumerate(weights["layers"]):
+        kc, vc = f64(caches[li][0]), f64(caches[li][1])
+        h = store(rmsnorm(x, lw["attn_norm"], w.eps), dt)
+        o = np.zeros((B, L, w.Hq, w.d))
+        bk = np.zeros((B, L, w.Hkv, w.d))
+        bv = np.zeros((B, L, w.Hkv, w.d))
+        for b in range(B):
+            q, k, v = _layer_kv(h[b * L:(b + 1) * L], lw, w, pos)
+            bk[b], bv[b] = k, v
+            kp = np.arange(P) if keep is None else np.asarray(keep[li][b])
+            keys = np.concatenate([kc[b][:, kp, :].transpose(1, 0, 2), k], axis=0)
+            vals = np.concatenate([vc[b][:, kp, :].transpose(1, 0, 2), v], axis=0)
+            kpos = np.concatenate([kp, pos])
+            o[b] = store(attention(q, keys, vals, pos, kpos, L), dt)
+        out["block_k"].append(bk)
+        out["block_v"].append(bv)
+        x = store(x + o.reshape(B * L, -1) @ f64(lw["w_o"]).T, dt)
+        if skip_last_ffn and li == n_layers - 1:
+            out["route"].append(None)
+            break
+        h2 = store(rmsnorm(x, lw["ffn_norm"], w.eps), dt)
+        ids, gates, _, margin = route(h2, lw["w_router"], lw["router_bias"], w.k)
+        out["route"].append((ids, gates, margin))
+        delta = moe_delta(h2, ids, gates, lw["w_gu"], lw["w_down"], lw["w_gu_shared"], lw["w_down_shared"], dt)
+        x = store(x + delta, dt)
+    out["x"] = x.reshape(B, L, H)
+    if want_logits:
+        xf = store(rmsnorm(x, weights["final_norm"], w.eps), dt)
+        Bl = B // 2 if w.cfg else B
+        row_pos = np.nonzero(np.asarray(mask)[:Bl].reshape(-1))[0]
+        rows = list(row_pos) + ([p + Bl * L for p in row_pos] if w.cfg else [])
+        wl = f64(weights["w_lm"][w.vocab_offset: w.vocab_offset + w.vlen])
+        out["logits"] = store(xf[rows] @ wl.T, dt)
+        out["row_pos"] = row_pos
+    return out
+
+
+def denoise_step(w, weights, caches, tokens, mask, t, keep=None):
+    """One denoising pass at step t: backbone, LM head over the masked rows, confidence, unmasking."""
+    f = forward_block(w, weights, caches, tokens, mask, keep=keep)
+    n = len(f["row_pos"])
+    zc, zu = (f["logits"][:n], f["logits"][n:]) if w.cfg else (f["logits"], None)
+    u = unmask(zc, f["row_pos"], tokens, mask, t, w.T_s, w.mode, w.tau, w.k_max, w.vocab_offset,
+               z_uncond=zu, cfg_scale=w.cfg_scale)
+    u["forward"] = f
+    return u
+
+
+def commit_block(w, weights, caches, tokens, keep=None):
+    """Pass over the finished block's clean tokens ([R] BDLM: earlier blocks are always clean context): each
+    layer's block K/V [B, L, Hkv, d] for cache rows [P, P + L). The last layer's FFN and the LM head have no
+    consumer and are skipped."""
+    mask = np.zeros_like(np.asarray(tokens))
+    f = forward_block(w, weights, caches, tokens, mask, keep=keep, want_logits=False, skip_last_ffn=True)
+    return f["block_k"], f["block_v"]
+
+
+def sprint_keep(w, caches):
+    """SPRINT selection at the first step of a block: per layer, per row, kept prefix positions."""
+    keep = []
+    for li in range(len(caches)):
+        kc = f64(caches[li][0])
+        keep.append([prefix_retain(kc[b][:, : w.P, :], w.keep_ratio)[0] for b in range(w.B)])
+    return keep

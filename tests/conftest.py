@@ -1,0 +1,19 @@
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+
+def pytest_configure(config):
+    config.addinivalue_line("markers", "gpu: needs a B200 and the built CUDA library")
+
+
+@pytest.fixture(scope="session")
+def lib():
+    """The C-ABI library through its binding; GPU tests only."""
+    from block_diffusion_moe_dllm_b200 import binding
+    return binding.load()

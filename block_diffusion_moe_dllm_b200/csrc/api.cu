@@ -1,0 +1,553 @@
+// C-ABI entry points: argument validation, workspace carving and the composition of one denoising pass.
+// Every entry point validates before launching; nothing is launched on error. No entry point allocates device
+// memory or synchronises, except dllm_status_check, which reads the workspace status word.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <cmath>
+#include "common.cuh"
+#include "kernels.h"
+#include "misc.h"
+
+#include <atomic>
+
+namespace dllm_host {
+static thread_local char g_err[512] = "";
+static std::atomic<unsigned long long> g_launches{0};
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+void set_error(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+}
+int cuda_status(cudaError_t e, const char* what) {
+  set_error("%s: %s", what, cudaGetErrorString(e));
+  return DLLM_ERR_CUDA;
+}
+}  // namespace dllm_host
+
+using namespace dllm;
+
+namespace {
+
+constexpr size_t kStatusBytes = 256;
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+inline int esize(int dtype) { return dtype == DLLM_BF16 ? 2 : 4; }
+inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+// Bump carver over a caller workspace (base == nullptr only measures).
+struct Carver {
+  char* base;
+  size_t off = kStatusBytes;
+  explicit Carver(void* b) : base(static_cast<char*>(b)) {}
+  template <typename T = void>
+  T* take(size_t bytes) {
+    off = align256(off);
+    T* p = base ? reinterpret_cast<T*>(base + off) : nullptr;
+    off += bytes;
+    return p;
+  }
+};
+
+#define REQ(cond, code, ...) DLLM_REQUIRE(cond, code, __VA_ARGS__)
+
+int check_ws(void* ws, size_t ws_bytes, size_t need) {
+  REQ(ws != nullptr, DLLM_ERR_WORKSPACE, "workspace is NULL");
+  REQ(((uintptr_t)ws & 255u) == 0, DLLM_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  REQ(ws_bytes >= need, DLLM_ERR_WORKSPACE, "workspace too small: %zu bytes given, %zu needed", ws_bytes, need);
+  return DLLM_OK;
+}
+
+int32_t* status_word(void* ws) { return static_cast<int32_t*>(ws); }
+
+// ------------------------------------------------------------------------------------------------ GEMM dispatch
+int run_gemm(GemmArgs& a, cudaStream_t s) {
+  return a.dtype == DLLM_BF16 ? gemm_bf16_tc(a, s) : gemm_f32_simt(a, s);
+}
+
+// ------------------------------------------------------------------------------------------------ experts
+struct ExpertBufs {
+  void* xp;
+  void* act;
+  float* y;
+  float* scratch;
+};
+
+void carve_experts(Carver& c, int dtype, int Tk, int H, int k, int I, int shared, ExpertBufs& b) {
+  const int64_t rows = (int64_t)Tk * k + (shared ? Tk : 0);
+  b.xp = c.take(rows * H * esize(dtype));
+  b.act = c.take(rows * I * esize(dtype));
+  b.y = c.take<float>(rows * H * 4);
+  b.scratch = dtype == DLLM_F32 ? c.take<float>(gemm_f32_scratch_bytes(rows, std::max(2 * I, H), 0)) : nullptr;
+}
+
+int expert_bn_hint(int Tk, int k, int E) {
+  const int avg = (Tk * k + E - 1) / E;
+  return std::min(Tk, std::max(64, 4 * avg));
+}
+
+int run_experts(int dtype, int Tk, int H, int E, int k, int I, const void* h, const void* w_gu, const void* w_down,
+                const void* w_gu_s, const void* w_down_s, const int32_t* counts, const int32_t* offsets,
+                const int32_t* perm, const int32_t* inv, const float* gates, void* x, const ExpertBufs& b,
+                int32_t* status, cudaStream_t s) {
+  const int shared = w_gu_s != nullptr;
+  const int n_assign = Tk * k;
+  const int64_t rows = (int64_t)n_assign + (shared ? Tk : 0);
+  int st = launch_gather_rows(dtype, h, perm, k, Tk, shared, b.xp, H, s);
+  if (st) return st;
+  GemmArgs g1;
+  g1.x = b.xp; g1.x_rows = rows;
+  g1.w = w_gu; g1.w_rows = (int64_t)E * 2 * I;
+  g1.w2 = w_gu_s; g1.w2_rows = 2 * I;
+  g1.K = H; g1.M = I; g1.swiglu = 1; g1.w_group_stride = 2 * I;
+  g1.n_dev = E; g1.grp_off = offsets; g1.grp_cnt = counts;
+  g1.has_extra = shared; g1.extra_off = n_assign; g1.extra_cnt = Tk;
+  g1.max_cnt = expert_bn_hint(Tk, k, E); g1.cnt_bound = Tk;
+  g1.dtype = dtype; g1.status = status; g1.f32_scratch = b.scratch;
+  g1.epi.kind = EPI_SWIGLU; g1.epi.out = b.act; g1.epi.ldo = I;
+  st = run_gemm(g1, s);
+  if (st) return st;
+  GemmArgs g2 = g1;
+  g2.x = b.act; g2.K = I; g2.M = H; g2.swiglu = 0;
+  g2.w = w_down; g2.w_rows = (int64_t)E * H; g2.w2 = w_down_s; g2.w2_rows = H; g2.w_group_stride = H;
+  g2.epi = EpiParams();
+  g2.epi.kind = EPI_STORE; g2.epi.out = b.y; g2.epi.ldo = H; g2.epi.out_f32 = 1;
+  st = run_gemm(g2, s);
+  if (st) return st;
+  return launch_combine(dtype, x, b.y, gates, inv, k, Tk, shared, H, s);
+}
+
+// ------------------------------------------------------------------------------------------------ step plan
+struct StepPlan {
+  int B, L, Bl, halves, Tk, vlen, n_keys, max_rows, n_chunks;
+  void* x;
+  void* h;
+  void* q;
+  void* ao;
+  void* attn_ws;
+  size_t attn_ws_bytes;
+  float* scores;
+  int32_t* ids;
+  float* gates;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* perm;
+  int32_t* inv;
+  ExpertBufs eb;
+  float* proj_scratch;
+  int32_t* row_pos;
+  int32_t* n_rows;
+  void* xf;
+  void* logits;
+  void* partials;
+  float* retain_raw;
+  size_t total;
+};
+
+int validate_step(const dllm_model* m, const dllm_state* st, const dllm_step_params* p) {
+  REQ(m && st && p, DLLM_ERR_INVALID_ARG, "denoise_step: NULL descriptor");
+  REQ(m->dtype == DLLM_BF16 || m->dtype == DLLM_F32, DLLM_ERR_INVALID_ARG, "denoise_step: bad dtype %d", m->dtype);
+  REQ(m->n_layers >= 1 && m->layers, DLLM_ERR_INVALID_ARG, "denoise_step: no layers");
+  REQ(m->H > 0 && m->Hq > 0 && m->Hkv > 0 && m->d > 0 && m->E > 0 && m->k > 0 && m->I > 0 && m->V > 0,
+      DLLM_ERR_SHAPE, "denoise_step: non-positive model dimension");
+  REQ(m->Hq % m->Hkv == 0, DLLM_ERR_SHAPE, "denoise_step: Hq %% Hkv != 0");
+  REQ(m->k <= m->E && m->k <= 32 && m->E <= 1024, DLLM_ERR_UNSUPPORTED, "denoise_step: k/E out of range");
+  REQ(m->H % 8 == 0, DLLM_ERR_SHAPE, "denoise_step: H must be a multiple of 8");
+  REQ(st->B >= 1 && st->L >= 1 && st->L <= 32 && st->P >= 0, DLLM_ERR_SHAPE, "denoise_step: bad B/L/P");
+  REQ(st->cap >= st->P + st->L, DLLM_ERR_SHAPE, "denoise_step: cap %d < P + L", st->cap);
+  REQ(st->tokens && st->mask, DLLM_ERR_INVALID_ARG, "denoise_step: NULL tokens/mask");
+  REQ(m->embed && m->final_norm && m->w_lm, DLLM_ERR_INVALID_ARG, "denoise_step: NULL embed/final_norm/w_lm");
+  REQ(p->T_s >= 1 && p->t >= 0 && p->t < p->T_s, DLLM_ERR_INVALID_ARG, "denoise_step: step %d of %d", p->t, p->T_s);
+  REQ(p->mode == DLLM_UNMASK_FIXED || p->mode == DLLM_UNMASK_THRESHOLD, DLLM_ERR_INVALID_ARG, "bad unmask mode");
+  REQ(!p->cfg || st->B % 2 == 0, DLLM_ERR_SHAPE, "denoise_step: cfg needs an even number of rows");
+  const int vlen = p->vocab_len ? p->vocab_len : m->V;
+  REQ(p->vocab_offset >= 0 && p->vocab_offset + vlen <= m->V, DLLM_ERR_SHAPE, "denoise_step: vocab slice out of range");
+  if (p->sprint) {
+    REQ(p->n_keep >= 1 && p->n_keep <= st->P && p->n_keep <= 8192, DLLM_ERR_SHAPE, "denoise_step: bad n_keep");
+    REQ(st->cap_thin >= p->n_keep + st->L, DLLM_ERR_SHAPE, "denoise_step: cap_thin too small");
+    REQ(st->P <= 8192, DLLM_ERR_UNSUPPORTED, "denoise_step: SPRINT needs P <= 8192");
+  }
+  if (!p->commit) REQ(p->sel && p->nsel && p->conf && p->remaining, DLLM_ERR_INVALID_ARG, "denoise_step: NULL outputs");
+  for (int l = 0; l < m->n_layers; ++l) {
+    const dllm_layer& L = m->layers[l];
+    REQ(L.attn_norm && L.w_qkv && L.w_o && L.ffn_norm && L.w_router && L.router_bias && L.w_gu && L.w_down &&
+            L.k_cache && L.v_cache,
+        DLLM_ERR_INVALID_ARG, "denoise_step: layer %d has a NULL weight or cache", l);
+    REQ((L.w_gu_shared == nullptr) == (L.w_down_shared == nullptr), DLLM_ERR_INVALID_ARG,
+        "denoise_step: layer %d: shared expert weights must both be set or both NULL", l);
+    if (p->sprint) REQ(L.k_thin && L.v_thin && L.keep_pos, DLLM_ERR_INVALID_ARG, "layer %d: NULL thinned cache", l);
+    if (m->dtype == DLLM_BF16)
+      REQ(aligned16(L.w_qkv) && aligned16(L.w_o) && aligned16(L.w_gu) && aligned16(L.w_down), DLLM_ERR_ALIGN,
+          "layer %d: weights must be 16-byte aligned", l);
+  }
+  if (m->dtype == DLLM_BF16) {
+    REQ(m->d == 128, DLLM_ERR_UNSUPPORTED, "denoise_step: bf16 path needs head dim 128");
+    REQ(m->H % 128 == 0 && m->I % 64 == 0, DLLM_ERR_UNSUPPORTED, "denoise_step: bf16 path needs H %% 128 == 0, I %% 64 == 0");
+    REQ(vlen % 128 == 0, DLLM_ERR_UNSUPPORTED, "denoise_step: scored vocabulary must be a multiple of 128");
+    REQ(aligned16(m->w_lm) && aligned16(m->embed), DLLM_ERR_ALIGN, "denoise_step: LM head / embedding alignment");
+  } else {
+    REQ(m->d <= 128 && m->d % 4 == 0, DLLM_ERR_UNSUPPORTED, "denoise_step: fp32 path needs d <= 128, d %% 4 == 0");
+  }
+  return DLLM_OK;
+}
+
+void plan_step(const dllm_model* m, const dllm_state* st, const dllm_step_params* p, void* ws, StepPlan& s) {
+  Carver c(ws);
+  const int es = esize(m->dtype);
+  s.B = st->B;
+  s.L = st->L;
+  s.halves = p->cfg ? 2 : 1;
+  s.Bl = st->B / s.halves;
+  s.Tk = st->B * st->L;
+  s.vlen = p->vocab_len ? p->vocab_len : m->V;
+  s.n_keys = p->sprint ? p->n_keep + st->L : st->P + st->L;
+  s.max_rows = s.Bl * st->L;
+  s.n_chunks = unmask_chunks(s.max_rows, s.vlen);
+  const int H = m->H, QD = m->Hq * m->d;
+  s.x = c.take((size_t)s.Tk * H * es);
+  s.h = c.take((size_t)s.Tk * H * es);
+  s.q = c.take((size_t)s.Tk * QD * es);
+  s.ao = c.take((size_t)s.Tk * QD * es);
+  s.attn_ws_bytes = attn_workspace_bytes(st->B, st->L, m->Hq, m->Hkv, m->d, s.n_keys);
+  s.attn_ws = c.take(s.attn_ws_bytes);
+  s.scores = c.take<float>((size_t)s.Tk * m->E * 4);
+  s.ids = c.take<int32_t>((size_t)s.Tk * m->k * 4);
+  s.gates = c.take<float>((size_t)s.Tk * m->k * 4);
+  s.counts = c.take<int32_t>((size_t)(m->E + 1) * 4);
+  s.offsets = c.take<int32_t>((size_t)(m->E + 1) * 4);
+  s.perm = c.take<int32_t>((size_t)s.Tk * m->k * 4);
+  s.inv = c.take<int32_t>((size_t)s.Tk * m->k * 4);
+  carve_experts(c, m->dtype, s.Tk, H, m->k, m->I, 1, s.eb);
+  const int proj_n = (m->Hq + 2 * m->Hkv) * m->d;
+  s.proj_scratch = m->dtype == DLLM_F32
+                       ? c.take<float>((size_t)std::max(s.Tk, s.halves * s.max_rows) *
+                                       std::max(std::max(proj_n, H), s.vlen) * 4)
+                       : nullptr;
+  s.row_pos = c.take<int32_t>((size_t)s.max_rows * 4);
+  s.n_rows = c.take<int32_t>(16);
+  s.xf = c.take((size_t)s.halves * s.max_rows * H * es);
+  s.logits = c.take((size_t)s.halves * s.max_rows * s.vlen * es);
+  s.partials = c.take(unmask_partials_bytes(s.max_rows, s.n_chunks));
+  s.retain_raw = p->sprint ? c.take<float>(retain_workspace_bytes(st->B, st->P)) : nullptr;
+  s.total = align256(c.off);
+}
+
+}  // namespace
+
+// ================================================================================================== ABI
+extern "C" {
+
+const char* dllm_version(void) { return "dllm-b200 0.1 (sm_100a)"; }
+const char* dllm_last_error(void) { return dllm_host::g_err; }
+unsigned long long dllm_launch_count(void) { return dllm_host::g_launches.load(std::memory_order_relaxed); }
+
+int dllm_status_check(void* ws, cudaStream_t stream) {
+  REQ(ws != nullptr, DLLM_ERR_WORKSPACE, "status_check: NULL workspace");
+  int32_t h = 0;
+  cudaError_t e = cudaMemcpyAsync(&h, ws, sizeof(int32_t), cudaMemcpyDeviceToHost, stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return dllm_host::cuda_status(e, "status_check");
+  if (h != 0) {
+    int32_t zero = 0;
+    cudaMemcpyAsync(ws, &zero, sizeof(int32_t), cudaMemcpyHostToDevice, stream);
+    cudaStreamSynchronize(stream);
+    dllm_host::set_error("a kernel gave up on a bounded wait (code %d)", h);
+    return DLLM_ERR_TIMEOUT;
+  }
+  return DLLM_OK;
+}
+
+// ------------------------------------------------------------------------------------------------ dense GEMM
+size_t dllm_gemm_workspace_size(const dllm_gemm_desc* d) {
+  if (!d) return 0;
+  size_t n = kStatusBytes;
+  if (d->dtype == DLLM_F32) n = align256(n) + gemm_f32_scratch_bytes(d->N, d->M, 0);
+  return align256(n);
+}
+
+int dllm_gemm(const dllm_gemm_desc* d, const void* x, const void* w, void* y, const int32_t* n_rows_dev, void* ws,
+              size_t ws_bytes, cudaStream_t stream) {
+  REQ(d && x && w && y, DLLM_ERR_INVALID_ARG, "gemm: NULL argument");
+  REQ(d->N >= 0 && d->M > 0 && d->K > 0 && d->ldy >= d->M, DLLM_ERR_SHAPE, "gemm: bad N/M/K/ldy");
+  REQ(d->dtype == DLLM_BF16 || d->dtype == DLLM_F32, DLLM_ERR_INVALID_ARG, "gemm: bad dtype");
+  int st = check_ws(ws, ws_bytes, dllm_gemm_workspace_size(d));
+  if (st) return st;
+  if (d->N == 0) return DLLM_OK;
+  if (d->dtype == DLLM_BF16) {
+    REQ(d->K % 64 == 0 && d->M % 128 == 0, DLLM_ERR_UNSUPPORTED, "gemm: bf16 needs K %% 64 == 0 and M %% 128 == 0");
+    REQ(aligned16(x) && aligned16(w), DLLM_ERR_ALIGN, "gemm: X and W must be 16-byte aligned");
+  }
+  Carver c(ws);
+  GemmArgs a;
+  a.x = x; a.x_rows = d->N; a.w = w; a.w_rows = d->M; a.K = d->K; a.M = d->M;
+  a.cnt_dev = n_rows_dev; a.host_cnt = d->N; a.max_cnt = d->N; a.cnt_bound = d->N;
+  a.dtype = d->dtype; a.status = status_word(ws);
+  a.f32_scratch = d->dtype == DLLM_F32 ? c.take<float>(gemm_f32_scratch_bytes(d->N, d->M, 0)) : nullptr;
+  a.epi.kind = d->residual ? EPI_RESID : EPI_STORE;
+  a.epi.out = y; a.epi.ldo = d->ldy; a.epi.out_f32 = d->y_f32 || d->dtype == DLLM_F32;
+  return run_gemm(a, stream);
+}
+
+// ------------------------------------------------------------------------------------------------ attention
+size_t dllm_block_attn_workspace_size(const dllm_attn_desc* d) {
+  if (!d) return 0;
+  return align256(align256(kStatusBytes) + attn_workspace_bytes(d->B, d->Lq, d->Hq, d->Hkv, d->d, d->n_keys));
+}
+
+int dllm_block_attn(const dllm_attn_desc* d, const void* q, const void* k_cache, const void* v_cache,
+                    const int32_t* key_pos, void* out, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  REQ(d && q && k_cache && v_cache && out, DLLM_ERR_INVALID_ARG, "block_attn: NULL argument");
+  REQ(d->B >= 1 && d->Lq >= 1 && d->Hq >= 1 && d->Hkv >= 1 && d->d >= 1 && d->blk_len >= 1 && d->n_keys >= 1 &&
+          d->q_pos0 >= 0,
+      DLLM_ERR_SHAPE, "block_attn: non-positive dimension");
+  REQ(d->Hq % d->Hkv == 0 && d->Hq / d->Hkv <= 64, DLLM_ERR_SHAPE, "block_attn: Hq must be a multiple of Hkv (group <= 64)");
+  REQ(d->cap >= d->n_keys, DLLM_ERR_SHAPE, "block_attn: cap < n_keys");
+  REQ(d->dtype == DLLM_BF16 || d->dtype == DLLM_F32, DLLM_ERR_INVALID_ARG, "block_attn: bad dtype");
+  REQ(d->dtype == DLLM_BF16 ? d->d == 128 : (d->d <= 128 && d->d % 4 == 0), DLLM_ERR_UNSUPPORTED,
+      "block_attn: unsupported head dim %d", d->d);
+  int st = check_ws(ws, ws_bytes, dllm_block_attn_workspace_size(d));
+  if (st) return st;
+  Carver c(ws);
+  AttnArgs a;
+  a.B = d->B; a.Lq = d->Lq; a.Hq = d->Hq; a.Hkv = d->Hkv; a.d = d->d; a.blk_len = d->blk_len; a.q_pos0 = d->q_pos0;
+  a.n_keys = d->n_keys; a.cap = d->cap; a.dtype = d->dtype; a.scale = d->scale;
+  a.q = q; a.k = k_cache; a.v = v_cache; a.key_pos = key_pos; a.out = out;
+  a.ws_bytes = attn_workspace_bytes(d->B, d->Lq, d->Hq, d->Hkv, d->d, d->n_keys);
+  a.ws = c.take(a.ws_bytes);
+  return launch_attn(a, stream);
+}
+
+// ------------------------------------------------------------------------------------------------ SPRINT
+size_t dllm_prefix_retain_workspace_size(const dllm_retain_desc* d) {
+  if (!d) return 0;
+  return align256(align256(kStatusBytes) + retain_workspace_bytes(d->B, d->P));
+}
+
+int dllm_prefix_retain(const dllm_retain_desc* d, const void* k_cache, const void* v_cache, int32_t* keep_pos,
+                       void* k_thin, void* v_thin, float* scores, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  REQ(d && k_cache && v_cache && keep_pos && k_thin && v_thin, DLLM_ERR_INVALID_ARG, "prefix_retain: NULL argument");
+  REQ(d->B >= 1 && d->Hkv >= 1 && d->d >= 1 && d->P >= 1 && d->cap >= d->P, DLLM_ERR_SHAPE, "prefix_retain: bad shape");
+  REQ(d->n_keep >= 1 && d->n_keep <= d->P && d->n_keep <= d->cap_thin, DLLM_ERR_SHAPE, "prefix_retain: bad n_keep");
+  REQ(d->P <= 8192, DLLM_ERR_UNSUPPORTED, "prefix_retain: P > 8192");
+  REQ(d->dtype == DLLM_BF16 || d->dtype == DLLM_F32, DLLM_ERR_INVALID_ARG, "prefix_retain: bad dtype");
+  REQ((d->d * esize(d->dtype)) % 16 == 0, DLLM_ERR_UNSUPPORTED, "prefix_retain: row bytes must be a multiple of 16");
+  int st = check_ws(ws, ws_bytes, dllm_prefix_retain_workspace_size(d));
+  if (st) return st;
+  Carver c(ws);
+  RetainArgs a;
+  a.B = d->B; a.Hkv = d->Hkv; a.d = d->d; a.P = d->P; a.cap = d->cap; a.n_keep = d->n_keep; a.cap_thin = d->cap_thin;
+  a.dtype = d->dtype; a.k = k_cache; a.v = v_cache; a.keep_pos = keep_pos; a.k_thin = k_thin; a.v_thin = v_thin;
+  a.scores = scores; a.raw = c.take<float>(retain_workspace_bytes(d->B, d->P)); a.block_len = 0;
+  return launch_retain(a, stream);
+}
+
+// ------------------------------------------------------------------------------------------------ router
+size_t dllm_moe_route_workspace_size(const dllm_route_desc* d) {
+  if (!d) return 0;
+  return align256(align256(kStatusBytes) + (size_t)d->Tk * d->E * 4);
+}
+
+int dllm_moe_route(const dllm_route_desc* d, const void* h, const void* w_router, const float* bias, int32_t* ids,
+                   float* gates, int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv, float* scores,
+                   void* ws, size_t ws_bytes, cudaStream_t stream) {
+  REQ(d && h && w_router && bias && ids && gates && counts && offsets && perm && inv, DLLM_ERR_INVALID_ARG,
+      "moe_route: NULL argument");
+  REQ(d->Tk >= 0 && d->H > 0 && d->E >= 1 && d->k >= 1, DLLM_ERR_SHAPE, "moe_route: bad shape");
+  REQ(d->E <= 1024 && d->k <= 32 && d->k <= d->E, DLLM_ERR_UNSUPPORTED, "moe_route: needs E <= 1024, k <= min(32, E)");
+  REQ(d->H % 8 == 0, DLLM_ERR_SHAPE, "moe_route: H must be a multiple of 8");
+  REQ(d->H * 32 <= 200 * 1024 / 1, DLLM_ERR_UNSUPPORTED, "moe_route: H too large");
+  REQ(d->dtype == DLLM_BF16 || d->dtype == DLLM_F32, DLLM_ERR_INVALID_ARG, "moe_route: bad dtype");
+  REQ(aligned16(h) && aligned16(w_router), DLLM_ERR_ALIGN, "moe_route: h and w_router must be 16-byte aligned");
+  int st = check_ws(ws, ws_bytes, dllm_moe_route_workspace_size(d));
+  if (st) return st;
+  Carver c(ws);
+  float* sc = scores ? scores : c.take<float>((size_t)d->Tk * d->E * 4);
+  return launch_route(d->dtype, h, w_router, bias, d->Tk, d->H, d->E, d->k, ids, gates, sc, counts, offsets, perm,
+                      inv, stream);
+}
+
+// ------------------------------------------------------------------------------------------------ experts
+size_t dllm_moe_experts_workspace_size(const dllm_expert_desc* d) {
+  if (!d) return 0;
+  Carver c(nullptr);
+  ExpertBufs b;
+  carve_experts(c, d->dtype, d->Tk, d->H, d->k, d->I, 1, b);
+  return align256(c.off);
+}
+
+int dllm_moe_experts(const dllm_expert_desc* d, const void* h, const void* w_gu, const void* w_down,
+                     const void* w_gu_shared, const void* w_down_shared, const int32_t* counts, const int32_t* offsets,
+                     const int32_t* perm, const int32_t* inv, const float* gates, void* x_inout, void* ws,
+                     size_t ws_bytes, cudaStream_t stream) {
+  REQ(d && h && w_gu && w_down && counts && offsets && perm && inv && gates && x_inout, DLLM_ERR_INVALID_ARG,
+      "moe_experts: NULL argument");
+  REQ((w_gu_shared == nullptr) == (w_down_shared == nullptr), DLLM_ERR_INVALID_ARG,
+      "moe_experts: shared expert weights must both be set or both NULL");
+  REQ(d->Tk >= 0 && d->H > 0 && d->E >= 1 && d->k >= 1 && d->k <= d->E && d->I > 0, DLLM_ERR_SHAPE,
+      "moe_experts: bad shape");
+  REQ(d->E <= 1024 && d->k <= 32, DLLM_ERR_UNSUPPORTED, "moe_experts: needs E <= 1024, k <= 32");
+  REQ(d->dtype == DLLM_BF16 || d->dtype == DLLM_F32, DLLM_ERR_INVALID_ARG, "moe_experts: bad dtype");
+  REQ((d->H * esize(d->dtype)) % 16 == 0, DLLM_ERR_SHAPE, "moe_experts: H row bytes must be a multiple of 16");
+  if (d->dtype == DLLM_BF16) {
+    REQ(d->H % 128 == 0 && d->I % 64 == 0, DLLM_ERR_UNSUPPORTED, "moe_experts: bf16 needs H %% 128 == 0, I %% 64 == 0");
+    REQ(aligned16(h) && aligned16(w_gu) && aligned16(w_down) && (!w_gu_shared || (aligned16(w_gu_shared) && aligned16(w_down_shared))),
+        DLLM_ERR_ALIGN, "moe_experts: operands must be 16-byte aligned");
+  }
+  int st = check_ws(ws, ws_bytes, dllm_moe_experts_workspace_size(d));
+  if (st) return st;
+  if (d->Tk == 0) return DLLM_OK;
+  Carver c(ws);
+  ExpertBufs b;
+  carve_experts(c, d->dtype, d->Tk, d->H, d->k, d->I, 1, b);
+  return run_experts(d->dtype, d->Tk, d->H, d->E, d->k, d->I, h, w_gu, w_down, w_gu_shared, w_down_shared, counts,
+                     offsets, perm, inv, gates, x_inout, b, status_word(ws), stream);
+}
+
+// ------------------------------------------------------------------------------------------------ unmask
+size_t dllm_unmask_workspace_size(const dllm_unmask_desc* d) {
+  if (!d) return 0;
+  return align256(align256(kStatusBytes) + unmask_partials_bytes(d->max_rows, unmask_chunks(d->max_rows, d->V)));
+}
+
+int dllm_unmask(const dllm_unmask_desc* d, const void* logits, const int32_t* row_pos, const int32_t* n_rows_dev,
+                int32_t* tokens, uint8_t* mask, int32_t* sel, int32_t* nsel, float* conf, int32_t* remaining,
+                void* ws, size_t ws_bytes, cudaStream_t stream) {
+  REQ(d && logits && row_pos && n_rows_dev && tokens && mask && sel && nsel && conf && remaining,
+      DLLM_ERR_INVALID_ARG, "unmask: NULL argument");
+  REQ(d->B >= 1 && d->L >= 1 && d->L <= 32 && d->V >= 1 && d->max_rows >= 0 && d->max_rows <= d->B * d->L,
+      DLLM_ERR_SHAPE, "unmask: bad shape (L <= 32, max_rows <= B*L)");
+  REQ(d->T_s >= 1 && d->t >= 0 && d->t < d->T_s, DLLM_ERR_INVALID_ARG, "unmask: step %d of %d", d->t, d->T_s);
+  REQ(d->mode == DLLM_UNMASK_FIXED || d->mode == DLLM_UNMASK_THRESHOLD, DLLM_ERR_INVALID_ARG, "unmask: bad mode");
+  REQ(d->mode == DLLM_UNMASK_FIXED || d->k_max >= 1, DLLM_ERR_INVALID_ARG, "unmask: k_max must be >= 1");
+  REQ(d->dtype == DLLM_BF16 || d->dtype == DLLM_F32, DLLM_ERR_INVALID_ARG, "unmask: bad dtype");
+  REQ(d->vocab_offset >= 0, DLLM_ERR_INVALID_ARG, "unmask: negative vocab_offset");
+  int st = check_ws(ws, ws_bytes, dllm_unmask_workspace_size(d));
+  if (st) return st;
+  Carver c(ws);
+  UnmaskArgs a;
+  a.B = d->B; a.L = d->L; a.V = d->V; a.max_rows = d->max_rows; a.t = d->t; a.T_s = d->T_s; a.mode = d->mode;
+  a.k_max = d->k_max; a.cfg = d->cfg; a.vocab_offset = d->vocab_offset; a.dtype = d->dtype; a.tau = d->tau;
+  a.cfg_scale = d->cfg_scale; a.logits = logits; a.row_pos = row_pos; a.n_rows = n_rows_dev; a.tokens = tokens;
+  a.mask = mask; a.sel = sel; a.nsel = nsel; a.conf = conf; a.remaining = remaining;
+  a.n_chunks = unmask_chunks(d->max_rows, d->V);
+  a.partials = c.take(unmask_partials_bytes(d->max_rows, a.n_chunks));
+  return launch_unmask(a, stream);
+}
+
+// ------------------------------------------------------------------------------------------------ step
+size_t dllm_denoise_step_workspace_size(const dllm_model* m, const dllm_state* st, const dllm_step_params* p) {
+  if (validate_step(m, st, p) != DLLM_OK) return 0;
+  StepPlan s;
+  plan_step(m, st, p, nullptr, s);
+  return s.total;
+}
+
+int dllm_denoise_step_views(const dllm_model* m, const dllm_state* st, const dllm_step_params* p, void* ws,
+                            size_t ws_bytes, dllm_step_views* v) {
+  int r = validate_step(m, st, p);
+  if (r) return r;
+  REQ(v != nullptr, DLLM_ERR_INVALID_ARG, "denoise_step_views: NULL views");
+  StepPlan s;
+  plan_step(m, st, p, nullptr, s);
+  r = check_ws(ws, ws_bytes, s.total);
+  if (r) return r;
+  plan_step(m, st, p, ws, s);
+  v->logits = s.logits;
+  v->row_pos = s.row_pos;
+  v->n_rows = s.n_rows;
+  v->x_final = s.x;
+  return DLLM_OK;
+}
+
+int dllm_denoise_step(const dllm_model* m, const dllm_state* st, const dllm_step_params* p, void* ws,
+                      size_t ws_bytes, cudaStream_t stream) {
+  int r = validate_step(m, st, p);
+  if (r) return r;
+  StepPlan s;
+  plan_step(m, st, p, nullptr, s);
+  r = check_ws(ws, ws_bytes, s.total);
+  if (r) return r;
+  plan_step(m, st, p, ws, s);
+  const int dt = m->dtype, H = m->H, QD = m->Hq * m->d, es = esize(dt);
+  const int P = st->P, L = st->L;
+  int32_t* status = status_word(ws);
+#define TRY(x)            \
+  do {                    \
+    int _r = (x);         \
+    if (_r) return _r;    \
+  } while (0)
+
+  if (!p->commit) TRY(launch_masked_rows(st->mask, s.Bl * L, s.halves, s.row_pos, s.n_rows, stream));
+  TRY(launch_embed(dt, st->tokens, p->commit ? nullptr : st->mask, m->mask_id, m->embed, s.x, s.Tk, H, stream));
+  for (int l = 0; l < m->n_layers; ++l) {
+    const dllm_layer& Ly = m->layers[l];
+    const bool last = l == m->n_layers - 1;
+    TRY(launch_rmsnorm(dt, s.x, Ly.attn_norm, s.h, s.Tk, H, m->eps, nullptr, nullptr, 0, 0, stream));
+    if (p->sprint && p->retain) {
+      RetainArgs ra;
+      ra.B = st->B; ra.Hkv = m->Hkv; ra.d = m->d; ra.P = P; ra.cap = st->cap; ra.n_keep = p->n_keep;
+      ra.cap_thin = st->cap_thin; ra.dtype = dt; ra.k = Ly.k_cache; ra.v = Ly.v_cache; ra.keep_pos = Ly.keep_pos;
+      ra.k_thin = Ly.k_thin; ra.v_thin = Ly.v_thin; ra.scores = nullptr; ra.raw = s.retain_raw; ra.block_len = L;
+      TRY(launch_retain(ra, stream));
+    }
+    // QKV projection + RoPE; block K/V into the cache the attention reads (and the full cache on commit)
+    GemmArgs g;
+    g.x = s.h; g.x_rows = s.Tk; g.w = Ly.w_qkv; g.w_rows = (int64_t)(m->Hq + 2 * m->Hkv) * m->d; g.K = H;
+    g.M = (m->Hq + 2 * m->Hkv) * m->d; g.host_cnt = s.Tk; g.max_cnt = s.Tk; g.cnt_bound = s.Tk; g.dtype = dt;
+    g.status = status; g.f32_scratch = s.proj_scratch;
+    g.epi.kind = EPI_QKV; g.epi.q_out = s.q; g.epi.Hq = m->Hq; g.epi.Hkv = m->Hkv; g.epi.d = m->d; g.epi.L = L;
+    g.epi.pos0 = P; g.epi.rope_base = m->rope_base;
+    if (p->sprint) {
+      g.epi.k_dst = Ly.k_thin; g.epi.v_dst = Ly.v_thin; g.epi.cap = st->cap_thin; g.epi.slot0 = p->n_keep;
+      if (p->commit) { g.epi.k_dst2 = Ly.k_cache; g.epi.v_dst2 = Ly.v_cache; g.epi.cap2 = st->cap; g.epi.slot2 = P; }
+    } else {
+      g.epi.k_dst = Ly.k_cache; g.epi.v_dst = Ly.v_cache; g.epi.cap = st->cap; g.epi.slot0 = P;
+    }
+    TRY(run_gemm(g, stream));
+    // block attention
+    AttnArgs aa;
+    aa.B = st->B; aa.Lq = L; aa.Hq = m->Hq; aa.Hkv = m->Hkv; aa.d = m->d; aa.blk_len = L; aa.q_pos0 = P;
+    aa.n_keys = s.n_keys; aa.cap = p->sprint ? st->cap_thin : st->cap; aa.dtype = dt; aa.scale = 0.f;
+    aa.q = s.q; aa.k = p->sprint ? Ly.k_thin : Ly.k_cache; aa.v = p->sprint ? Ly.v_thin : Ly.v_cache;
+    aa.key_pos = p->sprint ? Ly.keep_pos : nullptr; aa.out = s.ao; aa.ws = s.attn_ws; aa.ws_bytes = s.attn_ws_bytes;
+    TRY(launch_attn(aa, stream));
+    // output projection + residual
+    GemmArgs go;
+    go.x = s.ao; go.x_rows = s.Tk; go.w = Ly.w_o; go.w_rows = H; go.K = QD; go.M = H; go.host_cnt = s.Tk;
+    go.max_cnt = s.Tk; go.cnt_bound = s.Tk; go.dtype = dt; go.status = status; go.f32_scratch = s.proj_scratch;
+    go.epi.kind = EPI_RESID; go.epi.out = s.x; go.epi.ldo = H; go.epi.out_f32 = dt == DLLM_F32;
+    TRY(run_gemm(go, stream));
+    if (p->commit && last) break;  // the last layer's FFN output has no consumer in a commit pass
+    // MoE FFN
+    TRY(launch_rmsnorm(dt, s.x, Ly.ffn_norm, s.h, s.Tk, H, m->eps, nullptr, nullptr, 0, 0, stream));
+    TRY(launch_route(dt, s.h, Ly.w_router, Ly.router_bias, s.Tk, H, m->E, m->k, s.ids, s.gates, s.scores, s.counts,
+                     s.offsets, s.perm, s.inv, stream));
+    TRY(run_experts(dt, s.Tk, H, m->E, m->k, m->I, s.h, Ly.w_gu, Ly.w_down, Ly.w_gu_shared, Ly.w_down_shared,
+                    s.counts, s.offsets, s.perm, s.inv, s.gates, s.x, s.eb, status, stream));
+  }
+  if (p->commit) return DLLM_OK;
+  // final norm on the masked rows (cond, then uncond), LM head, confidence + unmasking
+  TRY(launch_rmsnorm(dt, s.x, m->final_norm, s.xf, s.halves * s.max_rows, H, m->eps, s.row_pos, s.n_rows,
+                     p->cfg, s.Bl * L, stream));
+  GemmArgs gl;
+  gl.x = s.xf; gl.x_rows = (int64_t)s.halves * s.max_rows;
+  gl.w = static_cast<const char*>(m->w_lm) + (size_t)p->vocab_offset * H * es; gl.w_rows = s.vlen;
+  gl.K = H; gl.M = s.vlen; gl.cnt_dev = s.n_rows + 1; gl.host_cnt = s.halves * s.max_rows;
+  gl.max_cnt = s.halves * s.max_rows; gl.cnt_bound = s.halves * s.max_rows; gl.dtype = dt; gl.status = status;
+  gl.f32_scratch = s.proj_scratch;
+  gl.epi.kind = EPI_STORE; gl.epi.out = s.logits; gl.epi.ldo = s.vlen; gl.epi.out_f32 = dt == DLLM_F32;
+  TRY(run_gemm(gl, stream));
+  UnmaskArgs ua;
+  ua.B = s.Bl; ua.L = L; ua.V = s.vlen; ua.max_rows = s.max_rows; ua.t = p->t; ua.T_s = p->T_s; ua.mode = p->mode;
+  ua.k_max = p->k_max; ua.cfg = p->cfg; ua.vocab_offset = p->vocab_offset; ua.dtype = dt; ua.tau = p->tau;
+  ua.cfg_scale = p->cfg_scale; ua.logits = s.logits; ua.row_pos = s.row_pos; ua.n_rows = s.n_rows;
+  ua.tokens = st->tokens; ua.mask = st->mask; ua.sel = p->sel; ua.nsel = p->nsel; ua.conf = p->conf;
+  ua.remaining = p->remaining; ua.partials = s.partials; ua.n_chunks = s.n_chunks;
+  TRY(launch_unmask(ua, stream));
+#undef TRY
+  return DLLM_OK;
+}
+
+}  // extern "C"

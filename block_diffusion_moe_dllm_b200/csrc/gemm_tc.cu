@@ -1,0 +1,463 @@
+// Weight-streaming grouped GEMM on the 5th-generation tensor cores (tcgen05 + TMEM), sm_100a.
+//
+// Y[row, m] = sum_k X[row, k] W[m, k] over groups of X rows (one group per expert, or a single group for the
+// dense projections and the LM head). At the decode shapes of the denoising step every weight tile is read
+// exactly once and the token count per group is small (1..64), so the kernel is built around streaming W:
+//   * swap-AB: the weight tile is the M = 128 operand (A), the group's tokens the N operand (B); the MMA's N
+//     is chosen per tile at run time (tokens rounded up to 16), so a group of 3 tokens issues N = 16 MMAs;
+//   * persistent CTAs (one per SM) walk a flat tile list (group, m-tile, n-tile) built on the device from the
+//     router's counts, so no host synchronisation is needed;
+//   * warp specialisation: warp 0 issues TMA loads into a STAGES-deep shared-memory ring, warp 1 issues
+//     tcgen05.mma from one thread into a double-buffered TMEM accumulator, warps 2..5 drain TMEM
+//     (tcgen05.ld), stage through shared memory and run the fused epilogue (store, residual add, SwiGLU, or
+//     RoPE + KV-cache write) with coalesced global stores;
+//   * weights are loaded with an L2 evict-first hint (read once), activations with evict-last.
+// Every mbarrier wait is bounded; on expiry the kernel records a status word and drains its own copies.
+#include "common.cuh"
+#include "tc.cuh"
+#include "kernels.h"
+#include <cuda.h>
+#include <mutex>
+
+namespace dllm {
+
+namespace {
+
+constexpr int BK = 64;                 // K elements per stage (one 128-byte swizzled row)
+constexpr int A_BYTES = 128 * BK * 2;  // 16 KB weight tile per stage
+constexpr int XBOX_ROWS = 32;          // X rows per TMA box
+constexpr int XBOX_BYTES = XBOX_ROWS * BK * 2;
+constexpr int STAGE_COLS = 32;         // epilogue column chunk
+constexpr int STAGING_BYTES = 128 * STAGE_COLS * 4;
+constexpr int MAX_GROUPS = 1040;
+constexpr int NUM_THREADS = 192;
+constexpr int SMEM_LIMIT = 232448;
+
+struct Smem {
+  uint64_t full[16];
+  uint64_t empty[16];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t done;
+  uint32_t tmem_base;
+  int abort_flag;
+  int n_groups;
+  int total_tiles;
+  int tile_prefix[MAX_GROUPS + 1];  // exclusive prefix of tiles per group
+  int grp_off[MAX_GROUPS];
+  int grp_cnt[MAX_GROUPS];
+  int chunk_sum[NUM_THREADS];
+};
+
+struct KParams {
+  int K, M, swiglu, m_tiles;
+  int64_t w_group_stride;
+  int n_dev, has_extra, extra_off, extra_cnt, host_cnt;
+  const int32_t* grp_off;
+  const int32_t* grp_cnt;
+  const int32_t* cnt_dev;
+  EpiParams epi;
+  int32_t* status;
+};
+
+__device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                         int32_t* status, int code) {
+  uint32_t n = 0;
+  while (!tc::mbar_try_wait(bar, parity)) {
+    if (*abort_flag) return false;
+    if (++n > (1u << 22)) {
+      *abort_flag = 1;
+      if (status) atomicExch(status, code);
+      return false;
+    }
+  }
+  return true;
+}
+
+// Tile t -> (group, m-tile, first row of the n-tile, rows in the n-tile). n-tiles of one weight tile are adjacent.
+template <int BN>
+__device__ __forceinline__ void decode_tile(const Smem& sm, int m_tiles, int t, int& g, int& mt, int& n0,
+                                            int& nval) {
+  int lo = 0, hi = sm.n_groups - 1;
+  while (lo < hi) {  // last g with tile_prefix[g] <= t
+    int mid = (lo + hi + 1) >> 1;
+    if (sm.tile_prefix[mid] <= t) lo = mid; else hi = mid - 1;
+  }
+  g = lo;
+  int local = t - sm.tile_prefix[g];
+  int ntl = (sm.grp_cnt[g] + BN - 1) / BN;
+  mt = local / ntl;
+  int nt = local - mt * ntl;
+  n0 = nt * BN;
+  nval = min(BN, sm.grp_cnt[g] - n0);
+}
+
+__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }
+
+template <int BN>
+__device__ void epilogue_chunk(const KParams& p, const float* stage, int g, int mt, int n0, int nval, int c0,
+                               int row0, int tid) {
+  const EpiParams& e = p.epi;
+  const int ncols = min(STAGE_COLS, nval - c0);
+  if (e.kind == EPI_SWIGLU) {
+    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(e.out);
+    for (int idx = tid; idx < ncols * 64; idx += 128) {
+      int j = idx >> 6, m = idx & 63;
+      float gt = stage[j * 128 + m], up = stage[j * 128 + 64 + m];
+      int64_t row = row0 + n0 + c0 + j;
+      out[row * e.ldo + mt * 64 + m] = __float2bfloat16_rn(silu_f(gt) * up);
+    }
+  } else if (e.kind == EPI_QKV) {
+    // m-tile = one head of d = 128 rows: q heads, then k heads, then v heads. RoPE pairs (i, i + 64).
+    const int hh = mt;
+    const bool rot = hh < e.Hq + e.Hkv;
+    const int m = tid & 63;
+    const double inv_freq = pow((double)e.rope_base, -2.0 * (double)m / 128.0);
+    for (int idx = tid; idx < ncols * 64; idx += 128) {
+      int j = idx >> 6;
+      int tr = row0 + n0 + c0 + j;  // token row = b * L + i
+      float x1 = stage[j * 128 + m], x2 = stage[j * 128 + 64 + m];
+      float y1 = x1, y2 = x2;
+      if (rot) {
+        int pos = e.pos0 + tr % e.L;
+        double sn, cs;
+        sincos((double)pos * inv_freq, &sn, &cs);
+        float c = (float)cs, s = (float)sn;
+        y1 = x1 * c - x2 * s;
+        y2 = x2 * c + x1 * s;
+      }
+      __nv_bfloat16 b1 = __float2bfloat16_rn(y1), b2 = __float2bfloat16_rn(y2);
+      if (hh < e.Hq) {
+        __nv_bfloat16* q = static_cast<__nv_bfloat16*>(e.q_out) + ((int64_t)tr * e.Hq + hh) * 128;
+        q[m] = b1;
+        q[m + 64] = b2;
+      } else {
+        int b = tr / e.L, i = tr % e.L;
+        bool is_k = hh < e.Hq + e.Hkv;
+        int gk = is_k ? hh - e.Hq : hh - e.Hq - e.Hkv;
+        __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(is_k ? e.k_dst : e.v_dst) +
+                             (((int64_t)b * e.Hkv + gk) * e.cap + e.slot0 + i) * 128;
+        dst[m] = b1;
+        dst[m + 64] = b2;
+        void* d2v = is_k ? e.k_dst2 : e.v_dst2;
+        if (d2v) {
+          __nv_bfloat16* d2 = static_cast<__nv_bfloat16*>(d2v) + (((int64_t)b * e.Hkv + gk) * e.cap2 + e.slot2 + i) * 128;
+          d2[m] = b1;
+          d2[m + 64] = b2;
+        }
+      }
+    }
+  } else {
+    const int64_t mbase = (int64_t)mt * 128;
+    for (int idx = tid; idx < ncols * 128; idx += 128) {
+      int j = idx >> 7, m = idx & 127;
+      float v = stage[j * 128 + m];
+      int64_t off = (int64_t)(row0 + n0 + c0 + j) * e.ldo + mbase + m;
+      if (e.out_f32) {
+        float* o = static_cast<float*>(e.out);
+        o[off] = (e.kind == EPI_RESID) ? o[off] + v : v;
+      } else {
+        __nv_bfloat16* o = static_cast<__nv_bfloat16*>(e.out);
+        float r = (e.kind == EPI_RESID) ? __bfloat162float(o[off]) + v : v;
+        o[off] = __float2bfloat16_rn(r);
+      }
+    }
+  }
+}
+
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_w2,
+               const __grid_constant__ CUtensorMap tmap_x, const KParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  constexpr int STAGE_BYTES = A_BYTES + BN * BK * 2;
+  uint8_t* stages = base;
+  float* staging = reinterpret_cast<float*>(base + STAGES * STAGE_BYTES);
+  Smem& sm = *reinterpret_cast<Smem*>(base + STAGES * STAGE_BYTES + STAGING_BYTES);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+
+  // ---- group table: counts, offsets and the exclusive prefix of tiles per group
+  const int n_groups = p.n_dev + p.has_extra + ((p.n_dev + p.has_extra) == 0 ? 1 : 0);
+  for (int g = tid; g < n_groups; g += NUM_THREADS) {
+    int off, cnt;
+    if (g < p.n_dev) {
+      off = p.grp_off[g];
+      cnt = p.grp_cnt[g];
+    } else if (p.has_extra) {
+      off = p.extra_off;
+      cnt = p.extra_cnt;
+    } else {
+      off = 0;
+      cnt = p.cnt_dev ? min(*p.cnt_dev, p.host_cnt) : p.host_cnt;
+    }
+    sm.grp_off[g] = off;
+    sm.grp_cnt[g] = max(cnt, 0);
+  }
+  if (tid == 0) {
+    sm.n_groups = n_groups;
+    sm.abort_flag = 0;
+    for (int s = 0; s < STAGES; ++s) {
+      tc::mbar_init(&sm.full[s], 1);
+      tc::mbar_init(&sm.empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      tc::mbar_init(&sm.tfull[b], 1);
+      tc::mbar_init(&sm.tempty[b], 128);
+    }
+    tc::mbar_init(&sm.done, 1);
+    tc::fence_mbar_init();
+  }
+  if (warp == 1) tc::tmem_alloc(&sm.tmem_base, 2 * BN);
+  __syncthreads();
+  // prefix of tiles per group: contiguous chunks per thread, then a scan of the chunk sums
+  {
+    int* chunk_sum = sm.chunk_sum;
+    const int per = (n_groups + NUM_THREADS - 1) / NUM_THREADS;
+    const int g0 = tid * per, g1 = min(n_groups, g0 + per);
+    int s = 0;
+    for (int g = g0; g < g1; ++g) s += ((sm.grp_cnt[g] + BN - 1) / BN) * p.m_tiles;
+    chunk_sum[tid] = s;
+    __syncthreads();
+    if (tid == 0) {
+      int run = 0;
+      for (int i = 0; i < NUM_THREADS; ++i) {
+        int v = chunk_sum[i];
+        chunk_sum[i] = run;
+        run += v;
+      }
+      sm.total_tiles = run;
+    }
+    __syncthreads();
+    int run = chunk_sum[tid];
+    for (int g = g0; g < g1; ++g) {
+      sm.tile_prefix[g] = run;
+      run += ((sm.grp_cnt[g] + BN - 1) / BN) * p.m_tiles;
+    }
+    __syncthreads();
+  }
+  const int total = sm.total_tiles;
+  volatile int* abort_flag = &sm.abort_flag;
+  const int kblocks = p.K / BK;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (tc::elect_one()) {
+      tc::prefetch_tmap(&tmap_w);
+      tc::prefetch_tmap(&tmap_x);
+      if (p.has_extra) tc::prefetch_tmap(&tmap_w2);
+      const uint64_t pol_w = tc::policy_evict_first();
+      const uint64_t pol_x = tc::policy_evict_last();
+      uint32_t it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        int g, mt, n0, nval;
+        decode_tile<BN>(sm, p.m_tiles, t, g, mt, n0, nval);
+        const bool extra = p.has_extra && g == p.n_dev;
+        const CUtensorMap* wm = extra ? &tmap_w2 : &tmap_w;
+        const int64_t wrow = extra ? 0 : (int64_t)g * p.w_group_stride;
+        const int nb = (nval + XBOX_ROWS - 1) / XBOX_ROWS;
+        const uint32_t bytes = A_BYTES + nb * XBOX_BYTES;
+        const int xrow = sm.grp_off[g] + n0;
+        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (!wait_bar(&sm.empty[s], ph ^ 1, abort_flag, p.status, ST_TIMEOUT_PRODUCER)) { ok = false; break; }
+          uint8_t* a = stages + s * STAGE_BYTES;
+          uint8_t* b = a + A_BYTES;
+          tc::mbar_arrive_expect_tx(&sm.full[s], bytes);
+          if (p.swiglu) {
+            tc::tma_load_2d(a, wm, kb * BK, (int)(wrow + mt * 64), &sm.full[s], pol_w);
+            tc::tma_load_2d(a + A_BYTES / 2, wm, kb * BK, (int)(wrow + p.M + mt * 64), &sm.full[s], pol_w);
+          } else {
+            tc::tma_load_2d(a, wm, kb * BK, (int)(wrow + mt * 128), &sm.full[s], pol_w);
+          }
+          for (int j = 0; j < nb; ++j)
+            tc::tma_load_2d(b + j * XBOX_BYTES, &tmap_x, kb * BK, xrow + j * XBOX_ROWS, &sm.full[s], pol_x);
+        }
+      }
+      if (!ok) {
+        // drain: wait (bounded) for the copies of the last issued stages to land before leaving
+        uint32_t first = it > (uint32_t)STAGES ? it - STAGES : 0;
+        for (uint32_t i = first; i < it; ++i) tc::mbar_wait(&sm.full[i % STAGES], (i / STAGES) & 1, 1u << 16);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (tc::elect_one()) {
+      uint32_t it = 0, tcount = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++tcount) {
+        int g, mt, n0, nval;
+        decode_tile<BN>(sm, p.m_tiles, t, g, mt, n0, nval);
+        const uint32_t buf = tcount & 1, tph = (tcount >> 1) & 1;
+        if (!wait_bar(&sm.tempty[buf], tph ^ 1, abort_flag, p.status, ST_TIMEOUT_MMA)) { ok = false; break; }
+        tc::fence_after_sync();
+        const uint32_t N = max(16, (nval + 15) & ~15);
+        const uint32_t idesc = tc::idesc_bf16_f32(128, N);
+        const uint32_t d = sm.tmem_base + buf * BN;
+        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (!wait_bar(&sm.full[s], ph, abort_flag, p.status, ST_TIMEOUT_MMA)) { ok = false; break; }
+          tc::fence_after_sync();
+          const uint32_t a = tc::smem_u32(stages + s * STAGE_BYTES);
+          const uint32_t b = a + A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            tc::mma_bf16(d, tc::sdesc_k128(a + kk * 32), tc::sdesc_k128(b + kk * 32), idesc, (kb | kk) != 0);
+          tc::mma_commit(&sm.empty[s]);
+        }
+        if (!ok) break;
+        tc::mma_commit(&sm.tfull[buf]);
+      }
+      // all issued MMAs complete before TMEM is released
+      tc::mma_commit(&sm.done);
+      tc::mbar_wait(&sm.done, 0, 1u << 20);
+    }
+  } else {
+    // ------------------------------------------------------------------ epilogue warps 2..5
+    const int q = warp & 3;          // TMEM lane quadrant this warp may access
+    const int row = q * 32 + lane;   // tile row m (TMEM lane)
+    const int etid = tid - 64;       // 0..127
+    uint32_t tcount = 0;
+    for (int t = blockIdx.x; t < total; t += gridDim.x, ++tcount) {
+      int g, mt, n0, nval;
+      decode_tile<BN>(sm, p.m_tiles, t, g, mt, n0, nval);
+      const uint32_t buf = tcount & 1, tph = (tcount >> 1) & 1;
+      if (!wait_bar(&sm.tfull[buf], tph, abort_flag, p.status, ST_TIMEOUT_EPILOGUE)) break;
+      tc::fence_after_sync();
+      for (int c0 = 0; c0 < nval; c0 += STAGE_COLS) {
+        float v[STAGE_COLS];
+        const uint32_t taddr = sm.tmem_base + ((uint32_t)(q * 32) << 16) + buf * BN + c0;
+        tc::tmem_ld16(taddr, v);
+        tc::tmem_ld16(taddr + 16, v + 16);
+        tc::named_bar_sync(1, 128);  // staging free (previous chunk consumed)
+#pragma unroll
+        for (int j = 0; j < STAGE_COLS; ++j) staging[j * 128 + row] = v[j];
+        tc::named_bar_sync(1, 128);
+        epilogue_chunk<BN>(p, staging, g, mt, n0, nval, c0, sm.grp_off[g], etid);
+      }
+      tc::fence_before_sync();
+      tc::mbar_arrive(&sm.tempty[buf]);
+    }
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(sm.tmem_base, 2 * BN);
+  }
+}
+
+// ---------------------------------------------------------------------------------------------------- host
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+int make_map(CUtensorMap* m, const void* ptr, int64_t rows, int K, int box_rows) {
+  EncodeTiledFn enc = get_encode();
+  if (!enc) {
+    dllm_host::set_error("cuTensorMapEncodeTiled unavailable");
+    return DLLM_ERR_CUDA;
+  }
+  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+  cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    dllm_host::set_error("cuTensorMapEncodeTiled failed (%d) rows=%lld K=%d box_rows=%d", (int)r, (long long)rows,
+                         K, box_rows);
+    return DLLM_ERR_CUDA;
+  }
+  return DLLM_OK;
+}
+
+template <int BN, int STAGES>
+int launch(const GemmArgs& a, const CUtensorMap& mw, const CUtensorMap& mw2, const CUtensorMap& mx,
+           const KParams& kp, cudaStream_t s) {
+  constexpr int STAGE_BYTES = A_BYTES + BN * BK * 2;
+  constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + STAGING_BYTES + (int)sizeof(Smem);
+  static_assert(SMEM <= SMEM_LIMIT, "shared memory budget");
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         SMEM);
+    if (e != cudaSuccess) return dllm_host::cuda_status(e, "cudaFuncSetAttribute(gemm_tc)");
+    configured = true;
+  }
+  gemm_tc_kernel<BN, STAGES><<<num_sms(), NUM_THREADS, SMEM, s>>>(mw, mw2, mx, kp);
+  DLLM_CHECK_LAUNCH("gemm_tc_kernel");
+  return DLLM_OK;
+}
+
+}  // namespace
+
+int gemm_bf16_tc(const GemmArgs& a, cudaStream_t s) {
+  DLLM_REQUIRE(a.K % BK == 0 && a.K > 0, DLLM_ERR_UNSUPPORTED, "gemm: K=%d must be a positive multiple of 64", a.K);
+  DLLM_REQUIRE(a.swiglu ? (a.M % 64 == 0) : (a.M % 128 == 0), DLLM_ERR_UNSUPPORTED,
+               "gemm: M=%d must be a multiple of %d", a.M, a.swiglu ? 64 : 128);
+  DLLM_REQUIRE(a.n_dev + a.has_extra <= MAX_GROUPS, DLLM_ERR_UNSUPPORTED, "gemm: too many groups");
+  DLLM_REQUIRE(((uintptr_t)a.x % 16 == 0) && ((uintptr_t)a.w % 16 == 0) && (!a.w2 || (uintptr_t)a.w2 % 16 == 0),
+               DLLM_ERR_ALIGN, "gemm: operands must be 16-byte aligned");
+  if (a.epi.kind == EPI_QKV)
+    DLLM_REQUIRE(a.epi.d == 128, DLLM_ERR_UNSUPPORTED, "gemm: QKV epilogue needs head dim 128");
+  const int box_rows = a.swiglu ? 64 : 128;
+  CUtensorMap mw, mw2, mx;
+  int st = make_map(&mw, a.w, a.w_rows, a.K, box_rows);
+  if (st) return st;
+  st = make_map(&mw2, a.w2 ? a.w2 : a.w, a.w2 ? a.w2_rows : a.w_rows, a.K, box_rows);
+  if (st) return st;
+  st = make_map(&mx, a.x, a.x_rows, a.K, XBOX_ROWS);
+  if (st) return st;
+  KParams kp;
+  kp.K = a.K;
+  kp.M = a.M;
+  kp.swiglu = a.swiglu;
+  kp.m_tiles = a.swiglu ? a.M / 64 : a.M / 128;
+  kp.w_group_stride = a.w_group_stride;
+  kp.n_dev = a.n_dev;
+  kp.has_extra = a.has_extra;
+  kp.extra_off = a.extra_off;
+  kp.extra_cnt = a.extra_cnt;
+  kp.host_cnt = a.host_cnt;
+  kp.grp_off = a.grp_off;
+  kp.grp_cnt = a.grp_cnt;
+  kp.cnt_dev = a.cnt_dev;
+  kp.epi = a.epi;
+  kp.status = a.status;
+  if (a.max_cnt <= 32) return launch<32, 9>(a, mw, mw2, mx, kp, s);
+  if (a.max_cnt <= 64) return launch<64, 8>(a, mw, mw2, mx, kp, s);
+  if (a.max_cnt <= 128) return launch<128, 6>(a, mw, mw2, mx, kp, s);
+  return launch<256, 4>(a, mw, mw2, mx, kp, s);
+}
+
+int num_sms() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+}  // namespace dllm

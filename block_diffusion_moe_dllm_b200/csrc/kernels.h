@@ -1,0 +1,68 @@
+// Internal host interface between the C-ABI entry points and the kernels (not part of the public ABI).
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stddef.h>
+
+namespace dllm {
+
+enum EpiKind : int {
+  EPI_STORE = 0,   // out[row, m] = acc                 (storage type, or fp32 if out_f32)
+  EPI_RESID = 1,   // out[row, m] = out[row, m] + acc   (rounded once)
+  EPI_SWIGLU = 2,  // out[row, i] = silu(acc_gate) * acc_up
+  EPI_QKV = 3,     // RoPE on q/k heads; q -> q_out, k/v -> cache rows
+};
+
+struct EpiParams {
+  int kind = EPI_STORE;
+  void* out = nullptr;
+  int64_t ldo = 0;
+  int out_f32 = 0;
+  // EPI_QKV
+  void* q_out = nullptr;            // [rows, Hq, d]
+  void* k_dst = nullptr;            // [B, Hkv, cap, d]
+  void* v_dst = nullptr;
+  void* k_dst2 = nullptr;           // optional second destination (nullable)
+  void* v_dst2 = nullptr;
+  int cap = 0, slot0 = 0, cap2 = 0, slot2 = 0;
+  int Hq = 0, Hkv = 0, d = 0, L = 1, pos0 = 0;
+  float rope_base = 10000.f;
+};
+
+// Y = X W^T over groups of X rows. Group g < n_dev reads rows [grp_off[g], grp_off[g] + grp_cnt[g]) of X and
+// weight rows [g * w_group_stride, ...) of W; the optional extra group reads rows [extra_off, extra_off +
+// extra_cnt) of X with weights W2. With no device groups and no extra group there is one group of X rows
+// [0, cnt) with cnt = *cnt_dev if cnt_dev else host_cnt.
+struct GemmArgs {
+  const void* x = nullptr;
+  int64_t x_rows = 0;
+  const void* w = nullptr;
+  int64_t w_rows = 0;
+  const void* w2 = nullptr;
+  int64_t w2_rows = 0;
+  int K = 0;
+  int M = 0;               // outputs per group (swiglu: I)
+  int swiglu = 0;          // weight tile = rows [m, m+64) and [I + m, I + m + 64)
+  int64_t w_group_stride = 0;
+  int n_dev = 0;
+  const int32_t* grp_off = nullptr;
+  const int32_t* grp_cnt = nullptr;
+  int has_extra = 0;
+  int extra_off = 0, extra_cnt = 0;
+  const int32_t* cnt_dev = nullptr;
+  int host_cnt = 0;
+  int max_cnt = 0;         // typical largest group (chooses the tensor-core N tile; larger groups take more tiles)
+  int cnt_bound = 0;       // true upper bound of rows in any group (sizes the SIMT grid)
+  int dtype = 0;           // DLLM_BF16 / DLLM_F32
+  EpiParams epi;
+  int32_t* status = nullptr;
+  float* f32_scratch = nullptr;  // f32 path: [x_rows, M (x2 for swiglu)] raw products
+};
+
+int gemm_bf16_tc(const GemmArgs& a, cudaStream_t s);
+int gemm_f32_simt(const GemmArgs& a, cudaStream_t s);
+size_t gemm_f32_scratch_bytes(int64_t x_rows, int M, int swiglu);
+
+int num_sms();
+
+}  // namespace dllm

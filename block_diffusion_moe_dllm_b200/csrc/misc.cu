@@ -1,0 +1,324 @@
+// Memory-bound helper kernels of the denoising step: embedding gather, RMSNorm, masked-row compaction,
+// expert-row gather, gate-weighted combine, and the fp32 SIMT projection path (storage type fp32).
+#include "common.cuh"
+#include "kernels.h"
+#include "misc.h"
+
+namespace dllm {
+
+// ------------------------------------------------------------------------------------------------ embedding
+// x[t] = embed[mask[t] ? mask_id : tokens[t]]  (block tokens, masked positions read the mask embedding row)
+template <typename T>
+__global__ void embed_kernel(const int32_t* __restrict__ tokens, const uint8_t* __restrict__ mask, int mask_id,
+                             const T* __restrict__ table, T* __restrict__ x, int H) {
+  const int t = blockIdx.x;
+  const int id = (mask && mask[t]) ? mask_id : tokens[t];
+  const uint4* src = reinterpret_cast<const uint4*>(table + (int64_t)id * H);
+  uint4* dst = reinterpret_cast<uint4*>(x + (int64_t)t * H);
+  const int nvec = H * (int)sizeof(T) / 16;
+  for (int i = threadIdx.x; i < nvec; i += blockDim.x) dst[i] = src[i];
+}
+
+int launch_embed(int dtype, const int32_t* tokens, const uint8_t* mask, int mask_id, const void* table, void* x,
+                 int rows, int H, cudaStream_t s) {
+  if (rows <= 0) return DLLM_OK;
+  if (dtype == DLLM_BF16)
+    embed_kernel<__nv_bfloat16><<<rows, 128, 0, s>>>(tokens, mask, mask_id, (const __nv_bfloat16*)table,
+                                                     (__nv_bfloat16*)x, H);
+  else
+    embed_kernel<float><<<rows, 128, 0, s>>>(tokens, mask, mask_id, (const float*)table, (float*)x, H);
+  DLLM_CHECK_LAUNCH("embed_kernel");
+  return DLLM_OK;
+}
+
+// ------------------------------------------------------------------------------------------------ RMSNorm
+// out[r] = x[src(r)] / sqrt(mean(x^2) + eps) * g, fp32 math. src(r) = r, or through a compacted row list:
+// rows r < n come from row_pos[r], rows n <= r < 2n from row_pos[r - n] + uncond_off (n = *n_dev).
+template <typename T>
+__global__ void rmsnorm_kernel(const T* __restrict__ x, const T* __restrict__ g, T* __restrict__ out, int H,
+                               float eps, const int32_t* __restrict__ row_pos, const int32_t* __restrict__ n_dev,
+                               int two_halves, int uncond_off) {
+  int r = blockIdx.x;
+  int src = r;
+  if (row_pos) {
+    const int n = *n_dev;
+    if (r >= n * (two_halves ? 2 : 1)) return;
+    src = (r < n) ? row_pos[r] : row_pos[r - n] + uncond_off;
+  }
+  const T* xr = x + (int64_t)src * H;
+  float ss = 0.f;
+  for (int i = threadIdx.x; i < H; i += blockDim.x) {
+    float v = to_f32(xr[i]);
+    ss += v * v;
+  }
+  __shared__ float red[32];
+  ss = warp_sum(ss);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+    v = warp_sum(v);
+    if (threadIdx.x == 0) red[0] = v;
+  }
+  __syncthreads();
+  const float inv = 1.0f / sqrtf(red[0] / (float)H + eps);
+  T* o = out + (int64_t)r * H;
+  for (int i = threadIdx.x; i < H; i += blockDim.x) o[i] = from_f32<T>(to_f32(xr[i]) * inv * to_f32(g[i]));
+}
+
+int launch_rmsnorm(int dtype, const void* x, const void* g, void* out, int rows, int H, float eps,
+                   const int32_t* row_pos, const int32_t* n_dev, int two_halves, int uncond_off, cudaStream_t s) {
+  if (rows <= 0) return DLLM_OK;
+  if (dtype == DLLM_BF16)
+    rmsnorm_kernel<__nv_bfloat16><<<rows, 256, 0, s>>>((const __nv_bfloat16*)x, (const __nv_bfloat16*)g,
+                                                       (__nv_bfloat16*)out, H, eps, row_pos, n_dev, two_halves,
+                                                       uncond_off);
+  else
+    rmsnorm_kernel<float><<<rows, 256, 0, s>>>((const float*)x, (const float*)g, (float*)out, H, eps, row_pos,
+                                               n_dev, two_halves, uncond_off);
+  DLLM_CHECK_LAUNCH("rmsnorm_kernel");
+  return DLLM_OK;
+}
+
+// ------------------------------------------------------------------------------------------------ masked rows
+// Ascending list of the still-masked flat positions of the first n_pos positions (the logical rows), their
+// count n_out[0] and n_out[1] = n_out[0] * halves (rows the LM head scores).
+__global__ void masked_rows_kernel(const uint8_t* __restrict__ mask, int n_pos, int halves, int32_t* row_pos,
+                                   int32_t* n_out) {
+  __shared__ int warp_tot[32];
+  __shared__ int base;
+  if (threadIdx.x == 0) base = 0;
+  __syncthreads();
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int c0 = 0; c0 < n_pos; c0 += blockDim.x) {
+    const int p = c0 + threadIdx.x;
+    const int f = (p < n_pos && mask[p]) ? 1 : 0;
+    const unsigned bal = __ballot_sync(0xffffffffu, f);
+    const int in_warp = __popc(bal & ((1u << lane) - 1u));
+    if (lane == 0) warp_tot[w] = __popc(bal);
+    __syncthreads();
+    int before = 0, tot = 0;
+    for (int i = 0; i < nw; ++i) {
+      if (i < w) before += warp_tot[i];
+      tot += warp_tot[i];
+    }
+    if (f) row_pos[base + before + in_warp] = p;
+    __syncthreads();
+    if (threadIdx.x == 0) base += tot;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    n_out[0] = base;
+    n_out[1] = base * halves;
+  }
+}
+
+int launch_masked_rows(const uint8_t* mask, int n_pos, int halves, int32_t* row_pos, int32_t* n_out,
+                       cudaStream_t s) {
+  masked_rows_kernel<<<1, 1024, 0, s>>>(mask, n_pos, halves, row_pos, n_out);
+  DLLM_CHECK_LAUNCH("masked_rows_kernel");
+  return DLLM_OK;
+}
+
+// ------------------------------------------------------------------------------------------------ expert rows
+// Xp[r] = h[perm[r] / k] for r < Tk * k (assignments grouped by expert), Xp[Tk * k + t] = h[t] (shared expert).
+template <typename T>
+__global__ void gather_rows_kernel(const T* __restrict__ h, const int32_t* __restrict__ perm, int k, int n_assign,
+                                   int shared, T* __restrict__ xp, int H) {
+  const int r = blockIdx.x;
+  int src;
+  if (r < n_assign) src = perm[r] / k;
+  else if (shared) src = r - n_assign;
+  else return;
+  const uint4* a = reinterpret_cast<const uint4*>(h + (int64_t)src * H);
+  uint4* b = reinterpret_cast<uint4*>(xp + (int64_t)r * H);
+  const int nvec = H * (int)sizeof(T) / 16;
+  for (int i = threadIdx.x; i < nvec; i += blockDim.x) b[i] = a[i];
+}
+
+int launch_gather_rows(int dtype, const void* h, const int32_t* perm, int k, int Tk, int shared, void* xp, int H,
+                       cudaStream_t s) {
+  const int rows = Tk * k + (shared ? Tk : 0);
+  if (rows <= 0) return DLLM_OK;
+  if (dtype == DLLM_BF16)
+    gather_rows_kernel<__nv_bfloat16><<<rows, 128, 0, s>>>((const __nv_bfloat16*)h, perm, k, Tk * k, shared,
+                                                           (__nv_bfloat16*)xp, H);
+  else
+    gather_rows_kernel<float><<<rows, 128, 0, s>>>((const float*)h, perm, k, Tk * k, shared, (float*)xp, H);
+  DLLM_CHECK_LAUNCH("gather_rows_kernel");
+  return DLLM_OK;
+}
+
+// ------------------------------------------------------------------------------------------------ combine
+// x[t] = x[t] + (y[Tk*k + t] + sum_j gates[t, j] * y[inv[t*k + j]]), summed in fp32 in slot order, rounded once.
+template <typename T>
+__global__ void combine_kernel(T* __restrict__ x, const float* __restrict__ y, const float* __restrict__ gates,
+                               const int32_t* __restrict__ inv, int k, int n_assign, int shared, int H) {
+  const int t = blockIdx.x;
+  __shared__ int rows[32];
+  __shared__ float gs[32];
+  if (threadIdx.x < k) {
+    rows[threadIdx.x] = inv[t * k + threadIdx.x];
+    gs[threadIdx.x] = gates[t * k + threadIdx.x];
+  }
+  __syncthreads();
+  const float* ys = y + (int64_t)(n_assign + t) * H;
+  T* xr = x + (int64_t)t * H;
+  for (int i = threadIdx.x; i < H; i += blockDim.x) {
+    float acc = shared ? ys[i] : 0.f;
+    for (int j = 0; j < k; ++j) acc += gs[j] * y[(int64_t)rows[j] * H + i];
+    xr[i] = from_f32<T>(to_f32(xr[i]) + acc);
+  }
+}
+
+int launch_combine(int dtype, void* x, const float* y, const float* gates, const int32_t* inv, int k, int Tk,
+                   int shared, int H, cudaStream_t s) {
+  if (Tk <= 0) return DLLM_OK;
+  if (dtype == DLLM_BF16)
+    combine_kernel<__nv_bfloat16><<<Tk, 256, 0, s>>>((__nv_bfloat16*)x, y, gates, inv, k, Tk * k, shared, H);
+  else
+    combine_kernel<float><<<Tk, 256, 0, s>>>((float*)x, y, gates, inv, k, Tk * k, shared, H);
+  DLLM_CHECK_LAUNCH("combine_kernel");
+  return DLLM_OK;
+}
+
+// ------------------------------------------------------------------------------------------------ fp32 path
+// SIMT GEMM over groups: raw[row, f] = sum_k X[row, k] W[g * wstride + f, k], f < Mw, fp32 throughout.
+// Tiles of 32 rows x 64 features, 256 threads, 2 x 4 outputs per thread.
+struct SimtGroups {
+  int n_dev, has_extra, extra_off, extra_cnt, host_cnt;
+  const int32_t* grp_off;
+  const int32_t* grp_cnt;
+  const int32_t* cnt_dev;
+};
+
+__device__ __forceinline__ void group_of(const SimtGroups& G, int g, int& off, int& cnt) {
+  if (g < G.n_dev) {
+    off = G.grp_off[g];
+    cnt = G.grp_cnt[g];
+  } else if (G.has_extra) {
+    off = G.extra_off;
+    cnt = G.extra_cnt;
+  } else {
+    off = 0;
+    cnt = G.cnt_dev ? min(*G.cnt_dev, G.host_cnt) : G.host_cnt;
+  }
+}
+
+__global__ void simt_gemm_f32_kernel(const float* __restrict__ X, const float* __restrict__ W,
+                                     const float* __restrict__ W2, int K, int Mw, int64_t wstride, SimtGroups G,
+                                     float* __restrict__ raw) {
+  const int g = blockIdx.z;
+  int off, cnt;
+  group_of(G, g, off, cnt);
+  const int n0 = blockIdx.x * 32, f0 = blockIdx.y * 64;
+  if (n0 >= cnt) return;
+  const bool extra = G.has_extra && g == G.n_dev;
+  const float* Wg = extra ? W2 : W + (int64_t)g * wstride * K;
+  __shared__ float xs[32][33];
+  __shared__ float ws[64][33];
+  const int ty = threadIdx.x >> 4, tx = threadIdx.x & 15;
+  float acc[2][4] = {};
+  for (int k0 = 0; k0 < K; k0 += 32) {
+    for (int i = threadIdx.x; i < 32 * 32; i += 256) {
+      int r = i >> 5, c = i & 31;
+      xs[r][c] = (n0 + r < cnt && k0 + c < K) ? X[(int64_t)(off + n0 + r) * K + k0 + c] : 0.f;
+    }
+    for (int i = threadIdx.x; i < 64 * 32; i += 256) {
+      int r = i >> 5, c = i & 31;
+      ws[r][c] = (f0 + r < Mw && k0 + c < K) ? Wg[(int64_t)(f0 + r) * K + k0 + c] : 0.f;
+    }
+    __syncthreads();
+    for (int c = 0; c < 32; ++c) {
+#pragma unroll
+      for (int a = 0; a < 2; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) acc[a][b] += xs[ty * 2 + a][c] * ws[tx * 4 + b][c];
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int a = 0; a < 2; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      int r = n0 + ty * 2 + a, f = f0 + tx * 4 + b;
+      if (r < cnt && f < Mw) raw[(int64_t)(off + r) * Mw + f] = acc[a][b];
+    }
+}
+
+// Epilogue of the fp32 path over every valid row of every group.
+__global__ void simt_epilogue_f32_kernel(const float* __restrict__ raw, int Mw, int M, SimtGroups G, EpiParams e) {
+  const int g = blockIdx.y;
+  int off, cnt;
+  group_of(G, g, off, cnt);
+  const int n = blockIdx.x;
+  if (n >= cnt) return;
+  const int row = off + n;
+  const float* rr = raw + (int64_t)row * Mw;
+  if (e.kind == EPI_SWIGLU) {
+    float* out = static_cast<float*>(e.out);
+    for (int i = threadIdx.x; i < M; i += blockDim.x) {
+      float gt = rr[i], up = rr[M + i];
+      out[(int64_t)row * e.ldo + i] = gt / (1.0f + expf(-gt)) * up;
+    }
+  } else if (e.kind == EPI_QKV) {
+    const int d = e.d, half = d / 2, nh = e.Hq + 2 * e.Hkv;
+    const int b = row / e.L, i = row % e.L, pos = e.pos0 + i;
+    for (int idx = threadIdx.x; idx < nh * half; idx += blockDim.x) {
+      const int hh = idx / half, m = idx % half;
+      float x1 = rr[hh * d + m], x2 = rr[hh * d + m + half];
+      float y1 = x1, y2 = x2;
+      if (hh < e.Hq + e.Hkv) {
+        double sn, cs;
+        sincos((double)pos * pow((double)e.rope_base, -2.0 * (double)m / (double)d), &sn, &cs);
+        float c = (float)cs, s = (float)sn;
+        y1 = x1 * c - x2 * s;
+        y2 = x2 * c + x1 * s;
+      }
+      float* dst;
+      if (hh < e.Hq) {
+        dst = static_cast<float*>(e.q_out) + ((int64_t)row * e.Hq + hh) * d;
+      } else {
+        const bool is_k = hh < e.Hq + e.Hkv;
+        const int gk = is_k ? hh - e.Hq : hh - e.Hq - e.Hkv;
+        dst = static_cast<float*>(is_k ? e.k_dst : e.v_dst) + (((int64_t)b * e.Hkv + gk) * e.cap + e.slot0 + i) * d;
+        void* d2v = is_k ? e.k_dst2 : e.v_dst2;
+        if (d2v) {
+          float* d2 = static_cast<float*>(d2v) + (((int64_t)b * e.Hkv + gk) * e.cap2 + e.slot2 + i) * d;
+          d2[m] = y1;
+          d2[m + half] = y2;
+        }
+      }
+      dst[m] = y1;
+      dst[m + half] = y2;
+    }
+  } else {
+    float* out = static_cast<float*>(e.out);
+    for (int f = threadIdx.x; f < M; f += blockDim.x) {
+      int64_t o = (int64_t)row * e.ldo + f;
+      out[o] = (e.kind == EPI_RESID) ? out[o] + rr[f] : rr[f];
+    }
+  }
+}
+
+size_t gemm_f32_scratch_bytes(int64_t x_rows, int M, int swiglu) {
+  return (size_t)x_rows * (size_t)(swiglu ? 2 * M : M) * sizeof(float);
+}
+
+int gemm_f32_simt(const GemmArgs& a, cudaStream_t s) {
+  DLLM_REQUIRE(a.f32_scratch != nullptr, DLLM_ERR_WORKSPACE, "fp32 projection needs scratch");
+  SimtGroups G{a.n_dev, a.has_extra, a.extra_off, a.extra_cnt, a.host_cnt, a.grp_off, a.grp_cnt, a.cnt_dev};
+  const int n_groups = a.n_dev + a.has_extra + ((a.n_dev + a.has_extra) == 0 ? 1 : 0);
+  const int Mw = a.swiglu ? 2 * a.M : a.M;
+  const int max_cnt = a.cnt_bound > 0 ? a.cnt_bound : 1;
+  dim3 grid((max_cnt + 31) / 32, (Mw + 63) / 64, n_groups);
+  simt_gemm_f32_kernel<<<grid, 256, 0, s>>>((const float*)a.x, (const float*)a.w, (const float*)a.w2, a.K, Mw,
+                                            a.w_group_stride, G, a.f32_scratch);
+  DLLM_CHECK_LAUNCH("simt_gemm_f32_kernel");
+  dim3 g2(max_cnt, n_groups);
+  simt_epilogue_f32_kernel<<<g2, 128, 0, s>>>(a.f32_scratch, Mw, a.M, G, a.epi);
+  DLLM_CHECK_LAUNCH("simt_epilogue_f32_kernel");
+  return DLLM_OK;
+}
+
+}  // namespace dllm

@@ -1,0 +1,77 @@
+// Internal launchers of the helper kernels (not part of the public ABI).
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stddef.h>
+
+namespace dllm {
+
+int launch_embed(int dtype, const int32_t* tokens, const uint8_t* mask, int mask_id, const void* table, void* x,
+                 int rows, int H, cudaStream_t s);
+int launch_rmsnorm(int dtype, const void* x, const void* g, void* out, int rows, int H, float eps,
+                   const int32_t* row_pos, const int32_t* n_dev, int two_halves, int uncond_off, cudaStream_t s);
+int launch_masked_rows(const uint8_t* mask, int n_pos, int halves, int32_t* row_pos, int32_t* n_out,
+                       cudaStream_t s);
+int launch_gather_rows(int dtype, const void* h, const int32_t* perm, int k, int Tk, int shared, void* xp, int H,
+                       cudaStream_t s);
+int launch_combine(int dtype, void* x, const float* y, const float* gates, const int32_t* inv, int k, int Tk,
+                   int shared, int H, cudaStream_t s);
+
+// router
+int num_sms();
+
+int launch_route(int dtype, const void* h, const void* w_router, const float* bias, int Tk, int H, int E, int k,
+                 int32_t* ids, float* gates, float* scores, int32_t* counts, int32_t* offsets, int32_t* perm,
+                 int32_t* inv, cudaStream_t s);
+
+// unmask
+struct UnmaskArgs {
+  int B, L, V, max_rows, t, T_s, mode, k_max, cfg, vocab_offset, dtype;
+  float tau, cfg_scale;
+  const void* logits;
+  const int32_t* row_pos;
+  const int32_t* n_rows;
+  int32_t* tokens;
+  uint8_t* mask;
+  int32_t* sel;
+  int32_t* nsel;
+  float* conf;
+  int32_t* remaining;
+  void* partials;  // workspace: max_rows * n_chunks entries
+  int n_chunks;
+};
+int unmask_chunks(int max_rows, int V);
+size_t unmask_partials_bytes(int max_rows, int n_chunks);
+int launch_unmask(const UnmaskArgs& a, cudaStream_t s);
+
+// attention
+struct AttnArgs {
+  int B, Lq, Hq, Hkv, d, blk_len, q_pos0, n_keys, cap, dtype;
+  float scale;
+  const void* q;
+  const void* k;
+  const void* v;
+  const int32_t* key_pos;
+  void* out;
+  void* ws;
+  size_t ws_bytes;
+};
+size_t attn_workspace_bytes(int B, int Lq, int Hq, int Hkv, int d, int n_keys);
+int launch_attn(const AttnArgs& a, cudaStream_t s);
+
+// SPRINT retention
+struct RetainArgs {
+  int B, Hkv, d, P, cap, n_keep, cap_thin, dtype;
+  const void* k;
+  const void* v;
+  int32_t* keep_pos;
+  void* k_thin;
+  void* v_thin;
+  float* scores;
+  float* raw;  // workspace [B, P]
+  int block_len;  // > 0: also write keep_pos[n_keep + i] = P + i for i < block_len
+};
+size_t retain_workspace_bytes(int B, int P);
+int launch_retain(const RetainArgs& a, cudaStream_t s);
+
+}  // namespace dllm

@@ -1,0 +1,248 @@
+// Confidence and unmasking: vocabulary-wide max / arg-max / sum-of-exponentials per still-masked position
+// (optionally on classifier-free-guided logits), then per block row the choice of the positions to unmask.
+// Source: LLaDA2.0-Uni paper review, section "SPRINT — 학습 없는 추론 가속" (c_i = max_v p(v | x_t); accept every
+// position with c above tau, at least ceil(m / (T - t)) per step; the standard schedule ceil(m / T)), and the
+// HF-mirror README, section "SPRINT 加速技术" (k = ceil(remaining / steps_left); batch acceptance above the
+// threshold).
+//
+// Reduction: one CTA per (row, vocabulary chunk); 256 threads stream the chunk with 16-byte non-allocating
+// loads, keep a running (max, lowest arg-max, sum of exp(z - max)) per thread (sum in fp64, exponentials in
+// fp32), merge in registers and shared memory and write one partial per CTA. Selection: one warp per block row
+// merges its rows' partials, computes c = 1 / sum, counts, ranks and writes tokens, mask and the step outputs.
+#include "common.cuh"
+#include "misc.h"
+
+namespace dllm {
+namespace {
+
+struct Partial {
+  float m;    // max logit
+  int idx;    // lowest index attaining m (absolute vocabulary index within the scored slice)
+  double s;   // sum over the chunk of exp(z - m)
+};
+
+DLLM_DEV void merge(Partial& a, const Partial& b) {
+  if (b.s == 0.0) return;
+  if (a.s == 0.0) { a = b; return; }
+  if (b.m > a.m || (b.m == a.m && b.idx < a.idx)) {
+    double f = (b.m == a.m) ? 1.0 : exp((double)a.m - (double)b.m);
+    a.s = a.s * f + b.s;
+    a.m = b.m;
+    a.idx = b.idx;
+  } else {
+    double f = (b.m == a.m) ? 1.0 : exp((double)b.m - (double)a.m);
+    a.s = a.s + b.s * f;
+  }
+}
+
+DLLM_DEV float guided(float zc, float zu, float s) {
+  // z = zu + s * (zc - zu), each operation rounded to fp32 in this order (no contraction)
+  return __fadd_rn(zu, __fmul_rn(s, __fsub_rn(zc, zu)));
+}
+
+// Running update of one thread's partial with 8 consecutive values starting at vocabulary index v.
+DLLM_DEV void update8(Partial& p, const float* z, int v) {
+  float vm = z[0];
+  int vi = 0;
+#pragma unroll
+  for (int u = 1; u < 8; ++u)
+    if (z[u] > vm) { vm = z[u]; vi = u; }
+  if (p.s == 0.0 || vm > p.m) {
+    p.s = (p.s == 0.0) ? 0.0 : p.s * exp((double)p.m - (double)vm);
+    p.m = vm;
+    p.idx = v + vi;
+  }
+  float acc = 0.f;
+#pragma unroll
+  for (int u = 0; u < 8; ++u) acc += expf(z[u] - p.m);
+  p.s += (double)acc;
+}
+
+DLLM_DEV void load8f(const __nv_bfloat16* p, float* f) { bf16x8_to_f32(ld_nc_v4(p), f); }
+DLLM_DEV void load8f(const float* p, float* f) {
+  uint4 a = ld_nc_v4(p), b = ld_nc_v4(p + 4);
+  f[0] = __uint_as_float(a.x); f[1] = __uint_as_float(a.y); f[2] = __uint_as_float(a.z); f[3] = __uint_as_float(a.w);
+  f[4] = __uint_as_float(b.x); f[5] = __uint_as_float(b.y); f[6] = __uint_as_float(b.z); f[7] = __uint_as_float(b.w);
+}
+
+template <typename T, bool CFG>
+__global__ void __launch_bounds__(256) unmask_reduce_kernel(const T* __restrict__ logits,
+                                                            const int32_t* __restrict__ n_rows, int V, int chunk,
+                                                            float cfg_scale, Partial* __restrict__ part,
+                                                            int n_chunks) {
+  const int r = blockIdx.x, c = blockIdx.y;
+  const int n = *n_rows;
+  if (r >= n) return;
+  const T* zc = logits + (int64_t)r * V;
+  const T* zu = logits + (int64_t)(r + n) * V;
+  const int v0 = c * chunk, v1 = min(V, v0 + chunk);
+  Partial p{-INFINITY, 0x7fffffff, 0.0};
+  const int nvec = (v1 - v0) >> 3;
+  const bool vec_ok = ((V * (int)sizeof(T)) % 16 == 0) && (v0 % 8 == 0);
+  if (vec_ok) {
+    int i = threadIdx.x;
+    // two vectors in flight per thread per iteration
+    for (; i + 256 < nvec; i += 512) {
+      float a[8], b[8];
+      load8f(zc + v0 + i * 8, a);
+      load8f(zc + v0 + (i + 256) * 8, b);
+      if (CFG) {
+        float ua[8], ub[8];
+        load8f(zu + v0 + i * 8, ua);
+        load8f(zu + v0 + (i + 256) * 8, ub);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) { a[u] = guided(a[u], ua[u], cfg_scale); b[u] = guided(b[u], ub[u], cfg_scale); }
+      }
+      update8(p, a, v0 + i * 8);
+      update8(p, b, v0 + (i + 256) * 8);
+    }
+    for (; i < nvec; i += 256) {
+      float a[8];
+      load8f(zc + v0 + i * 8, a);
+      if (CFG) {
+        float ua[8];
+        load8f(zu + v0 + i * 8, ua);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) a[u] = guided(a[u], ua[u], cfg_scale);
+      }
+      update8(p, a, v0 + i * 8);
+    }
+  }
+  // scalar part: the whole chunk when vector loads are not possible, else the tail
+  for (int v = v0 + (vec_ok ? nvec * 8 : 0) + threadIdx.x; v < v1; v += 256) {
+    float z = to_f32(zc[v]);
+    if (CFG) z = guided(z, to_f32(zu[v]), cfg_scale);
+    Partial q{z, v, 1.0};
+    merge(p, q);
+  }
+  // warp merge then block merge
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    Partial q;
+    q.m = __shfl_xor_sync(0xffffffffu, p.m, o);
+    q.idx = __shfl_xor_sync(0xffffffffu, p.idx, o);
+    q.s = __shfl_xor_sync(0xffffffffu, p.s, o);
+    merge(p, q);
+  }
+  __shared__ Partial wp[8];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  if (lane == 0) wp[w] = p;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    Partial a = wp[0];
+    for (int i = 1; i < 8; ++i) merge(a, wp[i]);
+    part[(int64_t)r * n_chunks + c] = a;
+  }
+}
+
+// One warp per logical block row b (L <= 32 positions, lane i = position i).
+__global__ void unmask_select_kernel(const Partial* __restrict__ part, int n_chunks, const int32_t* __restrict__ row_pos,
+                                     const int32_t* __restrict__ n_rows, int B, int L, int t, int T_s, int mode,
+                                     float tau, int k_max, int cfg, int vocab_offset, int32_t* tokens, uint8_t* mask,
+                                     int32_t* sel, int32_t* nsel, float* conf, int32_t* remaining) {
+  __shared__ int rem_w[32];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int n = *n_rows;
+  int rem_acc = 0;
+  for (int b = w; b < B; b += nw) {
+    const int p = b * L + lane;
+    const bool valid = lane < L;
+    const bool masked = valid && mask[p] != 0;
+    double c = 0.0;
+    int cand = -1;
+    if (masked) {
+      int lo = 0, hi = n - 1;  // row_pos is ascending: find r with row_pos[r] == p
+      while (lo < hi) {
+        int mid = (lo + hi) >> 1;
+        if (row_pos[mid] < p) lo = mid + 1; else hi = mid;
+      }
+      Partial a{-INFINITY, 0x7fffffff, 0.0};
+      for (int q = 0; q < n_chunks; ++q) merge(a, part[(int64_t)lo * n_chunks + q]);
+      c = 1.0 / a.s;
+      cand = a.idx + vocab_offset;
+    }
+    const unsigned mball = __ballot_sync(0xffffffffu, masked);
+    const int m = __popc(mball);
+    int kt = 0;
+    if (m > 0) {
+      const int floor_k = (m + (T_s - t) - 1) / (T_s - t);
+      if (mode == DLLM_UNMASK_FIXED) {
+        kt = min(m, floor_k);
+      } else {
+        const int above = __popc(__ballot_sync(0xffffffffu, masked && c > (double)tau));
+        kt = min(m, max(floor_k, min(k_max, above)));
+      }
+    }
+    // rank among masked positions: higher confidence first, lower position on equal confidence
+    int rank = 0;
+    for (int j = 0; j < 32; ++j) {
+      const double cj = __shfl_sync(0xffffffffu, c, j);
+      if (((mball >> j) & 1u) && (cj > c || (cj == c && j < lane))) ++rank;
+    }
+    const bool chosen = masked && rank < kt;
+    if (valid) {
+      sel[b * L + lane] = -1;
+      conf[b * L + lane] = masked ? (float)c : 0.f;
+    }
+    __syncwarp();
+    if (chosen) {
+      sel[b * L + rank] = lane;
+      tokens[p] = cand;
+      mask[p] = 0;
+      if (cfg) {
+        tokens[p + B * L] = cand;
+        mask[p + B * L] = 0;
+      }
+    }
+    if (lane == 0) {
+      nsel[b] = kt;
+      rem_acc += m - kt;
+    }
+  }
+  if (lane == 0) rem_w[w] = rem_acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int s = 0;
+    for (int i = 0; i < nw; ++i) s += rem_w[i];
+    *remaining = s;
+  }
+}
+
+}  // namespace
+
+int unmask_chunks(int max_rows, int V) {
+  // enough CTAs to cover the SMs a few times when every row is masked, chunks of at least 2048 entries
+  int want = (4 * num_sms() + max(max_rows, 1) - 1) / max(max_rows, 1);
+  int most = max(1, V / 2048);
+  return max(1, min(want, min(most, 64)));
+}
+
+size_t unmask_partials_bytes(int max_rows, int n_chunks) {
+  return (size_t)max(max_rows, 1) * (size_t)n_chunks * sizeof(Partial);
+}
+
+int launch_unmask(const UnmaskArgs& a, cudaStream_t s) {
+  const int chunk = ((a.V + a.n_chunks - 1) / a.n_chunks + 7) & ~7;
+  if (a.max_rows > 0) {
+    dim3 grid(a.max_rows, a.n_chunks);
+    Partial* part = static_cast<Partial*>(a.partials);
+    if (a.dtype == DLLM_BF16) {
+      const __nv_bfloat16* z = static_cast<const __nv_bfloat16*>(a.logits);
+      if (a.cfg) unmask_reduce_kernel<__nv_bfloat16, true><<<grid, 256, 0, s>>>(z, a.n_rows, a.V, chunk, a.cfg_scale, part, a.n_chunks);
+      else unmask_reduce_kernel<__nv_bfloat16, false><<<grid, 256, 0, s>>>(z, a.n_rows, a.V, chunk, a.cfg_scale, part, a.n_chunks);
+    } else {
+      const float* z = static_cast<const float*>(a.logits);
+      if (a.cfg) unmask_reduce_kernel<float, true><<<grid, 256, 0, s>>>(z, a.n_rows, a.V, chunk, a.cfg_scale, part, a.n_chunks);
+      else unmask_reduce_kernel<float, false><<<grid, 256, 0, s>>>(z, a.n_rows, a.V, chunk, a.cfg_scale, part, a.n_chunks);
+    }
+    DLLM_CHECK_LAUNCH("unmask_reduce_kernel");
+  }
+  const int threads = 32 * min(32, max(1, a.B));
+  unmask_select_kernel<<<1, threads, 0, s>>>(static_cast<const Partial*>(a.partials), a.n_chunks, a.row_pos, a.n_rows,
+                                             a.B, a.L, a.t, a.T_s, a.mode, a.tau, a.k_max, a.cfg, a.vocab_offset,
+                                             a.tokens, a.mask, a.sel, a.nsel, a.conf, a.remaining);
+  DLLM_CHECK_LAUNCH("unmask_select_kernel");
+  return DLLM_OK;
+}
+
+}  // namespace dllm

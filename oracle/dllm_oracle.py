@@ -137,14 +137,16 @@ def prefix_scores(k_prefix):
     return l / l.mean()
 
 
-def prefix_retain(k_prefix, ratio):
-    """Kept prefix positions, in position order: the ceil(ratio * P) largest l~_i, ties -> lower position.
+def prefix_retain(k_prefix, ratio, n_keep=None):
+    """Kept prefix positions, in position order: the ceil(ratio * P) largest l~_i (or n_keep of them when
+    given), ties -> lower position.
 
     Returns (keep_pos [n_keep] int64, scores [P], margin) where margin is the score gap between the last kept
     and the first dropped position (inf when nothing is dropped)."""
     sc = prefix_scores(k_prefix)
     P = sc.shape[0]
-    n_keep = int(math.ceil(ratio * P))
+    if n_keep is None:
+        n_keep = int(math.ceil(ratio * P))
     order = sorted(range(P), key=lambda i: (-sc[i], i))
     keep = np.array(sorted(order[:n_keep]), dtype=np.int64)
     margin = sc[order[n_keep - 1]] - sc[order[n_keep]] if n_keep < P else np.inf

@@ -1,0 +1,55 @@
+"""Helpers shared by the GPU parity tests (comparison criteria and small input builders)."""
+import numpy as np
+import torch
+
+# float tolerances of the parity bar: bf16 storage -> max-abs <= 2e-2 and relative L2 <= 5e-3; fp32 -> 1e-4.
+# A bf16 value whose magnitude exceeds 2.56 has a rounding step (one ulp, 2^-7 relative) above 2e-2: there the
+# per-element bound is one ulp of the value, since both sides round a result that differs by ~1e-6 relative
+# to the nearest bf16 and may land on the two neighbours of a rounding boundary.
+TOL = {"bf16": (2e-2, 5e-3), "f32": (1e-4, 1e-4)}
+
+
+def to64(t):
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def assert_close(got, want, dtype, what=""):
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    assert got.shape == want.shape, (what, got.shape, want.shape)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite values"
+    abs_tol, rel_tol = TOL[dtype]
+    err = np.abs(got - want)
+    max_abs = float(err.max()) if err.size else 0.0
+    rel_l2 = float(np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-30))
+    if dtype == "f32":
+        # fp32: 1e-4 absolute or relative per element
+        bad = err > abs_tol * np.maximum(1.0, np.abs(want))
+        assert not bad.any(), f"{what}: {int(bad.sum())} elements beyond 1e-4 (max abs {max_abs:.3g})"
+    else:
+        bound = np.maximum(abs_tol, np.abs(want) * 2.0 ** -7)
+        bad = err > bound
+        assert not bad.any(), (f"{what}: {int(bad.sum())} elements beyond max(2e-2, one bf16 ulp); "
+                               f"max-abs {max_abs:.4g}")
+        assert rel_l2 <= rel_tol, f"{what}: rel-L2 {rel_l2:.4g} > {rel_tol}"
+    return max_abs, rel_l2
+
+
+def assignment_tables(ids, E):
+    """counts, offsets, perm, inv of the (token, slot) assignments grouped by expert, stable in token order."""
+    T, k = ids.shape
+    flat = ids.reshape(-1)
+    counts = np.bincount(flat, minlength=E).astype(np.int32)
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    perm = np.argsort(flat, kind="stable").astype(np.int32)
+    inv = np.empty_like(perm)
+    inv[perm] = np.arange(len(perm), dtype=np.int32)
+    return counts, offsets, perm, inv
+
+
+def random_assignments(T, E, k, seed):
+    g = np.random.default_rng(seed)
+    ids = np.stack([g.choice(E, k, replace=False) for _ in range(T)]).astype(np.int32)
+    gates = g.uniform(0.1, 1.0, (T, k)).astype(np.float32)
+    gates = (gates / gates.sum(1, keepdims=True)).astype(np.float32)
+    return ids, gates

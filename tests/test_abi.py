@@ -1,0 +1,125 @@
+"""The C-ABI library: it loads, exports every entry point include/dllm.h declares, and rejects bad arguments on
+the host before touching the GPU (these calls launch nothing, so they run without a GPU)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from block_diffusion_moe_dllm_b200 import binding as bd
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dllm.h")
+
+
+def _declared():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"DLLM_API\s+[\w\s\*]+?\b(dllm_\w+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(bd.LIB_PATH):
+        from block_diffusion_moe_dllm_b200 import build
+        build.build()
+    return bd.load()
+
+
+def test_library_exports_every_declared_symbol(lib):
+    declared = _declared()
+    assert len(declared) >= 17
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert sorted(bd.EXPORTED) == declared
+
+
+def test_exports_nothing_else():
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", bd.LIB_PATH], capture_output=True, text=True).stdout
+    funcs = sorted(l.split()[-1] for l in out.splitlines() if " T " in l)
+    assert funcs == _declared()
+
+
+def test_version(lib):
+    assert "sm_100a" in lib.dllm_version().decode()
+
+
+FAKE = 0x10000  # never dereferenced: every call below fails validation first
+
+
+def test_gemm_rejects_bad_arguments(lib):
+    d = bd.GemmDesc(32, 128, 64, 128, bd.BF16, 0, 0)
+    assert lib.dllm_gemm(C.byref(d), None, FAKE, FAKE, None, FAKE, 1 << 20, None) == bd.ERR_INVALID_ARG
+    d.K = 0
+    assert lib.dllm_gemm(C.byref(d), FAKE, FAKE, FAKE, None, FAKE, 1 << 20, None) == bd.ERR_SHAPE
+    d.K = 64
+    assert lib.dllm_gemm(C.byref(d), FAKE, FAKE, FAKE, None, None, 1 << 20, None) == bd.ERR_WORKSPACE
+    assert lib.dllm_gemm(C.byref(d), FAKE, FAKE, FAKE, None, FAKE + 8, 1 << 20, None) == bd.ERR_WORKSPACE
+    assert lib.dllm_gemm(C.byref(d), FAKE, FAKE, FAKE, None, FAKE, 16, None) == bd.ERR_WORKSPACE
+    d.K = 96
+    assert lib.dllm_gemm(C.byref(d), FAKE, FAKE, FAKE, None, FAKE, 1 << 20, None) == bd.ERR_UNSUPPORTED
+    d.K = 64
+    assert lib.dllm_gemm(C.byref(d), FAKE + 2, FAKE, FAKE, None, FAKE, 1 << 20, None) == bd.ERR_ALIGN
+    assert "aligned" in lib.dllm_last_error().decode()
+
+
+def test_attention_rejects_bad_arguments(lib):
+    d = bd.AttnDesc(1, 32, 16, 4, 128, 32, 1024, 1056, 1056, bd.BF16, 0.0)
+    d.Hq = 15
+    assert lib.dllm_block_attn(C.byref(d), FAKE, FAKE, FAKE, None, FAKE, FAKE, 1 << 30, None) == bd.ERR_SHAPE
+    d.Hq = 16
+    d.cap = 100
+    assert lib.dllm_block_attn(C.byref(d), FAKE, FAKE, FAKE, None, FAKE, FAKE, 1 << 30, None) == bd.ERR_SHAPE
+    d.cap = 1056
+    d.d = 64
+    assert lib.dllm_block_attn(C.byref(d), FAKE, FAKE, FAKE, None, FAKE, FAKE, 1 << 30, None) == bd.ERR_UNSUPPORTED
+
+
+def test_route_and_experts_reject_bad_arguments(lib):
+    r = bd.RouteDesc(32, 2048, 2048, 8, bd.BF16)
+    args = [FAKE] * 9
+    assert lib.dllm_moe_route(C.byref(r), *args, None, FAKE, 1 << 30, None) == bd.ERR_UNSUPPORTED
+    r.E, r.k = 256, 300
+    assert lib.dllm_moe_route(C.byref(r), *args, None, FAKE, 1 << 30, None) == bd.ERR_UNSUPPORTED
+    e = bd.ExpertDesc(32, 2048, 256, 8, 512, bd.BF16)
+    # one shared weight without the other
+    assert lib.dllm_moe_experts(C.byref(e), FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                FAKE, 1 << 30, None) == bd.ERR_INVALID_ARG
+    e.I = 500
+    assert lib.dllm_moe_experts(C.byref(e), *([FAKE] * 11), FAKE, 1 << 30, None) == bd.ERR_UNSUPPORTED
+
+
+def test_unmask_rejects_bad_arguments(lib):
+    u = bd.UnmaskDesc(1, 64, 1024, 64, 0, 8, bd.FIXED, 0.9, 8, 0, 1.0, 0, bd.BF16)
+    assert lib.dllm_unmask(C.byref(u), *([FAKE] * 10), FAKE, 1 << 30, None) == bd.ERR_SHAPE   # L > 32
+    u.L, u.max_rows, u.t = 32, 32, 8
+    assert lib.dllm_unmask(C.byref(u), *([FAKE] * 10), FAKE, 1 << 30, None) == bd.ERR_INVALID_ARG  # t >= T_s
+
+
+def test_retain_rejects_bad_arguments(lib):
+    d = bd.RetainDesc(8, 4, 128, 4096, 4128, 0, 2080, bd.BF16)
+    assert lib.dllm_prefix_retain(C.byref(d), *([FAKE] * 6), FAKE, 1 << 30, None) == bd.ERR_SHAPE
+    d.n_keep, d.P, d.cap = 2048, 9000, 9100
+    assert lib.dllm_prefix_retain(C.byref(d), *([FAKE] * 6), FAKE, 1 << 30, None) == bd.ERR_UNSUPPORTED
+
+
+def test_step_rejects_bad_model(lib):
+    layers = (bd.Layer * 1)()
+    m = bd.Model(1, 2048, 16, 4, 128, 256, 8, 512, 157184, bd.BF16, 1e-6, 1e4, 0, FAKE, FAKE, FAKE, layers)
+    st = bd.State(1, 32, 1024, 1056, 0, FAKE, FAKE)
+    p = bd.StepParams(0, 8, 0, 0.9, 8, 0, 1.0, 0, 0, 0, 0, 0, 0, FAKE, FAKE, FAKE, FAKE)
+    # layer 0 has NULL weights
+    assert lib.dllm_denoise_step(C.byref(m), C.byref(st), C.byref(p), FAKE, 1 << 40, None) == bd.ERR_INVALID_ARG
+    assert lib.dllm_denoise_step_workspace_size(C.byref(m), C.byref(st), C.byref(p)) == 0
+    for name in ("attn_norm", "w_qkv", "w_o", "ffn_norm", "w_router", "router_bias", "w_gu", "w_down",
+                 "w_gu_shared", "w_down_shared", "k_cache", "v_cache"):
+        setattr(layers[0], name, FAKE)
+    assert lib.dllm_denoise_step_workspace_size(C.byref(m), C.byref(st), C.byref(p)) > 0
+    st.L = 40
+    assert lib.dllm_denoise_step(C.byref(m), C.byref(st), C.byref(p), FAKE, 1 << 40, None) == bd.ERR_SHAPE
+    st.L = 32
+    p.t = 9
+    assert lib.dllm_denoise_step(C.byref(m), C.byref(st), C.byref(p), FAKE, 1 << 40, None) == bd.ERR_INVALID_ARG
+    p.t = 0
+    m.d = 64
+    assert lib.dllm_denoise_step(C.byref(m), C.byref(st), C.byref(p), FAKE, 1 << 40, None) == bd.ERR_UNSUPPORTED

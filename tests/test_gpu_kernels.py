@@ -1,0 +1,286 @@
+"""Per-call parity of the CUDA library against the fp64 oracle on seeded inputs (GPU)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from block_diffusion_moe_dllm_b200 import binding as bd
+from block_diffusion_moe_dllm_b200 import synth
+from oracle import dllm_oracle as O
+from _util import TOL, assert_close, assignment_tables, random_assignments, to64
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+DT = {"bf16": bd.BF16, "f32": bd.F32}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    bd.load()
+
+
+def _tdt(name):
+    return synth.torch_dtype(name)
+
+
+# ------------------------------------------------------------------------------------------------ GEMM
+@pytest.mark.parametrize("N,M,K", [(1, 128, 64), (5, 256, 128), (32, 384, 2048), (77, 256, 512), (200, 128, 256),
+                                   (300, 256, 192), (513, 128, 64)])
+def test_gemm_bf16_store(N, M, K):
+    x = synth.normal((N, K), 1.0, 1, f"gx{N}", DEV)
+    w = synth.normal((M, K), 0.05, 1, f"gw{M}{K}", DEV)
+    y = torch.full((N, M), float("nan"), dtype=torch.bfloat16, device=DEV)
+    bd.gemm(x, w, y, N, M, K, bd.BF16)
+    torch.cuda.synchronize()
+    want = O.store(to64(x) @ to64(w).T, "bf16")
+    assert_close(to64(y), want, "bf16", "gemm")
+
+
+def test_gemm_bf16_residual_and_device_count():
+    N, M, K = 40, 256, 256
+    x = synth.normal((N, K), 1.0, 2, "rx", DEV)
+    w = synth.normal((M, K), 0.05, 2, "rw", DEV)
+    y0 = synth.normal((N, M), 1.0, 2, "ry", DEV)
+    y = y0.clone()
+    n_dev = torch.tensor([33], dtype=torch.int32, device=DEV)
+    bd.gemm(x, w, y, N, M, K, bd.BF16, residual=1, n_rows_dev=n_dev)
+    torch.cuda.synchronize()
+    want = O.store(to64(y0)[:33] + to64(x)[:33] @ to64(w).T, "bf16")
+    assert_close(to64(y)[:33], want, "bf16", "gemm residual")
+    assert torch.equal(y[33:], y0[33:]), "rows past the device count must be untouched"
+
+
+def test_gemm_bf16_f32_output():
+    N, M, K = 17, 128, 320
+    x = synth.normal((N, K), 1.0, 3, "fx", DEV)
+    w = synth.normal((M, K), 0.05, 3, "fw", DEV)
+    y = torch.zeros((N, M), dtype=torch.float32, device=DEV)
+    bd.gemm(x, w, y, N, M, K, bd.BF16, y_f32=1)
+    torch.cuda.synchronize()
+    want = to64(x) @ to64(w).T
+    assert np.max(np.abs(to64(y) - want)) < 1e-4
+
+
+def test_gemm_f32():
+    N, M, K = 23, 100, 70
+    x = synth.normal((N, K), 1.0, 4, "sx", DEV, torch.float32)
+    w = synth.normal((M, K), 0.05, 4, "sw", DEV, torch.float32)
+    y = torch.zeros((N, M), dtype=torch.float32, device=DEV)
+    bd.gemm(x, w, y, N, M, K, bd.F32)
+    torch.cuda.synchronize()
+    assert_close(to64(y), to64(x) @ to64(w).T, "f32", "gemm f32")
+
+
+# ------------------------------------------------------------------------------------------------ router
+@pytest.mark.parametrize("dtype,Tk,H,E,k", [("bf16", 1, 2048, 256, 8), ("bf16", 32, 2048, 256, 8),
+                                            ("bf16", 77, 2048, 256, 8), ("bf16", 512, 2048, 256, 8),
+                                            ("f32", 16, 256, 8, 2), ("bf16", 9, 256, 1024, 32)])
+def test_route(dtype, Tk, H, E, k):
+    t = _tdt(dtype)
+    h = synth.normal((Tk, H), 1.0, 5, f"rh{Tk}", DEV, t)
+    wr = synth.normal((E, H), 0.02, 5, f"rw{E}", DEV, t)
+    bias = synth.uniform((E,), -0.1, 0.1, 5, f"rb{E}", DEV)
+    ids = torch.empty((Tk, k), dtype=torch.int32, device=DEV)
+    gates = torch.empty((Tk, k), dtype=torch.float32, device=DEV)
+    counts = torch.empty(E, dtype=torch.int32, device=DEV)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=DEV)
+    perm = torch.empty(Tk * k, dtype=torch.int32, device=DEV)
+    inv = torch.empty(Tk * k, dtype=torch.int32, device=DEV)
+    scores = torch.empty((Tk, E), dtype=torch.float32, device=DEV)
+    bd.moe_route(h, wr, bias, ids, gates, counts, offsets, perm, inv, Tk, H, E, k, DT[dtype], scores=scores)
+    torch.cuda.synchronize()
+    o_ids, o_gates, o_s, margin = O.route(to64(h), to64(wr), to64(bias), k)
+    g_ids = ids.cpu().numpy()
+    assert np.max(np.abs(to64(scores) - o_s)) < 2e-6
+    flagged = margin < 1e-6
+    exact = ~flagged
+    assert np.array_equal(g_ids[exact], o_ids[exact]), "routed expert ids differ away from near-ties"
+    assert np.allclose(gates.cpu().numpy()[exact], o_gates[exact], rtol=2e-6, atol=2e-7)
+    # permutation tables are exactly those of the GPU's ids
+    c, off, p, iv = assignment_tables(g_ids, E)
+    assert np.array_equal(counts.cpu().numpy(), c)
+    assert np.array_equal(offsets.cpu().numpy(), off)
+    assert np.array_equal(perm.cpu().numpy(), p)
+    assert np.array_equal(inv.cpu().numpy(), iv)
+
+
+# ------------------------------------------------------------------------------------------------ experts
+@pytest.mark.parametrize("dtype,Tk,H,E,k,I,shared", [("bf16", 32, 2048, 256, 8, 512, True),
+                                                     ("bf16", 5, 256, 16, 4, 128, True),
+                                                     ("bf16", 70, 256, 8, 2, 192, False),
+                                                     ("bf16", 300, 256, 4, 2, 64, True),
+                                                     ("f32", 16, 256, 8, 2, 128, True)])
+def test_experts(dtype, Tk, H, E, k, I, shared):
+    t = _tdt(dtype)
+    h = synth.normal((Tk, H), 1.0, 6, "eh", DEV, t)
+    x0 = synth.normal((Tk, H), 1.0, 6, "ex", DEV, t)
+    wgu = synth.normal((E, 2 * I, H), 0.02, 6, "egu", DEV, t)
+    wd = synth.normal((E, H, I), 0.02, 6, "ed", DEV, t)
+    sgu = synth.normal((2 * I, H), 0.02, 6, "sgu", DEV, t) if shared else None
+    sd = synth.normal((H, I), 0.02, 6, "sd", DEV, t) if shared else None
+    ids, gates = random_assignments(Tk, E, k, seed=Tk + E)
+    counts, offsets, perm, inv = assignment_tables(ids, E)
+    cvt = lambda a: torch.from_numpy(a).to(DEV)
+    x = x0.clone()
+    bd.moe_experts(h, wgu, wd, sgu, sd, cvt(counts), cvt(offsets), cvt(perm), cvt(inv), cvt(gates), x, Tk, H, E, k,
+                   I, DT[dtype])
+    torch.cuda.synchronize()
+    delta = O.moe_delta(to64(h), ids, gates.astype(np.float64), to64(wgu), to64(wd),
+                        to64(sgu) if shared else None, to64(sd) if shared else None, dtype)
+    want = O.store(to64(x0) + delta, dtype)
+    assert_close(to64(x), want, dtype, "experts")
+
+
+# ------------------------------------------------------------------------------------------------ attention
+def _attn_case(dtype, B, Lq, Hq, Hkv, d, blk, q_pos0, n_keys, cap, key_pos=None, seed=0):
+    t = _tdt(dtype)
+    q = synth.normal((B, Lq, Hq, d), 1.0, seed, "aq", DEV, t)
+    kc = synth.normal((B, Hkv, cap, d), 1.0, seed, "ak", DEV, t)
+    vc = synth.normal((B, Hkv, cap, d), 1.0, seed, "av", DEV, t)
+    out = torch.full((B, Lq, Hq * d), float("nan"), dtype=t, device=DEV)
+    kp = None if key_pos is None else torch.from_numpy(key_pos.astype(np.int32)).to(DEV)
+    bd.block_attn(q, kc, vc, out, B, Lq, Hq, Hkv, d, blk, q_pos0, n_keys, cap, DT[dtype], key_pos=kp)
+    torch.cuda.synchronize()
+    got = to64(out).reshape(B, Lq, Hq, d)
+    for b in range(B):
+        kpos = np.arange(n_keys) if key_pos is None else key_pos[b]
+        want = O.store(O.attention(to64(q[b]), to64(kc[b, :, :n_keys]).transpose(1, 0, 2),
+                                   to64(vc[b, :, :n_keys]).transpose(1, 0, 2), np.arange(q_pos0, q_pos0 + Lq), kpos,
+                                   blk), dtype)
+        assert_close(got[b], want, dtype, f"attention row {b}")
+
+
+def test_attention_decode_block():
+    P, L = 1024, 32
+    _attn_case("bf16", 1, L, 16, 4, 128, L, P, P + L, P + L)
+
+
+def test_attention_decode_ragged_prefix_batch():
+    P, L = 100, 32
+    _attn_case("bf16", 3, L, 16, 4, 128, L, P, P + L, P + L + 5, seed=1)
+
+
+def test_attention_thinned_prefix():
+    P, L, n_keep, B = 300, 32, 150, 2
+    g = np.random.default_rng(7)
+    kp = np.stack([np.concatenate([np.sort(g.choice(P, n_keep, replace=False)), np.arange(P, P + L)])
+                   for _ in range(B)])
+    _attn_case("bf16", B, L, 16, 4, 128, L, P, n_keep + L, n_keep + L + 8, key_pos=kp, seed=2)
+
+
+def test_attention_prefill_block_causal():
+    _attn_case("bf16", 2, 96, 16, 4, 128, 32, 0, 96, 96, seed=3)
+
+
+def test_attention_ragged_queries_small_blocks():
+    _attn_case("bf16", 1, 70, 8, 2, 128, 16, 0, 70, 80, seed=4)
+
+
+def test_attention_long_prefix_split():
+    _attn_case("bf16", 2, 32, 16, 4, 128, 32, 4096, 4128, 4128, seed=5)
+
+
+def test_attention_f32_mha():
+    _attn_case("f32", 1, 16, 4, 4, 64, 16, 64, 80, 80, seed=6)
+
+
+# ------------------------------------------------------------------------------------------------ SPRINT
+@pytest.mark.parametrize("B,P,n_keep,cap_thin", [(2, 300, 150, 170), (1, 4096, 2048, 2080), (3, 64, 64, 64),
+                                                 (1, 33, 1, 8)])
+def test_prefix_retain(B, P, n_keep, cap_thin):
+    Hkv, d = 4, 128
+    cap = P + 16
+    kc = synth.normal((B, Hkv, cap, d), 1.0, 8, "pk", DEV)
+    vc = synth.normal((B, Hkv, cap, d), 1.0, 8, "pv", DEV)
+    if P > 20:
+        kc[:, :, 7] = kc[:, :, 3]          # exact ties: the lower position must win
+        kc[:, :, 19] = kc[:, :, 3]
+    keep = torch.full((B, cap_thin), -1, dtype=torch.int32, device=DEV)
+    kt = torch.zeros((B, Hkv, cap_thin, d), dtype=torch.bfloat16, device=DEV)
+    vt = torch.zeros_like(kt)
+    sc = torch.zeros((B, P), dtype=torch.float32, device=DEV)
+    bd.prefix_retain(kc, vc, keep, kt, vt, B, Hkv, d, P, cap, n_keep, cap_thin, bd.BF16, scores=sc)
+    torch.cuda.synchronize()
+    for b in range(B):
+        o_keep, o_sc, margin = O.prefix_retain(to64(kc[b, :, :P]), None, n_keep=n_keep)
+        assert len(o_keep) == n_keep
+        g_keep = keep[b, :n_keep].cpu().numpy()
+        assert np.allclose(to64(sc[b]), o_sc, rtol=2e-6)
+        if margin > 1e-6 * np.max(o_sc):
+            assert np.array_equal(g_keep, o_keep)
+        assert np.all(np.diff(g_keep) > 0)
+        idx = torch.from_numpy(g_keep.astype(np.int64)).to(DEV)
+        assert torch.equal(kt[b, :, :n_keep], kc[b][:, idx]) and torch.equal(vt[b, :, :n_keep], vc[b][:, idx])
+
+
+# ------------------------------------------------------------------------------------------------ unmask
+def _unmask_case(B, L, V, masked_frac, t, T_s, mode, std, cfg=False, scale=2.0, tau=0.9, k_max=8, voff=0,
+                 dtype="bf16", seed=0):
+    g = np.random.default_rng(seed)
+    Btot = 2 * B if cfg else B
+    mask = (g.uniform(size=(B, L)) < masked_frac).astype(np.uint8)
+    mask[0, 0] = 1
+    if cfg:
+        mask = np.concatenate([mask, mask])
+    tokens = np.where(mask == 1, V - 1, g.integers(0, V, (Btot, L))).astype(np.int32)
+    row_pos = np.nonzero(mask[:B].reshape(-1))[0].astype(np.int32)
+    n = len(row_pos)
+    t_dt = _tdt(dtype)
+    logits = synth.normal(((2 if cfg else 1) * n, V), std, seed, f"ul{V}", DEV, t_dt)
+    dm = torch.from_numpy(mask).to(DEV)
+    dt_ = torch.from_numpy(tokens).to(DEV)
+    sel = torch.empty((B, L), dtype=torch.int32, device=DEV)
+    nsel = torch.empty(B, dtype=torch.int32, device=DEV)
+    conf = torch.empty((B, L), dtype=torch.float32, device=DEV)
+    rem = torch.empty(1, dtype=torch.int32, device=DEV)
+    rp = torch.from_numpy(np.concatenate([row_pos, np.zeros(B * L - n, np.int32)])).to(DEV)
+    nd = torch.tensor([n], dtype=torch.int32, device=DEV)
+    bd.unmask(logits, rp, nd, dt_, dm, sel, nsel, conf, rem, B, L, V, B * L, t, T_s, DT[dtype], mode=mode, tau=tau,
+              k_max=k_max, cfg=int(cfg), cfg_scale=scale, vocab_offset=voff)
+    torch.cuda.synchronize()
+    zl = to64(logits)
+    u = O.unmask(zl[:n], row_pos, tokens, mask, t, T_s, mode, float(np.float32(tau)), k_max, voff,
+                 z_uncond=zl[n:] if cfg else None, cfg_scale=float(np.float32(scale)))
+    g_conf = conf.cpu().numpy().astype(np.float64)
+    m_ = mask[:B].astype(bool)
+    assert np.all(np.abs(g_conf[m_] - u["conf"][m_]) <= 1e-6 * np.maximum(u["conf"][m_], 1e-30) + 1e-12)
+    for b in range(B):
+        if u["tie_rank"][b] or u["tie_tau"][b]:
+            continue
+        assert nsel.cpu().numpy()[b] == u["nsel"][b]
+        assert list(sel.cpu().numpy()[b][: u["nsel"][b]]) == list(u["sel"][b])
+        assert np.array_equal(dt_.cpu().numpy()[b], u["tokens"][b])
+        assert np.array_equal(dm.cpu().numpy()[b], u["mask"][b])
+        if cfg:
+            assert np.array_equal(dt_.cpu().numpy()[b + B], u["tokens"][b + B])
+    assert rem.item() == int(dm[:B].sum().item())
+    return u
+
+
+@pytest.mark.parametrize("V", [157184, 16384, 1001])
+def test_unmask_fixed(V):
+    _unmask_case(2, 32, V, 0.8, 1, 8, bd.FIXED, 1.0, seed=V % 97)
+
+
+def test_unmask_first_step_all_masked_full_vocab():
+    _unmask_case(1, 32, 157184, 1.0, 0, 8, bd.FIXED, 1.0, seed=11)
+
+
+def test_unmask_threshold_crosses_tau():
+    # wide logits so that some confidences exceed 0.9 and the cap of 8 binds
+    u = _unmask_case(16, 32, 157184, 1.0, 0, 32, bd.THRESHOLD, 6.0, seed=12)
+    assert np.any(u["nsel"] > 1)
+
+
+def test_unmask_cfg_image_slice():
+    _unmask_case(1, 32, 16384, 0.7, 2, 8, bd.FIXED, 1.0, cfg=True, scale=2.0, voff=157184 - 16384, seed=13)
+
+
+def test_unmask_last_step_takes_all():
+    u = _unmask_case(3, 32, 4096, 0.3, 7, 8, bd.FIXED, 1.0, seed=14)
+    assert np.all(u["mask"] == 0)
+
+
+def test_unmask_f32():
+    _unmask_case(1, 16, 1024, 1.0, 0, 4, bd.FIXED, 1.0, dtype="f32", seed=15)

@@ -1,0 +1,239 @@
+"""End-to-end parity of dllm_denoise_step (the whole pass through the C ABI) against the fp64 oracle (GPU).
+
+Both sides start from the same seeded weights, caches and block state. The oracle never sees a value the
+library computed. Where the two may legitimately part (a routing or confidence near-tie that a rounding
+difference can flip), the affected rows are excluded and counted, and a block comparison stops at the first
+such step.
+"""
+import numpy as np
+import pytest
+import torch
+
+from block_diffusion_moe_dllm_b200 import binding as bd
+from block_diffusion_moe_dllm_b200 import synth
+from block_diffusion_moe_dllm_b200.configs import ONE_LAYER, TINY_F32, scaled
+from block_diffusion_moe_dllm_b200.engine import DenoiseEngine
+from oracle import dllm_oracle as O
+from _util import assert_close, to64
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+# small bf16 backbone with the tensor-core path's constraints (head dim 128, H % 128 == 0, I % 64 == 0)
+SMALL = scaled(ONE_LAYER, name="small-bf16", n_layers=2, H=256, Hq=2, Hkv=1, d=128, E=8, k=2, I=128, V=1024, B=2,
+               P=64, L=16, T_s=4)
+# Routing margins below this can flip when the two sides' bf16 router inputs differ by one ulp in a few
+# elements: one ulp (2^-7 relative, ~8e-3 at |h| ~ 1) times a router weight (~0.02) moves a logit by ~1.6e-4
+# and a sigmoid score by at most a quarter of that; 3e-4 leaves a margin for a handful of such elements.
+# fp32 storage: 1e-5.
+E2E_ROUTE_MARGIN = 3e-4
+E2E_CONF_MARGIN = 2e-2    # relative confidence margins below this can flip under one-ulp logit differences
+
+
+def _setup(w, seed=0, masked_fraction=1.0, random_gains=True):
+    wt = synth.make_weights(w, DEV, seed=seed, random_gains=random_gains)
+    caches = synth.make_prefix_cache(w, DEV, seed=seed)
+    tokens, mask = synth.make_block_state(w, DEV, seed=seed, masked_fraction=masked_fraction)
+    eng = DenoiseEngine(w, wt, caches, DEV)
+    eng.set_block(tokens, mask)
+    return wt, caches, eng, tokens.cpu().numpy(), mask.cpu().numpy()
+
+
+def _host(wt):
+    """Host copies of the weights for the oracle (the same bytes the library reads)."""
+    cp = lambda t: t.detach().cpu()
+    return {"embed": cp(wt["embed"]), "final_norm": cp(wt["final_norm"]), "w_lm": cp(wt["w_lm"]),
+            "layers": [{k: cp(v) for k, v in lw.items()} for lw in wt["layers"]]}
+
+
+def _host_caches(caches, P):
+    return [(c[0][:, :, :P].cpu(), c[1][:, :, :P].cpu()) for c in caches]
+
+
+def _route_margin(dtype):
+    return E2E_ROUTE_MARGIN if dtype == "bf16" else 1e-5
+
+
+def _flagged_tokens(f, dtype="bf16"):
+    flag = np.zeros(f["x"].shape[0] * f["x"].shape[1], dtype=bool)
+    for r in f["route"]:
+        if r is not None:
+            flag |= r[2] < _route_margin(dtype)
+    return flag
+
+
+def _check_pass(w, eng, f, dtype):
+    n = len(f["row_pos"])
+    flag = _flagged_tokens(f, dtype)
+    x = to64(eng.x_final()).reshape(w.B * w.L, w.H)
+    ok = ~flag
+    assert ok.sum() >= 0.5 * len(ok), "too many routing near-ties for a meaningful comparison"
+    assert_close(x[ok], f["x"].reshape(-1, w.H)[ok], dtype, "hidden state after the last layer")
+    lg = to64(eng.logits(n))
+    Bl = w.B // 2 if w.cfg else w.B
+    rows = list(f["row_pos"]) + ([p + Bl * w.L for p in f["row_pos"]] if w.cfg else [])
+    okr = ~flag[np.asarray(rows, dtype=np.int64)]
+    if w.cfg:  # a guided row needs both of its rows clean
+        okr = okr[:n] & okr[n:]
+        okr = np.concatenate([okr, okr])
+    assert_close(lg[okr], f["logits"][okr], dtype, "logits of the masked rows")
+    return flag
+
+
+def _decisions_agree(w, u_or, eng, flag):
+    """Compare the unmask decisions where the oracle's choice is not a near-tie."""
+    Bl = w.B // 2 if w.cfg else w.B
+    g_tok = eng.tokens.cpu().numpy()
+    g_mask = eng.mask.cpu().numpy()
+    g_nsel = eng.nsel.cpu().numpy()
+    clean = True
+    for b in range(Bl):
+        c = u_or["conf"][b]
+        m = u_or["sel"][b]
+        row_flag = flag[b * w.L:(b + 1) * w.L].any() or (w.cfg and flag[(b + Bl) * w.L:(b + Bl + 1) * w.L].any())
+        masked_c = np.sort(c[c > 0])[::-1]
+        k = u_or["nsel"][b]
+        near = False
+        if 0 < k < len(masked_c):
+            near = (masked_c[k - 1] - masked_c[k]) < E2E_CONF_MARGIN * masked_c[k - 1]
+        if w.mode == 1:
+            near |= bool(np.any(np.abs(c[c > 0] - w.tau) < E2E_CONF_MARGIN))
+        if near or row_flag:
+            clean = False
+            continue
+        assert g_nsel[b] == u_or["nsel"][b]
+        assert np.array_equal(g_mask[b], u_or["mask"][b]), f"row {b}: unmasked positions differ"
+    return clean
+
+
+def _check_candidates(w, eng, u_or, f, flag):
+    """Candidate tokens written this step agree wherever the oracle's top-2 logit gap is clear."""
+    Bl = w.B // 2 if w.cfg else w.B
+    n = len(f["row_pos"])
+    z = f["logits"][:n]
+    if w.cfg:
+        z = O.cfg_combine_f32(z, f["logits"][n:], w.cfg_scale)
+    top2 = np.sort(z, axis=1)[:, -2:]
+    clear = (top2[:, 1] - top2[:, 0]) > 0.05
+    g_tok = eng.tokens.cpu().numpy()
+    g_mask = eng.mask.cpu().numpy()
+    for r, p in enumerate(f["row_pos"]):
+        b, i = divmod(int(p), w.L)
+        if not clear[r] or flag[p] or g_mask[b, i] == 1 or u_or["mask"][b, i] == 1:
+            continue
+        assert g_tok[b, i] == u_or["cand"][b, i], f"candidate token at row {b} pos {i}"
+
+
+def _one_pass(w, seed=0, masked_fraction=1.0, t=0, random_gains=True):
+    wt, caches, eng, tok0, mask0 = _setup(w, seed, masked_fraction, random_gains)
+    hw, hc = _host(wt), _host_caches(caches, w.P)
+    keep = O.sprint_keep(w, hc) if w.sprint else None
+    eng.step(t)
+    torch.cuda.synchronize()
+    assert bd.status_check(eng.ws) == bd.OK
+    u = O.denoise_step(w, hw, hc, tok0, mask0, t, keep=keep)
+    flag = _check_pass(w, eng, u["forward"], w.dtype)
+    _decisions_agree(w, u, eng, flag)
+    _check_candidates(w, eng, u, u["forward"], flag)
+    if w.sprint:
+        for l in range(w.n_layers):
+            kp = eng.thin[l][2]
+            for b in range(w.B):
+                got = kp[b, : w.n_keep].cpu().numpy()
+                _, sc, margin = O.prefix_retain(O.f64(hc[l][0][b]), None, n_keep=w.n_keep)
+                if margin > 1e-6 * sc.max():
+                    assert np.array_equal(got, keep[l][b])
+                assert np.array_equal(kp[b, w.n_keep: w.n_keep + w.L].cpu().numpy(), np.arange(w.P, w.P + w.L))
+    return eng, u
+
+
+def test_step_tiny_fp32():
+    _one_pass(TINY_F32, seed=0)
+
+
+def test_step_small_bf16_all_masked():
+    _one_pass(SMALL, seed=1)
+
+
+def test_step_small_bf16_partly_masked_mid_block():
+    _one_pass(SMALL, seed=2, masked_fraction=0.5, t=2)
+
+
+def test_step_small_bf16_cfg_image_slice():
+    w = scaled(SMALL, B=2, cfg=1, cfg_scale=2.0, vocab_offset=1024 - 256, vocab_len=256)
+    _one_pass(w, seed=3)
+
+
+def test_step_small_bf16_sprint():
+    w = scaled(SMALL, B=3, P=96, sprint=1, keep_ratio=0.5)
+    _one_pass(w, seed=4)
+
+
+def test_step_small_bf16_threshold():
+    w = scaled(SMALL, mode=1, tau=0.9, k_max=8, T_s=16, lm_std=1.0)
+    _one_pass(w, seed=5)
+
+
+def test_step_one_layer_full_size():
+    """The one-layer bf16 workload at its full size (hidden 2048, 256 experts, vocab 157184, prefix 1024)."""
+    _one_pass(ONE_LAYER, seed=0, random_gains=False)
+
+
+@pytest.mark.parametrize("w", [TINY_F32, SMALL], ids=["tiny-f32", "small-bf16"])
+def test_block_decode(w):
+    """All T_s passes of a block. The oracle follows its own decisions from the same start; the two states are
+    compared after every step until a step whose decision is a near-tie (after which they may part)."""
+    wt, caches, eng, tok, mask = _setup(w, seed=7)
+    hw, hc = _host(wt), _host_caches(caches, w.P)
+    compared = 0
+    for t in range(w.T_s):
+        eng.step(t)
+        torch.cuda.synchronize()
+        if tok is None:
+            continue
+        u = O.denoise_step(w, hw, hc, tok, mask, t)
+        flag = _flagged_tokens(u["forward"], w.dtype)
+        clean = _decisions_agree(w, u, eng, flag)
+        _check_candidates(w, eng, u, u["forward"], flag)
+        if not np.array_equal(eng.mask.cpu().numpy(), u["mask"]):
+            assert not clean, f"step {t}: unmasked positions differ without a near-tie"
+            tok = None
+            continue
+        if not np.array_equal(eng.tokens.cpu().numpy(), u["tokens"]):
+            tok = None          # a candidate with an unclear top-2 gap was written (checked where clear)
+            continue
+        compared += 1
+        tok, mask = u["tokens"], u["mask"]
+    assert int(eng.mask.sum().item()) == 0, "every position is unmasked after the last step"
+
+
+@pytest.mark.parametrize("w", [TINY_F32, SMALL, scaled(SMALL, sprint=1, keep_ratio=0.5)],
+                         ids=["tiny-f32", "small-bf16", "small-bf16-sprint"])
+def test_commit_pass(w):
+    """The commit pass over a seeded clean block writes each layer's block K/V into cache rows [P, P + L)."""
+    wt, caches, eng, _, _ = _setup(w, seed=8)
+    hw, hc = _host(wt), _host_caches(caches, w.P)
+    clean = synth.randint((w.B, w.L), 0, w.V - 1, 8, "clean_block", DEV)
+    eng.set_block(clean, torch.zeros((w.B, w.L), dtype=torch.uint8, device=DEV))
+    keep = None
+    if w.sprint:
+        eng.step(0)          # selects the kept prefix (retain) for this block
+        keep = O.sprint_keep(w, hc)
+        eng.set_block(clean, torch.zeros((w.B, w.L), dtype=torch.uint8, device=DEV))
+    eng.commit()
+    torch.cuda.synchronize()
+    assert bd.status_check(eng.ws) == bd.OK
+    bk, bv = O.commit_block(w, hw, hc, clean.cpu().numpy(), keep=keep)
+    flag = np.zeros(w.B * w.L, dtype=bool)
+    f = O.forward_block(w, hw, hc, clean.cpu().numpy(), np.zeros((w.B, w.L), np.int64), keep=keep,
+                        want_logits=False, skip_last_ffn=True)
+    for l in range(w.n_layers):
+        kc, vc = caches[l]
+        got_k = to64(kc[:, :, w.P: w.P + w.L]).transpose(0, 2, 1, 3)
+        got_v = to64(vc[:, :, w.P: w.P + w.L]).transpose(0, 2, 1, 3)
+        ok = ~flag.reshape(w.B, w.L)
+        assert_close(got_k[ok], bk[l][ok], w.dtype, f"committed K layer {l}")
+        assert_close(got_v[ok], bv[l][ok], w.dtype, f"committed V layer {l}")
+        # routing near-ties in this layer can change the next layer's input: mark those tokens
+        if f["route"][l] is not None:
+            flag |= f["route"][l][2] < _route_margin(w.dtype)

@@ -91,6 +91,7 @@ _SIGS = {
     "dllm_moe_experts_workspace_size": ([C.POINTER(ExpertDesc)], sz),
     "dllm_unmask": ([C.POINTER(UnmaskDesc), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], C.c_int),
     "dllm_unmask_workspace_size": ([C.POINTER(UnmaskDesc)], sz),
+    "dllm_unmask_noalloc": ([C.POINTER(UnmaskDesc), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp], C.c_int),
     "dllm_denoise_step": ([C.POINTER(Model), C.POINTER(State), C.POINTER(StepParams), vp, sz, vp], C.c_int),
     "dllm_denoise_step_workspace_size": ([C.POINTER(Model), C.POINTER(State), C.POINTER(StepParams)], sz),
     "dllm_denoise_step_views": ([C.POINTER(Model), C.POINTER(State), C.POINTER(StepParams), vp, sz,

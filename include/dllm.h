@@ -207,6 +207,21 @@ DLLM_API int dllm_unmask(const dllm_unmask_desc* desc, const void* logits, const
                 void* ws, size_t ws_bytes, cudaStream_t stream);
 DLLM_API size_t dllm_unmask_workspace_size(const dllm_unmask_desc* desc);
 
+/*
+ * dllm_unmask without a workspace, for callers that cannot allocate device memory (a plug-in inside a host
+ * application that owns the device's memory pool and exposes no allocator; a serving loop that forbids cudaMalloc
+ * after start-up because it can synchronise the device). The paper has no counterpart: this is a deployment
+ * variant of the same computation. Same arguments and results as dllm_unmask minus ws / ws_bytes; the caller
+ * still owns every input and output. The per-chunk scratch lives in a fixed 1 MiB array inside the library,
+ * held on every GPU that loads it until the process exits; calls with max_rows x vocabulary chunks needing more
+ * (more than 65536 partial entries) return DLLM_ERR_UNSUPPORTED. The first call on each device looks up the
+ * array's device address (make it before any stream capture). All calls share the array: calls that overlap on
+ * the GPU race and must be ordered by the caller (one stream, or events).
+ */
+DLLM_API int dllm_unmask_noalloc(const dllm_unmask_desc* desc, const void* logits, const int32_t* row_pos,
+                                 const int32_t* n_rows_dev, int32_t* tokens, uint8_t* mask, int32_t* sel, int32_t* nsel,
+                                 float* conf, int32_t* remaining, cudaStream_t stream);
+
 /* ---------------------------------------------------------------------------------------------- B6 step */
 /* Weights of one layer (device pointers, storage type unless stated). */
 typedef struct {

@@ -267,59 +267,16 @@ def main():
 
 
 def kernel_rooflines(w, wt, eng, dev, stream):
-    """Per-kernel CUDA-event timings of the step's main kernels launched alone with the step's shapes."""
-    import torch
-    from block_diffusion_moe_dllm_b200 import binding as bd
-    peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
-        os.path.join(ROOT, "MEASURED_PEAKS.json")) else {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
-    hbm = peaks["hbm_gbs"]
-    rows = w.B * w.L
-    x = torch.randn((rows, w.H), device=dev).to(torch.bfloat16)
-    vlen = w.vlen
-    wl = wt["w_lm"][w.vocab_offset: w.vocab_offset + vlen]
-    y = torch.empty((rows, vlen), dtype=torch.bfloat16, device=dev)
-    ws = bd.Workspace(1 << 20, dev)
-
-    def timed(fn, reps=20):
-        for _ in range(3):
-            fn()
-        torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(reps):
-            fn()
-        b.record(stream)
-        torch.cuda.synchronize()
-        return a.elapsed_time(b) / 1000.0 / reps
-
-    t_lm = timed(lambda: bd.gemm(x, wl, y, rows, vlen, w.H, bd.BF16, ws=ws, stream=stream))
-    lm_bytes = vlen * w.H * 2 + rows * w.H * 2 + rows * vlen * 2
-    kernels = {"gemm_tc_kernel[lm_head]": {"us": t_lm * 1e6, "bytes": lm_bytes,
-                                           "GB/s": lm_bytes / t_lm / 1e9, "frac_hbm": lm_bytes / t_lm / 1e9 / hbm}}
-    # expert GEMMs of one layer: route the block's first-pass input, then time the experts call alone
-    lw = wt["layers"][0]
-    h = torch.randn((rows, w.H), device=dev).to(torch.bfloat16)
-    ids = torch.empty((rows, w.k), dtype=torch.int32, device=dev)
-    gates = torch.empty((rows, w.k), dtype=torch.float32, device=dev)
-    counts = torch.empty(w.E, dtype=torch.int32, device=dev)
-    offsets = torch.empty(w.E + 1, dtype=torch.int32, device=dev)
-    perm = torch.empty(rows * w.k, dtype=torch.int32, device=dev)
-    inv = torch.empty(rows * w.k, dtype=torch.int32, device=dev)
-    bd.moe_route(h, lw["w_router"], lw["router_bias"], ids, gates, counts, offsets, perm, inv, rows, w.H, w.E, w.k,
-                 bd.BF16, ws=ws, stream=stream)
-    torch.cuda.synchronize()
-    active = int((counts > 0).sum().item())
-    xo = torch.zeros((rows, w.H), dtype=torch.bfloat16, device=dev)
-    t_ex = timed(lambda: bd.moe_experts(h, lw["w_gu"], lw["w_down"], lw["w_gu_shared"], lw["w_down_shared"], counts,
-                                        offsets, perm, inv, gates, xo, rows, w.H, w.E, w.k, w.I, bd.BF16, ws=ws,
-                                        stream=stream))
-    ex_bytes = (active + 1) * 3 * w.I * w.H * 2
-    kernels["moe_experts[gather+2 gemm+combine]"] = {"us": t_ex * 1e6, "bytes": ex_bytes, "active_experts": active,
-                                                    "GB/s": ex_bytes / t_ex / 1e9,
-                                                    "frac_hbm": ex_bytes / t_ex / 1e9 / hbm}
+    """Per-kernel CUDA-event timings of the step's main calls launched alone with the step's shapes; the LM-head
+    GEMM (one launch of gemm_tc_kernel streaming 157184 x 2048 bf16) is the roofline kernel."""
+    from block_diffusion_moe_dllm_b200 import kernel_bench as kb
+    lm = kb.bench_lm_head(w, 20, dev, stream, weights=wt)
+    rest = kb.bench_experts(w, 20, dev, stream, weights=wt) + [kb.bench_unmask(w, 20, dev, stream),
+                                                               kb.bench_attn(w, 20, dev, stream)]
+    kernels = {r["kernel"]: {k: v for k, v in r.items() if k != "kernel"} for r in [lm] + rest}
     roof = {"kernel": "gemm_tc_kernel (LM head 157184x2048 bf16, 32 rows)", "bound": "hbm",
-            "achieved": lm_bytes / t_lm / 1e9, "peak": hbm, "unit": "GB/s", "frac": lm_bytes / t_lm / 1e9 / hbm,
-            "traffic": None, "peak_source": "measured (MEASURED_PEAKS.json hbm_gbs)"}
+            "achieved": lm["GB/s"], "peak": lm["peak_GBs"], "unit": "GB/s", "frac": lm["frac_hbm"],
+            "traffic": None, "peak_source": f"{lm['peak_source']} (MEASURED_PEAKS.json hbm_gbs, burst copy)"}
     return roof, kernels
 
 

@@ -1,0 +1,156 @@
+"""Per-kernel timing of the library's main calls at a workload's shapes (CUDA events, kernels launched alone).
+
+    python -m block_diffusion_moe_dllm_b200.kernel_bench [--kernel lm_head|experts|unmask|attn|route|all]
+                                                         [--workload NAME] [--reps N]
+
+Each line reports the mean time of one call, its algorithmic bytes (weights and activations it must move at
+least once) and the achieved fraction of the measured HBM bandwidth. Used by bench.py for the roofline object and
+as the target command of ncu captures.
+"""
+import argparse
+import json
+import os
+
+import torch
+
+from . import binding as bd
+from . import synth
+from .configs import BY_NAME, ONE_LAYER, Workload
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def hbm_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        return json.load(open(p))["hbm_gbs"], "measured"
+    return 6650.0, "fallback"
+
+
+def timed(fn, reps, stream, warm=3):
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(reps):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / 1000.0 / max(reps, 1)
+
+
+def _result(name, t, nbytes, extra=None):
+    peak, src = hbm_peak()
+    r = {"kernel": name, "us": t * 1e6, "bytes": nbytes, "GB/s": nbytes / t / 1e9, "frac_hbm": nbytes / t / 1e9 / peak,
+         "peak_GBs": peak, "peak_source": src}
+    if extra:
+        r.update(extra)
+    return r
+
+
+def bench_lm_head(w: Workload, reps, dev, stream, weights=None):
+    rows = (2 if w.cfg else 1) * (w.B // (2 if w.cfg else 1)) * w.L
+    wl = (weights["w_lm"] if weights else synth.normal((w.V, w.H), w.lm_std, w.seed, "w_lm", dev, chunk_rows=16384))
+    wl = wl[w.vocab_offset: w.vocab_offset + w.vlen]
+    x = synth.normal((rows, w.H), 1.0, 1, "kb_x", dev)
+    y = torch.empty((rows, w.vlen), dtype=torch.bfloat16, device=dev)
+    ws = bd.Workspace(1 << 16, dev)
+    t = timed(lambda: bd.gemm(x, wl, y, rows, w.vlen, w.H, bd.BF16, ws=ws, stream=stream), reps, stream)
+    nbytes = w.vlen * w.H * 2 + rows * w.H * 2 + rows * w.vlen * 2
+    return _result("gemm_tc_kernel[lm_head]", t, nbytes, {"rows": rows, "M": w.vlen, "K": w.H})
+
+
+def bench_experts(w: Workload, reps, dev, stream, weights=None):
+    rows = w.B * w.L
+    lw = weights["layers"][0] if weights else synth.make_weights(
+        Workload(**{**w.__dict__, "n_layers": 1, "V": 128}), dev)["layers"][0]
+    h = synth.normal((rows, w.H), 1.0, 2, "kb_h", dev)
+    ids = torch.empty((rows, w.k), dtype=torch.int32, device=dev)
+    gates = torch.empty((rows, w.k), dtype=torch.float32, device=dev)
+    counts = torch.empty(w.E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(w.E + 1, dtype=torch.int32, device=dev)
+    perm = torch.empty(rows * w.k, dtype=torch.int32, device=dev)
+    inv = torch.empty(rows * w.k, dtype=torch.int32, device=dev)
+    ws = bd.Workspace(1 << 20, dev)
+    bd.moe_route(h, lw["w_router"], lw["router_bias"], ids, gates, counts, offsets, perm, inv, rows, w.H, w.E, w.k,
+                 bd.BF16, ws=ws, stream=stream)
+    torch.cuda.synchronize()
+    active = int((counts > 0).sum().item())
+    x = torch.zeros((rows, w.H), dtype=torch.bfloat16, device=dev)
+    t = timed(lambda: bd.moe_experts(h, lw["w_gu"], lw["w_down"], lw["w_gu_shared"], lw["w_down_shared"], counts,
+                                     offsets, perm, inv, gates, x, rows, w.H, w.E, w.k, w.I, bd.BF16, ws=ws,
+                                     stream=stream), reps, stream)
+    nbytes = (active + 1) * 3 * w.I * w.H * 2 + 2 * rows * w.H * 2
+    troute = timed(lambda: bd.moe_route(h, lw["w_router"], lw["router_bias"], ids, gates, counts, offsets, perm, inv,
+                                        rows, w.H, w.E, w.k, bd.BF16, ws=ws, stream=stream), reps, stream)
+    rbytes = w.E * w.H * 2 + rows * w.H * 2
+    return [_result("moe_experts[gather+gemm_tc x2+combine]", t, nbytes, {"active_experts": active, "rows": rows}),
+            _result("moe_route[scores+topk+permute]", troute, rbytes, {"rows": rows})]
+
+
+def bench_unmask(w: Workload, reps, dev, stream):
+    Bl = w.B // 2 if w.cfg else w.B
+    n = Bl * w.L
+    logits = synth.normal(((2 if w.cfg else 1) * n, w.vlen), 3.0, 3, "kb_logits", dev)
+    row_pos = torch.arange(n, dtype=torch.int32, device=dev)
+    n_dev = torch.tensor([n], dtype=torch.int32, device=dev)
+    tok = torch.zeros((w.B, w.L), dtype=torch.int32, device=dev)
+    msk0 = torch.ones((w.B, w.L), dtype=torch.uint8, device=dev)
+    msk = msk0.clone()
+    sel = torch.empty((Bl, w.L), dtype=torch.int32, device=dev)
+    nsel = torch.empty(Bl, dtype=torch.int32, device=dev)
+    conf = torch.empty((Bl, w.L), dtype=torch.float32, device=dev)
+    rem = torch.empty(1, dtype=torch.int32, device=dev)
+    ws = bd.Workspace(1 << 22, dev)
+
+    def call():
+        msk.copy_(msk0)
+        bd.unmask(logits, row_pos, n_dev, tok, msk, sel, nsel, conf, rem, Bl, w.L, w.vlen, n, 0, w.T_s, bd.BF16,
+                  mode=w.mode, tau=w.tau, k_max=w.k_max, cfg=w.cfg, cfg_scale=w.cfg_scale,
+                  vocab_offset=w.vocab_offset, ws=ws, stream=stream)
+    t = timed(call, reps, stream)
+    nbytes = logits.numel() * 2
+    return _result("unmask[reduce+select]", t, nbytes, {"rows": n, "V": w.vlen})
+
+
+def bench_attn(w: Workload, reps, dev, stream):
+    n_keys = (w.n_keep if w.sprint else w.P) + w.L
+    cap = n_keys
+    q = synth.normal((w.B, w.L, w.Hq, w.d), 1.0, 4, "kb_q", dev)
+    kc = synth.normal((w.B, w.Hkv, cap, w.d), 1.0, 4, "kb_k", dev)
+    vc = synth.normal((w.B, w.Hkv, cap, w.d), 1.0, 4, "kb_v", dev)
+    out = torch.empty((w.B, w.L, w.Hq * w.d), dtype=torch.bfloat16, device=dev)
+    ws = bd.Workspace(1 << 26, dev)
+    t = timed(lambda: bd.block_attn(q, kc, vc, out, w.B, w.L, w.Hq, w.Hkv, w.d, w.L, w.P, n_keys, cap, bd.BF16,
+                                    ws=ws, stream=stream), reps, stream)
+    nbytes = 2 * w.B * w.Hkv * n_keys * w.d * 2 + 2 * w.B * w.L * w.Hq * w.d * 2
+    flops = 4.0 * w.B * w.L * w.Hq * n_keys * w.d
+    return _result("block_attn", t, nbytes, {"keys": n_keys, "TFLOP/s": flops / t / 1e12})
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--kernel", default="all")
+    ap.add_argument("--workload", default=ONE_LAYER.name)
+    ap.add_argument("--reps", type=int, default=20)
+    a = ap.parse_args()
+    w = BY_NAME[a.workload]
+    dev = "cuda"
+    bd.load()
+    stream = torch.cuda.current_stream()
+    out = []
+    if a.kernel in ("lm_head", "all"):
+        out.append(bench_lm_head(w, a.reps, dev, stream))
+    if a.kernel in ("experts", "route", "all"):
+        out.extend(bench_experts(w, a.reps, dev, stream))
+    if a.kernel in ("unmask", "all"):
+        out.append(bench_unmask(w, a.reps, dev, stream))
+    if a.kernel in ("attn", "all"):
+        out.append(bench_attn(w, a.reps, dev, stream))
+    for r in out:
+        print(json.dumps(r), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -10,6 +10,7 @@
 #include "misc.h"
 
 #include <atomic>
+#include <algorithm>
 
 namespace dllm_host {
 static thread_local char g_err[512] = "";
@@ -63,6 +64,13 @@ int check_ws(void* ws, size_t ws_bytes, size_t need) {
 int32_t* status_word(void* ws) { return static_cast<int32_t*>(ws); }
 
 // ------------------------------------------------------------------------------------------------ GEMM dispatch
+// Scratch a dense projection of `rows` rows needs for split-K (0 when it does not split).
+size_t dense_splitk_bytes(int dtype, int64_t rows, int M, int K) {
+  GemmArgs a;
+  a.dtype = dtype; a.x_rows = rows; a.M = M; a.K = K; a.max_cnt = (int)rows; a.host_cnt = (int)rows;
+  return gemm_splitk_scratch_bytes(a);
+}
+
 int run_gemm(GemmArgs& a, cudaStream_t s) {
   return a.dtype == DLLM_BF16 ? gemm_bf16_tc(a, s) : gemm_f32_simt(a, s);
 }
@@ -137,6 +145,7 @@ struct StepPlan {
   int32_t* inv;
   ExpertBufs eb;
   float* proj_scratch;
+  float* splitk;
   int32_t* row_pos;
   int32_t* n_rows;
   void* xf;
@@ -155,6 +164,8 @@ int validate_step(const dllm_model* m, const dllm_state* st, const dllm_step_par
   REQ(m->Hq % m->Hkv == 0, DLLM_ERR_SHAPE, "denoise_step: Hq %% Hkv != 0");
   REQ(m->k <= m->E && m->k <= 32 && m->E <= 1024, DLLM_ERR_UNSUPPORTED, "denoise_step: k/E out of range");
   REQ(m->H % 8 == 0, DLLM_ERR_SHAPE, "denoise_step: H must be a multiple of 8");
+  REQ((size_t)16 * m->H * (m->dtype == DLLM_BF16 ? 2 : 4) <= 200 * 1024, DLLM_ERR_UNSUPPORTED,
+      "denoise_step: H too large for the router");
   REQ(st->B >= 1 && st->L >= 1 && st->L <= 32 && st->P >= 0, DLLM_ERR_SHAPE, "denoise_step: bad B/L/P");
   REQ(st->cap >= st->P + st->L, DLLM_ERR_SHAPE, "denoise_step: cap %d < P + L", st->cap);
   REQ(st->tokens && st->mask, DLLM_ERR_INVALID_ARG, "denoise_step: NULL tokens/mask");
@@ -210,7 +221,7 @@ void plan_step(const dllm_model* m, const dllm_state* st, const dllm_step_params
   s.h = c.take((size_t)s.Tk * H * es);
   s.q = c.take((size_t)s.Tk * QD * es);
   s.ao = c.take((size_t)s.Tk * QD * es);
-  s.attn_ws_bytes = attn_workspace_bytes(st->B, st->L, m->Hq, m->Hkv, m->d, s.n_keys);
+  s.attn_ws_bytes = attn_workspace_bytes(st->B, st->L, m->Hq, m->Hkv, m->d, s.n_keys, m->dtype);
   s.attn_ws = c.take(s.attn_ws_bytes);
   s.scores = c.take<float>((size_t)s.Tk * m->E * 4);
   s.ids = c.take<int32_t>((size_t)s.Tk * m->k * 4);
@@ -225,6 +236,13 @@ void plan_step(const dllm_model* m, const dllm_state* st, const dllm_step_params
                        ? c.take<float>((size_t)std::max(s.Tk, s.halves * s.max_rows) *
                                        std::max(std::max(proj_n, H), s.vlen) * 4)
                        : nullptr;
+  {
+    const size_t a = dense_splitk_bytes(m->dtype, s.Tk, proj_n, H);
+    const size_t b = dense_splitk_bytes(m->dtype, s.Tk, H, QD);
+    const size_t l = dense_splitk_bytes(m->dtype, (int64_t)s.halves * s.max_rows, s.vlen, H);
+    const size_t need = std::max(a, std::max(b, l));
+    s.splitk = need ? c.take<float>(need) : nullptr;
+  }
   s.row_pos = c.take<int32_t>((size_t)s.max_rows * 4);
   s.n_rows = c.take<int32_t>(16);
   s.xf = c.take((size_t)s.halves * s.max_rows * H * es);
@@ -264,6 +282,7 @@ size_t dllm_gemm_workspace_size(const dllm_gemm_desc* d) {
   if (!d) return 0;
   size_t n = kStatusBytes;
   if (d->dtype == DLLM_F32) n = align256(n) + gemm_f32_scratch_bytes(d->N, d->M, 0);
+  else n = align256(n) + dense_splitk_bytes(d->dtype, d->N, d->M, d->K);
   return align256(n);
 }
 
@@ -285,6 +304,10 @@ int dllm_gemm(const dllm_gemm_desc* d, const void* x, const void* w, void* y, co
   a.cnt_dev = n_rows_dev; a.host_cnt = d->N; a.max_cnt = d->N; a.cnt_bound = d->N;
   a.dtype = d->dtype; a.status = status_word(ws);
   a.f32_scratch = d->dtype == DLLM_F32 ? c.take<float>(gemm_f32_scratch_bytes(d->N, d->M, 0)) : nullptr;
+  if (d->dtype == DLLM_BF16) {
+    const size_t sk = dense_splitk_bytes(d->dtype, d->N, d->M, d->K);
+    a.splitk_scratch = sk ? c.take<float>(sk) : nullptr;
+  }
   a.epi.kind = d->residual ? EPI_RESID : EPI_STORE;
   a.epi.out = y; a.epi.ldo = d->ldy; a.epi.out_f32 = d->y_f32 || d->dtype == DLLM_F32;
   return run_gemm(a, stream);
@@ -293,7 +316,7 @@ int dllm_gemm(const dllm_gemm_desc* d, const void* x, const void* w, void* y, co
 // ------------------------------------------------------------------------------------------------ attention
 size_t dllm_block_attn_workspace_size(const dllm_attn_desc* d) {
   if (!d) return 0;
-  return align256(align256(kStatusBytes) + attn_workspace_bytes(d->B, d->Lq, d->Hq, d->Hkv, d->d, d->n_keys));
+  return align256(align256(kStatusBytes) + attn_workspace_bytes(d->B, d->Lq, d->Hq, d->Hkv, d->d, d->n_keys, d->dtype));
 }
 
 int dllm_block_attn(const dllm_attn_desc* d, const void* q, const void* k_cache, const void* v_cache,
@@ -314,9 +337,9 @@ int dllm_block_attn(const dllm_attn_desc* d, const void* q, const void* k_cache,
   a.B = d->B; a.Lq = d->Lq; a.Hq = d->Hq; a.Hkv = d->Hkv; a.d = d->d; a.blk_len = d->blk_len; a.q_pos0 = d->q_pos0;
   a.n_keys = d->n_keys; a.cap = d->cap; a.dtype = d->dtype; a.scale = d->scale;
   a.q = q; a.k = k_cache; a.v = v_cache; a.key_pos = key_pos; a.out = out;
-  a.ws_bytes = attn_workspace_bytes(d->B, d->Lq, d->Hq, d->Hkv, d->d, d->n_keys);
+  a.ws_bytes = attn_workspace_bytes(d->B, d->Lq, d->Hq, d->Hkv, d->d, d->n_keys, d->dtype);
   a.ws = c.take(a.ws_bytes);
-  return launch_attn(a, stream);
+  return launch_attn(a, status_word(ws), stream);
 }
 
 // ------------------------------------------------------------------------------------------------ SPRINT
@@ -357,7 +380,7 @@ int dllm_moe_route(const dllm_route_desc* d, const void* h, const void* w_router
   REQ(d->Tk >= 0 && d->H > 0 && d->E >= 1 && d->k >= 1, DLLM_ERR_SHAPE, "moe_route: bad shape");
   REQ(d->E <= 1024 && d->k <= 32 && d->k <= d->E, DLLM_ERR_UNSUPPORTED, "moe_route: needs E <= 1024, k <= min(32, E)");
   REQ(d->H % 8 == 0, DLLM_ERR_SHAPE, "moe_route: H must be a multiple of 8");
-  REQ(d->H * 32 <= 200 * 1024 / 1, DLLM_ERR_UNSUPPORTED, "moe_route: H too large");
+  REQ((size_t)16 * d->H * (d->dtype == DLLM_BF16 ? 2 : 4) <= 200 * 1024, DLLM_ERR_UNSUPPORTED, "moe_route: H too large");
   REQ(d->dtype == DLLM_BF16 || d->dtype == DLLM_F32, DLLM_ERR_INVALID_ARG, "moe_route: bad dtype");
   REQ(aligned16(h) && aligned16(w_router), DLLM_ERR_ALIGN, "moe_route: h and w_router must be 16-byte aligned");
   int st = check_ws(ws, ws_bytes, dllm_moe_route_workspace_size(d));
@@ -496,7 +519,7 @@ int dllm_denoise_step(const dllm_model* m, const dllm_state* st, const dllm_step
     GemmArgs g;
     g.x = s.h; g.x_rows = s.Tk; g.w = Ly.w_qkv; g.w_rows = (int64_t)(m->Hq + 2 * m->Hkv) * m->d; g.K = H;
     g.M = (m->Hq + 2 * m->Hkv) * m->d; g.host_cnt = s.Tk; g.max_cnt = s.Tk; g.cnt_bound = s.Tk; g.dtype = dt;
-    g.status = status; g.f32_scratch = s.proj_scratch;
+    g.status = status; g.f32_scratch = s.proj_scratch; g.splitk_scratch = s.splitk;
     g.epi.kind = EPI_QKV; g.epi.q_out = s.q; g.epi.Hq = m->Hq; g.epi.Hkv = m->Hkv; g.epi.d = m->d; g.epi.L = L;
     g.epi.pos0 = P; g.epi.rope_base = m->rope_base;
     if (p->sprint) {
@@ -512,11 +535,12 @@ int dllm_denoise_step(const dllm_model* m, const dllm_state* st, const dllm_step
     aa.n_keys = s.n_keys; aa.cap = p->sprint ? st->cap_thin : st->cap; aa.dtype = dt; aa.scale = 0.f;
     aa.q = s.q; aa.k = p->sprint ? Ly.k_thin : Ly.k_cache; aa.v = p->sprint ? Ly.v_thin : Ly.v_cache;
     aa.key_pos = p->sprint ? Ly.keep_pos : nullptr; aa.out = s.ao; aa.ws = s.attn_ws; aa.ws_bytes = s.attn_ws_bytes;
-    TRY(launch_attn(aa, stream));
+    TRY(launch_attn(aa, status, stream));
     // output projection + residual
     GemmArgs go;
     go.x = s.ao; go.x_rows = s.Tk; go.w = Ly.w_o; go.w_rows = H; go.K = QD; go.M = H; go.host_cnt = s.Tk;
     go.max_cnt = s.Tk; go.cnt_bound = s.Tk; go.dtype = dt; go.status = status; go.f32_scratch = s.proj_scratch;
+    go.splitk_scratch = s.splitk;
     go.epi.kind = EPI_RESID; go.epi.out = s.x; go.epi.ldo = H; go.epi.out_f32 = dt == DLLM_F32;
     TRY(run_gemm(go, stream));
     if (p->commit && last) break;  // the last layer's FFN output has no consumer in a commit pass
@@ -536,7 +560,7 @@ int dllm_denoise_step(const dllm_model* m, const dllm_state* st, const dllm_step
   gl.w = static_cast<const char*>(m->w_lm) + (size_t)p->vocab_offset * H * es; gl.w_rows = s.vlen;
   gl.K = H; gl.M = s.vlen; gl.cnt_dev = s.n_rows + 1; gl.host_cnt = s.halves * s.max_rows;
   gl.max_cnt = s.halves * s.max_rows; gl.cnt_bound = s.halves * s.max_rows; gl.dtype = dt; gl.status = status;
-  gl.f32_scratch = s.proj_scratch;
+  gl.f32_scratch = s.proj_scratch; gl.splitk_scratch = s.splitk;
   gl.epi.kind = EPI_STORE; gl.epi.out = s.logits; gl.epi.ldo = s.vlen; gl.epi.out_f32 = dt == DLLM_F32;
   TRY(run_gemm(gl, stream));
   UnmaskArgs ua;

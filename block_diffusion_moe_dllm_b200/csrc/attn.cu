@@ -201,7 +201,7 @@ void plan(int B, int Lq, int Hq, int Hkv, int n_keys, int& qt_rows, int& n_qtile
 
 }  // namespace
 
-size_t attn_workspace_bytes(int B, int Lq, int Hq, int Hkv, int d, int n_keys) {
+size_t attn_simt_workspace_bytes(int B, int Lq, int Hq, int Hkv, int d, int n_keys) {
   int qt, nqt, ns, kps;
   plan(B, Lq, Hq, Hkv, n_keys, qt, nqt, ns, kps);
   if (ns <= 1) return 0;
@@ -209,7 +209,7 @@ size_t attn_workspace_bytes(int B, int Lq, int Hq, int Hkv, int d, int n_keys) {
   return ns * nq * (size_t)d * 4 + 2 * ns * nq * 4 + 512;
 }
 
-int launch_attn(const AttnArgs& a, cudaStream_t s) {
+int launch_attn_simt(const AttnArgs& a, cudaStream_t s) {
   AttnK p;
   p.B = a.B; p.Lq = a.Lq; p.Hq = a.Hq; p.Hkv = a.Hkv; p.d = a.d; p.blk_len = a.blk_len; p.q_pos0 = a.q_pos0;
   p.n_keys = a.n_keys; p.cap = a.cap;
@@ -245,6 +245,27 @@ int launch_attn(const AttnArgs& a, cudaStream_t s) {
     else attn_merge_kernel<float><<<nq, 128, 0, s>>>(p);
     DLLM_CHECK_LAUNCH("attn_merge_kernel");
   }
+  return DLLM_OK;
+}
+
+size_t attn_workspace_bytes(int B, int Lq, int Hq, int Hkv, int d, int n_keys, int dtype) {
+  if (attn_tc_supported(dtype, Hq, Hkv, d)) return attn_tc_workspace_bytes(B, Lq, Hq, Hkv, n_keys);
+  return attn_simt_workspace_bytes(B, Lq, Hq, Hkv, d, n_keys);
+}
+
+int launch_attn(const AttnArgs& a, int32_t* status, cudaStream_t s) {
+  if (attn_tc_supported(a.dtype, a.Hq, a.Hkv, a.d)) return launch_attn_tc(a, status, s);
+  return launch_attn_simt(a, s);
+}
+
+int launch_attn_merge(const AttnArgs& a, int n_splits, float* po, float* pm, float* pl, cudaStream_t s) {
+  AttnK p{};
+  p.B = a.B; p.Lq = a.Lq; p.Hq = a.Hq; p.d = a.d; p.n_splits = n_splits;
+  p.po = po; p.pm = pm; p.pl = pl; p.out = a.out;
+  const int nq = a.B * a.Lq * a.Hq;
+  if (a.dtype == DLLM_BF16) attn_merge_kernel<__nv_bfloat16><<<nq, 128, 0, s>>>(p);
+  else attn_merge_kernel<float><<<nq, 128, 0, s>>>(p);
+  DLLM_CHECK_LAUNCH("attn_merge_kernel");
   return DLLM_OK;
 }
 

@@ -18,6 +18,7 @@
 #include "kernels.h"
 #include <cuda.h>
 #include <mutex>
+#include <algorithm>
 
 namespace dllm {
 
@@ -47,10 +48,15 @@ struct Smem {
   int grp_off[MAX_GROUPS];
   int grp_cnt[MAX_GROUPS];
   int chunk_sum[NUM_THREADS];
+  int is_last;
 };
 
 struct KParams {
   int K, M, swiglu, m_tiles;
+  int ksplit;              // > 1: split-K; each split writes its raw fp32 partial, the last split of a tile to
+  float* partial;          // arrive sums all partials in split order and runs the epilogue
+  int64_t part_stride;     // elements between two splits' partials (x_rows * M)
+  int* tile_cnt;           // per-tile arrival counters (zero before the launch; reset by the last split)
   int64_t w_group_stride;
   int n_dev, has_extra, extra_off, extra_cnt, host_cnt;
   const int32_t* grp_off;
@@ -78,6 +84,7 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
 template <int BN>
 __device__ __forceinline__ void decode_tile(const Smem& sm, int m_tiles, int t, int& g, int& mt, int& n0,
                                             int& nval) {
+  // t is a tile index (work index / ksplit)
   int lo = 0, hi = sm.n_groups - 1;
   while (lo < hi) {  // last g with tile_prefix[g] <= t
     int mid = (lo + hi + 1) >> 1;
@@ -238,7 +245,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
     }
     __syncthreads();
   }
-  const int total = sm.total_tiles;
+  const int total = sm.total_tiles * p.ksplit;
   volatile int* abort_flag = &sm.abort_flag;
   const int kblocks = p.K / BK;
 
@@ -252,7 +259,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
       const uint64_t pol_x = tc::policy_evict_last();
       uint32_t it = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      for (int wk = blockIdx.x; wk < total && ok; wk += gridDim.x) {
+        const int t = wk / p.ksplit, ks = wk - t * p.ksplit;
+        const int kb0 = ks * kblocks / p.ksplit, kb1 = (ks + 1) * kblocks / p.ksplit;
         int g, mt, n0, nval;
         decode_tile<BN>(sm, p.m_tiles, t, g, mt, n0, nval);
         const bool extra = p.has_extra && g == p.n_dev;
@@ -261,7 +270,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
         const int nb = (nval + XBOX_ROWS - 1) / XBOX_ROWS;
         const uint32_t bytes = A_BYTES + nb * XBOX_BYTES;
         const int xrow = sm.grp_off[g] + n0;
-        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
           if (!wait_bar(&sm.empty[s], ph ^ 1, abort_flag, p.status, ST_TIMEOUT_PRODUCER)) { ok = false; break; }
@@ -289,7 +298,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
     if (tc::elect_one()) {
       uint32_t it = 0, tcount = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++tcount) {
+      for (int wk = blockIdx.x; wk < total && ok; wk += gridDim.x, ++tcount) {
+        const int t = wk / p.ksplit, ks = wk - t * p.ksplit;
+        const int kb0 = ks * kblocks / p.ksplit, kb1 = (ks + 1) * kblocks / p.ksplit;
         int g, mt, n0, nval;
         decode_tile<BN>(sm, p.m_tiles, t, g, mt, n0, nval);
         const uint32_t buf = tcount & 1, tph = (tcount >> 1) & 1;
@@ -298,7 +309,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
         const uint32_t N = max(16, (nval + 15) & ~15);
         const uint32_t idesc = tc::idesc_bf16_f32(128, N);
         const uint32_t d = sm.tmem_base + buf * BN;
-        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
           if (!wait_bar(&sm.full[s], ph, abort_flag, p.status, ST_TIMEOUT_MMA)) { ok = false; break; }
@@ -307,7 +318,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
           const uint32_t b = a + A_BYTES;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
-            tc::mma_bf16(d, tc::sdesc_k128(a + kk * 32), tc::sdesc_k128(b + kk * 32), idesc, (kb | kk) != 0);
+            tc::mma_bf16(d, tc::sdesc_k128(a + kk * 32), tc::sdesc_k128(b + kk * 32), idesc, (kb != kb0) || kk != 0);
           tc::mma_commit(&sm.empty[s]);
         }
         if (!ok) break;
@@ -323,25 +334,63 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
     const int row = q * 32 + lane;   // tile row m (TMEM lane)
     const int etid = tid - 64;       // 0..127
     uint32_t tcount = 0;
-    for (int t = blockIdx.x; t < total; t += gridDim.x, ++tcount) {
+    for (int wk = blockIdx.x; wk < total; wk += gridDim.x, ++tcount) {
+      const int t = wk / p.ksplit, ks = wk - t * p.ksplit;
       int g, mt, n0, nval;
       decode_tile<BN>(sm, p.m_tiles, t, g, mt, n0, nval);
       const uint32_t buf = tcount & 1, tph = (tcount >> 1) & 1;
       if (!wait_bar(&sm.tfull[buf], tph, abort_flag, p.status, ST_TIMEOUT_EPILOGUE)) break;
       tc::fence_after_sync();
-      for (int c0 = 0; c0 < nval; c0 += STAGE_COLS) {
-        float v[STAGE_COLS];
-        const uint32_t taddr = sm.tmem_base + ((uint32_t)(q * 32) << 16) + buf * BN + c0;
-        tc::tmem_ld16(taddr, v);
-        tc::tmem_ld16(taddr + 16, v + 16);
-        tc::named_bar_sync(1, 128);  // staging free (previous chunk consumed)
+      if (p.ksplit == 1) {
+        for (int c0 = 0; c0 < nval; c0 += STAGE_COLS) {
+          float v[STAGE_COLS];
+          const uint32_t taddr = sm.tmem_base + ((uint32_t)(q * 32) << 16) + buf * BN + c0;
+          tc::tmem_ld16(taddr, v);
+          tc::tmem_ld16(taddr + 16, v + 16);
+          tc::named_bar_sync(1, 128);  // staging free (previous chunk consumed)
 #pragma unroll
-        for (int j = 0; j < STAGE_COLS; ++j) staging[j * 128 + row] = v[j];
+          for (int j = 0; j < STAGE_COLS; ++j) staging[j * 128 + row] = v[j];
+          tc::named_bar_sync(1, 128);
+          epilogue_chunk<BN>(p, staging, g, mt, n0, nval, c0, sm.grp_off[g], etid);
+        }
+        tc::fence_before_sync();
+        tc::mbar_arrive(&sm.tempty[buf]);
+      } else {
+        // split-K: this split's raw partial straight from TMEM (thread = row m, columns = token rows)
+        float* dst = p.partial + ks * p.part_stride;
+        const int64_t col0 = (int64_t)mt * 128 + row;
+        for (int c0 = 0; c0 < nval; c0 += STAGE_COLS) {
+          float v[STAGE_COLS];
+          const uint32_t taddr = sm.tmem_base + ((uint32_t)(q * 32) << 16) + buf * BN + c0;
+          tc::tmem_ld16(taddr, v);
+          tc::tmem_ld16(taddr + 16, v + 16);
+          const int ncols = min(STAGE_COLS, nval - c0);
+          for (int j = 0; j < ncols; ++j)
+            dst[(int64_t)(sm.grp_off[g] + n0 + c0 + j) * p.M + col0] = v[j];
+        }
+        tc::fence_before_sync();
+        tc::mbar_arrive(&sm.tempty[buf]);
+        __threadfence();
         tc::named_bar_sync(1, 128);
-        epilogue_chunk<BN>(p, staging, g, mt, n0, nval, c0, sm.grp_off[g], etid);
+        if (etid == 0) sm.is_last = (atomicAdd(&p.tile_cnt[t], 1) == p.ksplit - 1);
+        tc::named_bar_sync(1, 128);
+        if (sm.is_last) {
+          __threadfence();
+          for (int c0 = 0; c0 < nval; c0 += STAGE_COLS) {
+            const int ncols = min(STAGE_COLS, nval - c0);
+            tc::named_bar_sync(1, 128);
+            for (int j = 0; j < ncols; ++j) {
+              const int64_t off = (int64_t)(sm.grp_off[g] + n0 + c0 + j) * p.M + col0;
+              float acc = 0.f;
+              for (int sp = 0; sp < p.ksplit; ++sp) acc += __ldcg(p.partial + sp * p.part_stride + off);
+              staging[j * 128 + row] = acc;
+            }
+            tc::named_bar_sync(1, 128);
+            epilogue_chunk<BN>(p, staging, g, mt, n0, nval, c0, sm.grp_off[g], etid);
+          }
+          if (etid == 0) p.tile_cnt[t] = 0;
+        }
       }
-      tc::fence_before_sync();
-      tc::mbar_arrive(&sm.tempty[buf]);
     }
   }
   __syncthreads();
@@ -443,10 +492,52 @@ int gemm_bf16_tc(const GemmArgs& a, cudaStream_t s) {
   kp.cnt_dev = a.cnt_dev;
   kp.epi = a.epi;
   kp.status = a.status;
-  if (a.max_cnt <= 32) return launch<32, 9>(a, mw, mw2, mx, kp, s);
-  if (a.max_cnt <= 64) return launch<64, 8>(a, mw, mw2, mx, kp, s);
-  if (a.max_cnt <= 128) return launch<128, 6>(a, mw, mw2, mx, kp, s);
-  return launch<256, 4>(a, mw, mw2, mx, kp, s);
+  kp.ksplit = 1;
+  kp.partial = nullptr;
+  kp.part_stride = 0;
+  const int bn = bn_for(a.max_cnt);
+  const int ks = gemm_splitk_factor(a, bn);
+  kp.tile_cnt = nullptr;
+  if (ks > 1) {
+    DLLM_REQUIRE(a.splitk_scratch != nullptr, DLLM_ERR_WORKSPACE, "gemm: split-K needs scratch");
+    kp.ksplit = ks;
+    kp.partial = a.splitk_scratch;
+    kp.part_stride = a.x_rows * (int64_t)a.M;
+    kp.tile_cnt = reinterpret_cast<int*>(a.splitk_scratch + (size_t)ks * a.x_rows * a.M);
+    const int tiles = (a.M / 128) * ((a.max_cnt + bn - 1) / bn);
+    cudaError_t e = cudaMemsetAsync(kp.tile_cnt, 0, (size_t)tiles * sizeof(int), s);
+    if (e != cudaSuccess) return dllm_host::cuda_status(e, "gemm: cudaMemsetAsync(split-K counters)");
+  }
+  int st2;
+  if (bn == 32) st2 = launch<32, 9>(a, mw, mw2, mx, kp, s);
+  else if (bn == 64) st2 = launch<64, 8>(a, mw, mw2, mx, kp, s);
+  else if (bn == 128) st2 = launch<128, 6>(a, mw, mw2, mx, kp, s);
+  else st2 = launch<256, 4>(a, mw, mw2, mx, kp, s);
+  return st2;
+}
+
+int bn_for(int max_cnt) {
+  if (max_cnt <= 32) return 32;
+  if (max_cnt <= 64) return 64;
+  if (max_cnt <= 128) return 128;
+  return 256;
+}
+
+// Split-K for dense projections whose output tiles would leave most SMs idle (a single group of rows known on
+// the host, no SwiGLU pairing): enough K slices to give every SM a tile, at least two 64-wide K blocks each.
+int gemm_splitk_factor(const GemmArgs& a, int bn) {
+  if (a.dtype != DLLM_BF16 || a.swiglu || a.n_dev || a.has_extra) return 1;
+  const int tiles = (a.M / 128) * ((a.max_cnt + bn - 1) / bn);
+  const int kblocks = a.K / BK;
+  if (tiles <= 0 || tiles * 2 > num_sms() || kblocks < 4) return 1;
+  return std::max(1, std::min(kblocks / 2, num_sms() / tiles));
+}
+
+size_t gemm_splitk_scratch_bytes(const GemmArgs& a) {
+  const int bn = bn_for(a.max_cnt);
+  const int ks = gemm_splitk_factor(a, bn);
+  const int tiles = (a.M / 128) * ((a.max_cnt + bn - 1) / bn);
+  return ks > 1 ? (size_t)ks * a.x_rows * a.M * sizeof(float) + (size_t)tiles * sizeof(int) : 0;
 }
 
 int num_sms() {

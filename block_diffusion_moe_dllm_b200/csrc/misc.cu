@@ -35,9 +35,11 @@ int launch_embed(int dtype, const int32_t* tokens, const uint8_t* mask, int mask
 // out[r] = x[src(r)] / sqrt(mean(x^2) + eps) * g, fp32 math. src(r) = r, or through a compacted row list:
 // rows r < n come from row_pos[r], rows n <= r < 2n from row_pos[r - n] + uncond_off (n = *n_dev).
 template <typename T>
-__global__ void rmsnorm_kernel(const T* __restrict__ x, const T* __restrict__ g, T* __restrict__ out, int H,
-                               float eps, const int32_t* __restrict__ row_pos, const int32_t* __restrict__ n_dev,
-                               int two_halves, int uncond_off) {
+__global__ void __launch_bounds__(256) rmsnorm_kernel(const T* __restrict__ x, const T* __restrict__ g,
+                                                      T* __restrict__ out, int H, float eps,
+                                                      const int32_t* __restrict__ row_pos,
+                                                      const int32_t* __restrict__ n_dev, int two_halves,
+                                                      int uncond_off) {
   int r = blockIdx.x;
   int src = r;
   if (row_pos) {
@@ -46,12 +48,35 @@ __global__ void rmsnorm_kernel(const T* __restrict__ x, const T* __restrict__ g,
     src = (r < n) ? row_pos[r] : row_pos[r - n] + uncond_off;
   }
   const T* xr = x + (int64_t)src * H;
-  float ss = 0.f;
-  for (int i = threadIdx.x; i < H; i += blockDim.x) {
-    float v = to_f32(xr[i]);
-    ss += v * v;
-  }
+  T* o = out + (int64_t)r * H;
+  constexpr int VE = 16 / sizeof(T);      // elements per 16-byte vector
+  constexpr int MAXV = 4;                 // vectors kept in registers per thread
+  const int nvec = H / VE;
   __shared__ float red[32];
+  float ss = 0.f;
+  const bool vec = (H % VE == 0) && nvec <= MAXV * (int)blockDim.x && ((reinterpret_cast<uintptr_t>(xr) |
+                   reinterpret_cast<uintptr_t>(o) | reinterpret_cast<uintptr_t>(g)) & 15) == 0;
+  uint4 keep[MAXV];
+  if (vec) {
+#pragma unroll
+    for (int k = 0; k < MAXV; ++k) {
+      const int i = threadIdx.x + k * blockDim.x;
+      if (i < nvec) {
+        keep[k] = reinterpret_cast<const uint4*>(xr)[i];
+        const T* e = reinterpret_cast<const T*>(&keep[k]);
+#pragma unroll
+        for (int u = 0; u < VE; ++u) {
+          const float v = to_f32(e[u]);
+          ss += v * v;
+        }
+      }
+    }
+  } else {
+    for (int i = threadIdx.x; i < H; i += blockDim.x) {
+      float v = to_f32(xr[i]);
+      ss += v * v;
+    }
+  }
   ss = warp_sum(ss);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
   __syncthreads();
@@ -62,8 +87,24 @@ __global__ void rmsnorm_kernel(const T* __restrict__ x, const T* __restrict__ g,
   }
   __syncthreads();
   const float inv = 1.0f / sqrtf(red[0] / (float)H + eps);
-  T* o = out + (int64_t)r * H;
-  for (int i = threadIdx.x; i < H; i += blockDim.x) o[i] = from_f32<T>(to_f32(xr[i]) * inv * to_f32(g[i]));
+  if (vec) {
+#pragma unroll
+    for (int k = 0; k < MAXV; ++k) {
+      const int i = threadIdx.x + k * blockDim.x;
+      if (i < nvec) {
+        const uint4 gv = reinterpret_cast<const uint4*>(g)[i];
+        const T* e = reinterpret_cast<const T*>(&keep[k]);
+        const T* ge = reinterpret_cast<const T*>(&gv);
+        uint4 res;
+        T* re = reinterpret_cast<T*>(&res);
+#pragma unroll
+        for (int u = 0; u < VE; ++u) re[u] = from_f32<T>(to_f32(e[u]) * inv * to_f32(ge[u]));
+        reinterpret_cast<uint4*>(o)[i] = res;
+      }
+    }
+  } else {
+    for (int i = threadIdx.x; i < H; i += blockDim.x) o[i] = from_f32<T>(to_f32(xr[i]) * inv * to_f32(g[i]));
+  }
 }
 
 int launch_rmsnorm(int dtype, const void* x, const void* g, void* out, int rows, int H, float eps,
@@ -152,32 +193,38 @@ int launch_gather_rows(int dtype, const void* h, const int32_t* perm, int k, int
 // ------------------------------------------------------------------------------------------------ combine
 // x[t] = x[t] + (y[Tk*k + t] + sum_j gates[t, j] * y[inv[t*k + j]]), summed in fp32 in slot order, rounded once.
 template <typename T>
-__global__ void combine_kernel(T* __restrict__ x, const float* __restrict__ y, const float* __restrict__ gates,
-                               const int32_t* __restrict__ inv, int k, int n_assign, int shared, int H) {
+__global__ void __launch_bounds__(128) combine_kernel(T* __restrict__ x, const float* __restrict__ y,
+                                                      const float* __restrict__ gates, const int32_t* __restrict__ inv,
+                                                      int k, int n_assign, int shared, int H) {
+  // grid (tokens, H / 512): each thread owns 4 consecutive hidden elements
   const int t = blockIdx.x;
-  __shared__ int rows[32];
-  __shared__ float gs[32];
-  if (threadIdx.x < k) {
-    rows[threadIdx.x] = inv[t * k + threadIdx.x];
-    gs[threadIdx.x] = gates[t * k + threadIdx.x];
+  const int h0 = (blockIdx.y * blockDim.x + threadIdx.x) * 4;
+  if (h0 >= H) return;
+  float4 acc = shared ? *reinterpret_cast<const float4*>(y + (int64_t)(n_assign + t) * H + h0)
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int j = 0; j < k; ++j) {
+    const float gj = gates[t * k + j];
+    const float4 v = *reinterpret_cast<const float4*>(y + (int64_t)inv[t * k + j] * H + h0);
+    acc.x += gj * v.x;
+    acc.y += gj * v.y;
+    acc.z += gj * v.z;
+    acc.w += gj * v.w;
   }
-  __syncthreads();
-  const float* ys = y + (int64_t)(n_assign + t) * H;
-  T* xr = x + (int64_t)t * H;
-  for (int i = threadIdx.x; i < H; i += blockDim.x) {
-    float acc = shared ? ys[i] : 0.f;
-    for (int j = 0; j < k; ++j) acc += gs[j] * y[(int64_t)rows[j] * H + i];
-    xr[i] = from_f32<T>(to_f32(xr[i]) + acc);
-  }
+  T* xr = x + (int64_t)t * H + h0;
+  xr[0] = from_f32<T>(to_f32(xr[0]) + acc.x);
+  xr[1] = from_f32<T>(to_f32(xr[1]) + acc.y);
+  xr[2] = from_f32<T>(to_f32(xr[2]) + acc.z);
+  xr[3] = from_f32<T>(to_f32(xr[3]) + acc.w);
 }
 
 int launch_combine(int dtype, void* x, const float* y, const float* gates, const int32_t* inv, int k, int Tk,
                    int shared, int H, cudaStream_t s) {
   if (Tk <= 0) return DLLM_OK;
+  dim3 grid(Tk, (H / 4 + 127) / 128);
   if (dtype == DLLM_BF16)
-    combine_kernel<__nv_bfloat16><<<Tk, 256, 0, s>>>((__nv_bfloat16*)x, y, gates, inv, k, Tk * k, shared, H);
+    combine_kernel<__nv_bfloat16><<<grid, 128, 0, s>>>((__nv_bfloat16*)x, y, gates, inv, k, Tk * k, shared, H);
   else
-    combine_kernel<float><<<Tk, 256, 0, s>>>((float*)x, y, gates, inv, k, Tk * k, shared, H);
+    combine_kernel<float><<<grid, 128, 0, s>>>((float*)x, y, gates, inv, k, Tk * k, shared, H);
   DLLM_CHECK_LAUNCH("combine_kernel");
   return DLLM_OK;
 }
@@ -246,8 +293,11 @@ __global__ void simt_gemm_f32_kernel(const float* __restrict__ X, const float* _
     }
 }
 
-// Epilogue of the fp32 path over every valid row of every group.
-__global__ void simt_epilogue_f32_kernel(const float* __restrict__ raw, int Mw, int M, SimtGroups G, EpiParams e) {
+// Epilogue of the fp32 SIMT path from raw fp32 products, over every valid row of every group (nsplit partials
+// split_stride elements apart are summed first). T is the storage type.
+template <typename T>
+__global__ void raw_epilogue_kernel(const float* __restrict__ raw, int nsplit, int64_t split_stride, int Mw, int M,
+                                    SimtGroups G, EpiParams e) {
   const int g = blockIdx.y;
   int off, cnt;
   group_of(G, g, off, cnt);
@@ -255,18 +305,23 @@ __global__ void simt_epilogue_f32_kernel(const float* __restrict__ raw, int Mw, 
   if (n >= cnt) return;
   const int row = off + n;
   const float* rr = raw + (int64_t)row * Mw;
+  auto val = [&](int f) {
+    float v = rr[f];
+    for (int s = 1; s < nsplit; ++s) v += rr[s * split_stride + f];
+    return v;
+  };
   if (e.kind == EPI_SWIGLU) {
-    float* out = static_cast<float*>(e.out);
+    T* out = static_cast<T*>(e.out);
     for (int i = threadIdx.x; i < M; i += blockDim.x) {
-      float gt = rr[i], up = rr[M + i];
-      out[(int64_t)row * e.ldo + i] = gt / (1.0f + expf(-gt)) * up;
+      float gt = val(i), up = val(M + i);
+      out[(int64_t)row * e.ldo + i] = from_f32<T>(gt / (1.0f + expf(-gt)) * up);
     }
   } else if (e.kind == EPI_QKV) {
     const int d = e.d, half = d / 2, nh = e.Hq + 2 * e.Hkv;
     const int b = row / e.L, i = row % e.L, pos = e.pos0 + i;
     for (int idx = threadIdx.x; idx < nh * half; idx += blockDim.x) {
       const int hh = idx / half, m = idx % half;
-      float x1 = rr[hh * d + m], x2 = rr[hh * d + m + half];
+      float x1 = val(hh * d + m), x2 = val(hh * d + m + half);
       float y1 = x1, y2 = x2;
       if (hh < e.Hq + e.Hkv) {
         double sn, cs;
@@ -275,28 +330,35 @@ __global__ void simt_epilogue_f32_kernel(const float* __restrict__ raw, int Mw, 
         y1 = x1 * c - x2 * s;
         y2 = x2 * c + x1 * s;
       }
-      float* dst;
+      const T t1 = from_f32<T>(y1), t2 = from_f32<T>(y2);
+      T* dst;
       if (hh < e.Hq) {
-        dst = static_cast<float*>(e.q_out) + ((int64_t)row * e.Hq + hh) * d;
+        dst = static_cast<T*>(e.q_out) + ((int64_t)row * e.Hq + hh) * d;
       } else {
         const bool is_k = hh < e.Hq + e.Hkv;
         const int gk = is_k ? hh - e.Hq : hh - e.Hq - e.Hkv;
-        dst = static_cast<float*>(is_k ? e.k_dst : e.v_dst) + (((int64_t)b * e.Hkv + gk) * e.cap + e.slot0 + i) * d;
+        dst = static_cast<T*>(is_k ? e.k_dst : e.v_dst) + (((int64_t)b * e.Hkv + gk) * e.cap + e.slot0 + i) * d;
         void* d2v = is_k ? e.k_dst2 : e.v_dst2;
         if (d2v) {
-          float* d2 = static_cast<float*>(d2v) + (((int64_t)b * e.Hkv + gk) * e.cap2 + e.slot2 + i) * d;
-          d2[m] = y1;
-          d2[m + half] = y2;
+          T* d2 = static_cast<T*>(d2v) + (((int64_t)b * e.Hkv + gk) * e.cap2 + e.slot2 + i) * d;
+          d2[m] = t1;
+          d2[m + half] = t2;
         }
       }
-      dst[m] = y1;
-      dst[m + half] = y2;
+      dst[m] = t1;
+      dst[m + half] = t2;
     }
-  } else {
+  } else if (e.out_f32) {
     float* out = static_cast<float*>(e.out);
     for (int f = threadIdx.x; f < M; f += blockDim.x) {
       int64_t o = (int64_t)row * e.ldo + f;
-      out[o] = (e.kind == EPI_RESID) ? out[o] + rr[f] : rr[f];
+      out[o] = (e.kind == EPI_RESID) ? out[o] + val(f) : val(f);
+    }
+  } else {
+    T* out = static_cast<T*>(e.out);
+    for (int f = threadIdx.x; f < M; f += blockDim.x) {
+      int64_t o = (int64_t)row * e.ldo + f;
+      out[o] = from_f32<T>((e.kind == EPI_RESID) ? to_f32(out[o]) + val(f) : val(f));
     }
   }
 }
@@ -316,8 +378,8 @@ int gemm_f32_simt(const GemmArgs& a, cudaStream_t s) {
                                             a.w_group_stride, G, a.f32_scratch);
   DLLM_CHECK_LAUNCH("simt_gemm_f32_kernel");
   dim3 g2(max_cnt, n_groups);
-  simt_epilogue_f32_kernel<<<g2, 128, 0, s>>>(a.f32_scratch, Mw, a.M, G, a.epi);
-  DLLM_CHECK_LAUNCH("simt_epilogue_f32_kernel");
+  raw_epilogue_kernel<float><<<g2, 128, 0, s>>>(a.f32_scratch, 1, 0, Mw, a.M, G, a.epi);
+  DLLM_CHECK_LAUNCH("raw_epilogue_kernel");
   return DLLM_OK;
 }
 

@@ -56,8 +56,15 @@ struct AttnArgs {
   void* ws;
   size_t ws_bytes;
 };
-size_t attn_workspace_bytes(int B, int Lq, int Hq, int Hkv, int d, int n_keys);
-int launch_attn(const AttnArgs& a, cudaStream_t s);
+size_t attn_workspace_bytes(int B, int Lq, int Hq, int Hkv, int d, int n_keys, int dtype);
+int launch_attn(const AttnArgs& a, int32_t* status, cudaStream_t s);
+// SIMT (any storage type) and tensor-core (bf16, d = 128) variants
+size_t attn_simt_workspace_bytes(int B, int Lq, int Hq, int Hkv, int d, int n_keys);
+int launch_attn_simt(const AttnArgs& a, cudaStream_t s);
+bool attn_tc_supported(int dtype, int Hq, int Hkv, int d);
+size_t attn_tc_workspace_bytes(int B, int Lq, int Hq, int Hkv, int n_keys);
+int launch_attn_tc(const AttnArgs& a, int32_t* status, cudaStream_t s);
+int launch_attn_merge(const AttnArgs& a, int n_splits, float* po, float* pm, float* pl, cudaStream_t s);
 
 // SPRINT retention
 struct RetainArgs {

@@ -8,8 +8,8 @@
 namespace dllm {
 namespace {
 
-constexpr int TPB = 8;   // tokens per CTA of the score kernel
-constexpr int EC = 32;   // experts per CTA of the score kernel
+constexpr int TT = 16;   // tokens per CTA of the score kernel
+constexpr int EW = 8;    // experts per CTA (one per warp)
 
 DLLM_DEV void load8(const __nv_bfloat16* p, float* f) { bf16x8_to_f32(*reinterpret_cast<const uint4*>(p), f); }
 DLLM_DEV void load8(const float* p, float* f) {
@@ -17,40 +17,49 @@ DLLM_DEV void load8(const float* p, float* f) {
   f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w; f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
 }
 
-// scores[t, e] = sigmoid(sum_i h[t, i] w[e, i]) in fp32. Lane l accumulates 8-element groups l, l + 32, ...
-// sequentially, then a fixed butterfly adds the lanes: the order is the same on every run.
+// scores[t, e] = sigmoid(sum_i h[t, i] w[e, i]) in fp32. One warp per expert streams its router row in 8-element
+// vectors (lane l owns elements l*8 + 256 j + u) and applies each vector to the CTA's TT token rows held in shared
+// memory; each lane sums its elements in increasing j, u, then a fixed butterfly adds the lanes, so the order of
+// the fp32 sum is the same on every run.
 template <typename T>
-__global__ void route_scores_kernel(const T* __restrict__ h, const T* __restrict__ w, int Tk, int H, int E,
-                                    float* __restrict__ scores) {
-  extern __shared__ float hs[];  // [TPB][H]
-  const int t0 = blockIdx.x * TPB, e0 = blockIdx.y * EC;
-  const int nt = min(TPB, Tk - t0);
-  for (int i = threadIdx.x; i < TPB * H; i += blockDim.x) {
-    int tt = i / H, c = i - tt * H;
-    hs[i] = tt < nt ? to_f32(h[(int64_t)(t0 + tt) * H + c]) : 0.f;
+__global__ void __launch_bounds__(256) route_scores_kernel(const T* __restrict__ h, const T* __restrict__ w, int Tk,
+                                                           int H, int E, float* __restrict__ scores) {
+  extern __shared__ __align__(16) unsigned char hs_raw[];
+  T* hs = reinterpret_cast<T*>(hs_raw);  // [TT][H]
+  const int e0 = blockIdx.x * EW, t0 = blockIdx.y * TT;
+  const int nt = min(TT, Tk - t0);
+  const int vec = 16 / (int)sizeof(T);
+  const int nvec = TT * H / vec;
+  for (int i = threadIdx.x; i < nvec; i += blockDim.x) {
+    const int tt = (i * vec) / H;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (tt < nt) v = reinterpret_cast<const uint4*>(h + (int64_t)t0 * H)[i];
+    reinterpret_cast<uint4*>(hs)[i] = v;
   }
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int e = e0 + warp; e < min(E, e0 + EC); e += (blockDim.x >> 5)) {
-    const T* wr = w + (int64_t)e * H;
-    float acc[TPB];
+  const int e = e0 + warp;
+  if (e >= E) return;
+  const T* wr = w + (int64_t)e * H;
+  float acc[TT];
 #pragma unroll
-    for (int tt = 0; tt < TPB; ++tt) acc[tt] = 0.f;
-    for (int c = lane * 8; c < H; c += 256) {
-      float wf[8];
-      load8(wr + c, wf);
+  for (int tt = 0; tt < TT; ++tt) acc[tt] = 0.f;
+#pragma unroll 4
+  for (int c = lane * 8; c < H; c += 256) {
+    float wf[8];
+    load8(wr + c, wf);
 #pragma unroll
-      for (int tt = 0; tt < TPB; ++tt) {
-        const float* hr = hs + tt * H + c;
+    for (int tt = 0; tt < TT; ++tt) {
+      float hf[8];
+      load8(hs + tt * H + c, hf);
 #pragma unroll
-        for (int u = 0; u < 8; ++u) acc[tt] = fmaf(wf[u], hr[u], acc[tt]);
-      }
+      for (int u = 0; u < 8; ++u) acc[tt] = fmaf(wf[u], hf[u], acc[tt]);
     }
+  }
 #pragma unroll
-    for (int tt = 0; tt < TPB; ++tt) {
-      float v = warp_sum(acc[tt]);
-      if (lane == 0 && tt < nt) scores[(int64_t)(t0 + tt) * E + e] = 1.0f / (1.0f + expf(-v));
-    }
+  for (int tt = 0; tt < TT; ++tt) {
+    const float v = warp_sum(acc[tt]);
+    if (lane == 0 && tt < nt) scores[(int64_t)(t0 + tt) * E + e] = 1.0f / (1.0f + expf(-v));
   }
 }
 
@@ -188,8 +197,8 @@ int launch_route(int dtype, const void* h, const void* w_router, const float* bi
                  int32_t* ids, float* gates, float* scores, int32_t* counts, int32_t* offsets, int32_t* perm,
                  int32_t* inv, cudaStream_t s) {
   if (Tk <= 0) return DLLM_OK;
-  dim3 g1((Tk + TPB - 1) / TPB, (E + EC - 1) / EC);
-  const size_t smem = (size_t)TPB * H * sizeof(float);
+  dim3 g1((E + EW - 1) / EW, (Tk + TT - 1) / TT);
+  const size_t smem = (size_t)TT * H * (dtype == DLLM_BF16 ? 2 : 4);
   if (dtype == DLLM_BF16) {
     static bool cfg = false;
     if (!cfg) {

@@ -90,6 +90,22 @@ class DenoiseEngine:
             self.step(t, stream)
         self.commit(stream)
 
+    def capture_block(self, tokens0=None, mask0=None):
+        """A CUDA graph of one block: optional reset of the block state from device tensors, the T_s passes and the
+        commit pass, captured once (kernel launches and their arguments are fixed; the block's data is not)."""
+        for _ in range(2):                                  # warm the library's one-time set-up outside capture
+            if tokens0 is not None:
+                self.set_block(tokens0, mask0)
+            self.decode_block()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            if tokens0 is not None:
+                self.tokens.copy_(tokens0)
+                self.mask.copy_(mask0)
+            self.decode_block(torch.cuda.current_stream())
+        return g
+
     def views(self, t=0):
         p = self.params(t)
         v = bd.StepViews()

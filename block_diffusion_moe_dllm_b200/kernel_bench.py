@@ -27,15 +27,23 @@ def hbm_peak():
     return 6650.0, "fallback"
 
 
-def timed(fn, reps, stream, warm=3):
+def timed(fn, reps, stream=None, warm=3):
+    """GPU time of one call: `reps` calls captured in a CUDA graph, the replay timed with CUDA events (host-side
+    launch cost excluded)."""
     for _ in range(warm):
         fn()
     torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(reps):
+            fn()
+    g.replay()
+    torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(reps):
-        fn()
-    b.record(stream)
+    a.record(s)
+    g.replay()
+    b.record(s)
     torch.cuda.synchronize()
     return a.elapsed_time(b) / 1000.0 / max(reps, 1)
 
@@ -56,7 +64,7 @@ def bench_lm_head(w: Workload, reps, dev, stream, weights=None):
     x = synth.normal((rows, w.H), 1.0, 1, "kb_x", dev)
     y = torch.empty((rows, w.vlen), dtype=torch.bfloat16, device=dev)
     ws = bd.Workspace(1 << 16, dev)
-    t = timed(lambda: bd.gemm(x, wl, y, rows, w.vlen, w.H, bd.BF16, ws=ws, stream=stream), reps, stream)
+    t = timed(lambda: bd.gemm(x, wl, y, rows, w.vlen, w.H, bd.BF16, ws=ws), reps, stream)
     nbytes = w.vlen * w.H * 2 + rows * w.H * 2 + rows * w.vlen * 2
     return _result("gemm_tc_kernel[lm_head]", t, nbytes, {"rows": rows, "M": w.vlen, "K": w.H})
 
@@ -74,16 +82,16 @@ def bench_experts(w: Workload, reps, dev, stream, weights=None):
     inv = torch.empty(rows * w.k, dtype=torch.int32, device=dev)
     ws = bd.Workspace(1 << 20, dev)
     bd.moe_route(h, lw["w_router"], lw["router_bias"], ids, gates, counts, offsets, perm, inv, rows, w.H, w.E, w.k,
-                 bd.BF16, ws=ws, stream=stream)
+                 bd.BF16, ws=ws)
     torch.cuda.synchronize()
     active = int((counts > 0).sum().item())
     x = torch.zeros((rows, w.H), dtype=torch.bfloat16, device=dev)
     t = timed(lambda: bd.moe_experts(h, lw["w_gu"], lw["w_down"], lw["w_gu_shared"], lw["w_down_shared"], counts,
-                                     offsets, perm, inv, gates, x, rows, w.H, w.E, w.k, w.I, bd.BF16, ws=ws,
-                                     stream=stream), reps, stream)
+                                     offsets, perm, inv, gates, x, rows, w.H, w.E, w.k, w.I, bd.BF16, ws=ws),
+              reps, stream)
     nbytes = (active + 1) * 3 * w.I * w.H * 2 + 2 * rows * w.H * 2
     troute = timed(lambda: bd.moe_route(h, lw["w_router"], lw["router_bias"], ids, gates, counts, offsets, perm, inv,
-                                        rows, w.H, w.E, w.k, bd.BF16, ws=ws, stream=stream), reps, stream)
+                                        rows, w.H, w.E, w.k, bd.BF16, ws=ws), reps, stream)
     rbytes = w.E * w.H * 2 + rows * w.H * 2
     return [_result("moe_experts[gather+gemm_tc x2+combine]", t, nbytes, {"active_experts": active, "rows": rows}),
             _result("moe_route[scores+topk+permute]", troute, rbytes, {"rows": rows})]
@@ -108,7 +116,7 @@ def bench_unmask(w: Workload, reps, dev, stream):
         msk.copy_(msk0)
         bd.unmask(logits, row_pos, n_dev, tok, msk, sel, nsel, conf, rem, Bl, w.L, w.vlen, n, 0, w.T_s, bd.BF16,
                   mode=w.mode, tau=w.tau, k_max=w.k_max, cfg=w.cfg, cfg_scale=w.cfg_scale,
-                  vocab_offset=w.vocab_offset, ws=ws, stream=stream)
+                  vocab_offset=w.vocab_offset, ws=ws)
     t = timed(call, reps, stream)
     nbytes = logits.numel() * 2
     return _result("unmask[reduce+select]", t, nbytes, {"rows": n, "V": w.vlen})
@@ -123,7 +131,7 @@ def bench_attn(w: Workload, reps, dev, stream):
     out = torch.empty((w.B, w.L, w.Hq * w.d), dtype=torch.bfloat16, device=dev)
     ws = bd.Workspace(1 << 26, dev)
     t = timed(lambda: bd.block_attn(q, kc, vc, out, w.B, w.L, w.Hq, w.Hkv, w.d, w.L, w.P, n_keys, cap, bd.BF16,
-                                    ws=ws, stream=stream), reps, stream)
+                                    ws=ws), reps, stream)
     nbytes = 2 * w.B * w.Hkv * n_keys * w.d * 2 + 2 * w.B * w.L * w.Hq * w.d * 2
     flops = 4.0 * w.B * w.L * w.Hq * n_keys * w.d
     return _result("block_attn", t, nbytes, {"keys": n_keys, "TFLOP/s": flops / t / 1e12})

@@ -37,6 +37,18 @@ def test_gemm_bf16_store(N, M, K):
     assert_close(to64(y), want, "bf16", "gemm")
 
 
+@pytest.mark.parametrize("N,M,K", [(32, 3072, 2048), (32, 2048, 2048), (7, 256, 1024)])
+def test_gemm_bf16_split_k(N, M, K):
+    """Few output tiles: the K reduction is split across CTAs and summed by the epilogue kernel."""
+    x = synth.normal((N, K), 1.0, 9, f"skx{N}", DEV)
+    w = synth.normal((M, K), 0.02, 9, f"skw{M}", DEV)
+    y0 = synth.normal((N, M), 1.0, 9, f"sky{N}{M}", DEV)
+    y = y0.clone()
+    bd.gemm(x, w, y, N, M, K, bd.BF16, residual=1)
+    torch.cuda.synchronize()
+    assert_close(to64(y), O.store(to64(y0) + to64(x) @ to64(w).T, "bf16"), "bf16", "split-K gemm")
+
+
 def test_gemm_bf16_residual_and_device_count():
     N, M, K = 40, 256, 256
     x = synth.normal((N, K), 1.0, 2, "rx", DEV)
@@ -133,11 +145,14 @@ def test_experts(dtype, Tk, H, E, k, I, shared):
 
 
 # ------------------------------------------------------------------------------------------------ attention
-def _attn_case(dtype, B, Lq, Hq, Hkv, d, blk, q_pos0, n_keys, cap, key_pos=None, seed=0):
+def _attn_case(dtype, B, Lq, Hq, Hkv, d, blk, q_pos0, n_keys, cap, key_pos=None, seed=0, nan_tail=False):
     t = _tdt(dtype)
     q = synth.normal((B, Lq, Hq, d), 1.0, seed, "aq", DEV, t)
     kc = synth.normal((B, Hkv, cap, d), 1.0, seed, "ak", DEV, t)
     vc = synth.normal((B, Hkv, cap, d), 1.0, seed, "av", DEV, t)
+    if nan_tail:      # cache rows past n_keys are never read
+        kc[:, :, n_keys:] = float("nan")
+        vc[:, :, n_keys:] = float("nan")
     out = torch.full((B, Lq, Hq * d), float("nan"), dtype=t, device=DEV)
     kp = None if key_pos is None else torch.from_numpy(key_pos.astype(np.int32)).to(DEV)
     bd.block_attn(q, kc, vc, out, B, Lq, Hq, Hkv, d, blk, q_pos0, n_keys, cap, DT[dtype], key_pos=kp)
@@ -179,6 +194,16 @@ def test_attention_ragged_queries_small_blocks():
 
 def test_attention_long_prefix_split():
     _attn_case("bf16", 2, 32, 16, 4, 128, 32, 4096, 4128, 4128, seed=5)
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (16, 2), (8, 4), (32, 1)])
+def test_attention_group_sizes(Hq, Hkv):
+    _attn_case("bf16", 2, 32, Hq, Hkv, 128, 32, 160, 192, 200, seed=7)
+
+
+def test_attention_cache_tail_never_read():
+    _attn_case("bf16", 2, 32, 16, 4, 128, 32, 200, 232, 300, seed=8, nan_tail=True)
+    _attn_case("f32", 1, 16, 4, 4, 64, 16, 40, 56, 80, seed=8, nan_tail=True)
 
 
 def test_attention_f32_mha():

@@ -273,8 +273,8 @@ def kernel_rooflines(w, wt, eng, dev, stream):
     GEMM (one launch of gemm_tc_kernel streaming 157184 x 2048 bf16) is the roofline kernel."""
     from block_diffusion_moe_dllm_b200 import kernel_bench as kb
     lm = kb.bench_lm_head(w, 20, dev, stream, weights=wt)
-    rest = kb.bench_experts(w, 20, dev, stream, weights=wt) + [kb.bench_unmask(w, 20, dev, stream),
-                                                               kb.bench_attn(w, 20, dev, stream)]
+    rest = (kb.bench_proj(w, 20, dev, stream, weights=wt) + kb.bench_experts(w, 20, dev, stream, weights=wt) +
+            [kb.bench_unmask(w, 20, dev, stream), kb.bench_attn(w, 20, dev, stream)])
     kernels = {r["kernel"]: {k: v for k, v in r.items() if k != "kernel"} for r in [lm] + rest}
     roof = {"kernel": "gemm_tc_kernel (LM head 157184x2048 bf16, 32 rows)", "bound": "hbm",
             "achieved": lm["GB/s"], "peak": lm["peak_GBs"], "unit": "GB/s", "frac": lm["frac_hbm"],

@@ -64,13 +64,6 @@ int check_ws(void* ws, size_t ws_bytes, size_t need) {
 int32_t* status_word(void* ws) { return static_cast<int32_t*>(ws); }
 
 // ------------------------------------------------------------------------------------------------ GEMM dispatch
-// Scratch a dense projection of `rows` rows needs for split-K (0 when it does not split).
-size_t dense_splitk_bytes(int dtype, int64_t rows, int M, int K) {
-  GemmArgs a;
-  a.dtype = dtype; a.x_rows = rows; a.M = M; a.K = K; a.max_cnt = (int)rows; a.host_cnt = (int)rows;
-  return gemm_splitk_scratch_bytes(a);
-}
-
 int run_gemm(GemmArgs& a, cudaStream_t s) {
   return a.dtype == DLLM_BF16 ? gemm_bf16_tc(a, s) : gemm_f32_simt(a, s);
 }
@@ -145,7 +138,6 @@ struct StepPlan {
   int32_t* inv;
   ExpertBufs eb;
   float* proj_scratch;
-  float* splitk;
   int32_t* row_pos;
   int32_t* n_rows;
   void* xf;
@@ -166,7 +158,8 @@ int validate_step(const dllm_model* m, const dllm_state* st, const dllm_step_par
   REQ(m->H % 8 == 0, DLLM_ERR_SHAPE, "denoise_step: H must be a multiple of 8");
   REQ((size_t)16 * m->H * (m->dtype == DLLM_BF16 ? 2 : 4) <= 200 * 1024, DLLM_ERR_UNSUPPORTED,
       "denoise_step: H too large for the router");
-  REQ(st->B >= 1 && st->L >= 1 && st->L <= 32 && st->P >= 0, DLLM_ERR_SHAPE, "denoise_step: bad B/L/P");
+  REQ(st->B >= 1 && st->B <= 1024 && st->L >= 1 && st->L <= 32 && st->P >= 0, DLLM_ERR_SHAPE,
+      "denoise_step: bad B/L/P (B <= 1024, L <= 32)");
   REQ(st->cap >= st->P + st->L, DLLM_ERR_SHAPE, "denoise_step: cap %d < P + L", st->cap);
   REQ(st->tokens && st->mask, DLLM_ERR_INVALID_ARG, "denoise_step: NULL tokens/mask");
   REQ(m->embed && m->final_norm && m->w_lm, DLLM_ERR_INVALID_ARG, "denoise_step: NULL embed/final_norm/w_lm");
@@ -236,13 +229,6 @@ void plan_step(const dllm_model* m, const dllm_state* st, const dllm_step_params
                        ? c.take<float>((size_t)std::max(s.Tk, s.halves * s.max_rows) *
                                        std::max(std::max(proj_n, H), s.vlen) * 4)
                        : nullptr;
-  {
-    const size_t a = dense_splitk_bytes(m->dtype, s.Tk, proj_n, H);
-    const size_t b = dense_splitk_bytes(m->dtype, s.Tk, H, QD);
-    const size_t l = dense_splitk_bytes(m->dtype, (int64_t)s.halves * s.max_rows, s.vlen, H);
-    const size_t need = std::max(a, std::max(b, l));
-    s.splitk = need ? c.take<float>(need) : nullptr;
-  }
   s.row_pos = c.take<int32_t>((size_t)s.max_rows * 4);
   s.n_rows = c.take<int32_t>(16);
   s.xf = c.take((size_t)s.halves * s.max_rows * H * es);
@@ -282,7 +268,6 @@ size_t dllm_gemm_workspace_size(const dllm_gemm_desc* d) {
   if (!d) return 0;
   size_t n = kStatusBytes;
   if (d->dtype == DLLM_F32) n = align256(n) + gemm_f32_scratch_bytes(d->N, d->M, 0);
-  else n = align256(n) + dense_splitk_bytes(d->dtype, d->N, d->M, d->K);
   return align256(n);
 }
 
@@ -304,10 +289,6 @@ int dllm_gemm(const dllm_gemm_desc* d, const void* x, const void* w, void* y, co
   a.cnt_dev = n_rows_dev; a.host_cnt = d->N; a.max_cnt = d->N; a.cnt_bound = d->N;
   a.dtype = d->dtype; a.status = status_word(ws);
   a.f32_scratch = d->dtype == DLLM_F32 ? c.take<float>(gemm_f32_scratch_bytes(d->N, d->M, 0)) : nullptr;
-  if (d->dtype == DLLM_BF16) {
-    const size_t sk = dense_splitk_bytes(d->dtype, d->N, d->M, d->K);
-    a.splitk_scratch = sk ? c.take<float>(sk) : nullptr;
-  }
   a.epi.kind = d->residual ? EPI_RESID : EPI_STORE;
   a.epi.out = y; a.epi.ldo = d->ldy; a.epi.out_f32 = d->y_f32 || d->dtype == DLLM_F32;
   return run_gemm(a, stream);
@@ -439,8 +420,9 @@ int dllm_unmask(const dllm_unmask_desc* d, const void* logits, const int32_t* ro
                 void* ws, size_t ws_bytes, cudaStream_t stream) {
   REQ(d && logits && row_pos && n_rows_dev && tokens && mask && sel && nsel && conf && remaining,
       DLLM_ERR_INVALID_ARG, "unmask: NULL argument");
-  REQ(d->B >= 1 && d->L >= 1 && d->L <= 32 && d->V >= 1 && d->max_rows >= 0 && d->max_rows <= d->B * d->L,
-      DLLM_ERR_SHAPE, "unmask: bad shape (L <= 32, max_rows <= B*L)");
+  REQ(d->B >= 1 && d->B <= 1024 && d->L >= 1 && d->L <= 32 && d->V >= 1 && d->max_rows >= 0 &&
+          d->max_rows <= d->B * d->L,
+      DLLM_ERR_SHAPE, "unmask: bad shape (B <= 1024, L <= 32, max_rows <= B*L)");
   REQ(d->T_s >= 1 && d->t >= 0 && d->t < d->T_s, DLLM_ERR_INVALID_ARG, "unmask: step %d of %d", d->t, d->T_s);
   REQ(d->mode == DLLM_UNMASK_FIXED || d->mode == DLLM_UNMASK_THRESHOLD, DLLM_ERR_INVALID_ARG, "unmask: bad mode");
   REQ(d->mode == DLLM_UNMASK_FIXED || d->k_max >= 1, DLLM_ERR_INVALID_ARG, "unmask: k_max must be >= 1");
@@ -519,7 +501,7 @@ int dllm_denoise_step(const dllm_model* m, const dllm_state* st, const dllm_step
     GemmArgs g;
     g.x = s.h; g.x_rows = s.Tk; g.w = Ly.w_qkv; g.w_rows = (int64_t)(m->Hq + 2 * m->Hkv) * m->d; g.K = H;
     g.M = (m->Hq + 2 * m->Hkv) * m->d; g.host_cnt = s.Tk; g.max_cnt = s.Tk; g.cnt_bound = s.Tk; g.dtype = dt;
-    g.status = status; g.f32_scratch = s.proj_scratch; g.splitk_scratch = s.splitk;
+    g.status = status; g.f32_scratch = s.proj_scratch;
     g.epi.kind = EPI_QKV; g.epi.q_out = s.q; g.epi.Hq = m->Hq; g.epi.Hkv = m->Hkv; g.epi.d = m->d; g.epi.L = L;
     g.epi.pos0 = P; g.epi.rope_base = m->rope_base;
     if (p->sprint) {
@@ -540,7 +522,6 @@ int dllm_denoise_step(const dllm_model* m, const dllm_state* st, const dllm_step
     GemmArgs go;
     go.x = s.ao; go.x_rows = s.Tk; go.w = Ly.w_o; go.w_rows = H; go.K = QD; go.M = H; go.host_cnt = s.Tk;
     go.max_cnt = s.Tk; go.cnt_bound = s.Tk; go.dtype = dt; go.status = status; go.f32_scratch = s.proj_scratch;
-    go.splitk_scratch = s.splitk;
     go.epi.kind = EPI_RESID; go.epi.out = s.x; go.epi.ldo = H; go.epi.out_f32 = dt == DLLM_F32;
     TRY(run_gemm(go, stream));
     if (p->commit && last) break;  // the last layer's FFN output has no consumer in a commit pass
@@ -560,7 +541,7 @@ int dllm_denoise_step(const dllm_model* m, const dllm_state* st, const dllm_step
   gl.w = static_cast<const char*>(m->w_lm) + (size_t)p->vocab_offset * H * es; gl.w_rows = s.vlen;
   gl.K = H; gl.M = s.vlen; gl.cnt_dev = s.n_rows + 1; gl.host_cnt = s.halves * s.max_rows;
   gl.max_cnt = s.halves * s.max_rows; gl.cnt_bound = s.halves * s.max_rows; gl.dtype = dt; gl.status = status;
-  gl.f32_scratch = s.proj_scratch; gl.splitk_scratch = s.splitk;
+  gl.f32_scratch = s.proj_scratch;
   gl.epi.kind = EPI_STORE; gl.epi.out = s.logits; gl.epi.ldo = s.vlen; gl.epi.out_f32 = dt == DLLM_F32;
   TRY(run_gemm(gl, stream));
   UnmaskArgs ua;

@@ -48,15 +48,12 @@ struct Smem {
   int grp_off[MAX_GROUPS];
   int grp_cnt[MAX_GROUPS];
   int chunk_sum[NUM_THREADS];
-  int is_last;
 };
 
 struct KParams {
   int K, M, swiglu, m_tiles;
-  int ksplit;              // > 1: split-K; each split writes its raw fp32 partial, the last split of a tile to
-  float* partial;          // arrive sums all partials in split order and runs the epilogue
-  int64_t part_stride;     // elements between two splits' partials (x_rows * M)
-  int* tile_cnt;           // per-tile arrival counters (zero before the launch; reset by the last split)
+  int ksplit;              // > 1: the K slices of one tile run as one thread-block cluster (rank = slice); the
+                           // slices' accumulators are summed through distributed shared memory in rank order
   int64_t w_group_stride;
   int n_dev, has_extra, extra_off, extra_cnt, host_cnt;
   const int32_t* grp_off;
@@ -101,6 +98,29 @@ __device__ __forceinline__ void decode_tile(const Smem& sm, int m_tiles, int t, 
 
 __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }
 
+// Barrier over every thread of every CTA of the cluster (release / acquire on shared memory).
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// fp32 load from the same shared-memory offset in the CTA of the cluster with the given rank.
+__device__ __forceinline__ float ld_dsmem(const float* local, uint32_t rank) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(tc::smem_u32(local)), "r"(rank));
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+  return v;
+}
+
+// cos and sin of pos * inv_freq: the angle is formed and reduced to [-pi, pi] in fp64, then evaluated in fp32
+// (absolute error ~1e-7 for any position).
+__device__ __forceinline__ void rope_cos_sin(int pos, double inv_freq, float* c, float* s) {
+  const double two_pi = 6.283185307179586476925286766559;
+  const double inv_two_pi = 0.15915494309189533576888376337251;
+  double a = (double)pos * inv_freq;
+  a -= two_pi * rint(a * inv_two_pi);
+  sincosf((float)a, s, c);
+}
+
 template <int BN>
 __device__ void epilogue_chunk(const KParams& p, const float* stage, int g, int mt, int n0, int nval, int c0,
                                int row0, int tid) {
@@ -126,10 +146,8 @@ __device__ void epilogue_chunk(const KParams& p, const float* stage, int g, int 
       float x1 = stage[j * 128 + m], x2 = stage[j * 128 + 64 + m];
       float y1 = x1, y2 = x2;
       if (rot) {
-        int pos = e.pos0 + tr % e.L;
-        double sn, cs;
-        sincos((double)pos * inv_freq, &sn, &cs);
-        float c = (float)cs, s = (float)sn;
+        float c, s;
+        rope_cos_sin(e.pos0 + tr % e.L, inv_freq, &c, &s);
         y1 = x1 * c - x2 * s;
         y2 = x2 * c + x1 * s;
       }
@@ -155,18 +173,28 @@ __device__ void epilogue_chunk(const KParams& p, const float* stage, int g, int 
       }
     }
   } else {
-    const int64_t mbase = (int64_t)mt * 128;
-    for (int idx = tid; idx < ncols * 128; idx += 128) {
-      int j = idx >> 7, m = idx & 127;
-      float v = stage[j * 128 + m];
-      int64_t off = (int64_t)(row0 + n0 + c0 + j) * e.ldo + mbase + m;
-      if (e.out_f32) {
-        float* o = static_cast<float*>(e.out);
-        o[off] = (e.kind == EPI_RESID) ? o[off] + v : v;
-      } else {
-        __nv_bfloat16* o = static_cast<__nv_bfloat16*>(e.out);
-        float r = (e.kind == EPI_RESID) ? __bfloat162float(o[off]) + v : v;
-        o[off] = __float2bfloat16_rn(r);
+    // thread = output feature m; 8 token rows per round so the residual loads of a round are in flight together
+    const int m = tid;
+    const int64_t col = (int64_t)mt * 128 + m;
+    const int64_t base = (int64_t)(row0 + n0 + c0) * e.ldo + col;
+    for (int j0 = 0; j0 < ncols; j0 += 8) {
+      float res[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        res[u] = 0.f;
+        if (e.kind == EPI_RESID && j0 + u < ncols) {
+          const int64_t off = base + (int64_t)(j0 + u) * e.ldo;
+          res[u] = e.out_f32 ? static_cast<const float*>(e.out)[off]
+                             : __bfloat162float(static_cast<const __nv_bfloat16*>(e.out)[off]);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (j0 + u >= ncols) break;
+        const int64_t off = base + (int64_t)(j0 + u) * e.ldo;
+        const float v = stage[(j0 + u) * 128 + m] + res[u];
+        if (e.out_f32) static_cast<float*>(e.out)[off] = v;
+        else static_cast<__nv_bfloat16*>(e.out)[off] = __float2bfloat16_rn(v);
       }
     }
   }
@@ -219,33 +247,41 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
   }
   if (warp == 1) tc::tmem_alloc(&sm.tmem_base, 2 * BN);
   __syncthreads();
-  // prefix of tiles per group: contiguous chunks per thread, then a scan of the chunk sums
+  // prefix of tiles per group: contiguous chunks per thread, a shuffle scan of the thread sums inside each warp,
+  // then the six warp totals
   {
-    int* chunk_sum = sm.chunk_sum;
+    int* warp_tot = sm.chunk_sum;
     const int per = (n_groups + NUM_THREADS - 1) / NUM_THREADS;
     const int g0 = tid * per, g1 = min(n_groups, g0 + per);
     int s = 0;
     for (int g = g0; g < g1; ++g) s += ((sm.grp_cnt[g] + BN - 1) / BN) * p.m_tiles;
-    chunk_sum[tid] = s;
-    __syncthreads();
-    if (tid == 0) {
-      int run = 0;
-      for (int i = 0; i < NUM_THREADS; ++i) {
-        int v = chunk_sum[i];
-        chunk_sum[i] = run;
-        run += v;
-      }
-      sm.total_tiles = run;
+    int inc = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
     }
+    if (lane == 31) warp_tot[warp] = inc;
     __syncthreads();
-    int run = chunk_sum[tid];
+    int before = 0, all = 0;
+#pragma unroll
+    for (int w2 = 0; w2 < NUM_THREADS / 32; ++w2) {
+      const int v = warp_tot[w2];
+      if (w2 < warp) before += v;
+      all += v;
+    }
+    int run = before + inc - s;
     for (int g = g0; g < g1; ++g) {
       sm.tile_prefix[g] = run;
       run += ((sm.grp_cnt[g] + BN - 1) / BN) * p.m_tiles;
     }
+    if (tid == 0) sm.total_tiles = all;
     __syncthreads();
   }
   const int total = sm.total_tiles * p.ksplit;
+  // persistent CTAs stride over the work list; in cluster split-K mode CTA (rank, tile) owns exactly one item
+  const int wk_begin = p.ksplit > 1 ? (int)(blockIdx.y * p.ksplit + blockIdx.x) : (int)blockIdx.x;
+  const int wk_step = p.ksplit > 1 ? total : (int)gridDim.x;
   volatile int* abort_flag = &sm.abort_flag;
   const int kblocks = p.K / BK;
 
@@ -259,7 +295,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
       const uint64_t pol_x = tc::policy_evict_last();
       uint32_t it = 0;
       bool ok = true;
-      for (int wk = blockIdx.x; wk < total && ok; wk += gridDim.x) {
+      for (int wk = wk_begin; wk < total && ok; wk += wk_step) {
         const int t = wk / p.ksplit, ks = wk - t * p.ksplit;
         const int kb0 = ks * kblocks / p.ksplit, kb1 = (ks + 1) * kblocks / p.ksplit;
         int g, mt, n0, nval;
@@ -298,7 +334,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
     if (tc::elect_one()) {
       uint32_t it = 0, tcount = 0;
       bool ok = true;
-      for (int wk = blockIdx.x; wk < total && ok; wk += gridDim.x, ++tcount) {
+      for (int wk = wk_begin; wk < total && ok; wk += wk_step, ++tcount) {
         const int t = wk / p.ksplit, ks = wk - t * p.ksplit;
         const int kb0 = ks * kblocks / p.ksplit, kb1 = (ks + 1) * kblocks / p.ksplit;
         int g, mt, n0, nval;
@@ -334,7 +370,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
     const int row = q * 32 + lane;   // tile row m (TMEM lane)
     const int etid = tid - 64;       // 0..127
     uint32_t tcount = 0;
-    for (int wk = blockIdx.x; wk < total; wk += gridDim.x, ++tcount) {
+    for (int wk = wk_begin; wk < total; wk += wk_step, ++tcount) {
       const int t = wk / p.ksplit, ks = wk - t * p.ksplit;
       int g, mt, n0, nval;
       decode_tile<BN>(sm, p.m_tiles, t, g, mt, n0, nval);
@@ -356,42 +392,42 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
         tc::fence_before_sync();
         tc::mbar_arrive(&sm.tempty[buf]);
       } else {
-        // split-K: this split's raw partial straight from TMEM (thread = row m, columns = token rows)
-        float* dst = p.partial + ks * p.part_stride;
-        const int64_t col0 = (int64_t)mt * 128 + row;
-        for (int c0 = 0; c0 < nval; c0 += STAGE_COLS) {
-          float v[STAGE_COLS];
-          const uint32_t taddr = sm.tmem_base + ((uint32_t)(q * 32) << 16) + buf * BN + c0;
-          tc::tmem_ld16(taddr, v);
-          tc::tmem_ld16(taddr + 16, v + 16);
-          const int ncols = min(STAGE_COLS, nval - c0);
-          for (int j = 0; j < ncols; ++j)
-            dst[(int64_t)(sm.grp_off[g] + n0 + c0 + j) * p.M + col0] = v[j];
-        }
+        // cluster split-K (BN == 32, one chunk): this slice's accumulator into this CTA's staging tile
+        float v[STAGE_COLS];
+        const uint32_t taddr = sm.tmem_base + ((uint32_t)(q * 32) << 16) + buf * BN;
+        tc::tmem_ld16(taddr, v);
+        tc::tmem_ld16(taddr + 16, v + 16);
+#pragma unroll
+        for (int j = 0; j < STAGE_COLS; ++j) staging[j * 128 + row] = v[j];
         tc::fence_before_sync();
         tc::mbar_arrive(&sm.tempty[buf]);
-        __threadfence();
-        tc::named_bar_sync(1, 128);
-        if (etid == 0) sm.is_last = (atomicAdd(&p.tile_cnt[t], 1) == p.ksplit - 1);
-        tc::named_bar_sync(1, 128);
-        if (sm.is_last) {
-          __threadfence();
-          for (int c0 = 0; c0 < nval; c0 += STAGE_COLS) {
-            const int ncols = min(STAGE_COLS, nval - c0);
-            tc::named_bar_sync(1, 128);
-            for (int j = 0; j < ncols; ++j) {
-              const int64_t off = (int64_t)(sm.grp_off[g] + n0 + c0 + j) * p.M + col0;
-              float acc = 0.f;
-              for (int sp = 0; sp < p.ksplit; ++sp) acc += __ldcg(p.partial + sp * p.part_stride + off);
-              staging[j * 128 + row] = acc;
-            }
-            tc::named_bar_sync(1, 128);
-            epilogue_chunk<BN>(p, staging, g, mt, n0, nval, c0, sm.grp_off[g], etid);
-          }
-          if (etid == 0) p.tile_cnt[t] = 0;
-        }
       }
     }
+  }
+  if (p.ksplit > 1) {
+    // every slice's staging tile is complete; rank r sums columns [r*nval/ks, (r+1)*nval/ks) over the slices in
+    // rank order (distributed shared memory) and runs the epilogue on them; a second cluster barrier keeps each
+    // CTA's shared memory alive until its peers have read it
+    __syncthreads();
+    cluster_sync();
+    if (warp >= 2 && !*abort_flag) {
+      const int t = (int)blockIdx.y;
+      const int rank = (int)blockIdx.x;
+      int g, mt, n0, nval;
+      decode_tile<BN>(sm, p.m_tiles, t, g, mt, n0, nval);
+      const int row = (warp & 3) * 32 + lane;
+      const int etid = tid - 64;
+      const int cb = rank * nval / p.ksplit, ce = (rank + 1) * nval / p.ksplit;
+      float* red = reinterpret_cast<float*>(stages);   // the operand ring is idle now
+      for (int j = cb; j < ce; ++j) {
+        float acc = 0.f;
+        for (int sp = 0; sp < p.ksplit; ++sp) acc += ld_dsmem(staging + j * 128 + row, (uint32_t)sp);
+        red[(j - cb) * 128 + row] = acc;
+      }
+      tc::named_bar_sync(1, 128);
+      if (ce > cb) epilogue_chunk<BN>(p, red, g, mt, n0 + cb, ce - cb, 0, sm.grp_off[g], etid);
+    }
+    cluster_sync();
   }
   __syncthreads();
   if (warp == 1) {
@@ -439,6 +475,10 @@ int make_map(CUtensorMap* m, const void* ptr, int64_t rows, int K, int box_rows)
   return DLLM_OK;
 }
 
+// Cluster split-K launch: grid (ksplit, tiles), cluster (ksplit, 1, 1), one work item per CTA.
+int launch_cluster_splitk(const GemmArgs& a, const CUtensorMap& mw, const CUtensorMap& mw2, const CUtensorMap& mx,
+                          const KParams& kp, cudaStream_t s);
+
 template <int BN, int STAGES>
 int launch(const GemmArgs& a, const CUtensorMap& mw, const CUtensorMap& mw2, const CUtensorMap& mx,
            const KParams& kp, cudaStream_t s) {
@@ -454,6 +494,36 @@ int launch(const GemmArgs& a, const CUtensorMap& mw, const CUtensorMap& mw2, con
   }
   gemm_tc_kernel<BN, STAGES><<<num_sms(), NUM_THREADS, SMEM, s>>>(mw, mw2, mx, kp);
   DLLM_CHECK_LAUNCH("gemm_tc_kernel");
+  return DLLM_OK;
+}
+
+int launch_cluster_splitk(const GemmArgs& a, const CUtensorMap& mw, const CUtensorMap& mw2, const CUtensorMap& mx,
+                          const KParams& kp, cudaStream_t s) {
+  constexpr int BN = 32, STAGES = 9;
+  constexpr int STAGE_BYTES = A_BYTES + BN * BK * 2;
+  constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + STAGING_BYTES + (int)sizeof(Smem);
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         SMEM);
+    if (e != cudaSuccess) return dllm_host::cuda_status(e, "cudaFuncSetAttribute(gemm_tc cluster)");
+    configured = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(kp.ksplit, a.M / 128, 1);
+  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kp.ksplit;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, STAGES>, mw, mw2, mx, kp);
+  if (e != cudaSuccess) return dllm_host::cuda_status(e, "cudaLaunchKernelEx(gemm_tc cluster split-K)");
+  DLLM_CHECK_LAUNCH("gemm_tc_kernel (cluster split-K)");
   return DLLM_OK;
 }
 
@@ -492,24 +562,12 @@ int gemm_bf16_tc(const GemmArgs& a, cudaStream_t s) {
   kp.cnt_dev = a.cnt_dev;
   kp.epi = a.epi;
   kp.status = a.status;
-  kp.ksplit = 1;
-  kp.partial = nullptr;
-  kp.part_stride = 0;
-  const int bn = bn_for(a.max_cnt);
+  const int bn = gemm_bn(a);
   const int ks = gemm_splitk_factor(a, bn);
-  kp.tile_cnt = nullptr;
-  if (ks > 1) {
-    DLLM_REQUIRE(a.splitk_scratch != nullptr, DLLM_ERR_WORKSPACE, "gemm: split-K needs scratch");
-    kp.ksplit = ks;
-    kp.partial = a.splitk_scratch;
-    kp.part_stride = a.x_rows * (int64_t)a.M;
-    kp.tile_cnt = reinterpret_cast<int*>(a.splitk_scratch + (size_t)ks * a.x_rows * a.M);
-    const int tiles = (a.M / 128) * ((a.max_cnt + bn - 1) / bn);
-    cudaError_t e = cudaMemsetAsync(kp.tile_cnt, 0, (size_t)tiles * sizeof(int), s);
-    if (e != cudaSuccess) return dllm_host::cuda_status(e, "gemm: cudaMemsetAsync(split-K counters)");
-  }
+  kp.ksplit = ks;
   int st2;
-  if (bn == 32) st2 = launch<32, 9>(a, mw, mw2, mx, kp, s);
+  if (ks > 1) st2 = launch_cluster_splitk(a, mw, mw2, mx, kp, s);
+  else if (bn == 32) st2 = launch<32, 9>(a, mw, mw2, mx, kp, s);
   else if (bn == 64) st2 = launch<64, 8>(a, mw, mw2, mx, kp, s);
   else if (bn == 128) st2 = launch<128, 6>(a, mw, mw2, mx, kp, s);
   else st2 = launch<256, 4>(a, mw, mw2, mx, kp, s);
@@ -523,21 +581,25 @@ int bn_for(int max_cnt) {
   return 256;
 }
 
-// Split-K for dense projections whose output tiles would leave most SMs idle (a single group of rows known on
-// the host, no SwiGLU pairing): enough K slices to give every SM a tile, at least two 64-wide K blocks each.
-int gemm_splitk_factor(const GemmArgs& a, int bn) {
-  if (a.dtype != DLLM_BF16 || a.swiglu || a.n_dev || a.has_extra) return 1;
-  const int tiles = (a.M / 128) * ((a.max_cnt + bn - 1) / bn);
-  const int kblocks = a.K / BK;
-  if (tiles <= 0 || tiles * 2 > num_sms() || kblocks < 4) return 1;
-  return std::max(1, std::min(kblocks / 2, num_sms() / tiles));
+static bool dense(const GemmArgs& a) { return !a.swiglu && !a.n_dev && !a.has_extra; }
+
+// N tile: the smallest that covers the largest group, except that a dense projection with too few output tiles to
+// occupy the SMs takes narrower N tiles first (the extra re-reads of its weight tiles hit L2).
+int gemm_bn(const GemmArgs& a) {
+  int bn = bn_for(a.max_cnt);
+  if (dense(a))
+    while (bn > 32 && (a.M / 128) * ((a.max_cnt + bn - 1) / bn) < 2 * num_sms()) bn /= 2;
+  return bn;
 }
 
-size_t gemm_splitk_scratch_bytes(const GemmArgs& a) {
-  const int bn = bn_for(a.max_cnt);
-  const int ks = gemm_splitk_factor(a, bn);
-  const int tiles = (a.M / 128) * ((a.max_cnt + bn - 1) / bn);
-  return ks > 1 ? (size_t)ks * a.x_rows * a.M * sizeof(float) + (size_t)tiles * sizeof(int) : 0;
+// Split-K for dense projections that still leave most SMs idle at N tile 32 (all rows in one tile): K slices of
+// at least two 64-wide blocks, at most 8 (the portable cluster size) and no more than fill the SMs.
+int gemm_splitk_factor(const GemmArgs& a, int bn) {
+  if (a.dtype != DLLM_BF16 || !dense(a) || bn != 32 || a.max_cnt > 32) return 1;
+  const int tiles = a.M / 128;
+  const int kblocks = a.K / BK;
+  if (tiles <= 0 || tiles * 2 > num_sms() || kblocks < 4) return 1;
+  return std::max(1, std::min(std::min(kblocks / 2, 8), num_sms() / tiles));
 }
 
 int num_sms() {

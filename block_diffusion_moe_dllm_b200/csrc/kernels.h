@@ -57,13 +57,12 @@ struct GemmArgs {
   EpiParams epi;
   int32_t* status = nullptr;
   float* f32_scratch = nullptr;  // f32 path: [x_rows, M (x2 for swiglu)] raw products
-  float* splitk_scratch = nullptr;  // bf16 split-K: [ksplit, x_rows, M] raw partial products
 };
 
 int gemm_bf16_tc(const GemmArgs& a, cudaStream_t s);
 int bn_for(int max_cnt);
+int gemm_bn(const GemmArgs& a);
 int gemm_splitk_factor(const GemmArgs& a, int bn);
-size_t gemm_splitk_scratch_bytes(const GemmArgs& a);
 
 int gemm_f32_simt(const GemmArgs& a, cudaStream_t s);
 size_t gemm_f32_scratch_bytes(int64_t x_rows, int M, int swiglu);

@@ -41,8 +41,11 @@ __global__ void retain_select_kernel(const float* __restrict__ raw, int P, int n
   __shared__ int red[32];
   __shared__ double dred[32];
   __shared__ int base;
+  __shared__ float rs[8192];     // this row's scores (P <= 8192): the 33 counting passes read shared memory
   const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, w = tid >> 5, nw = blockDim.x >> 5;
-  const float* r = raw + (int64_t)b * P;
+  for (int i = tid; i < P; i += blockDim.x) rs[i] = raw[(int64_t)b * P + i];
+  __syncthreads();
+  const float* r = rs;
 
   auto block_count = [&](uint32_t thr, bool strictly) -> int {
     int c = 0;

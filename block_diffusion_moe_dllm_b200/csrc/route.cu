@@ -4,6 +4,7 @@
 // "Load Balancing — Auxiliary-loss-free MoE Bias" (a per-expert bias that steers which experts are picked).
 #include "common.cuh"
 #include "misc.h"
+#include "kernels.h"
 
 namespace dllm {
 namespace {
@@ -30,11 +31,21 @@ __global__ void __launch_bounds__(256) route_scores_kernel(const T* __restrict__
   const int nt = min(TT, Tk - t0);
   const int vec = 16 / (int)sizeof(T);
   const int nvec = TT * H / vec;
-  for (int i = threadIdx.x; i < nvec; i += blockDim.x) {
-    const int tt = (i * vec) / H;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (tt < nt) v = reinterpret_cast<const uint4*>(h + (int64_t)t0 * H)[i];
-    reinterpret_cast<uint4*>(hs)[i] = v;
+  const int valid_vec = nt * H / vec;            // vectors of the valid token rows (rows are contiguous)
+  const uint4* src = reinterpret_cast<const uint4*>(h + (int64_t)t0 * H);
+  // 8 independent loads in flight per thread
+  for (int i0 = threadIdx.x; i0 < nvec; i0 += 8 * blockDim.x) {
+    uint4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * blockDim.x;
+      v[u] = (i < valid_vec) ? src[i] : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int i = i0 + u * blockDim.x;
+      if (i < nvec) reinterpret_cast<uint4*>(hs)[i] = v[u];
+    }
   }
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -64,47 +75,66 @@ __global__ void __launch_bounds__(256) route_scores_kernel(const T* __restrict__
 }
 
 // One warp per token: k rounds of warp arg-max over s + bias (ties -> lower expert id); gates = s / sum(s).
-__global__ void route_topk_kernel(const float* __restrict__ scores, const float* __restrict__ bias, int Tk, int E,
-                                  int k, int32_t* __restrict__ ids, float* __restrict__ gates) {
+// Lane l holds experts l, l + 32, ... in registers (biased and unbiased); the winner's unbiased score comes from the
+// owning lane by a shuffle, so the rounds touch no memory.
+// With from_logits the row holds router logits: the sigmoid scores replace them in place.
+__global__ void route_topk_kernel(float* __restrict__ scores, const float* __restrict__ bias, int Tk, int E, int k,
+                                  int from_logits, int32_t* __restrict__ ids, float* __restrict__ gates) {
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (warp >= Tk) return;
-  const float* s = scores + (int64_t)warp * E;
-  float val[32];
+  float* s = scores + (int64_t)warp * E;
+  float val[32], raw[32];
   const int per = (E + 31) / 32;
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
-    int e = i * 32 + lane;
-    val[i] = (i < per && e < E) ? s[e] + bias[e] : -INFINITY;
+    const int e = i * 32 + lane;
+    const bool in = i < per && e < E;
+    float v = in ? s[e] : 0.f;
+    if (from_logits && in) {
+      v = 1.0f / (1.0f + expf(-v));
+      s[e] = v;
+    }
+    raw[i] = v;
+    val[i] = in ? v + bias[e] : -INFINITY;
   }
-  float gsum = 0.f;
-  float sel_s[32];
-  int sel_e[32];
-  for (int j = 0; j < k; ++j) {
-    float bv = -INFINITY;
-    int be = 0x7fffffff;
+  float gsum = 0.f, my_gate = 0.f;
+  int my_id = 0;
+  // each lane's best (value, expert); only the winning lane rescans its own values after a round
+  auto lane_best = [&](float& bv, int& be) {
+    bv = -INFINITY;
+    be = 0x7fffffff;
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
-      int e = i * 32 + lane;
-      if (val[i] > bv || (val[i] == bv && e < be)) { bv = val[i]; be = e; }
+      const int e = i * 32 + lane;
+      if (i < per && (val[i] > bv || (val[i] == bv && e < be))) { bv = val[i]; be = e; }
     }
+  };
+  float lbv;
+  int lbe;
+  lane_best(lbv, lbe);
+  for (int j = 0; j < k; ++j) {
+    float bv = lbv;
+    int be = lbe;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
-      float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      int oe = __shfl_xor_sync(0xffffffffu, be, o);
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
       if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
     }
+    float mine = 0.f;
+    if ((be & 31) == lane) {
 #pragma unroll
-    for (int i = 0; i < 32; ++i)
-      if (i * 32 + lane == be) val[i] = -INFINITY;
-    sel_e[j] = be;
-    sel_s[j] = s[be];
-    gsum += sel_s[j];
-  }
-  if (lane == 0) {
-    for (int j = 0; j < k; ++j) {
-      ids[(int64_t)warp * k + j] = sel_e[j];
-      gates[(int64_t)warp * k + j] = sel_s[j] / gsum;
+      for (int i = 0; i < 32; ++i)
+        if (i * 32 + lane == be) { mine = raw[i]; val[i] = -INFINITY; }
+      lane_best(lbv, lbe);
     }
+    const float sc = __shfl_sync(0xffffffffu, mine, be & 31);
+    gsum += sc;
+    if (lane == j) { my_id = be; my_gate = sc; }
+  }
+  if (lane < k) {
+    ids[(int64_t)warp * k + lane] = my_id;
+    gates[(int64_t)warp * k + lane] = my_gate / gsum;
   }
 }
 
@@ -197,6 +227,22 @@ int launch_route(int dtype, const void* h, const void* w_router, const float* bi
                  int32_t* ids, float* gates, float* scores, int32_t* counts, int32_t* offsets, int32_t* perm,
                  int32_t* inv, cudaStream_t s) {
   if (Tk <= 0) return DLLM_OK;
+  // bf16 with a tensor-core friendly shape: router logits through the tcgen05 projection (fp32 out, accumulated
+  // in fp32 in the MMA's fixed order); otherwise the SIMT score kernel
+  const bool tc_logits = dtype == DLLM_BF16 && E % 128 == 0 && H % 64 == 0;
+  if (tc_logits) {
+    GemmArgs g;
+    g.x = h; g.x_rows = Tk; g.w = w_router; g.w_rows = E; g.K = H; g.M = E; g.host_cnt = Tk; g.max_cnt = Tk;
+    g.cnt_bound = Tk; g.dtype = DLLM_BF16;
+    g.epi.kind = EPI_STORE; g.epi.out = scores; g.epi.ldo = E; g.epi.out_f32 = 1;
+    int st = gemm_bf16_tc(g, s);
+    if (st) return st;
+    route_topk_kernel<<<(Tk + 7) / 8, 256, 0, s>>>(scores, bias, Tk, E, k, 1, ids, gates);
+    DLLM_CHECK_LAUNCH("route_topk_kernel");
+    route_permute_kernel<<<E, 256, 0, s>>>(ids, Tk * k, E, counts, offsets, perm, inv);
+    DLLM_CHECK_LAUNCH("route_permute_kernel");
+    return DLLM_OK;
+  }
   dim3 g1((E + EW - 1) / EW, (Tk + TT - 1) / TT);
   const size_t smem = (size_t)TT * H * (dtype == DLLM_BF16 ? 2 : 4);
   if (dtype == DLLM_BF16) {
@@ -217,7 +263,7 @@ int launch_route(int dtype, const void* h, const void* w_router, const float* bi
     route_scores_kernel<float><<<g1, 256, smem, s>>>((const float*)h, (const float*)w_router, Tk, H, E, scores);
   }
   DLLM_CHECK_LAUNCH("route_scores_kernel");
-  route_topk_kernel<<<(Tk + 7) / 8, 256, 0, s>>>(scores, bias, Tk, E, k, ids, gates);
+  route_topk_kernel<<<(Tk + 7) / 8, 256, 0, s>>>(scores, bias, Tk, E, k, 0, ids, gates);
   DLLM_CHECK_LAUNCH("route_topk_kernel");
   route_permute_kernel<<<E, 256, 0, s>>>(ids, Tk * k, E, counts, offsets, perm, inv);
   DLLM_CHECK_LAUNCH("route_permute_kernel");

@@ -25,12 +25,12 @@ DLLM_DEV void merge(Partial& a, const Partial& b) {
   if (b.s == 0.0) return;
   if (a.s == 0.0) { a = b; return; }
   if (b.m > a.m || (b.m == a.m && b.idx < a.idx)) {
-    double f = (b.m == a.m) ? 1.0 : exp((double)a.m - (double)b.m);
+    const double f = (b.m == a.m) ? 1.0 : (double)expf(a.m - b.m);
     a.s = a.s * f + b.s;
     a.m = b.m;
     a.idx = b.idx;
   } else {
-    double f = (b.m == a.m) ? 1.0 : exp((double)b.m - (double)a.m);
+    const double f = (b.m == a.m) ? 1.0 : (double)expf(b.m - a.m);
     a.s = a.s + b.s * f;
   }
 }
@@ -135,33 +135,56 @@ __global__ void __launch_bounds__(256) unmask_reduce_kernel(const T* __restrict_
   }
 }
 
-// One warp per logical block row b (L <= 32 positions, lane i = position i).
+// One warp per logical block row b (L <= 32 positions, lane i = position i). The still-masked flat positions are
+// the LM head's rows in increasing order, so the row of position (b, i) is the number of masked positions before it.
 __global__ void unmask_select_kernel(const Partial* __restrict__ part, int n_chunks, const int32_t* __restrict__ row_pos,
                                      const int32_t* __restrict__ n_rows, int B, int L, int t, int T_s, int mode,
                                      float tau, int k_max, int cfg, int vocab_offset, int32_t* tokens, uint8_t* mask,
                                      int32_t* sel, int32_t* nsel, float* conf, int32_t* remaining) {
   __shared__ int rem_w[32];
+  __shared__ int row_cnt[1024];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  const int n = *n_rows;
+  // masked count of every logical row, then the exclusive prefix (rows in order)
+  for (int b = w; b < B; b += nw) {
+    const bool mk = lane < L && mask[b * L + lane] != 0;
+    const int c = __popc(__ballot_sync(0xffffffffu, mk));
+    if (lane == 0) row_cnt[b] = c;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int run = 0;
+    for (int b = 0; b < B; ++b) {
+      const int c = row_cnt[b];
+      row_cnt[b] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
   int rem_acc = 0;
   for (int b = w; b < B; b += nw) {
     const int p = b * L + lane;
     const bool valid = lane < L;
     const bool masked = valid && mask[p] != 0;
+    const unsigned mball = __ballot_sync(0xffffffffu, masked);
     double c = 0.0;
     int cand = -1;
     if (masked) {
-      int lo = 0, hi = n - 1;  // row_pos is ascending: find r with row_pos[r] == p
-      while (lo < hi) {
-        int mid = (lo + hi) >> 1;
-        if (row_pos[mid] < p) lo = mid + 1; else hi = mid;
+      const int r = row_cnt[b] + __popc(mball & ((1u << lane) - 1u));
+      const Partial* pr = part + (int64_t)r * n_chunks;
+      Partial a = pr[0];
+      // batches of 8 independent loads, merged in chunk order
+      for (int q0 = 1; q0 < n_chunks; q0 += 8) {
+        Partial b8[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          if (q0 + u < n_chunks) b8[u] = pr[q0 + u];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          if (q0 + u < n_chunks) merge(a, b8[u]);
       }
-      Partial a{-INFINITY, 0x7fffffff, 0.0};
-      for (int q = 0; q < n_chunks; ++q) merge(a, part[(int64_t)lo * n_chunks + q]);
       c = 1.0 / a.s;
       cand = a.idx + vocab_offset;
     }
-    const unsigned mball = __ballot_sync(0xffffffffu, masked);
     const int m = __popc(mball);
     int kt = 0;
     if (m > 0) {
@@ -202,9 +225,9 @@ __global__ void unmask_select_kernel(const Partial* __restrict__ part, int n_chu
   if (lane == 0) rem_w[w] = rem_acc;
   __syncthreads();
   if (threadIdx.x == 0) {
-    int s = 0;
-    for (int i = 0; i < nw; ++i) s += rem_w[i];
-    *remaining = s;
+    int s2 = 0;
+    for (int i = 0; i < nw; ++i) s2 += rem_w[i];
+    *remaining = s2;
   }
 }
 

@@ -6,7 +6,7 @@
 // but cannot provide the workspace dllm_unmask needs for its per-chunk partial results. This entry point keeps
 // that scratch in a fixed array inside the library instead.
 //
-// The scratch is a file-scope __device__ array of kNoAllocScratchBytes (1 MiB). Every GPU that loads the library
+// The scratch is a file-scope __device__ array of kNoAllocScratchBytes (256 KiB: 16384 partial entries). Every GPU that loads the library
 // holds it until the process exits. Host code must never pass the array's name to a kernel: on the host that
 // name is a stand-in, not a device address. Its device address is taken once per device, with that device
 // current, through cudaGetSymbolAddress (the first call on each device does this set-up; make that first call
@@ -19,7 +19,7 @@
 
 namespace {
 
-constexpr size_t kNoAllocScratchBytes = size_t(1) << 20;
+constexpr size_t kNoAllocScratchBytes = size_t(256) << 10;
 constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_unmask_scratch[kNoAllocScratchBytes];
@@ -52,8 +52,9 @@ extern "C" int dllm_unmask_noalloc(const dllm_unmask_desc* d, const void* logits
   using namespace dllm;
   DLLM_REQUIRE(d && logits && row_pos && n_rows_dev && tokens && mask && sel && nsel && conf && remaining,
                DLLM_ERR_INVALID_ARG, "unmask_noalloc: NULL argument");
-  DLLM_REQUIRE(d->B >= 1 && d->L >= 1 && d->L <= 32 && d->V >= 1 && d->max_rows >= 0 && d->max_rows <= d->B * d->L,
-               DLLM_ERR_SHAPE, "unmask_noalloc: bad shape (L <= 32, max_rows <= B*L)");
+  DLLM_REQUIRE(d->B >= 1 && d->B <= 1024 && d->L >= 1 && d->L <= 32 && d->V >= 1 && d->max_rows >= 0 &&
+                   d->max_rows <= d->B * d->L,
+               DLLM_ERR_SHAPE, "unmask_noalloc: bad shape (B <= 1024, L <= 32, max_rows <= B*L)");
   DLLM_REQUIRE(d->T_s >= 1 && d->t >= 0 && d->t < d->T_s, DLLM_ERR_INVALID_ARG, "unmask_noalloc: step %d of %d", d->t,
                d->T_s);
   DLLM_REQUIRE(d->mode == DLLM_UNMASK_FIXED || d->mode == DLLM_UNMASK_THRESHOLD, DLLM_ERR_INVALID_ARG,

@@ -1,6 +1,6 @@
 """Per-kernel timing of the library's main calls at a workload's shapes (CUDA events, kernels launched alone).
 
-    python -m block_diffusion_moe_dllm_b200.kernel_bench [--kernel lm_head|experts|unmask|attn|route|all]
+    python -m block_diffusion_moe_dllm_b200.kernel_bench [--kernel lm_head|proj|experts|unmask|attn|route|all]
                                                          [--workload NAME] [--reps N]
 
 Each line reports the mean time of one call, its algorithmic bytes (weights and activations it must move at
@@ -67,6 +67,23 @@ def bench_lm_head(w: Workload, reps, dev, stream, weights=None):
     t = timed(lambda: bd.gemm(x, wl, y, rows, w.vlen, w.H, bd.BF16, ws=ws), reps, stream)
     nbytes = w.vlen * w.H * 2 + rows * w.H * 2 + rows * w.vlen * 2
     return _result("gemm_tc_kernel[lm_head]", t, nbytes, {"rows": rows, "M": w.vlen, "K": w.H})
+
+
+def bench_proj(w: Workload, reps, dev, stream, weights=None):
+    """The dense projections of one layer at the block's row count: QKV (M = (Hq + 2 Hkv) d) and output (M = H),
+    both written with a residual-free store (the step's epilogues move the same bytes)."""
+    rows = w.B * w.L
+    out = []
+    for name, M, K in (("qkv", (w.Hq + 2 * w.Hkv) * w.d, w.H), ("o_proj", w.H, w.Hq * w.d)):
+        wt = (weights["layers"][0]["w_qkv" if name == "qkv" else "w_o"] if weights else
+              synth.normal((M, K), w.w_std, w.seed, f"kb_{name}", dev))
+        x = synth.normal((rows, K), 1.0, 5, f"kb_{name}_x", dev)
+        y = torch.empty((rows, M), dtype=torch.bfloat16, device=dev)
+        ws = bd.Workspace(64 << 20, dev)
+        t = timed(lambda: bd.gemm(x, wt, y, rows, M, K, bd.BF16, ws=ws), reps, stream)
+        nbytes = M * K * 2 + rows * K * 2 + rows * M * 2
+        out.append(_result(f"gemm_tc_kernel[{name}]", t, nbytes, {"rows": rows, "M": M, "K": K}))
+    return out
 
 
 def bench_experts(w: Workload, reps, dev, stream, weights=None):
@@ -150,6 +167,8 @@ def main():
     out = []
     if a.kernel in ("lm_head", "all"):
         out.append(bench_lm_head(w, a.reps, dev, stream))
+    if a.kernel in ("proj", "all"):
+        out.extend(bench_proj(w, a.reps, dev, stream))
     if a.kernel in ("experts", "route", "all"):
         out.extend(bench_experts(w, a.reps, dev, stream))
     if a.kernel in ("unmask", "all"):

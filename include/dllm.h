@@ -184,11 +184,12 @@ DLLM_API size_t dllm_moe_experts_workspace_size(const dllm_expert_desc* desc);
  * zu = logits[n_rows + r]); candidate = vocab_offset + lowest argmax of z; c = 1 / sum_v exp(z_v - max z).
  * Per logical row b with m masked positions: k_t positions by c descending (ties -> lower position) get their
  * candidate written to tokens and their mask cleared; with cfg the uncond row b + B gets the same update.
- *   logits [n_rows * (1 + cfg), V] in the storage type; row_pos [>= n_rows] int32; n_rows_dev [1] int32
- *   (device count, <= max_rows); tokens [B * (1 + cfg), L] int32; mask [B * (1 + cfg), L] uint8;
+ *   logits [n_rows * (1 + cfg), V] in the storage type; row_pos [>= n_rows] int32: the still-masked flat
+ *   positions of the logical rows in increasing order (row r of the logits belongs to the r-th masked position);
+ *   n_rows_dev [1] int32 (device count of masked positions, <= max_rows); tokens [B * (1 + cfg), L] int32; mask [B * (1 + cfg), L] uint8;
  *   sel [B, L] int32 (chosen positions in rank order, -1 after nsel[b]); nsel [B]; conf [B, L] fp32 (0 at
  *   unmasked positions); remaining [1] int32: masked positions left over all logical rows.
- * Requires L <= 32 (one warp per block row for the selection).
+ * Requires L <= 32 (one warp per block row for the selection) and B <= 1024.
  */
 typedef struct {
   int32_t B, L, V;
@@ -212,9 +213,9 @@ DLLM_API size_t dllm_unmask_workspace_size(const dllm_unmask_desc* desc);
  * application that owns the device's memory pool and exposes no allocator; a serving loop that forbids cudaMalloc
  * after start-up because it can synchronise the device). The paper has no counterpart: this is a deployment
  * variant of the same computation. Same arguments and results as dllm_unmask minus ws / ws_bytes; the caller
- * still owns every input and output. The per-chunk scratch lives in a fixed 1 MiB array inside the library,
+ * still owns every input and output. The per-chunk scratch lives in a fixed 256 KiB array inside the library,
  * held on every GPU that loads it until the process exits; calls with max_rows x vocabulary chunks needing more
- * (more than 65536 partial entries) return DLLM_ERR_UNSUPPORTED. The first call on each device looks up the
+ * (more than 16384 partial entries of 16 bytes) return DLLM_ERR_UNSUPPORTED. The first call on each device looks up the
  * array's device address (make it before any stream capture). All calls share the array: calls that overlap on
  * the GPU race and must be ordered by the caller (one stream, or events).
  */

@@ -69,9 +69,9 @@ def test_unmask_noalloc_matches_workspace_version(B, L, V, t, T_s, mode, cfg):
 
 def test_unmask_noalloc_rejects_oversized_request():
     lib = bd.load()
-    # 131072 masked rows x 1 vocabulary chunk x 16 bytes = 2 MiB of partials, above the fixed 1 MiB: rejected
+    # 32768 masked rows x 1 vocabulary chunk x 16 bytes = 512 KiB of partials, above the fixed 256 KiB: rejected
     # on the host before any launch (the buffers below are never touched)
-    desc = bd.UnmaskDesc(4096, 32, 157184, 4096 * 32, 0, 8, bd.FIXED, 0.9, 8, 0, 1.0, 0, bd.BF16)
+    desc = bd.UnmaskDesc(1024, 32, 157184, 1024 * 32, 0, 8, bd.FIXED, 0.9, 8, 0, 1.0, 0, bd.BF16)
     z = torch.zeros(16, dtype=torch.int32, device=DEV)
     rc = lib.dllm_unmask_noalloc(C.byref(desc), bd.ptr(z), bd.ptr(z), bd.ptr(z), bd.ptr(z), bd.ptr(z), bd.ptr(z),
                                  bd.ptr(z), bd.ptr(z), bd.ptr(z), bd.stream_handle())

@@ -41,10 +41,8 @@ def parse():
 
 
 def dist_env():
-    ws = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    return ws, rank, local
+    from block_diffusion_moe_dllm_b200 import replicas
+    return replicas.env()
 
 
 # ---------------------------------------------------------------------------------------------- clocks
@@ -179,9 +177,11 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     bd.load()
 
-    wt = synth.make_weights(w, dev, seed=w.seed + rank)
-    caches = synth.make_prefix_cache(w, dev, seed=w.seed + rank)
-    tokens0, mask0 = synth.make_block_state(w, dev, seed=w.seed + rank)
+    from block_diffusion_moe_dllm_b200 import replicas
+    seed = replicas.replica_seed(w.seed, rank)
+    wt = synth.make_weights(w, dev, seed=seed)
+    caches = synth.make_prefix_cache(w, dev, seed=seed)
+    tokens0, mask0 = synth.make_block_state(w, dev, seed=seed)
     eng = DenoiseEngine(w, wt, caches, dev)
     stream = torch.cuda.current_stream()
 
@@ -210,15 +210,12 @@ def main():
     ev1.record(stream)
     torch.cuda.synchronize()
     launches = launches_per_step * args.steps
-    elapsed = ev0.elapsed_time(ev1) / 1000.0
+    elapsed = replicas.max_over_ranks(ev0.elapsed_time(ev1) / 1000.0, dev)
     if world > 1:
-        t = torch.tensor([elapsed], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed = float(t.item())
         dist.barrier()
     clk = clocks.stop()
     tokens_per_step = w.B * w.L * w.T_s
-    value = tokens_per_step * args.steps * world / elapsed
+    value = replicas.aggregate_throughput(tokens_per_step * args.steps, elapsed, world)
 
     # ---- end to end through the public API with host buffers: block state from pinned host memory in,
     # final tokens out, every step
@@ -237,12 +234,8 @@ def main():
         h_out.copy_(eng.tokens, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_t = e0.elapsed_time(e1) / 1000.0
-    if world > 1:
-        t = torch.tensor([e2e_t], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_t = float(t.item())
-    e2e = {"value": tokens_per_step * args.steps * world / e2e_t, "unit": "tokens/s",
+    e2e_t = replicas.max_over_ranks(e0.elapsed_time(e1) / 1000.0, dev)
+    e2e = {"value": replicas.aggregate_throughput(tokens_per_step * args.steps, e2e_t, world), "unit": "tokens/s",
            "h2d_bytes_per_step": h_tok.numel() * 4 + h_mask.numel(), "d2h_bytes_per_step": h_out.numel() * 4}
     del g_reset, g_plain
 

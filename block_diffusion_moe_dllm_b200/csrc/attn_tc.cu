@@ -22,13 +22,15 @@
 namespace dllm {
 namespace {
 
-constexpr int NT = 192;
+constexpr int NT = 320;                     // warp 0 TMA, warp 1 MMA, warps 2..9 softmax (two per query row)
 constexpr int KT = 128;                     // keys per tile
 constexpr int CHUNK = 128 * 64 * 2;         // one 64-wide K-major chunk of a 128-row tile: 16 KB
 constexpr int TILE = 2 * CHUNK;             // 128 rows x 128 elements: 32 KB
 constexpr int STAGES = 2;
 constexpr int BARS_BYTES = 2048;
-constexpr int SMEM = 1024 + TILE /*Q*/ + STAGES * 2 * TILE /*K,V*/ + TILE /*P*/ + BARS_BYTES;
+constexpr short kNoKey = 0x7fff;   // relative block of a key past n_keys (never visible)
+constexpr int SMEM = 1024 + TILE /*Q*/ + STAGES * 2 * TILE /*K,V*/ + 2 * TILE /*P, double buffered*/ + BARS_BYTES;
+static_assert(SMEM <= 232448, "shared memory budget");
 
 struct Bars {
   uint64_t q_full;
@@ -36,12 +38,14 @@ struct Bars {
   uint64_t kv_empty[STAGES];
   uint64_t s_full[2];
   uint64_t p_ready;
-  uint64_t o_full;
+  uint64_t o_full[2];
   uint64_t done;
   uint32_t tmem_base;
   int abort_flag;
-  int kblk[2][KT];      // block index of each key of the tile (INT_MAX past n_keys)
-  int all_vis[2];       // 1: every key of the tile is visible to every query of the CTA
+  short kblk[2][KT];    // block of each key of the tile relative to the CTA's first query block, clamped to
+                        // [-32768, 32766] (kNoKey past n_keys), per tile parity
+  unsigned vis_w[2][4]; // per tile, ballots of "key visible to every query of the CTA" (4 warps x 32 keys)
+  float rowmax[2][128]; // per column half, per row: the half-row maximum (the tile-start barrier separates uses)
 };
 static_assert(sizeof(Bars) <= BARS_BYTES, "barrier block exceeds its shared-memory reservation");
 
@@ -50,10 +54,7 @@ struct AttnTcParams {
   int n_splits, tiles_per_split;
   float scale_log2;
   const int32_t* key_pos;
-  __nv_bfloat16* out;   // [B, Lq, Hq, 128] when n_splits == 1
-  float* po;            // [splits, B, Lq, Hq, 128]
-  float* pm;            // [splits, B, Lq, Hq]
-  float* pl;
+  __nv_bfloat16* out;   // [B, Lq, Hq, 128]
   int32_t* status;
 };
 
@@ -99,6 +100,34 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t dsmem_addr(const void* local, uint32_t rank) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(tc::smem_u32(local)), "r"(rank));
+  return remote;
+}
+__device__ __forceinline__ float ld_dsmem(const float* local, uint32_t rank) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(dsmem_addr(local, rank)) : "memory");
+  return v;
+}
+__device__ __forceinline__ float4 ld_dsmem4(const float* local, uint32_t rank) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(dsmem_addr(local, rank))
+               : "memory");
+  return v;
+}
+
+// Each lane reads 64 consecutive 32-bit columns of its own TMEM lane.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float* v) {
+  tmem_ld32(taddr, v);
+  tmem_ld32(taddr + 32, v + 32);
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -111,16 +140,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   uint8_t* sQ = base;
   uint8_t* sK = sQ + TILE;                    // [STAGES][TILE]
   uint8_t* sV = sK + STAGES * TILE;           // [STAGES][TILE]
-  uint8_t* sP = sV + STAGES * TILE;
-  Bars& bar = *reinterpret_cast<Bars*>(sP + TILE);
+  uint8_t* sP = sV + STAGES * TILE;            // [2][TILE]
+  Bars& bar = *reinterpret_cast<Bars*>(sP + 2 * TILE);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  int bx = blockIdx.x;
+  int bx = blockIdx.y;
   const int qt = bx % p.n_qtiles;
   bx /= p.n_qtiles;
   const int g = bx % p.Hkv;
   const int b = bx / p.Hkv;
-  const int split = blockIdx.y;
+  const int split = blockIdx.x;      // = rank in the cluster of this tile's key splits
   const int q0 = qt * p.QT;
 
   // key tiles of this split; causal bound: a query tile never sees keys of blocks after its last query's block
@@ -144,8 +173,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
     tc::mbar_init(&bar.s_full[0], 1);
     tc::mbar_init(&bar.s_full[1], 1);
-    tc::mbar_init(&bar.p_ready, 128);
-    tc::mbar_init(&bar.o_full, 1);
+    tc::mbar_init(&bar.p_ready, 256);
+    tc::mbar_init(&bar.o_full[0], 1);
+    tc::mbar_init(&bar.o_full[1], 1);
     tc::mbar_init(&bar.done, 1);
     tc::fence_mbar_init();
   }
@@ -153,7 +183,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   __syncthreads();
   volatile int* abort_flag = &bar.abort_flag;
   const uint32_t tS = bar.tmem_base;          // S buffers at columns [0,128) and [128,256)
-  const uint32_t tO = bar.tmem_base + 256;    // O tile at columns [256, 384)
+  const uint32_t tO = bar.tmem_base + 256;    // O tiles at columns [256,384) and [384,512)
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
@@ -235,142 +265,142 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         tc::fence_after_sync();
         const int s = j % STAGES;
         const uint32_t aV = tc::smem_u32(sV + s * TILE);
+        const uint32_t aPj = aP + (j & 1) * TILE;
+        const uint32_t tOj = tO + (j & 1) * 128;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t offp = (kk >> 2) * CHUNK + (kk & 3) * 32;
-          tc::mma_bf16(tO, tc::sdesc_k128(aP + offp), sdesc_mn128(aV + kk * 2048, CHUNK), idesc_o, kk != 0);
+          tc::mma_bf16(tOj, tc::sdesc_k128(aPj + offp), sdesc_mn128(aV + kk * 2048, CHUNK), idesc_o, kk != 0);
         }
-        tc::mma_commit(&bar.o_full);
+        tc::mma_commit(&bar.o_full[j & 1]);
         tc::mma_commit(&bar.kv_empty[s]);
       }
       tc::mma_commit(&bar.done);
       tc::mbar_wait(&bar.done, 0, 1u << 20);
     }
   } else {
-    // ------------------------------------------------------------------ softmax / output warps 2..5
+    // ------------------------------------------------------------------ softmax / output warps 2..9
+    // Two threads per query row (TMEM lane): warp w in 2..5 takes keys / output columns [0, 64), warp w + 4 takes
+    // [64, 128). The half-row maxima are exchanged through shared memory once per tile.
     const int q4 = warp & 3;
     const int row = q4 * 32 + lane;      // TMEM lane = tile row
-    const int etid = tid - 64;           // 0..127
+    const int half = (warp - 2) >> 2;    // 0: columns [0, 64), 1: [64, 128)
+    const int etid = tid - 64;           // 0..255
     const int qi = row / p.G, hh = row % p.G;
     const int qg = q0 + qi;              // query index in the row
     const bool row_ok = qg < p.Lq;
-    const int qblk = (p.q_pos0 + qg) / p.blk_len;
     const int qblk_min = (p.q_pos0 + q0) / p.blk_len;  // rows of the tile past Lq never write output
+    const int qrel = (p.q_pos0 + qg) / p.blk_len - qblk_min;
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-    float o[128];
+    const int col0 = 64 * half;
+    float o[64];
 #pragma unroll
-    for (int c = 0; c < 128; ++c) o[c] = 0.f;
+    for (int c = 0; c < 64; ++c) o[c] = 0.f;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < ntile && ok; ++j) {
       const int jt = t_begin + j;
       // block index of every key of this tile, and whether the whole tile is visible to the whole query tile
-      {
-        const int c = etid;
-        const int key = jt * KT + c;
-        int kb = 0x7fffffff;
-        if (key < n_keys_eff) kb = (p.key_pos ? p.key_pos[(int64_t)b * p.n_keys + key] : key) / p.blk_len;
-        bar.kblk[j & 1][c] = kb;
-        const bool vis_all = kb <= qblk_min;
-        const unsigned bal = __ballot_sync(0xffffffffu, vis_all);
-        if (lane == 0) bar.all_vis[j & 1] = 1;
-        tc::named_bar_sync(1, 128);
-        if (lane == 0 && bal != 0xffffffffu) bar.all_vis[j & 1] = 0;
+      if (etid < 128) {
+        const int key = jt * KT + etid;
+        int rel = kNoKey;
+        if (key < n_keys_eff) {
+          const int kb = (p.key_pos ? p.key_pos[(int64_t)b * p.n_keys + key] : key) / p.blk_len;
+          rel = max(-32768, min(32766, kb - qblk_min));   // the queries' relative blocks lie in [0, 128]
+        }
+        bar.kblk[j & 1][etid] = (short)rel;
+        const unsigned bal = __ballot_sync(0xffffffffu, rel <= 0);
+        if (lane == 0) bar.vis_w[j & 1][etid >> 5] = bal;
       }
-      tc::named_bar_sync(1, 128);
-      const bool fast = bar.all_vis[j & 1] != 0;
+      tc::named_bar_sync(1, 256);
+      const bool fast = (bar.vis_w[j & 1][0] & bar.vis_w[j & 1][1] & bar.vis_w[j & 1][2] & bar.vis_w[j & 1][3]) ==
+                        0xffffffffu;
       if (!wait_bar(&bar.s_full[j & 1], (j >> 1) & 1, abort_flag, p.status, ST_TIMEOUT_EPILOGUE)) { ok = false; break; }
       tc::fence_after_sync();
-      const uint32_t sbase = tS + (j & 1) * 128 + lane_off;
-      const int* kbt = bar.kblk[j & 1];
-      // pass 1: row max of the visible scores
+      const uint32_t sbase = tS + (j & 1) * 128 + col0 + lane_off;
+      const short* kbt = bar.kblk[j & 1] + col0;
+      float v[64];
+      tmem_ld64(sbase, v);
+      // pass 1: half-row maximum of the visible scores, exchanged with the partner thread
       float mt = -INFINITY;
+      if (fast) {
 #pragma unroll
-      for (int c0 = 0; c0 < 128; c0 += 32) {
-        float v[32];
-        tmem_ld32(sbase + c0, v);
-        if (fast) {
+        for (int u = 0; u < 64; ++u) mt = fmaxf(mt, v[u]);
+      } else {
 #pragma unroll
-          for (int u = 0; u < 32; ++u) mt = fmaxf(mt, v[u]);
-        } else {
-#pragma unroll
-          for (int u = 0; u < 32; ++u)
-            if (kbt[c0 + u] <= qblk) mt = fmaxf(mt, v[u]);
-        }
+        for (int u = 0; u < 64; ++u)
+          if (kbt[u] <= qrel) mt = fmaxf(mt, v[u]);
       }
-      mt *= p.scale_log2;
+      bar.rowmax[half][row] = mt;
+      tc::named_bar_sync(2, 256);
+      mt = fmaxf(bar.rowmax[0][row], bar.rowmax[1][row]) * p.scale_log2;
       const float m_new = fmaxf(m, mt);
       const float alpha = (m_new == -INFINITY) ? 1.f : exp2f(m - m_new);
-      // fold in the previous tile's P V before rescaling
-      if (j > 0) {
-        if (!wait_bar(&bar.o_full, (j - 1) & 1, abort_flag, p.status, ST_TIMEOUT_EPILOGUE)) { ok = false; break; }
-        tc::fence_after_sync();
-#pragma unroll
-        for (int c0 = 0; c0 < 128; c0 += 32) {
-          float v[32];
-          tmem_ld32(tO + lane_off + c0, v);
-#pragma unroll
-          for (int u = 0; u < 32; ++u) o[c0 + u] += v[u];
-        }
-      }
-#pragma unroll
-      for (int c = 0; c < 128; ++c) o[c] *= alpha;
-      l *= alpha;
-      // pass 2: P = exp2(s - m_new) as bf16 into the swizzled K-major P tile
+      // pass 2: P = exp2(s - m_new) as bf16 into this half's chunk of the tile's swizzled K-major P buffer
+      uint8_t* sPj = sP + (j & 1) * TILE + half * CHUNK;
       float rs = 0.f;
 #pragma unroll
-      for (int c0 = 0; c0 < 128; c0 += 32) {
-        float v[32];
-        tmem_ld32(sbase + c0, v);
+      for (int u8 = 0; u8 < 8; ++u8) {
+        uint32_t packed[4];
 #pragma unroll
-        for (int u8 = 0; u8 < 4; ++u8) {
-          uint32_t packed[4];
+        for (int h2 = 0; h2 < 4; ++h2) {
+          float pv[2];
 #pragma unroll
-          for (int h2 = 0; h2 < 4; ++h2) {
-            float pv[2];
-#pragma unroll
-            for (int e2 = 0; e2 < 2; ++e2) {
-              const int c = c0 + u8 * 8 + h2 * 2 + e2;
-              const bool vis = (fast || kbt[c] <= qblk) && m_new != -INFINITY;
-              const float e = vis ? exp2f(v[u8 * 8 + h2 * 2 + e2] * p.scale_log2 - m_new) : 0.f;
-              pv[e2] = e;
-            }
-            __nv_bfloat162 pr = __floats2bfloat162_rn(pv[0], pv[1]);
-            rs += __bfloat162float(pr.x) + __bfloat162float(pr.y);
-            packed[h2] = *reinterpret_cast<uint32_t*>(&pr);
+          for (int e2 = 0; e2 < 2; ++e2) {
+            const int c = u8 * 8 + h2 * 2 + e2;
+            const bool vis = (fast || kbt[c] <= qrel) && m_new != -INFINITY;
+            pv[e2] = vis ? exp2f(v[c] * p.scale_log2 - m_new) : 0.f;
           }
-          const int key8 = (c0 >> 3) + u8;             // 16-byte unit index along the 128 keys
-          const int chunk = key8 >> 3, unit = key8 & 7;
-          uint8_t* dst = sP + chunk * CHUNK + row * 128 + ((unit ^ (row & 7)) << 4);
-          *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+          __nv_bfloat162 pr = __floats2bfloat162_rn(pv[0], pv[1]);
+          rs += __bfloat162float(pr.x) + __bfloat162float(pr.y);
+          packed[h2] = *reinterpret_cast<uint32_t*>(&pr);
         }
+        uint8_t* dst = sPj + row * 128 + ((u8 ^ (row & 7)) << 4);
+        *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
       }
-      l += rs;
-      m = m_new;
       fence_proxy_async_smem();
       tc::fence_before_sync();
       tc::mbar_arrive(&bar.p_ready);
+      // fold in the previous tile's P V (previous max's scale), then move to this tile's scale
+      if (j > 0) {
+        if (!wait_bar(&bar.o_full[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, p.status, ST_TIMEOUT_EPILOGUE)) {
+          ok = false;
+          break;
+        }
+        tc::fence_after_sync();
+        float w[64];
+        tmem_ld64(tO + ((j - 1) & 1) * 128 + col0 + lane_off, w);
+#pragma unroll
+        for (int u = 0; u < 64; ++u) o[u] += w[u];
+      }
+#pragma unroll
+      for (int c = 0; c < 64; ++c) o[c] *= alpha;
+      l = l * alpha + rs;          // this half's share of the row sum
+      m = m_new;
     }
     if (ok && ntile > 0) {
-      if (wait_bar(&bar.o_full, (ntile - 1) & 1, abort_flag, p.status, ST_TIMEOUT_EPILOGUE)) {
+      const int jl = ntile - 1;
+      if (wait_bar(&bar.o_full[jl & 1], (jl >> 1) & 1, abort_flag, p.status, ST_TIMEOUT_EPILOGUE)) {
         tc::fence_after_sync();
+        float w[64];
+        tmem_ld64(tO + (jl & 1) * 128 + col0 + lane_off, w);
 #pragma unroll
-        for (int c0 = 0; c0 < 128; c0 += 32) {
-          float v[32];
-          tmem_ld32(tO + lane_off + c0, v);
-#pragma unroll
-          for (int u = 0; u < 32; ++u) o[c0 + u] += v[u];
-        }
+        for (int u = 0; u < 64; ++u) o[u] += w[u];
       }
     }
-    if (row_ok && !*abort_flag) {
-      const int h = g * p.G + hh;
-      const int64_t qh = ((int64_t)b * p.Lq + qg) * p.Hq + h;
-      if (p.n_splits == 1) {
-        const float inv = l > 0.f ? 1.0f / l : 0.f;
-        uint4* dst = reinterpret_cast<uint4*>(p.out + qh * 128);
+    // row sums: the two halves' shares
+    float* lsum = &bar.rowmax[0][0];             // reused: [2][128]
+    tc::named_bar_sync(1, 256);
+    lsum[half * 128 + row] = l;
+    tc::named_bar_sync(1, 256);
+    const float l_row = lsum[row] + lsum[128 + row];
+    if (p.n_splits == 1) {
+      if (row_ok && !*abort_flag) {
+        const int64_t qh = ((int64_t)b * p.Lq + qg) * p.Hq + g * p.G + hh;
+        const float inv = l_row > 0.f ? 1.0f / l_row : 0.f;
+        uint4* dst = reinterpret_cast<uint4*>(p.out + qh * 128 + col0);
 #pragma unroll
-        for (int c = 0; c < 128; c += 8) {
+        for (int c = 0; c < 64; c += 8) {
           __nv_bfloat162 a0 = __floats2bfloat162_rn(o[c] * inv, o[c + 1] * inv);
           __nv_bfloat162 a1 = __floats2bfloat162_rn(o[c + 2] * inv, o[c + 3] * inv);
           __nv_bfloat162 a2 = __floats2bfloat162_rn(o[c + 4] * inv, o[c + 5] * inv);
@@ -378,16 +408,66 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           dst[c >> 3] = make_uint4(*reinterpret_cast<uint32_t*>(&a0), *reinterpret_cast<uint32_t*>(&a1),
                                    *reinterpret_cast<uint32_t*>(&a2), *reinterpret_cast<uint32_t*>(&a3));
         }
-      } else {
-        const int64_t nq = (int64_t)p.B * p.Lq * p.Hq;
-        float4* dst = reinterpret_cast<float4*>(p.po + ((int64_t)split * nq + qh) * 128);
+      }
+    } else {
+      // this split's unnormalised row (log2-domain max; an empty split leaves (-inf, 0)) into the idle K/V ring:
+      // o at [row][128] with the 16-byte units rotated by the row to spread banks, then m and l
+      float* so = reinterpret_cast<float*>(sK);
+      float4* orow = reinterpret_cast<float4*>(so + row * 128);
 #pragma unroll
-        for (int c = 0; c < 128; c += 4) dst[c >> 2] = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
-        // log2-domain max; an empty split leaves (-inf, 0)
-        p.pm[split * nq + qh] = m;
-        p.pl[split * nq + qh] = l;
+      for (int c = 0; c < 64; c += 4)
+        orow[(((col0 + c) >> 2) + row) & 31] = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
+      if (half == 0) {
+        so[128 * 128 + row] = m;
+        so[128 * 128 + 128 + row] = l_row;
       }
     }
+  }
+  if (p.n_splits > 1) {
+    // merge the splits of this tile: rank r owns rows [r*128/ns, (r+1)*128/ns); it reads every split's (o, m, l)
+    // of its rows through distributed shared memory, in rank order
+    __syncthreads();
+    cluster_sync();
+    if (warp >= 2 && !*abort_flag) {
+      const int ns = p.n_splits;
+      const int r0 = split * 128 / ns, r1 = (split + 1) * 128 / ns;
+      const float* so = reinterpret_cast<const float*>(sK);
+      const int etid = tid - 64;
+      const int d4 = etid & 31;               // this thread's 4 output columns
+      for (int rr = r0 + (etid >> 5); rr < r1; rr += 8) {
+        const int qi = rr / p.G, hh2 = rr % p.G, qg = q0 + qi;
+        float ms[8];
+        float M = -INFINITY;
+#pragma unroll
+        for (int sp = 0; sp < 8; ++sp) {
+          ms[sp] = sp < ns ? ld_dsmem(so + 128 * 128 + rr, (uint32_t)sp) : -INFINITY;
+          M = fmaxf(M, ms[sp]);
+        }
+        float L = 0.f;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int sp = 0; sp < 8; ++sp) {
+          const float w = (sp < ns && ms[sp] != -INFINITY) ? exp2f(ms[sp] - M) : 0.f;
+          if (w != 0.f) {
+            L += w * ld_dsmem(so + 128 * 128 + 128 + rr, (uint32_t)sp);
+            const float4 v4 = ld_dsmem4(so + rr * 128 + (((d4 + rr) & 31) << 2), (uint32_t)sp);
+            acc.x += w * v4.x;
+            acc.y += w * v4.y;
+            acc.z += w * v4.z;
+            acc.w += w * v4.w;
+          }
+        }
+        if (qg < p.Lq) {
+          const float inv = L > 0.f ? 1.0f / L : 0.f;
+          const int64_t qh = ((int64_t)b * p.Lq + qg) * p.Hq + g * p.G + hh2;
+          __nv_bfloat162 a0 = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+          __nv_bfloat162 a1 = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+          uint2* dst = reinterpret_cast<uint2*>(p.out + qh * 128 + d4 * 4);
+          *dst = make_uint2(*reinterpret_cast<uint32_t*>(&a0), *reinterpret_cast<uint32_t*>(&a1));
+        }
+      }
+    }
+    cluster_sync();
   }
   __syncthreads();
   if (warp == 1) {
@@ -437,8 +517,8 @@ void plan_tc(int B, int Lq, int Hq, int Hkv, int n_keys, int& QT, int& n_qtiles,
   n_qtiles = (Lq + QT - 1) / QT;
   const int tiles = (n_keys + KT - 1) / KT;
   const int base = B * Hkv * n_qtiles;
-  int want = (4 * num_sms() + base - 1) / base;
-  n_splits = max(1, min(want, tiles));
+  int want = (3 * num_sms() / 2 + base - 1) / base;
+  n_splits = max(1, min(min(want, tiles), 8));
   tps = (tiles + n_splits - 1) / n_splits;
   n_splits = max(1, (tiles + tps - 1) / tps);
 }
@@ -451,13 +531,7 @@ bool attn_tc_supported(int dtype, int Hq, int Hkv, int d) {
   return G >= 1 && G <= 128 && (128 % G) == 0;
 }
 
-size_t attn_tc_workspace_bytes(int B, int Lq, int Hq, int Hkv, int n_keys) {
-  int QT, nqt, ns, tps;
-  plan_tc(B, Lq, Hq, Hkv, n_keys, QT, nqt, ns, tps);
-  if (ns <= 1) return 0;
-  const size_t nq = (size_t)B * Lq * Hq;
-  return ns * nq * 128 * 4 + 2 * ns * nq * 4 + 512;
-}
+size_t attn_tc_workspace_bytes(int, int, int, int, int) { return 0; }  // splits merge on chip
 
 int launch_attn_tc(const AttnArgs& a, int32_t* status, cudaStream_t s) {
   DLLM_REQUIRE(((uintptr_t)a.q % 16 == 0) && ((uintptr_t)a.k % 16 == 0) && ((uintptr_t)a.v % 16 == 0),
@@ -470,17 +544,7 @@ int launch_attn_tc(const AttnArgs& a, int32_t* status, cudaStream_t s) {
   p.scale_log2 = scale * 1.4426950408889634f;
   p.key_pos = a.key_pos;
   p.out = static_cast<__nv_bfloat16*>(a.out);
-  p.po = p.pm = p.pl = nullptr;
   p.status = status;
-  if (p.n_splits > 1) {
-    const size_t nq = (size_t)a.B * a.Lq * a.Hq;
-    const size_t need = p.n_splits * nq * 128 * 4 + 2 * p.n_splits * nq * 4;
-    DLLM_REQUIRE(a.ws && a.ws_bytes >= need, DLLM_ERR_WORKSPACE, "attention workspace too small (%zu < %zu)",
-                 a.ws_bytes, need);
-    p.po = static_cast<float*>(a.ws);
-    p.pm = p.po + p.n_splits * nq * 128;
-    p.pl = p.pm + p.n_splits * nq;
-  }
   CUtensorMap mq, mk, mv;
   {
     cuuint64_t dims[4] = {128, (cuuint64_t)a.Hq, (cuuint64_t)a.Lq, (cuuint64_t)a.B};
@@ -505,10 +569,21 @@ int launch_attn_tc(const AttnArgs& a, int32_t* status, cudaStream_t s) {
     if (e != cudaSuccess) return dllm_host::cuda_status(e, "cudaFuncSetAttribute(attn_tc)");
     configured = true;
   }
-  dim3 grid(a.B * a.Hkv * p.n_qtiles, p.n_splits);
-  attn_tc_kernel<<<grid, NT, SMEM, s>>>(mq, mk, mv, p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.n_splits, a.B * a.Hkv * p.n_qtiles, 1);
+  cfg.blockDim = dim3(NT, 1, 1);
+  cfg.dynamicSmemBytes = SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = p.n_splits;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, attn_tc_kernel, mq, mk, mv, p);
+  if (e != cudaSuccess) return dllm_host::cuda_status(e, "cudaLaunchKernelEx(attn_tc_kernel)");
   DLLM_CHECK_LAUNCH("attn_tc_kernel");
-  if (p.n_splits > 1) return launch_attn_merge(a, p.n_splits, p.po, p.pm, p.pl, s);
   return DLLM_OK;
 }
 

@@ -15,6 +15,9 @@
 namespace dllm {
 namespace {
 
+constexpr int kRegVpt = 16;                      // 16-byte vectors per thread kept in registers
+constexpr int kRegChunk = kRegVpt * 256 * 8;     // vocabulary entries per CTA of the register path (32768)
+
 struct Partial {
   float m;    // max logit
   int idx;    // lowest index attaining m (absolute vocabulary index within the scored slice)
@@ -135,6 +138,85 @@ __global__ void __launch_bounds__(256) unmask_reduce_kernel(const T* __restrict_
   }
 }
 
+// bf16 logits without guidance: each thread keeps its VPT 16-byte vectors of the chunk in registers. Pass 1 finds
+// the maximum with packed bf16x2 max (and the first vector holding it); pass 2 sums exp(z - max) as
+// ex2((z - max) * log2(e)) in fp32 (z - max is exact near the maximum), accumulated per thread in fp32 over at most
+// VPT * 8 terms and then in fp64; the lowest arg-max comes from the first vector that holds the maximum.
+template <int VPT>
+__global__ void __launch_bounds__(256) unmask_reduce_bf16_kernel(const __nv_bfloat16* __restrict__ logits,
+                                                                 const int32_t* __restrict__ n_rows, int V, int chunk,
+                                                                 Partial* __restrict__ part, int n_chunks) {
+  const int r = blockIdx.x, c = blockIdx.y;
+  if (r >= *n_rows) return;
+  const __nv_bfloat16* z = logits + (int64_t)r * V;
+  const int v0 = c * chunk, v1 = min(V, v0 + chunk);
+  const int nvec = (v1 - v0) >> 3;
+  uint4 u[VPT];
+#pragma unroll
+  for (int k = 0; k < VPT; ++k) {
+    const int i = threadIdx.x + k * 256;
+    u[k] = i < nvec ? ld_nc_v4(z + v0 + i * 8) : make_uint4(0xff80ff80u, 0xff80ff80u, 0xff80ff80u, 0xff80ff80u);
+  }
+  // pass 1: maximum (bf16 -inf fills the missing vectors) and the first vector that attains it
+  float m = -INFINITY;
+  int best = -1;
+#pragma unroll
+  for (int k = 0; k < VPT; ++k) {
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u[k]);
+    const __nv_bfloat162 a = __hmax2(__hmax2(h[0], h[1]), __hmax2(h[2], h[3]));
+    const float vm = fmaxf(__low2float(a), __high2float(a));
+    if (vm > m) { m = vm; best = k; }
+  }
+  Partial p{-INFINITY, 0x7fffffff, 0.0};
+  if (best >= 0) {
+    // pass 2: sum of exponentials relative to the thread's maximum
+    const float log2e = 1.4426950408889634f;
+    float acc = 0.f;
+#pragma unroll
+    for (int k = 0; k < VPT; ++k) {
+      const uint32_t w[4] = {u[k].x, u[k].y, u[k].z, u[k].w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float lo = __uint_as_float(w[q] << 16), hi = __uint_as_float(w[q] & 0xffff0000u);
+        acc += exp2f((lo - m) * log2e) + exp2f((hi - m) * log2e);
+      }
+    }
+    // lowest index attaining m inside the first vector that holds it
+    const uint4 bv = ld_nc_v4(z + v0 + (threadIdx.x + best * 256) * 8);
+    float f[8];
+    bf16x8_to_f32(bv, f);
+    int e = 7;
+#pragma unroll
+    for (int q = 7; q >= 0; --q)
+      if (f[q] == m) e = q;
+    p.m = m;
+    p.idx = v0 + (threadIdx.x + best * 256) * 8 + e;
+    p.s = (double)acc;
+  }
+  // scalar tail of the chunk (chunk lengths are multiples of 8 except the row's last chunk)
+  for (int v = v0 + nvec * 8 + threadIdx.x; v < v1; v += 256) {
+    Partial q{__bfloat162float(z[v]), v, 1.0};
+    merge(p, q);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    Partial q;
+    q.m = __shfl_xor_sync(0xffffffffu, p.m, o);
+    q.idx = __shfl_xor_sync(0xffffffffu, p.idx, o);
+    q.s = __shfl_xor_sync(0xffffffffu, p.s, o);
+    merge(p, q);
+  }
+  __shared__ Partial wp[8];
+  const int lane = threadIdx.x & 31, wv = threadIdx.x >> 5;
+  if (lane == 0) wp[wv] = p;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    Partial a = wp[0];
+    for (int i = 1; i < 8; ++i) merge(a, wp[i]);
+    part[(int64_t)r * n_chunks + c] = a;
+  }
+}
+
 // One warp per logical block row b (L <= 32 positions, lane i = position i). The still-masked flat positions are
 // the LM head's rows in increasing order, so the row of position (b, i) is the number of masked positions before it.
 __global__ void unmask_select_kernel(const Partial* __restrict__ part, int n_chunks, const int32_t* __restrict__ row_pos,
@@ -234,10 +316,12 @@ __global__ void unmask_select_kernel(const Partial* __restrict__ part, int n_chu
 }  // namespace
 
 int unmask_chunks(int max_rows, int V) {
-  // enough CTAs to cover the SMs a few times when every row is masked, chunks of at least 2048 entries
+  // enough CTAs to cover the SMs a few times when every row is masked, chunks of at least 2048 entries, and at most
+  // kRegChunk entries so that a thread's share of a chunk fits in registers
   int want = (4 * num_sms() + max(max_rows, 1) - 1) / max(max_rows, 1);
   int most = max(1, V / 2048);
-  return max(1, min(want, min(most, 64)));
+  int least = (V + kRegChunk - 1) / kRegChunk;
+  return max(1, max(least, min(want, min(most, 64))));
 }
 
 size_t unmask_partials_bytes(int max_rows, int n_chunks) {
@@ -252,6 +336,8 @@ int launch_unmask(const UnmaskArgs& a, cudaStream_t s) {
     if (a.dtype == DLLM_BF16) {
       const __nv_bfloat16* z = static_cast<const __nv_bfloat16*>(a.logits);
       if (a.cfg) unmask_reduce_kernel<__nv_bfloat16, true><<<grid, 256, 0, s>>>(z, a.n_rows, a.V, chunk, a.cfg_scale, part, a.n_chunks);
+      else if (a.V % 8 == 0 && chunk <= kRegChunk)
+        unmask_reduce_bf16_kernel<kRegVpt><<<grid, 256, 0, s>>>(z, a.n_rows, a.V, chunk, part, a.n_chunks);
       else unmask_reduce_kernel<__nv_bfloat16, false><<<grid, 256, 0, s>>>(z, a.n_rows, a.V, chunk, a.cfg_scale, part, a.n_chunks);
     } else {
       const float* z = static_cast<const float*>(a.logits);

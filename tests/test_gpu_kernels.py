@@ -201,6 +201,14 @@ def test_attention_group_sizes(Hq, Hkv):
     _attn_case("bf16", 2, 32, Hq, Hkv, 128, 32, 160, 192, 200, seed=7)
 
 
+def test_attention_far_positions_small_blocks():
+    """Positions far past the cache rows with one-token blocks (block indices beyond 2^15)."""
+    _attn_case("bf16", 1, 32, 16, 4, 128, 1, 100000, 300, 300, seed=9)
+    g = np.random.default_rng(10)
+    kp = np.sort(g.choice(np.arange(60000, 100000), 300, replace=False))[None, :]
+    _attn_case("bf16", 1, 32, 16, 4, 128, 7, 99990, 300, 300, key_pos=kp, seed=10)
+
+
 def test_attention_cache_tail_never_read():
     _attn_case("bf16", 2, 32, 16, 4, 128, 32, 200, 232, 300, seed=8, nan_tail=True)
     _attn_case("f32", 1, 16, 4, 4, 64, 16, 40, 56, 80, seed=8, nan_tail=True)

@@ -1,0 +1,237 @@
+"""Parity at the full sizes of the 20-layer workloads (text-to-image, thinking with SPRINT, understanding).
+
+Per call, every kernel runs at the workload's exact shapes on seeded inputs and is compared with the oracle on
+sampled rows (the oracle computes those one by one). The whole 20-layer denoising pass, where compounded bf16
+rounding makes a token-by-token oracle comparison meaningless (routing near-ties in some layer for nearly every
+token), is checked through properties that hold at any size: determinism, the unmasking rule applied to the
+pass's own confidences, the choice of the most confident positions, mirrored guided rows, finite values.
+"""
+import gc
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from block_diffusion_moe_dllm_b200 import binding as bd
+from block_diffusion_moe_dllm_b200 import synth
+from block_diffusion_moe_dllm_b200.configs import T2I, THINKING, UNDERSTANDING
+from block_diffusion_moe_dllm_b200.engine import DenoiseEngine
+from oracle import dllm_oracle as O
+from _util import assert_close, assignment_tables, random_assignments, to64
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(autouse=True)
+def _free():
+    yield
+    gc.collect()
+    torch.cuda.empty_cache()
+
+
+# ------------------------------------------------------------------------------------------------ attention
+@pytest.mark.parametrize("w", [T2I, THINKING, UNDERSTANDING], ids=["t2i", "thinking", "understanding"])
+def test_full_attention(w):
+    L, Hq, Hkv, d = w.L, w.Hq, w.Hkv, w.d
+    key_pos = None
+    if w.sprint:
+        n_keys = w.n_keep + L
+        g = np.random.default_rng(21)
+        key_pos = np.stack([np.concatenate([np.sort(g.choice(w.P, w.n_keep, replace=False)), np.arange(w.P, w.P + L)])
+                            for _ in range(w.B)]).astype(np.int32)
+    else:
+        n_keys = w.P + L
+    cap = n_keys
+    q = synth.normal((w.B, L, Hq, d), 1.0, 20, "fa_q", DEV)
+    kc = synth.normal((w.B, Hkv, cap, d), 1.0, 20, "fa_k", DEV)
+    vc = synth.normal((w.B, Hkv, cap, d), 1.0, 20, "fa_v", DEV)
+    out = torch.full((w.B, L, Hq * d), float("nan"), dtype=torch.bfloat16, device=DEV)
+    kp = None if key_pos is None else torch.from_numpy(key_pos).to(DEV)
+    bd.block_attn(q, kc, vc, out, w.B, L, Hq, Hkv, d, L, w.P, n_keys, cap, bd.BF16, key_pos=kp)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out.float()).all()
+    for b in sorted({0, w.B - 1}):
+        kpos = np.arange(n_keys) if key_pos is None else key_pos[b]
+        want = O.store(O.attention(to64(q[b]), to64(kc[b]).transpose(1, 0, 2), to64(vc[b]).transpose(1, 0, 2),
+                                   np.arange(w.P, w.P + L), kpos, L), "bf16")
+        assert_close(to64(out[b]).reshape(L, Hq, d), want, "bf16", f"attention row {b}")
+
+
+# ------------------------------------------------------------------------------------------------ SPRINT
+def test_full_prefix_retain_thinking():
+    w = THINKING
+    B, Hkv, d, P = w.B, w.Hkv, w.d, w.P
+    cap, n_keep, cap_thin = P + w.L, w.n_keep, w.n_keep + w.L
+    kc = synth.normal((B, Hkv, cap, d), 1.0, 22, "fr_k", DEV)
+    vc = synth.normal((B, Hkv, cap, d), 1.0, 22, "fr_v", DEV)
+    keep = torch.full((B, cap_thin), -1, dtype=torch.int32, device=DEV)
+    kt = torch.zeros((B, Hkv, cap_thin, d), dtype=torch.bfloat16, device=DEV)
+    vt = torch.zeros_like(kt)
+    bd.prefix_retain(kc, vc, keep, kt, vt, B, Hkv, d, P, cap, n_keep, cap_thin, bd.BF16)
+    torch.cuda.synchronize()
+    for b in range(B):
+        o_keep, sc, margin = O.prefix_retain(to64(kc[b, :, :P]), None, n_keep=n_keep)
+        got = keep[b, :n_keep].cpu().numpy()
+        if margin > 1e-6 * sc.max():
+            assert np.array_equal(got, o_keep), f"row {b}"
+        idx = torch.from_numpy(got.astype(np.int64)).to(DEV)
+        assert torch.equal(kt[b, :, :n_keep], kc[b][:, idx]) and torch.equal(vt[b, :, :n_keep], vc[b][:, idx])
+
+
+# ------------------------------------------------------------------------------------------------ MoE
+def test_full_router_understanding():
+    w = UNDERSTANDING
+    Tk, H, E, k = w.Tk, w.H, w.E, w.k
+    h = synth.normal((Tk, H), 1.0, 23, "fro_h", DEV)
+    wr = synth.normal((E, H), 0.02, 23, "fro_w", DEV)
+    bias = synth.uniform((E,), -0.1, 0.1, 23, "fro_b", DEV)
+    ids = torch.empty((Tk, k), dtype=torch.int32, device=DEV)
+    gates = torch.empty((Tk, k), dtype=torch.float32, device=DEV)
+    counts = torch.empty(E, dtype=torch.int32, device=DEV)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=DEV)
+    perm = torch.empty(Tk * k, dtype=torch.int32, device=DEV)
+    inv = torch.empty(Tk * k, dtype=torch.int32, device=DEV)
+    bd.moe_route(h, wr, bias, ids, gates, counts, offsets, perm, inv, Tk, H, E, k, bd.BF16)
+    torch.cuda.synchronize()
+    o_ids, o_gates, _, margin = O.route(to64(h), to64(wr), to64(bias), k)
+    ok = margin >= 1e-6
+    assert ok.mean() > 0.9
+    assert np.array_equal(ids.cpu().numpy()[ok], o_ids[ok])
+    assert np.allclose(gates.cpu().numpy()[ok], o_gates[ok], rtol=5e-6, atol=5e-7)
+    c, off, p, iv = assignment_tables(ids.cpu().numpy(), E)
+    assert np.array_equal(perm.cpu().numpy(), p) and np.array_equal(inv.cpu().numpy(), iv)
+
+
+def test_full_experts_understanding():
+    w = UNDERSTANDING
+    Tk, H, E, k, I = w.Tk, w.H, w.E, w.k, w.I
+    h = synth.normal((Tk, H), 1.0, 24, "fe_h", DEV)
+    x0 = synth.normal((Tk, H), 1.0, 24, "fe_x", DEV)
+    wgu = synth.normal((E, 2 * I, H), 0.02, 24, "fe_gu", DEV, chunk_rows=16)
+    wd = synth.normal((E, H, I), 0.02, 24, "fe_d", DEV, chunk_rows=16)
+    sgu = synth.normal((2 * I, H), 0.02, 24, "fe_sgu", DEV)
+    sd = synth.normal((H, I), 0.02, 24, "fe_sd", DEV)
+    ids, gates = random_assignments(Tk, E, k, seed=24)
+    counts, offsets, perm, inv = assignment_tables(ids, E)
+    cvt = lambda a: torch.from_numpy(a).to(DEV)
+    x = x0.clone()
+    bd.moe_experts(h, wgu, wd, sgu, sd, cvt(counts), cvt(offsets), cvt(perm), cvt(inv), cvt(gates), x, Tk, H, E, k, I,
+                   bd.BF16)
+    torch.cuda.synchronize()
+    rows = np.random.default_rng(24).choice(Tk, 24, replace=False)
+    delta = O.moe_delta(to64(h[rows]), ids[rows], gates[rows].astype(np.float64), wgu, wd, sgu, sd, "bf16")
+    want = O.store(to64(x0[rows]) + delta, "bf16")
+    assert_close(to64(x[rows]), want, "bf16", "experts (sampled tokens)")
+
+
+# ------------------------------------------------------------------------------------------------ LM head
+def test_full_lm_head_understanding():
+    w = UNDERSTANDING
+    rows, V, H = w.B * w.L, w.V, w.H
+    x = synth.normal((rows, H), 1.0, 25, "fl_x", DEV)
+    wl = synth.normal((V, H), w.lm_std, 25, "fl_w", DEV, chunk_rows=16384)
+    y = torch.empty((rows, V), dtype=torch.bfloat16, device=DEV)
+    bd.gemm(x, wl, y, rows, V, H, bd.BF16)
+    torch.cuda.synchronize()
+    sample = np.random.default_rng(25).choice(rows, 6, replace=False)
+    xs = to64(x[sample])
+    want = np.concatenate([O.store(xs @ to64(wl[v0: v0 + 16384]).T, "bf16") for v0 in range(0, V, 16384)], axis=1)
+    assert_close(to64(y[sample]), want, "bf16", "LM head (sampled rows)")
+
+
+# ------------------------------------------------------------------------------------------------ unmask
+@pytest.mark.parametrize("w", [T2I, THINKING, UNDERSTANDING], ids=["t2i", "thinking", "understanding"])
+def test_full_unmask(w):
+    Bl = w.B // 2 if w.cfg else w.B
+    L, V = w.L, w.vlen
+    n = Bl * L
+    std = 6.0 if w.mode == 1 else 1.0
+    logits = synth.normal(((2 if w.cfg else 1) * n, V), std, 26, "fu_z", DEV)
+    mask = np.ones((w.B, L), dtype=np.uint8)
+    tokens = np.full((w.B, L), w.mask_id, dtype=np.int32)
+    row_pos = np.arange(n, dtype=np.int32)
+    dt, dm = torch.from_numpy(tokens).to(DEV), torch.from_numpy(mask).to(DEV)
+    sel = torch.empty((Bl, L), dtype=torch.int32, device=DEV)
+    nsel = torch.empty(Bl, dtype=torch.int32, device=DEV)
+    conf = torch.empty((Bl, L), dtype=torch.float32, device=DEV)
+    rem = torch.empty(1, dtype=torch.int32, device=DEV)
+    bd.unmask(logits, torch.from_numpy(row_pos).to(DEV), torch.tensor([n], dtype=torch.int32, device=DEV), dt, dm,
+              sel, nsel, conf, rem, Bl, L, V, n, 0, w.T_s, bd.BF16, mode=w.mode, tau=w.tau, k_max=w.k_max, cfg=w.cfg,
+              cfg_scale=w.cfg_scale, vocab_offset=w.vocab_offset)
+    torch.cuda.synchronize()
+    zl = to64(logits)
+    u = O.unmask(zl[:n], row_pos, tokens, mask, 0, w.T_s, w.mode, float(np.float32(w.tau)), w.k_max,
+                 w.vocab_offset, z_uncond=zl[n:] if w.cfg else None, cfg_scale=float(np.float32(w.cfg_scale)))
+    g_conf = conf.cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(g_conf - u["conf"]) <= 1e-6 * np.maximum(u["conf"], 1e-30) + 1e-12)
+    for b in range(Bl):
+        if u["tie_rank"][b] or u["tie_tau"][b]:
+            continue
+        assert nsel[b].item() == u["nsel"][b]
+        assert np.array_equal(dt.cpu().numpy()[b], u["tokens"][b]) and np.array_equal(dm.cpu().numpy()[b], u["mask"][b])
+
+
+# ------------------------------------------------------------------------------------------------ whole pass
+def _check_pass_properties(w, eng, tok0, mask0, t):
+    Bl = w.B // 2 if w.cfg else w.B
+    conf = eng.conf.cpu().numpy().astype(np.float64)
+    nsel = eng.nsel.cpu().numpy()
+    tok = eng.tokens.cpu().numpy()
+    msk = eng.mask.cpu().numpy()
+    m0 = mask0.cpu().numpy()
+    t0 = tok0.cpu().numpy()
+    for b in range(Bl):
+        masked = m0[b].astype(bool)
+        m = int(masked.sum())
+        c = conf[b]
+        assert np.all((c[masked] > 0) & (c[masked] <= 1.0)) and np.all(c[~masked] == 0)
+        floor_k = -(-m // (w.T_s - t))
+        if w.mode == 0:
+            k = min(m, floor_k)
+        else:
+            above = int(np.sum(c[masked] > np.float32(w.tau)))
+            k = min(m, max(floor_k, min(w.k_max, above)))
+        assert nsel[b] == k
+        newly = masked & (msk[b] == 0)
+        assert int(newly.sum()) == k
+        # the unmasked positions are the most confident masked ones
+        still = masked & (msk[b] == 1)
+        if newly.any() and still.any():
+            assert c[newly].min() >= c[still].max()
+        assert np.all((tok[b][newly] >= w.vocab_offset) & (tok[b][newly] < w.vocab_offset + w.vlen))
+        assert np.array_equal(tok[b][~newly], t0[b][~newly])
+        if w.cfg:
+            assert np.array_equal(tok[b + Bl], tok[b]) and np.array_equal(msk[b + Bl], msk[b])
+    assert eng.remaining.item() == int(msk[:Bl].sum())
+
+
+@pytest.mark.parametrize("w", [T2I, THINKING, UNDERSTANDING], ids=["t2i", "thinking", "understanding"])
+def test_full_denoise_pass_properties(w):
+    wt = synth.make_weights(w, DEV)
+    caches = synth.make_prefix_cache(w, DEV)
+    tok0, mask0 = synth.make_block_state(w, DEV)
+    eng = DenoiseEngine(w, wt, caches, DEV)
+    results = []
+    for rep in range(2):
+        eng.set_block(tok0, mask0)
+        eng.step(0)
+        torch.cuda.synchronize()
+        assert bd.status_check(eng.ws) == bd.OK
+        n = int(mask0[: (w.B // 2 if w.cfg else w.B)].sum().item())
+        lg = eng.logits(n)
+        assert torch.isfinite(lg.float()).all()
+        results.append((eng.tokens.clone(), eng.mask.clone(), eng.conf.clone(), lg.clone()))
+        if rep == 0:
+            _check_pass_properties(w, eng, tok0, mask0, 0)
+    # the pass is deterministic: identical bits on a second run from the same state
+    for a, b in zip(results[0], results[1]):
+        assert torch.equal(a, b)
+    # a full block then the commit pass finishes with every position unmasked
+    eng.set_block(tok0, mask0)
+    eng.decode_block()
+    torch.cuda.synchronize()
+    assert int(eng.mask.sum().item()) == 0
+    assert bd.status_check(eng.ws) == bd.OK
+    del eng, wt, caches

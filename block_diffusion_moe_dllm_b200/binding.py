@@ -79,6 +79,7 @@ _SIGS = {
     "dllm_last_error": ([], C.c_char_p),
     "dllm_status_check": ([vp, vp], C.c_int),
     "dllm_launch_count": ([], C.c_ulonglong),
+    "dllm_selftest_bounded_wait": ([vp, sz, vp], C.c_int),
     "dllm_gemm": ([C.POINTER(GemmDesc), vp, vp, vp, vp, vp, sz, vp], C.c_int),
     "dllm_gemm_workspace_size": ([C.POINTER(GemmDesc)], sz),
     "dllm_block_attn": ([C.POINTER(AttnDesc), vp, vp, vp, vp, vp, vp, sz, vp], C.c_int),

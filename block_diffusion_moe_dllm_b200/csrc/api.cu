@@ -8,6 +8,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "misc.h"
+#include "tc.cuh"
 
 #include <atomic>
 #include <algorithm>
@@ -240,8 +241,28 @@ void plan_step(const dllm_model* m, const dllm_state* st, const dllm_step_params
 
 }  // namespace
 
+// A kernel that waits on an mbarrier nothing ever arrives at, with the same bounded poll loop as the tensor-core
+// kernels (a short bound here), then records the timeout in the status word and returns.
+__global__ void selftest_wait_kernel(int32_t* status, uint32_t max_polls) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    dllm::tc::mbar_init(&bar, 1);
+    dllm::tc::fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && !dllm::tc::mbar_wait(&bar, 0, max_polls)) atomicExch(status, dllm::ST_TIMEOUT_MMA);
+}
+
 // ================================================================================================== ABI
 extern "C" {
+
+int dllm_selftest_bounded_wait(void* ws, size_t ws_bytes, cudaStream_t stream) {
+  int st = check_ws(ws, ws_bytes, kStatusBytes);
+  if (st) return st;
+  selftest_wait_kernel<<<1, 32, 0, stream>>>(status_word(ws), 1u << 12);
+  DLLM_CHECK_LAUNCH("selftest_wait_kernel");
+  return DLLM_OK;
+}
 
 const char* dllm_version(void) { return "dllm-b200 0.1 (sm_100a)"; }
 const char* dllm_last_error(void) { return dllm_host::g_err; }

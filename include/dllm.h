@@ -68,6 +68,12 @@ DLLM_API unsigned long long dllm_launch_count(void);
  * does). Returns DLLM_OK, DLLM_ERR_TIMEOUT (a kernel stopped after a bounded wait), or DLLM_ERR_CUDA. */
 DLLM_API int dllm_status_check(void* ws, cudaStream_t stream);
 
+/* Failure-path self-test: launches one kernel that waits on an mbarrier nothing arrives at, through the same
+ * bounded wait the tensor-core kernels use (with a short bound), so that it gives up, records DLLM_ERR_TIMEOUT's
+ * cause in the workspace status word and returns. dllm_status_check(ws) then reports DLLM_ERR_TIMEOUT (and clears
+ * the word). No GPU state is left behind. */
+DLLM_API int dllm_selftest_bounded_wait(void* ws, size_t ws_bytes, cudaStream_t stream);
+
 /* ---------------------------------------------------------------------------------------------- dense GEMM */
 /*
  * Y[n, m] = sum_k X[n, k] * W[m, k] for n < N, m < M: the projection primitive of the backbone (QKV, output

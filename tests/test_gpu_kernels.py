@@ -317,3 +317,16 @@ def test_unmask_last_step_takes_all():
 
 def test_unmask_f32():
     _unmask_case(1, 16, 1024, 1.0, 0, 4, bd.FIXED, 1.0, dtype="f32", seed=15)
+
+
+# ------------------------------------------------------------------------------------------------ failure path
+def test_bounded_wait_reports_timeout_and_recovers():
+    """A wait that can never complete gives up after its bound, the status word says so, the context stays usable."""
+    lib = bd.load()
+    ws = bd.Workspace(4096, DEV)
+    assert bd.status_check(ws) == bd.OK
+    bd.check(lib.dllm_selftest_bounded_wait(ws.addr, ws.nbytes, bd.stream_handle()))
+    assert bd.status_check(ws) == bd.ERR_TIMEOUT
+    assert bd.status_check(ws) == bd.OK                      # the check clears the word
+    x = torch.ones(8, device=DEV)                            # the context still works
+    assert float((x * 2).sum().item()) == 16.0

@@ -4,15 +4,22 @@
 //
 // One CTA per (batch row, kv head, tile of queries, key split). The 128-row M tile packs the G = Hq / Hkv query
 // heads that share the kv head with 128 / G queries (row r = query r / G, head r % G), so every K/V tile staged in
-// shared memory serves the whole group. Per 128-key tile:
-//   S = Q K^T      tcgen05.mma M=128 N=128 K=128 (Q, K K-major, TMA 128-byte swizzled) -> TMEM (double buffered)
-//   softmax        4 warps, one TMEM lane (query row) per thread: mask, scale, online max/sum, P = exp2(...) as
-//                  bf16 written to shared memory in the swizzled K-major layout
-//   O_t = P V      tcgen05.mma M=128 N=128 K=128 (P K-major, V MN-major straight from the [key][d] cache) -> TMEM
-//   o += O_t       accumulated in fp32 registers with the online-softmax rescale.
-// Warp 0 issues TMA (Q once; K and V tiles through a 2-stage ring), warp 1 issues the MMAs from one thread,
-// warps 2..5 run the softmax and write the output (or per-split partials merged by log-sum-exp).
-// Every mbarrier wait is bounded; on expiry the kernel records a status word and leaves.
+// shared memory serves the whole group. Per 128-key tile j:
+//   S_j = Q K_j^T   tcgen05.mma M=128 N=128 K=128 (Q, K K-major, TMA 128-byte swizzled) -> TMEM (two buffers)
+//   softmax         two groups of 4 warps take alternate tiles (group j mod 2), one thread per query row: mask,
+//                   scale, maximum; P_j = 2^(s - m_ref) as bf16, written back into the first 64 columns of S_j's
+//                   TMEM buffer (one buffer per group)
+//   O_g += P_j V_j  tcgen05.mma with A = P_j from TMEM and B = V_j (MN-major, straight from the [key][d] cache);
+//                   each group accumulates its own O_g in TMEM across its tiles, and the two are combined by
+//                   log-sum-exp at the end. While one group waits on loads, barriers and TMEM, the other's
+//                   exponentials keep the special-function unit busy.
+// m_ref is a per-row reference maximum that only moves when a tile's maximum exceeds it by more than 2^8 (then
+// O in TMEM and the row sum are rescaled once); in between, P values up to 2^8 are exact in bf16's range and the
+// result is the same softmax. Warp 0 issues TMA (Q once; K and V through a 3-stage ring), warp 1 issues the MMAs
+// from one thread, warps 2..9 run the softmax, combine O_0 and O_1 and write the output; with several key splits
+// (a thread-block cluster) every split pushes its unnormalised rows into the owning CTA's shared memory and the
+// owners merge them by log-sum-exp. Every mbarrier wait is bounded; on expiry the kernel records a status word
+// and leaves.
 #include "common.cuh"
 #include "tc.cuh"
 #include "misc.h"
@@ -26,32 +33,42 @@ constexpr int NT = 320;                     // warp 0 TMA, warp 1 MMA, warps 2..
 constexpr int KT = 128;                     // keys per tile
 constexpr int CHUNK = 128 * 64 * 2;         // one 64-wide K-major chunk of a 128-row tile: 16 KB
 constexpr int TILE = 2 * CHUNK;             // 128 rows x 128 elements: 32 KB
-constexpr int STAGES = 2;
+constexpr int STAGES = 3;
 constexpr int BARS_BYTES = 2048;
-constexpr short kNoKey = 0x7fff;   // relative block of a key past n_keys (never visible)
-constexpr int SMEM = 1024 + TILE /*Q*/ + STAGES * 2 * TILE /*K,V*/ + 2 * TILE /*P, double buffered*/ + BARS_BYTES;
+constexpr short kNoKey = 0x7fff;            // relative block of a key past n_keys (never visible)
+constexpr float kRescaleLog2 = 8.f;
+// named barriers: 1 + g = softmax group g's 128 threads inside its loop; kBarAll = all 256 softmax threads after
+// the loops (distinct ids, since one group can leave its loop while the other still synchronises inside its own)
+constexpr int kBarAll = 3;         // O and the row sum are rescaled when the maximum grows by > 2^8
+constexpr int kRecvStride = 132;            // floats per pushed row: o[128], m, l, 2 pad (16-byte multiple)
+constexpr int kRecvRowBytes = 130 * 4;      // bytes pushed per (split, row): o, m, l
+constexpr int SMEM = 1024 + TILE /*Q*/ + STAGES * 2 * TILE /*K,V*/ + BARS_BYTES;
 static_assert(SMEM <= 232448, "shared memory budget");
+static_assert(8 * 16 * kRecvStride * 4 <= STAGES * 2 * TILE && 7 * 19 * kRecvStride * 4 <= STAGES * 2 * TILE &&
+                  3 * 43 * kRecvStride * 4 <= STAGES * 2 * TILE,
+              "split merge buffer exceeds the K/V ring");
 
 struct Bars {
   uint64_t q_full;
   uint64_t kv_full[STAGES];
   uint64_t kv_empty[STAGES];
-  uint64_t s_full[2];
-  uint64_t p_ready;
-  uint64_t o_full[2];
+  uint64_t s_full[2];   // per softmax group: S of the group's next tile is in the group's TMEM buffer
+  uint64_t p_ready[2];  // per group: P of its tile written over S (and the group's O rescaled if needed)
+  uint64_t o_full[2];   // per group: phase i completes when the group's i-th P V is accumulated into its O
   uint64_t done;
+  uint64_t recv_full;   // split merge: completes when every split's rows owned by this CTA have arrived
   uint32_t tmem_base;
   int abort_flag;
-  short kblk[2][KT];    // block of each key of the tile relative to the CTA's first query block, clamped to
-                        // [-32768, 32766] (kNoKey past n_keys), per tile parity
-  unsigned vis_w[2][4]; // per tile, ballots of "key visible to every query of the CTA" (4 warps x 32 keys)
-  float rowmax[2][128]; // per column half, per row: the half-row maximum (the tile-start barrier separates uses)
+  short kblk[2][2][KT];     // [group][tile parity within the group][key]: block of the key relative to the CTA's
+                            // first query block, clamped to [-32768, 32766] (kNoKey past n_keys)
+  unsigned vis_w[2][2][4];  // [group][parity][warp]: ballots of "key visible to every query of the CTA"
 };
 static_assert(sizeof(Bars) <= BARS_BYTES, "barrier block exceeds its shared-memory reservation");
 
 struct AttnTcParams {
   int B, Lq, Hq, Hkv, G, QT, n_qtiles, n_keys, cap, blk_len, q_pos0;
   int n_splits, tiles_per_split;
+  uint32_t blk_magic, blk_shift;   // key position / blk_len = (pos * blk_magic) >> blk_shift for 0 <= pos < 2^31
   float scale_log2;
   const int32_t* key_pos;
   __nv_bfloat16* out;   // [B, Lq, Hq, 128]
@@ -71,6 +88,26 @@ __device__ __forceinline__ uint64_t sdesc_mn128(uint32_t addr, uint32_t lbo) {
   return d;
 }
 
+// D (TMEM) (+)= A (TMEM: 128 lanes = rows, two bf16 of K per 32-bit column) x B (shared memory descriptor).
+__device__ __forceinline__ void mma_bf16_tmem_a(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
+                                                uint32_t accumulate) {
+  uint32_t z = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %5, %5, %5}, p;\n\t}" ::"r"(tmem_d),
+      "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(z)
+      : "memory");
+}
+
+// Integer division by the block length without the divide sequence (which would queue on the special-function unit
+// behind the softmax's exponentials): multiply by m = ceil(2^(31+s) / d), 2^(s-1) < d <= 2^s, and keep the bits
+// above 31 + s; exact for 0 <= n < 2^31 since n (m d - 2^(31+s)) < 2^(31+s) (Granlund and Montgomery, "Division by
+// invariant integers using multiplication", 1994).
+__device__ __forceinline__ int div_blk(int n, uint32_t m, uint32_t shift) {
+  return (int)(((uint64_t)(uint32_t)n * m) >> shift);
+}
+
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int32_t* status,
                                          int code) {
   uint32_t n = 0;
@@ -83,6 +120,20 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
     }
   }
   return true;
+}
+
+// Named barrier over n threads that also ORs a predicate across them: every participant gets the same answer.
+__device__ __forceinline__ bool bar_sync_or(int id, int n, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.or.pred p, %2, %3, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
 }
 
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
@@ -100,26 +151,44 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+// Each lane writes 32 consecutive 32-bit columns of its own TMEM lane (completion: tmem_st_wait).
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
+      "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
+      "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
 }
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
 __device__ __forceinline__ uint32_t dsmem_addr(const void* local, uint32_t rank) {
   uint32_t remote;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(tc::smem_u32(local)), "r"(rank));
   return remote;
 }
-__device__ __forceinline__ float ld_dsmem(const float* local, uint32_t rank) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(dsmem_addr(local, rank)) : "memory");
-  return v;
-}
-__device__ __forceinline__ float4 ld_dsmem4(const float* local, uint32_t rank) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-               : "r"(dsmem_addr(local, rank))
+// Asynchronous store into another CTA's shared memory that counts its bytes on that CTA's mbarrier.
+__device__ __forceinline__ void st_async4(uint32_t remote, float a, float b, float c, float d, uint32_t remote_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
+                   remote),
+               "f"(a), "f"(b), "f"(c), "f"(d), "r"(remote_bar)
                : "memory");
-  return v;
+}
+__device__ __forceinline__ void st_async2(uint32_t remote, float a, float b, uint32_t remote_bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(remote),
+               "f"(a), "f"(b), "r"(remote_bar)
+               : "memory");
+}
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // Each lane reads 64 consecutive 32-bit columns of its own TMEM lane.
@@ -128,8 +197,30 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float* v) {
   tmem_ld32(taddr + 32, v + 32);
 }
 
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+// Packed fp32 pairs (sm_100 f32x2 instructions) and the hardware base-2 exponential (ex2.approx.ftz: relative
+// error about 2^-22; results below 2^-126 flush to 0, negligible next to the row's reference term 1).
+__device__ __forceinline__ uint64_t pk2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void upk2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ float ex2(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
 }
 
 __global__ void __launch_bounds__(NT, 1)
@@ -140,8 +231,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   uint8_t* sQ = base;
   uint8_t* sK = sQ + TILE;                    // [STAGES][TILE]
   uint8_t* sV = sK + STAGES * TILE;           // [STAGES][TILE]
-  uint8_t* sP = sV + STAGES * TILE;            // [2][TILE]
-  Bars& bar = *reinterpret_cast<Bars*>(sP + 2 * TILE);
+  Bars& bar = *reinterpret_cast<Bars*>(sV + STAGES * TILE);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   int bx = blockIdx.y;
@@ -171,19 +261,27 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       tc::mbar_init(&bar.kv_full[s], 1);
       tc::mbar_init(&bar.kv_empty[s], 1);
     }
-    tc::mbar_init(&bar.s_full[0], 1);
-    tc::mbar_init(&bar.s_full[1], 1);
-    tc::mbar_init(&bar.p_ready, 256);
-    tc::mbar_init(&bar.o_full[0], 1);
-    tc::mbar_init(&bar.o_full[1], 1);
+    for (int g2 = 0; g2 < 2; ++g2) {
+      tc::mbar_init(&bar.s_full[g2], 1);
+      tc::mbar_init(&bar.p_ready[g2], 128);
+      tc::mbar_init(&bar.o_full[g2], 1);
+    }
     tc::mbar_init(&bar.done, 1);
+    tc::mbar_init(&bar.recv_full, 1);
     tc::fence_mbar_init();
+    if (p.n_splits > 1) {
+      // every other split pushes each row this CTA owns; nothing can arrive before the cluster barrier that
+      // follows every CTA's main loop, long after this
+      const int LR = (128 + p.n_splits - 1) / p.n_splits;
+      const int n_loc = max(0, min(128, (split + 1) * LR) - split * LR);
+      tc::mbar_arrive_expect_tx(&bar.recv_full, (uint32_t)((p.n_splits - 1) * n_loc * kRecvRowBytes));
+    }
   }
   if (warp == 1) tc::tmem_alloc(&bar.tmem_base, 512);
   __syncthreads();
   volatile int* abort_flag = &bar.abort_flag;
-  const uint32_t tS = bar.tmem_base;          // S buffers at columns [0,128) and [128,256)
-  const uint32_t tO = bar.tmem_base + 256;    // O tiles at columns [256,384) and [384,512)
+  const uint32_t tS = bar.tmem_base;          // S buffers (group 0, group 1) at columns [0,128) and [128,256)
+  const uint32_t tO = bar.tmem_base + 256;    // O_0, O_1 at columns [256,384) and [384,512)
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
@@ -241,7 +339,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     if (tc::elect_one()) {
       const uint32_t idesc_s = tc::idesc_bf16_f32(128, 128);                  // A, B K-major
       const uint32_t idesc_o = tc::idesc_bf16_f32(128, 128) | (1u << 16);     // B MN-major
-      const uint32_t aQ = tc::smem_u32(sQ), aP = tc::smem_u32(sP);
+      const uint32_t aQ = tc::smem_u32(sQ);
       bool ok = ntile > 0 && wait_bar(&bar.q_full, 0, abort_flag, p.status, ST_TIMEOUT_MMA);
       auto issue_s = [&](int j) -> bool {
         const int s = j % STAGES;
@@ -258,216 +356,277 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         return true;
       };
       if (ok) ok = issue_s(0);
+      if (ok && ntile > 1) ok = issue_s(1);
       for (int j = 0; j < ntile && ok; ++j) {
-        if (j + 1 < ntile && !issue_s(j + 1)) { ok = false; break; }
-        // P_j written (and O tile of j-1 read) by the softmax warps
-        if (!wait_bar(&bar.p_ready, j & 1, abort_flag, p.status, ST_TIMEOUT_MMA)) { ok = false; break; }
+        const int g = j & 1;
+        // P_j written over S_j in group g's buffer (and O_g rescaled if needed)
+        if (!wait_bar(&bar.p_ready[g], (j >> 1) & 1, abort_flag, p.status, ST_TIMEOUT_MMA)) { ok = false; break; }
         tc::fence_after_sync();
         const int s = j % STAGES;
         const uint32_t aV = tc::smem_u32(sV + s * TILE);
-        const uint32_t aPj = aP + (j & 1) * TILE;
-        const uint32_t tOj = tO + (j & 1) * 128;
+        const uint32_t tP = tS + g * 128;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t offp = (kk >> 2) * CHUNK + (kk & 3) * 32;
-          tc::mma_bf16(tOj, tc::sdesc_k128(aPj + offp), sdesc_mn128(aV + kk * 2048, CHUNK), idesc_o, kk != 0);
-        }
-        tc::mma_commit(&bar.o_full[j & 1]);
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_tmem_a(tO + g * 128, tP + kk * 8, sdesc_mn128(aV + kk * 2048, CHUNK), idesc_o,
+                          (j >= 2 || kk != 0) ? 1u : 0u);
+        tc::mma_commit(&bar.o_full[g]);
         tc::mma_commit(&bar.kv_empty[s]);
+        // S_{j+2} reuses group g's buffer: the tcgen05 MMAs of this thread execute in issue order, so it cannot
+        // overwrite P_j before P_j V_j has read it
+        if (j + 2 < ntile && !issue_s(j + 2)) { ok = false; break; }
       }
       tc::mma_commit(&bar.done);
       tc::mbar_wait(&bar.done, 0, 1u << 20);
     }
-  } else {
-    // ------------------------------------------------------------------ softmax / output warps 2..9
-    // Two threads per query row (TMEM lane): warp w in 2..5 takes keys / output columns [0, 64), warp w + 4 takes
-    // [64, 128). The half-row maxima are exchanged through shared memory once per tile.
-    const int q4 = warp & 3;
-    const int row = q4 * 32 + lane;      // TMEM lane = tile row
-    const int half = (warp - 2) >> 2;    // 0: columns [0, 64), 1: [64, 128)
-    const int etid = tid - 64;           // 0..255
-    const int qi = row / p.G, hh = row % p.G;
+  }
+
+  // ------------------------------------------------------------------ softmax / output warps 2..9
+  // Group grp = 0 (warps 2..5) takes the split's tiles 0, 2, 4, ..., group 1 (warps 6..9) tiles 1, 3, 5, ...; in a
+  // group, one thread per query row (TMEM lane). At the end every thread of either group combines O_0 and O_1 for
+  // its row over output columns [64 grp, 64 grp + 64).
+  const int q4 = warp & 3;
+  const int row = q4 * 32 + lane;      // TMEM lane = tile row
+  const int grp = (warp - 2) >> 2;
+  const int gtid = ((warp - 2) & 3) * 32 + lane;   // 0..127 within the group
+  const int etid = tid - 64;           // 0..255
+  const int col0 = 64 * grp;
+  const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+  float o[64];
+  float m_ref = -INFINITY, l_row = 0.f;
+  if (warp >= 2) {
+    const int qi = row / p.G;
     const int qg = q0 + qi;              // query index in the row
-    const bool row_ok = qg < p.Lq;
     const int qblk_min = (p.q_pos0 + q0) / p.blk_len;  // rows of the tile past Lq never write output
     const int qrel = (p.q_pos0 + qg) / p.blk_len - qblk_min;
-    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-    const int col0 = 64 * half;
-    float o[64];
-#pragma unroll
-    for (int c = 0; c < 64; ++c) o[c] = 0.f;
-    float m = -INFINITY, l = 0.f;
+    const uint64_t scale2 = pk2(p.scale_log2, p.scale_log2);
+    const uint32_t tSg = tS + grp * 128 + lane_off;
+    const uint32_t tOg = tO + grp * 128 + lane_off;
+    const int n_my = ntile > grp ? (ntile - grp + 1) / 2 : 0;
+    float mg = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < ntile && ok; ++j) {
-      const int jt = t_begin + j;
+    // A failed wait marks this thread (and the shared abort flag); the group's 128 threads leave the loop
+    // together at the next tile-start barrier, so no named barrier is left waiting for threads that have gone.
+    for (int i = 0; i < n_my; ++i) {
+      const int jt = t_begin + grp + 2 * i;
       // block index of every key of this tile, and whether the whole tile is visible to the whole query tile
-      if (etid < 128) {
-        const int key = jt * KT + etid;
+      {
+        const int key = jt * KT + gtid;
         int rel = kNoKey;
         if (key < n_keys_eff) {
-          const int kb = (p.key_pos ? p.key_pos[(int64_t)b * p.n_keys + key] : key) / p.blk_len;
+          const int kb = div_blk(p.key_pos ? p.key_pos[(int64_t)b * p.n_keys + key] : key, p.blk_magic, p.blk_shift);
           rel = max(-32768, min(32766, kb - qblk_min));   // the queries' relative blocks lie in [0, 128]
         }
-        bar.kblk[j & 1][etid] = (short)rel;
+        bar.kblk[grp][i & 1][gtid] = (short)rel;
         const unsigned bal = __ballot_sync(0xffffffffu, rel <= 0);
-        if (lane == 0) bar.vis_w[j & 1][etid >> 5] = bal;
+        if (lane == 0) bar.vis_w[grp][i & 1][gtid >> 5] = bal;
       }
-      tc::named_bar_sync(1, 256);
-      const bool fast = (bar.vis_w[j & 1][0] & bar.vis_w[j & 1][1] & bar.vis_w[j & 1][2] & bar.vis_w[j & 1][3]) ==
-                        0xffffffffu;
-      if (!wait_bar(&bar.s_full[j & 1], (j >> 1) & 1, abort_flag, p.status, ST_TIMEOUT_EPILOGUE)) { ok = false; break; }
+      if (bar_sync_or(1 + grp, 128, !ok || *abort_flag)) { ok = false; break; }
+      const unsigned* vw = bar.vis_w[grp][i & 1];
+      const bool fast = (vw[0] & vw[1] & vw[2] & vw[3]) == 0xffffffffu;
+      const short* kbt = bar.kblk[grp][i & 1];
+      if (!wait_bar(&bar.s_full[grp], i & 1, abort_flag, p.status, ST_TIMEOUT_EPILOGUE)) ok = false;
       tc::fence_after_sync();
-      const uint32_t sbase = tS + (j & 1) * 128 + col0 + lane_off;
-      const short* kbt = bar.kblk[j & 1] + col0;
-      float v[64];
-      tmem_ld64(sbase, v);
-      // pass 1: half-row maximum of the visible scores, exchanged with the partner thread
+      // row maximum of the visible scores
       float mt = -INFINITY;
-      if (fast) {
 #pragma unroll
-        for (int u = 0; u < 64; ++u) mt = fmaxf(mt, v[u]);
-      } else {
+      for (int c = 0; c < 2; ++c) {
+        float v[64];
+        tmem_ld64(tSg + 64 * c, v);
+        if (fast) {
 #pragma unroll
-        for (int u = 0; u < 64; ++u)
-          if (kbt[u] <= qrel) mt = fmaxf(mt, v[u]);
+          for (int u = 0; u < 64; ++u) mt = fmaxf(mt, v[u]);
+        } else {
+#pragma unroll
+          for (int u = 0; u < 64; ++u)
+            if (kbt[64 * c + u] <= qrel) mt = fmaxf(mt, v[u]);
+        }
       }
-      bar.rowmax[half][row] = mt;
-      tc::named_bar_sync(2, 256);
-      mt = fmaxf(bar.rowmax[0][row], bar.rowmax[1][row]) * p.scale_log2;
-      const float m_new = fmaxf(m, mt);
-      const float alpha = (m_new == -INFINITY) ? 1.f : exp2f(m - m_new);
-      // pass 2: P = exp2(s - m_new) as bf16 into this half's chunk of the tile's swizzled K-major P buffer
-      uint8_t* sPj = sP + (j & 1) * TILE + half * CHUNK;
-      float rs = 0.f;
+      mt *= p.scale_log2;
+      // the reference maximum moves only when this tile's maximum exceeds it by more than 2^8
+      float alpha = 1.f;
+      if (mt > mg + kRescaleLog2) {
+        alpha = (mg == -INFINITY) ? 1.f : ex2(mg - mt);
+        mg = mt;
+      }
+      // P = 2^(s * scale - mg) as bf16 pairs, 64 keys at a time, written over the S columns already read; the
+      // row sum adds the fp32 values (the bf16 rounding of P is unbiased and below 2^-9 per term)
+      uint64_t rs2 = pk2(0.f, 0.f);
+      const uint64_t negm2 = pk2(-mg, -mg);
+      const bool any = mg != -INFINITY;
 #pragma unroll
-      for (int u8 = 0; u8 < 8; ++u8) {
-        uint32_t packed[4];
+      for (int c = 0; c < 2; ++c) {
+        float v[64];
+        tmem_ld64(tSg + 64 * c, v);
+        uint32_t pk[32];
+        if (fast) {     // every key visible: the tile maximum is finite, so mg is too
 #pragma unroll
-        for (int h2 = 0; h2 < 4; ++h2) {
-          float pv[2];
-#pragma unroll
-          for (int e2 = 0; e2 < 2; ++e2) {
-            const int c = u8 * 8 + h2 * 2 + e2;
-            const bool vis = (fast || kbt[c] <= qrel) && m_new != -INFINITY;
-            pv[e2] = vis ? exp2f(v[c] * p.scale_log2 - m_new) : 0.f;
+          for (int c2 = 0; c2 < 32; ++c2) {
+            float x0, x1;
+            upk2(fma2(pk2(v[2 * c2], v[2 * c2 + 1]), scale2, negm2), x0, x1);
+            const float e0 = ex2(x0), e1 = ex2(x1);
+            __nv_bfloat162 pr = __floats2bfloat162_rn(e0, e1);
+            pk[c2] = *reinterpret_cast<uint32_t*>(&pr);
+            rs2 = add2(rs2, pk2(e0, e1));
           }
-          __nv_bfloat162 pr = __floats2bfloat162_rn(pv[0], pv[1]);
-          rs += __bfloat162float(pr.x) + __bfloat162float(pr.y);
-          packed[h2] = *reinterpret_cast<uint32_t*>(&pr);
+        } else {
+#pragma unroll
+          for (int c2 = 0; c2 < 32; ++c2) {
+            float x0, x1;
+            upk2(fma2(pk2(v[2 * c2], v[2 * c2 + 1]), scale2, negm2), x0, x1);
+            float e0 = ex2(x0), e1 = ex2(x1);
+            if (!any || !(kbt[64 * c + 2 * c2] <= qrel)) e0 = 0.f;
+            if (!any || !(kbt[64 * c + 2 * c2 + 1] <= qrel)) e1 = 0.f;
+            __nv_bfloat162 pr = __floats2bfloat162_rn(e0, e1);
+            pk[c2] = *reinterpret_cast<uint32_t*>(&pr);
+            rs2 = add2(rs2, pk2(e0, e1));
+          }
         }
-        uint8_t* dst = sPj + row * 128 + ((u8 ^ (row & 7)) << 4);
-        *reinterpret_cast<uint4*>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        // keys [64c, 64c + 64) -> columns [32c, 32c + 32): S there has been read (c = 0: this chunk's first half;
+        // c = 1: chunk 0)
+        tmem_st32(tSg + 32 * c, pk);
       }
-      fence_proxy_async_smem();
+      // O_g holds the group's previous P V once that phase completes (every phase is waited in order, so the
+      // parity is unambiguous: the next phase needs this group's P)
+      if (i > 0 && !wait_bar(&bar.o_full[grp], (i - 1) & 1, abort_flag, p.status, ST_TIMEOUT_EPILOGUE)) ok = false;
+      if (__any_sync(0xffffffffu, alpha != 1.f)) {
+        tc::fence_after_sync();
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          float w[32];
+          tmem_ld32(tOg + 32 * c, w);
+          uint32_t r32[32];
+#pragma unroll
+          for (int u = 0; u < 32; ++u) r32[u] = __float_as_uint(w[u] * alpha);
+          tmem_st32(tOg + 32 * c, r32);
+        }
+      }
+      float rs0, rs1;
+      upk2(rs2, rs0, rs1);
+      l = l * alpha + (rs0 + rs1);
+      tmem_st_wait();
       tc::fence_before_sync();
-      tc::mbar_arrive(&bar.p_ready);
-      // fold in the previous tile's P V (previous max's scale), then move to this tile's scale
-      if (j > 0) {
-        if (!wait_bar(&bar.o_full[(j - 1) & 1], ((j - 1) >> 1) & 1, abort_flag, p.status, ST_TIMEOUT_EPILOGUE)) {
-          ok = false;
-          break;
-        }
-        tc::fence_after_sync();
-        float w[64];
-        tmem_ld64(tO + ((j - 1) & 1) * 128 + col0 + lane_off, w);
-#pragma unroll
-        for (int u = 0; u < 64; ++u) o[u] += w[u];
-      }
-#pragma unroll
-      for (int c = 0; c < 64; ++c) o[c] *= alpha;
-      l = l * alpha + rs;          // this half's share of the row sum
-      m = m_new;
+      tc::mbar_arrive(&bar.p_ready[grp]);
     }
-    if (ok && ntile > 0) {
-      const int jl = ntile - 1;
-      if (wait_bar(&bar.o_full[jl & 1], (jl >> 1) & 1, abort_flag, p.status, ST_TIMEOUT_EPILOGUE)) {
+    bool fin = ok && n_my > 0;
+    if (fin) fin = wait_bar(&bar.o_full[grp], (n_my - 1) & 1, abort_flag, p.status, ST_TIMEOUT_EPILOGUE);
+    // combine the groups: (m, l) through the K ring, idle once both groups' last P V have completed (every S
+    // product was issued before one of them), O_0 and O_1 straight from TMEM
+    tc::named_bar_sync(kBarAll, 256);
+    float2* xch = reinterpret_cast<float2*>(sK);      // [group][row]
+    xch[grp * 128 + row] = make_float2(fin ? mg : -INFINITY, fin ? l : 0.f);
+    tc::named_bar_sync(kBarAll, 256);
+    const float2 ma = xch[row], mb = xch[128 + row];
+    const float M = fmaxf(ma.x, mb.x);
+    const float wa = ma.x == -INFINITY ? 0.f : ex2(ma.x - M), wb = mb.x == -INFINITY ? 0.f : ex2(mb.x - M);
+    l_row = wa * ma.y + wb * mb.y;
+    m_ref = M;
+#pragma unroll
+    for (int u = 0; u < 64; ++u) o[u] = 0.f;
+#pragma unroll
+    for (int g2 = 0; g2 < 2; ++g2) {
+      const float w = g2 == 0 ? wa : wb;
+      if (__any_sync(0xffffffffu, w != 0.f)) {       // tcgen05.ld is warp-wide
         tc::fence_after_sync();
-        float w[64];
-        tmem_ld64(tO + (jl & 1) * 128 + col0 + lane_off, w);
+        float x[64];
+        tmem_ld64(tO + g2 * 128 + col0 + lane_off, x);
+        if (w != 0.f) {
 #pragma unroll
-        for (int u = 0; u < 64; ++u) o[u] += w[u];
-      }
-    }
-    // row sums: the two halves' shares
-    float* lsum = &bar.rowmax[0][0];             // reused: [2][128]
-    tc::named_bar_sync(1, 256);
-    lsum[half * 128 + row] = l;
-    tc::named_bar_sync(1, 256);
-    const float l_row = lsum[row] + lsum[128 + row];
-    if (p.n_splits == 1) {
-      if (row_ok && !*abort_flag) {
-        const int64_t qh = ((int64_t)b * p.Lq + qg) * p.Hq + g * p.G + hh;
-        const float inv = l_row > 0.f ? 1.0f / l_row : 0.f;
-        uint4* dst = reinterpret_cast<uint4*>(p.out + qh * 128 + col0);
-#pragma unroll
-        for (int c = 0; c < 64; c += 8) {
-          __nv_bfloat162 a0 = __floats2bfloat162_rn(o[c] * inv, o[c + 1] * inv);
-          __nv_bfloat162 a1 = __floats2bfloat162_rn(o[c + 2] * inv, o[c + 3] * inv);
-          __nv_bfloat162 a2 = __floats2bfloat162_rn(o[c + 4] * inv, o[c + 5] * inv);
-          __nv_bfloat162 a3 = __floats2bfloat162_rn(o[c + 6] * inv, o[c + 7] * inv);
-          dst[c >> 3] = make_uint4(*reinterpret_cast<uint32_t*>(&a0), *reinterpret_cast<uint32_t*>(&a1),
-                                   *reinterpret_cast<uint32_t*>(&a2), *reinterpret_cast<uint32_t*>(&a3));
+          for (int u = 0; u < 64; ++u) o[u] = fmaf(w, x[u], o[u]);
         }
       }
-    } else {
-      // this split's unnormalised row (log2-domain max; an empty split leaves (-inf, 0)) into the idle K/V ring:
-      // o at [row][128] with the 16-byte units rotated by the row to spread banks, then m and l
-      float* so = reinterpret_cast<float*>(sK);
-      float4* orow = reinterpret_cast<float4*>(so + row * 128);
+    }
+    tc::fence_before_sync();
+    // the exchange has been read by every consumer thread before the ring can receive other splits' rows
+    tc::named_bar_sync(kBarAll, 256);
+    if (p.n_splits > 1) {
+      fence_proxy_async_smem();
+      cluster_arrive();
+    }
+    if (p.n_splits == 1 && qg < p.Lq && !*abort_flag) {
+      const int64_t qh = ((int64_t)b * p.Lq + qg) * p.Hq + g * p.G + row % p.G;
+      const float inv = l_row > 0.f ? 1.0f / l_row : 0.f;
+      uint4* dst = reinterpret_cast<uint4*>(p.out + qh * 128 + col0);
 #pragma unroll
-      for (int c = 0; c < 64; c += 4)
-        orow[(((col0 + c) >> 2) + row) & 31] = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
-      if (half == 0) {
-        so[128 * 128 + row] = m;
-        so[128 * 128 + 128 + row] = l_row;
+      for (int c = 0; c < 64; c += 8) {
+        __nv_bfloat162 a0 = __floats2bfloat162_rn(o[c] * inv, o[c + 1] * inv);
+        __nv_bfloat162 a1 = __floats2bfloat162_rn(o[c + 2] * inv, o[c + 3] * inv);
+        __nv_bfloat162 a2 = __floats2bfloat162_rn(o[c + 4] * inv, o[c + 5] * inv);
+        __nv_bfloat162 a3 = __floats2bfloat162_rn(o[c + 6] * inv, o[c + 7] * inv);
+        dst[c >> 3] = make_uint4(*reinterpret_cast<uint32_t*>(&a0), *reinterpret_cast<uint32_t*>(&a1),
+                                 *reinterpret_cast<uint32_t*>(&a2), *reinterpret_cast<uint32_t*>(&a3));
       }
     }
   }
   if (p.n_splits > 1) {
-    // merge the splits of this tile: rank r owns rows [r*128/ns, (r+1)*128/ns); it reads every split's (o, m, l)
-    // of its rows through distributed shared memory, in rank order
-    __syncthreads();
-    cluster_sync();
-    if (warp >= 2 && !*abort_flag) {
-      const int ns = p.n_splits;
-      const int r0 = split * 128 / ns, r1 = (split + 1) * 128 / ns;
-      const float* so = reinterpret_cast<const float*>(sK);
-      const int etid = tid - 64;
+    // merge the splits of this query tile. Rank r owns rows [r*LR, (r+1)*LR). Every split pushes its
+    // unnormalised rows (o relative to its m_ref, and l) into the owner's idle K/V ring at [split][local row]
+    // with asynchronous stores counted on the owner's recv_full barrier; each owner waits for its bytes and
+    // merges its rows from its own shared memory, in split order.
+    const int ns = p.n_splits;
+    const int LR = (128 + ns - 1) / ns;
+    float* recv = reinterpret_cast<float*>(sK);
+    if (warp < 2) {
+      fence_proxy_async_smem();
+      cluster_arrive();        // warps 0 and 1 are done with the ring once their roles have returned
+    }
+    cluster_wait();
+    if (warp >= 2) {
+      const int owner = row / LR, local = row - owner * LR;
+      float* slot = recv + ((size_t)split * LR + local) * kRecvStride;
+      if (owner == split) {
+        // this CTA's own rows stay local
+#pragma unroll
+        for (int c = 0; c < 64; c += 4)
+          *reinterpret_cast<float4*>(slot + col0 + c) = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
+        if (grp == 0) *reinterpret_cast<float2*>(slot + 128) = make_float2(m_ref, l_row);
+      } else {
+        const uint32_t dst = dsmem_addr(slot, (uint32_t)owner);
+        const uint32_t rbar = dsmem_addr(&bar.recv_full, (uint32_t)owner);
+#pragma unroll
+        for (int c = 0; c < 64; c += 4)
+          st_async4(dst + (uint32_t)(col0 + c) * 4u, o[c], o[c + 1], o[c + 2], o[c + 3], rbar);
+        if (grp == 0) st_async2(dst + 128u * 4u, m_ref, l_row, rbar);
+      }
+      // rows this CTA owns: the other splits' bytes, and this split's local writes
+      const bool got = wait_bar(&bar.recv_full, 0, abort_flag, p.status, ST_TIMEOUT_EPILOGUE);
+      tc::named_bar_sync(kBarAll, 256);
+      const int r0 = split * LR, n_loc = min(128, r0 + LR) - r0;
       const int d4 = etid & 31;               // this thread's 4 output columns
-      for (int rr = r0 + (etid >> 5); rr < r1; rr += 8) {
-        const int qi = rr / p.G, hh2 = rr % p.G, qg = q0 + qi;
-        float ms[8];
+      for (int lr = etid >> 5; got && lr < n_loc; lr += 8) {
+        const int rr = r0 + lr;
+        float ms[8], ls[8];
+        float4 vs[8];
         float M = -INFINITY;
 #pragma unroll
         for (int sp = 0; sp < 8; ++sp) {
-          ms[sp] = sp < ns ? ld_dsmem(so + 128 * 128 + rr, (uint32_t)sp) : -INFINITY;
+          const float* rp = recv + ((size_t)sp * LR + lr) * kRecvStride;
+          ms[sp] = sp < ns ? rp[128] : -INFINITY;
+          ls[sp] = sp < ns ? rp[129] : 0.f;
+          vs[sp] = sp < ns ? *reinterpret_cast<const float4*>(rp + d4 * 4) : make_float4(0.f, 0.f, 0.f, 0.f);
           M = fmaxf(M, ms[sp]);
         }
         float L = 0.f;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int sp = 0; sp < 8; ++sp) {
-          const float w = (sp < ns && ms[sp] != -INFINITY) ? exp2f(ms[sp] - M) : 0.f;
-          if (w != 0.f) {
-            L += w * ld_dsmem(so + 128 * 128 + 128 + rr, (uint32_t)sp);
-            const float4 v4 = ld_dsmem4(so + rr * 128 + (((d4 + rr) & 31) << 2), (uint32_t)sp);
-            acc.x += w * v4.x;
-            acc.y += w * v4.y;
-            acc.z += w * v4.z;
-            acc.w += w * v4.w;
-          }
+          const float w = ms[sp] == -INFINITY ? 0.f : ex2(ms[sp] - M);
+          L += w * ls[sp];
+          acc.x += w * vs[sp].x;
+          acc.y += w * vs[sp].y;
+          acc.z += w * vs[sp].z;
+          acc.w += w * vs[sp].w;
         }
-        if (qg < p.Lq) {
+        const int qg2 = q0 + rr / p.G, hh2 = rr % p.G;
+        if (qg2 < p.Lq && !*abort_flag) {
           const float inv = L > 0.f ? 1.0f / L : 0.f;
-          const int64_t qh = ((int64_t)b * p.Lq + qg) * p.Hq + g * p.G + hh2;
+          const int64_t qh = ((int64_t)b * p.Lq + qg2) * p.Hq + g * p.G + hh2;
           __nv_bfloat162 a0 = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
           __nv_bfloat162 a1 = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
-          uint2* dst = reinterpret_cast<uint2*>(p.out + qh * 128 + d4 * 4);
-          *dst = make_uint2(*reinterpret_cast<uint32_t*>(&a0), *reinterpret_cast<uint32_t*>(&a1));
+          uint2* dstp = reinterpret_cast<uint2*>(p.out + qh * 128 + d4 * 4);
+          *dstp = make_uint2(*reinterpret_cast<uint32_t*>(&a0), *reinterpret_cast<uint32_t*>(&a1));
         }
       }
     }
-    cluster_sync();
   }
   __syncthreads();
   if (warp == 1) {
@@ -517,7 +676,9 @@ void plan_tc(int B, int Lq, int Hq, int Hkv, int n_keys, int& QT, int& n_qtiles,
   n_qtiles = (Lq + QT - 1) / QT;
   const int tiles = (n_keys + KT - 1) / KT;
   const int base = B * Hkv * n_qtiles;
-  int want = (3 * num_sms() / 2 + base - 1) / base;
+  // key splits fill at most one wave of the GPU (one CTA per SM): a second wave would repeat every split's
+  // fixed cost (setup, first loads, merge) for a sliver of the keys
+  const int want = num_sms() / base;
   n_splits = max(1, min(min(want, tiles), 8));
   tps = (tiles + n_splits - 1) / n_splits;
   n_splits = max(1, (tiles + tps - 1) / tps);
@@ -539,6 +700,12 @@ int launch_attn_tc(const AttnArgs& a, int32_t* status, cudaStream_t s) {
   AttnTcParams p;
   p.B = a.B; p.Lq = a.Lq; p.Hq = a.Hq; p.Hkv = a.Hkv; p.G = a.Hq / a.Hkv; p.n_keys = a.n_keys; p.cap = a.cap;
   p.blk_len = a.blk_len; p.q_pos0 = a.q_pos0;
+  {
+    uint32_t sh = 0;
+    while ((1u << sh) < (uint32_t)a.blk_len) ++sh;                     // 2^(sh-1) < blk_len <= 2^sh
+    p.blk_magic = (uint32_t)((((uint64_t)1 << (31 + sh)) + (uint64_t)a.blk_len - 1) / (uint64_t)a.blk_len);
+    p.blk_shift = 31 + sh;
+  }
   plan_tc(a.B, a.Lq, a.Hq, a.Hkv, a.n_keys, p.QT, p.n_qtiles, p.n_splits, p.tiles_per_split);
   const float scale = a.scale > 0.f ? a.scale : 1.0f / sqrtf((float)a.d);
   p.scale_log2 = scale * 1.4426950408889634f;

@@ -138,10 +138,36 @@ __global__ void __launch_bounds__(256) unmask_reduce_kernel(const T* __restrict_
   }
 }
 
+// Packed fp32 pairs (the sm_100 f32x2 instructions: one issue for two lanes' worth of add or multiply) and the
+// hardware base-2 exponential (ex2.approx.ftz: relative error about 2^-22, results below 2^-126 flushed to 0, which
+// against a maximum term of 1 is far below fp32 resolution).
+DLLM_DEV uint64_t pk2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+DLLM_DEV void upk2(uint64_t v, float& lo, float& hi) { asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v)); }
+DLLM_DEV uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+DLLM_DEV uint64_t mul2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+DLLM_DEV float ex2(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
 // bf16 logits without guidance: each thread keeps its VPT 16-byte vectors of the chunk in registers. Pass 1 finds
 // the maximum with packed bf16x2 max (and the first vector holding it); pass 2 sums exp(z - max) as
-// ex2((z - max) * log2(e)) in fp32 (z - max is exact near the maximum), accumulated per thread in fp32 over at most
-// VPT * 8 terms and then in fp64; the lowest arg-max comes from the first vector that holds the maximum.
+// 2^((z - max) * log2(e)) with the subtraction and the scaling done on fp32 pairs (z - max is exact near the
+// maximum), accumulated per thread in fp32 over at most VPT * 8 terms and then in fp64; the lowest arg-max comes
+// from the first vector that holds the maximum, re-read (from L2) before pass 2 so that its latency hides behind it.
 template <int VPT>
 __global__ void __launch_bounds__(256) unmask_reduce_bf16_kernel(const __nv_bfloat16* __restrict__ logits,
                                                                  const int32_t* __restrict__ n_rows, int V, int chunk,
@@ -169,20 +195,25 @@ __global__ void __launch_bounds__(256) unmask_reduce_bf16_kernel(const __nv_bflo
   }
   Partial p{-INFINITY, 0x7fffffff, 0.0};
   if (best >= 0) {
-    // pass 2: sum of exponentials relative to the thread's maximum
+    const uint4 bv = ld_nc_v4(z + v0 + (threadIdx.x + best * 256) * 8);
+    // pass 2: sum of exponentials relative to the thread's maximum, two terms per packed operation
     const float log2e = 1.4426950408889634f;
-    float acc = 0.f;
+    const uint64_t negm2 = pk2(-m, -m), log2e2 = pk2(log2e, log2e);
+    uint64_t acc2 = pk2(0.f, 0.f);
 #pragma unroll
     for (int k = 0; k < VPT; ++k) {
       const uint32_t w[4] = {u[k].x, u[k].y, u[k].z, u[k].w};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const float lo = __uint_as_float(w[q] << 16), hi = __uint_as_float(w[q] & 0xffff0000u);
-        acc += exp2f((lo - m) * log2e) + exp2f((hi - m) * log2e);
+        const uint64_t zz = pk2(__uint_as_float(w[q] << 16), __uint_as_float(w[q] & 0xffff0000u));
+        float e0, e1;
+        upk2(mul2(add2(zz, negm2), log2e2), e0, e1);
+        acc2 = add2(acc2, pk2(ex2(e0), ex2(e1)));
       }
     }
+    float a0, a1;
+    upk2(acc2, a0, a1);
     // lowest index attaining m inside the first vector that holds it
-    const uint4 bv = ld_nc_v4(z + v0 + (threadIdx.x + best * 256) * 8);
     float f[8];
     bf16x8_to_f32(bv, f);
     int e = 7;
@@ -191,7 +222,7 @@ __global__ void __launch_bounds__(256) unmask_reduce_bf16_kernel(const __nv_bflo
       if (f[q] == m) e = q;
     p.m = m;
     p.idx = v0 + (threadIdx.x + best * 256) * 8 + e;
-    p.s = (double)acc;
+    p.s = (double)a0 + (double)a1;
   }
   // scalar tail of the chunk (chunk lengths are multiples of 8 except the row's last chunk)
   for (int v = v0 + nvec * 8 + threadIdx.x; v < v1; v += 256) {

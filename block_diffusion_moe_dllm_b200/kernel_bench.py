@@ -27,6 +27,20 @@ def hbm_peak():
     return 6650.0, "fallback"
 
 
+def tensor_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        return json.load(open(p))["bf16_tflops"], "measured"
+    return 1590.0, "fallback"
+
+
+def _flops(extra, flops, t):
+    peak, src = tensor_peak()
+    extra.update({"TFLOP/s": flops / t / 1e12, "frac_tensor": flops / t / 1e12 / peak, "tensor_peak": peak,
+                  "tensor_peak_source": src})
+    return extra
+
+
 def timed(fn, reps, stream=None, warm=3):
     """GPU time of one call: `reps` calls captured in a CUDA graph, the replay timed with CUDA events (host-side
     launch cost excluded)."""
@@ -66,7 +80,8 @@ def bench_lm_head(w: Workload, reps, dev, stream, weights=None):
     ws = bd.Workspace(1 << 16, dev)
     t = timed(lambda: bd.gemm(x, wl, y, rows, w.vlen, w.H, bd.BF16, ws=ws), reps, stream)
     nbytes = w.vlen * w.H * 2 + rows * w.H * 2 + rows * w.vlen * 2
-    return _result("gemm_tc_kernel[lm_head]", t, nbytes, {"rows": rows, "M": w.vlen, "K": w.H})
+    return _result("gemm_tc_kernel[lm_head]", t, nbytes,
+                   _flops({"rows": rows, "M": w.vlen, "K": w.H}, 2.0 * rows * w.vlen * w.H, t))
 
 
 def bench_proj(w: Workload, reps, dev, stream, weights=None):
@@ -82,7 +97,8 @@ def bench_proj(w: Workload, reps, dev, stream, weights=None):
         ws = bd.Workspace(64 << 20, dev)
         t = timed(lambda: bd.gemm(x, wt, y, rows, M, K, bd.BF16, ws=ws), reps, stream)
         nbytes = M * K * 2 + rows * K * 2 + rows * M * 2
-        out.append(_result(f"gemm_tc_kernel[{name}]", t, nbytes, {"rows": rows, "M": M, "K": K}))
+        out.append(_result(f"gemm_tc_kernel[{name}]", t, nbytes,
+                           _flops({"rows": rows, "M": M, "K": K}, 2.0 * rows * M * K, t)))
     return out
 
 
@@ -110,7 +126,9 @@ def bench_experts(w: Workload, reps, dev, stream, weights=None):
     troute = timed(lambda: bd.moe_route(h, lw["w_router"], lw["router_bias"], ids, gates, counts, offsets, perm, inv,
                                         rows, w.H, w.E, w.k, bd.BF16, ws=ws), reps, stream)
     rbytes = w.E * w.H * 2 + rows * w.H * 2
-    return [_result("moe_experts[gather+gemm_tc x2+combine]", t, nbytes, {"active_experts": active, "rows": rows}),
+    flops = 6.0 * w.H * w.I * (w.k + 1) * rows
+    return [_result("moe_experts[gather+gemm_tc x2+combine]", t, nbytes,
+                    _flops({"active_experts": active, "rows": rows}, flops, t)),
             _result("moe_route[scores+topk+permute]", troute, rbytes, {"rows": rows})]
 
 
@@ -151,7 +169,7 @@ def bench_attn(w: Workload, reps, dev, stream):
                                     ws=ws), reps, stream)
     nbytes = 2 * w.B * w.Hkv * n_keys * w.d * 2 + 2 * w.B * w.L * w.Hq * w.d * 2
     flops = 4.0 * w.B * w.L * w.Hq * n_keys * w.d
-    return _result("block_attn", t, nbytes, {"keys": n_keys, "TFLOP/s": flops / t / 1e12})
+    return _result("block_attn", t, nbytes, _flops({"keys": n_keys, "rows": w.B * w.L}, flops, t))
 
 
 def main():

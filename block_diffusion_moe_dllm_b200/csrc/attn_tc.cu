@@ -40,13 +40,11 @@ constexpr float kRescaleLog2 = 8.f;
 // named barriers: 1 + g = softmax group g's 128 threads inside its loop; kBarAll = all 256 softmax threads after
 // the loops (distinct ids, since one group can leave its loop while the other still synchronises inside its own)
 constexpr int kBarAll = 3;         // O and the row sum are rescaled when the maximum grows by > 2^8
-constexpr int kRecvStride = 132;            // floats per pushed row: o[128], m, l, 2 pad (16-byte multiple)
-constexpr int kRecvRowBytes = 130 * 4;      // bytes pushed per (split, row): o, m, l
+constexpr int kRecvStride = 132;            // floats per exchanged row: o[128], m, l, 2 pad (16-byte multiple)
 constexpr int SMEM = 1024 + TILE /*Q*/ + STAGES * 2 * TILE /*K,V*/ + BARS_BYTES;
 static_assert(SMEM <= 232448, "shared memory budget");
-static_assert(8 * 16 * kRecvStride * 4 <= STAGES * 2 * TILE && 7 * 19 * kRecvStride * 4 <= STAGES * 2 * TILE &&
-                  3 * 43 * kRecvStride * 4 <= STAGES * 2 * TILE,
-              "split merge buffer exceeds the K/V ring");
+static_assert((128 + 135) * kRecvStride * 4 <= STAGES * 2 * TILE,
+              "split exchange staging (own rows + n_splits * ceil(128 / n_splits) others) exceeds the K/V ring");
 
 struct Bars {
   uint64_t q_full;
@@ -56,7 +54,7 @@ struct Bars {
   uint64_t p_ready[2];  // per group: P of its tile written over S (and the group's O rescaled if needed)
   uint64_t o_full[2];   // per group: phase i completes when the group's i-th P V is accumulated into its O
   uint64_t done;
-  uint64_t recv_full;   // split merge: completes when every split's rows owned by this CTA have arrived
+  uint64_t xch_full;    // split merge: the other splits' rows of this CTA have landed in shared memory
   uint32_t tmem_base;
   int abort_flag;
   short kblk[2][2][KT];     // [group][tile parity within the group][key]: block of the key relative to the CTA's
@@ -71,6 +69,7 @@ struct AttnTcParams {
   uint32_t blk_magic, blk_shift;   // key position / blk_len = (pos * blk_magic) >> blk_shift for 0 <= pos < 2^31
   float scale_log2;
   const int32_t* key_pos;
+  float* xscratch;      // split exchange: [B*Hkv*n_qtiles][n_splits][128 rows][kRecvStride] (n_splits > 1)
   __nv_bfloat16* out;   // [B, Lq, Hq, 128]
   int32_t* status;
 };
@@ -164,31 +163,30 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-__device__ __forceinline__ uint32_t dsmem_addr(const void* local, uint32_t rank) {
-  uint32_t remote;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(tc::smem_u32(local)), "r"(rank));
-  return remote;
-}
-// Asynchronous store into another CTA's shared memory that counts its bytes on that CTA's mbarrier.
-__device__ __forceinline__ void st_async4(uint32_t remote, float a, float b, float c, float d, uint32_t remote_bar) {
-  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(
-                   remote),
-               "f"(a), "f"(b), "f"(c), "f"(d), "r"(remote_bar)
+// Bulk copies between shared and global memory (the async proxy) for the split exchange.
+__device__ __forceinline__ void bulk_store_s2g(void* gdst, const void* ssrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(tc::smem_u32(ssrc)),
+               "r"(bytes)
                : "memory");
 }
-__device__ __forceinline__ void st_async2(uint32_t remote, float a, float b, uint32_t remote_bar) {
-  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.f32 [%0], {%1, %2}, [%3];" ::"r"(remote),
-               "f"(a), "f"(b), "r"(remote_bar)
+__device__ __forceinline__ void bulk_commit_and_wait() {
+  asm volatile("cp.async.bulk.commit_group;\n\tcp.async.bulk.wait_group 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_load_g2s(void* sdst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   tc::smem_u32(sdst)),
+               "l"(gsrc), "r"(bytes), "r"(tc::smem_u32(bar))
                : "memory");
 }
+__device__ __forceinline__ void fence_proxy_async_all() {
+  asm volatile("fence.proxy.async;" ::: "memory");
+}
+
 __device__ __forceinline__ void cluster_arrive() {
   asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
 }
 __device__ __forceinline__ void cluster_wait() {
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
-}
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // Each lane reads 64 consecutive 32-bit columns of its own TMEM lane.
@@ -267,15 +265,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       tc::mbar_init(&bar.o_full[g2], 1);
     }
     tc::mbar_init(&bar.done, 1);
-    tc::mbar_init(&bar.recv_full, 1);
+    tc::mbar_init(&bar.xch_full, 1);
     tc::fence_mbar_init();
-    if (p.n_splits > 1) {
-      // every other split pushes each row this CTA owns; nothing can arrive before the cluster barrier that
-      // follows every CTA's main loop, long after this
-      const int LR = (128 + p.n_splits - 1) / p.n_splits;
-      const int n_loc = max(0, min(128, (split + 1) * LR) - split * LR);
-      tc::mbar_arrive_expect_tx(&bar.recv_full, (uint32_t)((p.n_splits - 1) * n_loc * kRecvRowBytes));
-    }
   }
   if (warp == 1) tc::tmem_alloc(&bar.tmem_base, 512);
   __syncthreads();
@@ -536,12 +527,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       }
     }
     tc::fence_before_sync();
-    // the exchange has been read by every consumer thread before the ring can receive other splits' rows
-    tc::named_bar_sync(kBarAll, 256);
-    if (p.n_splits > 1) {
-      fence_proxy_async_smem();
-      cluster_arrive();
-    }
     if (p.n_splits == 1 && qg < p.Lq && !*abort_flag) {
       const int64_t qh = ((int64_t)b * p.Lq + qg) * p.Hq + g * p.G + row % p.G;
       const float inv = l_row > 0.f ? 1.0f / l_row : 0.f;
@@ -558,72 +543,90 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
   }
   if (p.n_splits > 1) {
-    // merge the splits of this query tile. Rank r owns rows [r*LR, (r+1)*LR). Every split pushes its
-    // unnormalised rows (o relative to its m_ref, and l) into the owner's idle K/V ring at [split][local row]
-    // with asynchronous stores counted on the owner's recv_full barrier; each owner waits for its bytes and
-    // merges its rows from its own shared memory, in split order.
+    // merge the splits of this query tile through L2. Rank r owns rows [r*LR, (r+1)*LR). Every split stages the
+    // unnormalised rows (o relative to its maximum, m, l) that other ranks own in its idle K/V ring and
+    // bulk-copies them to its slab of the exchange buffer; after one cluster barrier each owner bulk-copies the
+    // other splits' copies of its rows into its ring, and the two threads of every owned row fold them into the
+    // row they hold in registers (splits in order) and write the output.
     const int ns = p.n_splits;
     const int LR = (128 + ns - 1) / ns;
-    float* recv = reinterpret_cast<float*>(sK);
-    if (warp < 2) {
-      fence_proxy_async_smem();
-      cluster_arrive();        // warps 0 and 1 are done with the ring once their roles have returned
+    const int r0 = split * LR, n_loc = max(0, min(128, r0 + LR) - r0);
+    constexpr uint32_t kRowBytes = kRecvStride * 4;
+    float* stage = reinterpret_cast<float*>(sK);                 // [128 rows][kRecvStride]: rows others own
+    float* pbuf = stage + 128 * kRecvStride;                      // [ns][LR][kRecvStride]: the others' copies
+    float* slab0 = p.xscratch + (size_t)blockIdx.y * ns * 128 * kRecvStride;
+    const bool mine = row >= r0 && row < r0 + n_loc;
+    if (warp >= 2) {
+      tc::named_bar_sync(kBarAll, 256);              // every consumer has read the group exchange in the ring
+      if (!mine) {
+        float* srow = stage + (size_t)row * kRecvStride;
+#pragma unroll
+        for (int c = 0; c < 64; c += 4)
+          *reinterpret_cast<float4*>(srow + col0 + c) = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
+        if (grp == 0) *reinterpret_cast<float2*>(srow + 128) = make_float2(m_ref, l_row);
+      }
+      fence_proxy_async_all();                       // the staged rows are read by the bulk copy (async proxy)
+      tc::named_bar_sync(kBarAll, 256);
+      if (etid == 0) {
+        // rows [0, r0) and [r0 + n_loc, 128) to this split's slab
+        float* slab = slab0 + (size_t)split * 128 * kRecvStride;
+        if (r0 > 0) bulk_store_s2g(slab, stage, (uint32_t)r0 * kRowBytes);
+        if (r0 + n_loc < 128)
+          bulk_store_s2g(slab + (size_t)(r0 + n_loc) * kRecvStride, stage + (size_t)(r0 + n_loc) * kRecvStride,
+                         (uint32_t)(128 - r0 - n_loc) * kRowBytes);
+        bulk_commit_and_wait();
+        fence_proxy_async_all();
+      }
     }
+    cluster_arrive();
     cluster_wait();
     if (warp >= 2) {
-      const int owner = row / LR, local = row - owner * LR;
-      float* slot = recv + ((size_t)split * LR + local) * kRecvStride;
-      if (owner == split) {
-        // this CTA's own rows stay local
-#pragma unroll
-        for (int c = 0; c < 64; c += 4)
-          *reinterpret_cast<float4*>(slot + col0 + c) = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
-        if (grp == 0) *reinterpret_cast<float2*>(slot + 128) = make_float2(m_ref, l_row);
-      } else {
-        const uint32_t dst = dsmem_addr(slot, (uint32_t)owner);
-        const uint32_t rbar = dsmem_addr(&bar.recv_full, (uint32_t)owner);
-#pragma unroll
-        for (int c = 0; c < 64; c += 4)
-          st_async4(dst + (uint32_t)(col0 + c) * 4u, o[c], o[c + 1], o[c + 2], o[c + 3], rbar);
-        if (grp == 0) st_async2(dst + 128u * 4u, m_ref, l_row, rbar);
+      if (etid == 0) {
+        fence_proxy_async_all();
+        tc::mbar_arrive_expect_tx(&bar.xch_full, (uint32_t)((ns - 1) * n_loc) * kRowBytes);
+        for (int sp = 0; sp < ns; ++sp)
+          if (sp != split && n_loc > 0)
+            bulk_load_g2s(pbuf + (size_t)sp * LR * kRecvStride, slab0 + ((size_t)sp * 128 + r0) * kRecvStride,
+                          (uint32_t)n_loc * kRowBytes, &bar.xch_full);
       }
-      // rows this CTA owns: the other splits' bytes, and this split's local writes
-      const bool got = wait_bar(&bar.recv_full, 0, abort_flag, p.status, ST_TIMEOUT_EPILOGUE);
-      tc::named_bar_sync(kBarAll, 256);
-      const int r0 = split * LR, n_loc = min(128, r0 + LR) - r0;
-      const int d4 = etid & 31;               // this thread's 4 output columns
-      for (int lr = etid >> 5; got && lr < n_loc; lr += 8) {
-        const int rr = r0 + lr;
-        float ms[8], ls[8];
-        float4 vs[8];
-        float M = -INFINITY;
+      const bool got = wait_bar(&bar.xch_full, 0, abort_flag, p.status, ST_TIMEOUT_EPILOGUE);
+      const int qg = q0 + row / p.G;
+      if (mine && got && qg < p.Lq && !*abort_flag) {
+        const int lr = row - r0;
+        float M = m_ref;
+        for (int sp = 0; sp < ns; ++sp)
+          if (sp != split) M = fmaxf(M, pbuf[((size_t)sp * LR + lr) * kRecvStride + 128]);
+        const float ws0 = m_ref == -INFINITY ? 0.f : ex2(m_ref - M);
+        float L = ws0 * l_row;
 #pragma unroll
-        for (int sp = 0; sp < 8; ++sp) {
-          const float* rp = recv + ((size_t)sp * LR + lr) * kRecvStride;
-          ms[sp] = sp < ns ? rp[128] : -INFINITY;
-          ls[sp] = sp < ns ? rp[129] : 0.f;
-          vs[sp] = sp < ns ? *reinterpret_cast<const float4*>(rp + d4 * 4) : make_float4(0.f, 0.f, 0.f, 0.f);
-          M = fmaxf(M, ms[sp]);
-        }
-        float L = 0.f;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int u = 0; u < 64; ++u) o[u] *= ws0;
+        for (int sp = 0; sp < ns; ++sp) {
+          if (sp == split) continue;
+          const float* rp = pbuf + ((size_t)sp * LR + lr) * kRecvStride;
+          const float ms = rp[128];
+          if (ms == -INFINITY) continue;
+          const float w = ex2(ms - M);
+          L += w * rp[129];
 #pragma unroll
-        for (int sp = 0; sp < 8; ++sp) {
-          const float w = ms[sp] == -INFINITY ? 0.f : ex2(ms[sp] - M);
-          L += w * ls[sp];
-          acc.x += w * vs[sp].x;
-          acc.y += w * vs[sp].y;
-          acc.z += w * vs[sp].z;
-          acc.w += w * vs[sp].w;
+          for (int c = 0; c < 64; c += 4) {
+            const float4 v4 = *reinterpret_cast<const float4*>(rp + col0 + c);
+            o[c] = fmaf(w, v4.x, o[c]);
+            o[c + 1] = fmaf(w, v4.y, o[c + 1]);
+            o[c + 2] = fmaf(w, v4.z, o[c + 2]);
+            o[c + 3] = fmaf(w, v4.w, o[c + 3]);
+          }
         }
-        const int qg2 = q0 + rr / p.G, hh2 = rr % p.G;
-        if (qg2 < p.Lq && !*abort_flag) {
-          const float inv = L > 0.f ? 1.0f / L : 0.f;
-          const int64_t qh = ((int64_t)b * p.Lq + qg2) * p.Hq + g * p.G + hh2;
-          __nv_bfloat162 a0 = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-          __nv_bfloat162 a1 = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
-          uint2* dstp = reinterpret_cast<uint2*>(p.out + qh * 128 + d4 * 4);
-          *dstp = make_uint2(*reinterpret_cast<uint32_t*>(&a0), *reinterpret_cast<uint32_t*>(&a1));
+        const float inv = L > 0.f ? 1.0f / L : 0.f;
+        const int64_t qh = ((int64_t)b * p.Lq + qg) * p.Hq + g * p.G + row % p.G;
+        uint4* dst = reinterpret_cast<uint4*>(p.out + qh * 128 + col0);
+#pragma unroll
+        for (int c = 0; c < 64; c += 8) {
+          __nv_bfloat162 a0 = __floats2bfloat162_rn(o[c] * inv, o[c + 1] * inv);
+          __nv_bfloat162 a1 = __floats2bfloat162_rn(o[c + 2] * inv, o[c + 3] * inv);
+          __nv_bfloat162 a2 = __floats2bfloat162_rn(o[c + 4] * inv, o[c + 5] * inv);
+          __nv_bfloat162 a3 = __floats2bfloat162_rn(o[c + 6] * inv, o[c + 7] * inv);
+          dst[c >> 3] = make_uint4(*reinterpret_cast<uint32_t*>(&a0), *reinterpret_cast<uint32_t*>(&a1),
+                                   *reinterpret_cast<uint32_t*>(&a2), *reinterpret_cast<uint32_t*>(&a3));
         }
       }
     }
@@ -692,7 +695,12 @@ bool attn_tc_supported(int dtype, int Hq, int Hkv, int d) {
   return G >= 1 && G <= 128 && (128 % G) == 0;
 }
 
-size_t attn_tc_workspace_bytes(int, int, int, int, int) { return 0; }  // splits merge on chip
+size_t attn_tc_workspace_bytes(int B, int Lq, int Hq, int Hkv, int n_keys) {
+  int QT, n_qtiles, n_splits, tps;
+  plan_tc(B, Lq, Hq, Hkv, n_keys, QT, n_qtiles, n_splits, tps);
+  if (n_splits <= 1) return 0;
+  return (size_t)B * Hkv * n_qtiles * n_splits * 128 * kRecvStride * sizeof(float);
+}
 
 int launch_attn_tc(const AttnArgs& a, int32_t* status, cudaStream_t s) {
   DLLM_REQUIRE(((uintptr_t)a.q % 16 == 0) && ((uintptr_t)a.k % 16 == 0) && ((uintptr_t)a.v % 16 == 0),
@@ -710,6 +718,13 @@ int launch_attn_tc(const AttnArgs& a, int32_t* status, cudaStream_t s) {
   const float scale = a.scale > 0.f ? a.scale : 1.0f / sqrtf((float)a.d);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.key_pos = a.key_pos;
+  p.xscratch = static_cast<float*>(a.ws);
+  if (p.n_splits > 1) {
+    const size_t need = (size_t)a.B * a.Hkv * p.n_qtiles * p.n_splits * 128 * kRecvStride * sizeof(float);
+    DLLM_REQUIRE(a.ws != nullptr && a.ws_bytes >= need && ((uintptr_t)a.ws % 16) == 0, DLLM_ERR_WORKSPACE,
+                 "attention: split exchange needs %zu bytes of 16-byte aligned workspace (have %zu)", need,
+                 a.ws_bytes);
+  }
   p.out = static_cast<__nv_bfloat16*>(a.out);
   p.status = status;
   CUtensorMap mq, mk, mv;

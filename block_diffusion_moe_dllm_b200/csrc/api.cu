@@ -244,6 +244,7 @@ void plan_step(const dllm_model* m, const dllm_state* st, const dllm_step_params
 // A kernel that waits on an mbarrier nothing ever arrives at, with the same bounded poll loop as the tensor-core
 // kernels (a short bound here), then records the timeout in the status word and returns.
 __global__ void selftest_wait_kernel(int32_t* status, uint32_t max_polls) {
+  dllm::pdl_enter();
   __shared__ uint64_t bar;
   if (threadIdx.x == 0) {
     dllm::tc::mbar_init(&bar, 1);
@@ -259,7 +260,7 @@ extern "C" {
 int dllm_selftest_bounded_wait(void* ws, size_t ws_bytes, cudaStream_t stream) {
   int st = check_ws(ws, ws_bytes, kStatusBytes);
   if (st) return st;
-  selftest_wait_kernel<<<1, 32, 0, stream>>>(status_word(ws), 1u << 12);
+  dllm::launch_pdl(selftest_wait_kernel, 1, 32, 0, stream, status_word(ws), 1u << 12);
   DLLM_CHECK_LAUNCH("selftest_wait_kernel");
   return DLLM_OK;
 }

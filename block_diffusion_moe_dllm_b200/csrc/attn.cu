@@ -37,6 +37,7 @@ struct AttnK {
 
 template <typename T>
 __global__ void __launch_bounds__(256) attn_simt_kernel(const AttnK p) {
+  pdl_enter();
   extern __shared__ float sm[];
   float* qs = sm;                  // [ROWS][DP]
   float* ks = qs + ROWS * DP;      // [KB][DP]
@@ -166,6 +167,7 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(const AttnK p) {
 // out[q, h, :] = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s
 template <typename T>
 __global__ void attn_merge_kernel(const AttnK p) {
+  pdl_enter();
   const int64_t nq = (int64_t)p.B * p.Lq * p.Hq;
   const int64_t qh = blockIdx.x;
   if (qh >= nq) return;
@@ -232,17 +234,17 @@ int launch_attn_simt(const AttnArgs& a, cudaStream_t s) {
   if (a.dtype == DLLM_BF16) {
     static bool cfg = false;
     if (!cfg) { cudaFuncSetAttribute(attn_simt_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); cfg = true; }
-    attn_simt_kernel<__nv_bfloat16><<<grid, 256, smem, s>>>(p);
+    launch_pdl(attn_simt_kernel<__nv_bfloat16>, grid, 256, smem, s, p);
   } else {
     static bool cfg = false;
     if (!cfg) { cudaFuncSetAttribute(attn_simt_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem); cfg = true; }
-    attn_simt_kernel<float><<<grid, 256, smem, s>>>(p);
+    launch_pdl(attn_simt_kernel<float>, grid, 256, smem, s, p);
   }
   DLLM_CHECK_LAUNCH("attn_simt_kernel");
   if (p.n_splits > 1) {
     const int nq = a.B * a.Lq * a.Hq;
-    if (a.dtype == DLLM_BF16) attn_merge_kernel<__nv_bfloat16><<<nq, 128, 0, s>>>(p);
-    else attn_merge_kernel<float><<<nq, 128, 0, s>>>(p);
+    if (a.dtype == DLLM_BF16) launch_pdl(attn_merge_kernel<__nv_bfloat16>, nq, 128, 0, s, p);
+    else launch_pdl(attn_merge_kernel<float>, nq, 128, 0, s, p);
     DLLM_CHECK_LAUNCH("attn_merge_kernel");
   }
   return DLLM_OK;
@@ -263,8 +265,8 @@ int launch_attn_merge(const AttnArgs& a, int n_splits, float* po, float* pm, flo
   p.B = a.B; p.Lq = a.Lq; p.Hq = a.Hq; p.d = a.d; p.n_splits = n_splits;
   p.po = po; p.pm = pm; p.pl = pl; p.out = a.out;
   const int nq = a.B * a.Lq * a.Hq;
-  if (a.dtype == DLLM_BF16) attn_merge_kernel<__nv_bfloat16><<<nq, 128, 0, s>>>(p);
-  else attn_merge_kernel<float><<<nq, 128, 0, s>>>(p);
+  if (a.dtype == DLLM_BF16) launch_pdl(attn_merge_kernel<__nv_bfloat16>, nq, 128, 0, s, p);
+  else launch_pdl(attn_merge_kernel<float>, nq, 128, 0, s, p);
   DLLM_CHECK_LAUNCH("attn_merge_kernel");
   return DLLM_OK;
 }

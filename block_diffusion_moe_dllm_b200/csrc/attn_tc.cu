@@ -24,6 +24,7 @@
 #include "tc.cuh"
 #include "misc.h"
 #include <cuda.h>
+#include <algorithm>
 #include <mutex>
 
 namespace dllm {
@@ -43,6 +44,9 @@ constexpr int kBarAll = 3;         // O and the row sum are rescaled when the ma
 constexpr int kRecvStride = 132;            // floats per exchanged row: o[128], m, l, 2 pad (16-byte multiple)
 constexpr int SMEM = 1024 + TILE /*Q*/ + STAGES * 2 * TILE /*K,V*/ + BARS_BYTES;
 static_assert(SMEM <= 232448, "shared memory budget");
+// with programmatic dependent launch, tensor memory is allocated before the wait for earlier kernels: one such
+// CTA per SM (more than half the SM's shared memory) keeps a later kernel from holding columns an earlier needs
+static_assert(SMEM > 233472 / 2, "tensor-memory kernels must not share an SM");
 static_assert((128 + 135) * kRecvStride * 4 <= STAGES * 2 * TILE,
               "split exchange staging (own rows + n_splits * ceil(128 / n_splits) others) exceeds the K/V ring");
 
@@ -270,6 +274,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   }
   if (warp == 1) tc::tmem_alloc(&bar.tmem_base, 512);
   __syncthreads();
+  pdl_enter();         // everything above is on-chip set-up
   volatile int* abort_flag = &bar.abort_flag;
   const uint32_t tS = bar.tmem_base;          // S buffers (group 0, group 1) at columns [0,128) and [128,256)
   const uint32_t tO = bar.tmem_base + 256;    // O_0, O_1 at columns [256,384) and [384,512)
@@ -673,6 +678,39 @@ int encode(CUtensorMap* m, const void* ptr, int rank, const cuuint64_t* dims, co
   return DLLM_OK;
 }
 
+cudaError_t configure_attn() {
+  static cudaError_t st = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+  return st;
+}
+
+// How many clusters of ns CTAs can be resident at once (a cluster must fit inside one GPC); cached per size.
+int max_active_clusters(int ns) {
+  static int cache[9] = {0};
+  if (ns < 1 || ns > 8) return 0;
+  if (cache[ns] > 0) return cache[ns];
+  int n = 0;
+  if (configure_attn() == cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(ns, 1, 1);
+    cfg.blockDim = dim3(NT, 1, 1);
+    cfg.dynamicSmemBytes = SMEM;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = ns;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, attn_tc_kernel, &cfg) != cudaSuccess) n = 0;
+  }
+  if (n <= 0) {
+    cudaGetLastError();
+    n = num_sms() / (2 * ns);
+  }
+  cache[ns] = std::max(n, 1);
+  return cache[ns];
+}
+
 void plan_tc(int B, int Lq, int Hq, int Hkv, int n_keys, int& QT, int& n_qtiles, int& n_splits, int& tps) {
   const int G = Hq / Hkv;
   QT = 128 / G;
@@ -683,6 +721,7 @@ void plan_tc(int B, int Lq, int Hq, int Hkv, int n_keys, int& QT, int& n_qtiles,
   // fixed cost (setup, first loads, merge) for a sliver of the keys
   const int want = num_sms() / base;
   n_splits = max(1, min(min(want, tiles), 8));
+  while (n_splits > 1 && base > max_active_clusters(n_splits)) --n_splits;
   tps = (tiles + n_splits - 1) / n_splits;
   n_splits = max(1, (tiles + tps - 1) / tps);
 }
@@ -745,24 +784,24 @@ int launch_attn_tc(const AttnArgs& a, int32_t* status, cudaStream_t s) {
     st = encode(&mv, a.v, 3, dims, str, box);
     if (st) return st;
   }
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+  {
+    cudaError_t e = configure_attn();
     if (e != cudaSuccess) return dllm_host::cuda_status(e, "cudaFuncSetAttribute(attn_tc)");
-    configured = true;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(p.n_splits, a.B * a.Hkv * p.n_qtiles, 1);
   cfg.blockDim = dim3(NT, 1, 1);
   cfg.dynamicSmemBytes = SMEM;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = p.n_splits;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // see pdl_wait
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   cudaError_t e = cudaLaunchKernelEx(&cfg, attn_tc_kernel, mq, mk, mv, p);
   if (e != cudaSuccess) return dllm_host::cuda_status(e, "cudaLaunchKernelEx(attn_tc_kernel)");
   DLLM_CHECK_LAUNCH("attn_tc_kernel");

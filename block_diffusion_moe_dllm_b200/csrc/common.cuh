@@ -50,11 +50,40 @@ DLLM_DEV void bf16x8_to_f32(const uint4& u, float* f) {
   }
 }
 
+// Programmatic dependent launch. Every kernel of the library is launched so that the next kernel in the stream
+// may be scheduled before it finishes (pdl_trigger lets that happen as soon as every CTA has started), and every
+// kernel waits for the kernels before it to complete and their writes to be visible (pdl_wait) before it reads or
+// writes any global memory; only on-chip set-up (barriers, tensor memory, descriptor prefetch) may precede it.
+// Both are no-ops for a launch without the attribute.
+DLLM_DEV void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+DLLM_DEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+DLLM_DEV void pdl_enter() {
+  pdl_trigger();
+  pdl_wait();
+}
+
 DLLM_DEV uint4 ld_nc_v4(const void* p) {
   uint4 r;
   asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
                : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
   return r;
+}
+
+// Launch with programmatic stream serialization (see pdl_wait); errors surface through cudaGetLastError.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
 }  // namespace dllm

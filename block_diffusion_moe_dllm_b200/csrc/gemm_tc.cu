@@ -102,12 +102,22 @@ __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g));
 __device__ __forceinline__ void cluster_sync() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-// fp32 load from the same shared-memory offset in the CTA of the cluster with the given rank.
-__device__ __forceinline__ float ld_dsmem(const float* local, uint32_t rank) {
+// Split cluster barrier, usable from divergent code (no .aligned).
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
+}
+// 16-byte load from the same shared-memory offset in the CTA of the cluster with the given rank. Not volatile and
+// without a memory clobber, so that a thread's loads from every rank are issued back to back and their round
+// trips overlap; the cluster barriers (volatile, memory clobber) keep them inside the window where the data is
+// valid.
+__device__ __forceinline__ float4 ld_dsmem4(const float* local, uint32_t rank) {
   uint32_t remote;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(tc::smem_u32(local)), "r"(rank));
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+  asm("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(tc::smem_u32(local)), "r"(rank));
+  float4 v;
+  asm("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(remote));
   return v;
 }
 
@@ -214,23 +224,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
 
-  // ---- group table: counts, offsets and the exclusive prefix of tiles per group
   const int n_groups = p.n_dev + p.has_extra + ((p.n_dev + p.has_extra) == 0 ? 1 : 0);
-  for (int g = tid; g < n_groups; g += NUM_THREADS) {
-    int off, cnt;
-    if (g < p.n_dev) {
-      off = p.grp_off[g];
-      cnt = p.grp_cnt[g];
-    } else if (p.has_extra) {
-      off = p.extra_off;
-      cnt = p.extra_cnt;
-    } else {
-      off = 0;
-      cnt = p.cnt_dev ? min(*p.cnt_dev, p.host_cnt) : p.host_cnt;
-    }
-    sm.grp_off[g] = off;
-    sm.grp_cnt[g] = max(cnt, 0);
-  }
   if (tid == 0) {
     sm.n_groups = n_groups;
     sm.abort_flag = 0;
@@ -246,6 +240,24 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
     tc::fence_mbar_init();
   }
   if (warp == 1) tc::tmem_alloc(&sm.tmem_base, 2 * BN);
+  // everything above is on-chip set-up; the group counts below come from the kernels before this one
+  pdl_enter();
+  // ---- group table: counts, offsets and the exclusive prefix of tiles per group
+  for (int g = tid; g < n_groups; g += NUM_THREADS) {
+    int off, cnt;
+    if (g < p.n_dev) {
+      off = p.grp_off[g];
+      cnt = p.grp_cnt[g];
+    } else if (p.has_extra) {
+      off = p.extra_off;
+      cnt = p.extra_cnt;
+    } else {
+      off = 0;
+      cnt = p.cnt_dev ? min(*p.cnt_dev, p.host_cnt) : p.host_cnt;
+    }
+    sm.grp_off[g] = off;
+    sm.grp_cnt[g] = max(cnt, 0);
+  }
   __syncthreads();
   // prefix of tiles per group: contiguous chunks per thread, a shuffle scan of the thread sums inside each warp,
   // then the six warp totals
@@ -371,7 +383,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
     const int etid = tid - 64;       // 0..127
     uint32_t tcount = 0;
     for (int wk = wk_begin; wk < total; wk += wk_step, ++tcount) {
-      const int t = wk / p.ksplit, ks = wk - t * p.ksplit;
+      const int t = wk / p.ksplit;
       int g, mt, n0, nval;
       decode_tile<BN>(sm, p.m_tiles, t, g, mt, n0, nval);
       const uint32_t buf = tcount & 1, tph = (tcount >> 1) & 1;
@@ -406,28 +418,47 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
   }
   if (p.ksplit > 1) {
     // every slice's staging tile is complete; rank r sums columns [r*nval/ks, (r+1)*nval/ks) over the slices in
-    // rank order (distributed shared memory) and runs the epilogue on them; a second cluster barrier keeps each
-    // CTA's shared memory alive until its peers have read it
+    // rank order (distributed shared memory: each thread takes 8 rows of one column and has its loads from every
+    // rank in flight together) and runs the epilogue on them. The second cluster barrier keeps each CTA's shared
+    // memory alive until its peers have read it: arrive once the reads are done, wait at exit.
     __syncthreads();
     cluster_sync();
+    bool arrived = false;
     if (warp >= 2 && !*abort_flag) {
       const int t = (int)blockIdx.y;
       const int rank = (int)blockIdx.x;
       int g, mt, n0, nval;
       decode_tile<BN>(sm, p.m_tiles, t, g, mt, n0, nval);
-      const int row = (warp & 3) * 32 + lane;
       const int etid = tid - 64;
       const int cb = rank * nval / p.ksplit, ce = (rank + 1) * nval / p.ksplit;
       float* red = reinterpret_cast<float*>(stages);   // the operand ring is idle now
-      for (int j = cb; j < ce; ++j) {
-        float acc = 0.f;
-        for (int sp = 0; sp < p.ksplit; ++sp) acc += ld_dsmem(staging + j * 128 + row, (uint32_t)sp);
-        red[(j - cb) * 128 + row] = acc;
+      const int r8 = (etid & 15) * 8;                   // rows r8 .. r8 + 7
+      for (int j = cb + (etid >> 4); j < ce; j += 8) {
+        float4 lo[8], hi[8];
+#pragma unroll
+        for (int sp = 0; sp < 8; ++sp) {
+          const uint32_t rk = sp < p.ksplit ? (uint32_t)sp : 0u;
+          lo[sp] = ld_dsmem4(staging + j * 128 + r8, rk);
+          hi[sp] = ld_dsmem4(staging + j * 128 + r8 + 4, rk);
+        }
+        float4 a = lo[0], c = hi[0];
+#pragma unroll
+        for (int sp = 1; sp < 8; ++sp) {
+          if (sp < p.ksplit) {
+            a.x += lo[sp].x; a.y += lo[sp].y; a.z += lo[sp].z; a.w += lo[sp].w;
+            c.x += hi[sp].x; c.y += hi[sp].y; c.z += hi[sp].z; c.w += hi[sp].w;
+          }
+        }
+        *reinterpret_cast<float4*>(red + (j - cb) * 128 + r8) = a;
+        *reinterpret_cast<float4*>(red + (j - cb) * 128 + r8 + 4) = c;
       }
+      cluster_arrive();
+      arrived = true;
       tc::named_bar_sync(1, 128);
       if (ce > cb) epilogue_chunk<BN>(p, red, g, mt, n0 + cb, ce - cb, 0, sm.grp_off[g], etid);
     }
-    cluster_sync();
+    if (!arrived) cluster_arrive();
+    cluster_wait();
   }
   __syncthreads();
   if (warp == 1) {
@@ -485,6 +516,10 @@ int launch(const GemmArgs& a, const CUtensorMap& mw, const CUtensorMap& mw2, con
   constexpr int STAGE_BYTES = A_BYTES + BN * BK * 2;
   constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + STAGING_BYTES + (int)sizeof(Smem);
   static_assert(SMEM <= SMEM_LIMIT, "shared memory budget");
+  // With programmatic dependent launch a CTA allocates tensor memory before it waits for the kernels ahead of it.
+  // More than half an SM's shared memory per CTA keeps two tensor-memory kernels from sharing an SM, so a later
+  // kernel can never hold the columns an earlier one is still waiting to allocate.
+  static_assert(SMEM > 233472 / 2, "tensor-memory kernels must not share an SM");
   static bool configured = false;
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -492,36 +527,71 @@ int launch(const GemmArgs& a, const CUtensorMap& mw, const CUtensorMap& mw2, con
     if (e != cudaSuccess) return dllm_host::cuda_status(e, "cudaFuncSetAttribute(gemm_tc)");
     configured = true;
   }
-  gemm_tc_kernel<BN, STAGES><<<num_sms(), NUM_THREADS, SMEM, s>>>(mw, mw2, mx, kp);
+  launch_pdl((gemm_tc_kernel<BN, STAGES>), num_sms(), NUM_THREADS, SMEM, s, mw, mw2, mx, kp);
   DLLM_CHECK_LAUNCH("gemm_tc_kernel");
   return DLLM_OK;
 }
 
+constexpr int SPLITK_BN = 32, SPLITK_STAGES = 9;
+constexpr int SPLITK_SMEM = 1024 + SPLITK_STAGES * (A_BYTES + SPLITK_BN * BK * 2) + STAGING_BYTES + (int)sizeof(Smem);
+
+static cudaError_t configure_splitk() {
+  static cudaError_t st = cudaFuncSetAttribute(gemm_tc_kernel<SPLITK_BN, SPLITK_STAGES>,
+                                               cudaFuncAttributeMaxDynamicSharedMemorySize, SPLITK_SMEM);
+  return st;
+}
+
+// How many clusters of ks split-K CTAs can be resident at once (each cluster must sit inside one GPC, so sizes that
+// do not divide the GPCs' SM counts leave SMs unused); cached per size.
+static int max_active_clusters(int ks) {
+  static int cache[9] = {0};
+  if (ks < 1 || ks > 8) return 0;
+  if (cache[ks] > 0) return cache[ks];
+  int n = 0;
+  if (configure_splitk() == cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(ks, 1, 1);
+    cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = SPLITK_SMEM;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = ks;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel<SPLITK_BN, SPLITK_STAGES>, &cfg) != cudaSuccess) n = 0;
+  }
+  if (n <= 0) {
+    cudaGetLastError();
+    n = num_sms() / (2 * ks);   // conservative when the query is unavailable
+  }
+  cache[ks] = std::max(n, 1);
+  return cache[ks];
+}
+
 int launch_cluster_splitk(const GemmArgs& a, const CUtensorMap& mw, const CUtensorMap& mw2, const CUtensorMap& mx,
                           const KParams& kp, cudaStream_t s) {
-  constexpr int BN = 32, STAGES = 9;
-  constexpr int STAGE_BYTES = A_BYTES + BN * BK * 2;
-  constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + STAGING_BYTES + (int)sizeof(Smem);
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         SMEM);
+  constexpr int SMEM = SPLITK_SMEM;
+  {
+    cudaError_t e = configure_splitk();
     if (e != cudaSuccess) return dllm_host::cuda_status(e, "cudaFuncSetAttribute(gemm_tc cluster)");
-    configured = true;
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(kp.ksplit, a.M / 128, 1);
   cfg.blockDim = dim3(NUM_THREADS, 1, 1);
   cfg.dynamicSmemBytes = SMEM;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = kp.ksplit;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // see pdl_wait
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, STAGES>, mw, mw2, mx, kp);
+  cfg.numAttrs = 2;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<SPLITK_BN, SPLITK_STAGES>, mw, mw2, mx, kp);
   if (e != cudaSuccess) return dllm_host::cuda_status(e, "cudaLaunchKernelEx(gemm_tc cluster split-K)");
   DLLM_CHECK_LAUNCH("gemm_tc_kernel (cluster split-K)");
   return DLLM_OK;
@@ -593,13 +663,16 @@ int gemm_bn(const GemmArgs& a) {
 }
 
 // Split-K for dense projections that still leave most SMs idle at N tile 32 (all rows in one tile): K slices of
-// at least two 64-wide blocks, at most 8 (the portable cluster size) and no more than fill the SMs.
+// at least two 64-wide blocks, at most 8 (the portable cluster size), and only as many as let every tile's cluster
+// be resident at once (a second wave would double the kernel's time).
 int gemm_splitk_factor(const GemmArgs& a, int bn) {
   if (a.dtype != DLLM_BF16 || !dense(a) || bn != 32 || a.max_cnt > 32) return 1;
   const int tiles = a.M / 128;
   const int kblocks = a.K / BK;
   if (tiles <= 0 || tiles * 2 > num_sms() || kblocks < 4) return 1;
-  return std::max(1, std::min(std::min(kblocks / 2, 8), num_sms() / tiles));
+  int ks = std::max(1, std::min(std::min(kblocks / 2, 8), num_sms() / tiles));
+  while (ks > 1 && tiles > max_active_clusters(ks)) --ks;
+  return ks;
 }
 
 int num_sms() {

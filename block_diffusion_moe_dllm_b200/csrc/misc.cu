@@ -11,6 +11,7 @@ namespace dllm {
 template <typename T>
 __global__ void embed_kernel(const int32_t* __restrict__ tokens, const uint8_t* __restrict__ mask, int mask_id,
                              const T* __restrict__ table, T* __restrict__ x, int H) {
+  pdl_enter();
   const int t = blockIdx.x;
   const int id = (mask && mask[t]) ? mask_id : tokens[t];
   const uint4* src = reinterpret_cast<const uint4*>(table + (int64_t)id * H);
@@ -23,10 +24,10 @@ int launch_embed(int dtype, const int32_t* tokens, const uint8_t* mask, int mask
                  int rows, int H, cudaStream_t s) {
   if (rows <= 0) return DLLM_OK;
   if (dtype == DLLM_BF16)
-    embed_kernel<__nv_bfloat16><<<rows, 128, 0, s>>>(tokens, mask, mask_id, (const __nv_bfloat16*)table,
+    launch_pdl(embed_kernel<__nv_bfloat16>, rows, 128, 0, s, tokens, mask, mask_id, (const __nv_bfloat16*)table,
                                                      (__nv_bfloat16*)x, H);
   else
-    embed_kernel<float><<<rows, 128, 0, s>>>(tokens, mask, mask_id, (const float*)table, (float*)x, H);
+    launch_pdl(embed_kernel<float>, rows, 128, 0, s, tokens, mask, mask_id, (const float*)table, (float*)x, H);
   DLLM_CHECK_LAUNCH("embed_kernel");
   return DLLM_OK;
 }
@@ -40,6 +41,7 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const T* __restrict__ x, c
                                                       const int32_t* __restrict__ row_pos,
                                                       const int32_t* __restrict__ n_dev, int two_halves,
                                                       int uncond_off) {
+  pdl_enter();
   int r = blockIdx.x;
   int src = r;
   if (row_pos) {
@@ -111,11 +113,11 @@ int launch_rmsnorm(int dtype, const void* x, const void* g, void* out, int rows,
                    const int32_t* row_pos, const int32_t* n_dev, int two_halves, int uncond_off, cudaStream_t s) {
   if (rows <= 0) return DLLM_OK;
   if (dtype == DLLM_BF16)
-    rmsnorm_kernel<__nv_bfloat16><<<rows, 256, 0, s>>>((const __nv_bfloat16*)x, (const __nv_bfloat16*)g,
+    launch_pdl(rmsnorm_kernel<__nv_bfloat16>, rows, 256, 0, s, (const __nv_bfloat16*)x, (const __nv_bfloat16*)g,
                                                        (__nv_bfloat16*)out, H, eps, row_pos, n_dev, two_halves,
                                                        uncond_off);
   else
-    rmsnorm_kernel<float><<<rows, 256, 0, s>>>((const float*)x, (const float*)g, (float*)out, H, eps, row_pos,
+    launch_pdl(rmsnorm_kernel<float>, rows, 256, 0, s, (const float*)x, (const float*)g, (float*)out, H, eps, row_pos,
                                                n_dev, two_halves, uncond_off);
   DLLM_CHECK_LAUNCH("rmsnorm_kernel");
   return DLLM_OK;
@@ -126,6 +128,7 @@ int launch_rmsnorm(int dtype, const void* x, const void* g, void* out, int rows,
 // count n_out[0] and n_out[1] = n_out[0] * halves (rows the LM head scores).
 __global__ void masked_rows_kernel(const uint8_t* __restrict__ mask, int n_pos, int halves, int32_t* row_pos,
                                    int32_t* n_out) {
+  pdl_enter();
   __shared__ int warp_tot[32];
   __shared__ int base;
   if (threadIdx.x == 0) base = 0;
@@ -156,7 +159,7 @@ __global__ void masked_rows_kernel(const uint8_t* __restrict__ mask, int n_pos, 
 
 int launch_masked_rows(const uint8_t* mask, int n_pos, int halves, int32_t* row_pos, int32_t* n_out,
                        cudaStream_t s) {
-  masked_rows_kernel<<<1, 1024, 0, s>>>(mask, n_pos, halves, row_pos, n_out);
+  launch_pdl(masked_rows_kernel, 1, 1024, 0, s, mask, n_pos, halves, row_pos, n_out);
   DLLM_CHECK_LAUNCH("masked_rows_kernel");
   return DLLM_OK;
 }
@@ -166,6 +169,7 @@ int launch_masked_rows(const uint8_t* mask, int n_pos, int halves, int32_t* row_
 template <typename T>
 __global__ void gather_rows_kernel(const T* __restrict__ h, const int32_t* __restrict__ perm, int k, int n_assign,
                                    int shared, T* __restrict__ xp, int H) {
+  pdl_enter();
   const int r = blockIdx.x;
   int src;
   if (r < n_assign) src = perm[r] / k;
@@ -182,10 +186,10 @@ int launch_gather_rows(int dtype, const void* h, const int32_t* perm, int k, int
   const int rows = Tk * k + (shared ? Tk : 0);
   if (rows <= 0) return DLLM_OK;
   if (dtype == DLLM_BF16)
-    gather_rows_kernel<__nv_bfloat16><<<rows, 128, 0, s>>>((const __nv_bfloat16*)h, perm, k, Tk * k, shared,
+    launch_pdl(gather_rows_kernel<__nv_bfloat16>, rows, 128, 0, s, (const __nv_bfloat16*)h, perm, k, Tk * k, shared,
                                                            (__nv_bfloat16*)xp, H);
   else
-    gather_rows_kernel<float><<<rows, 128, 0, s>>>((const float*)h, perm, k, Tk * k, shared, (float*)xp, H);
+    launch_pdl(gather_rows_kernel<float>, rows, 128, 0, s, (const float*)h, perm, k, Tk * k, shared, (float*)xp, H);
   DLLM_CHECK_LAUNCH("gather_rows_kernel");
   return DLLM_OK;
 }
@@ -196,6 +200,7 @@ template <typename T>
 __global__ void __launch_bounds__(128) combine_kernel(T* __restrict__ x, const float* __restrict__ y,
                                                       const float* __restrict__ gates, const int32_t* __restrict__ inv,
                                                       int k, int n_assign, int shared, int H) {
+  pdl_enter();
   // grid (tokens, H / 512): each thread owns 4 consecutive hidden elements
   const int t = blockIdx.x;
   const int h0 = (blockIdx.y * blockDim.x + threadIdx.x) * 4;
@@ -222,9 +227,9 @@ int launch_combine(int dtype, void* x, const float* y, const float* gates, const
   if (Tk <= 0) return DLLM_OK;
   dim3 grid(Tk, (H / 4 + 127) / 128);
   if (dtype == DLLM_BF16)
-    combine_kernel<__nv_bfloat16><<<grid, 128, 0, s>>>((__nv_bfloat16*)x, y, gates, inv, k, Tk * k, shared, H);
+    launch_pdl(combine_kernel<__nv_bfloat16>, grid, 128, 0, s, (__nv_bfloat16*)x, y, gates, inv, k, Tk * k, shared, H);
   else
-    combine_kernel<float><<<grid, 128, 0, s>>>((float*)x, y, gates, inv, k, Tk * k, shared, H);
+    launch_pdl(combine_kernel<float>, grid, 128, 0, s, (float*)x, y, gates, inv, k, Tk * k, shared, H);
   DLLM_CHECK_LAUNCH("combine_kernel");
   return DLLM_OK;
 }
@@ -255,6 +260,7 @@ __device__ __forceinline__ void group_of(const SimtGroups& G, int g, int& off, i
 __global__ void simt_gemm_f32_kernel(const float* __restrict__ X, const float* __restrict__ W,
                                      const float* __restrict__ W2, int K, int Mw, int64_t wstride, SimtGroups G,
                                      float* __restrict__ raw) {
+  pdl_enter();
   const int g = blockIdx.z;
   int off, cnt;
   group_of(G, g, off, cnt);
@@ -298,6 +304,7 @@ __global__ void simt_gemm_f32_kernel(const float* __restrict__ X, const float* _
 template <typename T>
 __global__ void raw_epilogue_kernel(const float* __restrict__ raw, int nsplit, int64_t split_stride, int Mw, int M,
                                     SimtGroups G, EpiParams e) {
+  pdl_enter();
   const int g = blockIdx.y;
   int off, cnt;
   group_of(G, g, off, cnt);
@@ -374,11 +381,11 @@ int gemm_f32_simt(const GemmArgs& a, cudaStream_t s) {
   const int Mw = a.swiglu ? 2 * a.M : a.M;
   const int max_cnt = a.cnt_bound > 0 ? a.cnt_bound : 1;
   dim3 grid((max_cnt + 31) / 32, (Mw + 63) / 64, n_groups);
-  simt_gemm_f32_kernel<<<grid, 256, 0, s>>>((const float*)a.x, (const float*)a.w, (const float*)a.w2, a.K, Mw,
+  launch_pdl(simt_gemm_f32_kernel, grid, 256, 0, s, (const float*)a.x, (const float*)a.w, (const float*)a.w2, a.K, Mw,
                                             a.w_group_stride, G, a.f32_scratch);
   DLLM_CHECK_LAUNCH("simt_gemm_f32_kernel");
   dim3 g2(max_cnt, n_groups);
-  raw_epilogue_kernel<float><<<g2, 128, 0, s>>>(a.f32_scratch, 1, 0, Mw, a.M, G, a.epi);
+  launch_pdl(raw_epilogue_kernel<float>, g2, 128, 0, s, a.f32_scratch, 1, 0, Mw, a.M, G, a.epi);
   DLLM_CHECK_LAUNCH("raw_epilogue_kernel");
   return DLLM_OK;
 }

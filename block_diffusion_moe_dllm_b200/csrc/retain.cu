@@ -18,6 +18,7 @@ namespace {
 template <typename T>
 __global__ void retain_scores_kernel(const T* __restrict__ k, int B, int Hkv, int d, int P, int cap,
                                      float* __restrict__ raw) {
+  pdl_enter();
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (warp >= B * P) return;
   const int b = warp / P, i = warp - b * P;
@@ -38,6 +39,7 @@ __global__ void retain_scores_kernel(const T* __restrict__ k, int B, int Hkv, in
 // One CTA (1024 threads) per batch row: threshold search, stable selection, keep_pos and normalised scores.
 __global__ void retain_select_kernel(const float* __restrict__ raw, int P, int n_keep, int cap_thin,
                                      int32_t* __restrict__ keep_pos, float* __restrict__ scores, int block_len) {
+  pdl_enter();
   __shared__ int red[32];
   __shared__ double dred[32];
   __shared__ int base;
@@ -131,6 +133,7 @@ template <typename T>
 __global__ void retain_copy_kernel(const T* __restrict__ k, const T* __restrict__ v, const int32_t* __restrict__ keep_pos,
                                    int B, int Hkv, int d, int cap, int n_keep, int cap_thin, T* __restrict__ kt,
                                    T* __restrict__ vt) {
+  pdl_enter();
   const int64_t warp = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (warp >= (int64_t)B * Hkv * n_keep) return;
@@ -157,21 +160,21 @@ int launch_retain(const RetainArgs& a, cudaStream_t s) {
   const int64_t rows = (int64_t)a.B * a.P;
   const int blocks = (int)((rows * 32 + 255) / 256);
   if (a.dtype == DLLM_BF16)
-    retain_scores_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>((const __nv_bfloat16*)a.k, a.B, a.Hkv, a.d, a.P, a.cap, a.raw);
+    launch_pdl(retain_scores_kernel<__nv_bfloat16>, blocks, 256, 0, s, (const __nv_bfloat16*)a.k, a.B, a.Hkv, a.d, a.P, a.cap, a.raw);
   else
-    retain_scores_kernel<float><<<blocks, 256, 0, s>>>((const float*)a.k, a.B, a.Hkv, a.d, a.P, a.cap, a.raw);
+    launch_pdl(retain_scores_kernel<float>, blocks, 256, 0, s, (const float*)a.k, a.B, a.Hkv, a.d, a.P, a.cap, a.raw);
   DLLM_CHECK_LAUNCH("retain_scores_kernel");
-  retain_select_kernel<<<a.B, 1024, 0, s>>>(a.raw, a.P, a.n_keep, a.cap_thin, a.keep_pos, a.scores, a.block_len);
+  launch_pdl(retain_select_kernel, a.B, 1024, 0, s, a.raw, a.P, a.n_keep, a.cap_thin, a.keep_pos, a.scores, a.block_len);
   DLLM_CHECK_LAUNCH("retain_select_kernel");
   const int64_t copies = (int64_t)a.B * a.Hkv * a.n_keep;
   if (copies > 0) {
     const int cb = (int)((copies * 32 + 255) / 256);
     if (a.dtype == DLLM_BF16)
-      retain_copy_kernel<__nv_bfloat16><<<cb, 256, 0, s>>>((const __nv_bfloat16*)a.k, (const __nv_bfloat16*)a.v, a.keep_pos,
+      launch_pdl(retain_copy_kernel<__nv_bfloat16>, cb, 256, 0, s, (const __nv_bfloat16*)a.k, (const __nv_bfloat16*)a.v, a.keep_pos,
                                                           a.B, a.Hkv, a.d, a.cap, a.n_keep, a.cap_thin,
                                                           (__nv_bfloat16*)a.k_thin, (__nv_bfloat16*)a.v_thin);
     else
-      retain_copy_kernel<float><<<cb, 256, 0, s>>>((const float*)a.k, (const float*)a.v, a.keep_pos, a.B, a.Hkv, a.d,
+      launch_pdl(retain_copy_kernel<float>, cb, 256, 0, s, (const float*)a.k, (const float*)a.v, a.keep_pos, a.B, a.Hkv, a.d,
                                                    a.cap, a.n_keep, a.cap_thin, (float*)a.k_thin, (float*)a.v_thin);
     DLLM_CHECK_LAUNCH("retain_copy_kernel");
   }

@@ -25,6 +25,7 @@ DLLM_DEV void load8(const float* p, float* f) {
 template <typename T>
 __global__ void __launch_bounds__(256) route_scores_kernel(const T* __restrict__ h, const T* __restrict__ w, int Tk,
                                                            int H, int E, float* __restrict__ scores) {
+  pdl_enter();
   extern __shared__ __align__(16) unsigned char hs_raw[];
   T* hs = reinterpret_cast<T*>(hs_raw);  // [TT][H]
   const int e0 = blockIdx.x * EW, t0 = blockIdx.y * TT;
@@ -80,6 +81,7 @@ __global__ void __launch_bounds__(256) route_scores_kernel(const T* __restrict__
 // With from_logits the row holds router logits: the sigmoid scores replace them in place.
 __global__ void route_topk_kernel(float* __restrict__ scores, const float* __restrict__ bias, int Tk, int E, int k,
                                   int from_logits, int32_t* __restrict__ ids, float* __restrict__ gates) {
+  pdl_enter();
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (warp >= Tk) return;
   float* s = scores + (int64_t)warp * E;
@@ -178,6 +180,7 @@ __device__ void block_exclusive_scan(int* a, int n, int* total) {
 // increasing assignment order (t * k + j), which keeps the rows of an expert sorted by token.
 __global__ void route_permute_kernel(const int32_t* __restrict__ ids, int n_assign, int E, int32_t* counts,
                                      int32_t* offsets, int32_t* perm, int32_t* inv) {
+  pdl_enter();
   __shared__ int hist[1024];
   __shared__ int cnt_e;
   __shared__ int wtot[8];
@@ -237,9 +240,9 @@ int launch_route(int dtype, const void* h, const void* w_router, const float* bi
     g.epi.kind = EPI_STORE; g.epi.out = scores; g.epi.ldo = E; g.epi.out_f32 = 1;
     int st = gemm_bf16_tc(g, s);
     if (st) return st;
-    route_topk_kernel<<<(Tk + 7) / 8, 256, 0, s>>>(scores, bias, Tk, E, k, 1, ids, gates);
+    launch_pdl(route_topk_kernel, (Tk + 7) / 8, 256, 0, s, scores, bias, Tk, E, k, 1, ids, gates);
     DLLM_CHECK_LAUNCH("route_topk_kernel");
-    route_permute_kernel<<<E, 256, 0, s>>>(ids, Tk * k, E, counts, offsets, perm, inv);
+    launch_pdl(route_permute_kernel, E, 256, 0, s, ids, Tk * k, E, counts, offsets, perm, inv);
     DLLM_CHECK_LAUNCH("route_permute_kernel");
     return DLLM_OK;
   }
@@ -252,7 +255,7 @@ int launch_route(int dtype, const void* h, const void* w_router, const float* bi
                            200 * 1024);
       cfg = true;
     }
-    route_scores_kernel<__nv_bfloat16><<<g1, 256, smem, s>>>((const __nv_bfloat16*)h,
+    launch_pdl(route_scores_kernel<__nv_bfloat16>, g1, 256, smem, s, (const __nv_bfloat16*)h,
                                                              (const __nv_bfloat16*)w_router, Tk, H, E, scores);
   } else {
     static bool cfg = false;
@@ -260,12 +263,12 @@ int launch_route(int dtype, const void* h, const void* w_router, const float* bi
       cudaFuncSetAttribute(route_scores_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
       cfg = true;
     }
-    route_scores_kernel<float><<<g1, 256, smem, s>>>((const float*)h, (const float*)w_router, Tk, H, E, scores);
+    launch_pdl(route_scores_kernel<float>, g1, 256, smem, s, (const float*)h, (const float*)w_router, Tk, H, E, scores);
   }
   DLLM_CHECK_LAUNCH("route_scores_kernel");
-  route_topk_kernel<<<(Tk + 7) / 8, 256, 0, s>>>(scores, bias, Tk, E, k, 0, ids, gates);
+  launch_pdl(route_topk_kernel, (Tk + 7) / 8, 256, 0, s, scores, bias, Tk, E, k, 0, ids, gates);
   DLLM_CHECK_LAUNCH("route_topk_kernel");
-  route_permute_kernel<<<E, 256, 0, s>>>(ids, Tk * k, E, counts, offsets, perm, inv);
+  launch_pdl(route_permute_kernel, E, 256, 0, s, ids, Tk * k, E, counts, offsets, perm, inv);
   DLLM_CHECK_LAUNCH("route_permute_kernel");
   return DLLM_OK;
 }

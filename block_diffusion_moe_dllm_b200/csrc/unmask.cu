@@ -73,6 +73,7 @@ __global__ void __launch_bounds__(256) unmask_reduce_kernel(const T* __restrict_
                                                             const int32_t* __restrict__ n_rows, int V, int chunk,
                                                             float cfg_scale, Partial* __restrict__ part,
                                                             int n_chunks) {
+  pdl_enter();
   const int r = blockIdx.x, c = blockIdx.y;
   const int n = *n_rows;
   if (r >= n) return;
@@ -172,6 +173,7 @@ template <int VPT>
 __global__ void __launch_bounds__(256) unmask_reduce_bf16_kernel(const __nv_bfloat16* __restrict__ logits,
                                                                  const int32_t* __restrict__ n_rows, int V, int chunk,
                                                                  Partial* __restrict__ part, int n_chunks) {
+  pdl_enter();
   const int r = blockIdx.x, c = blockIdx.y;
   if (r >= *n_rows) return;
   const __nv_bfloat16* z = logits + (int64_t)r * V;
@@ -254,6 +256,7 @@ __global__ void unmask_select_kernel(const Partial* __restrict__ part, int n_chu
                                      const int32_t* __restrict__ n_rows, int B, int L, int t, int T_s, int mode,
                                      float tau, int k_max, int cfg, int vocab_offset, int32_t* tokens, uint8_t* mask,
                                      int32_t* sel, int32_t* nsel, float* conf, int32_t* remaining) {
+  pdl_enter();
   __shared__ int rem_w[32];
   __shared__ int row_cnt[1024];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
@@ -366,19 +369,19 @@ int launch_unmask(const UnmaskArgs& a, cudaStream_t s) {
     Partial* part = static_cast<Partial*>(a.partials);
     if (a.dtype == DLLM_BF16) {
       const __nv_bfloat16* z = static_cast<const __nv_bfloat16*>(a.logits);
-      if (a.cfg) unmask_reduce_kernel<__nv_bfloat16, true><<<grid, 256, 0, s>>>(z, a.n_rows, a.V, chunk, a.cfg_scale, part, a.n_chunks);
+      if (a.cfg) launch_pdl((unmask_reduce_kernel<__nv_bfloat16, true>), grid, 256, 0, s, z, a.n_rows, a.V, chunk, a.cfg_scale, part, a.n_chunks);
       else if (a.V % 8 == 0 && chunk <= kRegChunk)
-        unmask_reduce_bf16_kernel<kRegVpt><<<grid, 256, 0, s>>>(z, a.n_rows, a.V, chunk, part, a.n_chunks);
-      else unmask_reduce_kernel<__nv_bfloat16, false><<<grid, 256, 0, s>>>(z, a.n_rows, a.V, chunk, a.cfg_scale, part, a.n_chunks);
+        launch_pdl(unmask_reduce_bf16_kernel<kRegVpt>, grid, 256, 0, s, z, a.n_rows, a.V, chunk, part, a.n_chunks);
+      else launch_pdl((unmask_reduce_kernel<__nv_bfloat16, false>), grid, 256, 0, s, z, a.n_rows, a.V, chunk, a.cfg_scale, part, a.n_chunks);
     } else {
       const float* z = static_cast<const float*>(a.logits);
-      if (a.cfg) unmask_reduce_kernel<float, true><<<grid, 256, 0, s>>>(z, a.n_rows, a.V, chunk, a.cfg_scale, part, a.n_chunks);
-      else unmask_reduce_kernel<float, false><<<grid, 256, 0, s>>>(z, a.n_rows, a.V, chunk, a.cfg_scale, part, a.n_chunks);
+      if (a.cfg) launch_pdl((unmask_reduce_kernel<float, true>), grid, 256, 0, s, z, a.n_rows, a.V, chunk, a.cfg_scale, part, a.n_chunks);
+      else launch_pdl((unmask_reduce_kernel<float, false>), grid, 256, 0, s, z, a.n_rows, a.V, chunk, a.cfg_scale, part, a.n_chunks);
     }
     DLLM_CHECK_LAUNCH("unmask_reduce_kernel");
   }
   const int threads = 32 * min(32, max(1, a.B));
-  unmask_select_kernel<<<1, threads, 0, s>>>(static_cast<const Partial*>(a.partials), a.n_chunks, a.row_pos, a.n_rows,
+  launch_pdl(unmask_select_kernel, 1, threads, 0, s, static_cast<const Partial*>(a.partials), a.n_chunks, a.row_pos, a.n_rows,
                                              a.B, a.L, a.t, a.T_s, a.mode, a.tau, a.k_max, a.cfg, a.vocab_offset,
                                              a.tokens, a.mask, a.sel, a.nsel, a.conf, a.remaining);
   DLLM_CHECK_LAUNCH("unmask_select_kernel");

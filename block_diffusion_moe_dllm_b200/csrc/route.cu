@@ -79,64 +79,193 @@ __global__ void __launch_bounds__(256) route_scores_kernel(const T* __restrict__
 // Lane l holds experts l, l + 32, ... in registers (biased and unbiased); the winner's unbiased score comes from the
 // owning lane by a shuffle, so the rounds touch no memory.
 // With from_logits the row holds router logits: the sigmoid scores replace them in place.
-__global__ void route_topk_kernel(float* __restrict__ scores, const float* __restrict__ bias, int Tk, int E, int k,
-                                  int from_logits, int32_t* __restrict__ ids, float* __restrict__ gates) {
-  pdl_enter();
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-  if (warp >= Tk) return;
-  float* s = scores + (int64_t)warp * E;
-  float val[32], raw[32];
-  const int per = (E + 31) / 32;
+// Top-k of one token's expert scores, one warp. Lane l owns experts e = i * 32 + l (i < PER); the selection key is
+// the biased score val = raw + bias (ties to the lower expert), the gate the unbiased raw score, renormalised over
+// the chosen k. Each lane sorts its PER candidates with an insertion network (descending val, ascending e); then
+// k rounds take the warp-wide best head (a 5-step butterfly on (val, e)) and the winning lane pops its head.
+// With from_logits the raw scores are sigmoid(logit) and are written back over the logits.
+template <int PER>
+DLLM_DEV void warp_topk(float* __restrict__ srow, const float* __restrict__ bias, int E, int k, int from_logits,
+                        int lane, int& my_id, float& my_gate) {
+  float v[PER], r[PER];
+  int e[PER];
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const int e = i * 32 + lane;
-    const bool in = i < per && e < E;
-    float v = in ? s[e] : 0.f;
+  for (int i = 0; i < PER; ++i) {
+    const int ex = i * 32 + lane;
+    const bool in = ex < E;
+    float x = in ? srow[ex] : 0.f;
     if (from_logits && in) {
-      v = 1.0f / (1.0f + expf(-v));
-      s[e] = v;
+      x = 1.0f / (1.0f + expf(-x));
+      srow[ex] = x;
     }
-    raw[i] = v;
-    val[i] = in ? v + bias[e] : -INFINITY;
+    r[i] = x;
+    v[i] = in ? x + bias[ex] : -INFINITY;
+    e[i] = in ? ex : 0x7fffffff;
   }
-  float gsum = 0.f, my_gate = 0.f;
-  int my_id = 0;
-  // each lane's best (value, expert); only the winning lane rescans its own values after a round
-  auto lane_best = [&](float& bv, int& be) {
-    bv = -INFINITY;
-    be = 0x7fffffff;
+  // insertion network: after step i, entries [0, i] are sorted (PER <= 8; wider rows keep the unsorted
+  // candidates and the winning lane rescans them, below)
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      const int e = i * 32 + lane;
-      if (i < per && (val[i] > bv || (val[i] == bv && e < be))) { bv = val[i]; be = e; }
+  for (int i = 1; i < (PER <= 8 ? PER : 1); ++i) {
+#pragma unroll
+    for (int j = i; j > 0; --j) {
+      const bool sw = v[j] > v[j - 1] || (v[j] == v[j - 1] && e[j] < e[j - 1]);
+      const float tv = v[j], tr = r[j];
+      const int te = e[j];
+      v[j] = sw ? v[j - 1] : tv; r[j] = sw ? r[j - 1] : tr; e[j] = sw ? e[j - 1] : te;
+      v[j - 1] = sw ? tv : v[j - 1]; r[j - 1] = sw ? tr : r[j - 1]; e[j - 1] = sw ? te : e[j - 1];
     }
-  };
-  float lbv;
-  int lbe;
-  lane_best(lbv, lbe);
+  }
+  if (PER > 8) {
+#pragma unroll
+    for (int i = 1; i < PER; ++i) {
+      const bool sw = v[i] > v[0] || (v[i] == v[0] && e[i] < e[0]);
+      const float tv = v[i], tr = r[i];
+      const int te = e[i];
+      v[i] = sw ? v[0] : tv; r[i] = sw ? r[0] : tr; e[i] = sw ? e[0] : te;
+      v[0] = sw ? tv : v[0]; r[0] = sw ? tr : r[0]; e[0] = sw ? te : e[0];
+    }
+  }
+  float gsum = 0.f;
+  my_id = 0;
+  my_gate = 0.f;
   for (int j = 0; j < k; ++j) {
-    float bv = lbv;
-    int be = lbe;
+    float bv = v[0];
+    int be = e[0];
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
       const int oe = __shfl_xor_sync(0xffffffffu, be, o);
       if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
     }
-    float mine = 0.f;
-    if ((be & 31) == lane) {
+    const int win = be & 31;
+    const float sc = __shfl_sync(0xffffffffu, r[0], win);
+    if (lane == win) {
+      if (PER <= 8) {   // pop the sorted head
 #pragma unroll
-      for (int i = 0; i < 32; ++i)
-        if (i * 32 + lane == be) { mine = raw[i]; val[i] = -INFINITY; }
-      lane_best(lbv, lbe);
+        for (int i = 0; i + 1 < PER; ++i) { v[i] = v[i + 1]; r[i] = r[i + 1]; e[i] = e[i + 1]; }
+        v[PER - 1] = -INFINITY;
+        e[PER - 1] = 0x7fffffff;
+      } else {          // drop the winner and move this lane's next best to slot 0
+        v[0] = -INFINITY;
+        e[0] = 0x7fffffff;
+#pragma unroll
+        for (int i = 1; i < PER; ++i) {
+          const bool sw = v[i] > v[0] || (v[i] == v[0] && e[i] < e[0]);
+          const float tv = v[i], tr = r[i];
+          const int te = e[i];
+          v[i] = sw ? v[0] : tv; r[i] = sw ? r[0] : tr; e[i] = sw ? e[0] : te;
+          v[0] = sw ? tv : v[0]; r[0] = sw ? tr : r[0]; e[0] = sw ? te : e[0];
+        }
+      }
     }
-    const float sc = __shfl_sync(0xffffffffu, mine, be & 31);
     gsum += sc;
     if (lane == j) { my_id = be; my_gate = sc; }
   }
+  my_gate = my_gate / gsum;
+}
+
+// One warp per token.
+template <int PER>
+__global__ void route_topk_kernel(float* __restrict__ scores, const float* __restrict__ bias, int Tk, int E, int k,
+                                  int from_logits, int32_t* __restrict__ ids, float* __restrict__ gates) {
+  pdl_enter();
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (warp >= Tk) return;
+  int my_id;
+  float my_gate;
+  warp_topk<PER>(scores + (int64_t)warp * E, bias, E, k, from_logits, lane, my_id, my_gate);
   if (lane < k) {
     ids[(int64_t)warp * k + lane] = my_id;
-    gates[(int64_t)warp * k + lane] = my_gate / gsum;
+    gates[(int64_t)warp * k + lane] = my_gate;
+  }
+}
+
+// Few tokens (Tk <= 32, Tk * k <= 1024, E <= 256): top-k and the stable per-expert permutation in one CTA of
+// 1024 threads. Assignment a = t * k + j; chunk c = a / 32 is handled by one warp, whose lanes with the same expert
+// find each other with __match_any_sync: an assignment's position is offsets[e] + (assignments of e in earlier
+// chunks) + (lanes of e before it in its chunk), which is the order of a, as in the general permutation kernel.
+template <int PER>
+__global__ void __launch_bounds__(1024) route_small_kernel(float* __restrict__ scores, const float* __restrict__ bias,
+                                                           int Tk, int E, int k, int from_logits,
+                                                           int32_t* __restrict__ ids, float* __restrict__ gates,
+                                                           int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                                                           int32_t* __restrict__ perm, int32_t* __restrict__ inv) {
+  pdl_enter();
+  extern __shared__ int rs_sm[];
+  const int n = Tk * k, W = (n + 31) / 32;
+  int* hist = rs_sm;                 // [W][E]: counts per chunk, then their exclusive prefix over chunks
+  int* ids_s = hist + W * E;         // [n]
+  int* rk_s = ids_s + n;             // [n]: rank among the chunk's lanes with the same expert
+  int* off_s = rk_s + n;             // [E]
+  __shared__ int wtot[32];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nw = blockDim.x >> 5;
+  for (int i = tid; i < W * E; i += blockDim.x) hist[i] = 0;
+  for (int t = warp; t < Tk; t += nw) {
+    int my_id;
+    float my_gate;
+    warp_topk<PER>(scores + (int64_t)t * E, bias, E, k, from_logits, lane, my_id, my_gate);
+    if (lane < k) {
+      ids[(int64_t)t * k + lane] = my_id;
+      gates[(int64_t)t * k + lane] = my_gate;
+      ids_s[t * k + lane] = my_id;
+    }
+  }
+  __syncthreads();
+  for (int c = warp; c < W; c += nw) {
+    const int a = c * 32 + lane;
+    const int ex = a < n ? ids_s[a] : -1;
+    const unsigned grp = __match_any_sync(0xffffffffu, ex);
+    if (a < n) {
+      rk_s[a] = __popc(grp & ((1u << lane) - 1u));
+      if (lane == __ffs(grp) - 1) hist[c * E + ex] = __popc(grp);
+    }
+  }
+  __syncthreads();
+  // per expert: prefix over chunks, total count
+  for (int ex = tid; ex < E; ex += blockDim.x) {
+    int run = 0;
+    for (int c = 0; c < W; ++c) {
+      const int h = hist[c * E + ex];
+      hist[c * E + ex] = run;
+      run += h;
+    }
+    off_s[ex] = run;
+  }
+  __syncthreads();
+  // exclusive scan of the counts over experts (E <= 1024 = one entry per thread)
+  const int cnt = tid < E ? off_s[tid] : 0;
+  int inc = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += y;
+  }
+  if (lane == 31) wtot[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    int x = lane < nw ? wtot[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    wtot[lane] = x;   // inclusive over warps
+  }
+  __syncthreads();
+  const int excl = inc - cnt + (warp > 0 ? wtot[warp - 1] : 0);
+  __syncthreads();
+  if (tid < E) {
+    off_s[tid] = excl;
+    counts[tid] = cnt;
+    offsets[tid] = excl;
+  }
+  if (tid == 0) offsets[E] = n;
+  __syncthreads();
+  for (int a = tid; a < n; a += blockDim.x) {
+    const int ex = ids_s[a];
+    const int pos = off_s[ex] + hist[(a >> 5) * E + ex] + rk_s[a];
+    perm[pos] = a;
+    inv[a] = pos;
   }
 }
 
@@ -226,6 +355,42 @@ __global__ void route_permute_kernel(const int32_t* __restrict__ ids, int n_assi
 
 }  // namespace
 
+template <int PER>
+int launch_select_per(float* scores, const float* bias, int Tk, int E, int k, int from_logits, int32_t* ids,
+                      float* gates, int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv, cudaStream_t s) {
+  if constexpr (PER <= 8) {   // E <= 256: the single-CTA kernel fits its 64 registers per thread
+    const int n = Tk * k, W = (n + 31) / 32;
+    const size_t smem = ((size_t)W * E + 2 * (size_t)n + E) * sizeof(int);
+    if (Tk <= 32 && n <= 1024 && smem <= 96 * 1024) {
+      static bool cfg = false;
+      if (!cfg) {
+        cudaFuncSetAttribute(route_small_kernel<PER>, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
+        cfg = true;
+      }
+      launch_pdl(route_small_kernel<PER>, 1, 1024, smem, s, scores, bias, Tk, E, k, from_logits, ids, gates, counts,
+                 offsets, perm, inv);
+      DLLM_CHECK_LAUNCH("route_small_kernel");
+      return DLLM_OK;
+    }
+  }
+  launch_pdl(route_topk_kernel<PER>, (Tk + 7) / 8, 256, 0, s, scores, bias, Tk, E, k, from_logits, ids, gates);
+  DLLM_CHECK_LAUNCH("route_topk_kernel");
+  launch_pdl(route_permute_kernel, E, 256, 0, s, (const int32_t*)ids, Tk * k, E, counts, offsets, perm, inv);
+  DLLM_CHECK_LAUNCH("route_permute_kernel");
+  return DLLM_OK;
+}
+
+// Selection and permutation from fp32 scores (sigmoid applied here when from_logits), E <= 1024.
+int launch_select(float* scores, const float* bias, int Tk, int E, int k, int from_logits, int32_t* ids,
+                  float* gates, int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv, cudaStream_t s) {
+  if (E <= 32) return launch_select_per<1>(scores, bias, Tk, E, k, from_logits, ids, gates, counts, offsets, perm, inv, s);
+  if (E <= 64) return launch_select_per<2>(scores, bias, Tk, E, k, from_logits, ids, gates, counts, offsets, perm, inv, s);
+  if (E <= 128) return launch_select_per<4>(scores, bias, Tk, E, k, from_logits, ids, gates, counts, offsets, perm, inv, s);
+  if (E <= 256) return launch_select_per<8>(scores, bias, Tk, E, k, from_logits, ids, gates, counts, offsets, perm, inv, s);
+  if (E <= 512) return launch_select_per<16>(scores, bias, Tk, E, k, from_logits, ids, gates, counts, offsets, perm, inv, s);
+  return launch_select_per<32>(scores, bias, Tk, E, k, from_logits, ids, gates, counts, offsets, perm, inv, s);
+}
+
 int launch_route(int dtype, const void* h, const void* w_router, const float* bias, int Tk, int H, int E, int k,
                  int32_t* ids, float* gates, float* scores, int32_t* counts, int32_t* offsets, int32_t* perm,
                  int32_t* inv, cudaStream_t s) {
@@ -240,11 +405,7 @@ int launch_route(int dtype, const void* h, const void* w_router, const float* bi
     g.epi.kind = EPI_STORE; g.epi.out = scores; g.epi.ldo = E; g.epi.out_f32 = 1;
     int st = gemm_bf16_tc(g, s);
     if (st) return st;
-    launch_pdl(route_topk_kernel, (Tk + 7) / 8, 256, 0, s, scores, bias, Tk, E, k, 1, ids, gates);
-    DLLM_CHECK_LAUNCH("route_topk_kernel");
-    launch_pdl(route_permute_kernel, E, 256, 0, s, ids, Tk * k, E, counts, offsets, perm, inv);
-    DLLM_CHECK_LAUNCH("route_permute_kernel");
-    return DLLM_OK;
+    return launch_select(scores, bias, Tk, E, k, 1, ids, gates, counts, offsets, perm, inv, s);
   }
   dim3 g1((E + EW - 1) / EW, (Tk + TT - 1) / TT);
   const size_t smem = (size_t)TT * H * (dtype == DLLM_BF16 ? 2 : 4);
@@ -266,11 +427,7 @@ int launch_route(int dtype, const void* h, const void* w_router, const float* bi
     launch_pdl(route_scores_kernel<float>, g1, 256, smem, s, (const float*)h, (const float*)w_router, Tk, H, E, scores);
   }
   DLLM_CHECK_LAUNCH("route_scores_kernel");
-  launch_pdl(route_topk_kernel, (Tk + 7) / 8, 256, 0, s, scores, bias, Tk, E, k, 0, ids, gates);
-  DLLM_CHECK_LAUNCH("route_topk_kernel");
-  launch_pdl(route_permute_kernel, E, 256, 0, s, ids, Tk * k, E, counts, offsets, perm, inv);
-  DLLM_CHECK_LAUNCH("route_permute_kernel");
-  return DLLM_OK;
+  return launch_select(scores, bias, Tk, E, k, 0, ids, gates, counts, offsets, perm, inv, s);
 }
 
 }  // namespace dllm

@@ -87,7 +87,8 @@ def test_gemm_f32():
 # ------------------------------------------------------------------------------------------------ router
 @pytest.mark.parametrize("dtype,Tk,H,E,k", [("bf16", 1, 2048, 256, 8), ("bf16", 32, 2048, 256, 8),
                                             ("bf16", 77, 2048, 256, 8), ("bf16", 512, 2048, 256, 8),
-                                            ("f32", 16, 256, 8, 2), ("bf16", 9, 256, 1024, 32)])
+                                            ("f32", 16, 256, 8, 2), ("bf16", 9, 256, 1024, 32),
+                                            ("bf16", 20, 256, 512, 8), ("f32", 32, 128, 64, 32)])
 def test_route(dtype, Tk, H, E, k):
     t = _tdt(dtype)
     h = synth.normal((Tk, H), 1.0, 5, f"rh{Tk}", DEV, t)

@@ -90,10 +90,21 @@ int expert_bn_hint(int Tk, int k, int E) {
   return std::min(Tk, std::max(64, 4 * avg));
 }
 
+// The combine's follow-up RMSNorm, fused into it (PostNorm::g == nullptr: plain combine).
+struct PostNorm {
+  const void* g = nullptr;
+  float eps = 0.f;
+  void* out = nullptr;
+  int mode = NORM_NEXT;
+  const uint8_t* mask = nullptr;   // NORM_FINAL: block mask, positions per half, masked count
+  int n_half_pos = 0;
+  const int32_t* n_dev = nullptr;
+};
+
 int run_experts(int dtype, int Tk, int H, int E, int k, int I, const void* h, const void* w_gu, const void* w_down,
                 const void* w_gu_s, const void* w_down_s, const int32_t* counts, const int32_t* offsets,
                 const int32_t* perm, const int32_t* inv, const float* gates, void* x, const ExpertBufs& b,
-                int32_t* status, cudaStream_t s) {
+                int32_t* status, cudaStream_t s, const PostNorm& pn = PostNorm()) {
   const int shared = w_gu_s != nullptr;
   const int n_assign = Tk * k;
   const int64_t rows = (int64_t)n_assign + (shared ? Tk : 0);
@@ -118,7 +129,16 @@ int run_experts(int dtype, int Tk, int H, int E, int k, int I, const void* h, co
   g2.epi.kind = EPI_STORE; g2.epi.out = b.y; g2.epi.ldo = H; g2.epi.out_f32 = 1;
   st = run_gemm(g2, s);
   if (st) return st;
+  if (pn.g)
+    return launch_combine_norm(dtype, x, b.y, gates, inv, k, Tk, shared, H, pn.g, pn.eps, pn.out, pn.mode, pn.mask,
+                               pn.n_half_pos, pn.n_dev, s);
   return launch_combine(dtype, x, b.y, gates, inv, k, Tk, shared, H, s);
+}
+
+// Rows the fused row kernels handle: 16-byte vectors, at most kRowVecs of them per thread of a 256-thread CTA.
+static bool fused_rows_ok(int dtype, int H) {
+  const int ve = dtype == DLLM_BF16 ? 8 : 4;
+  return H % ve == 0 && H / ve <= kRowVecs * 256;
 }
 
 // ------------------------------------------------------------------------------------------------ step plan
@@ -506,12 +526,21 @@ int dllm_denoise_step(const dllm_model* m, const dllm_state* st, const dllm_step
     if (_r) return _r;    \
   } while (0)
 
-  if (!p->commit) TRY(launch_masked_rows(st->mask, s.Bl * L, s.halves, s.row_pos, s.n_rows, stream));
-  TRY(launch_embed(dt, st->tokens, p->commit ? nullptr : st->mask, m->mask_id, m->embed, s.x, s.Tk, H, stream));
+  const bool fuse = fused_rows_ok(dt, H);
+  if (fuse) {
+    // embedding, layer 0's attention-input norm and (denoising passes) the masked-row list in one launch
+    TRY(launch_embed_norm(dt, st->tokens, p->commit ? nullptr : st->mask, m->mask_id, m->embed, s.x, s.h,
+                          m->layers[0].attn_norm, s.Tk, H, m->eps, st->mask, s.Bl * L, s.halves,
+                          p->commit ? nullptr : s.row_pos, s.n_rows, stream));
+  } else {
+    if (!p->commit) TRY(launch_masked_rows(st->mask, s.Bl * L, s.halves, s.row_pos, s.n_rows, stream));
+    TRY(launch_embed(dt, st->tokens, p->commit ? nullptr : st->mask, m->mask_id, m->embed, s.x, s.Tk, H, stream));
+  }
   for (int l = 0; l < m->n_layers; ++l) {
     const dllm_layer& Ly = m->layers[l];
     const bool last = l == m->n_layers - 1;
-    TRY(launch_rmsnorm(dt, s.x, Ly.attn_norm, s.h, s.Tk, H, m->eps, nullptr, nullptr, 0, 0, stream));
+    // the attention-input norm comes fused with the embedding (layer 0) or the previous layer's combine
+    if (!fuse) TRY(launch_rmsnorm(dt, s.x, Ly.attn_norm, s.h, s.Tk, H, m->eps, nullptr, nullptr, 0, 0, stream));
     if (p->sprint && p->retain) {
       RetainArgs ra;
       ra.B = st->B; ra.Hkv = m->Hkv; ra.d = m->d; ra.P = P; ra.cap = st->cap; ra.n_keep = p->n_keep;
@@ -551,13 +580,21 @@ int dllm_denoise_step(const dllm_model* m, const dllm_state* st, const dllm_step
     TRY(launch_rmsnorm(dt, s.x, Ly.ffn_norm, s.h, s.Tk, H, m->eps, nullptr, nullptr, 0, 0, stream));
     TRY(launch_route(dt, s.h, Ly.w_router, Ly.router_bias, s.Tk, H, m->E, m->k, s.ids, s.gates, s.scores, s.counts,
                      s.offsets, s.perm, s.inv, stream));
+    PostNorm pn;
+    if (fuse && !last) {           // next layer's attention-input norm
+      pn.g = m->layers[l + 1].attn_norm; pn.eps = m->eps; pn.out = s.h; pn.mode = NORM_NEXT;
+    } else if (fuse && !p->commit) {   // final norm of the still-masked rows, in the LM head's row order
+      pn.g = m->final_norm; pn.eps = m->eps; pn.out = s.xf; pn.mode = NORM_FINAL; pn.mask = st->mask;
+      pn.n_half_pos = s.Bl * L; pn.n_dev = s.n_rows;
+    }
     TRY(run_experts(dt, s.Tk, H, m->E, m->k, m->I, s.h, Ly.w_gu, Ly.w_down, Ly.w_gu_shared, Ly.w_down_shared,
-                    s.counts, s.offsets, s.perm, s.inv, s.gates, s.x, s.eb, status, stream));
+                    s.counts, s.offsets, s.perm, s.inv, s.gates, s.x, s.eb, status, stream, pn));
   }
   if (p->commit) return DLLM_OK;
-  // final norm on the masked rows (cond, then uncond), LM head, confidence + unmasking
-  TRY(launch_rmsnorm(dt, s.x, m->final_norm, s.xf, s.halves * s.max_rows, H, m->eps, s.row_pos, s.n_rows,
-                     p->cfg, s.Bl * L, stream));
+  // final norm on the masked rows (cond, then uncond) unless fused above, LM head, confidence + unmasking
+  if (!fuse)
+    TRY(launch_rmsnorm(dt, s.x, m->final_norm, s.xf, s.halves * s.max_rows, H, m->eps, s.row_pos, s.n_rows,
+                       p->cfg, s.Bl * L, stream));
   GemmArgs gl;
   gl.x = s.xf; gl.x_rows = (int64_t)s.halves * s.max_rows;
   gl.w = static_cast<const char*>(m->w_lm) + (size_t)p->vocab_offset * H * es; gl.w_rows = s.vlen;

@@ -234,6 +234,208 @@ int launch_combine(int dtype, void* x, const float* y, const float* gates, const
   return DLLM_OK;
 }
 
+// ------------------------------------------------------------------------------------------------ fused rows
+// The step's row-wise stages that end in an RMSNorm are fused with the norm: the kernel that produces a residual
+// row keeps it in registers and writes both the row and its normalised copy, saving a launch and a re-read.
+// norm: out = v / sqrt(mean(v^2) + eps) * g in fp32 over the row as stored (rounded to T).
+
+// Sum over the CTA (256 threads) of one float per thread; every thread gets the total.
+DLLM_DEV float block_sum256(float v, float* red) {
+  v = warp_sum(v);
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float t = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) t += red[i];
+  return t;
+}
+
+template <typename T>
+DLLM_DEV void store_norm_row(const uint4* keep, int nvec, float inv, const T* __restrict__ g, T* __restrict__ o) {
+  constexpr int VE = 16 / sizeof(T);
+#pragma unroll
+  for (int k = 0; k < kRowVecs; ++k) {
+    const int i = threadIdx.x + k * 256;
+    if (i < nvec) {
+      const uint4 gv = reinterpret_cast<const uint4*>(g)[i];
+      const T* e = reinterpret_cast<const T*>(&keep[k]);
+      const T* ge = reinterpret_cast<const T*>(&gv);
+      uint4 res;
+      T* re = reinterpret_cast<T*>(&res);
+#pragma unroll
+      for (int u = 0; u < VE; ++u) re[u] = from_f32<T>(to_f32(e[u]) * inv * to_f32(ge[u]));
+      reinterpret_cast<uint4*>(o)[i] = res;
+    }
+  }
+}
+
+// CTA t < rows: x[t] = embed[mask[t] ? mask_id : tokens[t]] and h[t] = norm(x[t]) * g. With the masked-row list
+// requested, one extra CTA writes it (the ascending still-masked positions of the first n_pos, their count and
+// count * halves), as masked_rows_kernel does.
+template <typename T>
+__global__ void __launch_bounds__(256) embed_norm_kernel(const int32_t* __restrict__ tokens,
+                                                         const uint8_t* __restrict__ mask, int mask_id,
+                                                         const T* __restrict__ table, T* __restrict__ x,
+                                                         T* __restrict__ h, const T* __restrict__ g, int rows, int H,
+                                                         float eps, const uint8_t* __restrict__ list_mask, int n_pos,
+                                                         int halves, int32_t* row_pos, int32_t* n_out) {
+  pdl_enter();
+  __shared__ float red[8];
+  if ((int)blockIdx.x == rows) {
+    __shared__ int warp_tot[8];
+    __shared__ int base;
+    if (threadIdx.x == 0) base = 0;
+    __syncthreads();
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    for (int c0 = 0; c0 < n_pos; c0 += 256) {
+      const int p = c0 + threadIdx.x;
+      const int f = (p < n_pos && list_mask[p]) ? 1 : 0;
+      const unsigned bal = __ballot_sync(0xffffffffu, f);
+      if (lane == 0) warp_tot[w] = __popc(bal);
+      __syncthreads();
+      int before = 0, tot = 0;
+      for (int i = 0; i < 8; ++i) {
+        if (i < w) before += warp_tot[i];
+        tot += warp_tot[i];
+      }
+      if (f) row_pos[base + before + __popc(bal & ((1u << lane) - 1u))] = p;
+      __syncthreads();
+      if (threadIdx.x == 0) base += tot;
+      __syncthreads();
+    }
+    if (threadIdx.x == 0) {
+      n_out[0] = base;
+      n_out[1] = base * halves;
+    }
+    return;
+  }
+  constexpr int VE = 16 / sizeof(T);
+  const int t = blockIdx.x;
+  const int id = (mask && mask[t]) ? mask_id : tokens[t];
+  const uint4* src = reinterpret_cast<const uint4*>(table + (int64_t)id * H);
+  uint4* dst = reinterpret_cast<uint4*>(x + (int64_t)t * H);
+  const int nvec = H / VE;
+  uint4 keep[kRowVecs];
+  float ss = 0.f;
+#pragma unroll
+  for (int k = 0; k < kRowVecs; ++k) {
+    const int i = threadIdx.x + k * 256;
+    if (i < nvec) {
+      keep[k] = src[i];
+      dst[i] = keep[k];
+      const T* e = reinterpret_cast<const T*>(&keep[k]);
+#pragma unroll
+      for (int u = 0; u < VE; ++u) {
+        const float v = to_f32(e[u]);
+        ss += v * v;
+      }
+    }
+  }
+  ss = block_sum256(ss, red);
+  store_norm_row<T>(keep, nvec, 1.0f / sqrtf(ss / (float)H + eps), g, h + (int64_t)t * H);
+}
+
+int launch_embed_norm(int dtype, const int32_t* tokens, const uint8_t* mask, int mask_id, const void* table, void* x,
+                      void* h, const void* g, int rows, int H, float eps, const uint8_t* list_mask, int n_pos,
+                      int halves, int32_t* row_pos, int32_t* n_out, cudaStream_t s) {
+  if (rows <= 0) return DLLM_OK;
+  const int ctas = rows + (row_pos ? 1 : 0);
+  if (dtype == DLLM_BF16)
+    launch_pdl(embed_norm_kernel<__nv_bfloat16>, ctas, 256, 0, s, tokens, mask, mask_id,
+               (const __nv_bfloat16*)table, (__nv_bfloat16*)x, (__nv_bfloat16*)h, (const __nv_bfloat16*)g, rows, H,
+               eps, list_mask, n_pos, halves, row_pos, n_out);
+  else
+    launch_pdl(embed_norm_kernel<float>, ctas, 256, 0, s, tokens, mask, mask_id, (const float*)table, (float*)x,
+               (float*)h, (const float*)g, rows, H, eps, list_mask, n_pos, halves, row_pos, n_out);
+  DLLM_CHECK_LAUNCH("embed_norm_kernel");
+  return DLLM_OK;
+}
+
+// CTA t: x[t] += y[Tk*k + t] + sum_j gates[t, j] * y[inv[t*k + j]] (fp32, slot order, rounded once), then the
+// norm of the new row: mode NORM_NEXT writes out[t] (the next layer's attention input); mode NORM_FINAL writes the
+// final-norm row of a still-masked position only, at its place in the LM head's row list (rank among the masked
+// positions of its half, plus n for the unconditional half), which is the order masked_rows_kernel produces.
+template <typename T>
+__global__ void __launch_bounds__(256) combine_norm_kernel(T* __restrict__ x, const float* __restrict__ y,
+                                                           const float* __restrict__ gates,
+                                                           const int32_t* __restrict__ inv, int k, int n_assign,
+                                                           int shared, int H, const T* __restrict__ g, float eps,
+                                                           T* __restrict__ out, int mode,
+                                                           const uint8_t* __restrict__ mask, int n_half_pos,
+                                                           const int32_t* __restrict__ n_dev) {
+  pdl_enter();
+  __shared__ float red[8];
+  constexpr int VE = 16 / sizeof(T);
+  const int t = blockIdx.x;
+  const int nvec = H / VE;
+  T* xr = x + (int64_t)t * H;
+  uint4 keep[kRowVecs];
+  float ss = 0.f;
+#pragma unroll
+  for (int kk = 0; kk < kRowVecs; ++kk) {
+    const int i = threadIdx.x + kk * 256;
+    if (i < nvec) {
+      const int h0 = i * VE;
+      float acc[VE];
+#pragma unroll
+      for (int u = 0; u < VE; u += 4) {
+        const float4 v = shared ? *reinterpret_cast<const float4*>(y + (int64_t)(n_assign + t) * H + h0 + u)
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+        acc[u] = v.x; acc[u + 1] = v.y; acc[u + 2] = v.z; acc[u + 3] = v.w;
+      }
+      for (int j = 0; j < k; ++j) {
+        const float gj = gates[t * k + j];
+        const float* yr = y + (int64_t)inv[t * k + j] * H + h0;
+#pragma unroll
+        for (int u = 0; u < VE; u += 4) {
+          const float4 v = *reinterpret_cast<const float4*>(yr + u);
+          acc[u] += gj * v.x; acc[u + 1] += gj * v.y; acc[u + 2] += gj * v.z; acc[u + 3] += gj * v.w;
+        }
+      }
+      uint4 xv = reinterpret_cast<const uint4*>(xr)[i];
+      T* e = reinterpret_cast<T*>(&xv);
+#pragma unroll
+      for (int u = 0; u < VE; ++u) {
+        e[u] = from_f32<T>(to_f32(e[u]) + acc[u]);
+        const float v = to_f32(e[u]);
+        ss += v * v;
+      }
+      reinterpret_cast<uint4*>(xr)[i] = xv;
+      keep[kk] = xv;
+    }
+  }
+  int row = t;
+  if (mode == NORM_FINAL) {
+    // rank of this position among the masked positions of its half (counted by the whole CTA)
+    const int half = t / n_half_pos, tp = t - half * n_half_pos;
+    int c = 0;
+    for (int p = threadIdx.x; p < tp; p += 256) c += mask[p] ? 1 : 0;
+    const float tot = block_sum256((float)c, red);
+    if (!mask[tp]) {
+      ss = block_sum256(ss, red);   // every thread takes part in the reductions, then none of them writes
+      return;
+    }
+    row = (int)tot + half * n_dev[0];
+  }
+  ss = block_sum256(ss, red);
+  store_norm_row<T>(keep, nvec, 1.0f / sqrtf(ss / (float)H + eps), g, out + (int64_t)row * H);
+}
+
+int launch_combine_norm(int dtype, void* x, const float* y, const float* gates, const int32_t* inv, int k, int Tk,
+                        int shared, int H, const void* g, float eps, void* out, int mode, const uint8_t* mask,
+                        int n_half_pos, const int32_t* n_dev, cudaStream_t s) {
+  if (Tk <= 0) return DLLM_OK;
+  if (dtype == DLLM_BF16)
+    launch_pdl(combine_norm_kernel<__nv_bfloat16>, Tk, 256, 0, s, (__nv_bfloat16*)x, y, gates, inv, k, Tk * k, shared,
+               H, (const __nv_bfloat16*)g, eps, (__nv_bfloat16*)out, mode, mask, n_half_pos, n_dev);
+  else
+    launch_pdl(combine_norm_kernel<float>, Tk, 256, 0, s, (float*)x, y, gates, inv, k, Tk * k, shared, H,
+               (const float*)g, eps, (float*)out, mode, mask, n_half_pos, n_dev);
+  DLLM_CHECK_LAUNCH("combine_norm_kernel");
+  return DLLM_OK;
+}
+
 // ------------------------------------------------------------------------------------------------ fp32 path
 // SIMT GEMM over groups: raw[row, f] = sum_k X[row, k] W[g * wstride + f, k], f < Mw, fp32 throughout.
 // Tiles of 32 rows x 64 features, 256 threads, 2 x 4 outputs per thread.

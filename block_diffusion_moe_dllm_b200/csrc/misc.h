@@ -16,6 +16,15 @@ int launch_gather_rows(int dtype, const void* h, const int32_t* perm, int k, int
                        cudaStream_t s);
 int launch_combine(int dtype, void* x, const float* y, const float* gates, const int32_t* inv, int k, int Tk,
                    int shared, int H, cudaStream_t s);
+// Fused row stages (bf16 rows of up to 8192 elements, fp32 up to 4096: kRowVecs 16-byte vectors per thread).
+constexpr int kRowVecs = 4;
+enum NormMode { NORM_NEXT = 0, NORM_FINAL = 1 };
+int launch_embed_norm(int dtype, const int32_t* tokens, const uint8_t* mask, int mask_id, const void* table, void* x,
+                      void* h, const void* g, int rows, int H, float eps, const uint8_t* list_mask, int n_pos,
+                      int halves, int32_t* row_pos, int32_t* n_out, cudaStream_t s);
+int launch_combine_norm(int dtype, void* x, const float* y, const float* gates, const int32_t* inv, int k, int Tk,
+                        int shared, int H, const void* g, float eps, void* out, int mode, const uint8_t* mask,
+                        int n_half_pos, const int32_t* n_dev, cudaStream_t s);
 
 // router
 int num_sms();

@@ -61,6 +61,8 @@ struct KParams {
   const int32_t* cnt_dev;
   EpiParams epi;
   int32_t* status;
+  int prefetch_w;          // 1: dense with at most BN rows, so a CTA's first tile is m-tile = its first tile index and
+                           // its weight stages may be loaded before the kernels ahead of it finish
 };
 
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
@@ -240,7 +242,28 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
     tc::fence_mbar_init();
   }
   if (warp == 1) tc::tmem_alloc(&sm.tmem_base, 2 * BN);
-  // everything above is on-chip set-up; the group counts below come from the kernels before this one
+  __syncthreads();
+  // Weights are never written by the kernels ahead of this one: the first tile's first weight stages can stream
+  // in before the dependency wait (their transaction bytes are expected now; the arrival, with the activation
+  // bytes, comes in the producer loop). Every lane of warp 0 derives the same count.
+  const int kblocks = p.K / BK;
+  int npf = 0;
+  if (p.prefetch_w) {
+    const int t0 = p.ksplit > 1 ? (int)blockIdx.y : (int)blockIdx.x;
+    const int ks0 = p.ksplit > 1 ? (int)blockIdx.x : 0;
+    const int kb0 = ks0 * kblocks / p.ksplit, kb1 = (ks0 + 1) * kblocks / p.ksplit;
+    if (t0 < p.m_tiles) npf = min(STAGES, kb1 - kb0);
+    if (warp == 0 && npf > 0 && tc::elect_one()) {
+      tc::prefetch_tmap(&tmap_w);
+      const uint64_t pol_w = tc::policy_evict_first();
+      for (int i = 0; i < npf; ++i) {
+        tc::mbar_expect_tx(&sm.full[i], A_BYTES);
+        tc::tma_load_2d(stages + i * STAGE_BYTES, &tmap_w, (kb0 + i) * BK, t0 * 128, &sm.full[i], pol_w);
+      }
+    }
+  }
+  // everything above reads only the weights and on-chip state; the group counts below come from the kernels
+  // before this one
   pdl_enter();
   // ---- group table: counts, offsets and the exclusive prefix of tiles per group
   for (int g = tid; g < n_groups; g += NUM_THREADS) {
@@ -295,7 +318,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
   const int wk_begin = p.ksplit > 1 ? (int)(blockIdx.y * p.ksplit + blockIdx.x) : (int)blockIdx.x;
   const int wk_step = p.ksplit > 1 ? total : (int)gridDim.x;
   volatile int* abort_flag = &sm.abort_flag;
-  const int kblocks = p.K / BK;
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
@@ -324,12 +346,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
           if (!wait_bar(&sm.empty[s], ph ^ 1, abort_flag, p.status, ST_TIMEOUT_PRODUCER)) { ok = false; break; }
           uint8_t* a = stages + s * STAGE_BYTES;
           uint8_t* b = a + A_BYTES;
+          if (it < (uint32_t)npf) {   // weight stage already in flight: arrive with the activation bytes
+            tc::mbar_arrive_expect_tx(&sm.full[s], bytes - A_BYTES);
+          } else {
           tc::mbar_arrive_expect_tx(&sm.full[s], bytes);
           if (p.swiglu) {
             tc::tma_load_2d(a, wm, kb * BK, (int)(wrow + mt * 64), &sm.full[s], pol_w);
             tc::tma_load_2d(a + A_BYTES / 2, wm, kb * BK, (int)(wrow + p.M + mt * 64), &sm.full[s], pol_w);
           } else {
             tc::tma_load_2d(a, wm, kb * BK, (int)(wrow + mt * 128), &sm.full[s], pol_w);
+          }
           }
           for (int j = 0; j < nb; ++j)
             tc::tma_load_2d(b + j * XBOX_BYTES, &tmap_x, kb * BK, xrow + j * XBOX_ROWS, &sm.full[s], pol_x);
@@ -339,6 +365,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
         // drain: wait (bounded) for the copies of the last issued stages to land before leaving
         uint32_t first = it > (uint32_t)STAGES ? it - STAGES : 0;
         for (uint32_t i = first; i < it; ++i) tc::mbar_wait(&sm.full[i % STAGES], (i / STAGES) & 1, 1u << 16);
+      }
+      // prefetched weight stages no work item consumed (no rows after all): complete their phase and let the
+      // copies land before the CTA leaves
+      for (uint32_t i = it; i < (uint32_t)npf; ++i) {
+        tc::mbar_arrive(&sm.full[i]);
+        tc::mbar_wait(&sm.full[i], 0, 1u << 16);
       }
     }
   } else if (warp == 1) {
@@ -635,6 +667,7 @@ int gemm_bf16_tc(const GemmArgs& a, cudaStream_t s) {
   const int bn = gemm_bn(a);
   const int ks = gemm_splitk_factor(a, bn);
   kp.ksplit = ks;
+  kp.prefetch_w = (!a.swiglu && !a.n_dev && !a.has_extra && a.host_cnt <= (ks > 1 ? 32 : bn)) ? 1 : 0;
   int st2;
   if (ks > 1) st2 = launch_cluster_splitk(a, mw, mw2, mx, kp, s);
   else if (bn == 32) st2 = launch<32, 9>(a, mw, mw2, mx, kp, s);

@@ -212,6 +212,11 @@ int validate_step(const dllm_model* m, const dllm_state* st, const dllm_step_par
     REQ(m->H % 128 == 0 && m->I % 64 == 0, DLLM_ERR_UNSUPPORTED, "denoise_step: bf16 path needs H %% 128 == 0, I %% 64 == 0");
     REQ(vlen % 128 == 0, DLLM_ERR_UNSUPPORTED, "denoise_step: scored vocabulary must be a multiple of 128");
     REQ(aligned16(m->w_lm) && aligned16(m->embed), DLLM_ERR_ALIGN, "denoise_step: LM head / embedding alignment");
+    for (int l = 0; l < m->n_layers; ++l) {   // the QKV epilogue writes 16-byte vectors into the caches
+      const dllm_layer& L = m->layers[l];
+      REQ(aligned16(L.k_cache) && aligned16(L.v_cache) && (!p->sprint || (aligned16(L.k_thin) && aligned16(L.v_thin))),
+          DLLM_ERR_ALIGN, "layer %d: KV caches must be 16-byte aligned", l);
+    }
   } else {
     REQ(m->d <= 128 && m->d % 4 == 0, DLLM_ERR_UNSUPPORTED, "denoise_step: fp32 path needs d <= 128, d %% 4 == 0");
   }
@@ -324,6 +329,9 @@ int dllm_gemm(const dllm_gemm_desc* d, const void* x, const void* w, void* y, co
   if (d->dtype == DLLM_BF16) {
     REQ(d->K % 64 == 0 && d->M % 128 == 0, DLLM_ERR_UNSUPPORTED, "gemm: bf16 needs K %% 64 == 0 and M %% 128 == 0");
     REQ(aligned16(x) && aligned16(w), DLLM_ERR_ALIGN, "gemm: X and W must be 16-byte aligned");
+    // the epilogue writes 16-byte vectors of 8 (bf16) or 4 (fp32) outputs
+    REQ(aligned16(y) && d->ldy % (d->y_f32 ? 4 : 8) == 0, DLLM_ERR_ALIGN,
+        "gemm: Y must be 16-byte aligned with ldy a multiple of %d", d->y_f32 ? 4 : 8);
   }
   Carver c(ws);
   GemmArgs a;
@@ -406,6 +414,7 @@ int dllm_moe_route(const dllm_route_desc* d, const void* h, const void* w_router
   REQ((size_t)16 * d->H * (d->dtype == DLLM_BF16 ? 2 : 4) <= 200 * 1024, DLLM_ERR_UNSUPPORTED, "moe_route: H too large");
   REQ(d->dtype == DLLM_BF16 || d->dtype == DLLM_F32, DLLM_ERR_INVALID_ARG, "moe_route: bad dtype");
   REQ(aligned16(h) && aligned16(w_router), DLLM_ERR_ALIGN, "moe_route: h and w_router must be 16-byte aligned");
+  REQ(scores == nullptr || aligned16(scores), DLLM_ERR_ALIGN, "moe_route: scores must be 16-byte aligned");
   int st = check_ws(ws, ws_bytes, dllm_moe_route_workspace_size(d));
   if (st) return st;
   Carver c(ws);

@@ -133,80 +133,113 @@ __device__ __forceinline__ void rope_cos_sin(int pos, double inv_freq, float* c,
   sincosf((float)a, s, c);
 }
 
+// Eight consecutive staging values of token column j from feature m0 (two 16-byte shared-memory loads).
+__device__ __forceinline__ void stage8(const float* stage, int j, int m0, float* v) {
+  const float4 a = *reinterpret_cast<const float4*>(stage + j * 128 + m0);
+  const float4 b = *reinterpret_cast<const float4*>(stage + j * 128 + m0 + 4);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+__device__ __forceinline__ uint4 pack_bf16x8(const float* v) {
+  uint4 r;
+  __nv_bfloat162 t;
+  t = __floats2bfloat162_rn(v[0], v[1]); r.x = *reinterpret_cast<uint32_t*>(&t);
+  t = __floats2bfloat162_rn(v[2], v[3]); r.y = *reinterpret_cast<uint32_t*>(&t);
+  t = __floats2bfloat162_rn(v[4], v[5]); r.z = *reinterpret_cast<uint32_t*>(&t);
+  t = __floats2bfloat162_rn(v[6], v[7]); r.w = *reinterpret_cast<uint32_t*>(&t);
+  return r;
+}
+
+// Epilogue of up to STAGE_COLS token columns held in shared memory as stage[j * 128 + m] (m = tile row = output
+// feature). Every thread handles 8 consecutive features of one token, so each output write is one 16-byte store.
+// QKV rows keep their RoPE pair (m, m + 64) in the same thread; inv_freq holds rope_base^(-2 m / 128) of the
+// thread's 8 features m0 .. m0 + 7 (m0 = 8 (tid % 8)).
 template <int BN>
 __device__ void epilogue_chunk(const KParams& p, const float* stage, int g, int mt, int n0, int nval, int c0,
-                               int row0, int tid) {
+                               int row0, int tid, const double* inv_freq) {
   const EpiParams& e = p.epi;
   const int ncols = min(STAGE_COLS, nval - c0);
   if (e.kind == EPI_SWIGLU) {
+    // 64 gate rows then 64 up rows: 8 threads per token, 16 tokens per round
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(e.out);
-    for (int idx = tid; idx < ncols * 64; idx += 128) {
-      int j = idx >> 6, m = idx & 63;
-      float gt = stage[j * 128 + m], up = stage[j * 128 + 64 + m];
-      int64_t row = row0 + n0 + c0 + j;
-      out[row * e.ldo + mt * 64 + m] = __float2bfloat16_rn(silu_f(gt) * up);
+    const int m0 = (tid & 7) * 8;
+    for (int j = tid >> 3; j < ncols; j += 16) {
+      float gt[8], up[8], r[8];
+      stage8(stage, j, m0, gt);
+      stage8(stage, j, 64 + m0, up);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) r[u] = silu_f(gt[u]) * up[u];
+      const int64_t row = row0 + n0 + c0 + j;
+      *reinterpret_cast<uint4*>(out + row * e.ldo + mt * 64 + m0) = pack_bf16x8(r);
     }
   } else if (e.kind == EPI_QKV) {
     // m-tile = one head of d = 128 rows: q heads, then k heads, then v heads. RoPE pairs (i, i + 64).
     const int hh = mt;
     const bool rot = hh < e.Hq + e.Hkv;
-    const int m = tid & 63;
-    const double inv_freq = pow((double)e.rope_base, -2.0 * (double)m / 128.0);
-    for (int idx = tid; idx < ncols * 64; idx += 128) {
-      int j = idx >> 6;
-      int tr = row0 + n0 + c0 + j;  // token row = b * L + i
-      float x1 = stage[j * 128 + m], x2 = stage[j * 128 + 64 + m];
-      float y1 = x1, y2 = x2;
-      if (rot) {
-        float c, s;
-        rope_cos_sin(e.pos0 + tr % e.L, inv_freq, &c, &s);
-        y1 = x1 * c - x2 * s;
-        y2 = x2 * c + x1 * s;
+    const int m0 = (tid & 7) * 8;
+    for (int j = tid >> 3; j < ncols; j += 16) {
+      const int tr = row0 + n0 + c0 + j;  // token row = b * L + i
+      float x1[8], x2[8], y1[8], y2[8];
+      stage8(stage, j, m0, x1);
+      stage8(stage, j, 64 + m0, x2);
+      const int pos = e.pos0 + tr % e.L;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        y1[u] = x1[u];
+        y2[u] = x2[u];
+        if (rot) {
+          float c, sn;
+          rope_cos_sin(pos, inv_freq[u], &c, &sn);
+          y1[u] = x1[u] * c - x2[u] * sn;
+          y2[u] = x2[u] * c + x1[u] * sn;
+        }
       }
-      __nv_bfloat16 b1 = __float2bfloat16_rn(y1), b2 = __float2bfloat16_rn(y2);
+      const uint4 b1 = pack_bf16x8(y1), b2 = pack_bf16x8(y2);
       if (hh < e.Hq) {
         __nv_bfloat16* q = static_cast<__nv_bfloat16*>(e.q_out) + ((int64_t)tr * e.Hq + hh) * 128;
-        q[m] = b1;
-        q[m + 64] = b2;
+        *reinterpret_cast<uint4*>(q + m0) = b1;
+        *reinterpret_cast<uint4*>(q + 64 + m0) = b2;
       } else {
-        int b = tr / e.L, i = tr % e.L;
-        bool is_k = hh < e.Hq + e.Hkv;
-        int gk = is_k ? hh - e.Hq : hh - e.Hq - e.Hkv;
+        const int b = tr / e.L, i = tr % e.L;
+        const bool is_k = hh < e.Hq + e.Hkv;
+        const int gk = is_k ? hh - e.Hq : hh - e.Hq - e.Hkv;
         __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(is_k ? e.k_dst : e.v_dst) +
                              (((int64_t)b * e.Hkv + gk) * e.cap + e.slot0 + i) * 128;
-        dst[m] = b1;
-        dst[m + 64] = b2;
+        *reinterpret_cast<uint4*>(dst + m0) = b1;
+        *reinterpret_cast<uint4*>(dst + 64 + m0) = b2;
         void* d2v = is_k ? e.k_dst2 : e.v_dst2;
         if (d2v) {
           __nv_bfloat16* d2 = static_cast<__nv_bfloat16*>(d2v) + (((int64_t)b * e.Hkv + gk) * e.cap2 + e.slot2 + i) * 128;
-          d2[m] = b1;
-          d2[m + 64] = b2;
+          *reinterpret_cast<uint4*>(d2 + m0) = b1;
+          *reinterpret_cast<uint4*>(d2 + 64 + m0) = b2;
         }
       }
     }
   } else {
-    // thread = output feature m; 8 token rows per round so the residual loads of a round are in flight together
-    const int m = tid;
-    const int64_t col = (int64_t)mt * 128 + m;
-    const int64_t base = (int64_t)(row0 + n0 + c0) * e.ldo + col;
-    for (int j0 = 0; j0 < ncols; j0 += 8) {
-      float res[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        res[u] = 0.f;
-        if (e.kind == EPI_RESID && j0 + u < ncols) {
-          const int64_t off = base + (int64_t)(j0 + u) * e.ldo;
-          res[u] = e.out_f32 ? static_cast<const float*>(e.out)[off]
-                             : __bfloat162float(static_cast<const __nv_bfloat16*>(e.out)[off]);
+    // plain store or residual add: 16 threads per token, 8 tokens per round
+    const int m0 = (tid & 15) * 8;
+    const int64_t col = (int64_t)mt * 128 + m0;
+    for (int j = tid >> 4; j < ncols; j += 8) {
+      float v[8];
+      stage8(stage, j, m0, v);
+      const int64_t off = (int64_t)(row0 + n0 + c0 + j) * e.ldo + col;
+      if (e.out_f32) {
+        float4* o = reinterpret_cast<float4*>(static_cast<float*>(e.out) + off);
+        if (e.kind == EPI_RESID) {
+          const float4 r0 = o[0], r1 = o[1];
+          v[0] += r0.x; v[1] += r0.y; v[2] += r0.z; v[3] += r0.w;
+          v[4] += r1.x; v[5] += r1.y; v[6] += r1.z; v[7] += r1.w;
         }
-      }
+        o[0] = make_float4(v[0], v[1], v[2], v[3]);
+        o[1] = make_float4(v[4], v[5], v[6], v[7]);
+      } else {
+        uint4* o = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(e.out) + off);
+        if (e.kind == EPI_RESID) {
+          float r[8];
+          bf16x8_to_f32(*o, r);
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        if (j0 + u >= ncols) break;
-        const int64_t off = base + (int64_t)(j0 + u) * e.ldo;
-        const float v = stage[(j0 + u) * 128 + m] + res[u];
-        if (e.out_f32) static_cast<float*>(e.out)[off] = v;
-        else static_cast<__nv_bfloat16*>(e.out)[off] = __float2bfloat16_rn(v);
+          for (int u = 0; u < 8; ++u) v[u] += r[u];
+        }
+        *o = pack_bf16x8(v);
       }
     }
   }
@@ -413,6 +446,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
     const int q = warp & 3;          // TMEM lane quadrant this warp may access
     const int row = q * 32 + lane;   // tile row m (TMEM lane)
     const int etid = tid - 64;       // 0..127
+    double inv_freq[8];
+    if (p.epi.kind == EPI_QKV)
+#pragma unroll
+      for (int u = 0; u < 8; ++u) inv_freq[u] = pow((double)p.epi.rope_base, -2.0 * (double)((etid & 7) * 8 + u) / 128.0);
     uint32_t tcount = 0;
     for (int wk = wk_begin; wk < total; wk += wk_step, ++tcount) {
       const int t = wk / p.ksplit;
@@ -431,7 +468,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
 #pragma unroll
           for (int j = 0; j < STAGE_COLS; ++j) staging[j * 128 + row] = v[j];
           tc::named_bar_sync(1, 128);
-          epilogue_chunk<BN>(p, staging, g, mt, n0, nval, c0, sm.grp_off[g], etid);
+          epilogue_chunk<BN>(p, staging, g, mt, n0, nval, c0, sm.grp_off[g], etid, inv_freq);
         }
         tc::fence_before_sync();
         tc::mbar_arrive(&sm.tempty[buf]);
@@ -487,7 +524,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
       cluster_arrive();
       arrived = true;
       tc::named_bar_sync(1, 128);
-      if (ce > cb) epilogue_chunk<BN>(p, red, g, mt, n0 + cb, ce - cb, 0, sm.grp_off[g], etid);
+      double inv_freq[8];
+      if (p.epi.kind == EPI_QKV)
+#pragma unroll
+        for (int u = 0; u < 8; ++u) inv_freq[u] = pow((double)p.epi.rope_base, -2.0 * (double)((etid & 7) * 8 + u) / 128.0);
+      if (ce > cb) epilogue_chunk<BN>(p, red, g, mt, n0 + cb, ce - cb, 0, sm.grp_off[g], etid, inv_freq);
     }
     if (!arrived) cluster_arrive();
     cluster_wait();
@@ -687,11 +728,13 @@ int bn_for(int max_cnt) {
 static bool dense(const GemmArgs& a) { return !a.swiglu && !a.n_dev && !a.has_extra; }
 
 // N tile: the smallest that covers the largest group, except that a dense projection with too few output tiles to
-// occupy the SMs takes narrower N tiles first (the extra re-reads of its weight tiles hit L2).
+// occupy half the SMs takes narrower N tiles first (the extra re-reads of its weight tiles hit L2). Narrower still
+// loses: measured at 512 rows, N tile 128 (96 QKV tiles) beats 64 (192) and 32 (384), whose small MMAs and extra
+// operand traffic cost more than the idle SMs.
 int gemm_bn(const GemmArgs& a) {
   int bn = bn_for(a.max_cnt);
   if (dense(a))
-    while (bn > 32 && (a.M / 128) * ((a.max_cnt + bn - 1) / bn) < 2 * num_sms()) bn /= 2;
+    while (bn > 32 && (a.M / 128) * ((a.max_cnt + bn - 1) / bn) < num_sms() / 2) bn /= 2;
   return bn;
 }
 

@@ -61,6 +61,11 @@ def test_gemm_rejects_bad_arguments(lib):
     d.K = 64
     assert lib.dllm_gemm(C.byref(d), FAKE + 2, FAKE, FAKE, None, FAKE, 1 << 20, None) == bd.ERR_ALIGN
     assert "aligned" in lib.dllm_last_error().decode()
+    # the epilogue stores 16-byte vectors: Y's base and row stride must allow them
+    assert lib.dllm_gemm(C.byref(d), FAKE, FAKE, FAKE + 4, None, FAKE, 1 << 20, None) == bd.ERR_ALIGN
+    d.ldy = 132
+    assert lib.dllm_gemm(C.byref(d), FAKE, FAKE, FAKE, None, FAKE, 1 << 20, None) == bd.ERR_ALIGN
+    assert "ldy" in lib.dllm_last_error().decode()
 
 
 def test_attention_rejects_bad_arguments(lib):

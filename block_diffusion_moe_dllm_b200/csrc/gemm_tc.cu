@@ -17,6 +17,7 @@
 #include "tc.cuh"
 #include "kernels.h"
 #include <cuda.h>
+#include <cmath>
 #include <mutex>
 #include <algorithm>
 
@@ -150,67 +151,71 @@ __device__ __forceinline__ uint4 pack_bf16x8(const float* v) {
 }
 
 // Epilogue of up to STAGE_COLS token columns held in shared memory as stage[j * 128 + m] (m = tile row = output
-// feature). Every thread handles 8 consecutive features of one token, so each output write is one 16-byte store.
-// QKV rows keep their RoPE pair (m, m + 64) in the same thread; inv_freq holds rope_base^(-2 m / 128) of the
-// thread's 8 features m0 .. m0 + 7 (m0 = 8 (tid % 8)).
+// feature). Every thread handles 4 or 8 consecutive features of one token, so each output write is one 8- or
+// 16-byte store; QKV rows keep their RoPE pair (m, m + 64) in the same thread.
 template <int BN>
 __device__ void epilogue_chunk(const KParams& p, const float* stage, int g, int mt, int n0, int nval, int c0,
-                               int row0, int tid, const double* inv_freq) {
+                               int row0, int tid) {
   const EpiParams& e = p.epi;
   const int ncols = min(STAGE_COLS, nval - c0);
   if (e.kind == EPI_SWIGLU) {
-    // 64 gate rows then 64 up rows: 8 threads per token, 16 tokens per round
+    // 64 gate rows then 64 up rows: 16 threads per token (4 features each), 8 tokens per round
     __nv_bfloat16* out = static_cast<__nv_bfloat16*>(e.out);
-    const int m0 = (tid & 7) * 8;
-    for (int j = tid >> 3; j < ncols; j += 16) {
-      float gt[8], up[8], r[8];
-      stage8(stage, j, m0, gt);
-      stage8(stage, j, 64 + m0, up);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) r[u] = silu_f(gt[u]) * up[u];
+    const int m0 = (tid & 15) * 4;
+    for (int j = tid >> 4; j < ncols; j += 8) {
+      const float4 gt = *reinterpret_cast<const float4*>(stage + j * 128 + m0);
+      const float4 up = *reinterpret_cast<const float4*>(stage + j * 128 + 64 + m0);
+      __nv_bfloat162 t0 = __floats2bfloat162_rn(silu_f(gt.x) * up.x, silu_f(gt.y) * up.y);
+      __nv_bfloat162 t1 = __floats2bfloat162_rn(silu_f(gt.z) * up.z, silu_f(gt.w) * up.w);
       const int64_t row = row0 + n0 + c0 + j;
-      *reinterpret_cast<uint4*>(out + row * e.ldo + mt * 64 + m0) = pack_bf16x8(r);
+      *reinterpret_cast<uint2*>(out + row * e.ldo + mt * 64 + m0) =
+          make_uint2(*reinterpret_cast<uint32_t*>(&t0), *reinterpret_cast<uint32_t*>(&t1));
     }
   } else if (e.kind == EPI_QKV) {
-    // m-tile = one head of d = 128 rows: q heads, then k heads, then v heads. RoPE pairs (i, i + 64).
+    // m-tile = one head of d = 128 rows: q heads, then k heads, then v heads. RoPE pairs (i, i + 64); 16 threads
+    // per token (4 pairs each), 8 tokens per round
     const int hh = mt;
     const bool rot = hh < e.Hq + e.Hkv;
-    const int m0 = (tid & 7) * 8;
-    for (int j = tid >> 3; j < ncols; j += 16) {
+    const int m0 = (tid & 15) * 4;
+    for (int j = tid >> 4; j < ncols; j += 8) {
       const int tr = row0 + n0 + c0 + j;  // token row = b * L + i
-      float x1[8], x2[8], y1[8], y2[8];
-      stage8(stage, j, m0, x1);
-      stage8(stage, j, 64 + m0, x2);
+      const float4 a1 = *reinterpret_cast<const float4*>(stage + j * 128 + m0);
+      const float4 a2 = *reinterpret_cast<const float4*>(stage + j * 128 + 64 + m0);
+      const float x1[4] = {a1.x, a1.y, a1.z, a1.w}, x2[4] = {a2.x, a2.y, a2.z, a2.w};
+      float y1[4], y2[4];
       const int pos = e.pos0 + tr % e.L;
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
+      for (int u = 0; u < 4; ++u) {
         y1[u] = x1[u];
         y2[u] = x2[u];
         if (rot) {
           float c, sn;
-          rope_cos_sin(pos, inv_freq[u], &c, &sn);
+          rope_cos_sin(pos, e.inv_freq[m0 + u], &c, &sn);
           y1[u] = x1[u] * c - x2[u] * sn;
           y2[u] = x2[u] * c + x1[u] * sn;
         }
       }
-      const uint4 b1 = pack_bf16x8(y1), b2 = pack_bf16x8(y2);
+      __nv_bfloat162 t0 = __floats2bfloat162_rn(y1[0], y1[1]), t1 = __floats2bfloat162_rn(y1[2], y1[3]);
+      __nv_bfloat162 t2 = __floats2bfloat162_rn(y2[0], y2[1]), t3 = __floats2bfloat162_rn(y2[2], y2[3]);
+      const uint2 b1 = make_uint2(*reinterpret_cast<uint32_t*>(&t0), *reinterpret_cast<uint32_t*>(&t1));
+      const uint2 b2 = make_uint2(*reinterpret_cast<uint32_t*>(&t2), *reinterpret_cast<uint32_t*>(&t3));
       if (hh < e.Hq) {
         __nv_bfloat16* q = static_cast<__nv_bfloat16*>(e.q_out) + ((int64_t)tr * e.Hq + hh) * 128;
-        *reinterpret_cast<uint4*>(q + m0) = b1;
-        *reinterpret_cast<uint4*>(q + 64 + m0) = b2;
+        *reinterpret_cast<uint2*>(q + m0) = b1;
+        *reinterpret_cast<uint2*>(q + 64 + m0) = b2;
       } else {
         const int b = tr / e.L, i = tr % e.L;
         const bool is_k = hh < e.Hq + e.Hkv;
         const int gk = is_k ? hh - e.Hq : hh - e.Hq - e.Hkv;
         __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(is_k ? e.k_dst : e.v_dst) +
                              (((int64_t)b * e.Hkv + gk) * e.cap + e.slot0 + i) * 128;
-        *reinterpret_cast<uint4*>(dst + m0) = b1;
-        *reinterpret_cast<uint4*>(dst + 64 + m0) = b2;
+        *reinterpret_cast<uint2*>(dst + m0) = b1;
+        *reinterpret_cast<uint2*>(dst + 64 + m0) = b2;
         void* d2v = is_k ? e.k_dst2 : e.v_dst2;
         if (d2v) {
           __nv_bfloat16* d2 = static_cast<__nv_bfloat16*>(d2v) + (((int64_t)b * e.Hkv + gk) * e.cap2 + e.slot2 + i) * 128;
-          *reinterpret_cast<uint4*>(d2 + m0) = b1;
-          *reinterpret_cast<uint4*>(d2 + 64 + m0) = b2;
+          *reinterpret_cast<uint2*>(d2 + m0) = b1;
+          *reinterpret_cast<uint2*>(d2 + 64 + m0) = b2;
         }
       }
     }
@@ -446,10 +451,6 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
     const int q = warp & 3;          // TMEM lane quadrant this warp may access
     const int row = q * 32 + lane;   // tile row m (TMEM lane)
     const int etid = tid - 64;       // 0..127
-    double inv_freq[8];
-    if (p.epi.kind == EPI_QKV)
-#pragma unroll
-      for (int u = 0; u < 8; ++u) inv_freq[u] = pow((double)p.epi.rope_base, -2.0 * (double)((etid & 7) * 8 + u) / 128.0);
     uint32_t tcount = 0;
     for (int wk = wk_begin; wk < total; wk += wk_step, ++tcount) {
       const int t = wk / p.ksplit;
@@ -468,7 +469,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
 #pragma unroll
           for (int j = 0; j < STAGE_COLS; ++j) staging[j * 128 + row] = v[j];
           tc::named_bar_sync(1, 128);
-          epilogue_chunk<BN>(p, staging, g, mt, n0, nval, c0, sm.grp_off[g], etid, inv_freq);
+          epilogue_chunk<BN>(p, staging, g, mt, n0, nval, c0, sm.grp_off[g], etid);
         }
         tc::fence_before_sync();
         tc::mbar_arrive(&sm.tempty[buf]);
@@ -524,11 +525,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
       cluster_arrive();
       arrived = true;
       tc::named_bar_sync(1, 128);
-      double inv_freq[8];
-      if (p.epi.kind == EPI_QKV)
-#pragma unroll
-        for (int u = 0; u < 8; ++u) inv_freq[u] = pow((double)p.epi.rope_base, -2.0 * (double)((etid & 7) * 8 + u) / 128.0);
-      if (ce > cb) epilogue_chunk<BN>(p, red, g, mt, n0 + cb, ce - cb, 0, sm.grp_off[g], etid, inv_freq);
+      if (ce > cb) epilogue_chunk<BN>(p, red, g, mt, n0 + cb, ce - cb, 0, sm.grp_off[g], etid);
     }
     if (!arrived) cluster_arrive();
     cluster_wait();
@@ -704,6 +701,8 @@ int gemm_bf16_tc(const GemmArgs& a, cudaStream_t s) {
   kp.grp_cnt = a.grp_cnt;
   kp.cnt_dev = a.cnt_dev;
   kp.epi = a.epi;
+  if (kp.epi.kind == EPI_QKV)
+    for (int m = 0; m < 64; ++m) kp.epi.inv_freq[m] = std::pow((double)kp.epi.rope_base, -2.0 * (double)m / 128.0);
   kp.status = a.status;
   const int bn = gemm_bn(a);
   const int ks = gemm_splitk_factor(a, bn);

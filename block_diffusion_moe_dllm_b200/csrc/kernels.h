@@ -27,6 +27,7 @@ struct EpiParams {
   int cap = 0, slot0 = 0, cap2 = 0, slot2 = 0;
   int Hq = 0, Hkv = 0, d = 0, L = 1, pos0 = 0;
   float rope_base = 10000.f;
+  double inv_freq[64] = {};         // rope_base^(-2 m / 128), m < 64 (filled on the host by gemm_bf16_tc)
 };
 
 // Y = X W^T over groups of X rows. Group g < n_dev reads rows [grp_off[g], grp_off[g] + grp_cnt[g]) of X and

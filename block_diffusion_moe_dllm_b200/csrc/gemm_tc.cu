@@ -603,6 +603,9 @@ int launch(const GemmArgs& a, const CUtensorMap& mw, const CUtensorMap& mw2, con
 }
 
 constexpr int SPLITK_BN = 32, SPLITK_STAGES = 9;
+
+// Output tiles of a dense split-K GEMM: 128-row weight tiles x 32-row N tiles.
+static int splitk_tiles(const GemmArgs& a) { return (a.M / 128) * ((a.host_cnt + SPLITK_BN - 1) / SPLITK_BN); }
 constexpr int SPLITK_SMEM = 1024 + SPLITK_STAGES * (A_BYTES + SPLITK_BN * BK * 2) + STAGING_BYTES + (int)sizeof(Smem);
 
 static cudaError_t configure_splitk() {
@@ -648,7 +651,7 @@ int launch_cluster_splitk(const GemmArgs& a, const CUtensorMap& mw, const CUtens
     if (e != cudaSuccess) return dllm_host::cuda_status(e, "cudaFuncSetAttribute(gemm_tc cluster)");
   }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(kp.ksplit, a.M / 128, 1);
+  cfg.gridDim = dim3(kp.ksplit, splitk_tiles(a), 1);
   cfg.blockDim = dim3(NUM_THREADS, 1, 1);
   cfg.dynamicSmemBytes = SMEM;
   cfg.stream = s;
@@ -741,8 +744,11 @@ int gemm_bn(const GemmArgs& a) {
 // at least two 64-wide blocks, at most 8 (the portable cluster size), and only as many as let every tile's cluster
 // be resident at once (a second wave would double the kernel's time).
 int gemm_splitk_factor(const GemmArgs& a, int bn) {
-  if (a.dtype != DLLM_BF16 || !dense(a) || bn != 32 || a.max_cnt > 32) return 1;
-  const int tiles = a.M / 128;
+  // the grid is (slices, tiles) with the tile count fixed on the host: rows from a device count are excluded,
+  // except that a single N tile stays a single N tile for any count
+  if (a.dtype != DLLM_BF16 || !dense(a) || bn != 32) return 1;
+  if (a.cnt_dev && a.host_cnt > 32) return 1;
+  const int tiles = splitk_tiles(a);
   const int kblocks = a.K / BK;
   if (tiles <= 0 || tiles * 2 > num_sms() || kblocks < 4) return 1;
   int ks = std::max(1, std::min(std::min(kblocks / 2, 8), num_sms() / tiles));

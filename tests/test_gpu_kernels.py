@@ -37,9 +37,11 @@ def test_gemm_bf16_store(N, M, K):
     assert_close(to64(y), want, "bf16", "gemm")
 
 
-@pytest.mark.parametrize("N,M,K", [(32, 3072, 2048), (32, 2048, 2048), (7, 256, 1024)])
+@pytest.mark.parametrize("N,M,K", [(32, 3072, 2048), (32, 2048, 2048), (7, 256, 1024),
+                                   (512, 256, 2048), (77, 256, 512), (100, 512, 1024)])
 def test_gemm_bf16_split_k(N, M, K):
-    """Few output tiles: the K reduction is split across CTAs and summed by the epilogue kernel."""
+    """Few output tiles: the K slices of a tile run as one thread-block cluster and are summed through distributed
+    shared memory (one or several 32-row N tiles, ragged last tile)."""
     x = synth.normal((N, K), 1.0, 9, f"skx{N}", DEV)
     w = synth.normal((M, K), 0.02, 9, f"skw{M}", DEV)
     y0 = synth.normal((N, M), 1.0, 9, f"sky{N}{M}", DEV)

@@ -331,25 +331,29 @@ __global__ void route_permute_kernel(const int32_t* __restrict__ ids, int n_assi
     if (tid == 0) offsets[E] = total;
   }
   if (cnt_e == 0) return;
-  int base = 0;
-  for (int a0 = 0; a0 < n_assign; a0 += blockDim.x) {
-    const int a = a0 + tid;
-    const int f = (a < n_assign && ids[a] == e) ? 1 : 0;
+  // each of the 8 warps takes a contiguous segment of the assignments: count this expert's in it, one prefix
+  // over the warps, then write their positions in order (no block barrier inside the scans)
+  const int seg = (n_assign + 7) / 8;
+  const int s0 = min(n_assign, w * seg), s1 = min(n_assign, s0 + seg);
+  int c = 0;
+  for (int a0 = s0; a0 < s1; a0 += 32) {
+    const int a = a0 + lane;
+    c += __popc(__ballot_sync(0xffffffffu, a < s1 && __ldg(ids + a) == e));
+  }
+  if (lane == 0) wtot[w] = c;
+  __syncthreads();
+  int run = off;
+  for (int i = 0; i < w; ++i) run += wtot[i];
+  for (int a0 = s0; a0 < s1; a0 += 32) {
+    const int a = a0 + lane;
+    const bool f = a < s1 && __ldg(ids + a) == e;
     const unsigned bal = __ballot_sync(0xffffffffu, f);
-    if (lane == 0) wtot[w] = __popc(bal);
-    __syncthreads();
-    int before = 0, tot = 0;
-    for (int i = 0; i < 8; ++i) {
-      if (i < w) before += wtot[i];
-      tot += wtot[i];
-    }
     if (f) {
-      const int r = off + base + before + __popc(bal & ((1u << lane) - 1u));
+      const int r = run + __popc(bal & ((1u << lane) - 1u));
       perm[r] = a;
       inv[a] = r;
     }
-    base += tot;
-    __syncthreads();
+    run += __popc(bal);
   }
 }
 
@@ -373,7 +377,8 @@ int launch_select_per(float* scores, const float* bias, int Tk, int E, int k, in
       return DLLM_OK;
     }
   }
-  launch_pdl(route_topk_kernel<PER>, (Tk + 7) / 8, 256, 0, s, scores, bias, Tk, E, k, from_logits, ids, gates);
+  // one warp per token, 4 per CTA: many tokens spread over all the SMs
+  launch_pdl(route_topk_kernel<PER>, (Tk + 3) / 4, 128, 0, s, scores, bias, Tk, E, k, from_logits, ids, gates);
   DLLM_CHECK_LAUNCH("route_topk_kernel");
   launch_pdl(route_permute_kernel, E, 256, 0, s, (const int32_t*)ids, Tk * k, E, counts, offsets, perm, inv);
   DLLM_CHECK_LAUNCH("route_permute_kernel");

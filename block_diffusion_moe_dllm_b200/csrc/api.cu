@@ -164,6 +164,7 @@ struct StepPlan {
   void* xf;
   void* logits;
   void* partials;
+  int conf_parts;   // > 0: the LM head writes this many confidence partials per row (fused epilogue)
   float* retain_raw;
   size_t total;
 };
@@ -235,6 +236,13 @@ void plan_step(const dllm_model* m, const dllm_state* st, const dllm_step_params
   s.n_keys = p->sprint ? p->n_keep + st->L : st->P + st->L;
   s.max_rows = s.Bl * st->L;
   s.n_chunks = unmask_chunks(s.max_rows, s.vlen);
+  s.conf_parts = 0;
+  if (m->dtype == DLLM_BF16 && !p->cfg) {
+    GemmArgs g;   // the LM head's shape (see the step below)
+    g.dtype = DLLM_BF16; g.K = m->H; g.M = s.vlen; g.host_cnt = s.max_rows; g.max_cnt = s.max_rows;
+    g.cnt_bound = s.max_rows; g.epi.kind = EPI_STORE;
+    s.conf_parts = gemm_conf_parts(g);
+  }
   const int H = m->H, QD = m->Hq * m->d;
   s.x = c.take((size_t)s.Tk * H * es);
   s.h = c.take((size_t)s.Tk * H * es);
@@ -259,7 +267,7 @@ void plan_step(const dllm_model* m, const dllm_state* st, const dllm_step_params
   s.n_rows = c.take<int32_t>(16);
   s.xf = c.take((size_t)s.halves * s.max_rows * H * es);
   s.logits = c.take((size_t)s.halves * s.max_rows * s.vlen * es);
-  s.partials = c.take(unmask_partials_bytes(s.max_rows, s.n_chunks));
+  s.partials = c.take(unmask_partials_bytes(s.max_rows, std::max(s.n_chunks, s.conf_parts)));
   s.retain_raw = p->sprint ? c.take<float>(retain_workspace_bytes(st->B, st->P)) : nullptr;
   s.total = align256(c.off);
 }
@@ -611,13 +619,19 @@ int dllm_denoise_step(const dllm_model* m, const dllm_state* st, const dllm_step
   gl.max_cnt = s.halves * s.max_rows; gl.cnt_bound = s.halves * s.max_rows; gl.dtype = dt; gl.status = status;
   gl.f32_scratch = s.proj_scratch;
   gl.epi.kind = EPI_STORE; gl.epi.out = s.logits; gl.epi.ldo = s.vlen; gl.epi.out_f32 = dt == DLLM_F32;
+  if (s.conf_parts) {   // confidence partials from the LM head's epilogue: no separate reduction pass
+    gl.epi.conf_part = static_cast<ConfPartial*>(s.partials);
+    gl.epi.conf_nparts = s.conf_parts;
+  }
   TRY(run_gemm(gl, stream));
   UnmaskArgs ua;
   ua.B = s.Bl; ua.L = L; ua.V = s.vlen; ua.max_rows = s.max_rows; ua.t = p->t; ua.T_s = p->T_s; ua.mode = p->mode;
   ua.k_max = p->k_max; ua.cfg = p->cfg; ua.vocab_offset = p->vocab_offset; ua.dtype = dt; ua.tau = p->tau;
   ua.cfg_scale = p->cfg_scale; ua.logits = s.logits; ua.row_pos = s.row_pos; ua.n_rows = s.n_rows;
   ua.tokens = st->tokens; ua.mask = st->mask; ua.sel = p->sel; ua.nsel = p->nsel; ua.conf = p->conf;
-  ua.remaining = p->remaining; ua.partials = s.partials; ua.n_chunks = s.n_chunks;
+  ua.remaining = p->remaining; ua.partials = s.partials;
+  ua.n_chunks = s.conf_parts ? s.conf_parts : s.n_chunks;
+  ua.partials_ready = s.conf_parts ? 1 : 0;
   TRY(launch_unmask(ua, stream));
 #undef TRY
   return DLLM_OK;

@@ -250,6 +250,81 @@ __device__ void epilogue_chunk(const KParams& p, const float* stage, int g, int 
   }
 }
 
+// Running confidence partials of the four token rows whose 16-lane group this thread leads (rows (tid >> 4) + 8 i
+// of the single 32-row N tile).
+struct ConfRun {
+  float m[4];
+  int idx[4];
+  double s[4];
+};
+
+__device__ __forceinline__ float ex2_approx(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
+// LM-head epilogue with the confidence reduction fused (single 32-row N tile). Token row j of the tile is handled
+// by the 16 threads with tid >> 4 == j % 8 in round j / 8, each owning 8 consecutive vocabulary rows. The logits are
+// rounded to bf16 and stored, and the partial is taken over the rounded values, as a reduction reading them back
+// would see them: the 8-value maximum with its lowest index and the sum of 2^((z - max) log2 e) in fp32; then the
+// 16 lanes combine by the maximum M, each lane's sum rescaled to M and summed, and the lowest index among the lanes
+// at M. The group's first lane folds that into its running partial (fp64 sum; on equal maxima the lower index,
+// which comes first).
+__device__ __forceinline__ void epilogue_logits_conf(const KParams& p, const float* stage, int mt, int nval,
+                                                     int row0, int tid, ConfRun& run) {
+  __nv_bfloat16* out = static_cast<__nv_bfloat16*>(p.epi.out);
+  const int m0 = (tid & 15) * 8;
+  const int col = mt * 128 + m0;
+  const float log2e = 1.4426950408889634f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int j = (tid >> 4) + 8 * i;
+    const bool act = j < nval;   // uniform over the 16 lanes of the row
+    float lm = -INFINITY, ls = 0.f;
+    int li = 0x7fffffff;
+    if (act) {
+      float v[8];
+      stage8(stage, j, m0, v);
+      const uint4 pk = pack_bf16x8(v);
+      *reinterpret_cast<uint4*>(out + (int64_t)(row0 + j) * p.epi.ldo + col) = pk;
+      float f[8];
+      bf16x8_to_f32(pk, f);
+      lm = f[0];
+      li = 0;
+#pragma unroll
+      for (int q = 1; q < 8; ++q)
+        if (f[q] > lm) { lm = f[q]; li = q; }
+      li += col;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) ls += ex2_approx((f[q] - lm) * log2e);
+    }
+    float hm = lm;
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) hm = fmaxf(hm, __shfl_xor_sync(0xffffffffu, hm, o));
+    float sc = act ? ls * ex2_approx((lm - hm) * log2e) : 0.f;
+    int ci = (act && lm == hm) ? li : 0x7fffffff;
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) {
+      sc += __shfl_xor_sync(0xffffffffu, sc, o);
+      ci = min(ci, __shfl_xor_sync(0xffffffffu, ci, o));
+    }
+    if ((tid & 15) == 0 && act) {
+      if (run.s[i] == 0.0) {
+        run.m[i] = hm; run.idx[i] = ci; run.s[i] = sc;
+      } else if (hm > run.m[i]) {
+        run.s[i] = run.s[i] * (double)expf(run.m[i] - hm) + (double)sc;
+        run.m[i] = hm; run.idx[i] = ci;
+      } else if (hm == run.m[i]) {
+        run.s[i] += (double)sc;
+        run.idx[i] = min(run.idx[i], ci);
+      } else {
+        run.s[i] += (double)sc * (double)expf(hm - run.m[i]);
+      }
+    }
+  }
+}
+
 template <int BN, int STAGES>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_w2,
@@ -451,6 +526,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
     const int q = warp & 3;          // TMEM lane quadrant this warp may access
     const int row = q * 32 + lane;   // tile row m (TMEM lane)
     const int etid = tid - 64;       // 0..127
+    ConfRun run;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) { run.m[i] = -INFINITY; run.idx[i] = 0x7fffffff; run.s[i] = 0.0; }
     uint32_t tcount = 0;
     for (int wk = wk_begin; wk < total; wk += wk_step, ++tcount) {
       const int t = wk / p.ksplit;
@@ -469,6 +547,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
 #pragma unroll
           for (int j = 0; j < STAGE_COLS; ++j) staging[j * 128 + row] = v[j];
           tc::named_bar_sync(1, 128);
+          if constexpr (BN == 32) {
+            if (p.epi.conf_part) {
+              epilogue_logits_conf(p, staging, mt, nval, sm.grp_off[g] + n0, etid, run);
+              continue;
+            }
+          }
           epilogue_chunk<BN>(p, staging, g, mt, n0, nval, c0, sm.grp_off[g], etid);
         }
         tc::fence_before_sync();
@@ -483,6 +567,18 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
         for (int j = 0; j < STAGE_COLS; ++j) staging[j * 128 + row] = v[j];
         tc::fence_before_sync();
         tc::mbar_arrive(&sm.tempty[buf]);
+      }
+    }
+    if constexpr (BN == 32) {
+      // one confidence partial per token row and CTA (empty when this CTA produced no tile of the row)
+      if (p.epi.conf_part && (etid & 15) == 0) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int j = (etid >> 4) + 8 * i;
+          if (j < sm.grp_cnt[0])
+            p.epi.conf_part[(int64_t)(sm.grp_off[0] + j) * p.epi.conf_nparts + blockIdx.x] =
+                ConfPartial{run.m[i], run.idx[i], run.s[i]};
+        }
       }
     }
   }
@@ -709,6 +805,9 @@ int gemm_bf16_tc(const GemmArgs& a, cudaStream_t s) {
   kp.status = a.status;
   const int bn = gemm_bn(a);
   const int ks = gemm_splitk_factor(a, bn);
+  if (a.epi.conf_part)
+    DLLM_REQUIRE(a.epi.conf_nparts > 0 && gemm_conf_parts(a) == a.epi.conf_nparts, DLLM_ERR_UNSUPPORTED,
+                 "gemm: fused confidence epilogue unsupported for this shape");
   kp.ksplit = ks;
   kp.prefetch_w = (!a.swiglu && !a.n_dev && !a.has_extra && a.host_cnt <= (ks > 1 ? 32 : bn)) ? 1 : 0;
   int st2;
@@ -754,6 +853,14 @@ int gemm_splitk_factor(const GemmArgs& a, int bn) {
   int ks = std::max(1, std::min(std::min(kblocks / 2, 8), num_sms() / tiles));
   while (ks > 1 && tiles > max_active_clusters(ks)) --ks;
   return ks;
+}
+
+int gemm_conf_parts(const GemmArgs& a) {
+  if (a.dtype != DLLM_BF16 || !dense(a) || a.epi.kind != EPI_STORE || a.epi.out_f32) return 0;
+  if (a.host_cnt > 32 || a.max_cnt > 32) return 0;
+  const int bn = gemm_bn(a);
+  if (bn != 32 || gemm_splitk_factor(a, bn) != 1) return 0;
+  return num_sms();   // the persistent grid: every CTA writes its slot of every row
 }
 
 int num_sms() {

@@ -13,6 +13,15 @@ enum EpiKind : int {
   EPI_QKV = 3,     // RoPE on q/k heads; q -> q_out, k/v -> cache rows
 };
 
+// Confidence partial of one (token row, vocabulary slice): the slice's largest logit, the lowest vocabulary index
+// attaining it, and the sum over the slice of exp(z - m). Written by the confidence reduction and by the LM head's
+// fused epilogue, merged by the unmask selection.
+struct ConfPartial {
+  float m;
+  int idx;
+  double s;
+};
+
 struct EpiParams {
   int kind = EPI_STORE;
   void* out = nullptr;
@@ -28,6 +37,10 @@ struct EpiParams {
   int Hq = 0, Hkv = 0, d = 0, L = 1, pos0 = 0;
   float rope_base = 10000.f;
   double inv_freq[64] = {};         // rope_base^(-2 m / 128), m < 64 (filled on the host by gemm_bf16_tc)
+  // EPI_STORE of bf16 logits: also the confidence partial of every token row over the vocabulary rows this CTA
+  // produced, at conf_part[row * conf_nparts + CTA index] (only with gemm_conf_parts(...) == conf_nparts)
+  ConfPartial* conf_part = nullptr;
+  int conf_nparts = 0;
 };
 
 // Y = X W^T over groups of X rows. Group g < n_dev reads rows [grp_off[g], grp_off[g] + grp_cnt[g]) of X and
@@ -67,6 +80,11 @@ int gemm_splitk_factor(const GemmArgs& a, int bn);
 
 int gemm_f32_simt(const GemmArgs& a, cudaStream_t s);
 size_t gemm_f32_scratch_bytes(int64_t x_rows, int M, int swiglu);
+
+// Partial slots per token row when the LM-head GEMM described by a (dense, bf16, rows from a device count) can
+// fuse the confidence reduction into its epilogue: one per persistent CTA. 0 when it cannot (more rows than one
+// 32-row N tile, or split-K).
+int gemm_conf_parts(const GemmArgs& a);
 
 int num_sms();
 

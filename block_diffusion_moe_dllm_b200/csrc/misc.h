@@ -48,6 +48,7 @@ struct UnmaskArgs {
   int32_t* remaining;
   void* partials;  // workspace: max_rows * n_chunks entries
   int n_chunks;
+  int partials_ready = 0;  // 1: the partials were written by the LM head's fused epilogue (no reduction launch)
 };
 int unmask_chunks(int max_rows, int V);
 size_t unmask_partials_bytes(int max_rows, int n_chunks);

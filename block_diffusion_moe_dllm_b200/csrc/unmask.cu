@@ -10,6 +10,7 @@
 // fp32), merge in registers and shared memory and write one partial per CTA. Selection: one warp per block row
 // merges its rows' partials, computes c = 1 / sum, counts, ranks and writes tokens, mask and the step outputs.
 #include "common.cuh"
+#include "kernels.h"
 #include "misc.h"
 
 namespace dllm {
@@ -17,12 +18,10 @@ namespace {
 
 constexpr int kRegVpt = 16;                      // 16-byte vectors per thread kept in registers
 constexpr int kRegChunk = kRegVpt * 256 * 8;     // vocabulary entries per CTA of the register path (32768)
+constexpr int kMergeSerial = 8;                  // partials per row merged by one lane; more: a warp per row
 
-struct Partial {
-  float m;    // max logit
-  int idx;    // lowest index attaining m (absolute vocabulary index within the scored slice)
-  double s;   // sum over the chunk of exp(z - m)
-};
+// (max logit, lowest index attaining it within the scored slice, sum over the chunk of exp(z - max))
+using Partial = ConfPartial;
 
 DLLM_DEV void merge(Partial& a, const Partial& b) {
   if (b.s == 0.0) return;
@@ -164,6 +163,18 @@ DLLM_DEV float ex2(float x) {
   return r;
 }
 
+// Merge of the 32 lanes' partials (empty ones have s == 0): the lanes' maximum M, each sum rescaled by
+// 2^((m - M) log2 e), the fp64 sum of those, and the lowest index among the lanes with m == M. Every lane returns
+// the result.
+DLLM_DEV Partial warp_merge(Partial p) {
+  const bool has = p.s != 0.0;
+  const float M = warp_max(has ? p.m : -INFINITY);
+  double s = has ? p.s * (double)ex2((p.m - M) * 1.4426950408889634f) : 0.0;
+  s = warp_sum(s);
+  const int idx = __reduce_min_sync(0xffffffffu, (has && p.m == M) ? p.idx : 0x7fffffff);
+  return Partial{M, idx, s};
+}
+
 // bf16 logits without guidance: each thread keeps its VPT 16-byte vectors of the chunk in registers. Pass 1 finds
 // the maximum with packed bf16x2 max (and the first vector holding it); pass 2 sums exp(z - max) as
 // 2^((z - max) * log2(e)) with the subtraction and the scaling done on fp32 pairs (z - max is exact near the
@@ -231,28 +242,23 @@ __global__ void __launch_bounds__(256) unmask_reduce_bf16_kernel(const __nv_bflo
     Partial q{__bfloat162float(z[v]), v, 1.0};
     merge(p, q);
   }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    Partial q;
-    q.m = __shfl_xor_sync(0xffffffffu, p.m, o);
-    q.idx = __shfl_xor_sync(0xffffffffu, p.idx, o);
-    q.s = __shfl_xor_sync(0xffffffffu, p.s, o);
-    merge(p, q);
-  }
+  // warp, then block: the maximum, every sum rescaled to it, the sum, and the lowest index among the partials
+  // that attain it
+  p = warp_merge(p);
   __shared__ Partial wp[8];
   const int lane = threadIdx.x & 31, wv = threadIdx.x >> 5;
   if (lane == 0) wp[wv] = p;
   __syncthreads();
-  if (threadIdx.x == 0) {
-    Partial a = wp[0];
-    for (int i = 1; i < 8; ++i) merge(a, wp[i]);
-    part[(int64_t)r * n_chunks + c] = a;
+  if (wv == 0) {
+    Partial a = lane < 8 ? wp[lane] : Partial{-INFINITY, 0x7fffffff, 0.0};
+    a = warp_merge(a);
+    if (lane == 0) part[(int64_t)r * n_chunks + c] = a;
   }
 }
 
 // One warp per logical block row b (L <= 32 positions, lane i = position i). The still-masked flat positions are
 // the LM head's rows in increasing order, so the row of position (b, i) is the number of masked positions before it.
-__global__ void unmask_select_kernel(const Partial* __restrict__ part, int n_chunks, const int32_t* __restrict__ row_pos,
+__global__ void __launch_bounds__(1024) unmask_select_kernel(Partial* part, int n_chunks, const int32_t* __restrict__ row_pos,
                                      const int32_t* __restrict__ n_rows, int B, int L, int t, int T_s, int mode,
                                      float tau, int k_max, int cfg, int vocab_offset, int32_t* tokens, uint8_t* mask,
                                      int32_t* sel, int32_t* nsel, float* conf, int32_t* remaining) {
@@ -260,6 +266,30 @@ __global__ void unmask_select_kernel(const Partial* __restrict__ part, int n_chu
   __shared__ int rem_w[32];
   __shared__ int row_cnt[1024];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  // many partials per row (the LM head's fused epilogue writes one per CTA): a warp merges each row's partials
+  // into its first slot, then the selection below reads that slot alone
+  int n_merge = n_chunks;
+  if (n_chunks > kMergeSerial) {
+    const int nr = *n_rows;
+    for (int r = w; r < nr; r += nw) {
+      Partial* pr = part + (int64_t)r * n_chunks;
+      Partial a{-INFINITY, 0x7fffffff, 0.0};
+      for (int c0 = 0; c0 < n_chunks; c0 += 128) {
+        Partial b4[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int c = c0 + u * 32 + lane;
+          b4[u] = c < n_chunks ? pr[c] : Partial{-INFINITY, 0x7fffffff, 0.0};
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) merge(a, b4[u]);
+      }
+      a = warp_merge(a);
+      if (lane == 0) pr[0] = a;
+    }
+    __syncthreads();
+    n_merge = 1;
+  }
   // masked count of every logical row, then the exclusive prefix (rows in order)
   for (int b = w; b < B; b += nw) {
     const bool mk = lane < L && mask[b * L + lane] != 0;
@@ -289,14 +319,14 @@ __global__ void unmask_select_kernel(const Partial* __restrict__ part, int n_chu
       const Partial* pr = part + (int64_t)r * n_chunks;
       Partial a = pr[0];
       // batches of 8 independent loads, merged in chunk order
-      for (int q0 = 1; q0 < n_chunks; q0 += 8) {
+      for (int q0 = 1; q0 < n_merge; q0 += 8) {
         Partial b8[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u)
-          if (q0 + u < n_chunks) b8[u] = pr[q0 + u];
+          if (q0 + u < n_merge) b8[u] = pr[q0 + u];
 #pragma unroll
         for (int u = 0; u < 8; ++u)
-          if (q0 + u < n_chunks) merge(a, b8[u]);
+          if (q0 + u < n_merge) merge(a, b8[u]);
       }
       c = 1.0 / a.s;
       cand = a.idx + vocab_offset;
@@ -364,7 +394,7 @@ size_t unmask_partials_bytes(int max_rows, int n_chunks) {
 
 int launch_unmask(const UnmaskArgs& a, cudaStream_t s) {
   const int chunk = ((a.V + a.n_chunks - 1) / a.n_chunks + 7) & ~7;
-  if (a.max_rows > 0) {
+  if (a.max_rows > 0 && !a.partials_ready) {
     dim3 grid(a.max_rows, a.n_chunks);
     Partial* part = static_cast<Partial*>(a.partials);
     if (a.dtype == DLLM_BF16) {
@@ -380,8 +410,8 @@ int launch_unmask(const UnmaskArgs& a, cudaStream_t s) {
     }
     DLLM_CHECK_LAUNCH("unmask_reduce_kernel");
   }
-  const int threads = 32 * min(32, max(1, a.B));
-  launch_pdl(unmask_select_kernel, 1, threads, 0, s, static_cast<const Partial*>(a.partials), a.n_chunks, a.row_pos, a.n_rows,
+  const int threads = a.n_chunks > kMergeSerial ? 1024 : 32 * min(32, max(1, a.B));
+  launch_pdl(unmask_select_kernel, 1, threads, 0, s, static_cast<Partial*>(a.partials), a.n_chunks, a.row_pos, a.n_rows,
                                              a.B, a.L, a.t, a.T_s, a.mode, a.tau, a.k_max, a.cfg, a.vocab_offset,
                                              a.tokens, a.mask, a.sel, a.nsel, a.conf, a.remaining);
   DLLM_CHECK_LAUNCH("unmask_select_kernel");

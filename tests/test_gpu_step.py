@@ -175,6 +175,58 @@ def test_step_small_bf16_threshold():
     _one_pass(w, seed=5)
 
 
+# One logical row of at most 32 positions, no guidance, and a scored vocabulary of at least 74 weight tiles of 128
+# rows: the LM head writes the confidence partials from its epilogue (one per persistent CTA) and the step launches
+# no separate reduction.
+FUSED = scaled(SMALL, name="small-bf16-fused-confidence", B=1, L=32, V=20480)
+
+
+def test_step_fused_confidence_partly_masked():
+    _one_pass(FUSED, seed=21, masked_fraction=0.6, t=2)
+
+
+def test_step_fused_confidence_vocab_slice_threshold():
+    w = scaled(FUSED, vocab_offset=4096, vocab_len=128 * 80, mode=1, tau=0.9, k_max=8, T_s=16, lm_std=1.0)
+    _one_pass(w, seed=22)
+
+
+@pytest.mark.parametrize("masked_fraction", [1.0, 0.3])
+def test_fused_confidence_equals_reduction(masked_fraction):
+    """The fused confidence of a step equals the standalone reduction over the logits that step wrote. The
+    standalone reduction is itself held to the oracle within 1e-6 relative (the unmask tests), so this pins the
+    fused epilogue and the many-partial merge of the selection to the same arithmetic."""
+    w = scaled(FUSED, lm_std=0.5)
+    _, _, eng, tok0, mask0 = _setup(w, seed=23, masked_fraction=masked_fraction)
+    t = 1
+    eng.step(t)
+    torch.cuda.synchronize()
+    assert bd.status_check(eng.ws) == bd.OK
+    row_pos = np.nonzero(mask0.reshape(-1))[0].astype(np.int32)
+    n = len(row_pos)
+    logits = eng.logits(n).clone()
+    dm = torch.from_numpy(mask0).to(DEV)
+    dt_ = torch.from_numpy(tok0).to(DEV)
+    sel = torch.empty((1, w.L), dtype=torch.int32, device=DEV)
+    nsel = torch.empty(1, dtype=torch.int32, device=DEV)
+    conf = torch.empty((1, w.L), dtype=torch.float32, device=DEV)
+    rem = torch.empty(1, dtype=torch.int32, device=DEV)
+    rp = torch.from_numpy(np.concatenate([row_pos, np.zeros(w.L - n, np.int32)])).to(DEV)
+    nd = torch.tensor([n], dtype=torch.int32, device=DEV)
+    bd.unmask(logits, rp, nd, dt_, dm, sel, nsel, conf, rem, 1, w.L, w.vlen, w.L, t, w.T_s, bd.BF16, mode=w.mode,
+              tau=w.tau, k_max=w.k_max)
+    torch.cuda.synchronize()
+    m_ = mask0[0].astype(bool)
+    c_step = eng.conf.cpu().numpy()[0].astype(np.float64)
+    c_red = conf.cpu().numpy()[0].astype(np.float64)
+    assert np.all(np.abs(c_step[m_] - c_red[m_]) <= 2e-6 * c_red[m_])
+    cs = np.sort(c_red[m_])[::-1]
+    k = int(nsel.item())
+    if not (0 < k < len(cs) and cs[k - 1] - cs[k] < 1e-5 * cs[k - 1]):
+        assert int(eng.nsel[0].item()) == k
+        assert np.array_equal(eng.mask.cpu().numpy(), dm.cpu().numpy())
+        assert np.array_equal(eng.tokens.cpu().numpy(), dt_.cpu().numpy())
+
+
 def test_step_one_layer_full_size():
     """The one-layer bf16 workload at its full size (hidden 2048, 256 experts, vocab 157184, prefix 1024)."""
     _one_pass(ONE_LAYER, seed=0, random_gains=False)

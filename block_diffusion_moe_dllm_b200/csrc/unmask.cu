@@ -16,8 +16,12 @@
 namespace dllm {
 namespace {
 
-constexpr int kRegVpt = 16;                      // 16-byte vectors per thread kept in registers
+constexpr int kRegVpt = 16;                      // most 16-byte vectors a thread keeps in registers
 constexpr int kRegChunk = kRegVpt * 256 * 8;     // vocabulary entries per CTA of the register path (32768)
+
+// CTAs of the register path resident per SM for a given register depth (launch bound: registers per thread)
+constexpr int kPrefVpt = 16;                     // register depth the chunking aims for when rows are many
+template <int VPT> constexpr int reg_min_blocks() { return VPT >= 16 ? 3 : VPT >= 12 ? 4 : VPT >= 8 ? 5 : 6; }
 constexpr int kMergeSerial = 8;                  // partials per row merged by one lane; more: a warp per row
 
 // (max logit, lowest index attaining it within the scored slice, sum over the chunk of exp(z - max))
@@ -181,7 +185,7 @@ DLLM_DEV Partial warp_merge(Partial p) {
 // maximum), accumulated per thread in fp32 over at most VPT * 8 terms and then in fp64; the lowest arg-max comes
 // from the first vector that holds the maximum, re-read (from L2) before pass 2 so that its latency hides behind it.
 template <int VPT>
-__global__ void __launch_bounds__(256) unmask_reduce_bf16_kernel(const __nv_bfloat16* __restrict__ logits,
+__global__ void __launch_bounds__(256, reg_min_blocks<VPT>()) unmask_reduce_bf16_kernel(const __nv_bfloat16* __restrict__ logits,
                                                                  const int32_t* __restrict__ n_rows, int V, int chunk,
                                                                  Partial* __restrict__ part, int n_chunks) {
   pdl_enter();
@@ -381,10 +385,10 @@ __global__ void __launch_bounds__(1024) unmask_select_kernel(Partial* part, int 
 
 int unmask_chunks(int max_rows, int V) {
   // enough CTAs to cover the SMs a few times when every row is masked, chunks of at least 2048 entries, and at most
-  // kRegChunk entries so that a thread's share of a chunk fits in registers
+  // kPrefVpt * 2048 entries so that a thread's share of a chunk fits in registers
   int want = (4 * num_sms() + max(max_rows, 1) - 1) / max(max_rows, 1);
   int most = max(1, V / 2048);
-  int least = (V + kRegChunk - 1) / kRegChunk;
+  int least = (V + kPrefVpt * 2048 - 1) / (kPrefVpt * 2048);
   return max(1, max(least, min(want, min(most, 64))));
 }
 
@@ -400,8 +404,14 @@ int launch_unmask(const UnmaskArgs& a, cudaStream_t s) {
     if (a.dtype == DLLM_BF16) {
       const __nv_bfloat16* z = static_cast<const __nv_bfloat16*>(a.logits);
       if (a.cfg) launch_pdl((unmask_reduce_kernel<__nv_bfloat16, true>), grid, 256, 0, s, z, a.n_rows, a.V, chunk, a.cfg_scale, part, a.n_chunks);
-      else if (a.V % 8 == 0 && chunk <= kRegChunk)
-        launch_pdl(unmask_reduce_bf16_kernel<kRegVpt>, grid, 256, 0, s, z, a.n_rows, a.V, chunk, part, a.n_chunks);
+      else if (a.V % 8 == 0 && chunk <= kRegChunk) {
+        // the shallowest register depth that holds a thread's share of the chunk
+        const int vpt = (chunk / 8 + 255) / 256;
+        if (vpt <= 4) launch_pdl(unmask_reduce_bf16_kernel<4>, grid, 256, 0, s, z, a.n_rows, a.V, chunk, part, a.n_chunks);
+        else if (vpt <= 8) launch_pdl(unmask_reduce_bf16_kernel<8>, grid, 256, 0, s, z, a.n_rows, a.V, chunk, part, a.n_chunks);
+        else if (vpt <= 12) launch_pdl(unmask_reduce_bf16_kernel<12>, grid, 256, 0, s, z, a.n_rows, a.V, chunk, part, a.n_chunks);
+        else launch_pdl(unmask_reduce_bf16_kernel<16>, grid, 256, 0, s, z, a.n_rows, a.V, chunk, part, a.n_chunks);
+      }
       else launch_pdl((unmask_reduce_kernel<__nv_bfloat16, false>), grid, 256, 0, s, z, a.n_rows, a.V, chunk, a.cfg_scale, part, a.n_chunks);
     } else {
       const float* z = static_cast<const float*>(a.logits);

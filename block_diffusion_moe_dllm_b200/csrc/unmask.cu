@@ -46,6 +46,27 @@ DLLM_DEV float guided(float zc, float zu, float s) {
   return __fadd_rn(zu, __fmul_rn(s, __fsub_rn(zc, zu)));
 }
 
+// The hardware base-2 exponential (ex2.approx.ftz: relative error about 2^-22, results below 2^-126 flushed to 0,
+// which against a maximum term of 1 is far below fp32 resolution). Sums and scalings of fp32 pairs use the sm_100
+// packed instructions (__fadd2_rn / __fmul2_rn: one issue for two lanes' worth).
+DLLM_DEV float ex2(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
+// Merge of the 32 lanes' partials (empty ones have s == 0): the lanes' maximum M, each sum rescaled by
+// 2^((m - M) log2 e), the fp64 sum of those, and the lowest index among the lanes with m == M. Every lane returns
+// the result.
+DLLM_DEV Partial warp_merge(Partial p) {
+  const bool has = p.s != 0.0;
+  const float M = warp_max(has ? p.m : -INFINITY);
+  double s = !has ? 0.0 : p.m == M ? p.s : p.s * (double)ex2((p.m - M) * 1.4426950408889634f);
+  s = warp_sum(s);
+  const int idx = __reduce_min_sync(0xffffffffu, (has && p.m == M) ? p.idx : 0x7fffffff);
+  return Partial{M, idx, s};
+}
+
 // Running update of one thread's partial with 8 consecutive values starting at vocabulary index v.
 DLLM_DEV void update8(Partial& p, const float* z, int v) {
   float vm = z[0];
@@ -123,84 +144,26 @@ __global__ void __launch_bounds__(256) unmask_reduce_kernel(const T* __restrict_
     merge(p, q);
   }
   // warp merge then block merge
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    Partial q;
-    q.m = __shfl_xor_sync(0xffffffffu, p.m, o);
-    q.idx = __shfl_xor_sync(0xffffffffu, p.idx, o);
-    q.s = __shfl_xor_sync(0xffffffffu, p.s, o);
-    merge(p, q);
-  }
+  p = warp_merge(p);
   __shared__ Partial wp[8];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   if (lane == 0) wp[w] = p;
   __syncthreads();
-  if (threadIdx.x == 0) {
-    Partial a = wp[0];
-    for (int i = 1; i < 8; ++i) merge(a, wp[i]);
-    part[(int64_t)r * n_chunks + c] = a;
+  if (w == 0) {
+    Partial a = lane < 8 ? wp[lane] : Partial{-INFINITY, 0x7fffffff, 0.0};
+    a = warp_merge(a);
+    if (lane == 0) part[(int64_t)r * n_chunks + c] = a;
   }
 }
 
-// Packed fp32 pairs (the sm_100 f32x2 instructions: one issue for two lanes' worth of add or multiply) and the
-// hardware base-2 exponential (ex2.approx.ftz: relative error about 2^-22, results below 2^-126 flushed to 0, which
-// against a maximum term of 1 is far below fp32 resolution).
-DLLM_DEV uint64_t pk2(float lo, float hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-DLLM_DEV void upk2(uint64_t v, float& lo, float& hi) { asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v)); }
-DLLM_DEV uint64_t add2(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-DLLM_DEV uint64_t mul2(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
-DLLM_DEV float ex2(float x) {
-  float r;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
-  return r;
-}
-
-// Merge of the 32 lanes' partials (empty ones have s == 0): the lanes' maximum M, each sum rescaled by
-// 2^((m - M) log2 e), the fp64 sum of those, and the lowest index among the lanes with m == M. Every lane returns
-// the result.
-DLLM_DEV Partial warp_merge(Partial p) {
-  const bool has = p.s != 0.0;
-  const float M = warp_max(has ? p.m : -INFINITY);
-  double s = has ? p.s * (double)ex2((p.m - M) * 1.4426950408889634f) : 0.0;
-  s = warp_sum(s);
-  const int idx = __reduce_min_sync(0xffffffffu, (has && p.m == M) ? p.idx : 0x7fffffff);
-  return Partial{M, idx, s};
-}
-
-// bf16 logits without guidance: each thread keeps its VPT 16-byte vectors of the chunk in registers. Pass 1 finds
+// bf16 logits without guidance: each thread keeps its VPT 16-byte vectors of a chunk in registers. Pass 1 finds
 // the maximum with packed bf16x2 max (and the first vector holding it); pass 2 sums exp(z - max) as
 // 2^((z - max) * log2(e)) with the subtraction and the scaling done on fp32 pairs (z - max is exact near the
 // maximum), accumulated per thread in fp32 over at most VPT * 8 terms and then in fp64; the lowest arg-max comes
-// from the first vector that holds the maximum, re-read (from L2) before pass 2 so that its latency hides behind it.
-template <int VPT>
-__global__ void __launch_bounds__(256, reg_min_blocks<VPT>()) unmask_reduce_bf16_kernel(const __nv_bfloat16* __restrict__ logits,
-                                                                 const int32_t* __restrict__ n_rows, int V, int chunk,
-                                                                 Partial* __restrict__ part, int n_chunks) {
-  pdl_enter();
-  const int r = blockIdx.x, c = blockIdx.y;
-  if (r >= *n_rows) return;
-  const __nv_bfloat16* z = logits + (int64_t)r * V;
-  const int v0 = c * chunk, v1 = min(V, v0 + chunk);
-  const int nvec = (v1 - v0) >> 3;
-  uint4 u[VPT];
-#pragma unroll
-  for (int k = 0; k < VPT; ++k) {
-    const int i = threadIdx.x + k * 256;
-    u[k] = i < nvec ? ld_nc_v4(z + v0 + i * 8) : make_uint4(0xff80ff80u, 0xff80ff80u, 0xff80ff80u, 0xff80ff80u);
-  }
-  // pass 1: maximum (bf16 -inf fills the missing vectors) and the first vector that attains it
+// from the first vector that holds the maximum, fetched again (reload(k)) before pass 2 so that its latency hides
+// behind it. Missing vectors hold bf16 -inf.
+template <int VPT, typename Reload>
+DLLM_DEV Partial chunk_partial(const uint4 (&u)[VPT], int vbase, Reload reload) {
   float m = -INFINITY;
   int best = -1;
 #pragma unroll
@@ -212,24 +175,20 @@ __global__ void __launch_bounds__(256, reg_min_blocks<VPT>()) unmask_reduce_bf16
   }
   Partial p{-INFINITY, 0x7fffffff, 0.0};
   if (best >= 0) {
-    const uint4 bv = ld_nc_v4(z + v0 + (threadIdx.x + best * 256) * 8);
-    // pass 2: sum of exponentials relative to the thread's maximum, two terms per packed operation
+    const uint4 bv = reload(best);
     const float log2e = 1.4426950408889634f;
-    const uint64_t negm2 = pk2(-m, -m), log2e2 = pk2(log2e, log2e);
-    uint64_t acc2 = pk2(0.f, 0.f);
+    const float2 negm2 = make_float2(-m, -m), l2 = make_float2(log2e, log2e);
+    float2 acc = make_float2(0.f, 0.f);
 #pragma unroll
     for (int k = 0; k < VPT; ++k) {
       const uint32_t w[4] = {u[k].x, u[k].y, u[k].z, u[k].w};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const uint64_t zz = pk2(__uint_as_float(w[q] << 16), __uint_as_float(w[q] & 0xffff0000u));
-        float e0, e1;
-        upk2(mul2(add2(zz, negm2), log2e2), e0, e1);
-        acc2 = add2(acc2, pk2(ex2(e0), ex2(e1)));
+        const float2 zz = make_float2(__uint_as_float(w[q] << 16), __uint_as_float(w[q] & 0xffff0000u));
+        const float2 x = __fmul2_rn(__fadd2_rn(zz, negm2), l2);
+        acc = __fadd2_rn(acc, make_float2(ex2(x.x), ex2(x.y)));
       }
     }
-    float a0, a1;
-    upk2(acc2, a0, a1);
     // lowest index attaining m inside the first vector that holds it
     float f[8];
     bf16x8_to_f32(bv, f);
@@ -238,26 +197,52 @@ __global__ void __launch_bounds__(256, reg_min_blocks<VPT>()) unmask_reduce_bf16
     for (int q = 7; q >= 0; --q)
       if (f[q] == m) e = q;
     p.m = m;
-    p.idx = v0 + (threadIdx.x + best * 256) * 8 + e;
-    p.s = (double)a0 + (double)a1;
+    p.idx = vbase + (threadIdx.x + best * 256) * 8 + e;
+    p.s = (double)acc.x + (double)acc.y;
   }
-  // scalar tail of the chunk (chunk lengths are multiples of 8 except the row's last chunk)
-  for (int v = v0 + nvec * 8 + threadIdx.x; v < v1; v += 256) {
-    Partial q{__bfloat162float(z[v]), v, 1.0};
-    merge(p, q);
-  }
-  // warp, then block: the maximum, every sum rescaled to it, the sum, and the lowest index among the partials
-  // that attain it
+  return p;
+}
+
+// Block merge of the 256 threads' partials (warp, then block: the maximum, every sum rescaled to it, the sum, and
+// the lowest index among the partials that attain it); thread 0 stores the result. Reuses wp: the caller orders a
+// second use after the first with a barrier.
+DLLM_DEV void block_store(Partial p, Partial* wp, Partial* dst) {
   p = warp_merge(p);
-  __shared__ Partial wp[8];
   const int lane = threadIdx.x & 31, wv = threadIdx.x >> 5;
   if (lane == 0) wp[wv] = p;
   __syncthreads();
   if (wv == 0) {
     Partial a = lane < 8 ? wp[lane] : Partial{-INFINITY, 0x7fffffff, 0.0};
     a = warp_merge(a);
-    if (lane == 0) part[(int64_t)r * n_chunks + c] = a;
+    if (lane == 0) *dst = a;
   }
+}
+
+template <int VPT>
+DLLM_DEV void load_chunk_regs(uint4 (&u)[VPT], const __nv_bfloat16* src, int nvec) {
+#pragma unroll
+  for (int k = 0; k < VPT; ++k) {
+    const int i = threadIdx.x + k * 256;
+    u[k] = i < nvec ? ld_nc_v4(src + i * 8) : make_uint4(0xff80ff80u, 0xff80ff80u, 0xff80ff80u, 0xff80ff80u);
+  }
+}
+
+// One CTA per (row, chunk); a row's chunks are adjacent CTAs (contiguous memory). V % 8 == 0.
+template <int VPT>
+__global__ void __launch_bounds__(256, reg_min_blocks<VPT>()) unmask_reduce_bf16_kernel(const __nv_bfloat16* __restrict__ logits,
+                                                                 const int32_t* __restrict__ n_rows, int V, int chunk,
+                                                                 Partial* __restrict__ part, int n_chunks) {
+  pdl_enter();
+  const int r = blockIdx.y, c = blockIdx.x;
+  if (r >= *n_rows) return;
+  const __nv_bfloat16* z = logits + (int64_t)r * V;
+  const int v0 = c * chunk, v1 = min(V, v0 + chunk);
+  const int nvec = (v1 - v0) >> 3;
+  uint4 u[VPT];
+  load_chunk_regs<VPT>(u, z + v0, nvec);
+  const Partial p = chunk_partial<VPT>(u, v0, [&](int k) { return ld_nc_v4(z + v0 + (threadIdx.x + k * 256) * 8); });
+  __shared__ Partial wp[8];
+  block_store(p, wp, part + (int64_t)r * n_chunks + c);
 }
 
 // One warp per logical block row b (L <= 32 positions, lane i = position i). The still-masked flat positions are
@@ -407,10 +392,11 @@ int launch_unmask(const UnmaskArgs& a, cudaStream_t s) {
       else if (a.V % 8 == 0 && chunk <= kRegChunk) {
         // the shallowest register depth that holds a thread's share of the chunk
         const int vpt = (chunk / 8 + 255) / 256;
-        if (vpt <= 4) launch_pdl(unmask_reduce_bf16_kernel<4>, grid, 256, 0, s, z, a.n_rows, a.V, chunk, part, a.n_chunks);
-        else if (vpt <= 8) launch_pdl(unmask_reduce_bf16_kernel<8>, grid, 256, 0, s, z, a.n_rows, a.V, chunk, part, a.n_chunks);
-        else if (vpt <= 12) launch_pdl(unmask_reduce_bf16_kernel<12>, grid, 256, 0, s, z, a.n_rows, a.V, chunk, part, a.n_chunks);
-        else launch_pdl(unmask_reduce_bf16_kernel<16>, grid, 256, 0, s, z, a.n_rows, a.V, chunk, part, a.n_chunks);
+        const dim3 g2(a.n_chunks, a.max_rows);
+        if (vpt <= 4) launch_pdl(unmask_reduce_bf16_kernel<4>, g2, 256, 0, s, z, a.n_rows, a.V, chunk, part, a.n_chunks);
+        else if (vpt <= 8) launch_pdl(unmask_reduce_bf16_kernel<8>, g2, 256, 0, s, z, a.n_rows, a.V, chunk, part, a.n_chunks);
+        else if (vpt <= 12) launch_pdl(unmask_reduce_bf16_kernel<12>, g2, 256, 0, s, z, a.n_rows, a.V, chunk, part, a.n_chunks);
+        else launch_pdl(unmask_reduce_bf16_kernel<16>, g2, 256, 0, s, z, a.n_rows, a.V, chunk, part, a.n_chunks);
       }
       else launch_pdl((unmask_reduce_kernel<__nv_bfloat16, false>), grid, 256, 0, s, z, a.n_rows, a.V, chunk, a.cfg_scale, part, a.n_chunks);
     } else {

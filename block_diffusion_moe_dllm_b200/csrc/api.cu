@@ -157,6 +157,7 @@ struct StepPlan {
   int32_t* offsets;
   int32_t* perm;
   int32_t* inv;
+  int32_t* route_seg;
   ExpertBufs eb;
   float* proj_scratch;
   int32_t* row_pos;
@@ -257,6 +258,7 @@ void plan_step(const dllm_model* m, const dllm_state* st, const dllm_step_params
   s.offsets = c.take<int32_t>((size_t)(m->E + 1) * 4);
   s.perm = c.take<int32_t>((size_t)s.Tk * m->k * 4);
   s.inv = c.take<int32_t>((size_t)s.Tk * m->k * 4);
+  s.route_seg = c.take<int32_t>(route_scratch_bytes(s.Tk, m->E, m->k));
   carve_experts(c, m->dtype, s.Tk, H, m->k, m->I, 1, s.eb);
   const int proj_n = (m->Hq + 2 * m->Hkv) * m->d;
   s.proj_scratch = m->dtype == DLLM_F32
@@ -408,7 +410,7 @@ int dllm_prefix_retain(const dllm_retain_desc* d, const void* k_cache, const voi
 // ------------------------------------------------------------------------------------------------ router
 size_t dllm_moe_route_workspace_size(const dllm_route_desc* d) {
   if (!d) return 0;
-  return align256(align256(kStatusBytes) + (size_t)d->Tk * d->E * 4);
+  return align256(align256(align256(kStatusBytes) + (size_t)d->Tk * d->E * 4) + route_scratch_bytes(d->Tk, d->E, d->k));
 }
 
 int dllm_moe_route(const dllm_route_desc* d, const void* h, const void* w_router, const float* bias, int32_t* ids,
@@ -426,9 +428,11 @@ int dllm_moe_route(const dllm_route_desc* d, const void* h, const void* w_router
   int st = check_ws(ws, ws_bytes, dllm_moe_route_workspace_size(d));
   if (st) return st;
   Carver c(ws);
-  float* sc = scores ? scores : c.take<float>((size_t)d->Tk * d->E * 4);
+  float* sc = c.take<float>((size_t)d->Tk * d->E * 4);
+  if (scores) sc = scores;
+  int32_t* seg = c.take<int32_t>(route_scratch_bytes(d->Tk, d->E, d->k));
   return launch_route(d->dtype, h, w_router, bias, d->Tk, d->H, d->E, d->k, ids, gates, sc, counts, offsets, perm,
-                      inv, stream);
+                      inv, seg, stream);
 }
 
 // ------------------------------------------------------------------------------------------------ experts
@@ -596,7 +600,7 @@ int dllm_denoise_step(const dllm_model* m, const dllm_state* st, const dllm_step
     // MoE FFN
     TRY(launch_rmsnorm(dt, s.x, Ly.ffn_norm, s.h, s.Tk, H, m->eps, nullptr, nullptr, 0, 0, stream));
     TRY(launch_route(dt, s.h, Ly.w_router, Ly.router_bias, s.Tk, H, m->E, m->k, s.ids, s.gates, s.scores, s.counts,
-                     s.offsets, s.perm, s.inv, stream));
+                     s.offsets, s.perm, s.inv, s.route_seg, stream));
     PostNorm pn;
     if (fuse && !last) {           // next layer's attention-input norm
       pn.g = m->layers[l + 1].attn_norm; pn.eps = m->eps; pn.out = s.h; pn.mode = NORM_NEXT;

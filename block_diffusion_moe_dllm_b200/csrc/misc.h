@@ -29,9 +29,12 @@ int launch_combine_norm(int dtype, void* x, const float* y, const float* gates, 
 // router
 int num_sms();
 
+// seg_scratch: route_scratch_bytes(Tk, E, k) bytes (per-segment histograms of the permutation)
 int launch_route(int dtype, const void* h, const void* w_router, const float* bias, int Tk, int H, int E, int k,
                  int32_t* ids, float* gates, float* scores, int32_t* counts, int32_t* offsets, int32_t* perm,
-                 int32_t* inv, cudaStream_t s);
+                 int32_t* inv, int32_t* seg_scratch, cudaStream_t s);
+int route_segment(int n_assign);
+size_t route_scratch_bytes(int Tk, int E, int k);
 
 // unmask
 struct UnmaskArgs {

@@ -5,6 +5,7 @@
 #include "common.cuh"
 #include "misc.h"
 #include "kernels.h"
+#include <algorithm>
 
 namespace dllm {
 namespace {
@@ -269,91 +270,113 @@ __global__ void __launch_bounds__(1024) route_small_kernel(float* __restrict__ s
   }
 }
 
-// Exclusive scan of n <= 1024 ints in shared memory by 256 threads (4 consecutive items per thread).
-__device__ void block_exclusive_scan(int* a, int n, int* total) {
-  __shared__ int wsum[8];
-  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-  int v[4], s = 0;
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    int i = tid * 4 + u;
-    v[u] = i < n ? a[i] : 0;
-    s += v[u];
-  }
-  int inc = s;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    int y = __shfl_up_sync(0xffffffffu, inc, o);
-    if (lane >= o) inc += y;
-  }
-  if (lane == 31) wsum[w] = inc;
+// Stable permutation for many assignments, in three launches over segments of `seg` consecutive assignments
+// (seg a multiple of 256): per-segment expert histograms; one CTA turns them into counts, offsets and every segment's
+// first output position per expert; then each segment writes its assignments' positions in order. Positions within
+// an expert follow the assignment index a = t * k + j, so an expert's rows stay sorted by token.
+
+// seg_hist[s][e] = assignments of expert e in segment s.
+__global__ void __launch_bounds__(256) route_seg_hist_kernel(const int32_t* __restrict__ ids, int n, int E, int seg,
+                                                             int32_t* __restrict__ seg_hist) {
+  pdl_enter();
+  extern __shared__ int sh_hist[];
+  for (int i = threadIdx.x; i < E; i += blockDim.x) sh_hist[i] = 0;
   __syncthreads();
-  int before = 0, tot = 0;
-  for (int i = 0; i < 8; ++i) {
-    if (i < w) before += wsum[i];
-    tot += wsum[i];
-  }
-  int run = before + inc - s;
+  const int a0 = blockIdx.x * seg, a1 = min(n, a0 + seg);
+  for (int a = a0 + threadIdx.x; a < a1; a += blockDim.x) atomicAdd(&sh_hist[ids[a]], 1);
   __syncthreads();
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    int i = tid * 4 + u;
-    if (i < n) a[i] = run;
-    run += v[u];
-  }
-  if (total) *total = tot;
-  __syncthreads();
+  for (int i = threadIdx.x; i < E; i += blockDim.x) seg_hist[(int64_t)blockIdx.x * E + i] = sh_hist[i];
 }
 
-// One CTA per expert: histogram of all assignments, offsets by exclusive scan, then this expert's rows in
-// increasing assignment order (t * k + j), which keeps the rows of an expert sorted by token.
-__global__ void route_permute_kernel(const int32_t* __restrict__ ids, int n_assign, int E, int32_t* counts,
-                                     int32_t* offsets, int32_t* perm, int32_t* inv) {
+// One thread per expert (E <= 1024): counts = column sums, offsets = their exclusive scan over experts (offsets[E] =
+// n), and seg_hist[s][e] is replaced by offsets[e] + (assignments of e in segments before s).
+__global__ void __launch_bounds__(1024) route_seg_scan_kernel(int32_t* __restrict__ seg_hist, int S, int E, int n,
+                                                              int32_t* __restrict__ counts,
+                                                              int32_t* __restrict__ offsets) {
   pdl_enter();
-  __shared__ int hist[1024];
-  __shared__ int cnt_e;
-  __shared__ int wtot[8];
-  const int e = blockIdx.x, tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
-  for (int i = tid; i < E; i += blockDim.x) hist[i] = 0;
-  __syncthreads();
-  for (int a = tid; a < n_assign; a += blockDim.x) atomicAdd(&hist[ids[a]], 1);
-  __syncthreads();
-  if (tid == 0) cnt_e = hist[e];
-  __syncthreads();
-  int total = 0;
-  if (blockIdx.x == 0)
-    for (int i = tid; i < E; i += blockDim.x) counts[i] = hist[i];
-  __syncthreads();
-  block_exclusive_scan(hist, E, &total);
-  const int off = hist[e];
-  if (blockIdx.x == 0) {
-    for (int i = tid; i < E; i += blockDim.x) offsets[i] = hist[i];
-    if (tid == 0) offsets[E] = total;
+  __shared__ int wtot[32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+  int cnt = 0;
+  if (tid < E) {
+#pragma unroll 8
+    for (int sg = 0; sg < S; ++sg) cnt += seg_hist[(int64_t)sg * E + tid];
   }
-  if (cnt_e == 0) return;
-  // each of the 8 warps takes a contiguous segment of the assignments: count this expert's in it, one prefix
-  // over the warps, then write their positions in order (no block barrier inside the scans)
-  const int seg = (n_assign + 7) / 8;
-  const int s0 = min(n_assign, w * seg), s1 = min(n_assign, s0 + seg);
-  int c = 0;
-  for (int a0 = s0; a0 < s1; a0 += 32) {
-    const int a = a0 + lane;
-    c += __popc(__ballot_sync(0xffffffffu, a < s1 && __ldg(ids + a) == e));
+  int inc = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += y;
   }
-  if (lane == 0) wtot[w] = c;
+  if (lane == 31) wtot[warp] = inc;
   __syncthreads();
-  int run = off;
-  for (int i = 0; i < w; ++i) run += wtot[i];
-  for (int a0 = s0; a0 < s1; a0 += 32) {
-    const int a = a0 + lane;
-    const bool f = a < s1 && __ldg(ids + a) == e;
-    const unsigned bal = __ballot_sync(0xffffffffu, f);
-    if (f) {
-      const int r = run + __popc(bal & ((1u << lane) - 1u));
-      perm[r] = a;
-      inv[a] = r;
+  if (warp == 0) {
+    int x = lane < nw ? wtot[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
     }
-    run += __popc(bal);
+    wtot[lane] = x;   // inclusive over warps
+  }
+  __syncthreads();
+  const int excl = inc - cnt + (warp > 0 ? wtot[warp - 1] : 0);
+  if (tid < E) {
+    counts[tid] = cnt;
+    offsets[tid] = excl;
+    int run = excl;
+    for (int sg = 0; sg < S; ++sg) {
+      const int v = seg_hist[(int64_t)sg * E + tid];
+      seg_hist[(int64_t)sg * E + tid] = run;
+      run += v;
+    }
+  }
+  if (tid == 0) offsets[E] = n;
+}
+
+// Segment s: its 8 warps take seg / 8 consecutive assignments each (whole 32-assignment chunks). Pass 1 counts
+// each warp's assignments per expert (lanes with the same expert find each other with __match_any_sync and the
+// group's first lane adds the group size); the warps' counts are prefixed per expert on top of the segment's first
+// positions; pass 2 walks the chunks again and writes position = warp's running base + rank among the chunk's
+// lanes with the same expert.
+__global__ void __launch_bounds__(256) route_seg_scatter_kernel(const int32_t* __restrict__ ids, int n, int E, int seg,
+                                                                const int32_t* __restrict__ seg_base,
+                                                                int32_t* __restrict__ perm, int32_t* __restrict__ inv) {
+  pdl_enter();
+  extern __shared__ int wh[];   // [8][E]
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  for (int i = tid; i < 8 * E; i += blockDim.x) wh[i] = 0;
+  __syncthreads();
+  const int per = seg / 8;
+  const int w0 = blockIdx.x * seg + w * per, w1 = min(n, w0 + per);
+  for (int c = w0; c < w1; c += 32) {
+    const int a = c + lane;
+    const int ex = a < w1 ? ids[a] : -1;
+    const unsigned grp = __match_any_sync(0xffffffffu, ex);
+    if (a < w1 && lane == __ffs(grp) - 1) wh[w * E + ex] += __popc(grp);
+  }
+  __syncthreads();
+  for (int e = tid; e < E; e += blockDim.x) {
+    int run = seg_base[(int64_t)blockIdx.x * E + e];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const int v = wh[q * E + e];
+      wh[q * E + e] = run;
+      run += v;
+    }
+  }
+  __syncthreads();
+  for (int c = w0; c < w1; c += 32) {
+    const int a = c + lane;
+    const int ex = a < w1 ? ids[a] : -1;
+    const unsigned grp = __match_any_sync(0xffffffffu, ex);
+    if (a < w1) {
+      const int pos = wh[w * E + ex] + __popc(grp & ((1u << lane) - 1u));
+      perm[pos] = a;
+      inv[a] = pos;
+    }
+    __syncwarp();
+    if (a < w1 && lane == __ffs(grp) - 1) wh[w * E + ex] += __popc(grp);
+    __syncwarp();
   }
 }
 
@@ -361,7 +384,8 @@ __global__ void route_permute_kernel(const int32_t* __restrict__ ids, int n_assi
 
 template <int PER>
 int launch_select_per(float* scores, const float* bias, int Tk, int E, int k, int from_logits, int32_t* ids,
-                      float* gates, int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv, cudaStream_t s) {
+                      float* gates, int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv,
+                      int32_t* seg_scratch, cudaStream_t s) {
   if constexpr (PER <= 8) {   // E <= 256: the single-CTA kernel fits its 64 registers per thread
     const int n = Tk * k, W = (n + 31) / 32;
     const size_t smem = ((size_t)W * E + 2 * (size_t)n + E) * sizeof(int);
@@ -380,25 +404,42 @@ int launch_select_per(float* scores, const float* bias, int Tk, int E, int k, in
   // one warp per token, 4 per CTA: many tokens spread over all the SMs
   launch_pdl(route_topk_kernel<PER>, (Tk + 3) / 4, 128, 0, s, scores, bias, Tk, E, k, from_logits, ids, gates);
   DLLM_CHECK_LAUNCH("route_topk_kernel");
-  launch_pdl(route_permute_kernel, E, 256, 0, s, (const int32_t*)ids, Tk * k, E, counts, offsets, perm, inv);
-  DLLM_CHECK_LAUNCH("route_permute_kernel");
+  const int n = Tk * k, seg = route_segment(n), S = (n + seg - 1) / seg;
+  launch_pdl(route_seg_hist_kernel, S, 256, (size_t)E * sizeof(int), s, (const int32_t*)ids, n, E, seg, seg_scratch);
+  DLLM_CHECK_LAUNCH("route_seg_hist_kernel");
+  launch_pdl(route_seg_scan_kernel, 1, 32 * ((E + 31) / 32), 0, s, seg_scratch, S, E, n, counts, offsets);
+  DLLM_CHECK_LAUNCH("route_seg_scan_kernel");
+  launch_pdl(route_seg_scatter_kernel, S, 256, (size_t)8 * E * sizeof(int), s, (const int32_t*)ids, n, E, seg,
+             (const int32_t*)seg_scratch, perm, inv);
+  DLLM_CHECK_LAUNCH("route_seg_scatter_kernel");
   return DLLM_OK;
 }
 
 // Selection and permutation from fp32 scores (sigmoid applied here when from_logits), E <= 1024.
 int launch_select(float* scores, const float* bias, int Tk, int E, int k, int from_logits, int32_t* ids,
-                  float* gates, int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv, cudaStream_t s) {
-  if (E <= 32) return launch_select_per<1>(scores, bias, Tk, E, k, from_logits, ids, gates, counts, offsets, perm, inv, s);
-  if (E <= 64) return launch_select_per<2>(scores, bias, Tk, E, k, from_logits, ids, gates, counts, offsets, perm, inv, s);
-  if (E <= 128) return launch_select_per<4>(scores, bias, Tk, E, k, from_logits, ids, gates, counts, offsets, perm, inv, s);
-  if (E <= 256) return launch_select_per<8>(scores, bias, Tk, E, k, from_logits, ids, gates, counts, offsets, perm, inv, s);
-  if (E <= 512) return launch_select_per<16>(scores, bias, Tk, E, k, from_logits, ids, gates, counts, offsets, perm, inv, s);
-  return launch_select_per<32>(scores, bias, Tk, E, k, from_logits, ids, gates, counts, offsets, perm, inv, s);
+                  float* gates, int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv, int32_t* seg,
+                  cudaStream_t s) {
+  if (E <= 32) return launch_select_per<1>(scores, bias, Tk, E, k, from_logits, ids, gates, counts, offsets, perm, inv, seg, s);
+  if (E <= 64) return launch_select_per<2>(scores, bias, Tk, E, k, from_logits, ids, gates, counts, offsets, perm, inv, seg, s);
+  if (E <= 128) return launch_select_per<4>(scores, bias, Tk, E, k, from_logits, ids, gates, counts, offsets, perm, inv, seg, s);
+  if (E <= 256) return launch_select_per<8>(scores, bias, Tk, E, k, from_logits, ids, gates, counts, offsets, perm, inv, seg, s);
+  if (E <= 512) return launch_select_per<16>(scores, bias, Tk, E, k, from_logits, ids, gates, counts, offsets, perm, inv, seg, s);
+  return launch_select_per<32>(scores, bias, Tk, E, k, from_logits, ids, gates, counts, offsets, perm, inv, seg, s);
+}
+
+int route_segment(int n_assign) {
+  // a multiple of 256 assignments (8 warps x 32), at most about 128 segments
+  return std::max(256, ((n_assign + 127) / 128 + 255) / 256 * 256);
+}
+
+size_t route_scratch_bytes(int Tk, int E, int k) {
+  const int n = std::max(Tk, 0) * k, seg = route_segment(n);
+  return (size_t)std::max(1, (n + seg - 1) / seg) * (size_t)E * sizeof(int32_t);
 }
 
 int launch_route(int dtype, const void* h, const void* w_router, const float* bias, int Tk, int H, int E, int k,
                  int32_t* ids, float* gates, float* scores, int32_t* counts, int32_t* offsets, int32_t* perm,
-                 int32_t* inv, cudaStream_t s) {
+                 int32_t* inv, int32_t* seg_scratch, cudaStream_t s) {
   if (Tk <= 0) return DLLM_OK;
   // bf16 with a tensor-core friendly shape: router logits through the tcgen05 projection (fp32 out, accumulated
   // in fp32 in the MMA's fixed order); otherwise the SIMT score kernel
@@ -410,7 +451,7 @@ int launch_route(int dtype, const void* h, const void* w_router, const float* bi
     g.epi.kind = EPI_STORE; g.epi.out = scores; g.epi.ldo = E; g.epi.out_f32 = 1;
     int st = gemm_bf16_tc(g, s);
     if (st) return st;
-    return launch_select(scores, bias, Tk, E, k, 1, ids, gates, counts, offsets, perm, inv, s);
+    return launch_select(scores, bias, Tk, E, k, 1, ids, gates, counts, offsets, perm, inv, seg_scratch, s);
   }
   dim3 g1((E + EW - 1) / EW, (Tk + TT - 1) / TT);
   const size_t smem = (size_t)TT * H * (dtype == DLLM_BF16 ? 2 : 4);
@@ -432,7 +473,7 @@ int launch_route(int dtype, const void* h, const void* w_router, const float* bi
     launch_pdl(route_scores_kernel<float>, g1, 256, smem, s, (const float*)h, (const float*)w_router, Tk, H, E, scores);
   }
   DLLM_CHECK_LAUNCH("route_scores_kernel");
-  return launch_select(scores, bias, Tk, E, k, 0, ids, gates, counts, offsets, perm, inv, s);
+  return launch_select(scores, bias, Tk, E, k, 0, ids, gates, counts, offsets, perm, inv, seg_scratch, s);
 }
 
 }  // namespace dllm

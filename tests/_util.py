@@ -55,3 +55,30 @@ def random_assignments(T, E, k, seed):
     gates = g.uniform(0.1, 1.0, (T, k)).astype(np.float32)
     gates = (gates / gates.sum(1, keepdims=True)).astype(np.float32)
     return ids, gates
+
+
+# Router near-tie band. The library scores experts in fp32 (tensor-core accumulation over H), within 2e-6 of the
+# fp64 oracle's sigmoid scores (asserted by the router tests); two experts whose exact biased scores differ by less
+# than twice that can swap, so a selection whose oracle margin is below ROUTE_TIE is a near-tie.
+ROUTE_TIE = 4e-6
+
+
+def same_selection(g_ids, g_gates, o_ids, o_gates, rows, rtol, atol):
+    """The chosen expert sets agree on `rows`, and every chosen expert's gate agrees. The slot order is the
+    library's fp32 score order, which may differ from the exact order only between experts whose scores lie within
+    the fp32 error of each other; it decides nothing but the order of the combine's sum."""
+    g_ids, o_ids = np.asarray(g_ids)[rows], np.asarray(o_ids)[rows]
+    gs, os_ = np.argsort(g_ids, axis=1), np.argsort(o_ids, axis=1)
+    assert np.array_equal(np.take_along_axis(g_ids, gs, 1), np.take_along_axis(o_ids, os_, 1)), \
+        "routed expert sets differ away from near-ties"
+    assert np.allclose(np.take_along_axis(np.asarray(g_gates)[rows], gs, 1),
+                       np.take_along_axis(np.asarray(o_gates)[rows], os_, 1), rtol=rtol, atol=atol)
+
+
+def slot_order_valid(ids, scores, bias, guard=None):
+    """Slots are in non-increasing biased-score order up to the fp32 error band."""
+    guard = ROUTE_TIE if guard is None else guard
+    v = np.take_along_axis(np.asarray(scores, dtype=np.float64), np.asarray(ids, dtype=np.int64), 1) + \
+        np.asarray(bias, dtype=np.float64)[np.asarray(ids, dtype=np.int64)]
+    assert np.all(np.diff(v, axis=1) <= guard), "slots out of biased-score order"
+

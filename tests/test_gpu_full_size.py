@@ -15,10 +15,10 @@ import torch
 
 from block_diffusion_moe_dllm_b200 import binding as bd
 from block_diffusion_moe_dllm_b200 import synth
-from block_diffusion_moe_dllm_b200.configs import T2I, THINKING, UNDERSTANDING
+from block_diffusion_moe_dllm_b200.configs import PREFILL, T2I, THINKING, UNDERSTANDING
 from block_diffusion_moe_dllm_b200.engine import DenoiseEngine
 from oracle import dllm_oracle as O
-from _util import assert_close, assignment_tables, random_assignments, to64
+from _util import ROUTE_TIE, assert_close, assignment_tables, random_assignments, same_selection, to64
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -96,11 +96,34 @@ def test_full_router_understanding():
     bd.moe_route(h, wr, bias, ids, gates, counts, offsets, perm, inv, Tk, H, E, k, bd.BF16)
     torch.cuda.synchronize()
     o_ids, o_gates, _, margin = O.route(to64(h), to64(wr), to64(bias), k)
-    ok = margin >= 1e-6
+    ok = margin >= ROUTE_TIE
     assert ok.mean() > 0.9
-    assert np.array_equal(ids.cpu().numpy()[ok], o_ids[ok])
-    assert np.allclose(gates.cpu().numpy()[ok], o_gates[ok], rtol=5e-6, atol=5e-7)
+    same_selection(ids.cpu().numpy(), gates.cpu().numpy(), o_ids, o_gates, ok, rtol=5e-6, atol=5e-7)
     c, off, p, iv = assignment_tables(ids.cpu().numpy(), E)
+    assert np.array_equal(perm.cpu().numpy(), p) and np.array_equal(inv.cpu().numpy(), iv)
+
+
+def test_full_router_prefill():
+    """The router over the prefill shape's 32768 tokens (262144 assignments: 128 permutation segments)."""
+    w = PREFILL
+    Tk, H, E, k = w.Tk, w.H, w.E, w.k
+    h = synth.normal((Tk, H), 1.0, 25, "frp_h", DEV)
+    wr = synth.normal((E, H), 0.02, 25, "frp_w", DEV)
+    bias = synth.uniform((E,), -0.1, 0.1, 25, "frp_b", DEV)
+    ids = torch.empty((Tk, k), dtype=torch.int32, device=DEV)
+    gates = torch.empty((Tk, k), dtype=torch.float32, device=DEV)
+    counts = torch.empty(E, dtype=torch.int32, device=DEV)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=DEV)
+    perm = torch.empty(Tk * k, dtype=torch.int32, device=DEV)
+    inv = torch.empty(Tk * k, dtype=torch.int32, device=DEV)
+    bd.moe_route(h, wr, bias, ids, gates, counts, offsets, perm, inv, Tk, H, E, k, bd.BF16)
+    torch.cuda.synchronize()
+    o_ids, o_gates, _, margin = O.route(to64(h), to64(wr), to64(bias), k)
+    ok = margin >= ROUTE_TIE
+    assert ok.mean() > 0.9
+    same_selection(ids.cpu().numpy(), gates.cpu().numpy(), o_ids, o_gates, ok, rtol=5e-6, atol=5e-7)
+    c, off, p, iv = assignment_tables(ids.cpu().numpy(), E)
+    assert np.array_equal(counts.cpu().numpy(), c) and np.array_equal(offsets.cpu().numpy(), off)
     assert np.array_equal(perm.cpu().numpy(), p) and np.array_equal(inv.cpu().numpy(), iv)
 
 

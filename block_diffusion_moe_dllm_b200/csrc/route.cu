@@ -288,29 +288,43 @@ __global__ void __launch_bounds__(256) route_seg_hist_kernel(const int32_t* __re
   for (int i = threadIdx.x; i < E; i += blockDim.x) seg_hist[(int64_t)blockIdx.x * E + i] = sh_hist[i];
 }
 
-// One thread per expert (E <= 1024): counts = column sums, offsets = their exclusive scan over experts (offsets[E] =
-// n), and seg_hist[s][e] is replaced by offsets[e] + (assignments of e in segments before s).
+// counts = column sums of the segment histograms, offsets = their exclusive scan over experts (offsets[E] = n), and
+// seg_hist[s][e] replaced by offsets[e] + (assignments of e in segments before s). 1024 threads: G = 1024 / E32
+// groups of segments per expert column (E32 = E rounded up to 32), each summing its contiguous share of the
+// segments; the groups' sums are prefixed per expert in shared memory.
 __global__ void __launch_bounds__(1024) route_seg_scan_kernel(int32_t* __restrict__ seg_hist, int S, int E, int n,
                                                               int32_t* __restrict__ counts,
                                                               int32_t* __restrict__ offsets) {
   pdl_enter();
+  __shared__ int part[1024];   // [group][expert]
   __shared__ int wtot[32];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
-  int cnt = 0;
-  if (tid < E) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int E32 = (E + 31) & ~31, G = 1024 / E32;
+  const int g = tid / E32, e = tid - g * E32;
+  const int per = (S + G - 1) / G, s0 = min(S, g * per), s1 = min(S, s0 + per);
+  int sum = 0;
+  if (g < G && e < E) {
 #pragma unroll 8
-    for (int sg = 0; sg < S; ++sg) cnt += seg_hist[(int64_t)sg * E + tid];
+    for (int sg = s0; sg < s1; ++sg) sum += seg_hist[(int64_t)sg * E + e];
   }
+  part[tid] = sum;
+  __syncthreads();
+  // expert totals and their exclusive scan: threads of group 0 (one per expert column)
+  int cnt = 0;
+  if (tid < E32)
+    for (int q = 0; q < G; ++q) cnt += part[q * E32 + tid];
   int inc = cnt;
+  if (warp < E32 / 32) {
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, inc, o);
-    if (lane >= o) inc += y;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
+    }
+    if (lane == 31) wtot[warp] = inc;
   }
-  if (lane == 31) wtot[warp] = inc;
   __syncthreads();
   if (warp == 0) {
-    int x = lane < nw ? wtot[lane] : 0;
+    int x = lane < E32 / 32 ? wtot[lane] : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int y = __shfl_up_sync(0xffffffffu, x, o);
@@ -319,18 +333,27 @@ __global__ void __launch_bounds__(1024) route_seg_scan_kernel(int32_t* __restric
     wtot[lane] = x;   // inclusive over warps
   }
   __syncthreads();
-  const int excl = inc - cnt + (warp > 0 ? wtot[warp - 1] : 0);
-  if (tid < E) {
-    counts[tid] = cnt;
-    offsets[tid] = excl;
+  if (tid < E32) {
+    const int excl = inc - cnt + (warp > 0 ? wtot[warp - 1] : 0);
+    if (tid < E) { counts[tid] = cnt; offsets[tid] = excl; }
+    // the groups' starting positions per expert
     int run = excl;
-    for (int sg = 0; sg < S; ++sg) {
-      const int v = seg_hist[(int64_t)sg * E + tid];
-      seg_hist[(int64_t)sg * E + tid] = run;
+    for (int q = 0; q < G; ++q) {
+      const int v = part[q * E32 + tid];
+      part[q * E32 + tid] = run;
       run += v;
     }
   }
   if (tid == 0) offsets[E] = n;
+  __syncthreads();
+  if (g < G && e < E) {
+    int run = part[tid];
+    for (int sg = s0; sg < s1; ++sg) {
+      const int v = seg_hist[(int64_t)sg * E + e];
+      seg_hist[(int64_t)sg * E + e] = run;
+      run += v;
+    }
+  }
 }
 
 // Segment s: its 8 warps take seg / 8 consecutive assignments each (whole 32-assignment chunks). Pass 1 counts
@@ -401,13 +424,14 @@ int launch_select_per(float* scores, const float* bias, int Tk, int E, int k, in
       return DLLM_OK;
     }
   }
-  // one warp per token, 4 per CTA: many tokens spread over all the SMs
+  // one warp per token, 4 per CTA: many tokens spread over all the SMs (one thread per token, tried for thousands
+  // of tokens, reads each 1 KB score row with 32 lines in flight per warp instruction and was 2x slower)
   launch_pdl(route_topk_kernel<PER>, (Tk + 3) / 4, 128, 0, s, scores, bias, Tk, E, k, from_logits, ids, gates);
   DLLM_CHECK_LAUNCH("route_topk_kernel");
   const int n = Tk * k, seg = route_segment(n), S = (n + seg - 1) / seg;
   launch_pdl(route_seg_hist_kernel, S, 256, (size_t)E * sizeof(int), s, (const int32_t*)ids, n, E, seg, seg_scratch);
   DLLM_CHECK_LAUNCH("route_seg_hist_kernel");
-  launch_pdl(route_seg_scan_kernel, 1, 32 * ((E + 31) / 32), 0, s, seg_scratch, S, E, n, counts, offsets);
+  launch_pdl(route_seg_scan_kernel, 1, 1024, 0, s, seg_scratch, S, E, n, counts, offsets);
   DLLM_CHECK_LAUNCH("route_seg_scan_kernel");
   launch_pdl(route_seg_scatter_kernel, S, 256, (size_t)8 * E * sizeof(int), s, (const int32_t*)ids, n, E, seg,
              (const int32_t*)seg_scratch, perm, inv);

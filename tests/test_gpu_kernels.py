@@ -91,7 +91,8 @@ def test_gemm_f32():
                                             ("bf16", 77, 2048, 256, 8), ("bf16", 512, 2048, 256, 8),
                                             ("f32", 16, 256, 8, 2), ("bf16", 9, 256, 1024, 32),
                                             ("bf16", 20, 256, 512, 8), ("f32", 32, 128, 64, 32),
-                                            ("bf16", 4096, 512, 256, 8), ("bf16", 1001, 256, 1000, 3)])
+                                            ("bf16", 4096, 512, 256, 8), ("bf16", 1001, 256, 1000, 3),
+                                            ("f32", 4100, 64, 32, 2), ("bf16", 5000, 256, 96, 4)])
 def test_route(dtype, Tk, H, E, k):
     t = _tdt(dtype)
     h = synth.normal((Tk, H), 1.0, 5, f"rh{Tk}", DEV, t)

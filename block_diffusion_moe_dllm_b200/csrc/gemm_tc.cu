@@ -80,6 +80,20 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, volatil
   return true;
 }
 
+__device__ __forceinline__ bool wait_bar_cluster(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                                 int32_t* status, int code) {
+  uint32_t n = 0;
+  while (!tc::mbar_try_wait_cluster(bar, parity)) {
+    if (*abort_flag) return false;
+    if (++n > (1u << 22)) {
+      *abort_flag = 1;
+      if (status) atomicExch(status, code);
+      return false;
+    }
+  }
+  return true;
+}
+
 // Tile t -> (group, m-tile, first row of the n-tile, rows in the n-tile). n-tiles of one weight tile are adjacent.
 template <int BN>
 __device__ __forceinline__ void decode_tile(const Smem& sm, int m_tiles, int t, int& g, int& mt, int& n0,
@@ -633,6 +647,231 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
   }
 }
 
+// ---------------------------------------------------------------------------------------------------- CTA pairs
+// Compute-bound shapes (N tile 256): a (2, 1, 1) cluster shares every MMA (tcgen05.mma.cta_group::2, M = 256). Rank r
+// of the pair owns m-tile 2 mp + r of tile pair mp: it loads that m-tile's 128 weight rows and its half of the N
+// tile's token rows (the MMA takes N / 2 rows of B from each CTA, N rounded up to 32) and receives its m-tile's
+// accumulator in its own TMEM. Per CTA a stage moves 16 KB of weights and 16 KB of tokens for 128 x 256 x 64 MACs,
+// two thirds of a single-CTA 128 x 256 tile's 48 KB, which is what bounds the single-CTA mainloop (operand traffic
+// into shared memory per SM).
+// Roles: warp 0 of each CTA loads its own operands, both CTAs' copies completing on the leader's full barrier (the
+// leader arms it for both); warp 1 of the leader waits for it and issues the MMAs, committing stage release (empty)
+// and accumulator ready (tfull) to both CTAs at once; warps 2-5 of each CTA drain their TMEM half and arrive on the
+// leader's tempty (128 + 128 arrivals). Measured with the peer instead forwarding each landed stage to the leader
+// (a remote arrive after waiting on its own barrier): 2.5x slower, the extra hop stalling every stage.
+constexpr int PAIR_BN = 256;
+constexpr int PAIR_STAGES = 6;
+constexpr int PAIR_B_BYTES = (PAIR_BN / 2) * BK * 2;
+constexpr int PAIR_STAGE_BYTES = A_BYTES + PAIR_B_BYTES;
+constexpr int PAIR_SMEM = 1024 + PAIR_STAGES * PAIR_STAGE_BYTES + STAGING_BYTES + (int)sizeof(Smem);
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_w2,
+                    const __grid_constant__ CUtensorMap tmap_x, const KParams p) {
+  constexpr int STAGES = PAIR_STAGES;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* stages = base;
+  float* staging = reinterpret_cast<float*>(base + STAGES * PAIR_STAGE_BYTES);
+  Smem& sm = *reinterpret_cast<Smem*>(base + STAGES * PAIR_STAGE_BYTES + STAGING_BYTES);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = tc::cluster_ctarank();
+  const bool leader = rank == 0;
+  const int m_pairs = p.m_tiles / 2;
+
+  const int n_groups = p.n_dev + p.has_extra + ((p.n_dev + p.has_extra) == 0 ? 1 : 0);
+  if (tid == 0) {
+    sm.n_groups = n_groups;
+    sm.abort_flag = 0;
+    for (int s = 0; s < STAGES; ++s) {
+      tc::mbar_init(&sm.full[s], 1);
+      tc::mbar_init(&sm.empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      tc::mbar_init(&sm.tfull[b], 1);
+      tc::mbar_init(&sm.tempty[b], 256);
+    }
+    tc::mbar_init(&sm.done, 1);
+    tc::fence_mbar_init();
+  }
+  if (warp == 1) tc::tmem_alloc_pair(&sm.tmem_base, 2 * PAIR_BN);
+  __syncthreads();
+  cluster_sync();   // both CTAs' barriers exist before any cross-CTA arrive
+  pdl_enter();
+  // ---- group table (tiles counted in m-tile pairs)
+  for (int g = tid; g < n_groups; g += NUM_THREADS) {
+    int off, cnt;
+    if (g < p.n_dev) {
+      off = p.grp_off[g];
+      cnt = p.grp_cnt[g];
+    } else if (p.has_extra) {
+      off = p.extra_off;
+      cnt = p.extra_cnt;
+    } else {
+      off = 0;
+      cnt = p.cnt_dev ? min(*p.cnt_dev, p.host_cnt) : p.host_cnt;
+    }
+    sm.grp_off[g] = off;
+    sm.grp_cnt[g] = max(cnt, 0);
+  }
+  __syncthreads();
+  {
+    int* warp_tot = sm.chunk_sum;
+    const int per = (n_groups + NUM_THREADS - 1) / NUM_THREADS;
+    const int g0 = tid * per, g1 = min(n_groups, g0 + per);
+    int s = 0;
+    for (int g = g0; g < g1; ++g) s += ((sm.grp_cnt[g] + PAIR_BN - 1) / PAIR_BN) * m_pairs;
+    int inc = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
+    }
+    if (lane == 31) warp_tot[warp] = inc;
+    __syncthreads();
+    int before = 0, all = 0;
+#pragma unroll
+    for (int w2 = 0; w2 < NUM_THREADS / 32; ++w2) {
+      const int v = warp_tot[w2];
+      if (w2 < warp) before += v;
+      all += v;
+    }
+    int run = before + inc - s;
+    for (int g = g0; g < g1; ++g) {
+      sm.tile_prefix[g] = run;
+      run += ((sm.grp_cnt[g] + PAIR_BN - 1) / PAIR_BN) * m_pairs;
+    }
+    if (tid == 0) sm.total_tiles = all;
+    __syncthreads();
+  }
+  const int total = sm.total_tiles;
+  const int pair = (int)blockIdx.x >> 1, n_pairs = (int)gridDim.x >> 1;
+  const int kblocks = p.K / BK;
+  volatile int* abort_flag = &sm.abort_flag;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer (each CTA, its own halves)
+    if (tc::elect_one()) {
+      tc::prefetch_tmap(&tmap_w);
+      tc::prefetch_tmap(&tmap_x);
+      if (p.has_extra) tc::prefetch_tmap(&tmap_w2);
+      const uint64_t pol_w = tc::policy_evict_first();
+      const uint64_t pol_x = tc::policy_evict_last();
+      uint32_t it = 0;
+      bool ok = true;
+      const uint32_t full0 = tc::mapa_u32(tc::smem_u32(&sm.full[0]), 0);   // the leader's full barriers
+      for (int t = pair; t < total && ok; t += n_pairs) {
+        int g, mp, n0, nval;
+        decode_tile<PAIR_BN>(sm, m_pairs, t, g, mp, n0, nval);
+        const bool extra = p.has_extra && g == p.n_dev;
+        const CUtensorMap* wm = extra ? &tmap_w2 : &tmap_w;
+        const int64_t wrow = extra ? 0 : (int64_t)g * p.w_group_stride;
+        const int mt = 2 * mp + (int)rank;
+        const int half = min(PAIR_BN, (nval + 31) & ~31) / 2;
+        const int nb = (half + XBOX_ROWS - 1) / XBOX_ROWS;
+        const uint32_t bytes = A_BYTES + nb * XBOX_BYTES;
+        const int xrow = sm.grp_off[g] + n0 + (int)rank * half;
+        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (!wait_bar(&sm.empty[s], ph ^ 1, abort_flag, p.status, ST_TIMEOUT_PRODUCER)) { ok = false; break; }
+          uint8_t* a = stages + s * PAIR_STAGE_BYTES;
+          uint8_t* b = a + A_BYTES;
+          // both halves complete on the leader's full barrier, armed by the leader for both CTAs' bytes
+          if (leader) tc::mbar_arrive_expect_tx(&sm.full[s], 2 * bytes);
+          const uint32_t fb = full0 + 8u * s;
+          if (p.swiglu) {
+            tc::tma_load_2d_pair(a, wm, kb * BK, (int)(wrow + mt * 64), fb, pol_w);
+            tc::tma_load_2d_pair(a + A_BYTES / 2, wm, kb * BK, (int)(wrow + p.M + mt * 64), fb, pol_w);
+          } else {
+            tc::tma_load_2d_pair(a, wm, kb * BK, (int)(wrow + mt * 128), fb, pol_w);
+          }
+          for (int j = 0; j < nb; ++j)
+            tc::tma_load_2d_pair(b + j * XBOX_BYTES, &tmap_x, kb * BK, xrow + j * XBOX_ROWS, fb, pol_x);
+        }
+      }
+      if (leader) {
+        // every issued stage of both CTAs lands before the pair can leave (bounded); the peer passes the final
+        // cluster barrier only after this
+        const uint32_t first = it > (uint32_t)STAGES ? it - STAGES : 0;
+        for (uint32_t i = first; i < it; ++i) tc::mbar_wait(&sm.full[i % STAGES], (i / STAGES) & 1, 1u << 20);
+      } else if (!ok) {
+        // the peer cannot observe its own copies after an abort: give any in flight time to land
+        for (int i = 0; i < 200; ++i) __nanosleep(1000);
+      }
+    }
+  } else if (warp == 1) {
+    if (leader && tc::elect_one()) {
+      // ---------------------------------------------------------------- leader: MMA issuer for the pair
+      uint32_t it = 0, tcount = 0;
+      bool ok = true;
+      for (int t = pair; t < total && ok; t += n_pairs, ++tcount) {
+        int g, mp, n0, nval;
+        decode_tile<PAIR_BN>(sm, m_pairs, t, g, mp, n0, nval);
+        const uint32_t buf = tcount & 1, tph = (tcount >> 1) & 1;
+        if (!wait_bar_cluster(&sm.tempty[buf], tph ^ 1, abort_flag, p.status, ST_TIMEOUT_MMA)) { ok = false; break; }
+        tc::fence_after_sync();
+        const uint32_t N = (uint32_t)min(PAIR_BN, (nval + 31) & ~31);
+        const uint32_t idesc = tc::idesc_bf16_f32(256, N);
+        const uint32_t d = sm.tmem_base + buf * PAIR_BN;
+        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (!wait_bar(&sm.full[s], ph, abort_flag, p.status, ST_TIMEOUT_MMA)) { ok = false; break; }
+          tc::fence_after_sync();
+          const uint32_t a = tc::smem_u32(stages + s * PAIR_STAGE_BYTES);
+          const uint32_t b = a + A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            tc::mma_bf16_pair(d, tc::sdesc_k128(a + kk * 32), tc::sdesc_k128(b + kk * 32), idesc, kb != 0 || kk != 0);
+          tc::mma_commit_pair(&sm.empty[s], 0x3);
+        }
+        if (!ok) break;
+        tc::mma_commit_pair(&sm.tfull[buf], 0x3);
+      }
+      tc::mma_commit_pair(&sm.done, 0x1);   // all issued pair MMAs complete before TMEM is released
+      tc::mbar_wait(&sm.done, 0, 1u << 20);
+    }
+  } else {
+    // ------------------------------------------------------------------ epilogue warps 2..5 (each CTA, its half)
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const int etid = tid - 64;
+    const uint32_t tempty0 = tc::mapa_u32(tc::smem_u32(&sm.tempty[0]), 0);
+    uint32_t tcount = 0;
+    for (int t = pair; t < total; t += n_pairs, ++tcount) {
+      int g, mp, n0, nval;
+      decode_tile<PAIR_BN>(sm, m_pairs, t, g, mp, n0, nval);
+      const int mt = 2 * mp + (int)rank;
+      const uint32_t buf = tcount & 1, tph = (tcount >> 1) & 1;
+      if (!wait_bar(&sm.tfull[buf], tph, abort_flag, p.status, ST_TIMEOUT_EPILOGUE)) break;
+      tc::fence_after_sync();
+      for (int c0 = 0; c0 < nval; c0 += STAGE_COLS) {
+        float v[STAGE_COLS];
+        const uint32_t taddr = sm.tmem_base + ((uint32_t)(q * 32) << 16) + buf * PAIR_BN + c0;
+        tc::tmem_ld16(taddr, v);
+        tc::tmem_ld16(taddr + 16, v + 16);
+        tc::named_bar_sync(1, 128);
+#pragma unroll
+        for (int j = 0; j < STAGE_COLS; ++j) staging[j * 128 + row] = v[j];
+        tc::named_bar_sync(1, 128);
+        epilogue_chunk<PAIR_BN>(p, staging, g, mt, n0, nval, c0, sm.grp_off[g], etid);
+      }
+      tc::fence_before_sync();
+      tc::mbar_arrive_cluster(tempty0 + 8u * buf);
+    }
+  }
+  // neither CTA leaves (nor frees TMEM) while its peer may still signal its barriers or read its shared memory
+  __syncthreads();
+  cluster_sync();
+  if (warp == 1) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc_pair(sm.tmem_base, 2 * PAIR_BN);
+  }
+}
+
 // ---------------------------------------------------------------------------------------------------- host
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -766,6 +1005,58 @@ int launch_cluster_splitk(const GemmArgs& a, const CUtensorMap& mw, const CUtens
   return DLLM_OK;
 }
 
+static_assert(PAIR_SMEM <= SMEM_LIMIT, "shared memory budget (CTA pairs)");
+static_assert(PAIR_SMEM > 233472 / 2, "tensor-memory kernels must not share an SM");
+
+// Clusters of two resident at once for the CTA-pair kernel (cached).
+static int pair_clusters() {
+  static int n = 0;
+  if (n > 0) return n;
+  int m = 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2, 1, 1);
+  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = PAIR_SMEM;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaOccupancyMaxActiveClusters(&m, gemm_tc_pair_kernel, &cfg) != cudaSuccess || m <= 0) {
+    cudaGetLastError();
+    m = num_sms() / 2;
+  }
+  n = std::max(1, m);
+  return n;
+}
+
+int launch_pair(const CUtensorMap& mw, const CUtensorMap& mw2, const CUtensorMap& mx, const KParams& kp,
+                cudaStream_t s) {
+  static cudaError_t st = cudaFuncSetAttribute(gemm_tc_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               PAIR_SMEM);
+  if (st != cudaSuccess) return dllm_host::cuda_status(st, "cudaFuncSetAttribute(gemm_tc pair)");
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pair_clusters(), 1, 1);
+  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = PAIR_SMEM;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // see pdl_wait
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, gemm_tc_pair_kernel, mw, mw2, mx, kp);
+  if (e != cudaSuccess) return dllm_host::cuda_status(e, "cudaLaunchKernelEx(gemm_tc pair)");
+  DLLM_CHECK_LAUNCH("gemm_tc_pair_kernel");
+  return DLLM_OK;
+}
+
 }  // namespace
 
 int gemm_bf16_tc(const GemmArgs& a, cudaStream_t s) {
@@ -811,7 +1102,10 @@ int gemm_bf16_tc(const GemmArgs& a, cudaStream_t s) {
   kp.ksplit = ks;
   kp.prefetch_w = (!a.swiglu && !a.n_dev && !a.has_extra && a.host_cnt <= (ks > 1 ? 32 : bn)) ? 1 : 0;
   int st2;
-  if (ks > 1) st2 = launch_cluster_splitk(a, mw, mw2, mx, kp, s);
+  if (gemm_uses_pairs(a)) {
+    kp.prefetch_w = 0;
+    st2 = launch_pair(mw, mw2, mx, kp, s);
+  } else if (ks > 1) st2 = launch_cluster_splitk(a, mw, mw2, mx, kp, s);
   else if (bn == 32) st2 = launch<32, 9>(a, mw, mw2, mx, kp, s);
   else if (bn == 64) st2 = launch<64, 8>(a, mw, mw2, mx, kp, s);
   else if (bn == 128) st2 = launch<128, 6>(a, mw, mw2, mx, kp, s);
@@ -853,6 +1147,11 @@ int gemm_splitk_factor(const GemmArgs& a, int bn) {
   int ks = std::max(1, std::min(std::min(kblocks / 2, 8), num_sms() / tiles));
   while (ks > 1 && tiles > max_active_clusters(ks)) --ks;
   return ks;
+}
+
+bool gemm_uses_pairs(const GemmArgs& a) {
+  if (a.dtype != DLLM_BF16 || a.epi.conf_part || gemm_bn(a) != 256 || gemm_splitk_factor(a, 256) != 1) return false;
+  return a.swiglu ? (a.M / 64) % 2 == 0 : (a.M / 128) % 2 == 0;
 }
 
 int gemm_conf_parts(const GemmArgs& a) {

@@ -85,6 +85,8 @@ size_t gemm_f32_scratch_bytes(int64_t x_rows, int M, int swiglu);
 // fuse the confidence reduction into its epilogue: one per persistent CTA. 0 when it cannot (more rows than one
 // 32-row N tile, or split-K).
 int gemm_conf_parts(const GemmArgs& a);
+// True when the GEMM runs as CTA pairs sharing each MMA (N tile 256, an even number of 128-row weight tiles).
+bool gemm_uses_pairs(const GemmArgs& a);
 
 int num_sms();
 

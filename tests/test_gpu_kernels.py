@@ -51,6 +51,21 @@ def test_gemm_bf16_split_k(N, M, K):
     assert_close(to64(y), O.store(to64(y0) + to64(x) @ to64(w).T, "bf16"), "bf16", "split-K gemm")
 
 
+@pytest.mark.parametrize("N,M,K,residual", [(1200, 2048, 256, 0), (4100, 2048, 512, 1), (600, 4096, 128, 0)])
+def test_gemm_bf16_cta_pairs(N, M, K, residual):
+    """N tile 256 with enough tiles: CTA pairs share each MMA (M = 256 across two SMs, half of the N tile's rows
+    from each); ragged last N tiles (176, 4 and 88 rows)."""
+    x = synth.normal((N, K), 1.0, 10, f"px{N}", DEV)
+    w = synth.normal((M, K), 0.05, 10, f"pw{M}{K}", DEV)
+    y0 = synth.normal((N, M), 1.0, 10, f"py{N}{M}", DEV)
+    y = y0.clone()
+    bd.gemm(x, w, y, N, M, K, bd.BF16, residual=residual)
+    torch.cuda.synchronize()
+    acc = to64(x) @ to64(w).T
+    want = O.store(to64(y0) + acc, "bf16") if residual else O.store(acc, "bf16")
+    assert_close(to64(y), want, "bf16", "gemm (CTA pairs)")
+
+
 def test_gemm_bf16_residual_and_device_count():
     N, M, K = 40, 256, 256
     x = synth.normal((N, K), 1.0, 2, "rx", DEV)
@@ -127,6 +142,7 @@ def test_route(dtype, Tk, H, E, k):
                                                      ("bf16", 5, 256, 16, 4, 128, True),
                                                      ("bf16", 70, 256, 8, 2, 192, False),
                                                      ("bf16", 300, 256, 4, 2, 64, True),
+                                                     ("bf16", 600, 256, 4, 2, 128, True),
                                                      ("f32", 16, 256, 8, 2, 128, True)])
 def test_experts(dtype, Tk, H, E, k, I, shared):
     t = _tdt(dtype)

@@ -143,7 +143,9 @@ DLLM_API size_t dllm_prefix_retain_workspace_size(const dllm_retain_desc* desc);
 /*
  * MoE router ([R] "MoE 백본과 Block-wise Attention": top-k experts per token; [R] "Load Balancing": per-expert
  * bias used for selection only): s = sigmoid(h W_r^T) in fp32; ids = the k experts with the largest s + bias
- * (ties -> lower id), slots ordered by biased score; gates = s[ids] / sum(s[ids]).
+ * (ties -> lower id), slots ordered by biased score; gates = s[ids] / sum(s[ids]). s is accumulated in fp32 (on the
+ * tensor cores for bf16 with E % 128 == 0), so experts whose exact scores differ by less than its error (a few
+ * 1e-6 at H = 2048) can be chosen or ordered either way.
  * Then the token permutation used by the grouped expert GEMMs: counts[e] = #assignments to e; offsets =
  * exclusive prefix sum (offsets[E] = Tk * k); perm[r] = t * k + j of the assignment stored at sorted row r
  * (rows of one expert in increasing t); inv[t * k + j] = r.

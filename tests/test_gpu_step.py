@@ -227,6 +227,13 @@ def test_fused_confidence_equals_reduction(masked_fraction):
         assert np.array_equal(eng.tokens.cpu().numpy(), dt_.cpu().numpy())
 
 
+def test_step_cta_pairs():
+    """1024 tokens through 16 q / 4 kv heads: the QKV projection (24 weight tiles x 4 token tiles) and both expert
+    GEMMs (~256 rows per expert) run as CTA pairs sharing each MMA, through the RoPE/cache, SwiGLU and fp32 epilogues."""
+    w = scaled(SMALL, name="small-bf16-pairs", B=32, Hq=16, Hkv=4, P=64, L=32)
+    _one_pass(w, seed=31)
+
+
 def test_step_one_layer_full_size():
     """The one-layer bf16 workload at its full size (hidden 2048, 256 experts, vocab 157184, prefix 1024)."""
     _one_pass(ONE_LAYER, seed=0, random_gains=False)

@@ -245,23 +245,26 @@ __global__ void __launch_bounds__(256, reg_min_blocks<VPT>()) unmask_reduce_bf16
   block_store(p, wp, part + (int64_t)r * n_chunks + c);
 }
 
-// One warp per logical block row b (L <= 32 positions, lane i = position i). The still-masked flat positions are
-// the LM head's rows in increasing order, so the row of position (b, i) is the number of masked positions before it.
+// Selection, in two phases of one CTA. Phase A, per masked row r (the r-th still-masked position row_pos[r], cond
+// half): merge its partials (one thread per row, or a warp per row when there are many partials, as the LM head's
+// fused epilogue writes one per CTA), and park c = 1 / sum (fp32) and the candidate at the row's position in the
+// conf and sel outputs. Phase B, one warp per logical block row b (lane i = position i): the schedule, the rank of
+// each masked position (higher c first, lower position on equal c) and the writes. Positions whose confidences
+// are equal in fp32 rank by position.
 __global__ void __launch_bounds__(1024) unmask_select_kernel(Partial* part, int n_chunks, const int32_t* __restrict__ row_pos,
                                      const int32_t* __restrict__ n_rows, int B, int L, int t, int T_s, int mode,
                                      float tau, int k_max, int cfg, int vocab_offset, int32_t* tokens, uint8_t* mask,
                                      int32_t* sel, int32_t* nsel, float* conf, int32_t* remaining) {
   pdl_enter();
   __shared__ int rem_w[32];
-  __shared__ int row_cnt[1024];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  // many partials per row (the LM head's fused epilogue writes one per CTA): a warp merges each row's partials
-  // into its first slot, then the selection below reads that slot alone
-  int n_merge = n_chunks;
+  // this warp's first block row's mask, loaded ahead of phase A
+  const bool mk0 = w < B && lane < L && mask[w * L + lane] != 0;
+  const int nr = *n_rows;
   if (n_chunks > kMergeSerial) {
-    const int nr = *n_rows;
     for (int r = w; r < nr; r += nw) {
-      Partial* pr = part + (int64_t)r * n_chunks;
+      const Partial* pr = part + (int64_t)r * n_chunks;
+      const int pos = row_pos[r];
       Partial a{-INFINITY, 0x7fffffff, 0.0};
       for (int c0 = 0; c0 < n_chunks; c0 += 128) {
         Partial b4[4];
@@ -274,24 +277,30 @@ __global__ void __launch_bounds__(1024) unmask_select_kernel(Partial* part, int 
         for (int u = 0; u < 4; ++u) merge(a, b4[u]);
       }
       a = warp_merge(a);
-      if (lane == 0) pr[0] = a;
+      if (lane == 0 && pos >= 0 && pos < B * L) {
+        conf[pos] = (float)(1.0 / a.s);
+        sel[pos] = a.idx + vocab_offset;
+      }
     }
-    __syncthreads();
-    n_merge = 1;
-  }
-  // masked count of every logical row, then the exclusive prefix (rows in order)
-  for (int b = w; b < B; b += nw) {
-    const bool mk = lane < L && mask[b * L + lane] != 0;
-    const int c = __popc(__ballot_sync(0xffffffffu, mk));
-    if (lane == 0) row_cnt[b] = c;
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int run = 0;
-    for (int b = 0; b < B; ++b) {
-      const int c = row_cnt[b];
-      row_cnt[b] = run;
-      run += c;
+  } else {
+    for (int r = threadIdx.x; r < nr; r += blockDim.x) {
+      const Partial* pr = part + (int64_t)r * n_chunks;
+      const int pos = row_pos[r];
+      Partial a = pr[0];
+      // batches of 8 independent loads, merged in chunk order
+      for (int q0 = 1; q0 < n_chunks; q0 += 8) {
+        Partial b8[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          if (q0 + u < n_chunks) b8[u] = pr[q0 + u];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          if (q0 + u < n_chunks) merge(a, b8[u]);
+      }
+      if (pos >= 0 && pos < B * L) {
+        conf[pos] = (float)(1.0 / a.s);
+        sel[pos] = a.idx + vocab_offset;
+      }
     }
   }
   __syncthreads();
@@ -299,27 +308,11 @@ __global__ void __launch_bounds__(1024) unmask_select_kernel(Partial* part, int 
   for (int b = w; b < B; b += nw) {
     const int p = b * L + lane;
     const bool valid = lane < L;
-    const bool masked = valid && mask[p] != 0;
+    const bool masked = b == w ? mk0 : (valid && mask[p] != 0);
     const unsigned mball = __ballot_sync(0xffffffffu, masked);
-    double c = 0.0;
-    int cand = -1;
-    if (masked) {
-      const int r = row_cnt[b] + __popc(mball & ((1u << lane) - 1u));
-      const Partial* pr = part + (int64_t)r * n_chunks;
-      Partial a = pr[0];
-      // batches of 8 independent loads, merged in chunk order
-      for (int q0 = 1; q0 < n_merge; q0 += 8) {
-        Partial b8[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u)
-          if (q0 + u < n_merge) b8[u] = pr[q0 + u];
-#pragma unroll
-        for (int u = 0; u < 8; ++u)
-          if (q0 + u < n_merge) merge(a, b8[u]);
-      }
-      c = 1.0 / a.s;
-      cand = a.idx + vocab_offset;
-    }
+    const float c = masked ? conf[p] : 0.f;
+    const int cand = masked ? sel[p] : -1;
+    __syncwarp();
     const int m = __popc(mball);
     int kt = 0;
     if (m > 0) {
@@ -327,20 +320,19 @@ __global__ void __launch_bounds__(1024) unmask_select_kernel(Partial* part, int 
       if (mode == DLLM_UNMASK_FIXED) {
         kt = min(m, floor_k);
       } else {
-        const int above = __popc(__ballot_sync(0xffffffffu, masked && c > (double)tau));
+        const int above = __popc(__ballot_sync(0xffffffffu, masked && c > tau));
         kt = min(m, max(floor_k, min(k_max, above)));
       }
     }
-    // rank among masked positions: higher confidence first, lower position on equal confidence
     int rank = 0;
     for (int j = 0; j < 32; ++j) {
-      const double cj = __shfl_sync(0xffffffffu, c, j);
+      const float cj = __shfl_sync(0xffffffffu, c, j);
       if (((mball >> j) & 1u) && (cj > c || (cj == c && j < lane))) ++rank;
     }
     const bool chosen = masked && rank < kt;
     if (valid) {
       sel[b * L + lane] = -1;
-      conf[b * L + lane] = masked ? (float)c : 0.f;
+      conf[b * L + lane] = c;
     }
     __syncwarp();
     if (chosen) {

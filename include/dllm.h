@@ -190,7 +190,8 @@ DLLM_API size_t dllm_moe_experts_workspace_size(const dllm_expert_desc* desc);
  * For each still-masked position r (n_rows of them; row r is flat position row_pos[r] = b * L + i of the
  * logical rows): z = logits[r] (with cfg: z = zu + cfg_scale * (zc - zu) in fp32, zc = logits[r],
  * zu = logits[n_rows + r]); candidate = vocab_offset + lowest argmax of z; c = 1 / sum_v exp(z_v - max z).
- * Per logical row b with m masked positions: k_t positions by c descending (ties -> lower position) get their
+ * Per logical row b with m masked positions: k_t positions by c descending (c rounded to fp32; equal values ->
+ * lower position) get their
  * candidate written to tokens and their mask cleared; with cfg the uncond row b + B gets the same update.
  *   logits [n_rows * (1 + cfg), V] in the storage type; row_pos [>= n_rows] int32: the still-masked flat
  *   positions of the logical rows in increasing order (row r of the logits belongs to the r-th masked position);

@@ -656,7 +656,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
 // into shared memory per SM).
 // Roles: warp 0 of each CTA loads its own operands, both CTAs' copies completing on the leader's full barrier (the
 // leader arms it for both); warp 1 of the leader waits for it and issues the MMAs, committing stage release (empty)
-// and accumulator ready (tfull) to both CTAs at once; warps 2-5 of each CTA drain their TMEM half and arrive on the
+// and accumulator ready (tfull) to the barriers of both CTAs; warps 2-5 of each CTA drain their TMEM half and arrive on the
 // leader's tempty (128 + 128 arrivals). Measured with the peer instead forwarding each landed stage to the leader
 // (a remote arrive after waiting on its own barrier): 2.5x slower, the extra hop stalling every stage.
 constexpr int PAIR_BN = 256;
@@ -805,6 +805,8 @@ gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_con
   } else if (warp == 1) {
     if (leader && tc::elect_one()) {
       // ---------------------------------------------------------------- leader: MMA issuer for the pair
+      // stage release and accumulator-ready go to the barriers at the same offsets in both CTAs
+      const uint32_t own_cl = tc::mapa_u32(tc::smem_u32(&sm), 0), peer_cl = tc::mapa_u32(tc::smem_u32(&sm), 1);
       uint32_t it = 0, tcount = 0;
       bool ok = true;
       for (int t = pair; t < total && ok; t += n_pairs, ++tcount) {
@@ -826,12 +828,14 @@ gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_con
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
             tc::mma_bf16_pair(d, tc::sdesc_k128(a + kk * 32), tc::sdesc_k128(b + kk * 32), idesc, kb != 0 || kk != 0);
-          tc::mma_commit_pair(&sm.empty[s], 0x3);
+          tc::mma_commit_pair(own_cl + (uint32_t)((uint8_t*)&sm.empty[s] - (uint8_t*)&sm));
+          tc::mma_commit_pair(peer_cl + (uint32_t)((uint8_t*)&sm.empty[s] - (uint8_t*)&sm));
         }
         if (!ok) break;
-        tc::mma_commit_pair(&sm.tfull[buf], 0x3);
+        tc::mma_commit_pair(own_cl + (uint32_t)((uint8_t*)&sm.tfull[buf] - (uint8_t*)&sm));
+        tc::mma_commit_pair(peer_cl + (uint32_t)((uint8_t*)&sm.tfull[buf] - (uint8_t*)&sm));
       }
-      tc::mma_commit_pair(&sm.done, 0x1);   // all issued pair MMAs complete before TMEM is released
+      tc::mma_commit_pair(own_cl + (uint32_t)((uint8_t*)&sm.done - (uint8_t*)&sm));   // all pair MMAs done
       tc::mbar_wait(&sm.done, 0, 1u << 20);
     }
   } else {

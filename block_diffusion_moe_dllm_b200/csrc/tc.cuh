@@ -175,7 +175,7 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 // 2D tiled load into this CTA's shared memory whose completion is counted on an mbarrier of either CTA of the pair
-// (bar_cluster: shared::cluster address, here always the leader's). No multicast.
+// (bar_cluster: shared::cluster address, here always the leader's).
 __device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const CUtensorMap* map, int c0, int c1,
                                                  uint32_t bar_cluster, uint64_t policy) {
   asm volatile(
@@ -194,13 +194,11 @@ __device__ __forceinline__ void mma_bf16_pair(uint32_t tmem_d, uint64_t adesc, u
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(z)
       : "memory");
 }
-// Arrive once on the mbarrier at this offset in every CTA of cta_mask when this thread's MMAs have completed.
-__device__ __forceinline__ void mma_commit_pair(uint64_t* bar, uint16_t cta_mask) {
-  asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
-          smem_u32(bar)),
-      "h"(cta_mask)
-      : "memory");
+// Arrive once on the mbarrier at a shared::cluster address (this CTA's or the peer's) when every pair MMA issued so
+// far by this thread has completed.
+__device__ __forceinline__ void mma_commit_pair(uint32_t bar_cluster) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar_cluster)
+               : "memory");
 }
 // TMEM allocation for the pair: warp 1 of both CTAs executes it.
 __device__ __forceinline__ void tmem_alloc_pair(uint32_t* dst_smem, uint32_t ncols) {

@@ -476,13 +476,13 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
           if (it < (uint32_t)npf) {   // weight stage already in flight: arrive with the activation bytes
             tc::mbar_arrive_expect_tx(&sm.full[s], bytes - A_BYTES);
           } else {
-          tc::mbar_arrive_expect_tx(&sm.full[s], bytes);
-          if (p.swiglu) {
-            tc::tma_load_2d(a, wm, kb * BK, (int)(wrow + mt * 64), &sm.full[s], pol_w);
-            tc::tma_load_2d(a + A_BYTES / 2, wm, kb * BK, (int)(wrow + p.M + mt * 64), &sm.full[s], pol_w);
-          } else {
-            tc::tma_load_2d(a, wm, kb * BK, (int)(wrow + mt * 128), &sm.full[s], pol_w);
-          }
+            tc::mbar_arrive_expect_tx(&sm.full[s], bytes);
+            if (p.swiglu) {
+              tc::tma_load_2d(a, wm, kb * BK, (int)(wrow + mt * 64), &sm.full[s], pol_w);
+              tc::tma_load_2d(a + A_BYTES / 2, wm, kb * BK, (int)(wrow + p.M + mt * 64), &sm.full[s], pol_w);
+            } else {
+              tc::tma_load_2d(a, wm, kb * BK, (int)(wrow + mt * 128), &sm.full[s], pol_w);
+            }
           }
           for (int j = 0; j < nb; ++j)
             tc::tma_load_2d(b + j * XBOX_BYTES, &tmap_x, kb * BK, xrow + j * XBOX_ROWS, &sm.full[s], pol_x);

@@ -94,6 +94,20 @@ def test_route_and_experts_reject_bad_arguments(lib):
     assert lib.dllm_moe_experts(C.byref(e), *([FAKE] * 11), FAKE, 1 << 30, None) == bd.ERR_UNSUPPORTED
 
 
+def test_route_workspace_covers_scores_and_permutation_segments(lib):
+    """The router's workspace holds the fp32 scores and, past 32 tokens, one expert histogram per permutation
+    segment (segments of a multiple of 256 assignments, about 128 of them at most)."""
+    lib.dllm_moe_route_workspace_size.restype = C.c_size_t
+    for Tk, E, k in [(32, 256, 8), (512, 256, 8), (32768, 256, 8), (1001, 1000, 3), (5000, 96, 4)]:
+        n = Tk * k
+        seg = max(256, ((n + 127) // 128 + 255) // 256 * 256)
+        segments = (n + seg - 1) // seg
+        assert segments <= 129
+        need = Tk * E * 4 + segments * E * 4
+        r = bd.RouteDesc(Tk, 2048, E, k, bd.BF16)
+        assert lib.dllm_moe_route_workspace_size(C.byref(r)) >= need
+
+
 def test_unmask_rejects_bad_arguments(lib):
     u = bd.UnmaskDesc(1, 64, 1024, 64, 0, 8, bd.FIXED, 0.9, 8, 0, 1.0, 0, bd.BF16)
     assert lib.dllm_unmask(C.byref(u), *([FAKE] * 10), FAKE, 1 << 30, None) == bd.ERR_SHAPE   # L > 32

@@ -39,7 +39,8 @@ Readings where the pages are silent (each also listed in the design notes):
     divided by its mean over the prefix; keep ceil(r * P) largest, ties -> lower position; kept set in
     position order.
   * threshold rule (formula stripped on the page): k_t = min(m, max(ceil(m / (T_s - t)), min(k_max, #{c > tau}))).
-  * CFG: z = z_u + s (z_c - z_u) computed in float32 (the precision in which the argmax is decided).
+  * CFG: z = z_u + s (z_c - z_u), s = cfg_scale, in fp64; decisions within the float32 rounding bound of that
+    formula are flagged as near-ties (cfg_fp32_error_bound).
   * confidence c = max softmax at temperature 1 over the scored vocabulary; candidate = lowest argmax.
   * storage rounding: wherever the library stores a tensor in its storage type (bf16 or fp32) the oracle rounds
     its fp64 value to that type (round-to-nearest-even) at the same point; between those points it is fp64.
@@ -157,11 +158,13 @@ def sigmoid(x):
     return 1.0 / (1.0 + np.exp(-x))
 
 
-def route(h, w_router, bias, k):
+def route(h, w_router, bias, k, order=False):
     """[R] "MoE 백본" top-k router with the aux-loss-free bias of [R] "Load Balancing" used for selection only.
 
     h [T, H], w_router [E, H], bias [E] -> ids [T, k] (slots in biased-score order), gates [T, k],
-    scores [T, E], margin [T] (biased score of slot k-1 minus the best unchosen biased score)."""
+    scores [T, E], margin [T]: the biased score of slot k-1 minus the best unchosen biased score (the gap that
+    decides the chosen set), or with order=True the smallest gap between consecutive biased scores among the
+    best k + 1 (the gaps that decide the set and the slot order)."""
     s = sigmoid(f64(h) @ f64(w_router).T)
     b = f64(bias)
     T, E = s.shape
@@ -170,12 +173,15 @@ def route(h, w_router, bias, k):
     margin = np.full(T, np.inf)
     for t in range(T):
         biased = s[t] + b
-        order = sorted(range(E), key=lambda e: (-biased[e], e))
-        ids[t] = order[:k]
+        order_t = sorted(range(E), key=lambda e: (-biased[e], e))
+        ids[t] = order_t[:k]
         sel = s[t, ids[t]]
         gates[t] = sel / sel.sum()
-        if k < E:
-            margin[t] = biased[order[k - 1]] - biased[order[k]]
+        top = [biased[e] for e in order_t[:k + 1]]
+        if order and len(top) > 1:
+            margin[t] = min(top[j] - top[j + 1] for j in range(len(top) - 1))
+        elif k < E:
+            margin[t] = biased[order_t[k - 1]] - biased[order_t[k]]
     return ids, gates, s, margin
 
 
@@ -216,14 +222,21 @@ def moe_delta(h, ids, gates, w_gu, w_down, w_gu_shared, w_down_shared, dtype):
 # confidence and unmasking
 
 
-def cfg_combine_f32(zc, zu, scale):
-    """Classifier-free guidance z = z_u + s (z_c - z_u), each operation rounded to float32 in this order
-    (subtract, multiply, add)."""
-    zc = np.asarray(f64(zc), dtype=np.float32)
-    zu = np.asarray(f64(zu), dtype=np.float32)
-    diff = (zc - zu).astype(np.float32)
-    prod = (np.float32(scale) * diff).astype(np.float32)
-    return (zu + prod).astype(np.float32).astype(np.float64)
+def cfg_combine(zc, zu, scale):
+    """Classifier-free guidance z = z_u + s (z_c - z_u) (the guidance formula is not printed on the pages; this
+    is the plain reading, s = cfg_scale), in fp64."""
+    zc, zu = f64(zc), f64(zu)
+    return zu + float(scale) * (zc - zu)
+
+
+def cfg_fp32_error_bound(zc, zu, scale):
+    """Largest rounding error, per row, of any evaluation of z_u + s (z_c - z_u) in float32 that rounds each of its
+    three operations to nearest: with u = 2^-24, |fl(z) - z| <= u (2 |s (z_c - z_u)| + |z|) to first order (the
+    subtraction's and the product's errors scale with s (z_c - z_u), the sum's with z); 1 % is added for the
+    second-order terms. Comparison criteria use it to flag decisions that such rounding can flip."""
+    zc, zu = f64(zc), f64(zu)
+    d = float(scale) * (zc - zu)
+    return 1.01 * 2.0 ** -24 * np.max(2.0 * np.abs(d) + np.abs(zu + d), axis=-1)
 
 
 def confidence(z):
@@ -265,22 +278,42 @@ def unmask(z_rows, row_pos, tokens, mask, t, T_s, mode=0, tau=0.9, k_max=8, voca
     """One unmasking step over a batch of block rows.
 
     z_rows [n, V]: logits of the still-masked positions, row r belongs to flat position row_pos[r] = b*L + i of
-    the conditional rows. With ``z_uncond`` given, the rows are combined by CFG first, and the selection is
-    written to both halves of the batch (rows b and b + B/2).
-    Returns dict(tokens, mask, sel [Bl, k], nsel [Bl], conf [Bl, L], cand [Bl, L], tie_rank [Bl],
-    tie_tau [Bl]) where Bl is the number of logical rows."""
+    the conditional rows. With ``z_uncond`` given, the rows are combined by CFG first (fp64), and the selection
+    is written to both halves of the batch (rows b and b + B/2).
+
+    Near-tie flags (decisions a correct implementation may take either way): a confidence margin below 1e-6
+    relative between the last chosen and the first unchosen position (tie_rank), a confidence within 1e-6 of tau
+    (tie_tau). A library that evaluates the guidance in float32 perturbs each guided logit by up to
+    cfg_fp32_error_bound (z_err per row); the bands then widen by that amount: a candidate whose top-2 guided-logit
+    gap is at most 2 z_err (tie_cand), and confidences, which move by a relative 2 z_err at most (conf_rtol).
+    Returns dict(tokens, mask, sel [Bl, k], nsel [Bl], conf [Bl, L], cand [Bl, L], tie_rank [Bl], tie_tau [Bl],
+    tie_cand [Bl, L], conf_rtol [Bl, L]) where Bl is the number of logical rows."""
     tokens = np.array(tokens, dtype=np.int64, copy=True)
     mask = np.array(mask, dtype=np.int64, copy=True)
     B, L = mask.shape
     Bl = B // 2 if z_uncond is not None else B
-    z = cfg_combine_f32(z_rows, z_uncond, cfg_scale) if z_uncond is not None else f64(z_rows)
+    if z_uncond is not None:
+        z = cfg_combine(z_rows, z_uncond, cfg_scale)
+        z_err = cfg_fp32_error_bound(z_rows, z_uncond, cfg_scale)
+    else:
+        z = f64(z_rows)
+        z_err = np.zeros(z.shape[0])
     cand_r, conf_r, _, _ = confidence(z)
+    if z.shape[1] > 1:
+        top2 = np.sort(z, axis=1)[:, -2:]
+        gap_r = top2[:, 1] - top2[:, 0]
+    else:
+        gap_r = np.full(z.shape[0], np.inf)
     conf = np.zeros((Bl, L))
     cand = np.full((Bl, L), -1, dtype=np.int64)
+    tie_cand = np.zeros((Bl, L), dtype=bool)
+    conf_rtol = np.full((Bl, L), 1e-6)
     for r, p in enumerate(row_pos):
         b, i = divmod(int(p), L)
         conf[b, i] = conf_r[r]
         cand[b, i] = cand_r[r] + vocab_offset
+        tie_cand[b, i] = z_err[r] > 0 and gap_r[r] <= 2.0 * z_err[r]
+        conf_rtol[b, i] = 1e-6 + 2.0 * z_err[r]
     sel, nsel = [], np.zeros(Bl, dtype=np.int64)
     tie_rank = np.zeros(Bl, dtype=bool)
     tie_tau = np.zeros(Bl, dtype=bool)
@@ -290,9 +323,10 @@ def unmask(z_rows, row_pos, tokens, mask, t, T_s, mode=0, tau=0.9, k_max=8, voca
         cm = conf[b][masked]
         kt = unmask_count(m, t, T_s, mode, tau, k_max, cm)
         chosen, margin = select_positions(conf[b], masked, kt)
-        tie_rank[b] = margin < 1e-6 * max(conf[b].max(), 1e-30)
+        band = 2.0 * float(conf_rtol[b].max())
+        tie_rank[b] = margin < band * max(conf[b].max(), 1e-30)
         if mode == 1 and m:
-            tie_tau[b] = bool(np.any(np.abs(cm - tau) < 1e-6))
+            tie_tau[b] = bool(np.any(np.abs(cm - tau) < 1e-6 + conf_rtol[b][masked] * cm))
         for i in chosen:
             tokens[b, i] = cand[b, i]
             mask[b, i] = 0
@@ -302,7 +336,7 @@ def unmask(z_rows, row_pos, tokens, mask, t, T_s, mode=0, tau=0.9, k_max=8, voca
         sel.append(chosen)
         nsel[b] = kt
     return dict(tokens=tokens, mask=mask, sel=sel, nsel=nsel, conf=conf, cand=cand,
-                tie_rank=tie_rank, tie_tau=tie_tau)
+                tie_rank=tie_rank, tie_tau=tie_tau, tie_cand=tie_cand, conf_rtol=conf_rtol)
 
 
 # --------------------------------------------------------------------------------------------------------------

@@ -183,6 +183,28 @@ def test_prefix_scores_invariant_under_rope():
     assert abs(O.prefix_scores(k).mean() - 1.0) < 1e-14
 
 
+def test_prefix_scores_hand_computed_mean_of_head_norms():
+    """Hand-computed case in which the mean over kv heads of the per-head l2 norms ranks the positions differently
+    from the squared norm, the l2 norm of the whole key (all heads), the largest head norm and the l1 norm.
+    Head vectors (kv head 0 | kv head 1):
+      position 0: (3, 4) | (0, 0)    head norms 5, 0     -> mean 2.5   (l1 mean 3.5, max 5, squared mean 12.5)
+      position 1: (2, 0) | (0, 3.5)  head norms 2, 3.5   -> mean 2.75  (l1 mean 2.75, max 3.5, squared mean 8.125)
+      position 2: (0, 0) | (1, 0)    head norms 0, 1     -> mean 0.5
+    Mean over the prefix = 5.75 / 3, so the normalised scores are 30/23, 33/23, 6/23, and keeping one position
+    keeps position 1 (every alternative form listed would keep position 0)."""
+    k = np.zeros((2, 3, 2))
+    k[0, 0] = (3, 4)
+    k[0, 1] = (2, 0)
+    k[1, 1] = (0, 3.5)
+    k[1, 2] = (1, 0)
+    sc = O.prefix_scores(k)
+    assert np.allclose(sc, [30 / 23, 33 / 23, 6 / 23], rtol=0, atol=1e-15)
+    keep1, _, margin = O.prefix_retain(k, None, n_keep=1)
+    assert list(keep1) == [1] and abs(margin - 3 / 23) < 1e-15
+    keep2, _, _ = O.prefix_retain(k, 2 / 3)
+    assert list(keep2) == [0, 1]
+
+
 def test_prefix_retain_brute_force_and_ties():
     Hkv, P, d = 2, 9, 4
     k = rng.standard_normal((Hkv, P, d))
@@ -258,6 +280,19 @@ def test_router_ties_lower_expert_wins():
     h = np.zeros((1, 4))                                     # every sigmoid score is 0.5
     ids, gates, _, margin = O.route(h, np.ones((6, 4)), np.zeros(6), 2)
     assert list(ids[0]) == [0, 1] and np.allclose(gates, 0.5) and margin[0] == 0.0
+
+
+def test_router_margins_set_and_order():
+    """Hand-built biased scores: the set margin is the gap between slot k-1 and the best unchosen expert; the
+    order margin is the smallest gap between consecutive biased scores among the best k + 1."""
+    # zero router weights: every score is sigmoid(0) = 1/2, so the biased scores are 1/2 + bias
+    bias = np.array([0.30, 0.10, 0.29, -0.2, 0.05])
+    h = np.zeros((1, 3))
+    ids, gates, s, set_m = O.route(h, np.zeros((5, 3)), bias, 2)
+    _, _, _, ord_m = O.route(h, np.zeros((5, 3)), bias, 2, order=True)
+    assert list(ids[0]) == [0, 2] and np.allclose(gates, 0.5)
+    assert abs(set_m[0] - 0.19) < 1e-12          # 0.79 - 0.60
+    assert abs(ord_m[0] - 0.01) < 1e-12          # 0.80 - 0.79 (slots 0 and 1 nearly swap)
 
 
 def test_moe_permutation_equivariance():
@@ -371,11 +406,47 @@ def test_unmask_selection_and_writeback():
 def test_cfg_combine_special_scales():
     zc = rng.standard_normal((3, 50)).astype(np.float32).astype(np.float64)
     zu = rng.standard_normal((3, 50)).astype(np.float32).astype(np.float64)
-    # scale 0 gives z_u exactly; scale 1 gives z_c up to the float32 rounding of (z_c - z_u) and the add
-    assert np.array_equal(O.cfg_combine_f32(zc, zu, 0.0), zu)
-    assert np.allclose(O.cfg_combine_f32(zc, zu, 1.0), zc, rtol=0, atol=1e-6)
-    z2 = O.cfg_combine_f32(zc, zu, 2.0)
-    assert np.allclose(z2, 2 * zc - zu, atol=1e-5)
+    # scale 0 is the unconditional row, scale 1 the conditional one, scale 2 the extrapolation 2 z_c - z_u
+    # (all exact in fp64 for float32 inputs)
+    assert np.array_equal(O.cfg_combine(zc, zu, 0.0), zu)
+    assert np.array_equal(O.cfg_combine(zc, zu, 1.0), zc)
+    assert np.array_equal(O.cfg_combine(zc, zu, 2.0), 2 * zc - zu)
+    assert np.array_equal(O.cfg_combine(zc, zu, 0.5), 0.5 * (zc + zu))
+
+
+def test_cfg_fp32_error_bound_covers_float32_evaluation():
+    """The bound holds for a float32 evaluation (subtract, multiply, add, each rounded to nearest) at several
+    scales and magnitudes, and is tight to within a small factor (it is not vacuous)."""
+    worst = 0.0
+    for scale in (2.0, 1.5, 3.7, 0.3):
+        for mag in (1.0, 8.0, 100.0):
+            zc = (rng.standard_normal((4, 4096)) * mag).astype(np.float32)
+            zu = (rng.standard_normal((4, 4096)) * mag).astype(np.float32)
+            s32 = np.float32(scale)
+            fl = (zu + s32 * (zc - zu).astype(np.float32)).astype(np.float32).astype(np.float64)
+            exact = O.cfg_combine(zc, zu, float(s32))
+            err = np.abs(fl - exact).max(axis=1)
+            bound = O.cfg_fp32_error_bound(zc, zu, float(s32))
+            assert np.all(err <= bound)
+            worst = max(worst, float((err / bound).max()))
+    assert worst > 0.05
+
+
+def test_unmask_flags_guided_candidate_ties():
+    """Two candidates whose guided logits differ by less than the float32 rounding bound are flagged; a clear gap
+    is not; without guidance nothing is flagged as a candidate tie."""
+    V = 64
+    zc = np.zeros((2, V))
+    zu = np.zeros((2, V))
+    zc[0, 3], zc[0, 9] = 10.0, 10.0 + 2.0 ** -20     # guided gap 2^-19, inside the bound at |z| ~ 20
+    zc[1, 3], zc[1, 9] = 10.0, 10.5
+    tok = np.full((2, 4), V - 1)
+    msk = np.ones((2, 4), dtype=np.int64)
+    u = O.unmask(zc, [0, 1], tok, msk, 0, 4, z_uncond=zu, cfg_scale=2.0)
+    assert u["tie_cand"][0, 0] and not u["tie_cand"][0, 1]
+    assert u["cand"][0, 0] == 9 and u["cand"][0, 1] == 9
+    u0 = O.unmask(zc, [0, 1], tok[:1], msk[:1], 0, 4)
+    assert not u0["tie_cand"].any() and np.all(u0["conf_rtol"] == 1e-6)
 
 
 # ---------------------------------------------------------------------------------------------- composition

@@ -24,6 +24,11 @@ class GemmDesc(C.Structure):
     _fields_ = [("N", i32), ("M", i32), ("K", i32), ("ldy", i32), ("dtype", i32), ("y_f32", i32), ("residual", i32)]
 
 
+class GroupedGemmDesc(C.Structure):
+    _fields_ = [("G", i32), ("rows", i32), ("K", i32), ("M", i32), ("swiglu", i32), ("extra_rows", i32),
+                ("max_rows_hint", i32), ("dtype", i32), ("y_f32", i32)]
+
+
 class AttnDesc(C.Structure):
     _fields_ = [("B", i32), ("Lq", i32), ("Hq", i32), ("Hkv", i32), ("d", i32), ("blk_len", i32), ("q_pos0", i32),
                 ("n_keys", i32), ("cap", i32), ("dtype", i32), ("scale", f32)]
@@ -71,7 +76,8 @@ class StepParams(C.Structure):
 
 
 class StepViews(C.Structure):
-    _fields_ = [("logits", vp), ("row_pos", vp), ("n_rows", vp), ("x_final", vp)]
+    _fields_ = [("logits", vp), ("row_pos", vp), ("n_rows", vp), ("x_final", vp), ("expert_counts", vp),
+                ("live", vp)]
 
 
 _SIGS = {
@@ -82,6 +88,8 @@ _SIGS = {
     "dllm_selftest_bounded_wait": ([vp, sz, vp], C.c_int),
     "dllm_gemm": ([C.POINTER(GemmDesc), vp, vp, vp, vp, vp, sz, vp], C.c_int),
     "dllm_gemm_workspace_size": ([C.POINTER(GemmDesc)], sz),
+    "dllm_grouped_gemm": ([C.POINTER(GroupedGemmDesc), vp, vp, vp, vp, vp, vp, vp, sz, vp], C.c_int),
+    "dllm_grouped_gemm_workspace_size": ([C.POINTER(GroupedGemmDesc)], sz),
     "dllm_block_attn": ([C.POINTER(AttnDesc), vp, vp, vp, vp, vp, vp, sz, vp], C.c_int),
     "dllm_block_attn_workspace_size": ([C.POINTER(AttnDesc)], sz),
     "dllm_prefix_retain": ([C.POINTER(RetainDesc), vp, vp, vp, vp, vp, vp, vp, sz, vp], C.c_int),
@@ -169,6 +177,16 @@ def gemm(x, w, y, N, M, K, dtype, ldy=None, y_f32=0, residual=0, n_rows_dev=None
     ws = (ws or Workspace(need, x.device)).ensure(need)
     return check(lib.dllm_gemm(C.byref(d), ptr(x), ptr(w), ptr(y), ptr(n_rows_dev), ws.addr, ws.nbytes,
                                stream_handle(stream)))
+
+
+def grouped_gemm(x, w, w_extra, counts, offsets, y, G, rows, K, M, dtype, swiglu=0, extra_rows=0, max_rows_hint=0,
+                 y_f32=0, ws=None, stream=None):
+    lib = load()
+    d = GroupedGemmDesc(G, rows, K, M, swiglu, extra_rows, max_rows_hint, dtype, y_f32)
+    need = lib.dllm_grouped_gemm_workspace_size(C.byref(d))
+    ws = (ws or Workspace(need, x.device)).ensure(need)
+    return check(lib.dllm_grouped_gemm(C.byref(d), ptr(x), ptr(w), ptr(w_extra), ptr(counts), ptr(offsets), ptr(y),
+                                       ws.addr, ws.nbytes, stream_handle(stream)))
 
 
 def block_attn(q, k_cache, v_cache, out, B, Lq, Hq, Hkv, d, blk_len, q_pos0, n_keys, cap, dtype, key_pos=None,

@@ -104,11 +104,11 @@ struct PostNorm {
 int run_experts(int dtype, int Tk, int H, int E, int k, int I, const void* h, const void* w_gu, const void* w_down,
                 const void* w_gu_s, const void* w_down_s, const int32_t* counts, const int32_t* offsets,
                 const int32_t* perm, const int32_t* inv, const float* gates, void* x, const ExpertBufs& b,
-                int32_t* status, cudaStream_t s, const PostNorm& pn = PostNorm()) {
+                int32_t* status, cudaStream_t s, const PostNorm& pn = PostNorm(), const int32_t* live = nullptr) {
   const int shared = w_gu_s != nullptr;
   const int n_assign = Tk * k;
   const int64_t rows = (int64_t)n_assign + (shared ? Tk : 0);
-  int st = launch_gather_rows(dtype, h, perm, k, Tk, shared, b.xp, H, s);
+  int st = launch_gather_rows(dtype, h, perm, k, Tk, shared, b.xp, H, s, live);
   if (st) return st;
   GemmArgs g1;
   g1.x = b.xp; g1.x_rows = rows;
@@ -118,7 +118,7 @@ int run_experts(int dtype, int Tk, int H, int E, int k, int I, const void* h, co
   g1.n_dev = E; g1.grp_off = offsets; g1.grp_cnt = counts;
   g1.has_extra = shared; g1.extra_off = n_assign; g1.extra_cnt = Tk;
   g1.max_cnt = expert_bn_hint(Tk, k, E); g1.cnt_bound = Tk;
-  g1.dtype = dtype; g1.status = status; g1.f32_scratch = b.scratch;
+  g1.dtype = dtype; g1.status = status; g1.f32_scratch = b.scratch; g1.live = live;
   g1.epi.kind = EPI_SWIGLU; g1.epi.out = b.act; g1.epi.ldo = I;
   st = run_gemm(g1, s);
   if (st) return st;
@@ -131,8 +131,8 @@ int run_experts(int dtype, int Tk, int H, int E, int k, int I, const void* h, co
   if (st) return st;
   if (pn.g)
     return launch_combine_norm(dtype, x, b.y, gates, inv, k, Tk, shared, H, pn.g, pn.eps, pn.out, pn.mode, pn.mask,
-                               pn.n_half_pos, pn.n_dev, s);
-  return launch_combine(dtype, x, b.y, gates, inv, k, Tk, shared, H, s);
+                               pn.n_half_pos, pn.n_dev, s, live);
+  return launch_combine(dtype, x, b.y, gates, inv, k, Tk, shared, H, s, live);
 }
 
 // Rows the fused row kernels handle: 16-byte vectors, at most kRowVecs of them per thread of a 256-thread CTA.
@@ -254,7 +254,7 @@ void plan_step(const dllm_model* m, const dllm_state* st, const dllm_step_params
   s.scores = c.take<float>((size_t)s.Tk * m->E * 4);
   s.ids = c.take<int32_t>((size_t)s.Tk * m->k * 4);
   s.gates = c.take<float>((size_t)s.Tk * m->k * 4);
-  s.counts = c.take<int32_t>((size_t)(m->E + 1) * 4);
+  s.counts = c.take<int32_t>((size_t)m->n_layers * (m->E + 1) * 4);   // one histogram per layer (kept for views)
   s.offsets = c.take<int32_t>((size_t)(m->E + 1) * 4);
   s.perm = c.take<int32_t>((size_t)s.Tk * m->k * 4);
   s.inv = c.take<int32_t>((size_t)s.Tk * m->k * 4);
@@ -351,6 +351,43 @@ int dllm_gemm(const dllm_gemm_desc* d, const void* x, const void* w, void* y, co
   a.f32_scratch = d->dtype == DLLM_F32 ? c.take<float>(gemm_f32_scratch_bytes(d->N, d->M, 0)) : nullptr;
   a.epi.kind = d->residual ? EPI_RESID : EPI_STORE;
   a.epi.out = y; a.epi.ldo = d->ldy; a.epi.out_f32 = d->y_f32 || d->dtype == DLLM_F32;
+  return run_gemm(a, stream);
+}
+
+// ------------------------------------------------------------------------------------------------ grouped GEMM
+size_t dllm_grouped_gemm_workspace_size(const dllm_grouped_gemm_desc* d) {
+  if (!d) return 0;
+  return align256(kStatusBytes);
+}
+
+int dllm_grouped_gemm(const dllm_grouped_gemm_desc* d, const void* x, const void* w, const void* w_extra,
+                      const int32_t* counts, const int32_t* offsets, void* y, void* ws, size_t ws_bytes,
+                      cudaStream_t stream) {
+  REQ(d && x && w && counts && offsets && y, DLLM_ERR_INVALID_ARG, "grouped_gemm: NULL argument");
+  REQ(d->G >= 1 && d->G <= 4096 && d->rows >= 0 && d->K > 0 && d->M > 0 && d->extra_rows >= 0 &&
+          d->extra_rows <= d->rows,
+      DLLM_ERR_SHAPE, "grouped_gemm: bad G/rows/K/M/extra_rows");
+  REQ((w_extra != nullptr) == (d->extra_rows > 0), DLLM_ERR_INVALID_ARG,
+      "grouped_gemm: w_extra must be given exactly when extra_rows > 0");
+  REQ(d->dtype == DLLM_BF16, DLLM_ERR_UNSUPPORTED, "grouped_gemm: bf16 only");
+  REQ(d->K % 64 == 0 && (d->swiglu ? d->M % 64 == 0 : d->M % 128 == 0), DLLM_ERR_UNSUPPORTED,
+      "grouped_gemm: needs K %% 64 == 0 and M %% 128 == 0 (swiglu: M %% 64 == 0)");
+  REQ(!(d->swiglu && d->y_f32), DLLM_ERR_UNSUPPORTED, "grouped_gemm: swiglu output is in the storage type");
+  REQ(aligned16(x) && aligned16(w) && (!w_extra || aligned16(w_extra)) && aligned16(y), DLLM_ERR_ALIGN,
+      "grouped_gemm: X, W, W_extra and Y must be 16-byte aligned");
+  int st = check_ws(ws, ws_bytes, dllm_grouped_gemm_workspace_size(d));
+  if (st) return st;
+  if (d->rows == 0) return DLLM_OK;
+  const int Mw = d->swiglu ? 2 * d->M : d->M;
+  GemmArgs a;
+  a.x = x; a.x_rows = d->rows;
+  a.w = w; a.w_rows = (int64_t)d->G * Mw; a.w2 = w_extra; a.w2_rows = w_extra ? Mw : 0;
+  a.K = d->K; a.M = d->M; a.swiglu = d->swiglu; a.w_group_stride = Mw;
+  a.n_dev = d->G; a.grp_off = offsets; a.grp_cnt = counts;
+  a.has_extra = w_extra != nullptr; a.extra_off = d->rows - d->extra_rows; a.extra_cnt = d->extra_rows;
+  a.max_cnt = std::max(1, std::min(d->max_rows_hint > 0 ? d->max_rows_hint : d->rows, d->rows));
+  a.cnt_bound = d->rows; a.dtype = DLLM_BF16; a.status = status_word(ws);
+  a.epi.kind = d->swiglu ? EPI_SWIGLU : EPI_STORE; a.epi.out = y; a.epi.ldo = d->M; a.epi.out_f32 = d->y_f32;
   return run_gemm(a, stream);
 }
 
@@ -526,6 +563,8 @@ int dllm_denoise_step_views(const dllm_model* m, const dllm_state* st, const dll
   v->row_pos = s.row_pos;
   v->n_rows = s.n_rows;
   v->x_final = s.x;
+  v->expert_counts = s.counts;
+  v->live = s.n_rows + 2;
   return DLLM_OK;
 }
 
@@ -547,6 +586,10 @@ int dllm_denoise_step(const dllm_model* m, const dllm_state* st, const dllm_step
     if (_r) return _r;    \
   } while (0)
 
+  // live word of a denoising pass (written by the masked-row list below): once the block has no masked position
+  // left, every later kernel of the pass returns at once, so extra passes of a finished block cost only their
+  // launches. A commit pass always runs.
+  const int32_t* live = p->commit ? nullptr : s.n_rows + 2;
   const bool fuse = fused_rows_ok(dt, H);
   if (fuse) {
     // embedding, layer 0's attention-input norm and (denoising passes) the masked-row list in one launch
@@ -573,7 +616,7 @@ int dllm_denoise_step(const dllm_model* m, const dllm_state* st, const dllm_step
     GemmArgs g;
     g.x = s.h; g.x_rows = s.Tk; g.w = Ly.w_qkv; g.w_rows = (int64_t)(m->Hq + 2 * m->Hkv) * m->d; g.K = H;
     g.M = (m->Hq + 2 * m->Hkv) * m->d; g.host_cnt = s.Tk; g.max_cnt = s.Tk; g.cnt_bound = s.Tk; g.dtype = dt;
-    g.status = status; g.f32_scratch = s.proj_scratch;
+    g.status = status; g.f32_scratch = s.proj_scratch; g.live = live;
     g.epi.kind = EPI_QKV; g.epi.q_out = s.q; g.epi.Hq = m->Hq; g.epi.Hkv = m->Hkv; g.epi.d = m->d; g.epi.L = L;
     g.epi.pos0 = P; g.epi.rope_base = m->rope_base;
     if (p->sprint) {
@@ -589,18 +632,21 @@ int dllm_denoise_step(const dllm_model* m, const dllm_state* st, const dllm_step
     aa.n_keys = s.n_keys; aa.cap = p->sprint ? st->cap_thin : st->cap; aa.dtype = dt; aa.scale = 0.f;
     aa.q = s.q; aa.k = p->sprint ? Ly.k_thin : Ly.k_cache; aa.v = p->sprint ? Ly.v_thin : Ly.v_cache;
     aa.key_pos = p->sprint ? Ly.keep_pos : nullptr; aa.out = s.ao; aa.ws = s.attn_ws; aa.ws_bytes = s.attn_ws_bytes;
+    aa.live = live;
     TRY(launch_attn(aa, status, stream));
     // output projection + residual
     GemmArgs go;
     go.x = s.ao; go.x_rows = s.Tk; go.w = Ly.w_o; go.w_rows = H; go.K = QD; go.M = H; go.host_cnt = s.Tk;
     go.max_cnt = s.Tk; go.cnt_bound = s.Tk; go.dtype = dt; go.status = status; go.f32_scratch = s.proj_scratch;
+    go.live = live;
     go.epi.kind = EPI_RESID; go.epi.out = s.x; go.epi.ldo = H; go.epi.out_f32 = dt == DLLM_F32;
     TRY(run_gemm(go, stream));
     if (p->commit && last) break;  // the last layer's FFN output has no consumer in a commit pass
     // MoE FFN
     TRY(launch_rmsnorm(dt, s.x, Ly.ffn_norm, s.h, s.Tk, H, m->eps, nullptr, nullptr, 0, 0, stream));
-    TRY(launch_route(dt, s.h, Ly.w_router, Ly.router_bias, s.Tk, H, m->E, m->k, s.ids, s.gates, s.scores, s.counts,
-                     s.offsets, s.perm, s.inv, s.route_seg, stream));
+    int32_t* counts = s.counts + (size_t)l * (m->E + 1);
+    TRY(launch_route(dt, s.h, Ly.w_router, Ly.router_bias, s.Tk, H, m->E, m->k, s.ids, s.gates, s.scores, counts,
+                     s.offsets, s.perm, s.inv, s.route_seg, stream, live));
     PostNorm pn;
     if (fuse && !last) {           // next layer's attention-input norm
       pn.g = m->layers[l + 1].attn_norm; pn.eps = m->eps; pn.out = s.h; pn.mode = NORM_NEXT;
@@ -609,7 +655,7 @@ int dllm_denoise_step(const dllm_model* m, const dllm_state* st, const dllm_step
       pn.n_half_pos = s.Bl * L; pn.n_dev = s.n_rows;
     }
     TRY(run_experts(dt, s.Tk, H, m->E, m->k, m->I, s.h, Ly.w_gu, Ly.w_down, Ly.w_gu_shared, Ly.w_down_shared,
-                    s.counts, s.offsets, s.perm, s.inv, s.gates, s.x, s.eb, status, stream, pn));
+                    counts, s.offsets, s.perm, s.inv, s.gates, s.x, s.eb, status, stream, pn, live));
   }
   if (p->commit) return DLLM_OK;
   // final norm on the masked rows (cond, then uncond) unless fused above, LM head, confidence + unmasking

@@ -33,11 +33,13 @@ struct AttnK {
   float* po;  // [splits, B, Lq, Hq, d] partial outputs (unnormalised) when n_splits > 1
   float* pm;  // [splits, B, Lq, Hq] running max (log2 domain)
   float* pl;  // [splits, B, Lq, Hq] running sum
+  const int32_t* live;  // nullable: *live == 0 = nothing to do
 };
 
 template <typename T>
 __global__ void __launch_bounds__(256) attn_simt_kernel(const AttnK p) {
   pdl_enter();
+  if (p.live && *p.live == 0) return;   // a pass with no masked position left does nothing
   extern __shared__ float sm[];
   float* qs = sm;                  // [ROWS][DP]
   float* ks = qs + ROWS * DP;      // [KB][DP]
@@ -168,6 +170,7 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(const AttnK p) {
 template <typename T>
 __global__ void attn_merge_kernel(const AttnK p) {
   pdl_enter();
+  if (p.live && *p.live == 0) return;
   const int64_t nq = (int64_t)p.B * p.Lq * p.Hq;
   const int64_t qh = blockIdx.x;
   if (qh >= nq) return;
@@ -218,7 +221,7 @@ int launch_attn_simt(const AttnArgs& a, cudaStream_t s) {
   plan(a.B, a.Lq, a.Hq, a.Hkv, a.n_keys, p.qt_rows, p.n_qtiles, p.n_splits, p.keys_per_split);
   const float scale = a.scale > 0.f ? a.scale : 1.0f / sqrtf((float)a.d);
   p.scale_log2 = scale * 1.4426950408889634f;
-  p.q = a.q; p.k = a.k; p.v = a.v; p.key_pos = a.key_pos; p.out = a.out;
+  p.q = a.q; p.k = a.k; p.v = a.v; p.key_pos = a.key_pos; p.out = a.out; p.live = a.live;
   p.po = p.pm = p.pl = nullptr;
   if (p.n_splits > 1) {
     const size_t nq = (size_t)a.B * a.Lq * a.Hq;

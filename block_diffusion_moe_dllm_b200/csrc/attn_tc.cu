@@ -76,6 +76,7 @@ struct AttnTcParams {
   float* xscratch;      // split exchange: [B*Hkv*n_qtiles][n_splits][128 rows][kRecvStride] (n_splits > 1)
   __nv_bfloat16* out;   // [B, Lq, Hq, 128]
   int32_t* status;
+  const int32_t* live;  // nullable: *live == 0 = a denoising pass with no masked position left (nothing to do)
 };
 
 // Shared-memory descriptor of an MN-major operand with 128-byte swizzling: rows of 128 bytes along K (one key per
@@ -275,6 +276,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   if (warp == 1) tc::tmem_alloc(&bar.tmem_base, 512);
   __syncthreads();
   pdl_enter();         // everything above is on-chip set-up
+  if (p.live && *p.live == 0) {
+    // nothing to do: no copy or MMA was issued, so free the tensor memory and leave (every CTA of every cluster
+    // reads the same word and leaves here, before any cluster barrier or distributed shared memory access)
+    __syncthreads();
+    if (warp == 1) tc::tmem_dealloc(bar.tmem_base, 512);
+    return;
+  }
   volatile int* abort_flag = &bar.abort_flag;
   const uint32_t tS = bar.tmem_base;          // S buffers (group 0, group 1) at columns [0,128) and [128,256)
   const uint32_t tO = bar.tmem_base + 256;    // O_0, O_1 at columns [256,384) and [384,512)
@@ -766,6 +774,7 @@ int launch_attn_tc(const AttnArgs& a, int32_t* status, cudaStream_t s) {
   }
   p.out = static_cast<__nv_bfloat16*>(a.out);
   p.status = status;
+  p.live = a.live;
   CUtensorMap mq, mk, mv;
   {
     cuuint64_t dims[4] = {128, (cuuint64_t)a.Hq, (cuuint64_t)a.Lq, (cuuint64_t)a.B};

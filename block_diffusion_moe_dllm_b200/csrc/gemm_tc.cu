@@ -60,6 +60,7 @@ struct KParams {
   const int32_t* grp_off;
   const int32_t* grp_cnt;
   const int32_t* cnt_dev;
+  const int32_t* live;     // nullable: *live == 0 empties every group (a denoising pass with no masked position)
   EpiParams epi;
   int32_t* status;
   int prefetch_w;          // 1: dense with at most BN rows, so a CTA's first tile is m-tile = its first tile index and
@@ -393,6 +394,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
   // before this one
   pdl_enter();
   // ---- group table: counts, offsets and the exclusive prefix of tiles per group
+  const bool dead = p.live && *p.live == 0;
   for (int g = tid; g < n_groups; g += NUM_THREADS) {
     int off, cnt;
     if (g < p.n_dev) {
@@ -406,7 +408,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
       cnt = p.cnt_dev ? min(*p.cnt_dev, p.host_cnt) : p.host_cnt;
     }
     sm.grp_off[g] = off;
-    sm.grp_cnt[g] = max(cnt, 0);
+    sm.grp_cnt[g] = dead ? 0 : max(cnt, 0);
   }
   __syncthreads();
   // prefix of tiles per group: contiguous chunks per thread, a shuffle scan of the thread sums inside each warp,
@@ -604,7 +606,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
     __syncthreads();
     cluster_sync();
     bool arrived = false;
-    if (warp >= 2 && !*abort_flag) {
+    // a cluster past the device count's tiles (or of an emptied pass) owns no tile: nothing to reduce
+    if (warp >= 2 && !*abort_flag && (int)blockIdx.y < sm.total_tiles) {
       const int t = (int)blockIdx.y;
       const int rank = (int)blockIdx.x;
       int g, mt, n0, nval;
@@ -701,6 +704,7 @@ gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_con
   cluster_sync();   // both CTAs' barriers exist before any cross-CTA arrive
   pdl_enter();
   // ---- group table (tiles counted in m-tile pairs)
+  const bool dead = p.live && *p.live == 0;
   for (int g = tid; g < n_groups; g += NUM_THREADS) {
     int off, cnt;
     if (g < p.n_dev) {
@@ -714,7 +718,7 @@ gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_con
       cnt = p.cnt_dev ? min(*p.cnt_dev, p.host_cnt) : p.host_cnt;
     }
     sm.grp_off[g] = off;
-    sm.grp_cnt[g] = max(cnt, 0);
+    sm.grp_cnt[g] = dead ? 0 : max(cnt, 0);
   }
   __syncthreads();
   {
@@ -1094,6 +1098,7 @@ int gemm_bf16_tc(const GemmArgs& a, cudaStream_t s) {
   kp.grp_off = a.grp_off;
   kp.grp_cnt = a.grp_cnt;
   kp.cnt_dev = a.cnt_dev;
+  kp.live = a.live;
   kp.epi = a.epi;
   if (kp.epi.kind == EPI_QKV)
     for (int m = 0; m < 64; ++m) kp.epi.inv_freq[m] = std::pow((double)kp.epi.rope_base, -2.0 * (double)m / 128.0);

@@ -68,6 +68,7 @@ struct GemmArgs {
   int max_cnt = 0;         // typical largest group (chooses the tensor-core N tile; larger groups take more tiles)
   int cnt_bound = 0;       // true upper bound of rows in any group (sizes the SIMT grid)
   int dtype = 0;           // DLLM_BF16 / DLLM_F32
+  const int32_t* live = nullptr;  // nullable device word: 0 = the pass has nothing left to do (every group empty)
   EpiParams epi;
   int32_t* status = nullptr;
   float* f32_scratch = nullptr;  // f32 path: [x_rows, M (x2 for swiglu)] raw products

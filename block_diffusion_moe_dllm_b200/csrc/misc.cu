@@ -154,6 +154,7 @@ __global__ void masked_rows_kernel(const uint8_t* __restrict__ mask, int n_pos, 
   if (threadIdx.x == 0) {
     n_out[0] = base;
     n_out[1] = base * halves;
+    n_out[2] = base > 0;   // live word of the pass: 0 once the block has no masked position left
   }
 }
 
@@ -168,8 +169,9 @@ int launch_masked_rows(const uint8_t* mask, int n_pos, int halves, int32_t* row_
 // Xp[r] = h[perm[r] / k] for r < Tk * k (assignments grouped by expert), Xp[Tk * k + t] = h[t] (shared expert).
 template <typename T>
 __global__ void gather_rows_kernel(const T* __restrict__ h, const int32_t* __restrict__ perm, int k, int n_assign,
-                                   int shared, T* __restrict__ xp, int H) {
+                                   int shared, T* __restrict__ xp, int H, const int32_t* __restrict__ live) {
   pdl_enter();
+  if (live && *live == 0) return;   // a pass with no masked position left does nothing
   const int r = blockIdx.x;
   int src;
   if (r < n_assign) src = perm[r] / k;
@@ -182,14 +184,14 @@ __global__ void gather_rows_kernel(const T* __restrict__ h, const int32_t* __res
 }
 
 int launch_gather_rows(int dtype, const void* h, const int32_t* perm, int k, int Tk, int shared, void* xp, int H,
-                       cudaStream_t s) {
+                       cudaStream_t s, const int32_t* live) {
   const int rows = Tk * k + (shared ? Tk : 0);
   if (rows <= 0) return DLLM_OK;
   if (dtype == DLLM_BF16)
     launch_pdl(gather_rows_kernel<__nv_bfloat16>, rows, 128, 0, s, (const __nv_bfloat16*)h, perm, k, Tk * k, shared,
-                                                           (__nv_bfloat16*)xp, H);
+                                                           (__nv_bfloat16*)xp, H, live);
   else
-    launch_pdl(gather_rows_kernel<float>, rows, 128, 0, s, (const float*)h, perm, k, Tk * k, shared, (float*)xp, H);
+    launch_pdl(gather_rows_kernel<float>, rows, 128, 0, s, (const float*)h, perm, k, Tk * k, shared, (float*)xp, H, live);
   DLLM_CHECK_LAUNCH("gather_rows_kernel");
   return DLLM_OK;
 }
@@ -199,8 +201,10 @@ int launch_gather_rows(int dtype, const void* h, const int32_t* perm, int k, int
 template <typename T>
 __global__ void __launch_bounds__(128) combine_kernel(T* __restrict__ x, const float* __restrict__ y,
                                                       const float* __restrict__ gates, const int32_t* __restrict__ inv,
-                                                      int k, int n_assign, int shared, int H) {
+                                                      int k, int n_assign, int shared, int H,
+                                                      const int32_t* __restrict__ live) {
   pdl_enter();
+  if (live && *live == 0) return;   // a pass with no masked position left does nothing
   // grid (tokens, H / 512): each thread owns 4 consecutive hidden elements
   const int t = blockIdx.x;
   const int h0 = (blockIdx.y * blockDim.x + threadIdx.x) * 4;
@@ -223,13 +227,14 @@ __global__ void __launch_bounds__(128) combine_kernel(T* __restrict__ x, const f
 }
 
 int launch_combine(int dtype, void* x, const float* y, const float* gates, const int32_t* inv, int k, int Tk,
-                   int shared, int H, cudaStream_t s) {
+                   int shared, int H, cudaStream_t s, const int32_t* live) {
   if (Tk <= 0) return DLLM_OK;
   dim3 grid(Tk, (H / 4 + 127) / 128);
   if (dtype == DLLM_BF16)
-    launch_pdl(combine_kernel<__nv_bfloat16>, grid, 128, 0, s, (__nv_bfloat16*)x, y, gates, inv, k, Tk * k, shared, H);
+    launch_pdl(combine_kernel<__nv_bfloat16>, grid, 128, 0, s, (__nv_bfloat16*)x, y, gates, inv, k, Tk * k, shared, H,
+               live);
   else
-    launch_pdl(combine_kernel<float>, grid, 128, 0, s, (float*)x, y, gates, inv, k, Tk * k, shared, H);
+    launch_pdl(combine_kernel<float>, grid, 128, 0, s, (float*)x, y, gates, inv, k, Tk * k, shared, H, live);
   DLLM_CHECK_LAUNCH("combine_kernel");
   return DLLM_OK;
 }
@@ -307,6 +312,7 @@ __global__ void __launch_bounds__(256) embed_norm_kernel(const int32_t* __restri
     if (threadIdx.x == 0) {
       n_out[0] = base;
       n_out[1] = base * halves;
+      n_out[2] = base > 0;   // live word of the pass: 0 once the block has no masked position left
     }
     return;
   }
@@ -363,8 +369,10 @@ __global__ void __launch_bounds__(256) combine_norm_kernel(T* __restrict__ x, co
                                                            int shared, int H, const T* __restrict__ g, float eps,
                                                            T* __restrict__ out, int mode,
                                                            const uint8_t* __restrict__ mask, int n_half_pos,
-                                                           const int32_t* __restrict__ n_dev) {
+                                                           const int32_t* __restrict__ n_dev,
+                                                           const int32_t* __restrict__ live) {
   pdl_enter();
+  if (live && *live == 0) return;   // a pass with no masked position left does nothing (the whole CTA leaves)
   __shared__ float red[8];
   constexpr int VE = 16 / sizeof(T);
   const int t = blockIdx.x;
@@ -424,14 +432,14 @@ __global__ void __launch_bounds__(256) combine_norm_kernel(T* __restrict__ x, co
 
 int launch_combine_norm(int dtype, void* x, const float* y, const float* gates, const int32_t* inv, int k, int Tk,
                         int shared, int H, const void* g, float eps, void* out, int mode, const uint8_t* mask,
-                        int n_half_pos, const int32_t* n_dev, cudaStream_t s) {
+                        int n_half_pos, const int32_t* n_dev, cudaStream_t s, const int32_t* live) {
   if (Tk <= 0) return DLLM_OK;
   if (dtype == DLLM_BF16)
     launch_pdl(combine_norm_kernel<__nv_bfloat16>, Tk, 256, 0, s, (__nv_bfloat16*)x, y, gates, inv, k, Tk * k, shared,
-               H, (const __nv_bfloat16*)g, eps, (__nv_bfloat16*)out, mode, mask, n_half_pos, n_dev);
+               H, (const __nv_bfloat16*)g, eps, (__nv_bfloat16*)out, mode, mask, n_half_pos, n_dev, live);
   else
     launch_pdl(combine_norm_kernel<float>, Tk, 256, 0, s, (float*)x, y, gates, inv, k, Tk * k, shared, H,
-               (const float*)g, eps, (float*)out, mode, mask, n_half_pos, n_dev);
+               (const float*)g, eps, (float*)out, mode, mask, n_half_pos, n_dev, live);
   DLLM_CHECK_LAUNCH("combine_norm_kernel");
   return DLLM_OK;
 }
@@ -444,10 +452,14 @@ struct SimtGroups {
   const int32_t* grp_off;
   const int32_t* grp_cnt;
   const int32_t* cnt_dev;
+  const int32_t* live;   // nullable: *live == 0 empties every group
 };
 
 __device__ __forceinline__ void group_of(const SimtGroups& G, int g, int& off, int& cnt) {
-  if (g < G.n_dev) {
+  if (G.live && *G.live == 0) {
+    off = 0;
+    cnt = 0;
+  } else if (g < G.n_dev) {
     off = G.grp_off[g];
     cnt = G.grp_cnt[g];
   } else if (G.has_extra) {
@@ -578,7 +590,7 @@ size_t gemm_f32_scratch_bytes(int64_t x_rows, int M, int swiglu) {
 
 int gemm_f32_simt(const GemmArgs& a, cudaStream_t s) {
   DLLM_REQUIRE(a.f32_scratch != nullptr, DLLM_ERR_WORKSPACE, "fp32 projection needs scratch");
-  SimtGroups G{a.n_dev, a.has_extra, a.extra_off, a.extra_cnt, a.host_cnt, a.grp_off, a.grp_cnt, a.cnt_dev};
+  SimtGroups G{a.n_dev, a.has_extra, a.extra_off, a.extra_cnt, a.host_cnt, a.grp_off, a.grp_cnt, a.cnt_dev, a.live};
   const int n_groups = a.n_dev + a.has_extra + ((a.n_dev + a.has_extra) == 0 ? 1 : 0);
   const int Mw = a.swiglu ? 2 * a.M : a.M;
   const int max_cnt = a.cnt_bound > 0 ? a.cnt_bound : 1;

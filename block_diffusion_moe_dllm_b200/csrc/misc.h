@@ -12,10 +12,12 @@ int launch_rmsnorm(int dtype, const void* x, const void* g, void* out, int rows,
                    const int32_t* row_pos, const int32_t* n_dev, int two_halves, int uncond_off, cudaStream_t s);
 int launch_masked_rows(const uint8_t* mask, int n_pos, int halves, int32_t* row_pos, int32_t* n_out,
                        cudaStream_t s);
+// live (nullable, every launcher below that takes it): device word; 0 = the denoising pass has no masked position
+// left, and the kernel returns at once
 int launch_gather_rows(int dtype, const void* h, const int32_t* perm, int k, int Tk, int shared, void* xp, int H,
-                       cudaStream_t s);
+                       cudaStream_t s, const int32_t* live = nullptr);
 int launch_combine(int dtype, void* x, const float* y, const float* gates, const int32_t* inv, int k, int Tk,
-                   int shared, int H, cudaStream_t s);
+                   int shared, int H, cudaStream_t s, const int32_t* live = nullptr);
 // Fused row stages (bf16 rows of up to 8192 elements, fp32 up to 4096: kRowVecs 16-byte vectors per thread).
 constexpr int kRowVecs = 4;
 enum NormMode { NORM_NEXT = 0, NORM_FINAL = 1 };
@@ -24,16 +26,17 @@ int launch_embed_norm(int dtype, const int32_t* tokens, const uint8_t* mask, int
                       int halves, int32_t* row_pos, int32_t* n_out, cudaStream_t s);
 int launch_combine_norm(int dtype, void* x, const float* y, const float* gates, const int32_t* inv, int k, int Tk,
                         int shared, int H, const void* g, float eps, void* out, int mode, const uint8_t* mask,
-                        int n_half_pos, const int32_t* n_dev, cudaStream_t s);
+                        int n_half_pos, const int32_t* n_dev, cudaStream_t s, const int32_t* live = nullptr);
 
 // router
 int num_sms();
 
-// seg_scratch: route_scratch_bytes(Tk, E, k) bytes (per-segment histograms of the permutation)
+// seg_scratch: route_scratch_bytes(Tk, E, k) bytes, 256-byte aligned (per-segment histograms of the permutation and
+// the near-tie thresholds of the selection)
 int launch_route(int dtype, const void* h, const void* w_router, const float* bias, int Tk, int H, int E, int k,
                  int32_t* ids, float* gates, float* scores, int32_t* counts, int32_t* offsets, int32_t* perm,
-                 int32_t* inv, int32_t* seg_scratch, cudaStream_t s);
-int route_segment(int n_assign);
+                 int32_t* inv, void* seg_scratch, cudaStream_t s, const int32_t* live = nullptr);
+int route_segment_tokens(int Tk, int k);
 size_t route_scratch_bytes(int Tk, int E, int k);
 
 // unmask
@@ -68,6 +71,7 @@ struct AttnArgs {
   void* out;
   void* ws;
   size_t ws_bytes;
+  const int32_t* live = nullptr;   // nullable: *live == 0 = nothing to do (see launch_gather_rows)
 };
 size_t attn_workspace_bytes(int B, int Lq, int Hq, int Hkv, int d, int n_keys, int dtype);
 int launch_attn(const AttnArgs& a, int32_t* status, cudaStream_t s);

@@ -25,8 +25,10 @@ DLLM_DEV void load8(const float* p, float* f) {
 // the fp32 sum is the same on every run.
 template <typename T>
 __global__ void __launch_bounds__(256) route_scores_kernel(const T* __restrict__ h, const T* __restrict__ w, int Tk,
-                                                           int H, int E, float* __restrict__ scores) {
+                                                           int H, int E, float* __restrict__ scores,
+                                                           const int32_t* __restrict__ live) {
   pdl_enter();
+  if (live && *live == 0) return;   // a pass with no masked position left does nothing
   extern __shared__ __align__(16) unsigned char hs_raw[];
   T* hs = reinterpret_cast<T*>(hs_raw);  // [TT][H]
   const int e0 = blockIdx.x * EW, t0 = blockIdx.y * TT;
@@ -76,18 +78,24 @@ __global__ void __launch_bounds__(256) route_scores_kernel(const T* __restrict__
   }
 }
 
-// One warp per token: k rounds of warp arg-max over s + bias (ties -> lower expert id); gates = s / sum(s).
-// Lane l holds experts l, l + 32, ... in registers (biased and unbiased); the winner's unbiased score comes from the
-// owning lane by a shuffle, so the rounds touch no memory.
-// With from_logits the row holds router logits: the sigmoid scores replace them in place.
+// Guard band of the fp32 selection. The fp32 scores (tensor-core or SIMT accumulation over H, then an fp32
+// sigmoid) are within a few 1e-6 of the exact scores of the same inputs; a token whose fp32 biased scores have two
+// neighbours among its top k + 1 closer than kRouteGuard (so that rounding could change the chosen set or the slot
+// order) is decided again from exact scores (exact_redecide). Any expert whose fp32 biased score is below the
+// (k+1)-th by more than the guard cannot reach the top k, so only the experts within the guard of the (k+1)-th
+// score or above it are re-scored.
+constexpr float kRouteGuard = 2e-5f;
+
 // Top-k of one token's expert scores, one warp. Lane l owns experts e = i * 32 + l (i < PER); the selection key is
 // the biased score val = raw + bias (ties to the lower expert), the gate the unbiased raw score, renormalised over
 // the chosen k. Each lane sorts its PER candidates with an insertion network (descending val, ascending e); then
-// k rounds take the warp-wide best head (a 5-step butterfly on (val, e)) and the winning lane pops its head.
-// With from_logits the raw scores are sigmoid(logit) and are written back over the logits.
+// k rounds take the warp-wide best head (a 5-step butterfly on (val, e)) and the winning lane pops its head; one
+// more round reads the (k+1)-th value without popping it. With from_logits the raw scores are sigmoid(logit) and
+// are written back over the logits. Returns (warp-uniform) whether two consecutive values among the top k + 1
+// are closer than kRouteGuard; thr is then the (k+1)-th value minus the guard (-inf when k == E).
 template <int PER>
-DLLM_DEV void warp_topk(float* __restrict__ srow, const float* __restrict__ bias, int E, int k, int from_logits,
-                        int lane, int& my_id, float& my_gate) {
+DLLM_DEV bool warp_topk(float* __restrict__ srow, const float* __restrict__ bias, int E, int k, int from_logits,
+                        int lane, int& my_id, float& my_gate, float& thr) {
   float v[PER], r[PER];
   int e[PER];
 #pragma unroll
@@ -126,10 +134,13 @@ DLLM_DEV void warp_topk(float* __restrict__ srow, const float* __restrict__ bias
       v[0] = sw ? tv : v[0]; r[0] = sw ? tr : r[0]; e[0] = sw ? te : e[0];
     }
   }
-  float gsum = 0.f;
+  float gsum = 0.f, prev = 0.f;
+  bool near = false;
+  thr = -INFINITY;
   my_id = 0;
   my_gate = 0.f;
-  for (int j = 0; j < k; ++j) {
+  const int rounds = k < E ? k + 1 : k;
+  for (int j = 0; j < rounds; ++j) {
     float bv = v[0];
     int be = e[0];
 #pragma unroll
@@ -137,6 +148,12 @@ DLLM_DEV void warp_topk(float* __restrict__ srow, const float* __restrict__ bias
       const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
       const int oe = __shfl_xor_sync(0xffffffffu, be, o);
       if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
+    }
+    if (j > 0 && prev - bv < kRouteGuard) near = true;
+    prev = bv;
+    if (j == k) {   // the (k+1)-th value: read, not taken
+      thr = bv - kRouteGuard;
+      break;
     }
     const int win = be & 31;
     const float sc = __shfl_sync(0xffffffffu, r[0], win);
@@ -163,35 +180,128 @@ DLLM_DEV void warp_topk(float* __restrict__ srow, const float* __restrict__ bias
     if (lane == j) { my_id = be; my_gate = sc; }
   }
   my_gate = my_gate / gsum;
+  return near;
 }
 
-// One warp per token.
+// Exact dot product of two rows of H elements (H % 8 == 0), one warp; every lane returns the sum. A product of two
+// bf16 values is exact in fp32 (8 + 8 significant bits), so bf16 rows add fp32 products in fp64; fp32 rows use
+// fp64 fused multiply-adds. Either way the sum of H = 2048 terms is within about 1e-13 of the exact value.
+DLLM_DEV double warp_dot64(const __nv_bfloat16* __restrict__ a, const __nv_bfloat16* __restrict__ b, int H,
+                           int lane) {
+  double s0 = 0.0, s1 = 0.0;
+  for (int c = lane * 8; c < H; c += 256) {
+    float fa[8], fb[8];
+    bf16x8_to_f32(*reinterpret_cast<const uint4*>(a + c), fa);
+    bf16x8_to_f32(*reinterpret_cast<const uint4*>(b + c), fb);
+#pragma unroll
+    for (int u = 0; u < 8; u += 2) {
+      s0 += (double)(fa[u] * fb[u]);
+      s1 += (double)(fa[u + 1] * fb[u + 1]);
+    }
+  }
+  return warp_sum(s0 + s1);
+}
+DLLM_DEV double warp_dot64(const float* __restrict__ a, const float* __restrict__ b, int H, int lane) {
+  double s0 = 0.0, s1 = 0.0;
+  for (int c = lane * 8; c < H; c += 256) {
+    float fa[8], fb[8];
+    load8(a + c, fa);
+    load8(b + c, fb);
+#pragma unroll
+    for (int u = 0; u < 8; u += 2) {
+      s0 = fma((double)fa[u], (double)fb[u], s0);
+      s1 = fma((double)fa[u + 1], (double)fb[u + 1], s1);
+    }
+  }
+  return warp_sum(s0 + s1);
+}
+
+// The selection of one token decided from exact scores, one warp: every expert whose fp32 biased score is at
+// least thr (the (k+1)-th fp32 value minus the guard; -inf when k == E) is re-scored as sigmoid(h . w_e) + bias_e
+// in fp64 from the router's own inputs, then k rounds of warp arg-max over those (ties -> lower expert) give the
+// slots in order and the gates (unbiased fp64 scores renormalised, rounded once to fp32). Lane j < k returns slot j.
+template <int PER, typename T>
+DLLM_DEV void exact_redecide(const float* __restrict__ srow, const float* __restrict__ bias, int E, int k,
+                             const T* __restrict__ hrow, const T* __restrict__ w, int H, float thr, int lane,
+                             int& my_id, float& my_gate) {
+  __syncwarp();   // the warp's own write-back of the sigmoid scores is visible to every lane
+  double d[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int ex = i * 32 + lane;
+    d[i] = -INFINITY;
+    const bool cand = ex < E && srow[ex] + bias[ex] >= thr;
+    unsigned bal = __ballot_sync(0xffffffffu, cand);
+    while (bal) {
+      const int b = __ffs(bal) - 1;
+      bal &= bal - 1;
+      const int eb = i * 32 + b;
+      const double dot = warp_dot64(hrow, w + (int64_t)eb * H, H, lane);
+      if (lane == b) d[i] = 1.0 / (1.0 + exp(-dot)) + (double)bias[eb];
+    }
+  }
+  double gsum = 0.0, mine = 0.0;
+  my_id = 0;
+  for (int j = 0; j < k; ++j) {
+    double bv = -INFINITY;
+    int be = 0x7fffffff;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int ex = i * 32 + lane;
+      if (ex < E && (d[i] > bv || (d[i] == bv && ex < be))) { bv = d[i]; be = ex; }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const double ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+      if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
+    }
+#pragma unroll
+    for (int i = 0; i < PER; ++i)
+      if (i * 32 + lane == be) d[i] = -INFINITY;
+    const double sc = bv - (double)bias[be];
+    gsum += sc;
+    if (lane == j) { my_id = be; mine = sc; }
+  }
+  my_gate = (float)(mine / gsum);
+}
+
+// Many tokens: one warp per token, the fp32 selection. A token whose selection is a near-tie (see kRouteGuard) gets
+// fix_thr[t] = its candidate threshold, every other token NaN; the histogram launch decides those tokens again
+// before it counts.
 template <int PER>
 __global__ void route_topk_kernel(float* __restrict__ scores, const float* __restrict__ bias, int Tk, int E, int k,
-                                  int from_logits, int32_t* __restrict__ ids, float* __restrict__ gates) {
+                                  int from_logits, int32_t* __restrict__ ids, float* __restrict__ gates,
+                                  float* __restrict__ fix_thr, const int32_t* __restrict__ live) {
   pdl_enter();
+  if (live && *live == 0) return;   // a pass with no masked position left does nothing
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (warp >= Tk) return;
   int my_id;
-  float my_gate;
-  warp_topk<PER>(scores + (int64_t)warp * E, bias, E, k, from_logits, lane, my_id, my_gate);
+  float my_gate, thr;
+  const bool near = warp_topk<PER>(scores + (int64_t)warp * E, bias, E, k, from_logits, lane, my_id, my_gate, thr);
   if (lane < k) {
     ids[(int64_t)warp * k + lane] = my_id;
     gates[(int64_t)warp * k + lane] = my_gate;
   }
+  if (lane == 0) fix_thr[warp] = near ? thr : __int_as_float(0x7fc00000);
 }
 
-// Few tokens (Tk <= 32, Tk * k <= 1024, E <= 256): top-k and the stable per-expert permutation in one CTA of
-// 1024 threads. Assignment a = t * k + j; chunk c = a / 32 is handled by one warp, whose lanes with the same expert
-// find each other with __match_any_sync: an assignment's position is offsets[e] + (assignments of e in earlier
-// chunks) + (lanes of e before it in its chunk), which is the order of a, as in the general permutation kernel.
-template <int PER>
+// Few tokens (Tk <= 32, Tk * k <= 1024, E <= 256): top-k (with the exact re-decision of near-ties) and the stable
+// per-expert permutation in one CTA of 1024 threads. Assignment a = t * k + j; chunk c = a / 32 is handled by one
+// warp, whose lanes with the same expert find each other with __match_any_sync: an assignment's position is
+// offsets[e] + (assignments of e in earlier chunks) + (lanes of e before it in its chunk), which is the order of a,
+// as in the general permutation kernel.
+template <int PER, typename T>
 __global__ void __launch_bounds__(1024) route_small_kernel(float* __restrict__ scores, const float* __restrict__ bias,
                                                            int Tk, int E, int k, int from_logits,
+                                                           const T* __restrict__ h, const T* __restrict__ w, int H,
                                                            int32_t* __restrict__ ids, float* __restrict__ gates,
                                                            int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
-                                                           int32_t* __restrict__ perm, int32_t* __restrict__ inv) {
+                                                           int32_t* __restrict__ perm, int32_t* __restrict__ inv,
+                                                           const int32_t* __restrict__ live) {
   pdl_enter();
+  if (live && *live == 0) return;   // a pass with no masked position left does nothing
   extern __shared__ int rs_sm[];
   const int n = Tk * k, W = (n + 31) / 32;
   int* hist = rs_sm;                 // [W][E]: counts per chunk, then their exclusive prefix over chunks
@@ -203,8 +313,10 @@ __global__ void __launch_bounds__(1024) route_small_kernel(float* __restrict__ s
   for (int i = tid; i < W * E; i += blockDim.x) hist[i] = 0;
   for (int t = warp; t < Tk; t += nw) {
     int my_id;
-    float my_gate;
-    warp_topk<PER>(scores + (int64_t)t * E, bias, E, k, from_logits, lane, my_id, my_gate);
+    float my_gate, thr;
+    float* srow = scores + (int64_t)t * E;
+    if (warp_topk<PER>(srow, bias, E, k, from_logits, lane, my_id, my_gate, thr))
+      exact_redecide<PER>(srow, bias, E, k, h + (int64_t)t * H, w, H, thr, lane, my_id, my_gate);
     if (lane < k) {
       ids[(int64_t)t * k + lane] = my_id;
       gates[(int64_t)t * k + lane] = my_gate;
@@ -226,9 +338,9 @@ __global__ void __launch_bounds__(1024) route_small_kernel(float* __restrict__ s
   for (int ex = tid; ex < E; ex += blockDim.x) {
     int run = 0;
     for (int c = 0; c < W; ++c) {
-      const int h = hist[c * E + ex];
+      const int hh = hist[c * E + ex];
       hist[c * E + ex] = run;
-      run += h;
+      run += hh;
     }
     off_s[ex] = run;
   }
@@ -270,32 +382,63 @@ __global__ void __launch_bounds__(1024) route_small_kernel(float* __restrict__ s
   }
 }
 
-// Stable permutation for many assignments, in three launches over segments of `seg` consecutive assignments
-// (seg a multiple of 256): per-segment expert histograms; one CTA turns them into counts, offsets and every segment's
-// first output position per expert; then each segment writes its assignments' positions in order. Positions within
-// an expert follow the assignment index a = t * k + j, so an expert's rows stay sorted by token.
+// Stable permutation for many assignments, in three launches over segments of seg_tok consecutive tokens (seg_tok
+// * k assignments, a multiple of 256): per-segment expert histograms (after the segment's near-tie tokens are
+// decided again); one CTA turns them into counts, offsets and every segment's first output position per expert;
+// then each segment writes its assignments' positions in order. Positions within an expert follow the assignment
+// index a = t * k + j, so an expert's rows stay sorted by token.
 
-// seg_hist[s][e] = assignments of expert e in segment s.
-__global__ void __launch_bounds__(256) route_seg_hist_kernel(const int32_t* __restrict__ ids, int n, int E, int seg,
-                                                             int32_t* __restrict__ seg_hist) {
+// Exact re-decision of the segment's flagged tokens (a warp per token; fix_thr as written by route_topk_kernel),
+// then seg_hist[s][e] = assignments of expert e in segment s.
+template <int PER, typename T>
+__global__ void __launch_bounds__(256) route_seg_hist_kernel(int32_t* __restrict__ ids, float* __restrict__ gates,
+                                                             const float* __restrict__ scores,
+                                                             const float* __restrict__ bias,
+                                                             const float* __restrict__ fix_thr,
+                                                             const T* __restrict__ h, const T* __restrict__ w, int H,
+                                                             int Tk, int E, int k, int seg_tok,
+                                                             int32_t* __restrict__ seg_hist,
+                                                             const int32_t* __restrict__ live) {
   pdl_enter();
+  if (live && *live == 0) return;   // a pass with no masked position left does nothing
   extern __shared__ int sh_hist[];
   for (int i = threadIdx.x; i < E; i += blockDim.x) sh_hist[i] = 0;
-  __syncthreads();
-  const int a0 = blockIdx.x * seg, a1 = min(n, a0 + seg);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int t0 = blockIdx.x * seg_tok, t1 = min(Tk, t0 + seg_tok);
+  for (int tb = t0 + warp * 32; tb < t1; tb += 256) {
+    const int t = tb + lane;
+    const float th = t < t1 ? fix_thr[t] : __int_as_float(0x7fc00000);
+    unsigned bal = __ballot_sync(0xffffffffu, !isnan(th));
+    while (bal) {
+      const int j = __ffs(bal) - 1;
+      bal &= bal - 1;
+      const int tt = tb + j;
+      int my_id;
+      float my_gate;
+      exact_redecide<PER>(scores + (int64_t)tt * E, bias, E, k, h + (int64_t)tt * H, w, H,
+                          __shfl_sync(0xffffffffu, th, j), lane, my_id, my_gate);
+      if (lane < k) {
+        ids[(int64_t)tt * k + lane] = my_id;
+        gates[(int64_t)tt * k + lane] = my_gate;
+      }
+    }
+  }
+  __syncthreads();   // the re-decided ids (global writes of this CTA) are visible to the whole CTA
+  const int a0 = t0 * k, a1 = t1 * k;
   for (int a = a0 + threadIdx.x; a < a1; a += blockDim.x) atomicAdd(&sh_hist[ids[a]], 1);
   __syncthreads();
   for (int i = threadIdx.x; i < E; i += blockDim.x) seg_hist[(int64_t)blockIdx.x * E + i] = sh_hist[i];
 }
-
 // counts = column sums of the segment histograms, offsets = their exclusive scan over experts (offsets[E] = n), and
 // seg_hist[s][e] replaced by offsets[e] + (assignments of e in segments before s). 1024 threads: G = 1024 / E32
 // groups of segments per expert column (E32 = E rounded up to 32), each summing its contiguous share of the
 // segments; the groups' sums are prefixed per expert in shared memory.
 __global__ void __launch_bounds__(1024) route_seg_scan_kernel(int32_t* __restrict__ seg_hist, int S, int E, int n,
                                                               int32_t* __restrict__ counts,
-                                                              int32_t* __restrict__ offsets) {
+                                                              int32_t* __restrict__ offsets,
+                                                              const int32_t* __restrict__ live) {
   pdl_enter();
+  if (live && *live == 0) return;   // a pass with no masked position left does nothing
   __shared__ int part[1024];   // [group][expert]
   __shared__ int wtot[32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -363,8 +506,10 @@ __global__ void __launch_bounds__(1024) route_seg_scan_kernel(int32_t* __restric
 // lanes with the same expert.
 __global__ void __launch_bounds__(256) route_seg_scatter_kernel(const int32_t* __restrict__ ids, int n, int E, int seg,
                                                                 const int32_t* __restrict__ seg_base,
-                                                                int32_t* __restrict__ perm, int32_t* __restrict__ inv) {
+                                                                int32_t* __restrict__ perm, int32_t* __restrict__ inv,
+                                                                const int32_t* __restrict__ live) {
   pdl_enter();
+  if (live && *live == 0) return;   // a pass with no masked position left does nothing
   extern __shared__ int wh[];   // [8][E]
   const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
   for (int i = tid; i < 8 * E; i += blockDim.x) wh[i] = 0;
@@ -405,65 +550,96 @@ __global__ void __launch_bounds__(256) route_seg_scatter_kernel(const int32_t* _
 
 }  // namespace
 
-template <int PER>
-int launch_select_per(float* scores, const float* bias, int Tk, int E, int k, int from_logits, int32_t* ids,
-                      float* gates, int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv,
-                      int32_t* seg_scratch, cudaStream_t s) {
+// Layout of the router scratch: per-segment expert histograms, then one fp32 near-tie threshold per token.
+struct RouteScratch {
+  int seg_tok, S;
+  int32_t* seg_hist;
+  float* fix_thr;
+};
+
+RouteScratch route_scratch(int Tk, int E, int k, void* base) {
+  RouteScratch r;
+  r.seg_tok = route_segment_tokens(Tk, k);
+  r.S = std::max(1, (Tk + r.seg_tok - 1) / r.seg_tok);
+  const size_t hist = ((size_t)r.S * E * sizeof(int32_t) + 255) & ~size_t(255);
+  r.seg_hist = static_cast<int32_t*>(base);
+  r.fix_thr = base ? reinterpret_cast<float*>(static_cast<char*>(base) + hist) : nullptr;
+  return r;
+}
+
+template <int PER, typename T>
+int launch_select_per(float* scores, const float* bias, int Tk, int E, int k, int from_logits, const T* h,
+                      const T* w, int H, int32_t* ids, float* gates, int32_t* counts, int32_t* offsets, int32_t* perm,
+                      int32_t* inv, void* scratch, cudaStream_t s, const int32_t* live) {
   if constexpr (PER <= 8) {   // E <= 256: the single-CTA kernel fits its 64 registers per thread
     const int n = Tk * k, W = (n + 31) / 32;
     const size_t smem = ((size_t)W * E + 2 * (size_t)n + E) * sizeof(int);
     if (Tk <= 32 && n <= 1024 && smem <= 96 * 1024) {
       static bool cfg = false;
       if (!cfg) {
-        cudaFuncSetAttribute(route_small_kernel<PER>, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
+        cudaFuncSetAttribute(route_small_kernel<PER, T>, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
         cfg = true;
       }
-      launch_pdl(route_small_kernel<PER>, 1, 1024, smem, s, scores, bias, Tk, E, k, from_logits, ids, gates, counts,
-                 offsets, perm, inv);
+      launch_pdl(route_small_kernel<PER, T>, 1, 1024, smem, s, scores, bias, Tk, E, k, from_logits, h, w, H, ids,
+                 gates, counts, offsets, perm, inv, live);
       DLLM_CHECK_LAUNCH("route_small_kernel");
       return DLLM_OK;
     }
   }
+  const RouteScratch rs = route_scratch(Tk, E, k, scratch);
   // one warp per token, 4 per CTA: many tokens spread over all the SMs (one thread per token, tried for thousands
   // of tokens, reads each 1 KB score row with 32 lines in flight per warp instruction and was 2x slower)
-  launch_pdl(route_topk_kernel<PER>, (Tk + 3) / 4, 128, 0, s, scores, bias, Tk, E, k, from_logits, ids, gates);
+  launch_pdl(route_topk_kernel<PER>, (Tk + 3) / 4, 128, 0, s, scores, bias, Tk, E, k, from_logits, ids, gates,
+             rs.fix_thr, live);
   DLLM_CHECK_LAUNCH("route_topk_kernel");
-  const int n = Tk * k, seg = route_segment(n), S = (n + seg - 1) / seg;
-  launch_pdl(route_seg_hist_kernel, S, 256, (size_t)E * sizeof(int), s, (const int32_t*)ids, n, E, seg, seg_scratch);
+  const int n = Tk * k, seg = rs.seg_tok * k;
+  launch_pdl(route_seg_hist_kernel<PER, T>, rs.S, 256, (size_t)E * sizeof(int), s, ids, gates,
+             (const float*)scores, bias, (const float*)rs.fix_thr, h, w, H, Tk, E, k, rs.seg_tok, rs.seg_hist, live);
   DLLM_CHECK_LAUNCH("route_seg_hist_kernel");
-  launch_pdl(route_seg_scan_kernel, 1, 1024, 0, s, seg_scratch, S, E, n, counts, offsets);
+  launch_pdl(route_seg_scan_kernel, 1, 1024, 0, s, rs.seg_hist, rs.S, E, n, counts, offsets, live);
   DLLM_CHECK_LAUNCH("route_seg_scan_kernel");
-  launch_pdl(route_seg_scatter_kernel, S, 256, (size_t)8 * E * sizeof(int), s, (const int32_t*)ids, n, E, seg,
-             (const int32_t*)seg_scratch, perm, inv);
+  launch_pdl(route_seg_scatter_kernel, rs.S, 256, (size_t)8 * E * sizeof(int), s, (const int32_t*)ids, n, E, seg,
+             (const int32_t*)rs.seg_hist, perm, inv, live);
   DLLM_CHECK_LAUNCH("route_seg_scatter_kernel");
   return DLLM_OK;
 }
 
-// Selection and permutation from fp32 scores (sigmoid applied here when from_logits), E <= 1024.
-int launch_select(float* scores, const float* bias, int Tk, int E, int k, int from_logits, int32_t* ids,
-                  float* gates, int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv, int32_t* seg,
-                  cudaStream_t s) {
-  if (E <= 32) return launch_select_per<1>(scores, bias, Tk, E, k, from_logits, ids, gates, counts, offsets, perm, inv, seg, s);
-  if (E <= 64) return launch_select_per<2>(scores, bias, Tk, E, k, from_logits, ids, gates, counts, offsets, perm, inv, seg, s);
-  if (E <= 128) return launch_select_per<4>(scores, bias, Tk, E, k, from_logits, ids, gates, counts, offsets, perm, inv, seg, s);
-  if (E <= 256) return launch_select_per<8>(scores, bias, Tk, E, k, from_logits, ids, gates, counts, offsets, perm, inv, seg, s);
-  if (E <= 512) return launch_select_per<16>(scores, bias, Tk, E, k, from_logits, ids, gates, counts, offsets, perm, inv, seg, s);
-  return launch_select_per<32>(scores, bias, Tk, E, k, from_logits, ids, gates, counts, offsets, perm, inv, seg, s);
+// Selection and permutation from fp32 scores (sigmoid applied here when from_logits), E <= 1024; h and w are the
+// router's inputs, read again only for near-tie tokens.
+template <typename T>
+int launch_select(float* scores, const float* bias, int Tk, int E, int k, int from_logits, const T* h, const T* w,
+                  int H, int32_t* ids, float* gates, int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv,
+                  void* scratch, cudaStream_t s, const int32_t* live) {
+#define DLLM_SELECT(P) \
+  launch_select_per<P, T>(scores, bias, Tk, E, k, from_logits, h, w, H, ids, gates, counts, offsets, perm, inv, scratch, \
+                          s, live)
+  if (E <= 32) return DLLM_SELECT(1);
+  if (E <= 64) return DLLM_SELECT(2);
+  if (E <= 128) return DLLM_SELECT(4);
+  if (E <= 256) return DLLM_SELECT(8);
+  if (E <= 512) return DLLM_SELECT(16);
+  return DLLM_SELECT(32);
+#undef DLLM_SELECT
 }
 
-int route_segment(int n_assign) {
-  // a multiple of 256 assignments (8 warps x 32), at most about 128 segments
-  return std::max(256, ((n_assign + 127) / 128 + 255) / 256 * 256);
+int route_segment_tokens(int Tk, int k) {
+  // whole tokens per segment, seg_tok * k a multiple of 256 assignments (8 warps x 32), at most 128 segments
+  int g = 256, kk = std::max(k, 1);
+  while (kk) { const int t = g % kk; g = kk; kk = t; }   // gcd(256, k)
+  const int unit = 256 / g;
+  const int want = (std::max(Tk, 0) + 127) / 128;
+  return std::max(unit, (want + unit - 1) / unit * unit);
 }
 
 size_t route_scratch_bytes(int Tk, int E, int k) {
-  const int n = std::max(Tk, 0) * k, seg = route_segment(n);
-  return (size_t)std::max(1, (n + seg - 1) / seg) * (size_t)E * sizeof(int32_t);
+  const RouteScratch r = route_scratch(Tk, E, k, nullptr);
+  const size_t hist = ((size_t)r.S * E * sizeof(int32_t) + 255) & ~size_t(255);
+  return hist + (size_t)std::max(Tk, 1) * sizeof(float);
 }
 
 int launch_route(int dtype, const void* h, const void* w_router, const float* bias, int Tk, int H, int E, int k,
                  int32_t* ids, float* gates, float* scores, int32_t* counts, int32_t* offsets, int32_t* perm,
-                 int32_t* inv, int32_t* seg_scratch, cudaStream_t s) {
+                 int32_t* inv, void* seg_scratch, cudaStream_t s, const int32_t* live) {
   if (Tk <= 0) return DLLM_OK;
   // bf16 with a tensor-core friendly shape: router logits through the tcgen05 projection (fp32 out, accumulated
   // in fp32 in the MMA's fixed order); otherwise the SIMT score kernel
@@ -471,11 +647,12 @@ int launch_route(int dtype, const void* h, const void* w_router, const float* bi
   if (tc_logits) {
     GemmArgs g;
     g.x = h; g.x_rows = Tk; g.w = w_router; g.w_rows = E; g.K = H; g.M = E; g.host_cnt = Tk; g.max_cnt = Tk;
-    g.cnt_bound = Tk; g.dtype = DLLM_BF16;
+    g.cnt_bound = Tk; g.dtype = DLLM_BF16; g.live = live;
     g.epi.kind = EPI_STORE; g.epi.out = scores; g.epi.ldo = E; g.epi.out_f32 = 1;
     int st = gemm_bf16_tc(g, s);
     if (st) return st;
-    return launch_select(scores, bias, Tk, E, k, 1, ids, gates, counts, offsets, perm, inv, seg_scratch, s);
+    return launch_select(scores, bias, Tk, E, k, 1, (const __nv_bfloat16*)h, (const __nv_bfloat16*)w_router, H, ids,
+                         gates, counts, offsets, perm, inv, seg_scratch, s, live);
   }
   dim3 g1((E + EW - 1) / EW, (Tk + TT - 1) / TT);
   const size_t smem = (size_t)TT * H * (dtype == DLLM_BF16 ? 2 : 4);
@@ -487,17 +664,21 @@ int launch_route(int dtype, const void* h, const void* w_router, const float* bi
       cfg = true;
     }
     launch_pdl(route_scores_kernel<__nv_bfloat16>, g1, 256, smem, s, (const __nv_bfloat16*)h,
-                                                             (const __nv_bfloat16*)w_router, Tk, H, E, scores);
+                                                             (const __nv_bfloat16*)w_router, Tk, H, E, scores, live);
   } else {
     static bool cfg = false;
     if (!cfg) {
       cudaFuncSetAttribute(route_scores_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
       cfg = true;
     }
-    launch_pdl(route_scores_kernel<float>, g1, 256, smem, s, (const float*)h, (const float*)w_router, Tk, H, E, scores);
+    launch_pdl(route_scores_kernel<float>, g1, 256, smem, s, (const float*)h, (const float*)w_router, Tk, H, E, scores, live);
   }
   DLLM_CHECK_LAUNCH("route_scores_kernel");
-  return launch_select(scores, bias, Tk, E, k, 0, ids, gates, counts, offsets, perm, inv, seg_scratch, s);
+  if (dtype == DLLM_BF16)
+    return launch_select(scores, bias, Tk, E, k, 0, (const __nv_bfloat16*)h, (const __nv_bfloat16*)w_router, H, ids,
+                         gates, counts, offsets, perm, inv, seg_scratch, s, live);
+  return launch_select(scores, bias, Tk, E, k, 0, (const float*)h, (const float*)w_router, H, ids, gates, counts,
+                       offsets, perm, inv, seg_scratch, s, live);
 }
 
 }  // namespace dllm

@@ -94,12 +94,12 @@ DLLM_DEV void load8f(const float* p, float* f) {
 
 template <typename T, bool CFG>
 __global__ void __launch_bounds__(256) unmask_reduce_kernel(const T* __restrict__ logits,
-                                                            const int32_t* __restrict__ n_rows, int V, int chunk,
-                                                            float cfg_scale, Partial* __restrict__ part,
+                                                            const int32_t* __restrict__ n_rows, int max_rows, int V,
+                                                            int chunk, float cfg_scale, Partial* __restrict__ part,
                                                             int n_chunks) {
   pdl_enter();
   const int r = blockIdx.x, c = blockIdx.y;
-  const int n = *n_rows;
+  const int n = min(*n_rows, max_rows);   // the device count never exceeds the rows the buffers hold
   if (r >= n) return;
   const T* zc = logits + (int64_t)r * V;
   const T* zu = logits + (int64_t)(r + n) * V;
@@ -230,11 +230,11 @@ DLLM_DEV void load_chunk_regs(uint4 (&u)[VPT], const __nv_bfloat16* src, int nve
 // One CTA per (row, chunk); a row's chunks are adjacent CTAs (contiguous memory). V % 8 == 0.
 template <int VPT>
 __global__ void __launch_bounds__(256, reg_min_blocks<VPT>()) unmask_reduce_bf16_kernel(const __nv_bfloat16* __restrict__ logits,
-                                                                 const int32_t* __restrict__ n_rows, int V, int chunk,
-                                                                 Partial* __restrict__ part, int n_chunks) {
+                                                                 const int32_t* __restrict__ n_rows, int max_rows, int V,
+                                                                 int chunk, Partial* __restrict__ part, int n_chunks) {
   pdl_enter();
   const int r = blockIdx.y, c = blockIdx.x;
-  if (r >= *n_rows) return;
+  if (r >= min(*n_rows, max_rows)) return;
   const __nv_bfloat16* z = logits + (int64_t)r * V;
   const int v0 = c * chunk, v1 = min(V, v0 + chunk);
   const int nvec = (v1 - v0) >> 3;
@@ -252,7 +252,7 @@ __global__ void __launch_bounds__(256, reg_min_blocks<VPT>()) unmask_reduce_bf16
 // each masked position (higher c first, lower position on equal c) and the writes. Positions whose confidences
 // are equal in fp32 rank by position.
 __global__ void __launch_bounds__(1024) unmask_select_kernel(Partial* part, int n_chunks, const int32_t* __restrict__ row_pos,
-                                     const int32_t* __restrict__ n_rows, int B, int L, int t, int T_s, int mode,
+                                     const int32_t* __restrict__ n_rows, int max_rows, int B, int L, int t, int T_s, int mode,
                                      float tau, int k_max, int cfg, int vocab_offset, int32_t* tokens, uint8_t* mask,
                                      int32_t* sel, int32_t* nsel, float* conf, int32_t* remaining) {
   pdl_enter();
@@ -260,7 +260,7 @@ __global__ void __launch_bounds__(1024) unmask_select_kernel(Partial* part, int 
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
   // this warp's first block row's mask, loaded ahead of phase A
   const bool mk0 = w < B && lane < L && mask[w * L + lane] != 0;
-  const int nr = *n_rows;
+  const int nr = min(*n_rows, max_rows);   // partials exist for at most max_rows rows
   if (n_chunks > kMergeSerial) {
     for (int r = w; r < nr; r += nw) {
       const Partial* pr = part + (int64_t)r * n_chunks;
@@ -380,27 +380,27 @@ int launch_unmask(const UnmaskArgs& a, cudaStream_t s) {
     Partial* part = static_cast<Partial*>(a.partials);
     if (a.dtype == DLLM_BF16) {
       const __nv_bfloat16* z = static_cast<const __nv_bfloat16*>(a.logits);
-      if (a.cfg) launch_pdl((unmask_reduce_kernel<__nv_bfloat16, true>), grid, 256, 0, s, z, a.n_rows, a.V, chunk, a.cfg_scale, part, a.n_chunks);
+      if (a.cfg) launch_pdl((unmask_reduce_kernel<__nv_bfloat16, true>), grid, 256, 0, s, z, a.n_rows, a.max_rows, a.V, chunk, a.cfg_scale, part, a.n_chunks);
       else if (a.V % 8 == 0 && chunk <= kRegChunk) {
         // the shallowest register depth that holds a thread's share of the chunk
         const int vpt = (chunk / 8 + 255) / 256;
         const dim3 g2(a.n_chunks, a.max_rows);
-        if (vpt <= 4) launch_pdl(unmask_reduce_bf16_kernel<4>, g2, 256, 0, s, z, a.n_rows, a.V, chunk, part, a.n_chunks);
-        else if (vpt <= 8) launch_pdl(unmask_reduce_bf16_kernel<8>, g2, 256, 0, s, z, a.n_rows, a.V, chunk, part, a.n_chunks);
-        else if (vpt <= 12) launch_pdl(unmask_reduce_bf16_kernel<12>, g2, 256, 0, s, z, a.n_rows, a.V, chunk, part, a.n_chunks);
-        else launch_pdl(unmask_reduce_bf16_kernel<16>, g2, 256, 0, s, z, a.n_rows, a.V, chunk, part, a.n_chunks);
+        if (vpt <= 4) launch_pdl(unmask_reduce_bf16_kernel<4>, g2, 256, 0, s, z, a.n_rows, a.max_rows, a.V, chunk, part, a.n_chunks);
+        else if (vpt <= 8) launch_pdl(unmask_reduce_bf16_kernel<8>, g2, 256, 0, s, z, a.n_rows, a.max_rows, a.V, chunk, part, a.n_chunks);
+        else if (vpt <= 12) launch_pdl(unmask_reduce_bf16_kernel<12>, g2, 256, 0, s, z, a.n_rows, a.max_rows, a.V, chunk, part, a.n_chunks);
+        else launch_pdl(unmask_reduce_bf16_kernel<16>, g2, 256, 0, s, z, a.n_rows, a.max_rows, a.V, chunk, part, a.n_chunks);
       }
-      else launch_pdl((unmask_reduce_kernel<__nv_bfloat16, false>), grid, 256, 0, s, z, a.n_rows, a.V, chunk, a.cfg_scale, part, a.n_chunks);
+      else launch_pdl((unmask_reduce_kernel<__nv_bfloat16, false>), grid, 256, 0, s, z, a.n_rows, a.max_rows, a.V, chunk, a.cfg_scale, part, a.n_chunks);
     } else {
       const float* z = static_cast<const float*>(a.logits);
-      if (a.cfg) launch_pdl((unmask_reduce_kernel<float, true>), grid, 256, 0, s, z, a.n_rows, a.V, chunk, a.cfg_scale, part, a.n_chunks);
-      else launch_pdl((unmask_reduce_kernel<float, false>), grid, 256, 0, s, z, a.n_rows, a.V, chunk, a.cfg_scale, part, a.n_chunks);
+      if (a.cfg) launch_pdl((unmask_reduce_kernel<float, true>), grid, 256, 0, s, z, a.n_rows, a.max_rows, a.V, chunk, a.cfg_scale, part, a.n_chunks);
+      else launch_pdl((unmask_reduce_kernel<float, false>), grid, 256, 0, s, z, a.n_rows, a.max_rows, a.V, chunk, a.cfg_scale, part, a.n_chunks);
     }
     DLLM_CHECK_LAUNCH("unmask_reduce_kernel");
   }
   const int threads = a.n_chunks > kMergeSerial ? 1024 : 32 * min(32, max(1, a.B));
   launch_pdl(unmask_select_kernel, 1, threads, 0, s, static_cast<Partial*>(a.partials), a.n_chunks, a.row_pos, a.n_rows,
-                                             a.B, a.L, a.t, a.T_s, a.mode, a.tau, a.k_max, a.cfg, a.vocab_offset,
+                                             a.max_rows, a.B, a.L, a.t, a.T_s, a.mode, a.tau, a.k_max, a.cfg, a.vocab_offset,
                                              a.tokens, a.mask, a.sel, a.nsel, a.conf, a.remaining);
   DLLM_CHECK_LAUNCH("unmask_select_kernel");
   return DLLM_OK;

@@ -122,6 +122,14 @@ class DenoiseEngine:
         dt = torch_dtype(w.dtype)
         return _device_view(v.logits, numel, dt, self.ws.buf).reshape(halves * n_rows, w.vlen)
 
+    def expert_counts(self, v=None):
+        """Per layer, the assignments routed to each expert by the last pass that ran the layer: [n_layers, E + 1]
+        int32 view of the workspace (entry E unused)."""
+        w = self.w
+        v = v or self.views()
+        return _device_view(v.expert_counts, w.n_layers * (w.E + 1), torch.int32, self.ws.buf).reshape(
+            w.n_layers, w.E + 1)
+
     def x_final(self):
         w = self.w
         v = self.views()

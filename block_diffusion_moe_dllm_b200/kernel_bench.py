@@ -1,6 +1,7 @@
 """Per-kernel timing of the library's main calls at a workload's shapes (CUDA events, kernels launched alone).
 
-    python -m block_diffusion_moe_dllm_b200.kernel_bench [--kernel lm_head|proj|experts|unmask|attn|route|all]
+    python -m block_diffusion_moe_dllm_b200.kernel_bench [--kernel lm_head|proj|experts|expert_gemms|unmask|attn|
+                                                          route|all]
                                                          [--workload NAME] [--reps N]
 
 Each line reports the mean time of one call, its algorithmic bytes (weights and activations it must move at
@@ -132,6 +133,41 @@ def bench_experts(w: Workload, reps, dev, stream, weights=None):
             _result("moe_route[scores+topk+permute]", troute, rbytes, {"rows": rows})]
 
 
+def bench_expert_gemms(w: Workload, reps, dev, stream, weights=None):
+    """The two grouped expert GEMMs alone (dllm_grouped_gemm, the kernels the expert call launches), at the
+    workload's routed token rows (router output of random activations) plus the shared expert's rows: gate|up with
+    the SwiGLU epilogue, then down with fp32 rows."""
+    rows = w.B * w.L
+    lw = weights["layers"][0] if weights else synth.make_weights(
+        Workload(**{**w.__dict__, "n_layers": 1, "V": 128}), dev)["layers"][0]
+    h = synth.normal((rows, w.H), 1.0, 2, "kb_h", dev)
+    ids = torch.empty((rows, w.k), dtype=torch.int32, device=dev)
+    gates = torch.empty((rows, w.k), dtype=torch.float32, device=dev)
+    counts = torch.empty(w.E, dtype=torch.int32, device=dev)
+    offsets = torch.empty(w.E + 1, dtype=torch.int32, device=dev)
+    perm = torch.empty(rows * w.k, dtype=torch.int32, device=dev)
+    inv = torch.empty(rows * w.k, dtype=torch.int32, device=dev)
+    ws = bd.Workspace(1 << 20, dev)
+    bd.moe_route(h, lw["w_router"], lw["router_bias"], ids, gates, counts, offsets, perm, inv, rows, w.H, w.E, w.k,
+                 bd.BF16, ws=ws)
+    torch.cuda.synchronize()
+    active = int((counts > 0).sum().item())
+    n = rows * w.k + rows
+    hint = min(rows, max(64, 4 * ((rows * w.k + w.E - 1) // w.E)))
+    xp = synth.normal((n, w.H), 1.0, 6, "kb_xp", dev)
+    act = torch.empty((n, w.I), dtype=torch.bfloat16, device=dev)
+    y = torch.empty((n, w.H), dtype=torch.float32, device=dev)
+    t1 = timed(lambda: bd.grouped_gemm(xp, lw["w_gu"], lw["w_gu_shared"], counts, offsets, act, w.E, n, w.H, w.I,
+                                       bd.BF16, swiglu=1, extra_rows=rows, max_rows_hint=hint, ws=ws), reps, stream)
+    t2 = timed(lambda: bd.grouped_gemm(act, lw["w_down"], lw["w_down_shared"], counts, offsets, y, w.E, n, w.I, w.H,
+                                       bd.BF16, extra_rows=rows, max_rows_hint=hint, y_f32=1, ws=ws), reps, stream)
+    b1 = (active + 1) * 2 * w.I * w.H * 2 + n * w.H * 2 + n * w.I * 2
+    b2 = (active + 1) * w.H * w.I * 2 + n * w.I * 2 + n * w.H * 4
+    f1, f2 = 2.0 * n * 2 * w.I * w.H, 2.0 * n * w.H * w.I
+    return [_result("gemm_tc_kernel[experts_swiglu]", t1, b1, _flops({"active_experts": active, "rows": n}, f1, t1)),
+            _result("gemm_tc_kernel[experts_down]", t2, b2, _flops({"active_experts": active, "rows": n}, f2, t2))]
+
+
 def bench_unmask(w: Workload, reps, dev, stream):
     Bl = w.B // 2 if w.cfg else w.B
     n = Bl * w.L
@@ -189,6 +225,8 @@ def main():
         out.extend(bench_proj(w, a.reps, dev, stream))
     if a.kernel in ("experts", "route", "all"):
         out.extend(bench_experts(w, a.reps, dev, stream))
+    if a.kernel in ("experts", "expert_gemms", "all"):
+        out.extend(bench_expert_gemms(w, a.reps, dev, stream))
     if a.kernel in ("unmask", "all") and w.L <= 32:   # the prefill shape has no unmasking step
         out.append(bench_unmask(w, a.reps, dev, stream))
     if a.kernel in ("attn", "all"):

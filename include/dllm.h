@@ -92,6 +92,29 @@ DLLM_API int dllm_gemm(const dllm_gemm_desc* desc, const void* x, const void* w,
               void* ws, size_t ws_bytes, cudaStream_t stream);
 DLLM_API size_t dllm_gemm_workspace_size(const dllm_gemm_desc* desc);
 
+/*
+ * Grouped projection, the primitive of the routed experts (B4: [R] "MoE 백본과 Block-wise Attention", each token's
+ * chosen experts applied to it): rows [offsets[g], offsets[g] + counts[g]) of X form group g < G and are multiplied
+ * by the group's weight W[g] ([M', K], M' = 2M with swiglu: rows [0, M) gate, [M, 2M) up, else M' = M); with
+ * w_extra != NULL the last extra_rows rows of X form one more group with weight w_extra [M', K] (the shared
+ * expert). Y[r, :] = X[r] W_g^T, or with swiglu silu(X[r] W_gate^T) * (X[r] W_up^T) in fp32 rounded once to the
+ * storage type. X [rows, K]; Y [rows, M] in the storage type (fp32 when y_f32 != 0, not with swiglu); rows of X in
+ * no group are not written. counts, offsets: [G] int32 device arrays (groups may not overlap). max_rows_hint: the
+ * typical group size (chooses the tile width). bf16 only: K % 64 == 0, M % 128 == 0 (swiglu: M % 64 == 0).
+ */
+typedef struct {
+  int32_t G, rows, K, M;
+  int32_t swiglu;
+  int32_t extra_rows;
+  int32_t max_rows_hint;
+  int32_t dtype;
+  int32_t y_f32;
+} dllm_grouped_gemm_desc;
+DLLM_API int dllm_grouped_gemm(const dllm_grouped_gemm_desc* desc, const void* x, const void* w, const void* w_extra,
+                               const int32_t* counts, const int32_t* offsets, void* y, void* ws, size_t ws_bytes,
+                               cudaStream_t stream);
+DLLM_API size_t dllm_grouped_gemm_workspace_size(const dllm_grouped_gemm_desc* desc);
+
 /* ---------------------------------------------------------------------------------------------- B1 attention */
 /*
  * Block-causal attention ([R] "Block Diffusion Language Model (BDLM)", "MoE 백본과 Block-wise Attention"):
@@ -164,7 +187,10 @@ DLLM_API size_t dllm_moe_route_workspace_size(const dllm_route_desc* desc);
 
 /* ---------------------------------------------------------------------------------------------- B4 experts */
 /*
- * Routed experts plus shared expert, added to the residual:
+ * MoE FFN of the backbone ([R] "MoE 백본과 Block-wise Attention": each token's FFN is the mixture of the top-k
+ * experts the router picked, weighted by its gates; the shared expert, applied to every token, and the SwiGLU form
+ * of each expert are the stated layer configuration of this library's workloads). Routed experts plus shared
+ * expert, added to the residual:
  *   x[t] <- x[t] + shared(h[t]) + sum_j gates[t, j] * expert_{ids[t, j]}(h[t]),
  * expert_e(v) = W_down[e] (silu(W_gate[e] v) * (W_up[e] v)) (SwiGLU; the SwiGLU activation is stored in the
  * storage type), summed in slot order j = 0..k-1 in fp32 and rounded once.
@@ -194,8 +220,9 @@ DLLM_API size_t dllm_moe_experts_workspace_size(const dllm_expert_desc* desc);
  * lower position) get their
  * candidate written to tokens and their mask cleared; with cfg the uncond row b + B gets the same update.
  *   logits [n_rows * (1 + cfg), V] in the storage type; row_pos [>= n_rows] int32: the still-masked flat
- *   positions of the logical rows in increasing order (row r of the logits belongs to the r-th masked position);
- *   n_rows_dev [1] int32 (device count of masked positions, <= max_rows); tokens [B * (1 + cfg), L] int32; mask [B * (1 + cfg), L] uint8;
+ *   positions of the logical rows in increasing order (row r of the logits belongs to the r-th masked position;
+ *   every masked position must be listed, otherwise the results for the logical row are undefined);
+ *   n_rows_dev [1] int32 (device count of masked positions; a count above max_rows is read as max_rows); tokens [B * (1 + cfg), L] int32; mask [B * (1 + cfg), L] uint8;
  *   sel [B, L] int32 (chosen positions in rank order, -1 after nsel[b]); nsel [B]; conf [B, L] fp32 (0 at
  *   unmasked positions); remaining [1] int32: masked positions left over all logical rows.
  * Requires L <= 32 (one warp per block row for the selection) and B <= 1024.
@@ -304,6 +331,11 @@ typedef struct {
  *   output projection + residual, RMSNorm, router, routed + shared experts + residual] -> final RMSNorm ->
  *   LM head on the still-masked rows -> (CFG) -> confidence + unmasking.
  * B' = B / (1 + cfg) logical rows. Workspace from dllm_denoise_step_workspace_size with the same arguments.
+ * Early finish: a denoising pass over a block with no masked position left (threshold acceptance can finish a
+ * block before its last step) changes nothing: its first kernel finds no masked position, and every later kernel of
+ * the pass returns at entry (no weight or cache is read, no cache row written; sel is all -1, nsel 0, remaining 0),
+ * so the remaining passes of a finished block cost only their launches and need no host synchronisation. A commit
+ * pass always runs.
  */
 DLLM_API int dllm_denoise_step(const dllm_model* model, const dllm_state* state, const dllm_step_params* params, void* ws,
                       size_t ws_bytes, cudaStream_t stream);
@@ -317,6 +349,9 @@ typedef struct {
   const int32_t* row_pos;  /* [B' L] flat positions of the masked logical rows, ascending */
   const int32_t* n_rows;   /* [1] number of masked logical rows at the start of the pass */
   const void* x_final;     /* [B L, H] storage type: hidden state after the last layer (before the final norm) */
+  const int32_t* expert_counts; /* [n_layers, E + 1]: per layer, the assignments routed to each expert by the last
+                                   pass that ran that layer (entry E unused) */
+  const int32_t* live;     /* [1]: 1 if the last denoising pass found a masked position (and ran), else 0 */
 } dllm_step_views;
 DLLM_API int dllm_denoise_step_views(const dllm_model* model, const dllm_state* state, const dllm_step_params* params,
                             void* ws, size_t ws_bytes, dllm_step_views* views /* host */);

@@ -94,16 +94,31 @@ def test_route_and_experts_reject_bad_arguments(lib):
     assert lib.dllm_moe_experts(C.byref(e), *([FAKE] * 11), FAKE, 1 << 30, None) == bd.ERR_UNSUPPORTED
 
 
+def test_grouped_gemm_rejects_bad_arguments(lib):
+    d = bd.GroupedGemmDesc(8, 64, 256, 128, 0, 0, 0, bd.BF16, 0)
+    args = [FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, 1 << 20, None]
+    d.K = 100
+    assert lib.dllm_grouped_gemm(C.byref(d), *args) == bd.ERR_UNSUPPORTED
+    d.K, d.extra_rows = 256, 8          # an extra group without its weight
+    assert lib.dllm_grouped_gemm(C.byref(d), *args) == bd.ERR_INVALID_ARG
+    d.extra_rows, d.swiglu, d.y_f32 = 0, 1, 1
+    assert lib.dllm_grouped_gemm(C.byref(d), *args) == bd.ERR_UNSUPPORTED
+    d.swiglu, d.y_f32, d.dtype = 0, 0, bd.F32
+    assert lib.dllm_grouped_gemm(C.byref(d), *args) == bd.ERR_UNSUPPORTED
+
+
 def test_route_workspace_covers_scores_and_permutation_segments(lib):
-    """The router's workspace holds the fp32 scores and, past 32 tokens, one expert histogram per permutation
-    segment (segments of a multiple of 256 assignments, about 128 of them at most)."""
+    """The router's workspace holds the fp32 scores, one expert histogram per permutation segment (segments of
+    whole tokens, a multiple of 256 assignments, at most 128 of them) and one near-tie threshold per token."""
+    import math
     lib.dllm_moe_route_workspace_size.restype = C.c_size_t
-    for Tk, E, k in [(32, 256, 8), (512, 256, 8), (32768, 256, 8), (1001, 1000, 3), (5000, 96, 4)]:
-        n = Tk * k
-        seg = max(256, ((n + 127) // 128 + 255) // 256 * 256)
-        segments = (n + seg - 1) // seg
-        assert segments <= 129
-        need = Tk * E * 4 + segments * E * 4
+    for Tk, E, k in [(32, 256, 8), (512, 256, 8), (32768, 256, 8), (1001, 1000, 3), (5000, 96, 4), (77, 256, 6)]:
+        unit = 256 // math.gcd(k, 256)
+        seg_tok = max(unit, -(-(-(-Tk // 128)) // unit) * unit)
+        assert (seg_tok * k) % 256 == 0
+        segments = -(-Tk // seg_tok)
+        assert segments <= 128
+        need = Tk * E * 4 + segments * E * 4 + Tk * 4
         r = bd.RouteDesc(Tk, 2048, E, k, bd.BF16)
         assert lib.dllm_moe_route_workspace_size(C.byref(r)) >= need
 

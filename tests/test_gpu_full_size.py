@@ -18,7 +18,7 @@ from block_diffusion_moe_dllm_b200 import synth
 from block_diffusion_moe_dllm_b200.configs import PREFILL, T2I, THINKING, UNDERSTANDING
 from block_diffusion_moe_dllm_b200.engine import DenoiseEngine
 from oracle import dllm_oracle as O
-from _util import ROUTE_TIE, assert_close, assignment_tables, random_assignments, same_selection, to64
+from _util import ROUTE_TIE, assert_close, assignment_tables, check_unmask, random_assignments, same_routing, to64
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -95,10 +95,10 @@ def test_full_router_understanding():
     inv = torch.empty(Tk * k, dtype=torch.int32, device=DEV)
     bd.moe_route(h, wr, bias, ids, gates, counts, offsets, perm, inv, Tk, H, E, k, bd.BF16)
     torch.cuda.synchronize()
-    o_ids, o_gates, _, margin = O.route(to64(h), to64(wr), to64(bias), k)
+    o_ids, o_gates, _, margin = O.route(to64(h), to64(wr), to64(bias), k, order=True)
     ok = margin >= ROUTE_TIE
-    assert ok.mean() > 0.9
-    same_selection(ids.cpu().numpy(), gates.cpu().numpy(), o_ids, o_gates, ok, rtol=5e-6, atol=5e-7)
+    assert ok.mean() > 0.99
+    same_routing(ids.cpu().numpy(), gates.cpu().numpy(), o_ids, o_gates, ok, rtol=5e-6, atol=5e-7)
     c, off, p, iv = assignment_tables(ids.cpu().numpy(), E)
     assert np.array_equal(perm.cpu().numpy(), p) and np.array_equal(inv.cpu().numpy(), iv)
 
@@ -118,10 +118,13 @@ def test_full_router_prefill():
     inv = torch.empty(Tk * k, dtype=torch.int32, device=DEV)
     bd.moe_route(h, wr, bias, ids, gates, counts, offsets, perm, inv, Tk, H, E, k, bd.BF16)
     torch.cuda.synchronize()
-    o_ids, o_gates, _, margin = O.route(to64(h), to64(wr), to64(bias), k)
+    o_ids, o_gates, _, margin = O.route(to64(h), to64(wr), to64(bias), k, order=True)
     ok = margin >= ROUTE_TIE
-    assert ok.mean() > 0.9
-    same_selection(ids.cpu().numpy(), gates.cpu().numpy(), o_ids, o_gates, ok, rtol=5e-6, atol=5e-7)
+    assert ok.mean() > 0.99
+    # thousands of tokens have a neighbour gap between the band and a few times the fp32 score error: the case
+    # the exact re-decision exists for
+    assert np.sum((margin >= ROUTE_TIE) & (margin < 1e-5)) > 100
+    same_routing(ids.cpu().numpy(), gates.cpu().numpy(), o_ids, o_gates, ok, rtol=5e-6, atol=5e-7)
     c, off, p, iv = assignment_tables(ids.cpu().numpy(), E)
     assert np.array_equal(counts.cpu().numpy(), c) and np.array_equal(offsets.cpu().numpy(), off)
     assert np.array_equal(perm.cpu().numpy(), p) and np.array_equal(inv.cpu().numpy(), iv)
@@ -187,13 +190,8 @@ def test_full_unmask(w):
     zl = to64(logits)
     u = O.unmask(zl[:n], row_pos, tokens, mask, 0, w.T_s, w.mode, float(np.float32(w.tau)), w.k_max,
                  w.vocab_offset, z_uncond=zl[n:] if w.cfg else None, cfg_scale=float(np.float32(w.cfg_scale)))
-    g_conf = conf.cpu().numpy().astype(np.float64)
-    assert np.all(np.abs(g_conf - u["conf"]) <= 1e-6 * np.maximum(u["conf"], 1e-30) + 1e-12)
-    for b in range(Bl):
-        if u["tie_rank"][b] or u["tie_tau"][b]:
-            continue
-        assert nsel[b].item() == u["nsel"][b]
-        assert np.array_equal(dt.cpu().numpy()[b], u["tokens"][b]) and np.array_equal(dm.cpu().numpy()[b], u["mask"][b])
+    check_unmask(u, conf.cpu().numpy(), nsel.cpu().numpy(), sel.cpu().numpy(), dt.cpu().numpy(), dm.cpu().numpy(),
+                 Bl, w.cfg)
 
 
 # ------------------------------------------------------------------------------------------------ whole pass

@@ -113,7 +113,7 @@ def _check_candidates(w, eng, u_or, f, flag):
     n = len(f["row_pos"])
     z = f["logits"][:n]
     if w.cfg:
-        z = O.cfg_combine_f32(z, f["logits"][n:], w.cfg_scale)
+        z = O.cfg_combine(z, f["logits"][n:], w.cfg_scale)
     top2 = np.sort(z, axis=1)[:, -2:]
     clear = (top2[:, 1] - top2[:, 0]) > 0.05
     g_tok = eng.tokens.cpu().numpy()
@@ -297,3 +297,62 @@ def test_commit_pass(w):
         # routing near-ties in this layer can change the next layer's input: mark those tokens
         if f["route"][l] is not None:
             flag |= f["route"][l][2] < _route_margin(w.dtype)
+
+
+# ------------------------------------------------------------------------------------------------ early finish
+def _snapshot(eng, caches):
+    return (eng.tokens.clone(), eng.mask.clone(), [(k.clone(), v.clone()) for k, v in caches])
+
+
+def test_block_finished_early_later_passes_do_nothing():
+    """Threshold mode with tau = 0 and k_max >= L accepts every position at the first pass ([R] "SPRINT":
+    accept every c > tau). The block is then finished: the remaining passes of the block launch, see no masked
+    position and change nothing (tokens, mask, every layer's K/V cache); the commit pass still runs."""
+    w = scaled(SMALL, name="small-bf16-early", mode=1, tau=0.0, k_max=32, T_s=6)
+    wt, caches, eng, tok0, mask0 = _setup(w, seed=41)
+    hw, hc = _host(wt), _host_caches(caches, w.P)
+    eng.step(0)
+    torch.cuda.synchronize()
+    assert bd.status_check(eng.ws) == bd.OK
+    u = O.denoise_step(w, hw, hc, tok0, mask0, 0)
+    assert int(eng.remaining.item()) == 0 and int(eng.mask.sum().item()) == 0
+    assert np.array_equal(eng.nsel.cpu().numpy(), u["nsel"]) and np.all(u["nsel"] == w.L)
+    snap = _snapshot(eng, caches)
+    for t in range(1, w.T_s):
+        eng.step(t)
+    torch.cuda.synchronize()
+    assert bd.status_check(eng.ws) == bd.OK
+    assert torch.equal(eng.tokens, snap[0]) and torch.equal(eng.mask, snap[1])
+    for (k, v), (k0, v0) in zip(caches, snap[2]):
+        assert torch.equal(k, k0) and torch.equal(v, v0), "a finished block's pass wrote the cache"
+    assert int(eng.remaining.item()) == 0 and int(eng.nsel.sum().item()) == 0
+    eng.commit()
+    torch.cuda.synchronize()
+    assert bd.status_check(eng.ws) == bd.OK
+    assert not torch.equal(caches[0][0][:, :, w.P: w.P + w.L], snap[2][0][0][:, :, w.P: w.P + w.L])
+
+
+def test_finished_pass_costs_only_its_launches():
+    """At the one-layer workload's full size a pass over a finished block (every kernel returns at entry) takes
+    a fraction of a live pass (which streams about 1 GB of weights)."""
+    w = ONE_LAYER
+    wt, caches, eng, _, _ = _setup(w, seed=3, random_gains=False)
+    tokens, mask = synth.make_block_state(w, DEV, seed=3)
+    done = torch.zeros_like(mask)
+
+    def timed(m):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        ts = []
+        for _ in range(6):
+            eng.set_block(tokens, m)
+            torch.cuda.synchronize()
+            ev[0].record()
+            eng.step(1)
+            ev[1].record()
+            torch.cuda.synchronize()
+            ts.append(ev[0].elapsed_time(ev[1]))
+        return sorted(ts[1:])[2]
+
+    live, dead = timed(mask), timed(done)
+    assert bd.status_check(eng.ws) == bd.OK
+    assert dead < 0.5 * live, f"finished pass {dead * 1e3:.0f} us vs live pass {live * 1e3:.0f} us"

@@ -77,6 +77,28 @@ def f64(a):
 
 
 # --------------------------------------------------------------------------------------------------------------
+# FP8 weights (the FP8 checkpoint of the card news "FP8 추론" and the HF-mirror README's FP8 version: format not
+# given on the pages; read as OCP FP8 E4M3 codes with one fp32 scale per output row)
+
+
+def e4m3_value(q):
+    """Value of FP8 E4M3 codes (OCP 8-bit float, the variant without infinities): sign bit, 4 exponent bits with
+    bias 7, 3 mantissa bits; (-1)^s 2^(e-7) (1 + m/8) for e > 0, (-1)^s 2^-6 (m/8) for e = 0 (subnormals); the codes
+    with e = 15 and m = 7 are NaN. Returned in fp64 (exact)."""
+    q = np.asarray(q).astype(np.int64) & 0xFF
+    sgn, e, m = q >> 7, (q >> 3) & 0xF, q & 7
+    v = np.where(e == 0, (m / 8.0) * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2((e - 7).astype(np.float64)))
+    v = np.where((e == 15) & (m == 7), np.nan, v)
+    return np.where(sgn == 1, -v, v)
+
+
+def dequant_rows(q, scale):
+    """Weights of an FP8 matrix [..., M, K] with one scale per output row [..., M]: W[m, k] = value(q[m, k]) *
+    scale[m], exact in fp64."""
+    return e4m3_value(q) * f64(scale)[..., None]
+
+
+# --------------------------------------------------------------------------------------------------------------
 # per-layer building blocks
 
 

@@ -521,3 +521,32 @@ def test_denoise_block_end_to_end_tiny():
     assert mask.sum() == 0 and np.all(tokens < w.V)
     bk, bv = O.commit_block(w, wt, caches, tokens)
     assert len(bk) == w.n_layers and bk[0].shape == (w.B, w.L, w.Hkv, w.d)
+
+
+# ---------------------------------------------------------------------------------------------- FP8 weights
+
+def test_e4m3_values_match_torch_conversion_for_every_code():
+    """All 256 E4M3 codes decode to torch's float8_e4m3fn values (the same OCP format), NaN codes included."""
+    codes = np.arange(256, dtype=np.uint8)
+    want = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = O.e4m3_value(codes)
+    assert np.array_equal(np.isnan(got), np.isnan(want))
+    ok = ~np.isnan(want)
+    assert np.array_equal(got[ok], want[ok])
+
+
+def test_e4m3_closed_forms():
+    v = O.e4m3_value(np.array([0x00, 0x80, 0x38, 0xB8, 0x7E, 0x01, 0x08, 0x3C, 0x7F]))
+    assert v[0] == 0.0 and v[1] == 0.0 and np.signbit(v[1])
+    assert v[2] == 1.0 and v[3] == -1.0            # exponent 7 = bias, mantissa 0
+    assert v[4] == 448.0                           # largest finite: 2^8 * 1.75
+    assert v[5] == 2.0 ** -9                       # smallest subnormal: 2^-6 * 1/8
+    assert v[6] == 2.0 ** -6                       # smallest normal
+    assert v[7] == 1.5
+    assert np.isnan(v[8])
+
+
+def test_dequant_rows_scales_each_output_row():
+    q = np.array([[0x38, 0xB8], [0x40, 0x30]], dtype=np.uint8)      # [[1, -1], [2, 0.5]]
+    w = O.dequant_rows(q, np.array([0.5, 3.0], dtype=np.float32))
+    assert np.array_equal(w, [[0.5, -0.5], [6.0, 1.5]])

@@ -6,12 +6,12 @@ Default workload: understanding (20 layers, batch 16, hidden 2048, 16 q heads x 
 + shared, inter 512, vocab 157184, prefix 2688, block 32, 32 steps per block, threshold acceptance tau 0.9 with at
 most 8 tokens per step), the largest configuration that fits one GPU.
 
-One bench step decodes one block: the block state is reset from a device copy, then its T_s denoising passes
-(embedding, attention over the cached prefix, MoE FFN, LM head over the still-masked rows, confidence +
-unmasking) and the commit pass that writes the block's clean K/V into the cache, replayed as one CUDA graph.
-Threshold acceptance can finish a block before its last step; the passes after that find no masked position and
-return at entry (they cost their launches only). Metric: denoise-step tokens/s = B * L tokens for every pass that
-found a masked position, per second. Also reported: committed tokens/s (the block's B' * L tokens per block
+One bench step decodes one block: the block state is reset from a device copy, then the library's block graph
+(dllm_block_graph_create) runs its T_s denoising passes (embedding, attention over the cached prefix, MoE FFN, LM
+head over the still-masked rows, confidence + unmasking) and the commit pass that writes the block's clean K/V
+into the cache. Threshold acceptance can finish a block before its last step; each pass sits in a conditional
+node that runs it only while masked positions are left. Metric: denoise-step tokens/s = B * L tokens for every pass
+that ran, per second. Also reported: committed tokens/s (the block's B' * L tokens per block
 time), the live passes per block, the experts each layer routed to, and the step's algorithmic bytes against HBM.
 
 Timing: K steps between CUDA events after W warm-up steps, repeated until the timed units cover at least 2 s; the
@@ -282,15 +282,28 @@ def main():
     eng = DenoiseEngine(w, wt, caches, dev)
     stream = torch.cuda.current_stream()
 
-    # the whole block (state reset + T_s passes + commit) as one CUDA graph; the library's launches per block are
-    # counted while it is captured (two warm-up blocks + the captured one)
+    # the whole block as the library's block graph: the T_s passes, each inside a conditional node that runs it only
+    # while the block has masked positions, and the commit pass; every step resets the block state from a device
+    # copy first. Kernels per pass are counted on host-driven calls.
+    eng.set_block(tokens0, mask0)
+    eng.decode_block()                      # warms the library's one-time set-up outside capture
+    torch.cuda.synchronize()
     n0 = bd.launch_count()
-    g_reset = eng.capture_block(tokens0, mask0)
-    launches_per_step = (bd.launch_count() - n0) // 3
-    g_plain = eng.capture_block()                           # the same without the device-side reset (e2e arm)
+    eng.set_block(tokens0, mask0)
+    eng.step(0)
+    per_pass = bd.launch_count() - n0
+    n0 = bd.launch_count()
+    eng.commit()
+    per_commit = bd.launch_count() - n0
+    graph = eng.block_graph()
+
+    def block():
+        eng.tokens.copy_(tokens0)
+        eng.mask.copy_(mask0)
+        graph.launch(stream)
 
     for _ in range(args.warmup):
-        g_reset.replay()
+        block()
     torch.cuda.synchronize()
     assert bd.status_check(eng.ws) == bd.OK
 
@@ -305,7 +318,7 @@ def main():
         ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         ev0.record(stream)
         for _ in range(args.steps):
-            g_reset.replay()
+            block()
         ev1.record(stream)
         torch.cuda.synchronize()
         units.append(replicas.max_over_ranks(ev0.elapsed_time(ev1) / 1000.0, dev))
@@ -337,7 +350,7 @@ def main():
     h_mask = mask0.cpu().pin_memory()
     h_out = torch.empty_like(h_tok).pin_memory()
 
-    def e2e_run(graph):
+    def e2e_run(use_graph):
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
@@ -346,8 +359,8 @@ def main():
         for _ in range(args.steps):
             eng.tokens.copy_(h_tok, non_blocking=True)
             eng.mask.copy_(h_mask, non_blocking=True)
-            if graph:
-                g_plain.replay()
+            if use_graph:
+                graph.launch(stream)
             else:
                 eng.decode_block(stream)
             h_out.copy_(eng.tokens, non_blocking=True)
@@ -360,9 +373,9 @@ def main():
     e2e = {"value": e2e_run(False), "unit": "tokens/s", **io,
            "path": "dllm_denoise_step called from the host for every pass and the commit pass"}
     e2e_graph = {"value": e2e_run(True), "unit": "tokens/s", **io,
-                 "path": "the same calls replayed as one CUDA graph per block"}
+                 "path": "dllm_block_graph_launch per block (passes after the block finished are skipped)"}
     assert bd.status_check(eng.ws) == bd.OK
-    del g_reset, g_plain
+    del graph
 
     # ---- dominant kernel, timed alone with CUDA events at this workload's shapes
     roof, kernels = kernel_rooflines(w, wt, dev, stream)
@@ -371,8 +384,8 @@ def main():
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": 1000.0 * step_s, "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                "step": "one block: state reset, T_s denoising passes (those after the block finished return at "
-                        "entry) and the commit pass, replayed as one CUDA graph",
+                "step": "one block: state reset, then the library's block graph: T_s denoising passes, each in a "
+                        "conditional node that runs it only while masked positions are left, and the commit pass",
                 "config": bench_config(w, world),
                 "timed_units": {"n": len(units), "unit_s": units, "steps_per_unit": args.steps},
                 "committed_tokens_per_s": committed,
@@ -380,7 +393,7 @@ def main():
                                      "rows_per_live_pass": [p["rows"] for p in passes if p["live"]]},
                 "active_experts_per_layer": {"mean": statistics.mean(act) if act else 0,
                                              "min": min(act) if act else 0, "max": max(act) if act else 0},
-                "gpu_launches": launches_per_step * args.steps * len(units), "clocks": clk,
+                "gpu_launches": (live * per_pass + per_commit) * args.steps * len(units), "clocks": clk,
                 "e2e": e2e, "e2e_graph": e2e_graph, "roofline": roof, "step_roofline": step_roof,
                 "kernels": kernels}
         if not args.no_cpu_baseline and world == 1:

@@ -13,6 +13,7 @@ LIB_PATH = os.path.join(PKG, "libdllm.so")
 OK, ERR_INVALID_ARG, ERR_SHAPE, ERR_ALIGN, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = range(8)
 BF16, F32 = 0, 1
 FIXED, THRESHOLD = 0, 1
+WEIGHTS_BF16, WEIGHTS_FP8 = 0, 1
 
 STATUS_NAMES = {0: "DLLM_OK", 1: "DLLM_ERR_INVALID_ARG", 2: "DLLM_ERR_SHAPE", 3: "DLLM_ERR_ALIGN",
                 4: "DLLM_ERR_UNSUPPORTED", 5: "DLLM_ERR_WORKSPACE", 6: "DLLM_ERR_CUDA", 7: "DLLM_ERR_TIMEOUT"}
@@ -21,12 +22,13 @@ i32, f32, vp, sz = C.c_int32, C.c_float, C.c_void_p, C.c_size_t
 
 
 class GemmDesc(C.Structure):
-    _fields_ = [("N", i32), ("M", i32), ("K", i32), ("ldy", i32), ("dtype", i32), ("y_f32", i32), ("residual", i32)]
+    _fields_ = [("N", i32), ("M", i32), ("K", i32), ("ldy", i32), ("dtype", i32), ("y_f32", i32), ("residual", i32),
+                ("w_fp8", i32)]
 
 
 class GroupedGemmDesc(C.Structure):
     _fields_ = [("G", i32), ("rows", i32), ("K", i32), ("M", i32), ("swiglu", i32), ("extra_rows", i32),
-                ("max_rows_hint", i32), ("dtype", i32), ("y_f32", i32)]
+                ("max_rows_hint", i32), ("dtype", i32), ("y_f32", i32), ("w_fp8", i32)]
 
 
 class AttnDesc(C.Structure):
@@ -44,7 +46,7 @@ class RouteDesc(C.Structure):
 
 
 class ExpertDesc(C.Structure):
-    _fields_ = [("Tk", i32), ("H", i32), ("E", i32), ("k", i32), ("I", i32), ("dtype", i32)]
+    _fields_ = [("Tk", i32), ("H", i32), ("E", i32), ("k", i32), ("I", i32), ("dtype", i32), ("w_fp8", i32)]
 
 
 class UnmaskDesc(C.Structure):
@@ -56,13 +58,15 @@ class UnmaskDesc(C.Structure):
 class Layer(C.Structure):
     _fields_ = [("attn_norm", vp), ("w_qkv", vp), ("w_o", vp), ("ffn_norm", vp), ("w_router", vp),
                 ("router_bias", vp), ("w_gu", vp), ("w_down", vp), ("w_gu_shared", vp), ("w_down_shared", vp),
-                ("k_cache", vp), ("v_cache", vp), ("k_thin", vp), ("v_thin", vp), ("keep_pos", vp)]
+                ("k_cache", vp), ("v_cache", vp), ("k_thin", vp), ("v_thin", vp), ("keep_pos", vp),
+                ("w_gu_scale", vp), ("w_down_scale", vp), ("w_gu_shared_scale", vp), ("w_down_shared_scale", vp)]
 
 
 class Model(C.Structure):
     _fields_ = [("n_layers", i32), ("H", i32), ("Hq", i32), ("Hkv", i32), ("d", i32), ("E", i32), ("k", i32),
                 ("I", i32), ("V", i32), ("dtype", i32), ("eps", f32), ("rope_base", f32), ("mask_id", i32),
-                ("embed", vp), ("final_norm", vp), ("w_lm", vp), ("layers", C.POINTER(Layer))]
+                ("embed", vp), ("final_norm", vp), ("w_lm", vp), ("layers", C.POINTER(Layer)),
+                ("weight_format", i32), ("w_lm_scale", vp)]
 
 
 class State(C.Structure):
@@ -86,9 +90,9 @@ _SIGS = {
     "dllm_status_check": ([vp, vp], C.c_int),
     "dllm_launch_count": ([], C.c_ulonglong),
     "dllm_selftest_bounded_wait": ([vp, sz, vp], C.c_int),
-    "dllm_gemm": ([C.POINTER(GemmDesc), vp, vp, vp, vp, vp, sz, vp], C.c_int),
+    "dllm_gemm": ([C.POINTER(GemmDesc), vp, vp, vp, vp, vp, vp, sz, vp], C.c_int),
     "dllm_gemm_workspace_size": ([C.POINTER(GemmDesc)], sz),
-    "dllm_grouped_gemm": ([C.POINTER(GroupedGemmDesc), vp, vp, vp, vp, vp, vp, vp, sz, vp], C.c_int),
+    "dllm_grouped_gemm": ([C.POINTER(GroupedGemmDesc), vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], C.c_int),
     "dllm_grouped_gemm_workspace_size": ([C.POINTER(GroupedGemmDesc)], sz),
     "dllm_block_attn": ([C.POINTER(AttnDesc), vp, vp, vp, vp, vp, vp, sz, vp], C.c_int),
     "dllm_block_attn_workspace_size": ([C.POINTER(AttnDesc)], sz),
@@ -96,7 +100,7 @@ _SIGS = {
     "dllm_prefix_retain_workspace_size": ([C.POINTER(RetainDesc)], sz),
     "dllm_moe_route": ([C.POINTER(RouteDesc), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], C.c_int),
     "dllm_moe_route_workspace_size": ([C.POINTER(RouteDesc)], sz),
-    "dllm_moe_experts": ([C.POINTER(ExpertDesc), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], C.c_int),
+    "dllm_moe_experts": ([C.POINTER(ExpertDesc)] + [vp] * 16 + [sz, vp], C.c_int),
     "dllm_moe_experts_workspace_size": ([C.POINTER(ExpertDesc)], sz),
     "dllm_unmask": ([C.POINTER(UnmaskDesc), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], C.c_int),
     "dllm_unmask_workspace_size": ([C.POINTER(UnmaskDesc)], sz),
@@ -105,6 +109,10 @@ _SIGS = {
     "dllm_denoise_step_workspace_size": ([C.POINTER(Model), C.POINTER(State), C.POINTER(StepParams)], sz),
     "dllm_denoise_step_views": ([C.POINTER(Model), C.POINTER(State), C.POINTER(StepParams), vp, sz,
                                  C.POINTER(StepViews)], C.c_int),
+    "dllm_block_graph_create": ([C.POINTER(Model), C.POINTER(State), C.POINTER(StepParams), vp, sz, vp,
+                                 C.POINTER(vp)], C.c_int),
+    "dllm_block_graph_launch": ([vp, vp], C.c_int),
+    "dllm_block_graph_destroy": ([vp], None),
 }
 
 EXPORTED = sorted(_SIGS)
@@ -170,23 +178,26 @@ class Workspace:
 
 # ---------------------------------------------------------------------------------------------- call wrappers
 
-def gemm(x, w, y, N, M, K, dtype, ldy=None, y_f32=0, residual=0, n_rows_dev=None, ws=None, stream=None):
+def gemm(x, w, y, N, M, K, dtype, ldy=None, y_f32=0, residual=0, n_rows_dev=None, w_scale=None, ws=None,
+         stream=None):
+    """Dense projection; with w_scale given, w holds E4M3 codes (uint8) with one fp32 scale per row."""
     lib = load()
-    d = GemmDesc(N, M, K, ldy or M, dtype, y_f32, residual)
+    d = GemmDesc(N, M, K, ldy or M, dtype, y_f32, residual, int(w_scale is not None))
     need = lib.dllm_gemm_workspace_size(C.byref(d))
     ws = (ws or Workspace(need, x.device)).ensure(need)
-    return check(lib.dllm_gemm(C.byref(d), ptr(x), ptr(w), ptr(y), ptr(n_rows_dev), ws.addr, ws.nbytes,
+    return check(lib.dllm_gemm(C.byref(d), ptr(x), ptr(w), ptr(w_scale), ptr(y), ptr(n_rows_dev), ws.addr, ws.nbytes,
                                stream_handle(stream)))
 
 
 def grouped_gemm(x, w, w_extra, counts, offsets, y, G, rows, K, M, dtype, swiglu=0, extra_rows=0, max_rows_hint=0,
-                 y_f32=0, ws=None, stream=None):
+                 y_f32=0, w_scale=None, w_extra_scale=None, ws=None, stream=None):
+    """Grouped projection; with w_scale given, w (and w_extra) hold E4M3 codes with per-row fp32 scales."""
     lib = load()
-    d = GroupedGemmDesc(G, rows, K, M, swiglu, extra_rows, max_rows_hint, dtype, y_f32)
+    d = GroupedGemmDesc(G, rows, K, M, swiglu, extra_rows, max_rows_hint, dtype, y_f32, int(w_scale is not None))
     need = lib.dllm_grouped_gemm_workspace_size(C.byref(d))
     ws = (ws or Workspace(need, x.device)).ensure(need)
-    return check(lib.dllm_grouped_gemm(C.byref(d), ptr(x), ptr(w), ptr(w_extra), ptr(counts), ptr(offsets), ptr(y),
-                                       ws.addr, ws.nbytes, stream_handle(stream)))
+    return check(lib.dllm_grouped_gemm(C.byref(d), ptr(x), ptr(w), ptr(w_extra), ptr(w_scale), ptr(w_extra_scale),
+                                       ptr(counts), ptr(offsets), ptr(y), ws.addr, ws.nbytes, stream_handle(stream)))
 
 
 def block_attn(q, k_cache, v_cache, out, B, Lq, Hq, Hkv, d, blk_len, q_pos0, n_keys, cap, dtype, key_pos=None,
@@ -221,14 +232,16 @@ def moe_route(h, w_router, bias, ids, gates, counts, offsets, perm, inv, Tk, H, 
 
 
 def moe_experts(h, w_gu, w_down, w_gu_shared, w_down_shared, counts, offsets, perm, inv, gates, x_inout, Tk, H, E,
-                k, I, dtype, ws=None, stream=None):
+                k, I, dtype, scales=None, ws=None, stream=None):
+    """Routed + shared experts; scales = (gu, down, gu_shared, down_shared) row scales when the weights are E4M3."""
     lib = load()
-    desc = ExpertDesc(Tk, H, E, k, I, dtype)
+    desc = ExpertDesc(Tk, H, E, k, I, dtype, int(scales is not None))
+    sc = scales or (None, None, None, None)
     need = lib.dllm_moe_experts_workspace_size(C.byref(desc))
     ws = (ws or Workspace(need, h.device)).ensure(need)
     return check(lib.dllm_moe_experts(C.byref(desc), ptr(h), ptr(w_gu), ptr(w_down), ptr(w_gu_shared),
-                                      ptr(w_down_shared), ptr(counts), ptr(offsets), ptr(perm), ptr(inv), ptr(gates),
-                                      ptr(x_inout), ws.addr, ws.nbytes, stream_handle(stream)))
+                                      ptr(w_down_shared), *[ptr(t) for t in sc], ptr(counts), ptr(offsets), ptr(perm),
+                                      ptr(inv), ptr(gates), ptr(x_inout), ws.addr, ws.nbytes, stream_handle(stream)))
 
 
 def unmask(logits, row_pos, n_rows_dev, tokens, mask, sel, nsel, conf, remaining, B, L, V, max_rows, t, T_s,

@@ -42,6 +42,7 @@ class Workload:
     lm_std: float = 0.02
     bias_range: float = 0.1
     seed: int = 0
+    wfmt: str = "bf16"    # "fp8": expert and LM-head weights as E4M3 codes with per-row fp32 scales
 
     @property
     def Tk(self) -> int:
@@ -92,7 +93,11 @@ UNDERSTANDING = Workload("understanding-20layer-b16-p2688-thr0.9", "bf16", 20, 2
 # compute-bound prefill of the thinking-mode prompt: 1 layer, 8 rows x 4096 tokens under the block-causal mask
 PREFILL = Workload("prefill-1layer-b8-4096", "bf16", 1, 2048, 16, 4, 128, 256, 8, 512, 157184, 8, 0, 4096, 1)
 
-ALL = [TINY_F32, ONE_LAYER, T2I, THINKING, UNDERSTANDING, PREFILL]
+# the same two workloads with the FP8 checkpoint's expert and LM-head weights (E4M3 codes, per-row scales)
+ONE_LAYER_FP8 = replace(ONE_LAYER, name="moe-dllm-1layer-p1024-b1-fp8", wfmt="fp8")
+UNDERSTANDING_FP8 = replace(UNDERSTANDING, name="understanding-20layer-b16-p2688-thr0.9-fp8", wfmt="fp8")
+
+ALL = [TINY_F32, ONE_LAYER, T2I, THINKING, UNDERSTANDING, PREFILL, ONE_LAYER_FP8, UNDERSTANDING_FP8]
 BY_NAME = {w.name: w for w in ALL}
 
 

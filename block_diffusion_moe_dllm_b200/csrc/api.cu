@@ -101,10 +101,20 @@ struct PostNorm {
   const int32_t* n_dev = nullptr;
 };
 
+// Row scales of FP8 expert weights (all NULL for weights in the storage type).
+struct ExpertScales {
+  const float* gu = nullptr;
+  const float* down = nullptr;
+  const float* gu_shared = nullptr;
+  const float* down_shared = nullptr;
+};
+
 int run_experts(int dtype, int Tk, int H, int E, int k, int I, const void* h, const void* w_gu, const void* w_down,
                 const void* w_gu_s, const void* w_down_s, const int32_t* counts, const int32_t* offsets,
                 const int32_t* perm, const int32_t* inv, const float* gates, void* x, const ExpertBufs& b,
-                int32_t* status, cudaStream_t s, const PostNorm& pn = PostNorm(), const int32_t* live = nullptr) {
+                int32_t* status, cudaStream_t s, const PostNorm& pn = PostNorm(), const int32_t* live = nullptr,
+                const ExpertScales& sc = ExpertScales()) {
+  const int fp8 = sc.gu != nullptr;
   const int shared = w_gu_s != nullptr;
   const int n_assign = Tk * k;
   const int64_t rows = (int64_t)n_assign + (shared ? Tk : 0);
@@ -119,12 +129,14 @@ int run_experts(int dtype, int Tk, int H, int E, int k, int I, const void* h, co
   g1.has_extra = shared; g1.extra_off = n_assign; g1.extra_cnt = Tk;
   g1.max_cnt = expert_bn_hint(Tk, k, E); g1.cnt_bound = Tk;
   g1.dtype = dtype; g1.status = status; g1.f32_scratch = b.scratch; g1.live = live;
+  g1.w_fp8 = fp8; g1.w_scale = sc.gu; g1.w2_scale = sc.gu_shared;
   g1.epi.kind = EPI_SWIGLU; g1.epi.out = b.act; g1.epi.ldo = I;
   st = run_gemm(g1, s);
   if (st) return st;
   GemmArgs g2 = g1;
   g2.x = b.act; g2.K = I; g2.M = H; g2.swiglu = 0;
   g2.w = w_down; g2.w_rows = (int64_t)E * H; g2.w2 = w_down_s; g2.w2_rows = H; g2.w_group_stride = H;
+  g2.w_scale = sc.down; g2.w2_scale = sc.down_shared;
   g2.epi = EpiParams();
   g2.epi.kind = EPI_STORE; g2.epi.out = b.y; g2.epi.ldo = H; g2.epi.out_f32 = 1;
   st = run_gemm(g2, s);
@@ -209,6 +221,17 @@ int validate_step(const dllm_model* m, const dllm_state* st, const dllm_step_par
       REQ(aligned16(L.w_qkv) && aligned16(L.w_o) && aligned16(L.w_gu) && aligned16(L.w_down), DLLM_ERR_ALIGN,
           "layer %d: weights must be 16-byte aligned", l);
   }
+  REQ(m->weight_format == DLLM_WEIGHTS_BF16 || m->weight_format == DLLM_WEIGHTS_FP8, DLLM_ERR_INVALID_ARG,
+      "denoise_step: bad weight_format %d", m->weight_format);
+  if (m->weight_format == DLLM_WEIGHTS_FP8) {
+    REQ(m->dtype == DLLM_BF16, DLLM_ERR_UNSUPPORTED, "denoise_step: FP8 weights need bf16 storage");
+    REQ(m->w_lm_scale, DLLM_ERR_INVALID_ARG, "denoise_step: FP8 weights need w_lm_scale");
+    for (int l = 0; l < m->n_layers; ++l) {
+      const dllm_layer& L = m->layers[l];
+      REQ(L.w_gu_scale && L.w_down_scale && (!L.w_gu_shared || (L.w_gu_shared_scale && L.w_down_shared_scale)),
+          DLLM_ERR_INVALID_ARG, "denoise_step: layer %d: FP8 expert weights need their row scales", l);
+    }
+  }
   if (m->dtype == DLLM_BF16) {
     REQ(m->d == 128, DLLM_ERR_UNSUPPORTED, "denoise_step: bf16 path needs head dim 128");
     REQ(m->H % 128 == 0 && m->I % 64 == 0, DLLM_ERR_UNSUPPORTED, "denoise_step: bf16 path needs H %% 128 == 0, I %% 64 == 0");
@@ -241,7 +264,7 @@ void plan_step(const dllm_model* m, const dllm_state* st, const dllm_step_params
   if (m->dtype == DLLM_BF16 && !p->cfg) {
     GemmArgs g;   // the LM head's shape (see the step below)
     g.dtype = DLLM_BF16; g.K = m->H; g.M = s.vlen; g.host_cnt = s.max_rows; g.max_cnt = s.max_rows;
-    g.cnt_bound = s.max_rows; g.epi.kind = EPI_STORE;
+    g.cnt_bound = s.max_rows; g.epi.kind = EPI_STORE; g.w_fp8 = m->weight_format == DLLM_WEIGHTS_FP8;
     s.conf_parts = gemm_conf_parts(g);
   }
   const int H = m->H, QD = m->Hq * m->d;
@@ -328,11 +351,15 @@ size_t dllm_gemm_workspace_size(const dllm_gemm_desc* d) {
   return align256(n);
 }
 
-int dllm_gemm(const dllm_gemm_desc* d, const void* x, const void* w, void* y, const int32_t* n_rows_dev, void* ws,
-              size_t ws_bytes, cudaStream_t stream) {
+int dllm_gemm(const dllm_gemm_desc* d, const void* x, const void* w, const float* w_scale, void* y,
+              const int32_t* n_rows_dev, void* ws, size_t ws_bytes, cudaStream_t stream) {
   REQ(d && x && w && y, DLLM_ERR_INVALID_ARG, "gemm: NULL argument");
   REQ(d->N >= 0 && d->M > 0 && d->K > 0 && d->ldy >= d->M, DLLM_ERR_SHAPE, "gemm: bad N/M/K/ldy");
   REQ(d->dtype == DLLM_BF16 || d->dtype == DLLM_F32, DLLM_ERR_INVALID_ARG, "gemm: bad dtype");
+  if (d->w_fp8) {
+    REQ(d->dtype == DLLM_BF16 && !d->residual, DLLM_ERR_UNSUPPORTED, "gemm: FP8 weights need bf16 storage, no residual");
+    REQ(w_scale != nullptr, DLLM_ERR_INVALID_ARG, "gemm: FP8 weights need w_scale");
+  }
   int st = check_ws(ws, ws_bytes, dllm_gemm_workspace_size(d));
   if (st) return st;
   if (d->N == 0) return DLLM_OK;
@@ -348,6 +375,7 @@ int dllm_gemm(const dllm_gemm_desc* d, const void* x, const void* w, void* y, co
   a.x = x; a.x_rows = d->N; a.w = w; a.w_rows = d->M; a.K = d->K; a.M = d->M;
   a.cnt_dev = n_rows_dev; a.host_cnt = d->N; a.max_cnt = d->N; a.cnt_bound = d->N;
   a.dtype = d->dtype; a.status = status_word(ws);
+  a.w_fp8 = d->w_fp8; a.w_scale = d->w_fp8 ? w_scale : nullptr;
   a.f32_scratch = d->dtype == DLLM_F32 ? c.take<float>(gemm_f32_scratch_bytes(d->N, d->M, 0)) : nullptr;
   a.epi.kind = d->residual ? EPI_RESID : EPI_STORE;
   a.epi.out = y; a.epi.ldo = d->ldy; a.epi.out_f32 = d->y_f32 || d->dtype == DLLM_F32;
@@ -361,8 +389,8 @@ size_t dllm_grouped_gemm_workspace_size(const dllm_grouped_gemm_desc* d) {
 }
 
 int dllm_grouped_gemm(const dllm_grouped_gemm_desc* d, const void* x, const void* w, const void* w_extra,
-                      const int32_t* counts, const int32_t* offsets, void* y, void* ws, size_t ws_bytes,
-                      cudaStream_t stream) {
+                      const float* w_scale, const float* w_extra_scale, const int32_t* counts,
+                      const int32_t* offsets, void* y, void* ws, size_t ws_bytes, cudaStream_t stream) {
   REQ(d && x && w && counts && offsets && y, DLLM_ERR_INVALID_ARG, "grouped_gemm: NULL argument");
   REQ(d->G >= 1 && d->G <= 4096 && d->rows >= 0 && d->K > 0 && d->M > 0 && d->extra_rows >= 0 &&
           d->extra_rows <= d->rows,
@@ -373,6 +401,8 @@ int dllm_grouped_gemm(const dllm_grouped_gemm_desc* d, const void* x, const void
   REQ(d->K % 64 == 0 && (d->swiglu ? d->M % 64 == 0 : d->M % 128 == 0), DLLM_ERR_UNSUPPORTED,
       "grouped_gemm: needs K %% 64 == 0 and M %% 128 == 0 (swiglu: M %% 64 == 0)");
   REQ(!(d->swiglu && d->y_f32), DLLM_ERR_UNSUPPORTED, "grouped_gemm: swiglu output is in the storage type");
+  REQ(!d->w_fp8 || (w_scale && (!w_extra || w_extra_scale)), DLLM_ERR_INVALID_ARG,
+      "grouped_gemm: FP8 weights need their row scales");
   REQ(aligned16(x) && aligned16(w) && (!w_extra || aligned16(w_extra)) && aligned16(y), DLLM_ERR_ALIGN,
       "grouped_gemm: X, W, W_extra and Y must be 16-byte aligned");
   int st = check_ws(ws, ws_bytes, dllm_grouped_gemm_workspace_size(d));
@@ -387,6 +417,7 @@ int dllm_grouped_gemm(const dllm_grouped_gemm_desc* d, const void* x, const void
   a.has_extra = w_extra != nullptr; a.extra_off = d->rows - d->extra_rows; a.extra_cnt = d->extra_rows;
   a.max_cnt = std::max(1, std::min(d->max_rows_hint > 0 ? d->max_rows_hint : d->rows, d->rows));
   a.cnt_bound = d->rows; a.dtype = DLLM_BF16; a.status = status_word(ws);
+  a.w_fp8 = d->w_fp8; a.w_scale = d->w_fp8 ? w_scale : nullptr; a.w2_scale = d->w_fp8 ? w_extra_scale : nullptr;
   a.epi.kind = d->swiglu ? EPI_SWIGLU : EPI_STORE; a.epi.out = y; a.epi.ldo = d->M; a.epi.out_f32 = d->y_f32;
   return run_gemm(a, stream);
 }
@@ -482,9 +513,10 @@ size_t dllm_moe_experts_workspace_size(const dllm_expert_desc* d) {
 }
 
 int dllm_moe_experts(const dllm_expert_desc* d, const void* h, const void* w_gu, const void* w_down,
-                     const void* w_gu_shared, const void* w_down_shared, const int32_t* counts, const int32_t* offsets,
-                     const int32_t* perm, const int32_t* inv, const float* gates, void* x_inout, void* ws,
-                     size_t ws_bytes, cudaStream_t stream) {
+                     const void* w_gu_shared, const void* w_down_shared, const float* w_gu_scale,
+                     const float* w_down_scale, const float* w_gu_shared_scale, const float* w_down_shared_scale,
+                     const int32_t* counts, const int32_t* offsets, const int32_t* perm, const int32_t* inv,
+                     const float* gates, void* x_inout, void* ws, size_t ws_bytes, cudaStream_t stream) {
   REQ(d && h && w_gu && w_down && counts && offsets && perm && inv && gates && x_inout, DLLM_ERR_INVALID_ARG,
       "moe_experts: NULL argument");
   REQ((w_gu_shared == nullptr) == (w_down_shared == nullptr), DLLM_ERR_INVALID_ARG,
@@ -494,6 +526,11 @@ int dllm_moe_experts(const dllm_expert_desc* d, const void* h, const void* w_gu,
   REQ(d->E <= 1024 && d->k <= 32, DLLM_ERR_UNSUPPORTED, "moe_experts: needs E <= 1024, k <= 32");
   REQ(d->dtype == DLLM_BF16 || d->dtype == DLLM_F32, DLLM_ERR_INVALID_ARG, "moe_experts: bad dtype");
   REQ((d->H * esize(d->dtype)) % 16 == 0, DLLM_ERR_SHAPE, "moe_experts: H row bytes must be a multiple of 16");
+  if (d->w_fp8) {
+    REQ(d->dtype == DLLM_BF16, DLLM_ERR_UNSUPPORTED, "moe_experts: FP8 weights need bf16 storage");
+    REQ(w_gu_scale && w_down_scale && (!w_gu_shared || (w_gu_shared_scale && w_down_shared_scale)),
+        DLLM_ERR_INVALID_ARG, "moe_experts: FP8 weights need their row scales");
+  }
   if (d->dtype == DLLM_BF16) {
     REQ(d->H % 128 == 0 && d->I % 64 == 0, DLLM_ERR_UNSUPPORTED, "moe_experts: bf16 needs H %% 128 == 0, I %% 64 == 0");
     REQ(aligned16(h) && aligned16(w_gu) && aligned16(w_down) && (!w_gu_shared || (aligned16(w_gu_shared) && aligned16(w_down_shared))),
@@ -505,8 +542,12 @@ int dllm_moe_experts(const dllm_expert_desc* d, const void* h, const void* w_gu,
   Carver c(ws);
   ExpertBufs b;
   carve_experts(c, d->dtype, d->Tk, d->H, d->k, d->I, 1, b);
+  ExpertScales esc;
+  if (d->w_fp8) {
+    esc.gu = w_gu_scale; esc.down = w_down_scale; esc.gu_shared = w_gu_shared_scale; esc.down_shared = w_down_shared_scale;
+  }
   return run_experts(d->dtype, d->Tk, d->H, d->E, d->k, d->I, h, w_gu, w_down, w_gu_shared, w_down_shared, counts,
-                     offsets, perm, inv, gates, x_inout, b, status_word(ws), stream);
+                     offsets, perm, inv, gates, x_inout, b, status_word(ws), stream, PostNorm(), nullptr, esc);
 }
 
 // ------------------------------------------------------------------------------------------------ unmask
@@ -568,8 +609,12 @@ int dllm_denoise_step_views(const dllm_model* m, const dllm_state* st, const dll
   return DLLM_OK;
 }
 
-int dllm_denoise_step(const dllm_model* m, const dllm_state* st, const dllm_step_params* p, void* ws,
-                      size_t ws_bytes, cudaStream_t stream) {
+}  // extern "C"
+
+namespace {
+// One pass; with set_cond the unmask selection also sets the graph condition `cond` to (masked positions left > 0).
+int denoise_step_impl(const dllm_model* m, const dllm_state* st, const dllm_step_params* p, void* ws,
+                      size_t ws_bytes, cudaStream_t stream, cudaGraphConditionalHandle cond, int set_cond) {
   int r = validate_step(m, st, p);
   if (r) return r;
   StepPlan s;
@@ -654,8 +699,13 @@ int dllm_denoise_step(const dllm_model* m, const dllm_state* st, const dllm_step
       pn.g = m->final_norm; pn.eps = m->eps; pn.out = s.xf; pn.mode = NORM_FINAL; pn.mask = st->mask;
       pn.n_half_pos = s.Bl * L; pn.n_dev = s.n_rows;
     }
+    ExpertScales esc;
+    if (m->weight_format == DLLM_WEIGHTS_FP8) {
+      esc.gu = Ly.w_gu_scale; esc.down = Ly.w_down_scale;
+      esc.gu_shared = Ly.w_gu_shared_scale; esc.down_shared = Ly.w_down_shared_scale;
+    }
     TRY(run_experts(dt, s.Tk, H, m->E, m->k, m->I, s.h, Ly.w_gu, Ly.w_down, Ly.w_gu_shared, Ly.w_down_shared,
-                    counts, s.offsets, s.perm, s.inv, s.gates, s.x, s.eb, status, stream, pn, live));
+                    counts, s.offsets, s.perm, s.inv, s.gates, s.x, s.eb, status, stream, pn, live, esc));
   }
   if (p->commit) return DLLM_OK;
   // final norm on the masked rows (cond, then uncond) unless fused above, LM head, confidence + unmasking
@@ -664,7 +714,10 @@ int dllm_denoise_step(const dllm_model* m, const dllm_state* st, const dllm_step
                        p->cfg, s.Bl * L, stream));
   GemmArgs gl;
   gl.x = s.xf; gl.x_rows = (int64_t)s.halves * s.max_rows;
-  gl.w = static_cast<const char*>(m->w_lm) + (size_t)p->vocab_offset * H * es; gl.w_rows = s.vlen;
+  const bool lm_fp8 = m->weight_format == DLLM_WEIGHTS_FP8;
+  gl.w = static_cast<const char*>(m->w_lm) + (size_t)p->vocab_offset * H * (lm_fp8 ? 1 : es); gl.w_rows = s.vlen;
+  gl.w_fp8 = lm_fp8;
+  gl.w_scale = lm_fp8 ? m->w_lm_scale + p->vocab_offset : nullptr;
   gl.K = H; gl.M = s.vlen; gl.cnt_dev = s.n_rows + 1; gl.host_cnt = s.halves * s.max_rows;
   gl.max_cnt = s.halves * s.max_rows; gl.cnt_bound = s.halves * s.max_rows; gl.dtype = dt; gl.status = status;
   gl.f32_scratch = s.proj_scratch;
@@ -682,8 +735,121 @@ int dllm_denoise_step(const dllm_model* m, const dllm_state* st, const dllm_step
   ua.remaining = p->remaining; ua.partials = s.partials;
   ua.n_chunks = s.conf_parts ? s.conf_parts : s.n_chunks;
   ua.partials_ready = s.conf_parts ? 1 : 0;
+  ua.cond = cond;
+  ua.set_cond = set_cond;
   TRY(launch_unmask(ua, stream));
 #undef TRY
+  return DLLM_OK;
+}
+}  // namespace
+
+extern "C" {
+
+int dllm_denoise_step(const dllm_model* m, const dllm_state* st, const dllm_step_params* p, void* ws,
+                      size_t ws_bytes, cudaStream_t stream) {
+  return denoise_step_impl(m, st, p, ws, ws_bytes, stream, cudaGraphConditionalHandle(), 0);
+}
+
+// ------------------------------------------------------------------------------------------------ block graph
+struct dllm_block_graph {
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t exec = nullptr;
+  int passes = 0;
+};
+
+void dllm_block_graph_destroy(dllm_block_graph* g) {
+  if (!g) return;
+  if (g->exec) cudaGraphExecDestroy(g->exec);
+  if (g->graph) cudaGraphDestroy(g->graph);
+  delete g;
+}
+
+int dllm_block_graph_create(const dllm_model* m, const dllm_state* st, const dllm_step_params* p, void* ws,
+                            size_t ws_bytes, cudaStream_t capture_stream, dllm_block_graph** out) {
+  REQ(out != nullptr, DLLM_ERR_INVALID_ARG, "block_graph_create: NULL output");
+  *out = nullptr;
+  REQ(capture_stream != nullptr, DLLM_ERR_INVALID_ARG,
+      "block_graph_create: capture needs a created stream (not the legacy default stream)");
+  int r = validate_step(m, st, p);
+  if (r) return r;
+  REQ(!p->commit, DLLM_ERR_INVALID_ARG, "block_graph_create: the template must describe a denoising pass");
+  {
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    cudaError_t e = cudaStreamIsCapturing(capture_stream, &cs);
+    if (e != cudaSuccess) return dllm_host::cuda_status(e, "block_graph_create: cudaStreamIsCapturing");
+    REQ(cs == cudaStreamCaptureStatusNone, DLLM_ERR_INVALID_ARG, "block_graph_create: the stream is capturing");
+  }
+  // every pass (with and without SPRINT selection) and the commit pass fit the workspace
+  dllm_step_params pp = *p;
+  for (int variant = 0; variant < 3; ++variant) {
+    pp.retain = variant == 1 ? (p->sprint ? 1 : 0) : 0;
+    pp.commit = variant == 2;
+    StepPlan s;
+    plan_step(m, st, &pp, nullptr, s);
+    r = check_ws(ws, ws_bytes, s.total);
+    if (r) return r;
+  }
+  dllm_block_graph* g = new dllm_block_graph();
+  auto fail = [&](cudaError_t e, const char* what) {
+    dllm_block_graph_destroy(g);
+    return dllm_host::cuda_status(e, what);
+  };
+  cudaError_t e = cudaGraphCreate(&g->graph, 0);
+  if (e != cudaSuccess) return fail(e, "block_graph_create: cudaGraphCreate");
+  cudaGraphConditionalHandle cond;
+  e = cudaGraphConditionalHandleCreate(&cond, g->graph, 1, cudaGraphCondAssignDefault);
+  if (e != cudaSuccess) return fail(e, "block_graph_create: cudaGraphConditionalHandleCreate");
+  cudaGraphNode_t prev = nullptr;
+  for (int t = 0; t < p->T_s; ++t) {
+    cudaGraphNodeParams np = {};
+    np.type = cudaGraphNodeTypeConditional;
+    np.conditional.handle = cond;
+    np.conditional.type = cudaGraphCondTypeIf;
+    np.conditional.size = 1;
+    cudaGraphNode_t node;
+    e = cudaGraphAddNode(&node, g->graph, prev ? &prev : nullptr, prev ? 1 : 0, &np);
+    if (e != cudaSuccess) return fail(e, "block_graph_create: cudaGraphAddNode (conditional)");
+    cudaGraph_t body = np.conditional.phGraph_out[0];
+    e = cudaStreamBeginCaptureToGraph(capture_stream, body, nullptr, nullptr, 0, cudaStreamCaptureModeThreadLocal);
+    if (e != cudaSuccess) return fail(e, "block_graph_create: cudaStreamBeginCaptureToGraph");
+    pp = *p;
+    pp.t = t;
+    pp.commit = 0;
+    pp.retain = p->sprint && t == 0 ? 1 : 0;
+    r = denoise_step_impl(m, st, &pp, ws, ws_bytes, capture_stream, cond, 1);
+    cudaGraph_t captured = nullptr;
+    e = cudaStreamEndCapture(capture_stream, &captured);
+    if (r) {
+      dllm_block_graph_destroy(g);
+      return r;
+    }
+    if (e != cudaSuccess) return fail(e, "block_graph_create: cudaStreamEndCapture");
+    prev = node;
+  }
+  e = cudaStreamBeginCaptureToGraph(capture_stream, g->graph, &prev, nullptr, 1, cudaStreamCaptureModeThreadLocal);
+  if (e != cudaSuccess) return fail(e, "block_graph_create: cudaStreamBeginCaptureToGraph (commit)");
+  pp = *p;
+  pp.commit = 1;
+  pp.retain = 0;
+  r = denoise_step_impl(m, st, &pp, ws, ws_bytes, capture_stream, cudaGraphConditionalHandle(), 0);
+  cudaGraph_t captured = nullptr;
+  e = cudaStreamEndCapture(capture_stream, &captured);
+  if (r) {
+    dllm_block_graph_destroy(g);
+    return r;
+  }
+  if (e != cudaSuccess) return fail(e, "block_graph_create: cudaStreamEndCapture (commit)");
+  e = cudaGraphInstantiate(&g->exec, g->graph, 0);
+  if (e != cudaSuccess) return fail(e, "block_graph_create: cudaGraphInstantiate");
+  g->passes = p->T_s;
+  *out = g;
+  return DLLM_OK;
+}
+
+int dllm_block_graph_launch(const dllm_block_graph* g, cudaStream_t stream) {
+  REQ(g != nullptr && g->exec != nullptr, DLLM_ERR_INVALID_ARG, "block_graph_launch: NULL graph");
+  cudaError_t e = cudaGraphLaunch(g->exec, stream);
+  if (e != cudaSuccess) return dllm_host::cuda_status(e, "block_graph_launch: cudaGraphLaunch");
   return DLLM_OK;
 }
 

@@ -33,11 +33,14 @@ constexpr int STAGE_COLS = 32;         // epilogue column chunk
 constexpr int STAGING_BYTES = 128 * STAGE_COLS * 4;
 constexpr int MAX_GROUPS = 1040;
 constexpr int NUM_THREADS = 192;
+constexpr int NUM_THREADS_F8 = 320;    // FP8 weights: four more warps turn the E4M3 tiles into bf16 operand tiles
+constexpr int RAW_BYTES = 128 * BK;    // 8 KB E4M3 weight tile per stage
 constexpr int SMEM_LIMIT = 232448;
 
 struct Smem {
   uint64_t full[16];
   uint64_t empty[16];
+  uint64_t conv[16];                // FP8: the stage's bf16 weight tile is written (128 converter arrivals)
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t done;
@@ -48,7 +51,7 @@ struct Smem {
   int tile_prefix[MAX_GROUPS + 1];  // exclusive prefix of tiles per group
   int grp_off[MAX_GROUPS];
   int grp_cnt[MAX_GROUPS];
-  int chunk_sum[NUM_THREADS];
+  int chunk_sum[NUM_THREADS_F8];
 };
 
 struct KParams {
@@ -61,6 +64,8 @@ struct KParams {
   const int32_t* grp_cnt;
   const int32_t* cnt_dev;
   const int32_t* live;     // nullable: *live == 0 empties every group (a denoising pass with no masked position)
+  const float* w_scale;    // FP8 weights: per weight row of W / W2 (null otherwise)
+  const float* w2_scale;
   EpiParams epi;
   int32_t* status;
   int prefetch_w;          // 1: dense with at most BN rows, so a CTA's first tile is m-tile = its first tile index and
@@ -340,13 +345,54 @@ __device__ __forceinline__ void epilogue_logits_conf(const KParams& p, const flo
   }
 }
 
-template <int BN, int STAGES>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+// FP8 weights: one stage's E4M3 tile (128 rows x 64 codes, row r at byte r * 64, as the TMA box lands it) into the
+// bf16 operand tile the MMA reads (row r at byte r * 128, its eight 16-byte chunks XOR-swizzled by r & 7, the layout
+// a 128-byte-swizzling TMA load produces). Every E4M3 value is exact in bf16 (3 mantissa bits, exponents 2^-9 ..
+// 2^8), so the tile holds the codes' values unscaled; the per-row scale is applied to the accumulator. 128 threads,
+// four 16-byte pieces each (consecutive threads read consecutive 16 bytes).
+__device__ __forceinline__ void convert_e4m3_tile(const uint8_t* raw, uint8_t* a_tile, int ct) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int c = ct + 128 * i;
+    const int row = c >> 2, part = c & 3;
+    const uint4 q = *reinterpret_cast<const uint4*>(raw + row * 64 + part * 16);
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int h = 0; h < 8; ++h) {
+      const uint16_t pair = (uint16_t)(w[h >> 1] >> ((h & 1) * 16));
+      uint32_t f16x2;
+      asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(f16x2) : "h"(pair));
+      const __half2 hv = *reinterpret_cast<const __half2*>(&f16x2);
+      const float2 fv = __half22float2(hv);
+      const __nv_bfloat162 bv = __floats2bfloat162_rn(fv.x, fv.y);
+      o[h] = *reinterpret_cast<const uint32_t*>(&bv);
+    }
+    uint8_t* dst = a_tile + row * 128;
+    const int sw = row & 7;
+    *reinterpret_cast<uint4*>(dst + (((2 * part) ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+    *reinterpret_cast<uint4*>(dst + (((2 * part + 1) ^ sw) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+  }
+}
+
+// Scale of tile row r of tile (g, mt) for FP8 weights: the row of W (or W2 for the extra group) it came from.
+__device__ __forceinline__ float f8_row_scale(const KParams& p, int g, int mt, int r) {
+  const bool extra = p.has_extra && g == p.n_dev;
+  const float* sc = extra ? p.w2_scale : p.w_scale + (extra ? 0 : (int64_t)g * p.w_group_stride);
+  const int wr = p.swiglu ? (r < 64 ? mt * 64 + r : p.M + mt * 64 + r - 64) : mt * 128 + r;
+  return sc[wr];
+}
+
+template <int BN, int STAGES, bool F8 = false>
+__global__ void __launch_bounds__(F8 ? NUM_THREADS_F8 : NUM_THREADS, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_w2,
                const __grid_constant__ CUtensorMap tmap_x, const KParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  constexpr int STAGE_BYTES = A_BYTES + BN * BK * 2;
+  constexpr int NT = F8 ? NUM_THREADS_F8 : NUM_THREADS;
+  constexpr int B_BYTES = BN * BK * 2;
+  constexpr int STAGE_BYTES = A_BYTES + B_BYTES + (F8 ? RAW_BYTES : 0);   // [A bf16][B][E4M3 codes (FP8)]
+  constexpr uint32_t W_TX = F8 ? RAW_BYTES : A_BYTES;                     // weight bytes a stage's TMA brings
   uint8_t* stages = base;
   float* staging = reinterpret_cast<float*>(base + STAGES * STAGE_BYTES);
   Smem& sm = *reinterpret_cast<Smem*>(base + STAGES * STAGE_BYTES + STAGING_BYTES);
@@ -361,6 +407,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
     for (int s = 0; s < STAGES; ++s) {
       tc::mbar_init(&sm.full[s], 1);
       tc::mbar_init(&sm.empty[s], 1);
+      if (F8) tc::mbar_init(&sm.conv[s], 128);
     }
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(&sm.tfull[b], 1);
@@ -385,8 +432,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
       tc::prefetch_tmap(&tmap_w);
       const uint64_t pol_w = tc::policy_evict_first();
       for (int i = 0; i < npf; ++i) {
-        tc::mbar_expect_tx(&sm.full[i], A_BYTES);
-        tc::tma_load_2d(stages + i * STAGE_BYTES, &tmap_w, (kb0 + i) * BK, t0 * 128, &sm.full[i], pol_w);
+        tc::mbar_expect_tx(&sm.full[i], W_TX);
+        tc::tma_load_2d(stages + i * STAGE_BYTES + (F8 ? A_BYTES + B_BYTES : 0), &tmap_w, (kb0 + i) * BK, t0 * 128,
+                        &sm.full[i], pol_w);
       }
     }
   }
@@ -395,7 +443,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
   pdl_enter();
   // ---- group table: counts, offsets and the exclusive prefix of tiles per group
   const bool dead = p.live && *p.live == 0;
-  for (int g = tid; g < n_groups; g += NUM_THREADS) {
+  for (int g = tid; g < n_groups; g += NT) {
     int off, cnt;
     if (g < p.n_dev) {
       off = p.grp_off[g];
@@ -412,10 +460,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
   }
   __syncthreads();
   // prefix of tiles per group: contiguous chunks per thread, a shuffle scan of the thread sums inside each warp,
-  // then the six warp totals
+  // then the warp totals
   {
     int* warp_tot = sm.chunk_sum;
-    const int per = (n_groups + NUM_THREADS - 1) / NUM_THREADS;
+    const int per = (n_groups + NT - 1) / NT;
     const int g0 = tid * per, g1 = min(n_groups, g0 + per);
     int s = 0;
     for (int g = g0; g < g1; ++g) s += ((sm.grp_cnt[g] + BN - 1) / BN) * p.m_tiles;
@@ -429,7 +477,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
     __syncthreads();
     int before = 0, all = 0;
 #pragma unroll
-    for (int w2 = 0; w2 < NUM_THREADS / 32; ++w2) {
+    for (int w2 = 0; w2 < NT / 32; ++w2) {
       const int v = warp_tot[w2];
       if (w2 < warp) before += v;
       all += v;
@@ -467,7 +515,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
         const CUtensorMap* wm = extra ? &tmap_w2 : &tmap_w;
         const int64_t wrow = extra ? 0 : (int64_t)g * p.w_group_stride;
         const int nb = (nval + XBOX_ROWS - 1) / XBOX_ROWS;
-        const uint32_t bytes = A_BYTES + nb * XBOX_BYTES;
+        const uint32_t bytes = W_TX + nb * XBOX_BYTES;
         const int xrow = sm.grp_off[g] + n0;
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % STAGES;
@@ -475,15 +523,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
           if (!wait_bar(&sm.empty[s], ph ^ 1, abort_flag, p.status, ST_TIMEOUT_PRODUCER)) { ok = false; break; }
           uint8_t* a = stages + s * STAGE_BYTES;
           uint8_t* b = a + A_BYTES;
+          uint8_t* wdst = F8 ? a + A_BYTES + B_BYTES : a;   // FP8: the codes land after the B tile
           if (it < (uint32_t)npf) {   // weight stage already in flight: arrive with the activation bytes
-            tc::mbar_arrive_expect_tx(&sm.full[s], bytes - A_BYTES);
+            tc::mbar_arrive_expect_tx(&sm.full[s], bytes - W_TX);
           } else {
             tc::mbar_arrive_expect_tx(&sm.full[s], bytes);
             if (p.swiglu) {
-              tc::tma_load_2d(a, wm, kb * BK, (int)(wrow + mt * 64), &sm.full[s], pol_w);
-              tc::tma_load_2d(a + A_BYTES / 2, wm, kb * BK, (int)(wrow + p.M + mt * 64), &sm.full[s], pol_w);
+              tc::tma_load_2d(wdst, wm, kb * BK, (int)(wrow + mt * 64), &sm.full[s], pol_w);
+              tc::tma_load_2d(wdst + W_TX / 2, wm, kb * BK, (int)(wrow + p.M + mt * 64), &sm.full[s], pol_w);
             } else {
-              tc::tma_load_2d(a, wm, kb * BK, (int)(wrow + mt * 128), &sm.full[s], pol_w);
+              tc::tma_load_2d(wdst, wm, kb * BK, (int)(wrow + mt * 128), &sm.full[s], pol_w);
             }
           }
           for (int j = 0; j < nb; ++j)
@@ -521,7 +570,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
-          if (!wait_bar(&sm.full[s], ph, abort_flag, p.status, ST_TIMEOUT_MMA)) { ok = false; break; }
+          if (!wait_bar(F8 ? &sm.conv[s] : &sm.full[s], ph, abort_flag, p.status, ST_TIMEOUT_MMA)) { ok = false; break; }
           tc::fence_after_sync();
           const uint32_t a = tc::smem_u32(stages + s * STAGE_BYTES);
           const uint32_t b = a + A_BYTES;
@@ -536,6 +585,26 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
       // all issued MMAs complete before TMEM is released
       tc::mma_commit(&sm.done);
       tc::mbar_wait(&sm.done, 0, 1u << 20);
+    }
+  } else if (F8 && warp >= 6) {
+    // ------------------------------------------------------------------ FP8: converter warps 6..9
+    // the same stage sequence as the MMA issuer: wait for the stage's copies, write its bf16 weight tile, make the
+    // writes visible to the tensor core (async proxy) and arrive on the stage's conv barrier
+    const int ct = tid - 192;
+    uint32_t it = 0;
+    bool ok = true;
+    for (int wk = wk_begin; wk < total && ok; wk += wk_step) {
+      const int ks = wk - (wk / p.ksplit) * p.ksplit;
+      const int kb0 = ks * kblocks / p.ksplit, kb1 = (ks + 1) * kblocks / p.ksplit;
+      for (int kb = kb0; kb < kb1; ++kb, ++it) {
+        const int s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1;
+        if (!wait_bar(&sm.full[s], ph, abort_flag, p.status, ST_TIMEOUT_MMA)) { ok = false; break; }
+        uint8_t* a = stages + s * STAGE_BYTES;
+        convert_e4m3_tile(a + A_BYTES + B_BYTES, a, ct);
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        tc::mbar_arrive(&sm.conv[s]);
+      }
     }
   } else {
     // ------------------------------------------------------------------ epilogue warps 2..5
@@ -554,6 +623,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
       if (!wait_bar(&sm.tfull[buf], tph, abort_flag, p.status, ST_TIMEOUT_EPILOGUE)) break;
       tc::fence_after_sync();
       if (p.ksplit == 1) {
+        const float rs = F8 ? f8_row_scale(p, g, mt, row) : 1.f;
         for (int c0 = 0; c0 < nval; c0 += STAGE_COLS) {
           float v[STAGE_COLS];
           const uint32_t taddr = sm.tmem_base + ((uint32_t)(q * 32) << 16) + buf * BN + c0;
@@ -561,7 +631,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
           tc::tmem_ld16(taddr + 16, v + 16);
           tc::named_bar_sync(1, 128);  // staging free (previous chunk consumed)
 #pragma unroll
-          for (int j = 0; j < STAGE_COLS; ++j) staging[j * 128 + row] = v[j];
+          for (int j = 0; j < STAGE_COLS; ++j) staging[j * 128 + row] = F8 ? v[j] * rs : v[j];
           tc::named_bar_sync(1, 128);
           if constexpr (BN == 32) {
             if (p.epi.conf_part) {
@@ -898,18 +968,21 @@ EncodeTiledFn get_encode() {
   return fn;
 }
 
-int make_map(CUtensorMap* m, const void* ptr, int64_t rows, int K, int box_rows) {
+// bf16 [rows, K] with 128-byte swizzled boxes of 64 x box_rows, or (u8) E4M3 codes [rows, K] with plain boxes of
+// 64 bytes x box_rows (the converter warps read them row by row)
+int make_map(CUtensorMap* m, const void* ptr, int64_t rows, int K, int box_rows, bool u8 = false) {
   EncodeTiledFn enc = get_encode();
   if (!enc) {
     dllm_host::set_error("cuTensorMapEncodeTiled unavailable");
     return DLLM_ERR_CUDA;
   }
   cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+  cuuint64_t strides[1] = {(cuuint64_t)K * (u8 ? 1 : 2)};
   cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+  CUresult r = enc(m, u8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr),
+                   dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   u8 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     dllm_host::set_error("cuTensorMapEncodeTiled failed (%d) rows=%lld K=%d box_rows=%d", (int)r, (long long)rows,
@@ -923,10 +996,10 @@ int make_map(CUtensorMap* m, const void* ptr, int64_t rows, int K, int box_rows)
 int launch_cluster_splitk(const GemmArgs& a, const CUtensorMap& mw, const CUtensorMap& mw2, const CUtensorMap& mx,
                           const KParams& kp, cudaStream_t s);
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, bool F8 = false>
 int launch(const GemmArgs& a, const CUtensorMap& mw, const CUtensorMap& mw2, const CUtensorMap& mx,
            const KParams& kp, cudaStream_t s) {
-  constexpr int STAGE_BYTES = A_BYTES + BN * BK * 2;
+  constexpr int STAGE_BYTES = A_BYTES + BN * BK * 2 + (F8 ? RAW_BYTES : 0);
   constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + STAGING_BYTES + (int)sizeof(Smem);
   static_assert(SMEM <= SMEM_LIMIT, "shared memory budget");
   // With programmatic dependent launch a CTA allocates tensor memory before it waits for the kernels ahead of it.
@@ -935,12 +1008,12 @@ int launch(const GemmArgs& a, const CUtensorMap& mw, const CUtensorMap& mw2, con
   static_assert(SMEM > 233472 / 2, "tensor-memory kernels must not share an SM");
   static bool configured = false;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, STAGES, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          SMEM);
     if (e != cudaSuccess) return dllm_host::cuda_status(e, "cudaFuncSetAttribute(gemm_tc)");
     configured = true;
   }
-  launch_pdl((gemm_tc_kernel<BN, STAGES>), num_sms(), NUM_THREADS, SMEM, s, mw, mw2, mx, kp);
+  launch_pdl((gemm_tc_kernel<BN, STAGES, F8>), num_sms(), F8 ? NUM_THREADS_F8 : NUM_THREADS, SMEM, s, mw, mw2, mx, kp);
   DLLM_CHECK_LAUNCH("gemm_tc_kernel");
   return DLLM_OK;
 }
@@ -1077,10 +1150,16 @@ int gemm_bf16_tc(const GemmArgs& a, cudaStream_t s) {
   if (a.epi.kind == EPI_QKV)
     DLLM_REQUIRE(a.epi.d == 128, DLLM_ERR_UNSUPPORTED, "gemm: QKV epilogue needs head dim 128");
   const int box_rows = a.swiglu ? 64 : 128;
+  const bool f8 = a.w_fp8 != 0;
+  if (f8) {
+    DLLM_REQUIRE(a.w_scale && (!a.w2 || a.w2_scale), DLLM_ERR_INVALID_ARG, "gemm: FP8 weights need their row scales");
+    DLLM_REQUIRE(a.epi.kind == EPI_STORE || a.epi.kind == EPI_SWIGLU, DLLM_ERR_UNSUPPORTED,
+                 "gemm: FP8 weights take the store or SwiGLU epilogue");
+  }
   CUtensorMap mw, mw2, mx;
-  int st = make_map(&mw, a.w, a.w_rows, a.K, box_rows);
+  int st = make_map(&mw, a.w, a.w_rows, a.K, box_rows, f8);
   if (st) return st;
-  st = make_map(&mw2, a.w2 ? a.w2 : a.w, a.w2 ? a.w2_rows : a.w_rows, a.K, box_rows);
+  st = make_map(&mw2, a.w2 ? a.w2 : a.w, a.w2 ? a.w2_rows : a.w_rows, a.K, box_rows, f8);
   if (st) return st;
   st = make_map(&mx, a.x, a.x_rows, a.K, XBOX_ROWS);
   if (st) return st;
@@ -1099,6 +1178,8 @@ int gemm_bf16_tc(const GemmArgs& a, cudaStream_t s) {
   kp.grp_cnt = a.grp_cnt;
   kp.cnt_dev = a.cnt_dev;
   kp.live = a.live;
+  kp.w_scale = a.w_scale;
+  kp.w2_scale = a.w2_scale;
   kp.epi = a.epi;
   if (kp.epi.kind == EPI_QKV)
     for (int m = 0; m < 64; ++m) kp.epi.inv_freq[m] = std::pow((double)kp.epi.rope_base, -2.0 * (double)m / 128.0);
@@ -1111,7 +1192,11 @@ int gemm_bf16_tc(const GemmArgs& a, cudaStream_t s) {
   kp.ksplit = ks;
   kp.prefetch_w = (!a.swiglu && !a.n_dev && !a.has_extra && a.host_cnt <= (ks > 1 ? 32 : bn)) ? 1 : 0;
   int st2;
-  if (gemm_uses_pairs(a)) {
+  if (f8) {   // single-CTA tiles, no split-K (the weight-streaming shapes FP8 weights serve)
+    if (bn == 32) st2 = launch<32, 6, true>(a, mw, mw2, mx, kp, s);
+    else if (bn == 64) st2 = launch<64, 6, true>(a, mw, mw2, mx, kp, s);
+    else st2 = launch<128, 4, true>(a, mw, mw2, mx, kp, s);
+  } else if (gemm_uses_pairs(a)) {
     kp.prefetch_w = 0;
     st2 = launch_pair(mw, mw2, mx, kp, s);
   } else if (ks > 1) st2 = launch_cluster_splitk(a, mw, mw2, mx, kp, s);
@@ -1137,6 +1222,7 @@ static bool dense(const GemmArgs& a) { return !a.swiglu && !a.n_dev && !a.has_ex
 // operand traffic cost more than the idle SMs.
 int gemm_bn(const GemmArgs& a) {
   int bn = bn_for(a.max_cnt);
+  if (a.w_fp8) return std::min(bn, 128);   // FP8 weights: single-CTA tiles of at most 128 rows
   if (dense(a))
     while (bn > 32 && (a.M / 128) * ((a.max_cnt + bn - 1) / bn) < num_sms() / 2) bn /= 2;
   return bn;
@@ -1148,7 +1234,7 @@ int gemm_bn(const GemmArgs& a) {
 int gemm_splitk_factor(const GemmArgs& a, int bn) {
   // the grid is (slices, tiles) with the tile count fixed on the host: rows from a device count are excluded,
   // except that a single N tile stays a single N tile for any count
-  if (a.dtype != DLLM_BF16 || !dense(a) || bn != 32) return 1;
+  if (a.dtype != DLLM_BF16 || !dense(a) || bn != 32 || a.w_fp8) return 1;
   if (a.cnt_dev && a.host_cnt > 32) return 1;
   const int tiles = splitk_tiles(a);
   const int kblocks = a.K / BK;
@@ -1159,7 +1245,8 @@ int gemm_splitk_factor(const GemmArgs& a, int bn) {
 }
 
 bool gemm_uses_pairs(const GemmArgs& a) {
-  if (a.dtype != DLLM_BF16 || a.epi.conf_part || gemm_bn(a) != 256 || gemm_splitk_factor(a, 256) != 1) return false;
+  if (a.dtype != DLLM_BF16 || a.w_fp8 || a.epi.conf_part || gemm_bn(a) != 256 || gemm_splitk_factor(a, 256) != 1)
+    return false;
   return a.swiglu ? (a.M / 64) % 2 == 0 : (a.M / 128) % 2 == 0;
 }
 

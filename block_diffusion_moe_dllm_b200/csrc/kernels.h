@@ -69,6 +69,11 @@ struct GemmArgs {
   int cnt_bound = 0;       // true upper bound of rows in any group (sizes the SIMT grid)
   int dtype = 0;           // DLLM_BF16 / DLLM_F32
   const int32_t* live = nullptr;  // nullable device word: 0 = the pass has nothing left to do (every group empty)
+  // FP8 weights: W and W2 hold E4M3 codes (one byte each, same row layout) and w_scale / w2_scale one fp32 scale per
+  // weight row (w_scale indexed like the rows of W, w2_scale like those of W2); the output is scale[row] * (X q^T)
+  int w_fp8 = 0;
+  const float* w_scale = nullptr;
+  const float* w2_scale = nullptr;
   EpiParams epi;
   int32_t* status = nullptr;
   float* f32_scratch = nullptr;  // f32 path: [x_rows, M (x2 for swiglu)] raw products

@@ -55,6 +55,8 @@ struct UnmaskArgs {
   void* partials;  // workspace: max_rows * n_chunks entries
   int n_chunks;
   int partials_ready = 0;  // 1: the partials were written by the LM head's fused epilogue (no reduction launch)
+  cudaGraphConditionalHandle cond = 0;  // with set_cond: the selection sets this graph condition to (remaining > 0)
+  int set_cond = 0;
 };
 int unmask_chunks(int max_rows, int V);
 size_t unmask_partials_bytes(int max_rows, int n_chunks);

@@ -84,7 +84,7 @@ __global__ void __launch_bounds__(256) route_scores_kernel(const T* __restrict__
 // order) is decided again from exact scores (exact_redecide). Any expert whose fp32 biased score is below the
 // (k+1)-th by more than the guard cannot reach the top k, so only the experts within the guard of the (k+1)-th
 // score or above it are re-scored.
-constexpr float kRouteGuard = 2e-5f;
+constexpr float kRouteGuard = 1e-5f;
 
 // Top-k of one token's expert scores, one warp. Lane l owns experts e = i * 32 + l (i < PER); the selection key is
 // the biased score val = raw + bias (ties to the lower expert), the gate the unbiased raw score, renormalised over
@@ -185,32 +185,51 @@ DLLM_DEV bool warp_topk(float* __restrict__ srow, const float* __restrict__ bias
 
 // Exact dot product of two rows of H elements (H % 8 == 0), one warp; every lane returns the sum. A product of two
 // bf16 values is exact in fp32 (8 + 8 significant bits), so bf16 rows add fp32 products in fp64; fp32 rows use
-// fp64 fused multiply-adds. Either way the sum of H = 2048 terms is within about 1e-13 of the exact value.
-DLLM_DEV double warp_dot64(const __nv_bfloat16* __restrict__ a, const __nv_bfloat16* __restrict__ b, int H,
-                           int lane) {
-  double s0 = 0.0, s1 = 0.0;
-  for (int c = lane * 8; c < H; c += 256) {
-    float fa[8], fb[8];
-    bf16x8_to_f32(*reinterpret_cast<const uint4*>(a + c), fa);
-    bf16x8_to_f32(*reinterpret_cast<const uint4*>(b + c), fb);
+// fp64 fused multiply-adds. Either way the sum of H = 2048 terms is within about 1e-13 of the exact value. Each
+// lane has UNR 8-element chunks of both rows in flight at a time (the rows come from L2).
+DLLM_DEV void dot_chunk(const uint4& ua, const uint4& ub, double& s0, double& s1, const __nv_bfloat16*) {
+  float fa[8], fb[8];
+  bf16x8_to_f32(ua, fa);
+  bf16x8_to_f32(ub, fb);
 #pragma unroll
-    for (int u = 0; u < 8; u += 2) {
-      s0 += (double)(fa[u] * fb[u]);
-      s1 += (double)(fa[u + 1] * fb[u + 1]);
-    }
+  for (int u = 0; u < 8; u += 2) {
+    s0 += (double)(fa[u] * fb[u]);
+    s1 += (double)(fa[u + 1] * fb[u + 1]);
   }
-  return warp_sum(s0 + s1);
 }
-DLLM_DEV double warp_dot64(const float* __restrict__ a, const float* __restrict__ b, int H, int lane) {
+template <int UNR = 4, typename T>
+DLLM_DEV double warp_dot64(const T* __restrict__ a, const T* __restrict__ b, int H, int lane) {
+  constexpr int VE = 16 / sizeof(T);          // elements per 16-byte load
+  constexpr int CH = 8;                        // elements per lane per chunk
   double s0 = 0.0, s1 = 0.0;
-  for (int c = lane * 8; c < H; c += 256) {
-    float fa[8], fb[8];
-    load8(a + c, fa);
-    load8(b + c, fb);
+  for (int c0 = lane * CH; c0 < H; c0 += UNR * 32 * CH) {
+    uint4 ua[UNR][CH / VE], ub[UNR][CH / VE];
 #pragma unroll
-    for (int u = 0; u < 8; u += 2) {
-      s0 = fma((double)fa[u], (double)fb[u], s0);
-      s1 = fma((double)fa[u + 1], (double)fb[u + 1], s1);
+    for (int u = 0; u < UNR; ++u) {
+      const int c = c0 + u * 32 * CH;
+#pragma unroll
+      for (int v = 0; v < CH / VE; ++v) {
+        ua[u][v] = c < H ? *reinterpret_cast<const uint4*>(a + c + v * VE) : make_uint4(0, 0, 0, 0);
+        ub[u][v] = c < H ? *reinterpret_cast<const uint4*>(b + c + v * VE) : make_uint4(0, 0, 0, 0);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < UNR; ++u) {
+      if constexpr (sizeof(T) == 2) {
+        dot_chunk(ua[u][0], ub[u][0], s0, s1, a);
+      } else {
+#pragma unroll
+        for (int v = 0; v < CH / VE; ++v) {
+          const float fa[4] = {__uint_as_float(ua[u][v].x), __uint_as_float(ua[u][v].y), __uint_as_float(ua[u][v].z),
+                               __uint_as_float(ua[u][v].w)};
+          const float fb[4] = {__uint_as_float(ub[u][v].x), __uint_as_float(ub[u][v].y), __uint_as_float(ub[u][v].z),
+                               __uint_as_float(ub[u][v].w)};
+          s0 = fma((double)fa[0], (double)fb[0], s0);
+          s1 = fma((double)fa[1], (double)fb[1], s1);
+          s0 = fma((double)fa[2], (double)fb[2], s0);
+          s1 = fma((double)fa[3], (double)fb[3], s1);
+        }
+      }
     }
   }
   return warp_sum(s0 + s1);
@@ -236,7 +255,7 @@ DLLM_DEV void exact_redecide(const float* __restrict__ srow, const float* __rest
       const int b = __ffs(bal) - 1;
       bal &= bal - 1;
       const int eb = i * 32 + b;
-      const double dot = warp_dot64(hrow, w + (int64_t)eb * H, H, lane);
+      const double dot = warp_dot64<2>(hrow, w + (int64_t)eb * H, H, lane);
       if (lane == b) d[i] = 1.0 / (1.0 + exp(-dot)) + (double)bias[eb];
     }
   }
@@ -264,6 +283,95 @@ DLLM_DEV void exact_redecide(const float* __restrict__ srow, const float* __rest
     if (lane == j) { my_id = be; mine = sc; }
   }
   my_gate = (float)(mine / gsum);
+}
+
+// Cooperative exact re-decision of a CTA's near-tie tokens. The warps first list their flagged tokens; then, in
+// rounds of one flagged token per warp, (a) each warp lists its token's candidate experts (those whose fp32 biased
+// score is at least the token's threshold, at most 32 of them), (b) all warps of the CTA compute the candidates'
+// exact scores together (one warp per (token, expert) pair, so that a round costs about one dot product's latency),
+// (c) each warp ranks its token's candidates (lane j holds candidate j) into slots and gates. A token with more than
+// 32 candidates (only with many exactly tied scores) is decided by its warp alone (exact_redecide).
+constexpr int kMaxFlagged = 256;
+
+template <int NW>
+struct RedecideSmem {
+  int n_flag;
+  int ftok[kMaxFlagged];
+  float fthr[kMaxFlagged];
+  int cand_n[NW];
+  int cand_e[NW][32];
+  double cand_v[NW][32];
+};
+
+// Called by every thread of the CTA after each warp has appended its flagged tokens to rs (n_flag counted with
+// shared-memory atomics, then a barrier). out(t, lane, id, gate) writes lane's slot of token t.
+template <int PER, int NW, typename T, typename Out>
+DLLM_DEV void cta_redecide(RedecideSmem<NW>& rs, const float* __restrict__ scores, const float* __restrict__ bias,
+                           int E, int k, const T* __restrict__ h, const T* __restrict__ w, int H, Out out) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nf = min(rs.n_flag, kMaxFlagged);
+  for (int r0 = 0; r0 < nf; r0 += NW) {
+    const int f = r0 + warp;
+    if (f < nf) {   // (a) candidates of this warp's token
+      const int t = rs.ftok[f];
+      const float thr = rs.fthr[f];
+      const float* srow = scores + (int64_t)t * E;
+      int n = 0;
+#pragma unroll
+      for (int i = 0; i < PER; ++i) {
+        const int ex = i * 32 + lane;
+        const bool cand = ex < E && srow[ex] + bias[ex] >= thr;
+        const unsigned bal = __ballot_sync(0xffffffffu, cand);
+        const int slot = n + __popc(bal & ((1u << lane) - 1u));
+        if (cand && slot < 32) rs.cand_e[warp][slot] = ex;
+        n += __popc(bal);
+      }
+      if (lane == 0) rs.cand_n[warp] = n <= 32 ? n : -1;
+    } else if (lane == 0) {
+      rs.cand_n[warp] = 0;
+    }
+    __syncthreads();
+    // (b) every (token, candidate) pair of the round, one warp each
+    for (int p = warp; p < NW * 32; p += NW) {
+      const int ow = p >> 5, j = p & 31;
+      if (j >= rs.cand_n[ow]) continue;
+      const int t = rs.ftok[r0 + ow], e = rs.cand_e[ow][j];
+      const double dot = warp_dot64<NW >= 32 ? 2 : 4>(h + (int64_t)t * H, w + (int64_t)e * H, H, lane);
+      if (lane == 0) rs.cand_v[ow][j] = 1.0 / (1.0 + exp(-dot)) + (double)bias[e];
+    }
+    __syncthreads();
+    // (c) slots and gates of this warp's token
+    if (f < nf) {
+      const int t = rs.ftok[f], n = rs.cand_n[warp];
+      int my_id = 0;
+      float my_gate = 0.f;
+      if (n < 0) {
+        exact_redecide<PER>(scores + (int64_t)t * E, bias, E, k, h + (int64_t)t * H, w, H, rs.fthr[f], lane, my_id,
+                            my_gate);
+      } else {
+        double v = lane < n ? rs.cand_v[warp][lane] : -INFINITY;
+        const int e = lane < n ? rs.cand_e[warp][lane] : 0x7fffffff;
+        double gsum = 0.0, mine = 0.0;
+        for (int j = 0; j < k; ++j) {
+          double bv = v;
+          int be = e;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) {
+            const double ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+            if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
+          }
+          if (e == be) v = -INFINITY;
+          const double sc = bv - (double)bias[be];
+          gsum += sc;
+          if (lane == j) { my_id = be; mine = sc; }
+        }
+        my_gate = (float)(mine / gsum);
+      }
+      out(t, lane, my_id, my_gate);
+    }
+    __syncthreads();
+  }
 }
 
 // Many tokens: one warp per token, the fp32 selection. A token whose selection is a near-tie (see kRouteGuard) gets
@@ -310,19 +418,32 @@ __global__ void __launch_bounds__(1024) route_small_kernel(float* __restrict__ s
   int* off_s = rk_s + n;             // [E]
   __shared__ int wtot[32];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nw = blockDim.x >> 5;
+  __shared__ RedecideSmem<32> rd;
   for (int i = tid; i < W * E; i += blockDim.x) hist[i] = 0;
+  if (tid == 0) rd.n_flag = 0;
+  __syncthreads();
   for (int t = warp; t < Tk; t += nw) {
     int my_id;
     float my_gate, thr;
-    float* srow = scores + (int64_t)t * E;
-    if (warp_topk<PER>(srow, bias, E, k, from_logits, lane, my_id, my_gate, thr))
-      exact_redecide<PER>(srow, bias, E, k, h + (int64_t)t * H, w, H, thr, lane, my_id, my_gate);
+    if (warp_topk<PER>(scores + (int64_t)t * E, bias, E, k, from_logits, lane, my_id, my_gate, thr) && lane == 0) {
+      const int f = atomicAdd(&rd.n_flag, 1);   // Tk <= 32 <= kMaxFlagged
+      rd.ftok[f] = t;
+      rd.fthr[f] = thr;
+    }
     if (lane < k) {
       ids[(int64_t)t * k + lane] = my_id;
       gates[(int64_t)t * k + lane] = my_gate;
       ids_s[t * k + lane] = my_id;
     }
   }
+  __syncthreads();
+  cta_redecide<PER, 32>(rd, scores, bias, E, k, h, w, H, [&](int t, int ln, int id, float g) {
+    if (ln < k) {
+      ids[(int64_t)t * k + ln] = id;
+      gates[(int64_t)t * k + ln] = g;
+      ids_s[t * k + ln] = id;
+    }
+  });
   __syncthreads();
   for (int c = warp; c < W; c += nw) {
     const int a = c * 32 + lane;
@@ -402,16 +523,30 @@ __global__ void __launch_bounds__(256) route_seg_hist_kernel(int32_t* __restrict
   pdl_enter();
   if (live && *live == 0) return;   // a pass with no masked position left does nothing
   extern __shared__ int sh_hist[];
+  __shared__ RedecideSmem<8> rd;
   for (int i = threadIdx.x; i < E; i += blockDim.x) sh_hist[i] = 0;
+  if (threadIdx.x == 0) rd.n_flag = 0;
+  __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int t0 = blockIdx.x * seg_tok, t1 = min(Tk, t0 + seg_tok);
+  // the segment's near-tie tokens (fix_thr not NaN) into the list; past its capacity, a warp decides alone
   for (int tb = t0 + warp * 32; tb < t1; tb += 256) {
     const int t = tb + lane;
     const float th = t < t1 ? fix_thr[t] : __int_as_float(0x7fc00000);
-    unsigned bal = __ballot_sync(0xffffffffu, !isnan(th));
-    while (bal) {
-      const int j = __ffs(bal) - 1;
-      bal &= bal - 1;
+    const bool fl = !isnan(th);
+    const unsigned bal = __ballot_sync(0xffffffffu, fl);
+    int base = 0;
+    if (lane == 0 && bal) base = atomicAdd(&rd.n_flag, __popc(bal));
+    base = __shfl_sync(0xffffffffu, base, 0);
+    const int f = base + __popc(bal & ((1u << lane) - 1u));
+    if (fl && f < kMaxFlagged) {
+      rd.ftok[f] = t;
+      rd.fthr[f] = th;
+    }
+    unsigned over = __ballot_sync(0xffffffffu, fl && f >= kMaxFlagged);
+    while (over) {
+      const int j = __ffs(over) - 1;
+      over &= over - 1;
       const int tt = tb + j;
       int my_id;
       float my_gate;
@@ -423,6 +558,13 @@ __global__ void __launch_bounds__(256) route_seg_hist_kernel(int32_t* __restrict
       }
     }
   }
+  __syncthreads();
+  cta_redecide<PER, 8>(rd, scores, bias, E, k, h, w, H, [&](int t, int ln, int id, float g) {
+    if (ln < k) {
+      ids[(int64_t)t * k + ln] = id;
+      gates[(int64_t)t * k + ln] = g;
+    }
+  });
   __syncthreads();   // the re-decided ids (global writes of this CTA) are visible to the whole CTA
   const int a0 = t0 * k, a1 = t1 * k;
   for (int a = a0 + threadIdx.x; a < a1; a += blockDim.x) atomicAdd(&sh_hist[ids[a]], 1);

@@ -254,7 +254,8 @@ __global__ void __launch_bounds__(256, reg_min_blocks<VPT>()) unmask_reduce_bf16
 __global__ void __launch_bounds__(1024) unmask_select_kernel(Partial* part, int n_chunks, const int32_t* __restrict__ row_pos,
                                      const int32_t* __restrict__ n_rows, int max_rows, int B, int L, int t, int T_s, int mode,
                                      float tau, int k_max, int cfg, int vocab_offset, int32_t* tokens, uint8_t* mask,
-                                     int32_t* sel, int32_t* nsel, float* conf, int32_t* remaining) {
+                                     int32_t* sel, int32_t* nsel, float* conf, int32_t* remaining,
+                                     cudaGraphConditionalHandle cond, int set_cond) {
   pdl_enter();
   __shared__ int rem_w[32];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
@@ -355,6 +356,8 @@ __global__ void __launch_bounds__(1024) unmask_select_kernel(Partial* part, int 
     int s2 = 0;
     for (int i = 0; i < nw; ++i) s2 += rem_w[i];
     *remaining = s2;
+    // inside a block graph: the next pass runs only while masked positions are left
+    if (set_cond) cudaGraphSetConditional(cond, s2 > 0 ? 1u : 0u);
   }
 }
 
@@ -401,7 +404,8 @@ int launch_unmask(const UnmaskArgs& a, cudaStream_t s) {
   const int threads = a.n_chunks > kMergeSerial ? 1024 : 32 * min(32, max(1, a.B));
   launch_pdl(unmask_select_kernel, 1, threads, 0, s, static_cast<Partial*>(a.partials), a.n_chunks, a.row_pos, a.n_rows,
                                              a.max_rows, a.B, a.L, a.t, a.T_s, a.mode, a.tau, a.k_max, a.cfg, a.vocab_offset,
-                                             a.tokens, a.mask, a.sel, a.nsel, a.conf, a.remaining);
+                                             a.tokens, a.mask, a.sel, a.nsel, a.conf, a.remaining, a.cond,
+                                             a.set_cond);
   DLLM_CHECK_LAUNCH("unmask_select_kernel");
   return DLLM_OK;
 }

@@ -42,9 +42,14 @@ class DenoiseEngine:
                 setattr(L, name, bd.ptr(lw[name]))
             L.k_cache, L.v_cache = bd.ptr(kc), bd.ptr(vc)
             L.k_thin, L.v_thin, L.keep_pos = bd.ptr(kt), bd.ptr(vt), bd.ptr(kp)
+            if w.wfmt == "fp8":
+                for name in ("w_gu", "w_down", "w_gu_shared", "w_down_shared"):
+                    setattr(L, name + "_scale", bd.ptr(lw[name + "_scale"]))
+        fp8 = w.wfmt == "fp8"
         self.model = bd.Model(n, w.H, w.Hq, w.Hkv, w.d, w.E, w.k, w.I, w.V, self.dtype, w.eps, w.rope_base,
                               w.mask_id, bd.ptr(weights["embed"]), bd.ptr(weights["final_norm"]),
-                              bd.ptr(weights["w_lm"]), self._layers)
+                              bd.ptr(weights["w_lm"]), self._layers, bd.WEIGHTS_FP8 if fp8 else bd.WEIGHTS_BF16,
+                              bd.ptr(weights["w_lm_scale"]) if fp8 else None)
         self.tokens = torch.zeros((w.B, w.L), dtype=torch.int32, device=device)
         self.mask = torch.ones((w.B, w.L), dtype=torch.uint8, device=device)
         self.state = bd.State(w.B, w.L, w.P, self.cap, self.cap_thin, bd.ptr(self.tokens), bd.ptr(self.mask))
@@ -106,6 +111,12 @@ class DenoiseEngine:
             self.decode_block(torch.cuda.current_stream())
         return g
 
+    def block_graph(self, capture_stream=None):
+        """The library's block graph (dllm_block_graph_create): the T_s passes, each run only while the block has
+        masked positions, and the commit pass, captured once on a side stream. Warm the library's one-time set-up
+        (one decode_block) before the first call."""
+        return BlockGraph(self, capture_stream or torch.cuda.Stream(self.device))
+
     def views(self, t=0):
         p = self.params(t)
         v = bd.StepViews()
@@ -134,6 +145,27 @@ class DenoiseEngine:
         w = self.w
         v = self.views()
         return _device_view(v.x_final, w.Tk * w.H, torch_dtype(w.dtype), self.ws.buf).reshape(w.Tk, w.H)
+
+
+class BlockGraph:
+    """Owner of a dllm_block_graph handle (destroyed with the object)."""
+
+    def __init__(self, eng, capture_stream):
+        self.lib = eng.lib
+        self.eng = eng                     # keeps the tensors the graph's kernels address alive
+        self.handle = C.c_void_p()
+        p = eng.params(0)
+        bd.check(self.lib.dllm_block_graph_create(C.byref(eng.model), C.byref(eng.state), C.byref(p), eng.ws.addr,
+                                                  eng.ws.nbytes, bd.stream_handle(capture_stream),
+                                                  C.byref(self.handle)))
+
+    def launch(self, stream=None):
+        return bd.check(self.lib.dllm_block_graph_launch(self.handle, bd.stream_handle(stream)))
+
+    def __del__(self):
+        if getattr(self, "handle", None) and self.handle.value:
+            self.lib.dllm_block_graph_destroy(self.handle)
+            self.handle = C.c_void_p()
 
 
 def _device_view(addr, numel, dtype, owner):

@@ -56,8 +56,26 @@ def randint(shape, lo, hi, seed, tag, device="cpu"):
     return torch.randint(lo, hi, tuple(shape), generator=g, device=device, dtype=torch.int64).to(torch.int32)
 
 
+def fp8_rows(wb, chunk_rows=16384):
+    """An FP8 checkpoint of the bf16 matrix wb [..., M, K]: E4M3 codes (uint8) and one fp32 scale per row,
+    scale = max |row| / 448 (1 for an all-zero row), codes = round-to-nearest E4M3 of row / scale (torch's
+    float8_e4m3fn conversion), row by row in chunks."""
+    shape = wb.shape
+    flat = wb.reshape(-1, shape[-1])
+    codes = torch.empty(flat.shape, dtype=torch.uint8, device=wb.device)
+    scale = torch.empty(flat.shape[0], dtype=torch.float32, device=wb.device)
+    for r0 in range(0, flat.shape[0], chunk_rows):
+        f = flat[r0: r0 + chunk_rows].float()
+        amax = f.abs().amax(dim=1)
+        sc = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
+        codes[r0: r0 + chunk_rows] = (f / sc[:, None]).to(torch.float8_e4m3fn).view(torch.uint8)
+        scale[r0: r0 + chunk_rows] = sc
+    return codes.reshape(shape), scale.reshape(shape[:-1])
+
+
 def make_weights(w: Workload, device="cpu", seed=None, random_gains=False):
-    """All backbone weights of workload ``w``. Returns a dict of tensors on ``device``."""
+    """All backbone weights of workload ``w``. Returns a dict of tensors on ``device``. With w.wfmt == "fp8" the
+    expert and LM-head weights are replaced by their FP8 checkpoint (E4M3 codes, plus "<name>_scale" row scales)."""
     s = w.seed if seed is None else seed
     dt = torch_dtype(w.dtype)
     H, Hq, Hkv, d, E, I, V = w.H, w.Hq, w.Hkv, w.d, w.E, w.I, w.V
@@ -88,6 +106,11 @@ def make_weights(w: Workload, device="cpu", seed=None, random_gains=False):
             "w_gu_shared": normal((2 * I, H), w.w_std, s, p + "w_gu_shared", device, dt),
             "w_down_shared": normal((H, I), w.w_std, s, p + "w_down_shared", device, dt),
         })
+    if w.wfmt == "fp8":
+        wt["w_lm"], wt["w_lm_scale"] = fp8_rows(wt["w_lm"])
+        for lw in wt["layers"]:
+            for name in ("w_gu", "w_down", "w_gu_shared", "w_down_shared"):
+                lw[name], lw[name + "_scale"] = fp8_rows(lw[name])
     return wt
 
 

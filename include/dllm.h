@@ -74,12 +74,25 @@ DLLM_API int dllm_status_check(void* ws, cudaStream_t stream);
  * the word). No GPU state is left behind. */
 DLLM_API int dllm_selftest_bounded_wait(void* ws, size_t ws_bytes, cudaStream_t stream);
 
+/* ---------------------------------------------------------------------------------------------- weights */
+/*
+ * FP8 weights (the FP8 checkpoint of the card news "FP8 추론" and the HF-mirror README's FP8 version; the pages give
+ * no format): a matrix W [M, K] is stored as M x K E4M3 codes (OCP 8-bit float without infinities, one byte each,
+ * row-major) plus one fp32 scale per row, W[m, k] = value(code[m, k]) * scale[m]. Products with FP8 weights are
+ * scale[m] * sum_k x[k] value(code[m, k]) accumulated in fp32 (the codes' values are exact in bf16). Only the large
+ * matrices take this form: the routed and shared experts and the LM head.
+ */
+#define DLLM_WEIGHTS_BF16 0 /* weights in the storage type */
+#define DLLM_WEIGHTS_FP8 1  /* experts and LM head as E4M3 codes with per-row fp32 scales */
+
 /* ---------------------------------------------------------------------------------------------- dense GEMM */
 /*
  * Y[n, m] = sum_k X[n, k] * W[m, k] for n < N, m < M: the projection primitive of the backbone (QKV, output
  * projection, LM head). X [N, K], W [M, K], Y [N, M] with row stride ldy elements; Y has the storage type
  * (or fp32 when y_f32 != 0). bf16 path: K % 64 == 0, M % 128 == 0. If residual != 0, Y = Y_in + X W^T
  * (in place, rounded once). n_rows_dev (nullable) overrides N with a device-resident count <= N.
+ * w_fp8 != 0: W holds E4M3 codes and w_scale [M] their row scales (bf16 storage only, no residual); otherwise
+ * w_scale is ignored (may be NULL).
  */
 typedef struct {
   int32_t N, M, K;
@@ -87,9 +100,10 @@ typedef struct {
   int32_t dtype;
   int32_t y_f32;
   int32_t residual;
+  int32_t w_fp8;
 } dllm_gemm_desc;
-DLLM_API int dllm_gemm(const dllm_gemm_desc* desc, const void* x, const void* w, void* y, const int32_t* n_rows_dev,
-              void* ws, size_t ws_bytes, cudaStream_t stream);
+DLLM_API int dllm_gemm(const dllm_gemm_desc* desc, const void* x, const void* w, const float* w_scale, void* y,
+                       const int32_t* n_rows_dev, void* ws, size_t ws_bytes, cudaStream_t stream);
 DLLM_API size_t dllm_gemm_workspace_size(const dllm_gemm_desc* desc);
 
 /*
@@ -101,6 +115,7 @@ DLLM_API size_t dllm_gemm_workspace_size(const dllm_gemm_desc* desc);
  * storage type. X [rows, K]; Y [rows, M] in the storage type (fp32 when y_f32 != 0, not with swiglu); rows of X in
  * no group are not written. counts, offsets: [G] int32 device arrays (groups may not overlap). max_rows_hint: the
  * typical group size (chooses the tile width). bf16 only: K % 64 == 0, M % 128 == 0 (swiglu: M % 64 == 0).
+ * w_fp8 != 0: W and w_extra hold E4M3 codes, w_scale [G, M'] and w_extra_scale [M'] their row scales.
  */
 typedef struct {
   int32_t G, rows, K, M;
@@ -109,10 +124,11 @@ typedef struct {
   int32_t max_rows_hint;
   int32_t dtype;
   int32_t y_f32;
+  int32_t w_fp8;
 } dllm_grouped_gemm_desc;
 DLLM_API int dllm_grouped_gemm(const dllm_grouped_gemm_desc* desc, const void* x, const void* w, const void* w_extra,
-                               const int32_t* counts, const int32_t* offsets, void* y, void* ws, size_t ws_bytes,
-                               cudaStream_t stream);
+                               const float* w_scale, const float* w_extra_scale, const int32_t* counts,
+                               const int32_t* offsets, void* y, void* ws, size_t ws_bytes, cudaStream_t stream);
 DLLM_API size_t dllm_grouped_gemm_workspace_size(const dllm_grouped_gemm_desc* desc);
 
 /* ---------------------------------------------------------------------------------------------- B1 attention */
@@ -198,15 +214,19 @@ DLLM_API size_t dllm_moe_route_workspace_size(const dllm_route_desc* desc);
  *   w_down_shared [H, I] (both NULL: no shared expert); counts/offsets/perm/inv/gates as produced by
  *   dllm_moe_route; x_inout [Tk, H].
  * bf16: H % 128 == 0, I % 64 == 0.
+ * w_fp8 != 0: the four weights hold E4M3 codes with row scales w_gu_scale [E, 2I], w_down_scale [E, H],
+ * w_gu_shared_scale [2I], w_down_shared_scale [H] (NULL without a shared expert).
  */
 typedef struct {
   int32_t Tk, H, E, k, I;
   int32_t dtype;
+  int32_t w_fp8;
 } dllm_expert_desc;
 DLLM_API int dllm_moe_experts(const dllm_expert_desc* desc, const void* h, const void* w_gu, const void* w_down,
-                     const void* w_gu_shared, const void* w_down_shared, const int32_t* counts,
-                     const int32_t* offsets, const int32_t* perm, const int32_t* inv, const float* gates,
-                     void* x_inout, void* ws, size_t ws_bytes, cudaStream_t stream);
+                     const void* w_gu_shared, const void* w_down_shared, const float* w_gu_scale,
+                     const float* w_down_scale, const float* w_gu_shared_scale, const float* w_down_shared_scale,
+                     const int32_t* counts, const int32_t* offsets, const int32_t* perm, const int32_t* inv,
+                     const float* gates, void* x_inout, void* ws, size_t ws_bytes, cudaStream_t stream);
 DLLM_API size_t dllm_moe_experts_workspace_size(const dllm_expert_desc* desc);
 
 /* ---------------------------------------------------------------------------------------------- B5 unmask */
@@ -277,6 +297,12 @@ typedef struct {
   void* k_thin;              /* [B, Hkv, cap_thin, d] SPRINT-thinned cache (NULL without SPRINT) */
   void* v_thin;
   int32_t* keep_pos;         /* [B, cap_thin] positions of the thinned rows (NULL without SPRINT) */
+  /* row scales of the expert weights when the model's weight_format is DLLM_WEIGHTS_FP8 (the weights above then
+     hold E4M3 codes), else NULL */
+  const float* w_gu_scale;          /* [E, 2I] */
+  const float* w_down_scale;        /* [E, H] */
+  const float* w_gu_shared_scale;   /* [2I] */
+  const float* w_down_shared_scale; /* [H] */
 } dllm_layer;
 
 typedef struct {
@@ -289,6 +315,8 @@ typedef struct {
   const void* final_norm; /* [H] */
   const void* w_lm;       /* [V, H] */
   const dllm_layer* layers; /* host array of n_layers */
+  int32_t weight_format;    /* DLLM_WEIGHTS_BF16, or DLLM_WEIGHTS_FP8 (bf16 storage only): experts and w_lm as E4M3 codes */
+  const float* w_lm_scale;  /* [V] row scales of w_lm with DLLM_WEIGHTS_FP8, else NULL */
 } dllm_model;
 
 /* Decoding state of one block (device pointers except the sizes). */
@@ -341,6 +369,25 @@ DLLM_API int dllm_denoise_step(const dllm_model* model, const dllm_state* state,
                       size_t ws_bytes, cudaStream_t stream);
 DLLM_API size_t dllm_denoise_step_workspace_size(const dllm_model* model, const dllm_state* state,
                                         const dllm_step_params* params);
+
+/*
+ * A whole block as one CUDA graph: the T_s denoising passes (t = 0 .. T_s - 1, SPRINT selection at t = 0 when
+ * params->sprint) and the commit pass, every pass inside a conditional node that runs it only while the block still
+ * has masked positions (the unmasking of each pass sets the condition on the device), so the passes after a
+ * threshold-mode block finished are not launched at all. The passes are those dllm_denoise_step would run with the
+ * same arguments (params is the template: t, retain and commit are set per pass; it must describe a denoising
+ * pass). The graph is captured on capture_stream (a created stream, not capturing, not the legacy default stream),
+ * once; its kernels read the state, caches and outputs at the addresses given here on every launch, so the caller
+ * refills tokens / mask and launches it again for the next block of the same shapes. Host memory only: the library
+ * allocates no device memory (instantiating the graph may reserve driver resources). Destroy with
+ * dllm_block_graph_destroy.
+ */
+typedef struct dllm_block_graph dllm_block_graph;
+DLLM_API int dllm_block_graph_create(const dllm_model* model, const dllm_state* state, const dllm_step_params* params,
+                                     void* ws, size_t ws_bytes, cudaStream_t capture_stream,
+                                     dllm_block_graph** out /* host */);
+DLLM_API int dllm_block_graph_launch(const dllm_block_graph* graph, cudaStream_t stream);
+DLLM_API void dllm_block_graph_destroy(dllm_block_graph* graph);
 
 /* Device addresses, inside a step workspace, of intermediate results of the last dllm_denoise_step that used it
  * (read-only views for inspection; valid until the workspace is reused). */

@@ -48,24 +48,28 @@ FAKE = 0x10000  # never dereferenced: every call below fails validation first
 
 
 def test_gemm_rejects_bad_arguments(lib):
-    d = bd.GemmDesc(32, 128, 64, 128, bd.BF16, 0, 0)
-    assert lib.dllm_gemm(C.byref(d), None, FAKE, FAKE, None, FAKE, 1 << 20, None) == bd.ERR_INVALID_ARG
+    d = bd.GemmDesc(32, 128, 64, 128, bd.BF16, 0, 0, 0)
+    assert lib.dllm_gemm(C.byref(d), None, FAKE, None, FAKE, None, FAKE, 1 << 20, None) == bd.ERR_INVALID_ARG
     d.K = 0
-    assert lib.dllm_gemm(C.byref(d), FAKE, FAKE, FAKE, None, FAKE, 1 << 20, None) == bd.ERR_SHAPE
+    assert lib.dllm_gemm(C.byref(d), FAKE, FAKE, None, FAKE, None, FAKE, 1 << 20, None) == bd.ERR_SHAPE
     d.K = 64
-    assert lib.dllm_gemm(C.byref(d), FAKE, FAKE, FAKE, None, None, 1 << 20, None) == bd.ERR_WORKSPACE
-    assert lib.dllm_gemm(C.byref(d), FAKE, FAKE, FAKE, None, FAKE + 8, 1 << 20, None) == bd.ERR_WORKSPACE
-    assert lib.dllm_gemm(C.byref(d), FAKE, FAKE, FAKE, None, FAKE, 16, None) == bd.ERR_WORKSPACE
+    assert lib.dllm_gemm(C.byref(d), FAKE, FAKE, None, FAKE, None, None, 1 << 20, None) == bd.ERR_WORKSPACE
+    assert lib.dllm_gemm(C.byref(d), FAKE, FAKE, None, FAKE, None, FAKE + 8, 1 << 20, None) == bd.ERR_WORKSPACE
+    assert lib.dllm_gemm(C.byref(d), FAKE, FAKE, None, FAKE, None, FAKE, 16, None) == bd.ERR_WORKSPACE
     d.K = 96
-    assert lib.dllm_gemm(C.byref(d), FAKE, FAKE, FAKE, None, FAKE, 1 << 20, None) == bd.ERR_UNSUPPORTED
+    assert lib.dllm_gemm(C.byref(d), FAKE, FAKE, None, FAKE, None, FAKE, 1 << 20, None) == bd.ERR_UNSUPPORTED
     d.K = 64
-    assert lib.dllm_gemm(C.byref(d), FAKE + 2, FAKE, FAKE, None, FAKE, 1 << 20, None) == bd.ERR_ALIGN
+    assert lib.dllm_gemm(C.byref(d), FAKE + 2, FAKE, None, FAKE, None, FAKE, 1 << 20, None) == bd.ERR_ALIGN
     assert "aligned" in lib.dllm_last_error().decode()
     # the epilogue stores 16-byte vectors: Y's base and row stride must allow them
-    assert lib.dllm_gemm(C.byref(d), FAKE, FAKE, FAKE + 4, None, FAKE, 1 << 20, None) == bd.ERR_ALIGN
+    assert lib.dllm_gemm(C.byref(d), FAKE, FAKE, None, FAKE + 4, None, FAKE, 1 << 20, None) == bd.ERR_ALIGN
     d.ldy = 132
-    assert lib.dllm_gemm(C.byref(d), FAKE, FAKE, FAKE, None, FAKE, 1 << 20, None) == bd.ERR_ALIGN
+    assert lib.dllm_gemm(C.byref(d), FAKE, FAKE, None, FAKE, None, FAKE, 1 << 20, None) == bd.ERR_ALIGN
     assert "ldy" in lib.dllm_last_error().decode()
+    d.ldy, d.w_fp8 = 128, 1             # FP8 weights without their row scales
+    assert lib.dllm_gemm(C.byref(d), FAKE, FAKE, None, FAKE, None, FAKE, 1 << 20, None) == bd.ERR_INVALID_ARG
+    d.residual = 1
+    assert lib.dllm_gemm(C.byref(d), FAKE, FAKE, FAKE, FAKE, None, FAKE, 1 << 20, None) == bd.ERR_UNSUPPORTED
 
 
 def test_attention_rejects_bad_arguments(lib):
@@ -86,17 +90,22 @@ def test_route_and_experts_reject_bad_arguments(lib):
     assert lib.dllm_moe_route(C.byref(r), *args, None, FAKE, 1 << 30, None) == bd.ERR_UNSUPPORTED
     r.E, r.k = 256, 300
     assert lib.dllm_moe_route(C.byref(r), *args, None, FAKE, 1 << 30, None) == bd.ERR_UNSUPPORTED
-    e = bd.ExpertDesc(32, 2048, 256, 8, 512, bd.BF16)
+    e = bd.ExpertDesc(32, 2048, 256, 8, 512, bd.BF16, 0)
+    no_scales = [None] * 4
     # one shared weight without the other
-    assert lib.dllm_moe_experts(C.byref(e), FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
-                                FAKE, 1 << 30, None) == bd.ERR_INVALID_ARG
+    assert lib.dllm_moe_experts(C.byref(e), FAKE, FAKE, FAKE, FAKE, None, *no_scales, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                FAKE, FAKE, 1 << 30, None) == bd.ERR_INVALID_ARG
     e.I = 500
-    assert lib.dllm_moe_experts(C.byref(e), *([FAKE] * 11), FAKE, 1 << 30, None) == bd.ERR_UNSUPPORTED
+    assert lib.dllm_moe_experts(C.byref(e), *([FAKE] * 5), *no_scales, *([FAKE] * 6), FAKE, 1 << 30,
+                                None) == bd.ERR_UNSUPPORTED
+    e.I, e.w_fp8 = 512, 1                # FP8 expert weights without their row scales
+    assert lib.dllm_moe_experts(C.byref(e), *([FAKE] * 5), *no_scales, *([FAKE] * 6), FAKE, 1 << 30,
+                                None) == bd.ERR_INVALID_ARG
 
 
 def test_grouped_gemm_rejects_bad_arguments(lib):
-    d = bd.GroupedGemmDesc(8, 64, 256, 128, 0, 0, 0, bd.BF16, 0)
-    args = [FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, 1 << 20, None]
+    d = bd.GroupedGemmDesc(8, 64, 256, 128, 0, 0, 0, bd.BF16, 0, 0)
+    args = [FAKE, FAKE, None, None, None, FAKE, FAKE, FAKE, FAKE, 1 << 20, None]
     d.K = 100
     assert lib.dllm_grouped_gemm(C.byref(d), *args) == bd.ERR_UNSUPPORTED
     d.K, d.extra_rows = 256, 8          # an extra group without its weight
@@ -105,6 +114,8 @@ def test_grouped_gemm_rejects_bad_arguments(lib):
     assert lib.dllm_grouped_gemm(C.byref(d), *args) == bd.ERR_UNSUPPORTED
     d.swiglu, d.y_f32, d.dtype = 0, 0, bd.F32
     assert lib.dllm_grouped_gemm(C.byref(d), *args) == bd.ERR_UNSUPPORTED
+    d.dtype, d.w_fp8 = bd.BF16, 1        # FP8 weights without their row scales
+    assert lib.dllm_grouped_gemm(C.byref(d), *args) == bd.ERR_INVALID_ARG
 
 
 def test_route_workspace_covers_scores_and_permutation_segments(lib):

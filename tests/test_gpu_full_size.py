@@ -256,3 +256,91 @@ def test_full_denoise_pass_properties(w):
     assert int(eng.mask.sum().item()) == 0
     assert bd.status_check(eng.ws) == bd.OK
     del eng, wt, caches
+
+
+# ------------------------------------------------------------------------------------------------ prefill shape
+# The compute-bound shape on which the tensor-core fractions are measured: 8 rows x 4096 tokens under the
+# block-causal mask (one layer of the thinking-mode prompt's prefill).
+
+def test_prefill_attention_block_causal():
+    """dllm_block_attn at 8 x 4096 queries over their own 4096 keys with 32-token blocks (tensor-core path, key
+    splits), compared with the oracle's two-pass masked softmax on sampled queries of every row (early, middle and
+    last blocks) in every head."""
+    w = PREFILL
+    B, Lq, Hq, Hkv, d, blk = w.B, w.L, w.Hq, w.Hkv, w.d, 32
+    q = synth.normal((B, Lq, Hq, d), 1.0, 30, "pa_q", DEV)
+    kc = synth.normal((B, Hkv, Lq, d), 1.0, 30, "pa_k", DEV)
+    vc = synth.normal((B, Hkv, Lq, d), 1.0, 30, "pa_v", DEV)
+    out = torch.full((B, Lq, Hq * d), float("nan"), dtype=torch.bfloat16, device=DEV)
+    bd.block_attn(q, kc, vc, out, B, Lq, Hq, Hkv, d, blk, 0, Lq, Lq, bd.BF16)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out.float()).all()
+    g = np.random.default_rng(30)
+    for b in range(B):
+        qi = np.unique(np.concatenate([[0, 31, 32, Lq - 1], g.integers(0, Lq, 6)]))
+        kk = to64(kc[b]).transpose(1, 0, 2)
+        vv = to64(vc[b]).transpose(1, 0, 2)
+        want = O.store(O.attention(to64(q[b, qi]), kk, vv, qi, np.arange(Lq), blk), "bf16")
+        got = to64(out[b, qi]).reshape(len(qi), Hq, d)
+        assert_close(got, want, "bf16", f"prefill attention row {b}")
+
+
+def test_prefill_router_and_experts():
+    """The MoE FFN at the prefill shape's 32768 tokens: router output (ids, gates, permutation of 262144
+    assignments) fed to dllm_moe_experts (CTA-pair grouped GEMMs with ~1024 rows per expert), compared with the
+    oracle's per-token expert mixture on 24 sampled tokens."""
+    w = PREFILL
+    Tk, H, E, k, I = w.Tk, w.H, w.E, w.k, w.I
+    h = synth.normal((Tk, H), 1.0, 31, "pe_h", DEV)
+    x0 = synth.normal((Tk, H), 1.0, 31, "pe_x", DEV)
+    wr = synth.normal((E, H), 0.02, 31, "pe_r", DEV)
+    bias = synth.uniform((E,), -0.1, 0.1, 31, "pe_b", DEV)
+    wgu = synth.normal((E, 2 * I, H), 0.02, 31, "pe_gu", DEV, chunk_rows=16)
+    wd = synth.normal((E, H, I), 0.02, 31, "pe_d", DEV, chunk_rows=16)
+    sgu = synth.normal((2 * I, H), 0.02, 31, "pe_sgu", DEV)
+    sd = synth.normal((H, I), 0.02, 31, "pe_sd", DEV)
+    ids = torch.empty((Tk, k), dtype=torch.int32, device=DEV)
+    gates = torch.empty((Tk, k), dtype=torch.float32, device=DEV)
+    counts = torch.empty(E, dtype=torch.int32, device=DEV)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=DEV)
+    perm = torch.empty(Tk * k, dtype=torch.int32, device=DEV)
+    inv = torch.empty(Tk * k, dtype=torch.int32, device=DEV)
+    bd.moe_route(h, wr, bias, ids, gates, counts, offsets, perm, inv, Tk, H, E, k, bd.BF16)
+    x = x0.clone()
+    bd.moe_experts(h, wgu, wd, sgu, sd, counts, offsets, perm, inv, gates, x, Tk, H, E, k, I, bd.BF16)
+    torch.cuda.synchronize()
+    assert int(counts.max().item()) > 512            # groups span several 256-row pair tiles
+    rows = np.random.default_rng(31).choice(Tk, 24, replace=False)
+    g_ids, g_gates = ids.cpu().numpy()[rows], gates.cpu().numpy()[rows].astype(np.float64)
+    delta = O.moe_delta(to64(h[rows]), g_ids, g_gates, wgu, wd, sgu, sd, "bf16")
+    want = O.store(to64(x0[rows]) + delta, "bf16")
+    assert_close(to64(x[rows]), want, "bf16", "prefill experts (sampled tokens)")
+
+
+def test_step_at_prefill_row_count():
+    """One denoising pass over 1024 rows x 32 tokens (32768 token rows, as many as the prefill shape) of a layer of
+    the full width: the QKV projection with RoPE and cache writes, the output projection and both expert GEMMs
+    run as CTA pairs at this row count, the router takes its many-token path. Batch rows are independent, so the
+    oracle runs the layer for three sampled rows alone and the hidden states after the layer are compared there."""
+    from block_diffusion_moe_dllm_b200.configs import ONE_LAYER, scaled
+    w = scaled(ONE_LAYER, name="prefill-rows", B=1024, P=32, L=32, V=1024, T_s=8)
+    wt = synth.make_weights(w, DEV, seed=32, random_gains=True)
+    caches = synth.make_prefix_cache(w, DEV, seed=32)
+    tokens, mask = synth.make_block_state(w, DEV, seed=32, masked_fraction=0.5)
+    eng = DenoiseEngine(w, wt, caches, DEV)
+    eng.set_block(tokens, mask)
+    eng.step(1)
+    torch.cuda.synchronize()
+    assert bd.status_check(eng.ws) == bd.OK
+    x = to64(eng.x_final()).reshape(w.B, w.L, w.H)
+    sample = [0, 517, 1023]
+    ws = scaled(w, B=len(sample))
+    cp = lambda t: t.detach().cpu()
+    hw = {"embed": cp(wt["embed"]), "final_norm": cp(wt["final_norm"]), "w_lm": cp(wt["w_lm"]),
+          "layers": [{kk: cp(v) for kk, v in lw.items()} for lw in wt["layers"]]}
+    hc = [(c[0][sample, :, : w.P].cpu(), c[1][sample, :, : w.P].cpu()) for c in caches]
+    f = O.forward_block(ws, hw, hc, tokens[sample].cpu().numpy(), mask[sample].cpu().numpy(), want_logits=False)
+    ok = f["route"][0][2] >= 3e-4     # tokens whose routing a one-ulp input difference cannot flip
+    assert ok.mean() > 0.5
+    assert_close(x[sample].reshape(-1, w.H)[ok], f["x"].reshape(-1, w.H)[ok], "bf16",
+                 "hidden state after the layer (sampled rows)", ulps=2)

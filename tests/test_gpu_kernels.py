@@ -195,6 +195,56 @@ def test_grouped_gemm(Tk, E, k, I, H, swiglu):
             assert np.all(np.abs(ys[r] - want) <= 1e-4 * np.maximum(1.0, np.abs(want))), "grouped GEMM rows"
 
 
+@pytest.mark.parametrize("Tk,E,k,I,H,swiglu", [(512, 256, 8, 512, 2048, 1), (512, 256, 8, 512, 2048, 0),
+                                                  (40, 16, 4, 128, 256, 1), (300, 8, 2, 128, 256, 0)])
+def test_grouped_gemm_fp8(Tk, E, k, I, H, swiglu):
+    """dllm_grouped_gemm with E4M3 weights and per-row scales (the FP8 checkpoint) against the oracle's products
+    with the dequantized weights, on sampled rows of every group (N tiles of 32, 64 and 128 rows)."""
+    ids, _ = random_assignments(Tk, E, k, seed=Tk + I + 1)
+    counts, offsets, perm, _ = assignment_tables(ids, E)
+    n = Tk * k + Tk
+    K, M = (H, I) if swiglu else (I, H)
+    Mw = 2 * M if swiglu else M
+    x = synth.normal((n, K), 1.0, 10, f"gf_x{K}", DEV)
+    wq, ws_ = synth.fp8_rows(synth.normal((E, Mw, K), 0.02, 10, f"gf_w{M}", DEV))
+    xq, xs = synth.fp8_rows(synth.normal((Mw, K), 0.02, 10, f"gf_s{M}", DEV))
+    y = torch.full((n, M), -3.0, dtype=torch.bfloat16 if swiglu else torch.float32, device=DEV)
+    cvt = lambda a: torch.from_numpy(a).to(DEV)
+    bd.grouped_gemm(x, wq, xq, cvt(counts), cvt(offsets[:-1].copy()), y, E, n, K, M, bd.BF16, swiglu=swiglu,
+                    extra_rows=Tk, max_rows_hint=max(32, 4 * (Tk * k // E)), y_f32=0 if swiglu else 1, w_scale=ws_,
+                    w_extra_scale=xs)
+    torch.cuda.synchronize()
+    xs64, ys = to64(x), to64(y)
+    g = np.random.default_rng(4)
+    groups = [(int(offsets[e]), int(counts[e]), e) for e in range(E) if counts[e] > 0] + [(Tk * k, Tk, -1)]
+    for off, cnt, e in groups:
+        q, sc = (xq, xs) if e < 0 else (wq[e], ws_[e])
+        we = O.dequant_rows(q.cpu().numpy(), sc.cpu().numpy())
+        r = np.unique(g.integers(off, off + cnt, min(cnt, 4)))
+        if swiglu:
+            want = O.store(O.silu(xs64[r] @ we[:M].T) * (xs64[r] @ we[M:].T), "bf16")
+            assert_close(ys[r], want, "bf16", "grouped SwiGLU rows (FP8 weights)")
+        else:
+            want = xs64[r] @ we.T
+            assert np.all(np.abs(ys[r] - want) <= 1e-4 * np.maximum(1.0, np.abs(want))), "grouped rows (FP8)"
+
+
+@pytest.mark.parametrize("N", [32, 200])
+def test_gemm_fp8_lm_head_shape(N):
+    """The dense projection with E4M3 weights (the LM head of the FP8 checkpoint, 16384 rows x 2048) for 32 and
+    200 token rows, against the dequantized product on sampled columns."""
+    M, K = 16384, 2048
+    x = synth.normal((N, K), 1.0, 11, "gfl_x", DEV)
+    wq, sc = synth.fp8_rows(synth.normal((M, K), 0.02, 11, "gfl_w", DEV))
+    y = torch.empty((N, M), dtype=torch.bfloat16, device=DEV)
+    bd.gemm(x, wq, y, N, M, K, bd.BF16, w_scale=sc)
+    torch.cuda.synchronize()
+    cols = np.random.default_rng(5).choice(M, 256, replace=False)
+    we = O.dequant_rows(wq[cols].cpu().numpy(), sc[cols].cpu().numpy())
+    want = O.store(to64(x) @ we.T, "bf16")
+    assert_close(to64(y)[:, cols], want, "bf16", "FP8 LM-head logits")
+
+
 # ------------------------------------------------------------------------------------------------ attention
 def _attn_case(dtype, B, Lq, Hq, Hkv, d, blk, q_pos0, n_keys, cap, key_pos=None, seed=0, nan_tail=False):
     t = _tdt(dtype)

@@ -40,10 +40,16 @@ def _setup(w, seed=0, masked_fraction=1.0, random_gains=True):
 
 
 def _host(wt):
-    """Host copies of the weights for the oracle (the same bytes the library reads)."""
+    """Host copies of the weights for the oracle (the same bytes the library reads); FP8 matrices (codes with a
+    "<name>_scale" entry) are handed over as their dequantized values (the oracle's E4M3 definition, exact)."""
     cp = lambda t: t.detach().cpu()
-    return {"embed": cp(wt["embed"]), "final_norm": cp(wt["final_norm"]), "w_lm": cp(wt["w_lm"]),
-            "layers": [{k: cp(v) for k, v in lw.items()} for lw in wt["layers"]]}
+
+    def conv(d, name):
+        if name + "_scale" in d:
+            return O.dequant_rows(cp(d[name]).numpy(), cp(d[name + "_scale"]).numpy())
+        return cp(d[name])
+    return {"embed": cp(wt["embed"]), "final_norm": cp(wt["final_norm"]), "w_lm": conv(wt, "w_lm"),
+            "layers": [{k: conv(lw, k) for k in lw if not k.endswith("_scale")} for lw in wt["layers"]]}
 
 
 def _host_caches(caches, P):
@@ -173,6 +179,30 @@ def test_step_small_bf16_sprint():
 def test_step_small_bf16_threshold():
     w = scaled(SMALL, mode=1, tau=0.9, k_max=8, T_s=16, lm_std=1.0)
     _one_pass(w, seed=5)
+
+
+# ------------------------------------------------------------------------------------------------ FP8 weights
+# The expert and LM-head weights as E4M3 codes with per-row scales (the FP8 checkpoint); the oracle runs the same
+# pass on the codes' exact values.
+
+def test_step_small_fp8_weights():
+    _one_pass(scaled(SMALL, name="small-fp8", wfmt="fp8"), seed=51)
+
+
+def test_step_small_fp8_weights_cfg_threshold():
+    w = scaled(SMALL, name="small-fp8-cfg", wfmt="fp8", B=2, cfg=1, cfg_scale=2.0, vocab_offset=1024 - 256,
+               vocab_len=256)
+    _one_pass(w, seed=52)
+
+
+def test_step_fp8_fused_confidence():
+    _one_pass(scaled(SMALL, name="small-fp8-fused", B=1, L=32, V=20480, wfmt="fp8"), seed=53, masked_fraction=0.6,
+              t=2)
+
+
+def test_step_fp8_cta_rows():
+    """512 token rows with 16 q / 4 kv heads through FP8 experts (N tiles of 64 and 128 rows: groups of ~60 rows)."""
+    _one_pass(scaled(SMALL, name="small-fp8-rows", wfmt="fp8", B=16, Hq=16, Hkv=4, P=64, L=32), seed=54)
 
 
 # One logical row of at most 32 positions, no guidance, and a scored vocabulary of at least 74 weight tiles of 128
@@ -356,3 +386,34 @@ def test_finished_pass_costs_only_its_launches():
     live, dead = timed(mask), timed(done)
     assert bd.status_check(eng.ws) == bd.OK
     assert dead < 0.5 * live, f"finished pass {dead * 1e3:.0f} us vs live pass {live * 1e3:.0f} us"
+
+
+@pytest.mark.parametrize("early", [False, True], ids=["fixed-schedule", "finishes-at-first-pass"])
+def test_block_graph_matches_host_driven_block(early):
+    """dllm_block_graph_create captures a block (T_s passes, each inside a conditional node that runs it only while
+    masked positions are left, then the commit pass). Launched from the same start it leaves the same tokens, mask,
+    caches and step outputs as the passes called one by one from the host, launched twice in a row."""
+    w = scaled(SMALL, name="small-bf16-graph", mode=1, tau=0.0, k_max=32, T_s=6) if early else SMALL
+    wt, caches, eng, _, _ = _setup(w, seed=43)
+    tokens0, mask0 = eng.tokens.clone(), eng.mask.clone()
+    caches0 = [(k.clone(), v.clone()) for k, v in caches]
+    eng.decode_block()                         # host-driven reference (also warms the library's set-up)
+    torch.cuda.synchronize()
+    want = _snapshot(eng, caches)
+    want_sel = (eng.sel.clone(), eng.nsel.clone(), eng.remaining.clone())
+    g = eng.block_graph()
+    for _ in range(2):
+        for (k, v), (k0, v0) in zip(caches, caches0):
+            k.copy_(k0)
+            v.copy_(v0)
+        eng.set_block(tokens0, mask0)
+        g.launch()
+        torch.cuda.synchronize()
+        assert bd.status_check(eng.ws) == bd.OK
+        assert torch.equal(eng.tokens, want[0]) and torch.equal(eng.mask, want[1])
+        for (k, v), (k1, v1) in zip(caches, want[2]):
+            assert torch.equal(k, k1) and torch.equal(v, v1)
+        if not early:     # with an early finish the graph skips passes whose step outputs the host loop rewrote
+            assert torch.equal(eng.sel, want_sel[0]) and torch.equal(eng.nsel, want_sel[1])
+        assert int(eng.remaining.item()) == 0 and int(eng.mask.sum().item()) == 0
+    del g

@@ -59,6 +59,7 @@ def bench_config(w, world):
     """The workload description both arms print (identical keys and values)."""
     return {"workload": w.name, "B": w.B, "L": w.L, "T_s": w.T_s, "P": w.P, "H": w.H, "Hq": w.Hq, "Hkv": w.Hkv,
             "d": w.d, "E": w.E, "k": w.k, "I": w.I, "V": w.V, "vocab_scored": w.vlen, "layers": w.n_layers,
+            "weights": "fp8 e4m3 experts + lm head, per-row fp32 scales" if w.wfmt == "fp8" else "bf16",
             "mode": "threshold" if w.mode else "fixed", "tau": w.tau if w.mode else None,
             "k_max": w.k_max if w.mode else None, "cfg": w.cfg_scale if w.cfg else None,
             "sprint_keep": w.keep_ratio if w.sprint else None,
@@ -230,14 +231,15 @@ def algorithmic_bytes(w, passes, commit_active):
     """Bytes a block must move at least once from HBM: every live pass reads each layer's attention and router
     weights, the weights of every expert it routed to plus the shared expert, the K/V it attends over, and the
     LM-head rows it scores; SPRINT re-reads the full prefix K and writes the thinned copies at the first pass; the
-    commit pass reads the layer weights again (the last layer without its FFN). Activations (a few MB) are left
-    out."""
+    commit pass reads the layer weights again (the last layer without its FFN). FP8 expert and LM-head weights
+    count one byte per weight plus their row scales. Activations (a few MB) are left out."""
     H, QD = w.H, w.Hq * w.d
+    wb = 1 if w.wfmt == "fp8" else 2            # FP8 checkpoint: one byte per expert / LM-head weight (+ row scales)
     attn_w = ((w.Hq + 2 * w.Hkv) * w.d * H + H * QD + w.E * H) * 2
-    expert_w = 3 * w.I * H * 2
+    expert_w = 3 * w.I * H * wb + ((2 * w.I + H) * 4 if wb == 1 else 0)   # gate/up and down row scales
     n_keys = (w.n_keep if w.sprint else w.P) + w.L
     kv = 2 * w.B * w.Hkv * n_keys * w.d * 2
-    head = w.vlen * H * 2
+    head = w.vlen * H * wb + (w.vlen * 4 if wb == 1 else 0)
     total = 0
     for p in passes:
         if not p["live"]:

@@ -46,6 +46,7 @@ struct Smem {
   uint64_t done;
   uint32_t tmem_base;
   int abort_flag;
+  int drained;                      // CTA pairs: the leader saw every issued stage of both CTAs land
   int n_groups;
   int total_tiles;
   int tile_prefix[MAX_GROUPS + 1];  // exclusive prefix of tiles per group
@@ -758,6 +759,7 @@ gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_con
   if (tid == 0) {
     sm.n_groups = n_groups;
     sm.abort_flag = 0;
+    sm.drained = 1;   // the leader overwrites the peer's copy at its end (before the final cluster barrier)
     for (int s = 0; s < STAGES; ++s) {
       tc::mbar_init(&sm.full[s], 1);
       tc::mbar_init(&sm.empty[s], 1);
@@ -868,12 +870,14 @@ gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_con
       }
       if (leader) {
         // every issued stage of both CTAs lands before the pair can leave (bounded); the peer passes the final
-        // cluster barrier only after this
+        // cluster barrier only after this and then reads whether it succeeded
         const uint32_t first = it > (uint32_t)STAGES ? it - STAGES : 0;
-        for (uint32_t i = first; i < it; ++i) tc::mbar_wait(&sm.full[i % STAGES], (i / STAGES) & 1, 1u << 20);
-      } else if (!ok) {
-        // the peer cannot observe its own copies after an abort: give any in flight time to land
-        for (int i = 0; i < 200; ++i) __nanosleep(1000);
+        bool landed = true;
+        for (uint32_t i = first; i < it; ++i)
+          landed = tc::mbar_wait(&sm.full[i % STAGES], (i / STAGES) & 1, 1u << 20) && landed;
+        // tell the peer (its own shared memory; visible to it after the final cluster barrier)
+        asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(tc::mapa_u32(tc::smem_u32(&sm.drained), 1)),
+                     "r"(landed ? 1 : 0) : "memory");
       }
     }
   } else if (warp == 1) {
@@ -944,6 +948,17 @@ gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_con
   // neither CTA leaves (nor frees TMEM) while its peer may still signal its barriers or read its shared memory
   __syncthreads();
   cluster_sync();
+  if (!leader && tid == 0) {
+    // the peer's copies complete on the leader's barriers, which the leader drained and reported here: if that
+    // drain gave up, copies into this CTA's shared memory may still be in flight. Report it and give them a
+    // bounded time to land.
+    const int drained = *reinterpret_cast<volatile int*>(&sm.drained);
+    if (!drained) {
+      if (p.status) atomicExch(p.status, ST_TIMEOUT_PRODUCER);
+      for (int i = 0; i < 1000; ++i) __nanosleep(1000);
+    }
+  }
+  __syncthreads();
   if (warp == 1) {
     tc::fence_after_sync();
     tc::tmem_dealloc_pair(sm.tmem_base, 2 * PAIR_BN);

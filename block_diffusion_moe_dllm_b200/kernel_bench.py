@@ -72,15 +72,26 @@ def _result(name, t, nbytes, extra=None):
     return r
 
 
+def wbytes(w: Workload):
+    """Bytes per element of the expert and LM-head weights (FP8 checkpoint: one, plus a 4-byte scale per row)."""
+    return 1 if w.wfmt == "fp8" else 2
+
+
 def bench_lm_head(w: Workload, reps, dev, stream, weights=None):
     rows = (2 if w.cfg else 1) * (w.B // (2 if w.cfg else 1)) * w.L
-    wl = (weights["w_lm"] if weights else synth.normal((w.V, w.H), w.lm_std, w.seed, "w_lm", dev, chunk_rows=16384))
+    if weights:
+        wl, sc = weights["w_lm"], weights.get("w_lm_scale")
+    else:
+        wl, sc = synth.normal((w.V, w.H), w.lm_std, w.seed, "w_lm", dev, chunk_rows=16384), None
+        if w.wfmt == "fp8":
+            wl, sc = synth.fp8_rows(wl)
     wl = wl[w.vocab_offset: w.vocab_offset + w.vlen]
+    sc = sc[w.vocab_offset: w.vocab_offset + w.vlen] if sc is not None else None
     x = synth.normal((rows, w.H), 1.0, 1, "kb_x", dev)
     y = torch.empty((rows, w.vlen), dtype=torch.bfloat16, device=dev)
     ws = bd.Workspace(1 << 16, dev)
-    t = timed(lambda: bd.gemm(x, wl, y, rows, w.vlen, w.H, bd.BF16, ws=ws), reps, stream)
-    nbytes = w.vlen * w.H * 2 + rows * w.H * 2 + rows * w.vlen * 2
+    t = timed(lambda: bd.gemm(x, wl, y, rows, w.vlen, w.H, bd.BF16, w_scale=sc, ws=ws), reps, stream)
+    nbytes = w.vlen * w.H * wbytes(w) + (w.vlen * 4 if sc is not None else 0) + rows * w.H * 2 + rows * w.vlen * 2
     return _result("gemm_tc_kernel[lm_head]", t, nbytes,
                    _flops({"rows": rows, "M": w.vlen, "K": w.H}, 2.0 * rows * w.vlen * w.H, t))
 
@@ -120,10 +131,13 @@ def bench_experts(w: Workload, reps, dev, stream, weights=None):
     torch.cuda.synchronize()
     active = int((counts > 0).sum().item())
     x = torch.zeros((rows, w.H), dtype=torch.bfloat16, device=dev)
+    scales = tuple(lw[n + "_scale"] for n in ("w_gu", "w_down", "w_gu_shared", "w_down_shared")) \
+        if "w_gu_scale" in lw else None
     t = timed(lambda: bd.moe_experts(h, lw["w_gu"], lw["w_down"], lw["w_gu_shared"], lw["w_down_shared"], counts,
-                                     offsets, perm, inv, gates, x, rows, w.H, w.E, w.k, w.I, bd.BF16, ws=ws),
+                                     offsets, perm, inv, gates, x, rows, w.H, w.E, w.k, w.I, bd.BF16, scales=scales,
+                                     ws=ws),
               reps, stream)
-    nbytes = (active + 1) * 3 * w.I * w.H * 2 + 2 * rows * w.H * 2
+    nbytes = (active + 1) * 3 * w.I * w.H * wbytes(w) + 2 * rows * w.H * 2
     troute = timed(lambda: bd.moe_route(h, lw["w_router"], lw["router_bias"], ids, gates, counts, offsets, perm, inv,
                                         rows, w.H, w.E, w.k, bd.BF16, ws=ws), reps, stream)
     rbytes = w.E * w.H * 2 + rows * w.H * 2
@@ -157,12 +171,16 @@ def bench_expert_gemms(w: Workload, reps, dev, stream, weights=None):
     xp = synth.normal((n, w.H), 1.0, 6, "kb_xp", dev)
     act = torch.empty((n, w.I), dtype=torch.bfloat16, device=dev)
     y = torch.empty((n, w.H), dtype=torch.float32, device=dev)
+    f8 = "w_gu_scale" in lw
+    sc = (lambda name: lw[name + "_scale"] if f8 else None)
     t1 = timed(lambda: bd.grouped_gemm(xp, lw["w_gu"], lw["w_gu_shared"], counts, offsets, act, w.E, n, w.H, w.I,
-                                       bd.BF16, swiglu=1, extra_rows=rows, max_rows_hint=hint, ws=ws), reps, stream)
+                                       bd.BF16, swiglu=1, extra_rows=rows, max_rows_hint=hint, w_scale=sc("w_gu"),
+                                       w_extra_scale=sc("w_gu_shared"), ws=ws), reps, stream)
     t2 = timed(lambda: bd.grouped_gemm(act, lw["w_down"], lw["w_down_shared"], counts, offsets, y, w.E, n, w.I, w.H,
-                                       bd.BF16, extra_rows=rows, max_rows_hint=hint, y_f32=1, ws=ws), reps, stream)
-    b1 = (active + 1) * 2 * w.I * w.H * 2 + n * w.H * 2 + n * w.I * 2
-    b2 = (active + 1) * w.H * w.I * 2 + n * w.I * 2 + n * w.H * 4
+                                       bd.BF16, extra_rows=rows, max_rows_hint=hint, y_f32=1, w_scale=sc("w_down"),
+                                       w_extra_scale=sc("w_down_shared"), ws=ws), reps, stream)
+    b1 = (active + 1) * 2 * w.I * w.H * wbytes(w) + n * w.H * 2 + n * w.I * 2
+    b2 = (active + 1) * w.H * w.I * wbytes(w) + n * w.I * 2 + n * w.H * 4
     f1, f2 = 2.0 * n * 2 * w.I * w.H, 2.0 * n * w.H * w.I
     return [_result("gemm_tc_kernel[experts_swiglu]", t1, b1, _flops({"active_experts": active, "rows": n}, f1, t1)),
             _result("gemm_tc_kernel[experts_down]", t2, b2, _flops({"active_experts": active, "rows": n}, f2, t2))]

@@ -298,6 +298,7 @@ def main():
     eng.commit()
     per_commit = bd.launch_count() - n0
     graph = eng.block_graph()
+    graph_cond = graph.conditional
 
     def block():
         eng.tokens.copy_(tokens0)
@@ -391,11 +392,13 @@ def main():
                 "config": bench_config(w, world),
                 "timed_units": {"n": len(units), "unit_s": units, "steps_per_unit": args.steps},
                 "committed_tokens_per_s": committed,
-                "passes_per_block": {"live": live, "launched": w.T_s,
+                "block_graph_conditional": graph_cond,
+                "passes_per_block": {"live": live, "launched": live if graph_cond else w.T_s,
                                      "rows_per_live_pass": [p["rows"] for p in passes if p["live"]]},
                 "active_experts_per_layer": {"mean": statistics.mean(act) if act else 0,
                                              "min": min(act) if act else 0, "max": max(act) if act else 0},
-                "gpu_launches": (live * per_pass + per_commit) * args.steps * len(units), "clocks": clk,
+                "gpu_launches": ((live if graph_cond else w.T_s) * per_pass + per_commit) * args.steps * len(units),
+                "clocks": clk,
                 "e2e": e2e, "e2e_graph": e2e_graph, "roofline": roof, "step_roofline": step_roof,
                 "kernels": kernels}
         if not args.no_cpu_baseline and world == 1:

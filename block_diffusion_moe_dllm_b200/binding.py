@@ -113,6 +113,7 @@ _SIGS = {
                                  C.POINTER(vp)], C.c_int),
     "dllm_block_graph_launch": ([vp, vp], C.c_int),
     "dllm_block_graph_destroy": ([vp], None),
+    "dllm_block_graph_skips_finished_passes": ([vp], C.c_int),
 }
 
 EXPORTED = sorted(_SIGS)

@@ -12,6 +12,9 @@
 
 #include <atomic>
 #include <algorithm>
+#include <cuda.h>
+#include <mutex>
+#include <vector>
 
 namespace dllm_host {
 static thread_local char g_err[512] = "";
@@ -755,6 +758,7 @@ struct dllm_block_graph {
   cudaGraph_t graph = nullptr;
   cudaGraphExec_t exec = nullptr;
   int passes = 0;
+  int conditional = 0;   // 1: the passes sit in conditional nodes (passes after an early finish are skipped)
 };
 
 void dllm_block_graph_destroy(dllm_block_graph* g) {
@@ -763,6 +767,65 @@ void dllm_block_graph_destroy(dllm_block_graph* g) {
   if (g->graph) cudaGraphDestroy(g->graph);
   delete g;
 }
+
+int dllm_block_graph_skips_finished_passes(const dllm_block_graph* g) { return g ? g->conditional : 0; }
+
+}  // extern "C"
+
+namespace {
+// Conditional (IF) nodes through the driver API, with the context given explicitly (the node, its handle and the
+// kernels of its body must share one context: the current one).
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CondHandleCreateFn)(CUgraphConditionalHandle*, CUgraph, CUcontext, unsigned int, unsigned int);
+typedef CUresult (*GraphAddNodeFn)(CUgraphNode*, CUgraph, const CUgraphNode*, size_t, CUgraphNodeParams*);
+
+struct CondApi {
+  CtxGetCurrentFn ctx_get = nullptr;
+  CondHandleCreateFn handle_create = nullptr;
+  GraphAddNodeFn add_node = nullptr;
+};
+
+const CondApi& cond_api() {
+  static CondApi api;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    auto get = [](const char* name) -> void* {
+      void* p = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess)
+        return nullptr;
+      return p;
+    };
+    api.ctx_get = reinterpret_cast<CtxGetCurrentFn>(get("cuCtxGetCurrent"));
+    api.handle_create = reinterpret_cast<CondHandleCreateFn>(get("cuGraphConditionalHandleCreate"));
+    api.add_node = reinterpret_cast<GraphAddNodeFn>(get("cuGraphAddNode"));
+  });
+  return api;
+}
+
+// One IF node after `prev` (nullable) in `graph`; its body graph is returned in *body.
+bool add_if_node(cudaGraph_t graph, cudaGraphConditionalHandle cond, CUcontext ctx, cudaGraphNode_t prev,
+                 cudaGraphNode_t* node, cudaGraph_t* body) {
+  const CondApi& api = cond_api();
+  if (!api.add_node) return false;
+  CUgraphNodeParams np;
+  memset(&np, 0, sizeof(np));
+  np.type = CU_GRAPH_NODE_TYPE_CONDITIONAL;
+  np.conditional.handle = cond;
+  np.conditional.type = CU_GRAPH_COND_TYPE_IF;
+  np.conditional.size = 1;
+  np.conditional.ctx = ctx;
+  CUgraphNode n = nullptr;
+  CUgraphNode dep = reinterpret_cast<CUgraphNode>(prev);
+  if (api.add_node(&n, reinterpret_cast<CUgraph>(graph), prev ? &dep : nullptr, prev ? 1 : 0, &np) != CUDA_SUCCESS)
+    return false;
+  *node = reinterpret_cast<cudaGraphNode_t>(n);
+  *body = reinterpret_cast<cudaGraph_t>(np.conditional.phGraph_out[0]);
+  return true;
+}
+}  // namespace
+
+extern "C" {
 
 int dllm_block_graph_create(const dllm_model* m, const dllm_state* st, const dllm_step_params* p, void* ws,
                             size_t ws_bytes, cudaStream_t capture_stream, dllm_block_graph** out) {
@@ -796,52 +859,79 @@ int dllm_block_graph_create(const dllm_model* m, const dllm_state* st, const dll
   };
   cudaError_t e = cudaGraphCreate(&g->graph, 0);
   if (e != cudaSuccess) return fail(e, "block_graph_create: cudaGraphCreate");
-  cudaGraphConditionalHandle cond;
-  e = cudaGraphConditionalHandleCreate(&cond, g->graph, 1, cudaGraphCondAssignDefault);
-  if (e != cudaSuccess) return fail(e, "block_graph_create: cudaGraphConditionalHandleCreate");
-  cudaGraphNode_t prev = nullptr;
-  for (int t = 0; t < p->T_s; ++t) {
-    cudaGraphNodeParams np = {};
-    np.type = cudaGraphNodeTypeConditional;
-    np.conditional.handle = cond;
-    np.conditional.type = cudaGraphCondTypeIf;
-    np.conditional.size = 1;
-    cudaGraphNode_t node;
-    e = cudaGraphAddNode(&node, g->graph, prev ? &prev : nullptr, prev ? 1 : 0, &np);
-    if (e != cudaSuccess) return fail(e, "block_graph_create: cudaGraphAddNode (conditional)");
-    cudaGraph_t body = np.conditional.phGraph_out[0];
-    e = cudaStreamBeginCaptureToGraph(capture_stream, body, nullptr, nullptr, 0, cudaStreamCaptureModeThreadLocal);
+  // conditional passes when the driver offers them (the handle and the nodes on the current context); otherwise
+  // the passes follow one another unconditionally and those after an early finish return at entry
+  const CondApi& api = cond_api();
+  CUcontext ctx = nullptr;
+  cudaGraphConditionalHandle cond = 0;
+  bool use_cond = api.ctx_get && api.handle_create && api.add_node && api.ctx_get(&ctx) == CUDA_SUCCESS && ctx &&
+                  api.handle_create(reinterpret_cast<CUgraphConditionalHandle*>(&cond),
+                                    reinterpret_cast<CUgraph>(g->graph), ctx, 1,
+                                    CU_GRAPH_COND_ASSIGN_DEFAULT) == CUDA_SUCCESS;
+  cudaGraphNode_t first = nullptr;
+  cudaGraph_t first_body = nullptr;
+  if (use_cond && !add_if_node(g->graph, cond, ctx, nullptr, &first, &first_body)) {
+    // the conditional node was refused: a fresh graph without conditions (the handle stays unused)
+    use_cond = false;
+    cudaGraphDestroy(g->graph);
+    g->graph = nullptr;
+    e = cudaGraphCreate(&g->graph, 0);
+    if (e != cudaSuccess) return fail(e, "block_graph_create: cudaGraphCreate");
+  }
+  auto capture_pass = [&](cudaGraph_t target, const cudaGraphNode_t* deps, size_t n_deps, int t, int commit,
+                          bool set_cond) -> int {
+    cudaError_t ce = cudaStreamBeginCaptureToGraph(capture_stream, target, deps, nullptr, n_deps,
+                                                   cudaStreamCaptureModeThreadLocal);
+    if (ce != cudaSuccess) return dllm_host::cuda_status(ce, "block_graph_create: cudaStreamBeginCaptureToGraph");
+    dllm_step_params q = *p;
+    q.t = commit ? 0 : t;
+    q.commit = commit;
+    q.retain = !commit && p->sprint && t == 0 ? 1 : 0;
+    int rr = denoise_step_impl(m, st, &q, ws, ws_bytes, capture_stream, cond, set_cond ? 1 : 0);
+    cudaGraph_t captured = nullptr;
+    ce = cudaStreamEndCapture(capture_stream, &captured);
+    if (rr) return rr;
+    if (ce != cudaSuccess) return dllm_host::cuda_status(ce, "block_graph_create: cudaStreamEndCapture");
+    return DLLM_OK;
+  };
+  if (use_cond) {
+    cudaGraphNode_t prev = first;
+    r = capture_pass(first_body, nullptr, 0, 0, 0, true);
+    for (int t = 1; t < p->T_s && !r; ++t) {
+      cudaGraphNode_t node = nullptr;
+      cudaGraph_t body = nullptr;
+      if (!add_if_node(g->graph, cond, ctx, prev, &node, &body)) {
+        dllm_block_graph_destroy(g);
+        dllm_host::set_error("block_graph_create: a conditional node was refused after the first was accepted");
+        return DLLM_ERR_CUDA;
+      }
+      r = capture_pass(body, nullptr, 0, t, 0, true);
+      prev = node;
+    }
+    if (!r) r = capture_pass(g->graph, &prev, 1, 0, 1, false);
+  } else {
+    // one capture of the whole block: the passes and the commit pass in stream order
+    e = cudaStreamBeginCaptureToGraph(capture_stream, g->graph, nullptr, nullptr, 0, cudaStreamCaptureModeThreadLocal);
     if (e != cudaSuccess) return fail(e, "block_graph_create: cudaStreamBeginCaptureToGraph");
-    pp = *p;
-    pp.t = t;
-    pp.commit = 0;
-    pp.retain = p->sprint && t == 0 ? 1 : 0;
-    r = denoise_step_impl(m, st, &pp, ws, ws_bytes, capture_stream, cond, 1);
+    for (int t = 0; t <= p->T_s && !r; ++t) {
+      dllm_step_params q = *p;
+      q.t = t < p->T_s ? t : 0;
+      q.commit = t == p->T_s;
+      q.retain = !q.commit && p->sprint && t == 0 ? 1 : 0;
+      r = denoise_step_impl(m, st, &q, ws, ws_bytes, capture_stream, cudaGraphConditionalHandle(), 0);
+    }
     cudaGraph_t captured = nullptr;
     e = cudaStreamEndCapture(capture_stream, &captured);
-    if (r) {
-      dllm_block_graph_destroy(g);
-      return r;
-    }
-    if (e != cudaSuccess) return fail(e, "block_graph_create: cudaStreamEndCapture");
-    prev = node;
+    if (!r && e != cudaSuccess) r = dllm_host::cuda_status(e, "block_graph_create: cudaStreamEndCapture");
   }
-  e = cudaStreamBeginCaptureToGraph(capture_stream, g->graph, &prev, nullptr, 1, cudaStreamCaptureModeThreadLocal);
-  if (e != cudaSuccess) return fail(e, "block_graph_create: cudaStreamBeginCaptureToGraph (commit)");
-  pp = *p;
-  pp.commit = 1;
-  pp.retain = 0;
-  r = denoise_step_impl(m, st, &pp, ws, ws_bytes, capture_stream, cudaGraphConditionalHandle(), 0);
-  cudaGraph_t captured = nullptr;
-  e = cudaStreamEndCapture(capture_stream, &captured);
   if (r) {
     dllm_block_graph_destroy(g);
     return r;
   }
-  if (e != cudaSuccess) return fail(e, "block_graph_create: cudaStreamEndCapture (commit)");
   e = cudaGraphInstantiate(&g->exec, g->graph, 0);
   if (e != cudaSuccess) return fail(e, "block_graph_create: cudaGraphInstantiate");
   g->passes = p->T_s;
+  g->conditional = use_cond ? 1 : 0;
   *out = g;
   return DLLM_OK;
 }

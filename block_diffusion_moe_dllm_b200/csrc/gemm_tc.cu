@@ -40,7 +40,9 @@ constexpr int SMEM_LIMIT = 232448;
 struct Smem {
   uint64_t full[16];
   uint64_t empty[16];
-  uint64_t conv[16];                // FP8: the stage's bf16 weight tile is written (128 converter arrivals)
+  uint64_t conv[16];                // FP8: operand slot's bf16 weight tile written (128 converter arrivals)
+  uint64_t bfull[16];               // FP8: operand slot's activation tile landed (TMA transaction bytes)
+  uint64_t mempty[16];              // FP8: operand slot free again (MMA commit)
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t done;
@@ -392,11 +394,18 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   constexpr int NT = F8 ? NUM_THREADS_F8 : NUM_THREADS;
   constexpr int B_BYTES = BN * BK * 2;
-  constexpr int STAGE_BYTES = A_BYTES + B_BYTES + (F8 ? RAW_BYTES : 0);   // [A bf16][B][E4M3 codes (FP8)]
+  // bf16 weights: STAGES stages of [A weight tile][B activation tile]. FP8 weights: a deep ring of STAGES E4M3
+  // weight tiles (the HBM stream) and a shallow ring of MS operand slots [A bf16 tile][B activation tile] that the
+  // converter warps fill (activations come from L2, so two or three slots keep the MMA fed).
+  constexpr int MS = F8 ? (BN >= 128 ? 2 : 3) : 0;
+  constexpr int MSD = MS > 0 ? MS : 1;        // slot count as a divisor (the bf16 instantiations use no slots)
+  constexpr int STAGE_BYTES = F8 ? RAW_BYTES : A_BYTES + B_BYTES;
+  constexpr int SLOT_BYTES = A_BYTES + B_BYTES;
   constexpr uint32_t W_TX = F8 ? RAW_BYTES : A_BYTES;                     // weight bytes a stage's TMA brings
   uint8_t* stages = base;
-  float* staging = reinterpret_cast<float*>(base + STAGES * STAGE_BYTES);
-  Smem& sm = *reinterpret_cast<Smem*>(base + STAGES * STAGE_BYTES + STAGING_BYTES);
+  uint8_t* slots = base + STAGES * STAGE_BYTES;                           // FP8 operand slots
+  float* staging = reinterpret_cast<float*>(slots + MS * SLOT_BYTES);
+  Smem& sm = *reinterpret_cast<Smem*>(reinterpret_cast<uint8_t*>(staging) + STAGING_BYTES);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -407,8 +416,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
     sm.abort_flag = 0;
     for (int s = 0; s < STAGES; ++s) {
       tc::mbar_init(&sm.full[s], 1);
-      tc::mbar_init(&sm.empty[s], 1);
-      if (F8) tc::mbar_init(&sm.conv[s], 128);
+      tc::mbar_init(&sm.empty[s], F8 ? 128 : 1);   // FP8: released by the converters once they read the codes
+    }
+    for (int s = 0; s < MS; ++s) {
+      tc::mbar_init(&sm.conv[s], 128);
+      tc::mbar_init(&sm.bfull[s], 1);
+      tc::mbar_init(&sm.mempty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(&sm.tfull[b], 1);
@@ -433,9 +446,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
       tc::prefetch_tmap(&tmap_w);
       const uint64_t pol_w = tc::policy_evict_first();
       for (int i = 0; i < npf; ++i) {
-        tc::mbar_expect_tx(&sm.full[i], W_TX);
-        tc::tma_load_2d(stages + i * STAGE_BYTES + (F8 ? A_BYTES + B_BYTES : 0), &tmap_w, (kb0 + i) * BK, t0 * 128,
-                        &sm.full[i], pol_w);
+        if (F8) tc::mbar_arrive_expect_tx(&sm.full[i], W_TX);   // the weight ring's stage is complete with it
+        else tc::mbar_expect_tx(&sm.full[i], W_TX);
+        tc::tma_load_2d(stages + i * STAGE_BYTES, &tmap_w, (kb0 + i) * BK, t0 * 128, &sm.full[i], pol_w);
       }
     }
   }
@@ -516,28 +529,29 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
         const CUtensorMap* wm = extra ? &tmap_w2 : &tmap_w;
         const int64_t wrow = extra ? 0 : (int64_t)g * p.w_group_stride;
         const int nb = (nval + XBOX_ROWS - 1) / XBOX_ROWS;
-        const uint32_t bytes = W_TX + nb * XBOX_BYTES;
+        const uint32_t bytes = W_TX + (F8 ? 0 : nb * XBOX_BYTES);
         const int xrow = sm.grp_off[g] + n0;
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
+          if (F8 && it < (uint32_t)npf) continue;   // weight stage already in flight and armed
           if (!wait_bar(&sm.empty[s], ph ^ 1, abort_flag, p.status, ST_TIMEOUT_PRODUCER)) { ok = false; break; }
           uint8_t* a = stages + s * STAGE_BYTES;
           uint8_t* b = a + A_BYTES;
-          uint8_t* wdst = F8 ? a + A_BYTES + B_BYTES : a;   // FP8: the codes land after the B tile
           if (it < (uint32_t)npf) {   // weight stage already in flight: arrive with the activation bytes
             tc::mbar_arrive_expect_tx(&sm.full[s], bytes - W_TX);
           } else {
             tc::mbar_arrive_expect_tx(&sm.full[s], bytes);
             if (p.swiglu) {
-              tc::tma_load_2d(wdst, wm, kb * BK, (int)(wrow + mt * 64), &sm.full[s], pol_w);
-              tc::tma_load_2d(wdst + W_TX / 2, wm, kb * BK, (int)(wrow + p.M + mt * 64), &sm.full[s], pol_w);
+              tc::tma_load_2d(a, wm, kb * BK, (int)(wrow + mt * 64), &sm.full[s], pol_w);
+              tc::tma_load_2d(a + W_TX / 2, wm, kb * BK, (int)(wrow + p.M + mt * 64), &sm.full[s], pol_w);
             } else {
-              tc::tma_load_2d(wdst, wm, kb * BK, (int)(wrow + mt * 128), &sm.full[s], pol_w);
+              tc::tma_load_2d(a, wm, kb * BK, (int)(wrow + mt * 128), &sm.full[s], pol_w);
             }
           }
-          for (int j = 0; j < nb; ++j)
-            tc::tma_load_2d(b + j * XBOX_BYTES, &tmap_x, kb * BK, xrow + j * XBOX_ROWS, &sm.full[s], pol_x);
+          if (!F8)
+            for (int j = 0; j < nb; ++j)
+              tc::tma_load_2d(b + j * XBOX_BYTES, &tmap_x, kb * BK, xrow + j * XBOX_ROWS, &sm.full[s], pol_x);
         }
       }
       if (!ok) {
@@ -548,7 +562,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
       // prefetched weight stages no work item consumed (no rows after all): complete their phase and let the
       // copies land before the CTA leaves
       for (uint32_t i = it; i < (uint32_t)npf; ++i) {
-        tc::mbar_arrive(&sm.full[i]);
+        if (!F8) tc::mbar_arrive(&sm.full[i]);
         tc::mbar_wait(&sm.full[i], 0, 1u << 16);
       }
     }
@@ -569,16 +583,25 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
         const uint32_t idesc = tc::idesc_bf16_f32(128, N);
         const uint32_t d = sm.tmem_base + buf * BN;
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
-          const int s = it % STAGES;
-          const uint32_t ph = (it / STAGES) & 1;
-          if (!wait_bar(F8 ? &sm.conv[s] : &sm.full[s], ph, abort_flag, p.status, ST_TIMEOUT_MMA)) { ok = false; break; }
+          uint32_t a;
+          if constexpr (F8) {
+            const int ms = it % MSD;
+            const uint32_t mph = (it / MSD) & 1;
+            if (!wait_bar(&sm.conv[ms], mph, abort_flag, p.status, ST_TIMEOUT_MMA) ||
+                !wait_bar(&sm.bfull[ms], mph, abort_flag, p.status, ST_TIMEOUT_MMA)) { ok = false; break; }
+            a = tc::smem_u32(slots + ms * SLOT_BYTES);
+          } else {
+            const int s = it % STAGES;
+            const uint32_t ph = (it / STAGES) & 1;
+            if (!wait_bar(&sm.full[s], ph, abort_flag, p.status, ST_TIMEOUT_MMA)) { ok = false; break; }
+            a = tc::smem_u32(stages + s * STAGE_BYTES);
+          }
           tc::fence_after_sync();
-          const uint32_t a = tc::smem_u32(stages + s * STAGE_BYTES);
           const uint32_t b = a + A_BYTES;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
             tc::mma_bf16(d, tc::sdesc_k128(a + kk * 32), tc::sdesc_k128(b + kk * 32), idesc, (kb != kb0) || kk != 0);
-          tc::mma_commit(&sm.empty[s]);
+          tc::mma_commit(F8 ? &sm.mempty[it % MSD] : &sm.empty[it % STAGES]);
         }
         if (!ok) break;
         tc::mma_commit(&sm.tfull[buf]);
@@ -589,23 +612,45 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
     }
   } else if (F8 && warp >= 6) {
     // ------------------------------------------------------------------ FP8: converter warps 6..9
-    // the same stage sequence as the MMA issuer: wait for the stage's copies, write its bf16 weight tile, make the
-    // writes visible to the tensor core (async proxy) and arrive on the stage's conv barrier
+    // per k-block, in the MMA's order: once the operand slot is free, thread 0 loads the slot's activation tile
+    // (TMA, on the slot's bfull barrier); every thread then waits for the weight stage, writes its share of the
+    // slot's bf16 weight tile, releases the weight stage, makes its writes visible to the tensor core (async proxy)
+    // and arrives on the slot's conv barrier
     const int ct = tid - 192;
-    uint32_t it = 0;
+    const uint64_t pol_x = tc::policy_evict_last();
+    if (ct == 0) tc::prefetch_tmap(&tmap_x);
+    uint32_t it = 0, issued = 0;
     bool ok = true;
     for (int wk = wk_begin; wk < total && ok; wk += wk_step) {
-      const int ks = wk - (wk / p.ksplit) * p.ksplit;
+      const int t = wk / p.ksplit, ks = wk - t * p.ksplit;
       const int kb0 = ks * kblocks / p.ksplit, kb1 = (ks + 1) * kblocks / p.ksplit;
+      int g, mt, n0, nval;
+      decode_tile<BN>(sm, p.m_tiles, t, g, mt, n0, nval);
+      const int nb = (nval + XBOX_ROWS - 1) / XBOX_ROWS;
+      const int xrow = sm.grp_off[g] + n0;
       for (int kb = kb0; kb < kb1; ++kb, ++it) {
-        const int s = it % STAGES;
-        const uint32_t ph = (it / STAGES) & 1;
+        const int s = it % STAGES, ms = it % MSD;
+        const uint32_t ph = (it / STAGES) & 1, mph = (it / MSD) & 1;
+        if (!wait_bar(&sm.mempty[ms], mph ^ 1, abort_flag, p.status, ST_TIMEOUT_MMA)) { ok = false; break; }
+        uint8_t* slot = slots + ms * SLOT_BYTES;
+        if (ct == 0) {
+          tc::mbar_arrive_expect_tx(&sm.bfull[ms], (uint32_t)(nb * XBOX_BYTES));
+          for (int j = 0; j < nb; ++j)
+            tc::tma_load_2d(slot + A_BYTES + j * XBOX_BYTES, &tmap_x, kb * BK, xrow + j * XBOX_ROWS, &sm.bfull[ms],
+                            pol_x);
+          issued = it + 1;
+        }
         if (!wait_bar(&sm.full[s], ph, abort_flag, p.status, ST_TIMEOUT_MMA)) { ok = false; break; }
-        uint8_t* a = stages + s * STAGE_BYTES;
-        convert_e4m3_tile(a + A_BYTES + B_BYTES, a, ct);
+        convert_e4m3_tile(stages + s * STAGE_BYTES, slot, ct);
+        tc::mbar_arrive(&sm.empty[s]);
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        tc::mbar_arrive(&sm.conv[s]);
+        tc::mbar_arrive(&sm.conv[ms]);
       }
+    }
+    if (ct == 0 && !ok) {
+      // drain: the activation copies this thread issued land before the CTA leaves (bounded)
+      const uint32_t first = issued > (uint32_t)MSD ? issued - MSD : 0;
+      for (uint32_t i = first; i < issued; ++i) tc::mbar_wait(&sm.bfull[i % MSD], (i / MSD) & 1, 1u << 16);
     }
   } else {
     // ------------------------------------------------------------------ epilogue warps 2..5
@@ -1014,8 +1059,10 @@ int launch_cluster_splitk(const GemmArgs& a, const CUtensorMap& mw, const CUtens
 template <int BN, int STAGES, bool F8 = false>
 int launch(const GemmArgs& a, const CUtensorMap& mw, const CUtensorMap& mw2, const CUtensorMap& mx,
            const KParams& kp, cudaStream_t s) {
-  constexpr int STAGE_BYTES = A_BYTES + BN * BK * 2 + (F8 ? RAW_BYTES : 0);
-  constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + STAGING_BYTES + (int)sizeof(Smem);
+  // (matches the kernel's layout: bf16 stages, or FP8 weight stages plus operand slots)
+  constexpr int MS = F8 ? (BN >= 128 ? 2 : 3) : 0;
+  constexpr int STAGE_BYTES = F8 ? RAW_BYTES : A_BYTES + BN * BK * 2;
+  constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + MS * (A_BYTES + BN * BK * 2) + STAGING_BYTES + (int)sizeof(Smem);
   static_assert(SMEM <= SMEM_LIMIT, "shared memory budget");
   // With programmatic dependent launch a CTA allocates tensor memory before it waits for the kernels ahead of it.
   // More than half an SM's shared memory per CTA keeps two tensor-memory kernels from sharing an SM, so a later
@@ -1208,9 +1255,9 @@ int gemm_bf16_tc(const GemmArgs& a, cudaStream_t s) {
   kp.prefetch_w = (!a.swiglu && !a.n_dev && !a.has_extra && a.host_cnt <= (ks > 1 ? 32 : bn)) ? 1 : 0;
   int st2;
   if (f8) {   // single-CTA tiles, no split-K (the weight-streaming shapes FP8 weights serve)
-    if (bn == 32) st2 = launch<32, 6, true>(a, mw, mw2, mx, kp, s);
-    else if (bn == 64) st2 = launch<64, 6, true>(a, mw, mw2, mx, kp, s);
-    else st2 = launch<128, 4, true>(a, mw, mw2, mx, kp, s);
+    if (bn == 32) st2 = launch<32, 16, true>(a, mw, mw2, mx, kp, s);
+    else if (bn == 64) st2 = launch<64, 14, true>(a, mw, mw2, mx, kp, s);
+    else st2 = launch<128, 13, true>(a, mw, mw2, mx, kp, s);
   } else if (gemm_uses_pairs(a)) {
     kp.prefetch_w = 0;
     st2 = launch_pair(mw, mw2, mx, kp, s);

@@ -162,6 +162,11 @@ class BlockGraph:
     def launch(self, stream=None):
         return bd.check(self.lib.dllm_block_graph_launch(self.handle, bd.stream_handle(stream)))
 
+    @property
+    def conditional(self):
+        """True when the passes sit in conditional nodes (passes after an early finish are not launched)."""
+        return bool(self.lib.dllm_block_graph_skips_finished_passes(self.handle))
+
     def __del__(self):
         if getattr(self, "handle", None) and self.handle.value:
             self.lib.dllm_block_graph_destroy(self.handle)

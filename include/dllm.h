@@ -380,7 +380,9 @@ DLLM_API size_t dllm_denoise_step_workspace_size(const dllm_model* model, const 
  * once; its kernels read the state, caches and outputs at the addresses given here on every launch, so the caller
  * refills tokens / mask and launches it again for the next block of the same shapes. Host memory only: the library
  * allocates no device memory (instantiating the graph may reserve driver resources). Destroy with
- * dllm_block_graph_destroy.
+ * dllm_block_graph_destroy. Where the driver refuses conditional nodes the passes follow one another unconditionally
+ * (those after an early finish then return at entry, see dllm_denoise_step); dllm_block_graph_skips_finished_passes
+ * tells which (1: conditional).
  */
 typedef struct dllm_block_graph dllm_block_graph;
 DLLM_API int dllm_block_graph_create(const dllm_model* model, const dllm_state* state, const dllm_step_params* params,
@@ -388,6 +390,7 @@ DLLM_API int dllm_block_graph_create(const dllm_model* model, const dllm_state* 
                                      dllm_block_graph** out /* host */);
 DLLM_API int dllm_block_graph_launch(const dllm_block_graph* graph, cudaStream_t stream);
 DLLM_API void dllm_block_graph_destroy(dllm_block_graph* graph);
+DLLM_API int dllm_block_graph_skips_finished_passes(const dllm_block_graph* graph);
 
 /* Device addresses, inside a step workspace, of intermediate results of the last dllm_denoise_step that used it
  * (read-only views for inspection; valid until the workspace is reused). */

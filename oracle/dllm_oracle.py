@@ -271,6 +271,36 @@ def confidence(z):
     return cand.astype(np.int64), np.exp(zmax - lse), lse, zmax
 
 
+SCORES = ("low_confidence", "top_k_margin", "neg_entropy")
+
+
+def position_scores(z, score="low_confidence"):
+    """Score by which [M] "SPRINT 加速技术" ranks the still-masked positions (its strategies low_confidence,
+    top_k_margin, neg_entropy; the formulas are not on the pages, these are the plain readings of the names), from
+    p = softmax(z) at temperature 1 over the scored vocabulary:
+      low_confidence: p_(1), the largest probability (the c_i of [R] "SPRINT");
+      top_k_margin:   p_(1) - p_(2), the two largest probabilities over distinct vocabulary entries (0 when the
+                      largest logit occurs twice);
+      neg_entropy:    sum_v p_v log p_v, the negated entropy (0 for a one-hot distribution, -log V for a uniform
+                      one).
+    z [n, V] -> score [n] (fp64)."""
+    z = f64(z)
+    zmax = z.max(axis=1, keepdims=True)
+    e = np.exp(z - zmax)
+    ssum = e.sum(axis=1)
+    p = e / ssum[:, None]
+    if score == "low_confidence":
+        return p.max(axis=1)
+    if score == "top_k_margin":
+        top2 = np.sort(p, axis=1)[:, -2:] if p.shape[1] > 1 else np.concatenate([np.zeros_like(p), p], axis=1)
+        return top2[:, 1] - top2[:, 0]
+    if score == "neg_entropy":
+        # sum_v p_v log p_v with log p_v = (z_v - zmax) - log(sum); terms with p_v = 0 contribute 0
+        logp = (z - zmax) - np.log(ssum)[:, None]
+        return (p * logp).sum(axis=1)
+    raise ValueError(score)
+
+
 def unmask_count(m, t, T_s, mode, tau=None, k_max=None, conf_masked=None):
     """Positions to unmask at step t (0-based) of T_s with m still masked.
 
@@ -296,7 +326,7 @@ def select_positions(conf_row, masked_row, k):
 
 
 def unmask(z_rows, row_pos, tokens, mask, t, T_s, mode=0, tau=0.9, k_max=8, vocab_offset=0,
-           z_uncond=None, cfg_scale=1.0):
+           z_uncond=None, cfg_scale=1.0, score="low_confidence"):
     """One unmasking step over a batch of block rows.
 
     z_rows [n, V]: logits of the still-masked positions, row r belongs to flat position row_pos[r] = b*L + i of
@@ -308,8 +338,12 @@ def unmask(z_rows, row_pos, tokens, mask, t, T_s, mode=0, tau=0.9, k_max=8, voca
     (tie_tau). A library that evaluates the guidance in float32 perturbs each guided logit by up to
     cfg_fp32_error_bound (z_err per row); the bands then widen by that amount: a candidate whose top-2 guided-logit
     gap is at most 2 z_err (tie_cand), and confidences, which move by a relative 2 z_err at most (conf_rtol).
-    Returns dict(tokens, mask, sel [Bl, k], nsel [Bl], conf [Bl, L], cand [Bl, L], tie_rank [Bl], tie_tau [Bl],
-    tie_cand [Bl, L], conf_rtol [Bl, L]) where Bl is the number of logical rows."""
+    score: the strategy that ranks the positions (position_scores); the threshold acceptance always counts the
+    positions whose largest probability exceeds tau ([M] "SPRINT 加速技术": tokens whose probability exceeds the
+    threshold are accepted).
+    Returns dict(tokens, mask, sel [Bl, k], nsel [Bl], conf [Bl, L] (largest probability), rank [Bl, L] (ranking
+    score), cand [Bl, L], tie_rank [Bl], tie_tau [Bl], tie_cand [Bl, L], conf_rtol [Bl, L]) where Bl is the number
+    of logical rows."""
     tokens = np.array(tokens, dtype=np.int64, copy=True)
     mask = np.array(mask, dtype=np.int64, copy=True)
     B, L = mask.shape
@@ -321,18 +355,21 @@ def unmask(z_rows, row_pos, tokens, mask, t, T_s, mode=0, tau=0.9, k_max=8, voca
         z = f64(z_rows)
         z_err = np.zeros(z.shape[0])
     cand_r, conf_r, _, _ = confidence(z)
+    rank_r = conf_r if score == "low_confidence" else position_scores(z, score)
     if z.shape[1] > 1:
         top2 = np.sort(z, axis=1)[:, -2:]
         gap_r = top2[:, 1] - top2[:, 0]
     else:
         gap_r = np.full(z.shape[0], np.inf)
     conf = np.zeros((Bl, L))
+    rank = np.zeros((Bl, L))
     cand = np.full((Bl, L), -1, dtype=np.int64)
     tie_cand = np.zeros((Bl, L), dtype=bool)
     conf_rtol = np.full((Bl, L), 1e-6)
     for r, p in enumerate(row_pos):
         b, i = divmod(int(p), L)
         conf[b, i] = conf_r[r]
+        rank[b, i] = rank_r[r]
         cand[b, i] = cand_r[r] + vocab_offset
         tie_cand[b, i] = z_err[r] > 0 and gap_r[r] <= 2.0 * z_err[r]
         conf_rtol[b, i] = 1e-6 + 2.0 * z_err[r]
@@ -344,9 +381,9 @@ def unmask(z_rows, row_pos, tokens, mask, t, T_s, mode=0, tau=0.9, k_max=8, voca
         m = int(masked.sum())
         cm = conf[b][masked]
         kt = unmask_count(m, t, T_s, mode, tau, k_max, cm)
-        chosen, margin = select_positions(conf[b], masked, kt)
+        chosen, margin = select_positions(rank[b], masked, kt)
         band = 2.0 * float(conf_rtol[b].max())
-        tie_rank[b] = margin < band * max(conf[b].max(), 1e-30)
+        tie_rank[b] = margin < band * max(np.abs(rank[b][masked]).max() if m else 0.0, 1e-30)
         if mode == 1 and m:
             tie_tau[b] = bool(np.any(np.abs(cm - tau) < 1e-6 + conf_rtol[b][masked] * cm))
         for i in chosen:
@@ -357,7 +394,7 @@ def unmask(z_rows, row_pos, tokens, mask, t, T_s, mode=0, tau=0.9, k_max=8, voca
                 mask[b + Bl, i] = 0
         sel.append(chosen)
         nsel[b] = kt
-    return dict(tokens=tokens, mask=mask, sel=sel, nsel=nsel, conf=conf, cand=cand,
+    return dict(tokens=tokens, mask=mask, sel=sel, nsel=nsel, conf=conf, rank=rank, cand=cand,
                 tie_rank=tie_rank, tie_tau=tie_tau, tie_cand=tie_cand, conf_rtol=conf_rtol)
 
 

@@ -550,3 +550,54 @@ def test_dequant_rows_scales_each_output_row():
     q = np.array([[0x38, 0xB8], [0x40, 0x30]], dtype=np.uint8)      # [[1, -1], [2, 0.5]]
     w = O.dequant_rows(q, np.array([0.5, 3.0], dtype=np.float32))
     assert np.array_equal(w, [[0.5, -0.5], [6.0, 1.5]])
+
+
+# ---------------------------------------------------------------------------------------------- position scores
+
+def test_position_scores_closed_forms():
+    V = 50
+    zu = np.zeros((1, V))                            # uniform: p = 1/V everywhere
+    assert abs(O.position_scores(zu, "low_confidence")[0] - 1 / V) < 1e-15
+    assert abs(O.position_scores(zu, "top_k_margin")[0]) < 1e-15
+    assert abs(O.position_scores(zu, "neg_entropy")[0] + math.log(V)) < 1e-12
+    d = 3.0                                          # one spike: p1 = e^d / (e^d + V - 1), the rest 1 / (e^d + V - 1)
+    zs = np.zeros((1, V))
+    zs[0, 7] = d
+    S = math.exp(d) + V - 1
+    p1, p0 = math.exp(d) / S, 1 / S
+    assert abs(O.position_scores(zs, "top_k_margin")[0] - (p1 - p0)) < 1e-15
+    ent = p1 * math.log(p1) + (V - 1) * p0 * math.log(p0)
+    assert abs(O.position_scores(zs, "neg_entropy")[0] - ent) < 1e-12
+    z2 = np.zeros((1, V))                            # the largest logit twice: margin 0
+    z2[0, 3] = z2[0, 9] = 2.0
+    assert O.position_scores(z2, "top_k_margin")[0] == 0.0
+
+
+def test_position_scores_brute_force_small_vocab():
+    for _ in range(20):
+        z = rng.standard_normal((3, 7)) * 2
+        p = np.exp(z) / np.exp(z).sum(axis=1, keepdims=True)
+        srt = np.sort(p, axis=1)
+        assert np.allclose(O.position_scores(z, "top_k_margin"), srt[:, -1] - srt[:, -2], atol=1e-15)
+        assert np.allclose(O.position_scores(z, "neg_entropy"), (p * np.log(p)).sum(axis=1), atol=1e-13)
+        assert np.allclose(O.position_scores(z, "low_confidence"), p.max(axis=1), atol=1e-15)
+
+
+def test_unmask_ranks_by_score_and_counts_by_probability():
+    """The strategies rank differently: position 0 (p = 0.60, 0.39, ...) has the larger top probability, position 1
+    (p = 0.55, 0.05, ...) the larger margin and the lower entropy. The threshold count always uses the largest
+    probability (here none exceeds tau, so one position per step is taken)."""
+    V = 10
+    pa = np.array([0.60, 0.39] + [0.01 / 8] * 8)
+    pb = np.array([0.55] + [0.05] * 9)
+    z = np.log(np.stack([pa, pb]))
+    tok = np.full((1, 2), V - 1)
+    msk = np.ones((1, 2), dtype=np.int64)
+    args = dict(mode=1, tau=0.9, k_max=2)
+    assert list(O.unmask(z, [0, 1], tok, msk, 0, 2, score="low_confidence", **args)["sel"][0]) == [0]
+    assert list(O.unmask(z, [0, 1], tok, msk, 0, 2, score="top_k_margin", **args)["sel"][0]) == [1]
+    ent_a, ent_b = (pa * np.log(pa)).sum(), (pb * np.log(pb)).sum()
+    assert ent_b < ent_a                     # position 0 has the lower entropy: neg_entropy ranks it first
+    assert list(O.unmask(z, [0, 1], tok, msk, 0, 2, score="neg_entropy", **args)["sel"][0]) == [0]
+    u = O.unmask(z, [0, 1], tok, msk, 0, 2, score="top_k_margin", **args)
+    assert np.allclose(u["rank"][0], [0.60 - 0.39, 0.55 - 0.05]) and np.allclose(u["conf"][0], [0.60, 0.55])

@@ -14,6 +14,7 @@ OK, ERR_INVALID_ARG, ERR_SHAPE, ERR_ALIGN, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_C
 BF16, F32 = 0, 1
 FIXED, THRESHOLD = 0, 1
 WEIGHTS_BF16, WEIGHTS_FP8 = 0, 1
+SCORE_LOW_CONFIDENCE, SCORE_TOP_K_MARGIN, SCORE_NEG_ENTROPY = 0, 1, 2
 
 STATUS_NAMES = {0: "DLLM_OK", 1: "DLLM_ERR_INVALID_ARG", 2: "DLLM_ERR_SHAPE", 3: "DLLM_ERR_ALIGN",
                 4: "DLLM_ERR_UNSUPPORTED", 5: "DLLM_ERR_WORKSPACE", 6: "DLLM_ERR_CUDA", 7: "DLLM_ERR_TIMEOUT"}
@@ -52,7 +53,7 @@ class ExpertDesc(C.Structure):
 class UnmaskDesc(C.Structure):
     _fields_ = [("B", i32), ("L", i32), ("V", i32), ("max_rows", i32), ("t", i32), ("T_s", i32), ("mode", i32),
                 ("tau", f32), ("k_max", i32), ("cfg", i32), ("cfg_scale", f32), ("vocab_offset", i32),
-                ("dtype", i32)]
+                ("dtype", i32), ("score", i32)]
 
 
 class Layer(C.Structure):
@@ -76,7 +77,8 @@ class State(C.Structure):
 class StepParams(C.Structure):
     _fields_ = [("t", i32), ("T_s", i32), ("mode", i32), ("tau", f32), ("k_max", i32), ("cfg", i32),
                 ("cfg_scale", f32), ("vocab_offset", i32), ("vocab_len", i32), ("sprint", i32), ("n_keep", i32),
-                ("retain", i32), ("commit", i32), ("sel", vp), ("nsel", vp), ("conf", vp), ("remaining", vp)]
+                ("retain", i32), ("commit", i32), ("sel", vp), ("nsel", vp), ("conf", vp), ("remaining", vp),
+                ("score", i32)]
 
 
 class StepViews(C.Structure):
@@ -246,9 +248,10 @@ def moe_experts(h, w_gu, w_down, w_gu_shared, w_down_shared, counts, offsets, pe
 
 
 def unmask(logits, row_pos, n_rows_dev, tokens, mask, sel, nsel, conf, remaining, B, L, V, max_rows, t, T_s,
-           dtype, mode=FIXED, tau=0.9, k_max=8, cfg=0, cfg_scale=1.0, vocab_offset=0, ws=None, stream=None):
+           dtype, mode=FIXED, tau=0.9, k_max=8, cfg=0, cfg_scale=1.0, vocab_offset=0, score=SCORE_LOW_CONFIDENCE,
+           ws=None, stream=None):
     lib = load()
-    desc = UnmaskDesc(B, L, V, max_rows, t, T_s, mode, tau, k_max, cfg, cfg_scale, vocab_offset, dtype)
+    desc = UnmaskDesc(B, L, V, max_rows, t, T_s, mode, tau, k_max, cfg, cfg_scale, vocab_offset, dtype, score)
     need = lib.dllm_unmask_workspace_size(C.byref(desc))
     ws = (ws or Workspace(need, logits.device)).ensure(need)
     return check(lib.dllm_unmask(C.byref(desc), ptr(logits), ptr(row_pos), ptr(n_rows_dev), ptr(tokens), ptr(mask),

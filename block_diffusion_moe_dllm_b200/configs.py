@@ -43,6 +43,7 @@ class Workload:
     bias_range: float = 0.1
     seed: int = 0
     wfmt: str = "bf16"    # "fp8": expert and LM-head weights as E4M3 codes with per-row fp32 scales
+    score: int = 0        # ranking of the masked positions: 0 largest probability, 1 top-2 margin, 2 negated entropy
 
     @property
     def Tk(self) -> int:

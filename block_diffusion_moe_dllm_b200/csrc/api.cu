@@ -181,6 +181,7 @@ struct StepPlan {
   void* logits;
   void* partials;
   int conf_parts;   // > 0: the LM head writes this many confidence partials per row (fused epilogue)
+  void* unmask_extras;   // the other position scores' statistics (null for the largest probability)
   float* retain_raw;
   size_t total;
 };
@@ -203,6 +204,8 @@ int validate_step(const dllm_model* m, const dllm_state* st, const dllm_step_par
   REQ(m->embed && m->final_norm && m->w_lm, DLLM_ERR_INVALID_ARG, "denoise_step: NULL embed/final_norm/w_lm");
   REQ(p->T_s >= 1 && p->t >= 0 && p->t < p->T_s, DLLM_ERR_INVALID_ARG, "denoise_step: step %d of %d", p->t, p->T_s);
   REQ(p->mode == DLLM_UNMASK_FIXED || p->mode == DLLM_UNMASK_THRESHOLD, DLLM_ERR_INVALID_ARG, "bad unmask mode");
+  REQ(p->score >= DLLM_SCORE_LOW_CONFIDENCE && p->score <= DLLM_SCORE_NEG_ENTROPY, DLLM_ERR_INVALID_ARG,
+      "denoise_step: bad score %d", p->score);
   REQ(!p->cfg || st->B % 2 == 0, DLLM_ERR_SHAPE, "denoise_step: cfg needs an even number of rows");
   const int vlen = p->vocab_len ? p->vocab_len : m->V;
   REQ(p->vocab_offset >= 0 && p->vocab_offset + vlen <= m->V, DLLM_ERR_SHAPE, "denoise_step: vocab slice out of range");
@@ -264,7 +267,7 @@ void plan_step(const dllm_model* m, const dllm_state* st, const dllm_step_params
   s.max_rows = s.Bl * st->L;
   s.n_chunks = unmask_chunks(s.max_rows, s.vlen);
   s.conf_parts = 0;
-  if (m->dtype == DLLM_BF16 && !p->cfg) {
+  if (m->dtype == DLLM_BF16 && !p->cfg && p->score == DLLM_SCORE_LOW_CONFIDENCE) {
     GemmArgs g;   // the LM head's shape (see the step below)
     g.dtype = DLLM_BF16; g.K = m->H; g.M = s.vlen; g.host_cnt = s.max_rows; g.max_cnt = s.max_rows;
     g.cnt_bound = s.max_rows; g.epi.kind = EPI_STORE; g.w_fp8 = m->weight_format == DLLM_WEIGHTS_FP8;
@@ -296,6 +299,10 @@ void plan_step(const dllm_model* m, const dllm_state* st, const dllm_step_params
   s.xf = c.take((size_t)s.halves * s.max_rows * H * es);
   s.logits = c.take((size_t)s.halves * s.max_rows * s.vlen * es);
   s.partials = c.take(unmask_partials_bytes(s.max_rows, std::max(s.n_chunks, s.conf_parts)));
+  {
+    const size_t exb = unmask_extras_bytes(p->score, s.max_rows, s.n_chunks, s.Bl, st->L);
+    s.unmask_extras = exb ? c.take(exb) : nullptr;
+  }
   s.retain_raw = p->sprint ? c.take<float>(retain_workspace_bytes(st->B, st->P)) : nullptr;
   s.total = align256(c.off);
 }
@@ -556,7 +563,9 @@ int dllm_moe_experts(const dllm_expert_desc* d, const void* h, const void* w_gu,
 // ------------------------------------------------------------------------------------------------ unmask
 size_t dllm_unmask_workspace_size(const dllm_unmask_desc* d) {
   if (!d) return 0;
-  return align256(align256(kStatusBytes) + unmask_partials_bytes(d->max_rows, unmask_chunks(d->max_rows, d->V)));
+  const int nc = unmask_chunks(d->max_rows, d->V);
+  return align256(align256(align256(kStatusBytes) + unmask_partials_bytes(d->max_rows, nc)) +
+                  unmask_extras_bytes(d->score, d->max_rows, nc, d->B, d->L));
 }
 
 int dllm_unmask(const dllm_unmask_desc* d, const void* logits, const int32_t* row_pos, const int32_t* n_rows_dev,
@@ -572,6 +581,8 @@ int dllm_unmask(const dllm_unmask_desc* d, const void* logits, const int32_t* ro
   REQ(d->mode == DLLM_UNMASK_FIXED || d->k_max >= 1, DLLM_ERR_INVALID_ARG, "unmask: k_max must be >= 1");
   REQ(d->dtype == DLLM_BF16 || d->dtype == DLLM_F32, DLLM_ERR_INVALID_ARG, "unmask: bad dtype");
   REQ(d->vocab_offset >= 0, DLLM_ERR_INVALID_ARG, "unmask: negative vocab_offset");
+  REQ(d->score >= DLLM_SCORE_LOW_CONFIDENCE && d->score <= DLLM_SCORE_NEG_ENTROPY, DLLM_ERR_INVALID_ARG,
+      "unmask: bad score %d", d->score);
   int st = check_ws(ws, ws_bytes, dllm_unmask_workspace_size(d));
   if (st) return st;
   Carver c(ws);
@@ -582,6 +593,9 @@ int dllm_unmask(const dllm_unmask_desc* d, const void* logits, const int32_t* ro
   a.mask = mask; a.sel = sel; a.nsel = nsel; a.conf = conf; a.remaining = remaining;
   a.n_chunks = unmask_chunks(d->max_rows, d->V);
   a.partials = c.take(unmask_partials_bytes(d->max_rows, a.n_chunks));
+  a.score = d->score;
+  const size_t exb = unmask_extras_bytes(d->score, d->max_rows, a.n_chunks, d->B, d->L);
+  a.extras = exb ? c.take(exb) : nullptr;
   return launch_unmask(a, stream);
 }
 
@@ -740,6 +754,8 @@ int denoise_step_impl(const dllm_model* m, const dllm_state* st, const dllm_step
   ua.partials_ready = s.conf_parts ? 1 : 0;
   ua.cond = cond;
   ua.set_cond = set_cond;
+  ua.score = p->score;
+  ua.extras = s.unmask_extras;
   TRY(launch_unmask(ua, stream));
 #undef TRY
   return DLLM_OK;

@@ -22,6 +22,15 @@ struct ConfPartial {
   double s;
 };
 
+// The statistics the other position scores need, beside a ConfPartial of the same slice: the second largest
+// logit m2 (over distinct vocabulary entries, so equal to m when the largest value occurs twice; -inf for one entry)
+// and t = sum over the slice of exp(z - m) (z - m), from which the entropy follows.
+struct ConfExtra {
+  float m2;
+  float pad;
+  double t;
+};
+
 struct EpiParams {
   int kind = EPI_STORE;
   void* out = nullptr;

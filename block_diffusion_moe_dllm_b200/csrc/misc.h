@@ -57,9 +57,13 @@ struct UnmaskArgs {
   int partials_ready = 0;  // 1: the partials were written by the LM head's fused epilogue (no reduction launch)
   cudaGraphConditionalHandle cond = 0;  // with set_cond: the selection sets this graph condition to (remaining > 0)
   int set_cond = 0;
+  int score = 0;                 // DLLM_SCORE_*: how positions are ranked (the threshold counts largest probabilities)
+  void* extras = nullptr;        // score != 0: max_rows * n_chunks ConfExtra, then B * L floats of ranking scores
 };
 int unmask_chunks(int max_rows, int V);
 size_t unmask_partials_bytes(int max_rows, int n_chunks);
+// scratch beside the partials for the scores other than the largest probability (0 for that one)
+size_t unmask_extras_bytes(int score, int max_rows, int n_chunks, int B, int L);
 int launch_unmask(const UnmaskArgs& a, cudaStream_t s);
 
 // attention

@@ -156,6 +156,111 @@ __global__ void __launch_bounds__(256) unmask_reduce_kernel(const T* __restrict_
   }
 }
 
+// ---- the statistics of the other position scores (top-2 margin, entropy)
+// A running (m, idx, s) with (m2, t): m2 the second largest value seen (over entries), t = sum exp(z - m) (z - m).
+struct ExtPartial {
+  float m;
+  int idx;
+  double s;
+  float m2;
+  double t;
+};
+
+DLLM_DEV ExtPartial ext_empty() { return ExtPartial{-INFINITY, 0x7fffffff, 0.0, -INFINITY, 0.0}; }
+
+// Union of two partials. The maximum M, each side's sums moved to it (t by t' = e^(m - M) (t + (m - M) s)), the
+// lowest index at M, and the second largest value of the union.
+DLLM_DEV void ext_merge(ExtPartial& a, const ExtPartial& b) {
+  if (b.s == 0.0) return;
+  if (a.s == 0.0) { a = b; return; }
+  const float M = fmaxf(a.m, b.m);
+  const double fa = a.m == M ? 1.0 : exp((double)a.m - (double)M);
+  const double fb = b.m == M ? 1.0 : exp((double)b.m - (double)M);
+  const double ta = fa * (a.t + ((double)a.m - (double)M) * a.s);
+  const double tb = fb * (b.t + ((double)b.m - (double)M) * b.s);
+  float m2;
+  int idx;
+  if (a.m > b.m) { m2 = fmaxf(a.m2, b.m); idx = a.idx; }
+  else if (b.m > a.m) { m2 = fmaxf(b.m2, a.m); idx = b.idx; }
+  else { m2 = a.m; idx = min(a.idx, b.idx); }   // the maximum occurs on both sides
+  a = ExtPartial{M, idx, a.s * fa + b.s * fb, m2, ta + tb};
+}
+
+DLLM_DEV ExtPartial ext_one(float z, int v) { return ExtPartial{z, v, 1.0, -INFINITY, 0.0}; }
+
+// One more value z (vocabulary index v, visited in increasing v by this thread) into a running partial; the
+// per-value exponential in fp32, the sums in fp64.
+DLLM_DEV void ext_add(ExtPartial& p, float z, int v) {
+  if (p.s == 0.0) { p = ext_one(z, v); return; }
+  if (z > p.m) {
+    const float d = p.m - z;                      // < 0: the old terms scale by e^d
+    const double f = (double)expf(d);
+    p.t = f * (p.t + (double)d * p.s);
+    p.s = p.s * f + 1.0;
+    p.m2 = p.m;
+    p.m = z;
+    p.idx = v;
+  } else {
+    const float d = z - p.m;
+    const double e = (double)expf(d);
+    p.s += e;
+    p.t += e * (double)d;
+    p.m2 = fmaxf(p.m2, z);
+  }
+}
+
+DLLM_DEV ExtPartial ext_warp_merge(ExtPartial p) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    ExtPartial q;
+    q.m = __shfl_xor_sync(0xffffffffu, p.m, o);
+    q.idx = __shfl_xor_sync(0xffffffffu, p.idx, o);
+    q.s = __shfl_xor_sync(0xffffffffu, p.s, o);
+    q.m2 = __shfl_xor_sync(0xffffffffu, p.m2, o);
+    q.t = __shfl_xor_sync(0xffffffffu, p.t, o);
+    // merge in a fixed order (lower lane first) so that every lane computes the same result
+    if ((threadIdx.x & o) == 0) ext_merge(p, q);
+    else { ext_merge(q, p); p = q; }
+  }
+  return p;
+}
+
+// CTA per (row, chunk), any storage type, optional guidance: the extended partial of the chunk, stored as the
+// ConfPartial (m, idx, s) and its ConfExtra (m2, t).
+template <typename T, bool CFG>
+__global__ void __launch_bounds__(256) unmask_reduce_ext_kernel(const T* __restrict__ logits,
+                                                                const int32_t* __restrict__ n_rows, int max_rows,
+                                                                int V, int chunk, float cfg_scale,
+                                                                Partial* __restrict__ part,
+                                                                ConfExtra* __restrict__ extra, int n_chunks) {
+  pdl_enter();
+  const int r = blockIdx.x, c = blockIdx.y;
+  const int n = min(*n_rows, max_rows);
+  if (r >= n) return;
+  const T* zc = logits + (int64_t)r * V;
+  const T* zu = logits + (int64_t)(r + n) * V;
+  const int v0 = c * chunk, v1 = min(V, v0 + chunk);
+  ExtPartial p = ext_empty();
+  for (int v = v0 + threadIdx.x; v < v1; v += 256) {
+    float z = to_f32(zc[v]);
+    if (CFG) z = guided(z, to_f32(zu[v]), cfg_scale);
+    ext_add(p, z, v);
+  }
+  p = ext_warp_merge(p);
+  __shared__ ExtPartial wp[8];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  if (lane == 0) wp[w] = p;
+  __syncthreads();
+  if (w == 0) {
+    ExtPartial a = lane < 8 ? wp[lane] : ext_empty();
+    a = ext_warp_merge(a);
+    if (lane == 0) {
+      part[(int64_t)r * n_chunks + c] = Partial{a.m, a.idx, a.s};
+      extra[(int64_t)r * n_chunks + c] = ConfExtra{a.m2, 0.f, a.t};
+    }
+  }
+}
+
 // bf16 logits without guidance: each thread keeps its VPT 16-byte vectors of a chunk in registers. Pass 1 finds
 // the maximum with packed bf16x2 max (and the first vector holding it); pass 2 sums exp(z - max) as
 // 2^((z - max) * log2(e)) with the subtraction and the scaling done on fp32 pairs (z - max is exact near the
@@ -255,14 +360,36 @@ __global__ void __launch_bounds__(1024) unmask_select_kernel(Partial* part, int 
                                      const int32_t* __restrict__ n_rows, int max_rows, int B, int L, int t, int T_s, int mode,
                                      float tau, int k_max, int cfg, int vocab_offset, int32_t* tokens, uint8_t* mask,
                                      int32_t* sel, int32_t* nsel, float* conf, int32_t* remaining,
-                                     cudaGraphConditionalHandle cond, int set_cond) {
+                                     cudaGraphConditionalHandle cond, int set_cond, int score,
+                                     const ConfExtra* __restrict__ extra, float* __restrict__ rank) {
   pdl_enter();
   __shared__ int rem_w[32];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
   // this warp's first block row's mask, loaded ahead of phase A
   const bool mk0 = w < B && lane < L && mask[w * L + lane] != 0;
   const int nr = min(*n_rows, max_rows);   // partials exist for at most max_rows rows
-  if (n_chunks > kMergeSerial) {
+  if (extra) {
+    // other position scores: a thread per row merges its partials with their extras in chunk order, parks the
+    // largest probability (threshold) in conf and the ranking score in rank
+    for (int r = threadIdx.x; r < nr; r += blockDim.x) {
+      const int pos = row_pos[r];
+      ExtPartial a = ext_empty();
+      for (int c = 0; c < n_chunks; ++c) {
+        const Partial q = part[(int64_t)r * n_chunks + c];
+        const ConfExtra x = extra[(int64_t)r * n_chunks + c];
+        ext_merge(a, ExtPartial{q.m, q.idx, q.s, x.m2, x.t});
+      }
+      if (pos >= 0 && pos < B * L) {
+        const double p1 = 1.0 / a.s;
+        double sc;
+        if (score == DLLM_SCORE_TOP_K_MARGIN) sc = (1.0 - exp((double)a.m2 - (double)a.m)) * p1;
+        else sc = a.t * p1 - log(a.s);   // neg_entropy: sum p log p = t / s - log s
+        conf[pos] = (float)p1;
+        rank[pos] = (float)sc;
+        sel[pos] = a.idx + vocab_offset;
+      }
+    }
+  } else if (n_chunks > kMergeSerial) {
     for (int r = w; r < nr; r += nw) {
       const Partial* pr = part + (int64_t)r * n_chunks;
       const int pos = row_pos[r];
@@ -312,6 +439,7 @@ __global__ void __launch_bounds__(1024) unmask_select_kernel(Partial* part, int 
     const bool masked = b == w ? mk0 : (valid && mask[p] != 0);
     const unsigned mball = __ballot_sync(0xffffffffu, masked);
     const float c = masked ? conf[p] : 0.f;
+    const float rk = masked ? (extra ? rank[p] : c) : 0.f;   // the ranking score (the threshold counts c)
     const int cand = masked ? sel[p] : -1;
     __syncwarp();
     const int m = __popc(mball);
@@ -325,19 +453,19 @@ __global__ void __launch_bounds__(1024) unmask_select_kernel(Partial* part, int 
         kt = min(m, max(floor_k, min(k_max, above)));
       }
     }
-    int rank = 0;
+    int rnk = 0;
     for (int j = 0; j < 32; ++j) {
-      const float cj = __shfl_sync(0xffffffffu, c, j);
-      if (((mball >> j) & 1u) && (cj > c || (cj == c && j < lane))) ++rank;
+      const float rj = __shfl_sync(0xffffffffu, rk, j);
+      if (((mball >> j) & 1u) && (rj > rk || (rj == rk && j < lane))) ++rnk;
     }
-    const bool chosen = masked && rank < kt;
+    const bool chosen = masked && rnk < kt;
     if (valid) {
       sel[b * L + lane] = -1;
       conf[b * L + lane] = c;
     }
     __syncwarp();
     if (chosen) {
-      sel[b * L + rank] = lane;
+      sel[b * L + rnk] = lane;
       tokens[p] = cand;
       mask[p] = 0;
       if (cfg) {
@@ -376,9 +504,38 @@ size_t unmask_partials_bytes(int max_rows, int n_chunks) {
   return (size_t)max(max_rows, 1) * (size_t)n_chunks * sizeof(Partial);
 }
 
+size_t unmask_extras_bytes(int score, int max_rows, int n_chunks, int B, int L) {
+  if (score == DLLM_SCORE_LOW_CONFIDENCE) return 0;
+  const size_t ex = ((size_t)max(max_rows, 1) * (size_t)n_chunks * sizeof(ConfExtra) + 255) & ~size_t(255);
+  return ex + (size_t)B * L * sizeof(float);
+}
+
 int launch_unmask(const UnmaskArgs& a, cudaStream_t s) {
   const int chunk = ((a.V + a.n_chunks - 1) / a.n_chunks + 7) & ~7;
-  if (a.max_rows > 0 && !a.partials_ready) {
+  const bool ext = a.score != DLLM_SCORE_LOW_CONFIDENCE;
+  ConfExtra* extra = nullptr;
+  float* rank = nullptr;
+  if (ext) {
+    DLLM_REQUIRE(a.extras != nullptr && !a.partials_ready, DLLM_ERR_INVALID_ARG,
+                 "unmask: the position scores need their scratch and the separate reduction");
+    extra = static_cast<ConfExtra*>(a.extras);
+    const size_t ex = ((size_t)max(a.max_rows, 1) * (size_t)a.n_chunks * sizeof(ConfExtra) + 255) & ~size_t(255);
+    rank = reinterpret_cast<float*>(static_cast<char*>(a.extras) + ex);
+  }
+  if (a.max_rows > 0 && ext) {
+    dim3 grid(a.max_rows, a.n_chunks);
+    Partial* part = static_cast<Partial*>(a.partials);
+    if (a.dtype == DLLM_BF16) {
+      const __nv_bfloat16* z = static_cast<const __nv_bfloat16*>(a.logits);
+      if (a.cfg) launch_pdl((unmask_reduce_ext_kernel<__nv_bfloat16, true>), grid, 256, 0, s, z, a.n_rows, a.max_rows, a.V, chunk, a.cfg_scale, part, extra, a.n_chunks);
+      else launch_pdl((unmask_reduce_ext_kernel<__nv_bfloat16, false>), grid, 256, 0, s, z, a.n_rows, a.max_rows, a.V, chunk, a.cfg_scale, part, extra, a.n_chunks);
+    } else {
+      const float* z = static_cast<const float*>(a.logits);
+      if (a.cfg) launch_pdl((unmask_reduce_ext_kernel<float, true>), grid, 256, 0, s, z, a.n_rows, a.max_rows, a.V, chunk, a.cfg_scale, part, extra, a.n_chunks);
+      else launch_pdl((unmask_reduce_ext_kernel<float, false>), grid, 256, 0, s, z, a.n_rows, a.max_rows, a.V, chunk, a.cfg_scale, part, extra, a.n_chunks);
+    }
+    DLLM_CHECK_LAUNCH("unmask_reduce_ext_kernel");
+  } else if (a.max_rows > 0 && !a.partials_ready) {
     dim3 grid(a.max_rows, a.n_chunks);
     Partial* part = static_cast<Partial*>(a.partials);
     if (a.dtype == DLLM_BF16) {
@@ -401,11 +558,11 @@ int launch_unmask(const UnmaskArgs& a, cudaStream_t s) {
     }
     DLLM_CHECK_LAUNCH("unmask_reduce_kernel");
   }
-  const int threads = a.n_chunks > kMergeSerial ? 1024 : 32 * min(32, max(1, a.B));
+  const int threads = (a.n_chunks > kMergeSerial || ext) ? 1024 : 32 * min(32, max(1, a.B));
   launch_pdl(unmask_select_kernel, 1, threads, 0, s, static_cast<Partial*>(a.partials), a.n_chunks, a.row_pos, a.n_rows,
                                              a.max_rows, a.B, a.L, a.t, a.T_s, a.mode, a.tau, a.k_max, a.cfg, a.vocab_offset,
                                              a.tokens, a.mask, a.sel, a.nsel, a.conf, a.remaining, a.cond,
-                                             a.set_cond);
+                                             a.set_cond, a.score, (const ConfExtra*)extra, rank);
   DLLM_CHECK_LAUNCH("unmask_select_kernel");
   return DLLM_OK;
 }

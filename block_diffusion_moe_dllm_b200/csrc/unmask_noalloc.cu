@@ -62,8 +62,11 @@ extern "C" int dllm_unmask_noalloc(const dllm_unmask_desc* d, const void* logits
   DLLM_REQUIRE(d->mode == DLLM_UNMASK_FIXED || d->k_max >= 1, DLLM_ERR_INVALID_ARG, "unmask_noalloc: k_max must be >= 1");
   DLLM_REQUIRE(d->dtype == DLLM_BF16 || d->dtype == DLLM_F32, DLLM_ERR_INVALID_ARG, "unmask_noalloc: bad dtype");
   DLLM_REQUIRE(d->vocab_offset >= 0, DLLM_ERR_INVALID_ARG, "unmask_noalloc: negative vocab_offset");
+  DLLM_REQUIRE(d->score >= DLLM_SCORE_LOW_CONFIDENCE && d->score <= DLLM_SCORE_NEG_ENTROPY, DLLM_ERR_INVALID_ARG,
+               "unmask_noalloc: bad score %d", d->score);
   const int n_chunks = unmask_chunks(d->max_rows, d->V);
-  const size_t need = unmask_partials_bytes(d->max_rows, n_chunks);
+  const size_t part_bytes = (unmask_partials_bytes(d->max_rows, n_chunks) + 255) & ~size_t(255);
+  const size_t need = part_bytes + unmask_extras_bytes(d->score, d->max_rows, n_chunks, d->B, d->L);
   DLLM_REQUIRE(need <= kNoAllocScratchBytes, DLLM_ERR_UNSUPPORTED,
                "unmask_noalloc: %d rows x %d vocabulary chunks need %zu bytes of scratch, above the fixed %zu",
                d->max_rows, n_chunks, need, kNoAllocScratchBytes);
@@ -77,5 +80,7 @@ extern "C" int dllm_unmask_noalloc(const dllm_unmask_desc* d, const void* logits
   a.mask = mask; a.sel = sel; a.nsel = nsel; a.conf = conf; a.remaining = remaining;
   a.partials = scratch;
   a.n_chunks = n_chunks;
+  a.score = d->score;
+  a.extras = d->score != DLLM_SCORE_LOW_CONFIDENCE ? static_cast<char*>(scratch) + part_bytes : nullptr;
   return launch_unmask(a, stream);
 }

@@ -73,7 +73,7 @@ class DenoiseEngine:
             retain = bool(w.sprint and t == 0 and not commit)
         return bd.StepParams(t, w.T_s, w.mode, w.tau, w.k_max, w.cfg, w.cfg_scale, w.vocab_offset, w.vocab_len,
                              w.sprint, w.n_keep if w.sprint else 0, int(retain), int(commit), bd.ptr(self.sel),
-                             bd.ptr(self.nsel), bd.ptr(self.conf), bd.ptr(self.remaining))
+                             bd.ptr(self.nsel), bd.ptr(self.conf), bd.ptr(self.remaining), w.score)
 
     def set_block(self, tokens, mask):
         self.tokens.copy_(tokens)

@@ -57,6 +57,13 @@ extern "C" {
 #define DLLM_UNMASK_FIXED 0     /* k_t = ceil(m / (T_s - t)) */
 #define DLLM_UNMASK_THRESHOLD 1 /* k_t = min(m, max(ceil(m / (T_s - t)), min(k_max, #{c > tau}))) */
 
+/* How the still-masked positions are ranked ([M] "SPRINT 加速技术" names the strategies low_confidence, top_k_margin
+ * and neg_entropy; their formulas are not on the pages, these are the plain readings), from p = softmax(z). The
+ * threshold acceptance counts the positions whose largest probability exceeds tau whatever the ranking. */
+#define DLLM_SCORE_LOW_CONFIDENCE 0 /* p_(1), the largest probability */
+#define DLLM_SCORE_TOP_K_MARGIN 1   /* p_(1) - p_(2), the two largest probabilities over vocabulary entries */
+#define DLLM_SCORE_NEG_ENTROPY 2    /* sum_v p_v log p_v */
+
 /* ---------------------------------------------------------------------------------------------- B7 helpers */
 /* Library version string (host, static storage). */
 DLLM_API const char* dllm_version(void);
@@ -236,15 +243,15 @@ DLLM_API size_t dllm_moe_experts_workspace_size(const dllm_expert_desc* desc);
  * For each still-masked position r (n_rows of them; row r is flat position row_pos[r] = b * L + i of the
  * logical rows): z = logits[r] (with cfg: z = zu + cfg_scale * (zc - zu) in fp32, zc = logits[r],
  * zu = logits[n_rows + r]); candidate = vocab_offset + lowest argmax of z; c = 1 / sum_v exp(z_v - max z).
- * Per logical row b with m masked positions: k_t positions by c descending (c rounded to fp32; equal values ->
- * lower position) get their
+ * Per logical row b with m masked positions: k_t positions by the ranking score descending (c itself by default;
+ * rounded to fp32; equal values -> lower position) get their
  * candidate written to tokens and their mask cleared; with cfg the uncond row b + B gets the same update.
  *   logits [n_rows * (1 + cfg), V] in the storage type; row_pos [>= n_rows] int32: the still-masked flat
  *   positions of the logical rows in increasing order (row r of the logits belongs to the r-th masked position;
  *   every masked position must be listed, otherwise the results for the logical row are undefined);
  *   n_rows_dev [1] int32 (device count of masked positions; a count above max_rows is read as max_rows); tokens [B * (1 + cfg), L] int32; mask [B * (1 + cfg), L] uint8;
- *   sel [B, L] int32 (chosen positions in rank order, -1 after nsel[b]); nsel [B]; conf [B, L] fp32 (0 at
- *   unmasked positions); remaining [1] int32: masked positions left over all logical rows.
+ *   sel [B, L] int32 (chosen positions in rank order, -1 after nsel[b]); nsel [B]; conf [B, L] fp32 (the largest
+ *   probability; 0 at unmasked positions); remaining [1] int32: masked positions left over all logical rows.
  * Requires L <= 32 (one warp per block row for the selection) and B <= 1024.
  */
 typedef struct {
@@ -258,6 +265,7 @@ typedef struct {
   float cfg_scale;
   int32_t vocab_offset;
   int32_t dtype;
+  int32_t score;     /* DLLM_SCORE_*: the ranking of the positions */
 } dllm_unmask_desc;
 DLLM_API int dllm_unmask(const dllm_unmask_desc* desc, const void* logits, const int32_t* row_pos, const int32_t* n_rows_dev,
                 int32_t* tokens, uint8_t* mask, int32_t* sel, int32_t* nsel, float* conf, int32_t* remaining,
@@ -349,6 +357,7 @@ typedef struct {
   int32_t* nsel;      /* [B'] */
   float* conf;        /* [B', L] */
   int32_t* remaining; /* [1] */
+  int32_t score;      /* DLLM_SCORE_*: the ranking of the still-masked positions */
 } dllm_step_params;
 
 /*

@@ -475,7 +475,7 @@ def denoise_step(w, weights, caches, tokens, mask, t, keep=None):
     n = len(f["row_pos"])
     zc, zu = (f["logits"][:n], f["logits"][n:]) if w.cfg else (f["logits"], None)
     u = unmask(zc, f["row_pos"], tokens, mask, t, w.T_s, w.mode, w.tau, w.k_max, w.vocab_offset,
-               z_uncond=zu, cfg_scale=w.cfg_scale)
+               z_uncond=zu, cfg_scale=w.cfg_scale, score=SCORES[getattr(w, "score", 0)])
     u["forward"] = f
     return u
 

@@ -350,7 +350,7 @@ def test_prefix_retain(B, P, n_keep, cap_thin):
 
 # ------------------------------------------------------------------------------------------------ unmask
 def _unmask_case(B, L, V, masked_frac, t, T_s, mode, std, cfg=False, scale=2.0, tau=0.9, k_max=8, voff=0,
-                 dtype="bf16", seed=0, count_excess=None):
+                 dtype="bf16", seed=0, count_excess=None, score=0):
     """count_excess: the call's row capacity is exactly the masked count n and the device count says
     n + count_excess; the library must treat it as n (the logits hold n rows per half)."""
     g = np.random.default_rng(seed)
@@ -374,11 +374,11 @@ def _unmask_case(B, L, V, masked_frac, t, T_s, mode, std, cfg=False, scale=2.0, 
     nd = torch.tensor([n if count_excess is None else n + count_excess], dtype=torch.int32, device=DEV)
     cap = B * L if count_excess is None else n
     bd.unmask(logits, rp, nd, dt_, dm, sel, nsel, conf, rem, B, L, V, cap, t, T_s, DT[dtype], mode=mode, tau=tau,
-              k_max=k_max, cfg=int(cfg), cfg_scale=scale, vocab_offset=voff)
+              k_max=k_max, cfg=int(cfg), cfg_scale=scale, vocab_offset=voff, score=score)
     torch.cuda.synchronize()
     zl = to64(logits)
     u = O.unmask(zl[:n], row_pos, tokens, mask, t, T_s, mode, float(np.float32(tau)), k_max, voff,
-                 z_uncond=zl[n:] if cfg else None, cfg_scale=float(np.float32(scale)))
+                 z_uncond=zl[n:] if cfg else None, cfg_scale=float(np.float32(scale)), score=O.SCORES[score])
     check_unmask(u, conf.cpu().numpy(), nsel.cpu().numpy(), sel.cpu().numpy(), dt_.cpu().numpy(), dm.cpu().numpy(),
                  B, cfg)
     assert rem.item() == int(dm[:B].sum().item())
@@ -411,6 +411,20 @@ def test_unmask_last_step_takes_all():
 
 def test_unmask_f32():
     _unmask_case(1, 16, 1024, 1.0, 0, 4, bd.FIXED, 1.0, dtype="f32", seed=15)
+
+
+@pytest.mark.parametrize("score", [1, 2], ids=["top_k_margin", "neg_entropy"])
+@pytest.mark.parametrize("mode", [0, 1], ids=["fixed", "threshold"])
+def test_unmask_position_scores(score, mode):
+    """The other ranking strategies (top-2 margin, negated entropy): confidences (largest probability), counts,
+    chosen positions in rank order and written tokens against the oracle, on rows whose logits spread widely enough
+    that the threshold and the ranking both matter."""
+    _unmask_case(4, 32, 16384, 0.9, 0, 8, mode, 4.0, seed=40 + score + 2 * mode, score=score)
+
+
+@pytest.mark.parametrize("score", [1, 2], ids=["top_k_margin", "neg_entropy"])
+def test_unmask_position_scores_cfg_full_vocab(score):
+    _unmask_case(1, 32, 157184, 1.0, 1, 8, 1, 3.0, cfg=True, scale=2.0, seed=45 + score, score=score)
 
 
 @pytest.mark.parametrize("cfg", [False, True])

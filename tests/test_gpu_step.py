@@ -88,21 +88,21 @@ def _check_pass(w, eng, f, dtype):
 
 
 def _decisions_agree(w, u_or, eng, flag):
-    """Compare the unmask decisions where the oracle's choice is not a near-tie."""
+    """Compare the unmask decisions where the oracle's choice is not a near-tie (ranking by the workload's score,
+    threshold on the largest probability)."""
     Bl = w.B // 2 if w.cfg else w.B
-    g_tok = eng.tokens.cpu().numpy()
     g_mask = eng.mask.cpu().numpy()
     g_nsel = eng.nsel.cpu().numpy()
     clean = True
     for b in range(Bl):
         c = u_or["conf"][b]
-        m = u_or["sel"][b]
+        rk = u_or["rank"][b][c > 0]
         row_flag = flag[b * w.L:(b + 1) * w.L].any() or (w.cfg and flag[(b + Bl) * w.L:(b + Bl + 1) * w.L].any())
-        masked_c = np.sort(c[c > 0])[::-1]
+        ranked = np.sort(rk)[::-1]
         k = u_or["nsel"][b]
         near = False
-        if 0 < k < len(masked_c):
-            near = (masked_c[k - 1] - masked_c[k]) < E2E_CONF_MARGIN * masked_c[k - 1]
+        if 0 < k < len(ranked):
+            near = (ranked[k - 1] - ranked[k]) < E2E_CONF_MARGIN * max(abs(ranked[k - 1]), 1e-30)
         if w.mode == 1:
             near |= bool(np.any(np.abs(c[c > 0] - w.tau) < E2E_CONF_MARGIN))
         if near or row_flag:
@@ -174,6 +174,12 @@ def test_step_small_bf16_cfg_image_slice():
 def test_step_small_bf16_sprint():
     w = scaled(SMALL, B=3, P=96, sprint=1, keep_ratio=0.5)
     _one_pass(w, seed=4)
+
+
+@pytest.mark.parametrize("score", [1, 2], ids=["top_k_margin", "neg_entropy"])
+def test_step_small_bf16_position_scores(score):
+    _one_pass(scaled(SMALL, name=f"small-bf16-score{score}", mode=1, tau=0.9, k_max=8, T_s=16, lm_std=1.0,
+                     score=score), seed=6 + score)
 
 
 def test_step_small_bf16_threshold():

@@ -39,7 +39,7 @@ class AttnDesc(C.Structure):
 
 class RetainDesc(C.Structure):
     _fields_ = [("B", i32), ("Hkv", i32), ("d", i32), ("P", i32), ("cap", i32), ("n_keep", i32), ("cap_thin", i32),
-                ("dtype", i32)]
+                ("dtype", i32), ("alpha", f32), ("n_keep_img", i32)]
 
 
 class RouteDesc(C.Structure):
@@ -71,14 +71,15 @@ class Model(C.Structure):
 
 
 class State(C.Structure):
-    _fields_ = [("B", i32), ("L", i32), ("P", i32), ("cap", i32), ("cap_thin", i32), ("tokens", vp), ("mask", vp)]
+    _fields_ = [("B", i32), ("L", i32), ("P", i32), ("cap", i32), ("cap_thin", i32), ("tokens", vp), ("mask", vp),
+                ("prefix_conf", vp), ("prefix_modality", vp)]
 
 
 class StepParams(C.Structure):
     _fields_ = [("t", i32), ("T_s", i32), ("mode", i32), ("tau", f32), ("k_max", i32), ("cfg", i32),
                 ("cfg_scale", f32), ("vocab_offset", i32), ("vocab_len", i32), ("sprint", i32), ("n_keep", i32),
                 ("retain", i32), ("commit", i32), ("sel", vp), ("nsel", vp), ("conf", vp), ("remaining", vp),
-                ("score", i32)]
+                ("score", i32), ("sprint_alpha", f32), ("n_keep_img", i32)]
 
 
 class StepViews(C.Structure):
@@ -98,7 +99,7 @@ _SIGS = {
     "dllm_grouped_gemm_workspace_size": ([C.POINTER(GroupedGemmDesc)], sz),
     "dllm_block_attn": ([C.POINTER(AttnDesc), vp, vp, vp, vp, vp, vp, sz, vp], C.c_int),
     "dllm_block_attn_workspace_size": ([C.POINTER(AttnDesc)], sz),
-    "dllm_prefix_retain": ([C.POINTER(RetainDesc), vp, vp, vp, vp, vp, vp, vp, sz, vp], C.c_int),
+    "dllm_prefix_retain": ([C.POINTER(RetainDesc), vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], C.c_int),
     "dllm_prefix_retain_workspace_size": ([C.POINTER(RetainDesc)], sz),
     "dllm_moe_route": ([C.POINTER(RouteDesc), vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp], C.c_int),
     "dllm_moe_route_workspace_size": ([C.POINTER(RouteDesc)], sz),
@@ -214,13 +215,14 @@ def block_attn(q, k_cache, v_cache, out, B, Lq, Hq, Hkv, d, blk_len, q_pos0, n_k
 
 
 def prefix_retain(k_cache, v_cache, keep_pos, k_thin, v_thin, B, Hkv, d, P, cap, n_keep, cap_thin, dtype,
-                  scores=None, ws=None, stream=None):
+                  scores=None, conf=None, alpha=1.0, modality=None, n_keep_img=0, ws=None, stream=None):
     lib = load()
-    desc = RetainDesc(B, Hkv, d, P, cap, n_keep, cap_thin, dtype)
+    desc = RetainDesc(B, Hkv, d, P, cap, n_keep, cap_thin, dtype, alpha, n_keep_img)
     need = lib.dllm_prefix_retain_workspace_size(C.byref(desc))
     ws = (ws or Workspace(need, k_cache.device)).ensure(need)
-    return check(lib.dllm_prefix_retain(C.byref(desc), ptr(k_cache), ptr(v_cache), ptr(keep_pos), ptr(k_thin),
-                                        ptr(v_thin), ptr(scores), ws.addr, ws.nbytes, stream_handle(stream)))
+    return check(lib.dllm_prefix_retain(C.byref(desc), ptr(k_cache), ptr(v_cache), ptr(conf), ptr(modality),
+                                        ptr(keep_pos), ptr(k_thin), ptr(v_thin), ptr(scores), ws.addr, ws.nbytes,
+                                        stream_handle(stream)))
 
 
 def moe_route(h, w_router, bias, ids, gates, counts, offsets, perm, inv, Tk, H, E, k, dtype, scores=None, ws=None,

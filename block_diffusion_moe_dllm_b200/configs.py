@@ -44,6 +44,9 @@ class Workload:
     seed: int = 0
     wfmt: str = "bf16"    # "fp8": expert and LM-head weights as E4M3 codes with per-row fp32 scales
     score: int = 0        # ranking of the masked positions: 0 largest probability, 1 top-2 margin, 2 negated entropy
+    sprint_alpha: float = 1.0   # SPRINT importance = alpha * key norm + (1 - alpha) * confidence
+    n_img_prefix: int = 0       # > 0: the first n_img_prefix prefix positions are image tokens (modality counts)
+    img_keep_ratio: float = 1.0 # with image positions: keep ceil(ratio * n_img) of them, the rest of n_keep text
 
     @property
     def Tk(self) -> int:
@@ -59,7 +62,15 @@ class Workload:
 
     @property
     def n_keep(self) -> int:
-        return int(math.ceil(self.keep_ratio * self.P)) if self.sprint else self.P
+        if not self.sprint:
+            return self.P
+        if self.n_img_prefix:   # modality keep ratios: images at img_keep_ratio, text at keep_ratio
+            return self.n_keep_img + int(math.ceil(self.keep_ratio * (self.P - self.n_img_prefix)))
+        return int(math.ceil(self.keep_ratio * self.P))
+
+    @property
+    def n_keep_img(self) -> int:
+        return int(math.ceil(self.img_keep_ratio * self.n_img_prefix)) if self.n_img_prefix else 0
 
     @property
     def cap(self) -> int:

@@ -211,6 +211,11 @@ int validate_step(const dllm_model* m, const dllm_state* st, const dllm_step_par
   REQ(p->vocab_offset >= 0 && p->vocab_offset + vlen <= m->V, DLLM_ERR_SHAPE, "denoise_step: vocab slice out of range");
   if (p->sprint) {
     REQ(p->n_keep >= 1 && p->n_keep <= st->P && p->n_keep <= 8192, DLLM_ERR_SHAPE, "denoise_step: bad n_keep");
+    REQ(p->sprint_alpha >= 0.f && p->sprint_alpha <= 1.f, DLLM_ERR_INVALID_ARG, "denoise_step: sprint_alpha in [0, 1]");
+    REQ(p->sprint_alpha == 1.f || st->prefix_conf, DLLM_ERR_INVALID_ARG,
+        "denoise_step: sprint_alpha < 1 needs state->prefix_conf");
+    REQ(!st->prefix_modality || (p->n_keep_img >= 0 && p->n_keep_img <= p->n_keep), DLLM_ERR_INVALID_ARG,
+        "denoise_step: n_keep_img must be in [0, n_keep]");
     REQ(st->cap_thin >= p->n_keep + st->L, DLLM_ERR_SHAPE, "denoise_step: cap_thin too small");
     REQ(st->P <= 8192, DLLM_ERR_UNSUPPORTED, "denoise_step: SPRINT needs P <= 8192");
   }
@@ -467,14 +472,18 @@ size_t dllm_prefix_retain_workspace_size(const dllm_retain_desc* d) {
   return align256(align256(kStatusBytes) + retain_workspace_bytes(d->B, d->P));
 }
 
-int dllm_prefix_retain(const dllm_retain_desc* d, const void* k_cache, const void* v_cache, int32_t* keep_pos,
-                       void* k_thin, void* v_thin, float* scores, void* ws, size_t ws_bytes, cudaStream_t stream) {
+int dllm_prefix_retain(const dllm_retain_desc* d, const void* k_cache, const void* v_cache, const float* conf,
+                       const uint8_t* modality, int32_t* keep_pos, void* k_thin, void* v_thin, float* scores,
+                       void* ws, size_t ws_bytes, cudaStream_t stream) {
   REQ(d && k_cache && v_cache && keep_pos && k_thin && v_thin, DLLM_ERR_INVALID_ARG, "prefix_retain: NULL argument");
   REQ(d->B >= 1 && d->Hkv >= 1 && d->d >= 1 && d->P >= 1 && d->cap >= d->P, DLLM_ERR_SHAPE, "prefix_retain: bad shape");
   REQ(d->n_keep >= 1 && d->n_keep <= d->P && d->n_keep <= d->cap_thin, DLLM_ERR_SHAPE, "prefix_retain: bad n_keep");
   REQ(d->P <= 8192, DLLM_ERR_UNSUPPORTED, "prefix_retain: P > 8192");
   REQ(d->dtype == DLLM_BF16 || d->dtype == DLLM_F32, DLLM_ERR_INVALID_ARG, "prefix_retain: bad dtype");
   REQ((d->d * esize(d->dtype)) % 16 == 0, DLLM_ERR_UNSUPPORTED, "prefix_retain: row bytes must be a multiple of 16");
+  REQ(d->alpha >= 0.f && d->alpha <= 1.f, DLLM_ERR_INVALID_ARG, "prefix_retain: alpha must be in [0, 1]");
+  REQ(!modality || (d->n_keep_img >= 0 && d->n_keep_img <= d->n_keep), DLLM_ERR_INVALID_ARG,
+      "prefix_retain: n_keep_img must be in [0, n_keep]");
   int st = check_ws(ws, ws_bytes, dllm_prefix_retain_workspace_size(d));
   if (st) return st;
   Carver c(ws);
@@ -482,6 +491,8 @@ int dllm_prefix_retain(const dllm_retain_desc* d, const void* k_cache, const voi
   a.B = d->B; a.Hkv = d->Hkv; a.d = d->d; a.P = d->P; a.cap = d->cap; a.n_keep = d->n_keep; a.cap_thin = d->cap_thin;
   a.dtype = d->dtype; a.k = k_cache; a.v = v_cache; a.keep_pos = keep_pos; a.k_thin = k_thin; a.v_thin = v_thin;
   a.scores = scores; a.raw = c.take<float>(retain_workspace_bytes(d->B, d->P)); a.block_len = 0;
+  a.conf = conf; a.conf_stride = d->P; a.alpha = conf ? d->alpha : 1.f; a.modality = modality;
+  a.n_keep_img = d->n_keep_img;
   return launch_retain(a, stream);
 }
 
@@ -672,6 +683,8 @@ int denoise_step_impl(const dllm_model* m, const dllm_state* st, const dllm_step
       ra.B = st->B; ra.Hkv = m->Hkv; ra.d = m->d; ra.P = P; ra.cap = st->cap; ra.n_keep = p->n_keep;
       ra.cap_thin = st->cap_thin; ra.dtype = dt; ra.k = Ly.k_cache; ra.v = Ly.v_cache; ra.keep_pos = Ly.keep_pos;
       ra.k_thin = Ly.k_thin; ra.v_thin = Ly.v_thin; ra.scores = nullptr; ra.raw = s.retain_raw; ra.block_len = L;
+      ra.conf = p->sprint_alpha < 1.f ? st->prefix_conf : nullptr; ra.conf_stride = st->cap;
+      ra.alpha = p->sprint_alpha; ra.modality = st->prefix_modality; ra.n_keep_img = p->n_keep_img;
       TRY(launch_retain(ra, stream));
     }
     // QKV projection + RoPE; block K/V into the cache the attention reads (and the full cache on commit)
@@ -756,6 +769,9 @@ int denoise_step_impl(const dllm_model* m, const dllm_state* st, const dllm_step
   ua.set_cond = set_cond;
   ua.score = p->score;
   ua.extras = s.unmask_extras;
+  ua.conf_hist = st->prefix_conf;
+  ua.conf_hist_stride = st->cap;
+  ua.conf_hist_off = P;
   TRY(launch_unmask(ua, stream));
 #undef TRY
   return DLLM_OK;

@@ -59,6 +59,8 @@ struct UnmaskArgs {
   int set_cond = 0;
   int score = 0;                 // DLLM_SCORE_*: how positions are ranked (the threshold counts largest probabilities)
   void* extras = nullptr;        // score != 0: max_rows * n_chunks ConfExtra, then B * L floats of ranking scores
+  float* conf_hist = nullptr;    // nullable: accepted positions' confidences at conf_hist[row * stride + off + i]
+  int conf_hist_stride = 0, conf_hist_off = 0;
 };
 int unmask_chunks(int max_rows, int V);
 size_t unmask_partials_bytes(int max_rows, int n_chunks);
@@ -100,6 +102,11 @@ struct RetainArgs {
   float* scores;
   float* raw;  // workspace [B, P]
   int block_len;  // > 0: also write keep_pos[n_keep + i] = P + i for i < block_len
+  const float* conf = nullptr;        // [B, conf_stride] top-1 confidences of the prefix positions (nullable)
+  int conf_stride = 0;
+  float alpha = 1.0f;                 // importance = alpha * normalised key norm + (1 - alpha) * conf
+  const uint8_t* modality = nullptr;  // [P] 1 = image position (nullable: one selection over the prefix)
+  int n_keep_img = 0;                 // image positions kept (with a modality mask); the rest of n_keep are text
 };
 size_t retain_workspace_bytes(int B, int P);
 int launch_retain(const RetainArgs& a, cudaStream_t s);

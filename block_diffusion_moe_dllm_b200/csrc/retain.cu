@@ -1,6 +1,7 @@
-// SPRINT sparse prefix retention, key-norm term: per batch row, score every cached prefix position by the mean
-// over kv heads of the L2 norm of its key, keep the n_keep best (ties -> lower position) and compact their K/V
-// rows, in position order, into the thinned cache that the attention of the following steps reads.
+// SPRINT sparse prefix retention: per batch row, score every cached prefix position by the mean over kv heads of
+// the L2 norm of its key (optionally mixed with the position's top-1 confidence, and per modality), keep the n_keep
+// best (ties -> lower position) and compact their K/V rows, in position order, into the thinned cache that the
+// attention of the following steps reads.
 // Source: LLaDA2.0-Uni paper review, section "SPRINT — 학습 없는 추론 가속" (importance from the mean-normalised
 // key norm; pruning at the first step of each block), HF-mirror README, section "SPRINT 加速技术" (keep_ratio;
 // the prefix KV is computed once and reused).
@@ -36,25 +37,31 @@ __global__ void retain_scores_kernel(const T* __restrict__ k, int B, int Hkv, in
   if (lane == 0) raw[warp] = tot / (float)Hkv;
 }
 
-// One CTA (1024 threads) per batch row: threshold search, stable selection, keep_pos and normalised scores.
+// One CTA (1024 threads) per batch row: importance, threshold search, stable selection, keep_pos and scores.
+// Importance: the key norm, or with confidences alpha * (key norm / its mean over the prefix) + (1 - alpha) * conf
+// (fp32, non-negative). With a modality mask the image positions (mask 1) keep n_keep_img and the text positions the
+// rest, each its best ones (a modality with fewer positions than its count keeps them all and the other modality
+// keeps the rest, so exactly n_keep positions are kept).
 __global__ void retain_select_kernel(const float* __restrict__ raw, int P, int n_keep, int cap_thin,
-                                     int32_t* __restrict__ keep_pos, float* __restrict__ scores, int block_len) {
+                                     int32_t* __restrict__ keep_pos, float* __restrict__ scores, int block_len,
+                                     const float* __restrict__ conf, int conf_stride, float alpha,
+                                     const uint8_t* __restrict__ modality, int n_keep_img) {
   pdl_enter();
   __shared__ int red[32];
   __shared__ double dred[32];
   __shared__ int base;
-  __shared__ float rs[8192];     // this row's scores (P <= 8192): the 33 counting passes read shared memory
+  __shared__ float rs[8192];     // this row's importance (P <= 8192): the counting passes read shared memory
+  __shared__ uint8_t grp[8192];  // modality of each position (0 without a mask)
+  __shared__ uint32_t thr_s[2];
+  __shared__ int need_s[2];
   const int b = blockIdx.x, tid = threadIdx.x, lane = tid & 31, w = tid >> 5, nw = blockDim.x >> 5;
-  for (int i = tid; i < P; i += blockDim.x) rs[i] = raw[(int64_t)b * P + i];
+  for (int i = tid; i < P; i += blockDim.x) {
+    rs[i] = raw[(int64_t)b * P + i];
+    grp[i] = modality ? (modality[i] ? 1 : 0) : 0;
+  }
   __syncthreads();
-  const float* r = rs;
 
-  auto block_count = [&](uint32_t thr, bool strictly) -> int {
-    int c = 0;
-    for (int i = tid; i < P; i += blockDim.x) {
-      uint32_t u = __float_as_uint(r[i]);
-      c += strictly ? (u > thr) : (u >= thr);
-    }
+  auto block_sum_i = [&](int c) -> int {
     c = warp_sum_i(c);
     __syncthreads();
     if (lane == 0) red[w] = c;
@@ -63,52 +70,97 @@ __global__ void retain_select_kernel(const float* __restrict__ raw, int P, int n
     for (int i = 0; i < nw; ++i) t += red[i];
     return t;
   };
+  // positions of group g (g < 0: every position) whose bit pattern is >= thr (> thr when strictly)
+  auto block_count = [&](int g, uint32_t thr, bool strictly) -> int {
+    int c = 0;
+    for (int i = tid; i < P; i += blockDim.x) {
+      const uint32_t u = __float_as_uint(rs[i]);
+      c += (g < 0 || grp[i] == g) && (strictly ? (u > thr) : (u >= thr));
+    }
+    return block_sum_i(c);
+  };
 
-  // mean-normalised scores (optional output)
-  if (scores) {
+  // mean of the key norms (for the normalised scores and the mixed importance)
+  const bool mix = conf != nullptr && alpha != 1.0f;
+  if (scores || mix) {
     double s = 0.0;
-    for (int i = tid; i < P; i += blockDim.x) s += (double)r[i];
+    for (int i = tid; i < P; i += blockDim.x) s += (double)rs[i];
     s = warp_sum(s);
     if (lane == 0) dred[w] = s;
     __syncthreads();
     double tot = 0.0;
     for (int i = 0; i < nw; ++i) tot += dred[i];
     const float mean = (float)(tot / (double)P);
-    for (int i = tid; i < P; i += blockDim.x) scores[(int64_t)b * P + i] = r[i] / mean;
+    __syncthreads();
+    for (int i = tid; i < P; i += blockDim.x) {
+      float v = rs[i] / mean;
+      if (mix) v = alpha * v + (1.0f - alpha) * conf[(int64_t)b * conf_stride + i];
+      if (mix) rs[i] = fmaxf(v, 0.0f);
+      if (scores) scores[(int64_t)b * P + i] = mix ? rs[i] : v;
+    }
     __syncthreads();
   }
 
-  // T = largest bit pattern with #{u >= T} >= n_keep
-  uint32_t prefix = 0;
-  for (int bit = 31; bit >= 0; --bit) {
-    const uint32_t cand = prefix | (1u << bit);
-    if (block_count(cand, false) >= n_keep) prefix = cand;
+  // per selection group: the count it keeps, the largest bit pattern T with #{u >= T} >= count, and how many
+  // positions equal to T it takes
+  const int ng = modality ? 2 : 1;
+  int nk[2] = {n_keep, 0};
+  if (modality) {
+    const int n_img = block_count(1, 0u, false);
+    const int n_txt = P - n_img;
+    int ki = min(n_keep_img, n_img);
+    int kt = n_keep - ki;
+    if (kt > n_txt) { kt = n_txt; ki = n_keep - n_txt; }
+    nk[0] = ki;
+    nk[1] = kt;
   }
-  const int n_gt = block_count(prefix, true);
-  const int need_eq = n_keep - n_gt;
+  for (int gi = 0; gi < ng; ++gi) {
+    const int g = modality ? (gi == 0 ? 1 : 0) : -1;
+    uint32_t prefix = 0;
+    int need_eq = 0;
+    if (nk[gi] > 0) {
+      for (int bit = 31; bit >= 0; --bit) {
+        const uint32_t cand = prefix | (1u << bit);
+        if (block_count(g, cand, false) >= nk[gi]) prefix = cand;
+      }
+      need_eq = nk[gi] - block_count(g, prefix, true);
+    } else {
+      prefix = 0xffffffffu;   // no position has a larger pattern (importance is finite): nothing kept
+      need_eq = 0;
+    }
+    if (tid == 0) { thr_s[gi] = prefix; need_s[gi] = need_eq; }
+  }
+  __syncthreads();
 
-  // stable compaction: kept = (u > T) or (u == T and among the first need_eq equal positions)
-  if (tid == 0) base = 0;
-  __shared__ int eq_base;
-  if (tid == 0) eq_base = 0;
+  // stable compaction: kept = (u > T_g) or (u == T_g and among the first need_g equal positions of group g)
+  __shared__ int eq_base[2];
+  if (tid == 0) { base = 0; eq_base[0] = 0; eq_base[1] = 0; }
   __syncthreads();
   for (int c0 = 0; c0 < P; c0 += blockDim.x) {
     const int i = c0 + tid;
-    uint32_t u = i < P ? __float_as_uint(r[i]) : 0u;
-    const int is_eq = (i < P && u == prefix) ? 1 : 0;
-    // rank of this equal position among equal positions
-    unsigned bal = __ballot_sync(0xffffffffu, is_eq);
-    if (lane == 0) red[w] = __popc(bal);
-    __syncthreads();
-    int before = 0, tot = 0;
-    for (int k2 = 0; k2 < nw; ++k2) {
-      if (k2 < w) before += red[k2];
-      tot += red[k2];
+    const int gi = (i < P && modality) ? (grp[i] ? 0 : 1) : 0;
+    const uint32_t u = i < P ? __float_as_uint(rs[i]) : 0u;
+    const uint32_t T = thr_s[gi];
+    int keep = 0;
+    int tot_eq[2] = {0, 0};
+    for (int q = 0; q < ng; ++q) {
+      // rank of this position among the equal positions of selection group q
+      const int is_eq = (i < P && gi == q && u == thr_s[q] && thr_s[q] != 0xffffffffu) ? 1 : 0;
+      const unsigned bal = __ballot_sync(0xffffffffu, is_eq);
+      if (lane == 0) red[w] = __popc(bal);
+      __syncthreads();
+      int before = 0, tot = 0;
+      for (int k2 = 0; k2 < nw; ++k2) {
+        if (k2 < w) before += red[k2];
+        tot += red[k2];
+      }
+      const int eq_rank = eq_base[q] + before + __popc(bal & ((1u << lane) - 1u));
+      __syncthreads();
+      if (is_eq && eq_rank < need_s[q]) keep = 1;
+      tot_eq[q] = tot;
     }
-    const int eq_rank = eq_base + before + __popc(bal & ((1u << lane) - 1u));
-    __syncthreads();
-    const int keep = (i < P) && (u > prefix || (is_eq && eq_rank < need_eq));
-    bal = __ballot_sync(0xffffffffu, keep);
+    if (i < P && T != 0xffffffffu && u > T) keep = 1;
+    const unsigned bal = __ballot_sync(0xffffffffu, keep);
     if (lane == 0) red[w] = __popc(bal);
     __syncthreads();
     int kb = 0, ktot = 0;
@@ -120,7 +172,8 @@ __global__ void retain_select_kernel(const float* __restrict__ raw, int P, int n
     __syncthreads();
     if (tid == 0) {
       base += ktot;
-      eq_base += tot;
+      eq_base[0] += tot_eq[0];
+      eq_base[1] += tot_eq[1];
     }
     __syncthreads();
   }
@@ -164,7 +217,8 @@ int launch_retain(const RetainArgs& a, cudaStream_t s) {
   else
     launch_pdl(retain_scores_kernel<float>, blocks, 256, 0, s, (const float*)a.k, a.B, a.Hkv, a.d, a.P, a.cap, a.raw);
   DLLM_CHECK_LAUNCH("retain_scores_kernel");
-  launch_pdl(retain_select_kernel, a.B, 1024, 0, s, a.raw, a.P, a.n_keep, a.cap_thin, a.keep_pos, a.scores, a.block_len);
+  launch_pdl(retain_select_kernel, a.B, 1024, 0, s, a.raw, a.P, a.n_keep, a.cap_thin, a.keep_pos, a.scores, a.block_len,
+             a.conf, a.conf_stride, a.alpha, a.modality, a.n_keep_img);
   DLLM_CHECK_LAUNCH("retain_select_kernel");
   const int64_t copies = (int64_t)a.B * a.Hkv * a.n_keep;
   if (copies > 0) {

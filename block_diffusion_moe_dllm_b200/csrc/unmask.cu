@@ -361,7 +361,8 @@ __global__ void __launch_bounds__(1024) unmask_select_kernel(Partial* part, int 
                                      float tau, int k_max, int cfg, int vocab_offset, int32_t* tokens, uint8_t* mask,
                                      int32_t* sel, int32_t* nsel, float* conf, int32_t* remaining,
                                      cudaGraphConditionalHandle cond, int set_cond, int score,
-                                     const ConfExtra* __restrict__ extra, float* __restrict__ rank) {
+                                     const ConfExtra* __restrict__ extra, float* __restrict__ rank,
+                                     float* __restrict__ conf_hist, int hist_stride, int hist_off) {
   pdl_enter();
   __shared__ int rem_w[32];
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, nw = blockDim.x >> 5;
@@ -472,6 +473,10 @@ __global__ void __launch_bounds__(1024) unmask_select_kernel(Partial* part, int 
         tokens[p + B * L] = cand;
         mask[p + B * L] = 0;
       }
+      if (conf_hist) {   // the accepted position's confidence, for the importance of later SPRINT selections
+        conf_hist[(int64_t)b * hist_stride + hist_off + lane] = c;
+        if (cfg) conf_hist[(int64_t)(b + B) * hist_stride + hist_off + lane] = c;
+      }
     }
     if (lane == 0) {
       nsel[b] = kt;
@@ -562,7 +567,8 @@ int launch_unmask(const UnmaskArgs& a, cudaStream_t s) {
   launch_pdl(unmask_select_kernel, 1, threads, 0, s, static_cast<Partial*>(a.partials), a.n_chunks, a.row_pos, a.n_rows,
                                              a.max_rows, a.B, a.L, a.t, a.T_s, a.mode, a.tau, a.k_max, a.cfg, a.vocab_offset,
                                              a.tokens, a.mask, a.sel, a.nsel, a.conf, a.remaining, a.cond,
-                                             a.set_cond, a.score, (const ConfExtra*)extra, rank);
+                                             a.set_cond, a.score, (const ConfExtra*)extra, rank, a.conf_hist,
+                                             a.conf_hist_stride, a.conf_hist_off);
   DLLM_CHECK_LAUNCH("unmask_select_kernel");
   return DLLM_OK;
 }

@@ -52,7 +52,17 @@ class DenoiseEngine:
                               bd.ptr(weights["w_lm_scale"]) if fp8 else None)
         self.tokens = torch.zeros((w.B, w.L), dtype=torch.int32, device=device)
         self.mask = torch.ones((w.B, w.L), dtype=torch.uint8, device=device)
-        self.state = bd.State(w.B, w.L, w.P, self.cap, self.cap_thin, bd.ptr(self.tokens), bd.ptr(self.mask))
+        # per-position top-1 confidences of the cache (prompt positions 1) and the prefix modality, for SPRINT's
+        # mixed importance and modality counts
+        self.prefix_conf = None
+        self.prefix_modality = None
+        if w.sprint and w.sprint_alpha < 1.0:
+            self.prefix_conf = torch.ones((w.B, self.cap), dtype=torch.float32, device=device)
+        if w.sprint and w.n_img_prefix:
+            self.prefix_modality = torch.zeros(self.cap, dtype=torch.uint8, device=device)
+            self.prefix_modality[: w.n_img_prefix] = 1
+        self.state = bd.State(w.B, w.L, w.P, self.cap, self.cap_thin, bd.ptr(self.tokens), bd.ptr(self.mask),
+                              bd.ptr(self.prefix_conf), bd.ptr(self.prefix_modality))
         Bl = w.B // 2 if w.cfg else w.B
         self.sel = torch.full((Bl, w.L), -1, dtype=torch.int32, device=device)
         self.nsel = torch.zeros(Bl, dtype=torch.int32, device=device)
@@ -73,7 +83,8 @@ class DenoiseEngine:
             retain = bool(w.sprint and t == 0 and not commit)
         return bd.StepParams(t, w.T_s, w.mode, w.tau, w.k_max, w.cfg, w.cfg_scale, w.vocab_offset, w.vocab_len,
                              w.sprint, w.n_keep if w.sprint else 0, int(retain), int(commit), bd.ptr(self.sel),
-                             bd.ptr(self.nsel), bd.ptr(self.conf), bd.ptr(self.remaining), w.score)
+                             bd.ptr(self.nsel), bd.ptr(self.conf), bd.ptr(self.remaining), w.score, w.sprint_alpha,
+                             w.n_keep_img)
 
     def set_block(self, tokens, mask):
         self.tokens.copy_(tokens)

@@ -168,21 +168,29 @@ DLLM_API size_t dllm_block_attn_workspace_size(const dllm_attn_desc* desc);
 
 /* ---------------------------------------------------------------------------------------------- B2 SPRINT */
 /*
- * SPRINT sparse prefix retention ([R] "SPRINT — 학습 없는 추론 가속"; [M] "SPRINT 加速技术", keep_ratio), key-norm
- * term: per row b, score_i = mean over kv heads of ||K[b, h, i, :]||_2 divided by its mean over i < P; the
- * n_keep highest-scoring positions are kept (ties -> lower position), listed in increasing position in
- * keep_pos[b, 0:n_keep], and their K/V rows are copied, in that order, to rows [0, n_keep) of k_thin / v_thin.
+ * SPRINT sparse prefix retention ([R] "SPRINT — 학습 없는 추론 가속"; [M] "SPRINT 加速技术", keep_ratio and the
+ * modality keep ratios): per row b, the key norm l_i = mean over kv heads of ||K[b, h, i, :]||_2, normalised by its
+ * mean over i < P (l~_i); the importance s_i = alpha l~_i + (1 - alpha) conf[b, i] (alpha = 1 or conf == NULL: the
+ * key-norm term alone; the page's alpha is 0.5, conf the position's top-1 confidence). The n_keep highest-importance
+ * positions are kept (ties -> lower position), listed in increasing position in keep_pos[b, 0:n_keep], and their K/V
+ * rows are copied, in that order, to rows [0, n_keep) of k_thin / v_thin. With modality != NULL ([P] uint8, 1 =
+ * image position) n_keep_img of them are image positions and the rest text positions, each the best of its
+ * modality (a modality with fewer positions than its count keeps all of them and the other keeps the rest).
  *   k_cache, v_cache [B, Hkv, cap, d];  k_thin, v_thin [B, Hkv, cap_thin, d];  keep_pos [B, cap_thin] int32
- *   scores [B, P] fp32 (nullable): the mean-normalised scores.
- * Requires n_keep <= P <= 8192 and n_keep <= cap_thin.
+ *   conf [B, P] fp32 (nullable); modality [P] uint8 (nullable);
+ *   scores [B, P] fp32 (nullable): the importance (the mean-normalised key norm without confidences).
+ * Requires n_keep <= P <= 8192, n_keep <= cap_thin, 0 <= alpha <= 1, 0 <= n_keep_img <= n_keep.
  */
 typedef struct {
   int32_t B, Hkv, d, P, cap;
   int32_t n_keep, cap_thin;
   int32_t dtype;
+  float alpha;
+  int32_t n_keep_img;
 } dllm_retain_desc;
-DLLM_API int dllm_prefix_retain(const dllm_retain_desc* desc, const void* k_cache, const void* v_cache, int32_t* keep_pos,
-                       void* k_thin, void* v_thin, float* scores, void* ws, size_t ws_bytes, cudaStream_t stream);
+DLLM_API int dllm_prefix_retain(const dllm_retain_desc* desc, const void* k_cache, const void* v_cache,
+                       const float* conf, const uint8_t* modality, int32_t* keep_pos, void* k_thin, void* v_thin,
+                       float* scores, void* ws, size_t ws_bytes, cudaStream_t stream);
 DLLM_API size_t dllm_prefix_retain_workspace_size(const dllm_retain_desc* desc);
 
 /* ---------------------------------------------------------------------------------------------- B3 router */
@@ -336,6 +344,10 @@ typedef struct {
   int32_t cap_thin;  /* rows of the thinned caches, >= n_keep + L */
   int32_t* tokens;   /* [B, L] */
   uint8_t* mask;     /* [B, L] 1 = still masked */
+  float* prefix_conf;              /* [B, cap] (nullable): top-1 confidence of every cache position; each denoising
+                                      pass writes the confidences of the positions it accepts at P + i, SPRINT
+                                      selection reads [0, P) when sprint_alpha < 1 (prompt positions: the caller's) */
+  const uint8_t* prefix_modality;  /* [cap] (nullable): 1 = image position, for the modality keep counts */
 } dllm_state;
 
 typedef struct {
@@ -358,6 +370,8 @@ typedef struct {
   float* conf;        /* [B', L] */
   int32_t* remaining; /* [1] */
   int32_t score;      /* DLLM_SCORE_*: the ranking of the still-masked positions */
+  float sprint_alpha;   /* SPRINT importance mix (1: key norm alone; needs state->prefix_conf otherwise) */
+  int32_t n_keep_img;   /* with state->prefix_modality: image positions among the n_keep kept */
 } dllm_step_params;
 
 /*

@@ -160,20 +160,52 @@ def prefix_scores(k_prefix):
     return l / l.mean()
 
 
-def prefix_retain(k_prefix, ratio, n_keep=None):
-    """Kept prefix positions, in position order: the ceil(ratio * P) largest l~_i (or n_keep of them when
-    given), ties -> lower position.
-
-    Returns (keep_pos [n_keep] int64, scores [P], margin) where margin is the score gap between the last kept
-    and the first dropped position (inf when nothing is dropped)."""
+def prefix_importance(k_prefix, conf=None, alpha=1.0):
+    """[R] "SPRINT": importance of prefix position i mixing the mean-normalised key norm l~_i with the top-1
+    confidence c_i, alpha = 0.5 on the page (the formula itself was lost in extraction; the plain reading of the
+    surrounding prose is the convex combination s_i = alpha l~_i + (1 - alpha) c_i). alpha = 1 (or no confidences)
+    is the key-norm term alone. k_prefix [Hkv, P, d], conf [P] -> s [P]."""
     sc = prefix_scores(k_prefix)
+    if conf is None or alpha == 1.0:
+        return sc
+    return alpha * sc + (1.0 - alpha) * f64(conf)
+
+
+def prefix_retain(k_prefix, ratio, n_keep=None, conf=None, alpha=1.0, modality=None, n_keep_img=None):
+    """Kept prefix positions, in position order. Without modality: the ceil(ratio * P) (or n_keep) positions of
+    highest importance, ties -> lower position. With a modality mask ([M] "SPRINT 加速技术": modality-level keep
+    ratios; [R] "SPRINT": image tokens are pruned more than text tokens): n_keep_img of the image positions
+    (modality 1) and n_keep - n_keep_img of the text positions (modality 0), each the highest-importance ones of
+    its modality, ties -> lower position.
+
+    Returns (keep_pos [n_keep] int64, importance [P], margin) where margin is the smallest gap, within each
+    modality, between the last kept and the first dropped position (inf when nothing is dropped)."""
+    sc = prefix_importance(k_prefix, conf, alpha)
     P = sc.shape[0]
     if n_keep is None:
         n_keep = int(math.ceil(ratio * P))
-    order = sorted(range(P), key=lambda i: (-sc[i], i))
-    keep = np.array(sorted(order[:n_keep]), dtype=np.int64)
-    margin = sc[order[n_keep - 1]] - sc[order[n_keep]] if n_keep < P else np.inf
-    return keep, sc, margin
+    if modality is None:
+        groups = [(list(range(P)), n_keep)]
+    else:
+        # a modality with fewer positions than its count keeps them all and the other keeps the rest (n_keep kept)
+        mod = np.asarray(modality).astype(bool)
+        img = [i for i in range(P) if mod[i]]
+        txt = [i for i in range(P) if not mod[i]]
+        ki = min(n_keep_img, len(img))
+        kt = n_keep - ki
+        if kt > len(txt):
+            kt = len(txt)
+            ki = n_keep - kt
+        groups = [(img, ki), (txt, kt)]
+    keep, margin = [], np.inf
+    for pos, nk in groups:
+        order = sorted(pos, key=lambda i: (-sc[i], i))
+        keep += order[:nk]
+        if 0 < nk < len(order):
+            margin = min(margin, sc[order[nk - 1]] - sc[order[nk]])
+        elif nk == 0 and order:
+            margin = min(margin, np.inf)
+    return np.array(sorted(keep), dtype=np.int64), sc, margin
 
 
 def sigmoid(x):
@@ -489,10 +521,16 @@ def commit_block(w, weights, caches, tokens, keep=None):
     return f["block_k"], f["block_v"]
 
 
-def sprint_keep(w, caches):
-    """SPRINT selection at the first step of a block: per layer, per row, kept prefix positions."""
+def sprint_keep(w, caches, conf=None, modality=None):
+    """SPRINT selection at the first step of a block: per layer, per row, kept prefix positions (conf [B, P] and
+    modality [P] as in prefix_retain, with the workload's alpha and keep counts)."""
     keep = []
+    alpha = getattr(w, "sprint_alpha", 1.0)
+    n_img = getattr(w, "n_keep_img", None)
     for li in range(len(caches)):
         kc = f64(caches[li][0])
-        keep.append([prefix_retain(kc[b][:, : w.P, :], w.keep_ratio)[0] for b in range(w.B)])
+        keep.append([prefix_retain(kc[b][:, : w.P, :], w.keep_ratio, n_keep=w.n_keep,
+                                   conf=None if conf is None else conf[b][: w.P], alpha=alpha,
+                                   modality=None if modality is None else modality[: w.P], n_keep_img=n_img)[0]
+                     for b in range(w.B)])
     return keep

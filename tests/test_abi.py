@@ -143,9 +143,9 @@ def test_unmask_rejects_bad_arguments(lib):
 
 def test_retain_rejects_bad_arguments(lib):
     d = bd.RetainDesc(8, 4, 128, 4096, 4128, 0, 2080, bd.BF16)
-    assert lib.dllm_prefix_retain(C.byref(d), *([FAKE] * 6), FAKE, 1 << 30, None) == bd.ERR_SHAPE
+    assert lib.dllm_prefix_retain(C.byref(d), FAKE, FAKE, None, None, *([FAKE] * 4), FAKE, 1 << 30, None) == bd.ERR_SHAPE
     d.n_keep, d.P, d.cap = 2048, 9000, 9100
-    assert lib.dllm_prefix_retain(C.byref(d), *([FAKE] * 6), FAKE, 1 << 30, None) == bd.ERR_UNSUPPORTED
+    assert lib.dllm_prefix_retain(C.byref(d), FAKE, FAKE, None, None, *([FAKE] * 4), FAKE, 1 << 30, None) == bd.ERR_UNSUPPORTED
 
 
 def test_step_rejects_bad_model(lib):

@@ -348,6 +348,41 @@ def test_prefix_retain(B, P, n_keep, cap_thin):
         assert torch.equal(kt[b, :, :n_keep], kc[b][:, idx]) and torch.equal(vt[b, :, :n_keep], vc[b][:, idx])
 
 
+@pytest.mark.parametrize("B,P,n_keep,n_img,n_keep_img,alpha", [(2, 300, 150, 200, 100, 0.5), (1, 4096, 2048, 2560, 1536, 0.5),
+                                                             (2, 96, 60, 40, 40, 0.0), (3, 64, 40, 50, 30, 1.0),
+                                                             (1, 40, 30, 10, 20, 0.5)])
+def test_prefix_retain_mixed_importance_and_modality(B, P, n_keep, n_img, n_keep_img, alpha):
+    """SPRINT selection with the importance alpha l~ + (1 - alpha) c and per-modality counts (the first n_img
+    positions are image tokens): kept positions against the oracle wherever each modality's selection margin is
+    clear, exactly n_keep of them, n_keep_img images (or all images with the rest text when there are fewer)."""
+    Hkv, d = 4, 128
+    cap = P + 16
+    kc = synth.normal((B, Hkv, cap, d), 1.0, 9, "pmk", DEV)
+    vc = synth.normal((B, Hkv, cap, d), 1.0, 9, "pmv", DEV)
+    conf = synth.uniform((B, P), 0.0, 1.0, 9, "pmc", DEV)
+    mod = torch.zeros(P, dtype=torch.uint8, device=DEV)
+    mod[:n_img] = 1
+    keep = torch.full((B, n_keep + 4), -1, dtype=torch.int32, device=DEV)
+    kt = torch.zeros((B, Hkv, n_keep + 4, d), dtype=torch.bfloat16, device=DEV)
+    vt = torch.zeros_like(kt)
+    sc = torch.zeros((B, P), dtype=torch.float32, device=DEV)
+    bd.prefix_retain(kc, vc, keep, kt, vt, B, Hkv, d, P, cap, n_keep, n_keep + 4, bd.BF16, scores=sc, conf=conf,
+                     alpha=alpha, modality=mod, n_keep_img=n_keep_img)
+    torch.cuda.synchronize()
+    m = mod.cpu().numpy()
+    for b in range(B):
+        o_keep, o_sc, margin = O.prefix_retain(to64(kc[b, :, :P]), None, n_keep=n_keep, conf=to64(conf[b]),
+                                               alpha=alpha, modality=m, n_keep_img=n_keep_img)
+        g_keep = keep[b, :n_keep].cpu().numpy()
+        assert np.allclose(to64(sc[b]), o_sc, rtol=2e-6, atol=1e-7)
+        assert len(o_keep) == n_keep and np.all(np.diff(g_keep) > 0) and g_keep.min() >= 0 and g_keep.max() < P
+        assert int(m[g_keep].sum()) == int(m[o_keep].sum())
+        if margin > 1e-6 * np.max(o_sc):
+            assert np.array_equal(g_keep, o_keep)
+        idx = torch.from_numpy(g_keep.astype(np.int64)).to(DEV)
+        assert torch.equal(kt[b, :, :n_keep], kc[b][:, idx]) and torch.equal(vt[b, :, :n_keep], vc[b][:, idx])
+
+
 # ------------------------------------------------------------------------------------------------ unmask
 def _unmask_case(B, L, V, masked_frac, t, T_s, mode, std, cfg=False, scale=2.0, tau=0.9, k_max=8, voff=0,
                  dtype="bf16", seed=0, count_excess=None, score=0):

@@ -134,7 +134,11 @@ def _check_candidates(w, eng, u_or, f, flag):
 def _one_pass(w, seed=0, masked_fraction=1.0, t=0, random_gains=True):
     wt, caches, eng, tok0, mask0 = _setup(w, seed, masked_fraction, random_gains)
     hw, hc = _host(wt), _host_caches(caches, w.P)
-    keep = O.sprint_keep(w, hc) if w.sprint else None
+    keep = None
+    if w.sprint:
+        conf = eng.prefix_conf.cpu().numpy() if eng.prefix_conf is not None else None
+        mod = eng.prefix_modality.cpu().numpy() if eng.prefix_modality is not None else None
+        keep = O.sprint_keep(w, hc, conf=conf, modality=mod)
     eng.step(t)
     torch.cuda.synchronize()
     assert bd.status_check(eng.ws) == bd.OK
@@ -147,7 +151,10 @@ def _one_pass(w, seed=0, masked_fraction=1.0, t=0, random_gains=True):
             kp = eng.thin[l][2]
             for b in range(w.B):
                 got = kp[b, : w.n_keep].cpu().numpy()
-                _, sc, margin = O.prefix_retain(O.f64(hc[l][0][b]), None, n_keep=w.n_keep)
+                _, sc, margin = O.prefix_retain(O.f64(hc[l][0][b]), None, n_keep=w.n_keep,
+                                                conf=None if conf is None else conf[b][: w.P], alpha=w.sprint_alpha,
+                                                modality=None if mod is None else mod[: w.P],
+                                                n_keep_img=w.n_keep_img)
                 if margin > 1e-6 * sc.max():
                     assert np.array_equal(got, keep[l][b])
                 assert np.array_equal(kp[b, w.n_keep: w.n_keep + w.L].cpu().numpy(), np.arange(w.P, w.P + w.L))
@@ -180,6 +187,18 @@ def test_step_small_bf16_sprint():
 def test_step_small_bf16_position_scores(score):
     _one_pass(scaled(SMALL, name=f"small-bf16-score{score}", mode=1, tau=0.9, k_max=8, T_s=16, lm_std=1.0,
                      score=score), seed=6 + score)
+
+
+def test_step_small_bf16_sprint_mixed_modality():
+    """SPRINT with the mixed importance (alpha 0.5, prompt confidences 1) and modality counts: the first 64 of 96
+    prefix positions are image tokens, half of them kept, all text kept."""
+    w = scaled(SMALL, name="small-bf16-sprint-mixed", B=3, P=96, sprint=1, keep_ratio=1.0, sprint_alpha=0.5,
+               n_img_prefix=64, img_keep_ratio=0.5)
+    eng, _ = _one_pass(w, seed=9)
+    assert w.n_keep == 32 + 32
+    for l in range(w.n_layers):
+        kp = eng.thin[l][2][:, : w.n_keep].cpu().numpy()
+        assert np.all((kp < 64).sum(axis=1) == 32)
 
 
 def test_step_small_bf16_threshold():

@@ -601,3 +601,50 @@ def test_unmask_ranks_by_score_and_counts_by_probability():
     assert list(O.unmask(z, [0, 1], tok, msk, 0, 2, score="neg_entropy", **args)["sel"][0]) == [0]
     u = O.unmask(z, [0, 1], tok, msk, 0, 2, score="top_k_margin", **args)
     assert np.allclose(u["rank"][0], [0.60 - 0.39, 0.55 - 0.05]) and np.allclose(u["conf"][0], [0.60, 0.55])
+
+
+# ---------------------------------------------------------------------------------------------- SPRINT mixed score
+
+def test_prefix_importance_mixes_key_norm_and_confidence():
+    """s = alpha l~ + (1 - alpha) c: alpha = 1 is the key-norm term, alpha = 0 the confidence alone, alpha = 0.5
+    their mean (the hand-computed key norms of the kv-head pin: 30/23, 33/23, 6/23)."""
+    k = np.zeros((2, 3, 2))
+    k[0, 0] = (3, 4)
+    k[0, 1] = (2, 0)
+    k[1, 1] = (0, 3.5)
+    k[1, 2] = (1, 0)
+    c = np.array([0.9, 0.1, 0.5])
+    assert np.allclose(O.prefix_importance(k, c, 1.0), [30 / 23, 33 / 23, 6 / 23], atol=1e-15)
+    assert np.allclose(O.prefix_importance(k, c, 0.0), c, atol=1e-15)
+    half = O.prefix_importance(k, c, 0.5)
+    assert np.allclose(half, [0.5 * 30 / 23 + 0.45, 0.5 * 33 / 23 + 0.05, 0.5 * 6 / 23 + 0.25], atol=1e-15)
+    keep, _, _ = O.prefix_retain(k, None, n_keep=1, conf=c, alpha=0.5)
+    assert list(keep) == [0]          # 1.102 > 0.767 > 0.380: the confidence moves the choice from 1 to 0
+
+
+def test_prefix_retain_per_modality_counts_brute_force():
+    """With a modality mask, n_keep_img image positions and n_keep - n_keep_img text positions are kept, each the
+    best of its modality (brute force over subsets), in position order."""
+    import itertools
+    Hkv, P, d = 2, 10, 4
+    k = rng.standard_normal((Hkv, P, d))
+    c = rng.uniform(size=P)
+    mod = np.array([1, 1, 0, 1, 0, 1, 1, 0, 0, 1])
+    sc = O.prefix_importance(k, c, 0.5)
+    for n_img, n_txt in [(3, 2), (6, 0), (0, 4), (2, 4)]:   # the mask has 6 image and 4 text positions
+        keep, _, _ = O.prefix_retain(k, None, n_keep=n_img + n_txt, conf=c, alpha=0.5, modality=mod,
+                                     n_keep_img=n_img)
+        assert len(keep) == n_img + n_txt and list(keep) == sorted(keep)
+        assert int(mod[keep].sum()) == n_img
+        img = [i for i in range(P) if mod[i]]
+        best = max(itertools.combinations(img, n_img), key=lambda s: sorted([sc[i] for i in s]))
+        assert set(best) == {i for i in keep if mod[i]}
+
+
+def test_prefix_retain_modality_shortfall_moves_to_the_other_modality():
+    k = rng.standard_normal((1, 6, 4))
+    mod = np.array([1, 0, 1, 0, 0, 0])                # 2 image, 4 text positions
+    keep, _, _ = O.prefix_retain(k, None, n_keep=5, modality=mod, n_keep_img=4)
+    assert len(keep) == 5 and set(keep) >= {0, 2}      # both images kept, 3 of the 4 text positions
+    keep, _, _ = O.prefix_retain(k, None, n_keep=5, modality=mod, n_keep_img=0)
+    assert len(keep) == 5 and len(set(keep) & {0, 2}) == 1   # 4 text positions, then one image

@@ -299,6 +299,7 @@ def main():
     per_commit = bd.launch_count() - n0
     graph = eng.block_graph()
     graph_cond = graph.conditional
+    graph_note = graph.note
 
     def block():
         eng.tokens.copy_(tokens0)
@@ -392,7 +393,7 @@ def main():
                 "config": bench_config(w, world),
                 "timed_units": {"n": len(units), "unit_s": units, "steps_per_unit": args.steps},
                 "committed_tokens_per_s": committed,
-                "block_graph_conditional": graph_cond,
+                "block_graph_conditional": graph_cond if graph_cond else f"no: {graph_note}",
                 "passes_per_block": {"live": live, "launched": live if graph_cond else w.T_s,
                                      "rows_per_live_pass": [p["rows"] for p in passes if p["live"]]},
                 "active_experts_per_layer": {"mean": statistics.mean(act) if act else 0,

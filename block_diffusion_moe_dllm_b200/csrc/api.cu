@@ -835,6 +835,9 @@ const CondApi& cond_api() {
   return api;
 }
 
+// Why the last block graph was built without conditional nodes (CUresult codes), for dllm_last_error.
+static thread_local char g_cond_note[160] = "";
+
 // One IF node after `prev` (nullable) in `graph`; its body graph is returned in *body.
 bool add_if_node(cudaGraph_t graph, cudaGraphConditionalHandle cond, CUcontext ctx, cudaGraphNode_t prev,
                  cudaGraphNode_t* node, cudaGraph_t* body) {
@@ -849,8 +852,11 @@ bool add_if_node(cudaGraph_t graph, cudaGraphConditionalHandle cond, CUcontext c
   np.conditional.ctx = ctx;
   CUgraphNode n = nullptr;
   CUgraphNode dep = reinterpret_cast<CUgraphNode>(prev);
-  if (api.add_node(&n, reinterpret_cast<CUgraph>(graph), prev ? &dep : nullptr, prev ? 1 : 0, &np) != CUDA_SUCCESS)
+  const CUresult rc = api.add_node(&n, reinterpret_cast<CUgraph>(graph), prev ? &dep : nullptr, prev ? 1 : 0, &np);
+  if (rc != CUDA_SUCCESS) {
+    snprintf(g_cond_note, sizeof(g_cond_note), "conditional node refused: cuGraphAddNode returned %d", (int)rc);
     return false;
+  }
   *node = reinterpret_cast<cudaGraphNode_t>(n);
   *body = reinterpret_cast<cudaGraph_t>(np.conditional.phGraph_out[0]);
   return true;
@@ -896,10 +902,22 @@ int dllm_block_graph_create(const dllm_model* m, const dllm_state* st, const dll
   const CondApi& api = cond_api();
   CUcontext ctx = nullptr;
   cudaGraphConditionalHandle cond = 0;
-  bool use_cond = api.ctx_get && api.handle_create && api.add_node && api.ctx_get(&ctx) == CUDA_SUCCESS && ctx &&
-                  api.handle_create(reinterpret_cast<CUgraphConditionalHandle*>(&cond),
-                                    reinterpret_cast<CUgraph>(g->graph), ctx, 1,
-                                    CU_GRAPH_COND_ASSIGN_DEFAULT) == CUDA_SUCCESS;
+  bool use_cond = false;
+  g_cond_note[0] = 0;
+  if (!(api.ctx_get && api.handle_create && api.add_node)) {
+    snprintf(g_cond_note, sizeof(g_cond_note), "conditional nodes: driver entry points unavailable");
+  } else {
+    const CUresult rc0 = api.ctx_get(&ctx);
+    const CUresult rc1 = (rc0 == CUDA_SUCCESS && ctx)
+                             ? api.handle_create(reinterpret_cast<CUgraphConditionalHandle*>(&cond),
+                                                 reinterpret_cast<CUgraph>(g->graph), ctx, 1,
+                                                 CU_GRAPH_COND_ASSIGN_DEFAULT)
+                             : CUDA_ERROR_INVALID_CONTEXT;
+    use_cond = rc1 == CUDA_SUCCESS;
+    if (!use_cond)
+      snprintf(g_cond_note, sizeof(g_cond_note), "conditional handle refused: cuCtxGetCurrent %d, handle %d",
+               (int)rc0, (int)rc1);
+  }
   cudaGraphNode_t first = nullptr;
   cudaGraph_t first_body = nullptr;
   if (use_cond && !add_if_node(g->graph, cond, ctx, nullptr, &first, &first_body)) {
@@ -964,6 +982,8 @@ int dllm_block_graph_create(const dllm_model* m, const dllm_state* st, const dll
   if (e != cudaSuccess) return fail(e, "block_graph_create: cudaGraphInstantiate");
   g->passes = p->T_s;
   g->conditional = use_cond ? 1 : 0;
+  // leave the reason for a graph without conditions in the thread's last-error text (the call still succeeds)
+  if (!use_cond) dllm_host::set_error("block_graph_create: passes unconditional (%s)", g_cond_note);
   *out = g;
   return DLLM_OK;
 }

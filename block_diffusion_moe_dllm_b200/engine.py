@@ -169,6 +169,8 @@ class BlockGraph:
         bd.check(self.lib.dllm_block_graph_create(C.byref(eng.model), C.byref(eng.state), C.byref(p), eng.ws.addr,
                                                   eng.ws.nbytes, bd.stream_handle(capture_stream),
                                                   C.byref(self.handle)))
+        # why the passes are unconditional, when they are (the library leaves it in the last-error text)
+        self.note = "" if self.conditional else self.lib.dllm_last_error().decode()
 
     def launch(self, stream=None):
         return bd.check(self.lib.dllm_block_graph_launch(self.handle, bd.stream_handle(stream)))

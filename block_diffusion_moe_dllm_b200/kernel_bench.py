@@ -1,7 +1,7 @@
 """Per-kernel timing of the library's main calls at a workload's shapes (CUDA events, kernels launched alone).
 
     python -m block_diffusion_moe_dllm_b200.kernel_bench [--kernel lm_head|proj|experts|expert_gemms|unmask|attn|
-                                                          route|all]
+                                                          route|all|step]
                                                          [--workload NAME] [--reps N]
 
 Each line reports the mean time of one call, its algorithmic bytes (weights and activations it must move at
@@ -226,6 +226,33 @@ def bench_attn(w: Workload, reps, dev, stream):
     return _result("block_attn", t, nbytes, _flops({"keys": n_keys, "rows": w.B * w.L}, flops, t))
 
 
+def bench_step(w: Workload, reps, dev, stream):
+    """One whole denoising pass (dllm_denoise_step at the block's first step, every position masked) called from the
+    host, timed with CUDA events around `reps` passes (the block state reset before each), after one warm-up pass.
+    Also the command the pass's ncu launch list is taken with."""
+    from .engine import DenoiseEngine
+    wt = synth.make_weights(w, dev)
+    caches = synth.make_prefix_cache(w, dev)
+    tokens, mask = synth.make_block_state(w, dev)
+    eng = DenoiseEngine(w, wt, caches, dev)
+    eng.set_block(tokens, mask)
+    eng.step(0)
+    torch.cuda.synchronize()
+    n0 = bd.launch_count()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ts = []
+    for _ in range(reps):
+        eng.set_block(tokens, mask)
+        a.record(stream)
+        eng.step(0)
+        b.record(stream)
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b) / 1000.0)
+    t = sorted(ts)[len(ts) // 2]
+    return {"kernel": "denoise_pass", "us": t * 1e6, "launches_per_pass": (bd.launch_count() - n0) // max(reps, 1),
+            "rows": w.B * w.L, "layers": w.n_layers}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--kernel", default="all")
@@ -249,6 +276,8 @@ def main():
         out.append(bench_unmask(w, a.reps, dev, stream))
     if a.kernel in ("attn", "all"):
         out.append(bench_attn(w, a.reps, dev, stream))
+    if a.kernel == "step":
+        out.append(bench_step(w, a.reps, dev, stream))
     for r in out:
         print(json.dumps(r), flush=True)
 

@@ -92,18 +92,6 @@ __device__ __forceinline__ uint64_t sdesc_mn128(uint32_t addr, uint32_t lbo) {
   return d;
 }
 
-// D (TMEM) (+)= A (TMEM: 128 lanes = rows, two bf16 of K per 32-bit column) x B (shared memory descriptor).
-__device__ __forceinline__ void mma_bf16_tmem_a(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
-                                                uint32_t accumulate) {
-  uint32_t z = 0;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %5, %5, %5}, p;\n\t}" ::"r"(tmem_d),
-      "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(z)
-      : "memory");
-}
-
 // Integer division by the block length without the divide sequence (which would queue on the special-function unit
 // behind the softmax's exponentials): multiply by m = ceil(2^(31+s) / d), 2^(s-1) < d <= 2^s, and keep the bits
 // above 31 + s; exact for 0 <= n < 2^31 since n (m d - 2^(31+s)) < 2^(31+s) (Granlund and Montgomery, "Division by
@@ -154,19 +142,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
-
-// Each lane writes 32 consecutive 32-bit columns of its own TMEM lane (completion: tmem_st_wait).
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
-      "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
-      "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
-      : "memory");
-}
-__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 // Bulk copies between shared and global memory (the async proxy) for the split exchange.
 __device__ __forceinline__ void bulk_store_s2g(void* gdst, const void* ssrc, uint32_t bytes) {
@@ -371,7 +346,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const uint32_t tP = tS + g * 128;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_tmem_a(tO + g * 128, tP + kk * 8, sdesc_mn128(aV + kk * 2048, CHUNK), idesc_o,
+          tc::mma_bf16_tmem_a(tO + g * 128, tP + kk * 8, sdesc_mn128(aV + kk * 2048, CHUNK), idesc_o,
                           (j >= 2 || kk != 0) ? 1u : 0u);
         tc::mma_commit(&bar.o_full[g]);
         tc::mma_commit(&bar.kv_empty[s]);
@@ -487,7 +462,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
         // keys [64c, 64c + 64) -> columns [32c, 32c + 32): S there has been read (c = 0: this chunk's first half;
         // c = 1: chunk 0)
-        tmem_st32(tSg + 32 * c, pk);
+        tc::tmem_st32(tSg + 32 * c, pk);
       }
       // O_g holds the group's previous P V once that phase completes (every phase is waited in order, so the
       // parity is unambiguous: the next phase needs this group's P)
@@ -501,13 +476,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
           uint32_t r32[32];
 #pragma unroll
           for (int u = 0; u < 32; ++u) r32[u] = __float_as_uint(w[u] * alpha);
-          tmem_st32(tOg + 32 * c, r32);
+          tc::tmem_st32(tOg + 32 * c, r32);
         }
       }
       float rs0, rs1;
       upk2(rs2, rs0, rs1);
       l = l * alpha + (rs0 + rs1);
-      tmem_st_wait();
+      tc::tmem_st_wait();
       tc::fence_before_sync();
       tc::mbar_arrive(&bar.p_ready[grp]);
     }

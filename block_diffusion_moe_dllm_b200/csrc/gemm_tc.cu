@@ -40,9 +40,8 @@ constexpr int SMEM_LIMIT = 232448;
 struct Smem {
   uint64_t full[16];
   uint64_t empty[16];
-  uint64_t conv[16];                // FP8: operand slot's bf16 weight tile written (128 converter arrivals)
-  uint64_t bfull[16];               // FP8: operand slot's activation tile landed (TMA transaction bytes)
-  uint64_t mempty[16];              // FP8: operand slot free again (MMA commit)
+  uint64_t conv[16];                // FP8: A slot's 128 TMEM rows written (128 converter arrivals)
+  uint64_t mempty[16];              // FP8: A slot free again (MMA commit)
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t done;
@@ -348,34 +347,29 @@ __device__ __forceinline__ void epilogue_logits_conf(const KParams& p, const flo
   }
 }
 
-// FP8 weights: one stage's E4M3 tile (128 rows x 64 codes, row r at byte r * 64, as the TMA box lands it) into the
-// bf16 operand tile the MMA reads (row r at byte r * 128, its eight 16-byte chunks XOR-swizzled by r & 7, the layout
-// a 128-byte-swizzling TMA load produces). Every E4M3 value is exact in bf16 (3 mantissa bits, exponents 2^-9 ..
-// 2^8), so the tile holds the codes' values unscaled; the per-row scale is applied to the accumulator. 128 threads,
-// four 16-byte pieces each (consecutive threads read consecutive 16 bytes).
-__device__ __forceinline__ void convert_e4m3_tile(const uint8_t* raw, uint8_t* a_tile, int ct) {
+// FP8 weights: row r of one stage's E4M3 tile as 32 columns of bf16 pairs in TMEM lane r, the A operand the MMA
+// reads from tensor memory. The TMA box lands row r at byte r * 64 of the stage with 64-byte swizzling (its four
+// 16-byte pieces XOR-permuted by (r >> 1) & 3), so the eight rows a quarter-warp reads hit eight different bank
+// groups. Every E4M3 value is exact in bf16 (3 mantissa bits, exponents 2^-9 .. 2^8), so the tile holds the codes'
+// values unscaled; the per-row scale is applied to the accumulator.
+__device__ __forceinline__ void convert_e4m3_row_to_tmem(const uint8_t* raw, int row, uint32_t taddr) {
+  uint32_t o[32];
+  const int sw = (row >> 1) & 3;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int c = ct + 128 * i;
-    const int row = c >> 2, part = c & 3;
-    const uint4 q = *reinterpret_cast<const uint4*>(raw + row * 64 + part * 16);
+  for (int part = 0; part < 4; ++part) {
+    const uint4 q = *reinterpret_cast<const uint4*>(raw + row * 64 + ((part ^ sw) << 4));
     const uint32_t w[4] = {q.x, q.y, q.z, q.w};
-    uint32_t o[8];
 #pragma unroll
     for (int h = 0; h < 8; ++h) {
       const uint16_t pair = (uint16_t)(w[h >> 1] >> ((h & 1) * 16));
       uint32_t f16x2;
       asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(f16x2) : "h"(pair));
-      const __half2 hv = *reinterpret_cast<const __half2*>(&f16x2);
-      const float2 fv = __half22float2(hv);
+      const float2 fv = __half22float2(*reinterpret_cast<const __half2*>(&f16x2));
       const __nv_bfloat162 bv = __floats2bfloat162_rn(fv.x, fv.y);
-      o[h] = *reinterpret_cast<const uint32_t*>(&bv);
+      o[part * 8 + h] = *reinterpret_cast<const uint32_t*>(&bv);
     }
-    uint8_t* dst = a_tile + row * 128;
-    const int sw = row & 7;
-    *reinterpret_cast<uint4*>(dst + (((2 * part) ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-    *reinterpret_cast<uint4*>(dst + (((2 * part + 1) ^ sw) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
   }
+  tc::tmem_st32(taddr, o);
 }
 
 // Scale of tile row r of tile (g, mt) for FP8 weights: the row of W (or W2 for the extra group) it came from.
@@ -394,17 +388,17 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   constexpr int NT = F8 ? NUM_THREADS_F8 : NUM_THREADS;
   constexpr int B_BYTES = BN * BK * 2;
-  // bf16 weights: STAGES stages of [A weight tile][B activation tile]. FP8 weights: a deep ring of STAGES E4M3
-  // weight tiles (the HBM stream) and a shallow ring of MS operand slots [A bf16 tile][B activation tile] that the
-  // converter warps fill (activations come from L2, so two or three slots keep the MMA fed).
-  constexpr int MS = F8 ? (BN >= 128 ? 2 : 3) : 0;
+  // bf16 weights: STAGES stages of [A weight tile][B activation tile]. FP8 weights: STAGES stages of [E4M3 weight
+  // codes][B activation tile] (half the weight bytes, so a deeper ring), and MS A operand slots of 32 columns in
+  // tensor memory that the converter warps fill from the codes.
+  constexpr int MS = F8 ? 3 : 0;
   constexpr int MSD = MS > 0 ? MS : 1;        // slot count as a divisor (the bf16 instantiations use no slots)
-  constexpr int STAGE_BYTES = F8 ? RAW_BYTES : A_BYTES + B_BYTES;
-  constexpr int SLOT_BYTES = A_BYTES + B_BYTES;
-  constexpr uint32_t W_TX = F8 ? RAW_BYTES : A_BYTES;                     // weight bytes a stage's TMA brings
+  constexpr int W_BYTES = F8 ? RAW_BYTES : A_BYTES;
+  constexpr int STAGE_BYTES = W_BYTES + B_BYTES;
+  constexpr uint32_t W_TX = W_BYTES;                                      // weight bytes a stage's TMA brings
+  constexpr uint32_t TMEM_COLS = F8 ? (2 * BN + MS * 32 <= 256 ? 256 : 512) : 2 * BN;
   uint8_t* stages = base;
-  uint8_t* slots = base + STAGES * STAGE_BYTES;                           // FP8 operand slots
-  float* staging = reinterpret_cast<float*>(slots + MS * SLOT_BYTES);
+  float* staging = reinterpret_cast<float*>(base + STAGES * STAGE_BYTES);
   Smem& sm = *reinterpret_cast<Smem*>(reinterpret_cast<uint8_t*>(staging) + STAGING_BYTES);
 
   const int tid = threadIdx.x;
@@ -416,12 +410,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
     sm.abort_flag = 0;
     for (int s = 0; s < STAGES; ++s) {
       tc::mbar_init(&sm.full[s], 1);
-      tc::mbar_init(&sm.empty[s], F8 ? 128 : 1);   // FP8: released by the converters once they read the codes
+      tc::mbar_init(&sm.empty[s], 1);
     }
     for (int s = 0; s < MS; ++s) {
-      tc::mbar_init(&sm.conv[s], 128);
-      tc::mbar_init(&sm.bfull[s], 1);
-      tc::mbar_init(&sm.mempty[s], 1);
+      tc::mbar_init(&sm.conv[s], 128);   // the slot's 128 TMEM rows written
+      tc::mbar_init(&sm.mempty[s], 1);   // the slot read by the MMAs
     }
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(&sm.tfull[b], 1);
@@ -430,7 +423,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
     tc::mbar_init(&sm.done, 1);
     tc::fence_mbar_init();
   }
-  if (warp == 1) tc::tmem_alloc(&sm.tmem_base, 2 * BN);
+  if (warp == 1) tc::tmem_alloc(&sm.tmem_base, TMEM_COLS);
   __syncthreads();
   // Weights are never written by the kernels ahead of this one: the first tile's first weight stages can stream
   // in before the dependency wait (their transaction bytes are expected now; the arrival, with the activation
@@ -446,8 +439,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
       tc::prefetch_tmap(&tmap_w);
       const uint64_t pol_w = tc::policy_evict_first();
       for (int i = 0; i < npf; ++i) {
-        if (F8) tc::mbar_arrive_expect_tx(&sm.full[i], W_TX);   // the weight ring's stage is complete with it
-        else tc::mbar_expect_tx(&sm.full[i], W_TX);
+        tc::mbar_expect_tx(&sm.full[i], W_TX);
         tc::tma_load_2d(stages + i * STAGE_BYTES, &tmap_w, (kb0 + i) * BK, t0 * 128, &sm.full[i], pol_w);
       }
     }
@@ -529,15 +521,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
         const CUtensorMap* wm = extra ? &tmap_w2 : &tmap_w;
         const int64_t wrow = extra ? 0 : (int64_t)g * p.w_group_stride;
         const int nb = (nval + XBOX_ROWS - 1) / XBOX_ROWS;
-        const uint32_t bytes = W_TX + (F8 ? 0 : nb * XBOX_BYTES);
+        const uint32_t bytes = W_TX + nb * XBOX_BYTES;
         const int xrow = sm.grp_off[g] + n0;
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1;
-          if (F8 && it < (uint32_t)npf) continue;   // weight stage already in flight and armed
           if (!wait_bar(&sm.empty[s], ph ^ 1, abort_flag, p.status, ST_TIMEOUT_PRODUCER)) { ok = false; break; }
           uint8_t* a = stages + s * STAGE_BYTES;
-          uint8_t* b = a + A_BYTES;
+          uint8_t* b = a + W_BYTES;
           if (it < (uint32_t)npf) {   // weight stage already in flight: arrive with the activation bytes
             tc::mbar_arrive_expect_tx(&sm.full[s], bytes - W_TX);
           } else {
@@ -549,9 +540,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
               tc::tma_load_2d(a, wm, kb * BK, (int)(wrow + mt * 128), &sm.full[s], pol_w);
             }
           }
-          if (!F8)
-            for (int j = 0; j < nb; ++j)
-              tc::tma_load_2d(b + j * XBOX_BYTES, &tmap_x, kb * BK, xrow + j * XBOX_ROWS, &sm.full[s], pol_x);
+          for (int j = 0; j < nb; ++j)
+            tc::tma_load_2d(b + j * XBOX_BYTES, &tmap_x, kb * BK, xrow + j * XBOX_ROWS, &sm.full[s], pol_x);
         }
       }
       if (!ok) {
@@ -562,7 +552,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
       // prefetched weight stages no work item consumed (no rows after all): complete their phase and let the
       // copies land before the CTA leaves
       for (uint32_t i = it; i < (uint32_t)npf; ++i) {
-        if (!F8) tc::mbar_arrive(&sm.full[i]);
+        tc::mbar_arrive(&sm.full[i]);
         tc::mbar_wait(&sm.full[i], 0, 1u << 16);
       }
     }
@@ -583,25 +573,28 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
         const uint32_t idesc = tc::idesc_bf16_f32(128, N);
         const uint32_t d = sm.tmem_base + buf * BN;
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
-          uint32_t a;
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (!wait_bar(&sm.full[s], ph, abort_flag, p.status, ST_TIMEOUT_MMA)) { ok = false; break; }
+          const uint32_t a = tc::smem_u32(stages + s * STAGE_BYTES);
+          const uint32_t b = a + W_BYTES;
           if constexpr (F8) {
+            // A from tensor memory: the converted slot of this k-block
             const int ms = it % MSD;
-            const uint32_t mph = (it / MSD) & 1;
-            if (!wait_bar(&sm.conv[ms], mph, abort_flag, p.status, ST_TIMEOUT_MMA) ||
-                !wait_bar(&sm.bfull[ms], mph, abort_flag, p.status, ST_TIMEOUT_MMA)) { ok = false; break; }
-            a = tc::smem_u32(slots + ms * SLOT_BYTES);
-          } else {
-            const int s = it % STAGES;
-            const uint32_t ph = (it / STAGES) & 1;
-            if (!wait_bar(&sm.full[s], ph, abort_flag, p.status, ST_TIMEOUT_MMA)) { ok = false; break; }
-            a = tc::smem_u32(stages + s * STAGE_BYTES);
-          }
-          tc::fence_after_sync();
-          const uint32_t b = a + A_BYTES;
+            if (!wait_bar(&sm.conv[ms], (it / MSD) & 1, abort_flag, p.status, ST_TIMEOUT_MMA)) { ok = false; break; }
+            tc::fence_after_sync();
+            const uint32_t ta = sm.tmem_base + 2 * BN + ms * 32;
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)
-            tc::mma_bf16(d, tc::sdesc_k128(a + kk * 32), tc::sdesc_k128(b + kk * 32), idesc, (kb != kb0) || kk != 0);
-          tc::mma_commit(F8 ? &sm.mempty[it % MSD] : &sm.empty[it % STAGES]);
+            for (int kk = 0; kk < BK / 16; ++kk)
+              tc::mma_bf16_tmem_a(d, ta + kk * 8, tc::sdesc_k128(b + kk * 32), idesc, (kb != kb0) || kk != 0);
+            tc::mma_commit(&sm.mempty[ms]);
+          } else {
+            tc::fence_after_sync();
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk)
+              tc::mma_bf16(d, tc::sdesc_k128(a + kk * 32), tc::sdesc_k128(b + kk * 32), idesc, (kb != kb0) || kk != 0);
+          }
+          tc::mma_commit(&sm.empty[s]);
         }
         if (!ok) break;
         tc::mma_commit(&sm.tfull[buf]);
@@ -612,45 +605,26 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
     }
   } else if (F8 && warp >= 6) {
     // ------------------------------------------------------------------ FP8: converter warps 6..9
-    // per k-block, in the MMA's order: once the operand slot is free, thread 0 loads the slot's activation tile
-    // (TMA, on the slot's bfull barrier); every thread then waits for the weight stage, writes its share of the
-    // slot's bf16 weight tile, releases the weight stage, makes its writes visible to the tensor core (async proxy)
-    // and arrives on the slot's conv barrier
-    const int ct = tid - 192;
-    const uint64_t pol_x = tc::policy_evict_last();
-    if (ct == 0) tc::prefetch_tmap(&tmap_x);
-    uint32_t it = 0, issued = 0;
+    // per k-block, in the MMA's order: once the A slot is free and the stage's codes have landed, each thread writes
+    // its TMEM lane (the warp's quadrant) of the slot from its row of codes, waits for its stores, and arrives on the
+    // slot's conv barrier
+    const int row = (warp & 3) * 32 + lane;   // the TMEM lane this warp may access
+    uint32_t it = 0;
     bool ok = true;
     for (int wk = wk_begin; wk < total && ok; wk += wk_step) {
-      const int t = wk / p.ksplit, ks = wk - t * p.ksplit;
+      const int ks = wk - (wk / p.ksplit) * p.ksplit;
       const int kb0 = ks * kblocks / p.ksplit, kb1 = (ks + 1) * kblocks / p.ksplit;
-      int g, mt, n0, nval;
-      decode_tile<BN>(sm, p.m_tiles, t, g, mt, n0, nval);
-      const int nb = (nval + XBOX_ROWS - 1) / XBOX_ROWS;
-      const int xrow = sm.grp_off[g] + n0;
       for (int kb = kb0; kb < kb1; ++kb, ++it) {
         const int s = it % STAGES, ms = it % MSD;
-        const uint32_t ph = (it / STAGES) & 1, mph = (it / MSD) & 1;
-        if (!wait_bar(&sm.mempty[ms], mph ^ 1, abort_flag, p.status, ST_TIMEOUT_MMA)) { ok = false; break; }
-        uint8_t* slot = slots + ms * SLOT_BYTES;
-        if (ct == 0) {
-          tc::mbar_arrive_expect_tx(&sm.bfull[ms], (uint32_t)(nb * XBOX_BYTES));
-          for (int j = 0; j < nb; ++j)
-            tc::tma_load_2d(slot + A_BYTES + j * XBOX_BYTES, &tmap_x, kb * BK, xrow + j * XBOX_ROWS, &sm.bfull[ms],
-                            pol_x);
-          issued = it + 1;
-        }
-        if (!wait_bar(&sm.full[s], ph, abort_flag, p.status, ST_TIMEOUT_MMA)) { ok = false; break; }
-        convert_e4m3_tile(stages + s * STAGE_BYTES, slot, ct);
-        tc::mbar_arrive(&sm.empty[s]);
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        if (!wait_bar(&sm.mempty[ms], ((it / MSD) & 1) ^ 1, abort_flag, p.status, ST_TIMEOUT_MMA) ||
+            !wait_bar(&sm.full[s], (it / STAGES) & 1, abort_flag, p.status, ST_TIMEOUT_MMA)) { ok = false; break; }
+        tc::fence_after_sync();
+        convert_e4m3_row_to_tmem(stages + s * STAGE_BYTES, row,
+                                 sm.tmem_base + ((uint32_t)((warp & 3) * 32) << 16) + 2 * BN + ms * 32);
+        tc::tmem_st_wait();
+        tc::fence_before_sync();
         tc::mbar_arrive(&sm.conv[ms]);
       }
-    }
-    if (ct == 0 && !ok) {
-      // drain: the activation copies this thread issued land before the CTA leaves (bounded)
-      const uint32_t first = issued > (uint32_t)MSD ? issued - MSD : 0;
-      for (uint32_t i = first; i < issued; ++i) tc::mbar_wait(&sm.bfull[i % MSD], (i / MSD) & 1, 1u << 16);
     }
   } else {
     // ------------------------------------------------------------------ epilogue warps 2..5
@@ -762,7 +736,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
   __syncthreads();
   if (warp == 1) {
     tc::fence_after_sync();
-    tc::tmem_dealloc(sm.tmem_base, 2 * BN);
+    tc::tmem_dealloc(sm.tmem_base, TMEM_COLS);
   }
 }
 
@@ -1028,8 +1002,8 @@ EncodeTiledFn get_encode() {
   return fn;
 }
 
-// bf16 [rows, K] with 128-byte swizzled boxes of 64 x box_rows, or (u8) E4M3 codes [rows, K] with plain boxes of
-// 64 bytes x box_rows (the converter warps read them row by row)
+// bf16 [rows, K] with 128-byte swizzled boxes of 64 x box_rows, or (u8) E4M3 codes [rows, K] with 64-byte swizzled
+// boxes of 64 bytes x box_rows (the converter warps read them row by row)
 int make_map(CUtensorMap* m, const void* ptr, int64_t rows, int K, int box_rows, bool u8 = false) {
   EncodeTiledFn enc = get_encode();
   if (!enc) {
@@ -1042,7 +1016,7 @@ int make_map(CUtensorMap* m, const void* ptr, int64_t rows, int K, int box_rows,
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(m, u8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr),
                    dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   u8 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   u8 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     dllm_host::set_error("cuTensorMapEncodeTiled failed (%d) rows=%lld K=%d box_rows=%d", (int)r, (long long)rows,
@@ -1059,10 +1033,9 @@ int launch_cluster_splitk(const GemmArgs& a, const CUtensorMap& mw, const CUtens
 template <int BN, int STAGES, bool F8 = false>
 int launch(const GemmArgs& a, const CUtensorMap& mw, const CUtensorMap& mw2, const CUtensorMap& mx,
            const KParams& kp, cudaStream_t s) {
-  // (matches the kernel's layout: bf16 stages, or FP8 weight stages plus operand slots)
-  constexpr int MS = F8 ? (BN >= 128 ? 2 : 3) : 0;
-  constexpr int STAGE_BYTES = F8 ? RAW_BYTES : A_BYTES + BN * BK * 2;
-  constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + MS * (A_BYTES + BN * BK * 2) + STAGING_BYTES + (int)sizeof(Smem);
+  // (matches the kernel's layout: stages of [weights (bf16 or E4M3)][activations])
+  constexpr int STAGE_BYTES = (F8 ? RAW_BYTES : A_BYTES) + BN * BK * 2;
+  constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + STAGING_BYTES + (int)sizeof(Smem);
   static_assert(SMEM <= SMEM_LIMIT, "shared memory budget");
   // With programmatic dependent launch a CTA allocates tensor memory before it waits for the kernels ahead of it.
   // More than half an SM's shared memory per CTA keeps two tensor-memory kernels from sharing an SM, so a later
@@ -1256,8 +1229,8 @@ int gemm_bf16_tc(const GemmArgs& a, cudaStream_t s) {
   int st2;
   if (f8) {   // single-CTA tiles, no split-K (the weight-streaming shapes FP8 weights serve)
     if (bn == 32) st2 = launch<32, 16, true>(a, mw, mw2, mx, kp, s);
-    else if (bn == 64) st2 = launch<64, 14, true>(a, mw, mw2, mx, kp, s);
-    else st2 = launch<128, 13, true>(a, mw, mw2, mx, kp, s);
+    else if (bn == 64) st2 = launch<64, 12, true>(a, mw, mw2, mx, kp, s);
+    else st2 = launch<128, 8, true>(a, mw, mw2, mx, kp, s);
   } else if (gemm_uses_pairs(a)) {
     kp.prefetch_w = 0;
     st2 = launch_pair(mw, mw2, mx, kp, s);

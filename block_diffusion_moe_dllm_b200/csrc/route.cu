@@ -374,6 +374,44 @@ DLLM_DEV void cta_redecide(RedecideSmem<NW>& rs, const float* __restrict__ score
   }
 }
 
+// Tokens [t0, t1) whose fix_thr is not NaN (near-ties flagged by route_topk_kernel) into the CTA's list; past the
+// list's capacity, the token's warp decides it alone. Every warp of the CTA calls this; rs.n_flag starts at 0.
+template <int PER, int NW, typename T>
+DLLM_DEV void collect_flagged(RedecideSmem<NW>& rd, int t0, int t1, const float* __restrict__ fix_thr,
+                              const float* __restrict__ scores, const float* __restrict__ bias, int E, int k,
+                              const T* __restrict__ h, const T* __restrict__ w, int H, int32_t* __restrict__ ids,
+                              float* __restrict__ gates) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int tb = t0 + warp * 32; tb < t1; tb += NW * 32) {
+    const int t = tb + lane;
+    const float th = t < t1 ? fix_thr[t] : __int_as_float(0x7fc00000);
+    const bool fl = !isnan(th);
+    const unsigned bal = __ballot_sync(0xffffffffu, fl);
+    int base = 0;
+    if (lane == 0 && bal) base = atomicAdd(&rd.n_flag, __popc(bal));
+    base = __shfl_sync(0xffffffffu, base, 0);
+    const int f = base + __popc(bal & ((1u << lane) - 1u));
+    if (fl && f < kMaxFlagged) {
+      rd.ftok[f] = t;
+      rd.fthr[f] = th;
+    }
+    unsigned over = __ballot_sync(0xffffffffu, fl && f >= kMaxFlagged);
+    while (over) {
+      const int j = __ffs(over) - 1;
+      over &= over - 1;
+      const int tt = tb + j;
+      int my_id;
+      float my_gate;
+      exact_redecide<PER>(scores + (int64_t)tt * E, bias, E, k, h + (int64_t)tt * H, w, H,
+                          __shfl_sync(0xffffffffu, th, j), lane, my_id, my_gate);
+      if (lane < k) {
+        ids[(int64_t)tt * k + lane] = my_id;
+        gates[(int64_t)tt * k + lane] = my_gate;
+      }
+    }
+  }
+}
+
 // Many tokens: one warp per token, the fp32 selection. A token whose selection is a near-tie (see kRouteGuard) gets
 // fix_thr[t] = its candidate threshold, every other token NaN; the histogram launch decides those tokens again
 // before it counts.
@@ -527,37 +565,8 @@ __global__ void __launch_bounds__(256) route_seg_hist_kernel(int32_t* __restrict
   for (int i = threadIdx.x; i < E; i += blockDim.x) sh_hist[i] = 0;
   if (threadIdx.x == 0) rd.n_flag = 0;
   __syncthreads();
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int t0 = blockIdx.x * seg_tok, t1 = min(Tk, t0 + seg_tok);
-  // the segment's near-tie tokens (fix_thr not NaN) into the list; past its capacity, a warp decides alone
-  for (int tb = t0 + warp * 32; tb < t1; tb += 256) {
-    const int t = tb + lane;
-    const float th = t < t1 ? fix_thr[t] : __int_as_float(0x7fc00000);
-    const bool fl = !isnan(th);
-    const unsigned bal = __ballot_sync(0xffffffffu, fl);
-    int base = 0;
-    if (lane == 0 && bal) base = atomicAdd(&rd.n_flag, __popc(bal));
-    base = __shfl_sync(0xffffffffu, base, 0);
-    const int f = base + __popc(bal & ((1u << lane) - 1u));
-    if (fl && f < kMaxFlagged) {
-      rd.ftok[f] = t;
-      rd.fthr[f] = th;
-    }
-    unsigned over = __ballot_sync(0xffffffffu, fl && f >= kMaxFlagged);
-    while (over) {
-      const int j = __ffs(over) - 1;
-      over &= over - 1;
-      const int tt = tb + j;
-      int my_id;
-      float my_gate;
-      exact_redecide<PER>(scores + (int64_t)tt * E, bias, E, k, h + (int64_t)tt * H, w, H,
-                          __shfl_sync(0xffffffffu, th, j), lane, my_id, my_gate);
-      if (lane < k) {
-        ids[(int64_t)tt * k + lane] = my_id;
-        gates[(int64_t)tt * k + lane] = my_gate;
-      }
-    }
-  }
+  collect_flagged<PER, 8>(rd, t0, t1, fix_thr, scores, bias, E, k, h, w, H, ids, gates);
   __syncthreads();
   cta_redecide<PER, 8>(rd, scores, bias, E, k, h, w, H, [&](int t, int ln, int id, float g) {
     if (ln < k) {
@@ -690,6 +699,105 @@ __global__ void __launch_bounds__(256) route_seg_scatter_kernel(const int32_t* _
   }
 }
 
+// Mid-size routing (E <= 256, Tk * k <= kPermCtaMax): after route_topk_kernel, one CTA of 1024 threads decides the
+// flagged near-tie tokens again and builds counts, offsets and the stable permutation, in place of the segmented
+// three launches. Warp w takes the assignments [w per, (w + 1) per) (per a multiple of 32); pass 1 counts them per
+// expert (__match_any_sync groups), the 32 warps' counts are prefixed per expert on top of the expert's offset, and
+// pass 2 writes position = warp's running base + rank among the chunk's lanes with the same expert, so positions
+// within an expert follow the assignment index a = t k + j, as in the other permutation kernels.
+constexpr int kPermCtaMax = 8192;
+
+template <int PER, typename T>
+__global__ void __launch_bounds__(1024) route_perm_cta_kernel(int32_t* __restrict__ ids, float* __restrict__ gates,
+                                                              const float* __restrict__ scores,
+                                                              const float* __restrict__ bias,
+                                                              const float* __restrict__ fix_thr,
+                                                              const T* __restrict__ h, const T* __restrict__ w, int H,
+                                                              int Tk, int E, int k, int32_t* __restrict__ counts,
+                                                              int32_t* __restrict__ offsets,
+                                                              int32_t* __restrict__ perm, int32_t* __restrict__ inv,
+                                                              const int32_t* __restrict__ live) {
+  pdl_enter();
+  if (live && *live == 0) return;   // a pass with no masked position left does nothing
+  extern __shared__ int wh[];        // [32][E]
+  __shared__ RedecideSmem<32> rd;
+  __shared__ int wtot[32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int i = tid; i < 32 * E; i += blockDim.x) wh[i] = 0;
+  if (tid == 0) rd.n_flag = 0;
+  __syncthreads();
+  collect_flagged<PER, 32>(rd, 0, Tk, fix_thr, scores, bias, E, k, h, w, H, ids, gates);
+  __syncthreads();
+  cta_redecide<PER, 32>(rd, scores, bias, E, k, h, w, H, [&](int t, int ln, int id, float g) {
+    if (ln < k) {
+      ids[(int64_t)t * k + ln] = id;
+      gates[(int64_t)t * k + ln] = g;
+    }
+  });
+  __syncthreads();   // the re-decided ids (global writes of this CTA) are visible to the whole CTA
+  const int n = Tk * k;
+  const int per = ((n + 31) / 32 + 31) & ~31;
+  const int a0 = min(n, warp * per), a1 = min(n, a0 + per);
+  for (int c = a0; c < a1; c += 32) {
+    const int a = c + lane;
+    const int ex = a < a1 ? ids[a] : -1;
+    const unsigned grp = __match_any_sync(0xffffffffu, ex);
+    if (a < a1 && lane == __ffs(grp) - 1) wh[warp * E + ex] += __popc(grp);
+  }
+  __syncthreads();
+  // per expert (one thread each, E <= 1024): prefix over the warps, total count, then the exclusive scan of the
+  // totals over experts
+  int cnt = 0;
+  if (tid < E) {
+#pragma unroll 8
+    for (int q = 0; q < 32; ++q) {
+      const int v = wh[q * E + tid];
+      wh[q * E + tid] = cnt;
+      cnt += v;
+    }
+  }
+  int inc = cnt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += y;
+  }
+  if (lane == 31) wtot[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    int x = wtot[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    wtot[lane] = x;   // inclusive over warps
+  }
+  __syncthreads();
+  if (tid < E) {
+    const int excl = inc - cnt + (warp > 0 ? wtot[warp - 1] : 0);
+    counts[tid] = cnt;
+    offsets[tid] = excl;
+#pragma unroll 8
+    for (int q = 0; q < 32; ++q) wh[q * E + tid] += excl;
+  }
+  if (tid == 0) offsets[E] = n;
+  __syncthreads();
+  for (int c = a0; c < a1; c += 32) {
+    const int a = c + lane;
+    const int ex = a < a1 ? ids[a] : -1;
+    const unsigned grp = __match_any_sync(0xffffffffu, ex);
+    if (a < a1) {
+      const int pos = wh[warp * E + ex] + __popc(grp & ((1u << lane) - 1u));
+      perm[pos] = a;
+      inv[a] = pos;
+    }
+    __syncwarp();
+    if (a < a1 && lane == __ffs(grp) - 1) wh[warp * E + ex] += __popc(grp);
+    __syncwarp();
+  }
+}
+
 }  // namespace
 
 // Layout of the router scratch: per-segment expert histograms, then one fp32 near-tie threshold per token.
@@ -735,6 +843,20 @@ int launch_select_per(float* scores, const float* bias, int Tk, int E, int k, in
              rs.fix_thr, live);
   DLLM_CHECK_LAUNCH("route_topk_kernel");
   const int n = Tk * k, seg = rs.seg_tok * k;
+  if constexpr (PER <= 8) {
+    if (n <= kPermCtaMax) {   // one CTA decides the flagged tokens again and builds the permutation
+      const size_t smem = (size_t)32 * E * sizeof(int);
+      static bool cfg = false;
+      if (!cfg) {
+        cudaFuncSetAttribute(route_perm_cta_kernel<PER, T>, cudaFuncAttributeMaxDynamicSharedMemorySize, 32 * 1024);
+        cfg = true;
+      }
+      launch_pdl(route_perm_cta_kernel<PER, T>, 1, 1024, smem, s, ids, gates, (const float*)scores, bias,
+                 (const float*)rs.fix_thr, h, w, H, Tk, E, k, counts, offsets, perm, inv, live);
+      DLLM_CHECK_LAUNCH("route_perm_cta_kernel");
+      return DLLM_OK;
+    }
+  }
   launch_pdl(route_seg_hist_kernel<PER, T>, rs.S, 256, (size_t)E * sizeof(int), s, ids, gates,
              (const float*)scores, bias, (const float*)rs.fix_thr, h, w, H, Tk, E, k, rs.seg_tok, rs.seg_hist, live);
   DLLM_CHECK_LAUNCH("route_seg_hist_kernel");

@@ -107,7 +107,8 @@ def test_gemm_f32():
                                             ("f32", 16, 256, 8, 2), ("bf16", 9, 256, 1024, 32),
                                             ("bf16", 20, 256, 512, 8), ("f32", 32, 128, 64, 32),
                                             ("bf16", 4096, 512, 256, 8), ("bf16", 1001, 256, 1000, 3),
-                                            ("f32", 4100, 64, 32, 2), ("bf16", 5000, 256, 96, 4)])
+                                            ("f32", 4100, 64, 32, 2), ("bf16", 5000, 256, 96, 4),
+                                            ("bf16", 1024, 512, 128, 8), ("f32", 4096, 64, 32, 2)])
 def test_route(dtype, Tk, H, E, k):
     t = _tdt(dtype)
     h = synth.normal((Tk, H), 1.0, 5, f"rh{Tk}", DEV, t)
@@ -128,6 +129,54 @@ def test_route(dtype, Tk, H, E, k):
     assert np.max(np.abs(to64(scores) - o_s)) < 2e-6
     same_routing(g_ids, gates.cpu().numpy(), o_ids, o_gates, margin >= ROUTE_TIE, rtol=2e-6, atol=2e-7)
     # permutation tables are exactly those of the GPU's ids
+    c, off, p, iv = assignment_tables(g_ids, E)
+    assert np.array_equal(counts.cpu().numpy(), c)
+    assert np.array_equal(offsets.cpu().numpy(), off)
+    assert np.array_equal(perm.cpu().numpy(), p)
+    assert np.array_equal(inv.cpu().numpy(), iv)
+
+
+@pytest.mark.parametrize("dtype,Tk", [("f32", 2000), ("bf16", 2000), ("bf16", 300)])
+def test_route_planted_near_ties(dtype, Tk):
+    """Every token's second slot is contested by two experts whose scores differ by 1e-6 .. 1e-5 (inside the
+    library's fp32 guard, outside the 1e-6 band the comparison forgives): expert 0 always wins slot 1 (bias 2),
+    experts 1 and 2 (bias 1) differ only by a tiny weight perturbation, so nearly every token is re-decided exactly,
+    more of them than one CTA's flagged list holds."""
+    t = _tdt(dtype)
+    H, E, k = 256, 64, 2
+    g = torch.Generator().manual_seed(1234)
+    h = torch.randn((Tk, H), generator=g, dtype=torch.float64)
+    w = torch.randn((E, H), generator=g, dtype=torch.float64) * 0.02
+    bias = (torch.rand(E, generator=g, dtype=torch.float64) - 0.5) * 0.2
+    bias[0], bias[1], bias[2] = 2.0, 1.0, 1.0
+    if dtype == "f32":
+        w[2] = w[1] + 1e-6 * torch.randn(H, generator=g, dtype=torch.float64)
+        hd, wd = h.to(t), w.to(t)
+    else:
+        j = 7
+        w[1, j] = 0.02
+        sgn = torch.where(torch.rand(Tk, generator=g) < 0.5, -1.0, 1.0).to(torch.float64)
+        h[:, j] = sgn * (0.04 + 0.26 * torch.rand(Tk, generator=g, dtype=torch.float64))
+        hd, wd = h.to(t), w.to(t)
+        wb = wd.view(torch.int16)
+        wb[2] = wb[1]
+        wb[2, j] += 1                      # one bf16 ulp apart in one coordinate
+    hd, wd = hd.to(DEV), wd.to(DEV)
+    bias_d = bias.to(torch.float32).to(DEV)
+    ids = torch.empty((Tk, k), dtype=torch.int32, device=DEV)
+    gates = torch.empty((Tk, k), dtype=torch.float32, device=DEV)
+    counts = torch.empty(E, dtype=torch.int32, device=DEV)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=DEV)
+    perm = torch.empty(Tk * k, dtype=torch.int32, device=DEV)
+    inv = torch.empty(Tk * k, dtype=torch.int32, device=DEV)
+    bd.moe_route(hd, wd, bias_d, ids, gates, counts, offsets, perm, inv, Tk, H, E, k, DT[dtype])
+    torch.cuda.synchronize()
+    o_ids, o_gates, _, margin = O.route(to64(hd), to64(wd), to64(bias_d), k, order=True)
+    checked = margin >= ROUTE_TIE
+    near = checked & (margin < 1e-5)
+    assert near.sum() >= min(257, Tk // 3), "the planted ties should put many tokens inside the guard"
+    g_ids = ids.cpu().numpy()
+    same_routing(g_ids, gates.cpu().numpy(), o_ids, o_gates, checked, rtol=2e-6, atol=2e-7)
     c, off, p, iv = assignment_tables(g_ids, E)
     assert np.array_equal(counts.cpu().numpy(), c)
     assert np.array_equal(offsets.cpu().numpy(), off)

@@ -47,8 +47,8 @@ static_assert(SMEM <= 232448, "shared memory budget");
 // with programmatic dependent launch, tensor memory is allocated before the wait for earlier kernels: one such
 // CTA per SM (more than half the SM's shared memory) keeps a later kernel from holding columns an earlier needs
 static_assert(SMEM > 233472 / 2, "tensor-memory kernels must not share an SM");
-static_assert((128 + 135) * kRecvStride * 4 <= STAGES * 2 * TILE,
-              "split exchange staging (own rows + n_splits * ceil(128 / n_splits) others) exceeds the K/V ring");
+static_assert(135 * kRecvStride * 4 <= STAGES * 2 * TILE,
+              "split exchange (n_splits * ceil(128 / n_splits) rows, at most 8 splits) exceeds the K/V ring");
 
 struct Bars {
   uint64_t q_full;
@@ -58,7 +58,6 @@ struct Bars {
   uint64_t p_ready[2];  // per group: P of its tile written over S (and the group's O rescaled if needed)
   uint64_t o_full[2];   // per group: phase i completes when the group's i-th P V is accumulated into its O
   uint64_t done;
-  uint64_t xch_full;    // split merge: the other splits' rows of this CTA have landed in shared memory
   uint32_t tmem_base;
   int abort_flag;
   short kblk[2][2][KT];     // [group][tile parity within the group][key]: block of the key relative to the CTA's
@@ -73,7 +72,6 @@ struct AttnTcParams {
   uint32_t blk_magic, blk_shift;   // key position / blk_len = (pos * blk_magic) >> blk_shift for 0 <= pos < 2^31
   float scale_log2;
   const int32_t* key_pos;
-  float* xscratch;      // split exchange: [B*Hkv*n_qtiles][n_splits][128 rows][kRecvStride] (n_splits > 1)
   __nv_bfloat16* out;   // [B, Lq, Hq, 128]
   int32_t* status;
   const int32_t* live;  // nullable: *live == 0 = a denoising pass with no masked position left (nothing to do)
@@ -141,25 +139,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-// Bulk copies between shared and global memory (the async proxy) for the split exchange.
-__device__ __forceinline__ void bulk_store_s2g(void* gdst, const void* ssrc, uint32_t bytes) {
-  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(gdst), "r"(tc::smem_u32(ssrc)),
-               "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void bulk_commit_and_wait() {
-  asm volatile("cp.async.bulk.commit_group;\n\tcp.async.bulk.wait_group 0;" ::: "memory");
-}
-__device__ __forceinline__ void bulk_load_g2s(void* sdst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                   tc::smem_u32(sdst)),
-               "l"(gsrc), "r"(bytes), "r"(tc::smem_u32(bar))
-               : "memory");
-}
-__device__ __forceinline__ void fence_proxy_async_all() {
-  asm volatile("fence.proxy.async;" ::: "memory");
 }
 
 __device__ __forceinline__ void cluster_arrive() {
@@ -245,7 +224,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       tc::mbar_init(&bar.o_full[g2], 1);
     }
     tc::mbar_init(&bar.done, 1);
-    tc::mbar_init(&bar.xch_full, 1);
     tc::fence_mbar_init();
   }
   if (warp == 1) tc::tmem_alloc(&bar.tmem_base, 512);
@@ -288,6 +266,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const int s = it % STAGES;
         const uint32_t ph = (it / STAGES) & 1;
         if (!wait_bar(&bar.kv_empty[s], ph ^ 1, abort_flag, p.status, ST_TIMEOUT_PRODUCER)) { ok = false; break; }
+        // the rest of the ring only once the first tile has landed: every CTA of the launch requests its first
+        // tile alone, so those arrive first (with the whole ring requested at once by every CTA, the first tiles
+        // came in late, behind the others' later stages)
+        if (it == 1 && !wait_bar(&bar.kv_full[0], 0, abort_flag, p.status, ST_TIMEOUT_PRODUCER)) { ok = false; break; }
         const int key0 = (t_begin + j) * KT;
         const int bg = b * p.Hkv + g;
         tc::mbar_arrive_expect_tx(&bar.kv_full[s], 2 * TILE);
@@ -367,7 +349,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
   const int row = q4 * 32 + lane;      // TMEM lane = tile row
   const int grp = (warp - 2) >> 2;
   const int gtid = ((warp - 2) & 3) * 32 + lane;   // 0..127 within the group
-  const int etid = tid - 64;           // 0..255
   const int col0 = 64 * grp;
   const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
   float o[64];
@@ -531,55 +512,38 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     }
   }
   if (p.n_splits > 1) {
-    // merge the splits of this query tile through L2. Rank r owns rows [r*LR, (r+1)*LR). Every split stages the
-    // unnormalised rows (o relative to its maximum, m, l) that other ranks own in its idle K/V ring and
-    // bulk-copies them to its slab of the exchange buffer; after one cluster barrier each owner bulk-copies the
-    // other splits' copies of its rows into its ring, and the two threads of every owned row fold them into the
-    // row they hold in registers (splits in order) and write the output.
+    // merge the splits of this query tile inside the cluster. Rank r owns rows [r*LR, (r+1)*LR). Once every CTA
+    // of the cluster is done with its K/V ring (first cluster barrier), the threads of each row another rank owns
+    // store their unnormalised row (o relative to their maximum, m, l) straight into the owner's ring through
+    // distributed shared memory; after the second cluster barrier (release / acquire: the stores are visible) the
+    // two threads of every owned row fold the other splits' copies into the row they hold in registers (splits in
+    // order) and write the output.
     const int ns = p.n_splits;
     const int LR = (128 + ns - 1) / ns;
     const int r0 = split * LR, n_loc = max(0, min(128, r0 + LR) - r0);
-    constexpr uint32_t kRowBytes = kRecvStride * 4;
-    float* stage = reinterpret_cast<float*>(sK);                 // [128 rows][kRecvStride]: rows others own
-    float* pbuf = stage + 128 * kRecvStride;                      // [ns][LR][kRecvStride]: the others' copies
-    float* slab0 = p.xscratch + (size_t)blockIdx.y * ns * 128 * kRecvStride;
+    float* pbuf = reinterpret_cast<float*>(sK);                   // [ns][LR][kRecvStride]: the others' copies
     const bool mine = row >= r0 && row < r0 + n_loc;
-    if (warp >= 2) {
-      tc::named_bar_sync(kBarAll, 256);              // every consumer has read the group exchange in the ring
-      if (!mine) {
-        float* srow = stage + (size_t)row * kRecvStride;
+    cluster_arrive();
+    cluster_wait();
+    if (warp >= 2 && !mine && !*abort_flag) {
+      const int owner = row / LR, lr = row - owner * LR;
+      const uint32_t dst =
+          tc::mapa_u32(tc::smem_u32(pbuf + ((size_t)split * LR + lr) * kRecvStride + col0), (uint32_t)owner);
 #pragma unroll
-        for (int c = 0; c < 64; c += 4)
-          *reinterpret_cast<float4*>(srow + col0 + c) = make_float4(o[c], o[c + 1], o[c + 2], o[c + 3]);
-        if (grp == 0) *reinterpret_cast<float2*>(srow + 128) = make_float2(m_ref, l_row);
-      }
-      fence_proxy_async_all();                       // the staged rows are read by the bulk copy (async proxy)
-      tc::named_bar_sync(kBarAll, 256);
-      if (etid == 0) {
-        // rows [0, r0) and [r0 + n_loc, 128) to this split's slab
-        float* slab = slab0 + (size_t)split * 128 * kRecvStride;
-        if (r0 > 0) bulk_store_s2g(slab, stage, (uint32_t)r0 * kRowBytes);
-        if (r0 + n_loc < 128)
-          bulk_store_s2g(slab + (size_t)(r0 + n_loc) * kRecvStride, stage + (size_t)(r0 + n_loc) * kRecvStride,
-                         (uint32_t)(128 - r0 - n_loc) * kRowBytes);
-        bulk_commit_and_wait();
-        fence_proxy_async_all();
-      }
+      for (int c = 0; c < 64; c += 4)
+        asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(dst + c * 4), "f"(o[c]),
+                     "f"(o[c + 1]), "f"(o[c + 2]), "f"(o[c + 3])
+                     : "memory");
+      if (grp == 0)
+        asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(dst + (128 - col0) * 4), "f"(m_ref),
+                     "f"(l_row)
+                     : "memory");
     }
     cluster_arrive();
     cluster_wait();
     if (warp >= 2) {
-      if (etid == 0) {
-        fence_proxy_async_all();
-        tc::mbar_arrive_expect_tx(&bar.xch_full, (uint32_t)((ns - 1) * n_loc) * kRowBytes);
-        for (int sp = 0; sp < ns; ++sp)
-          if (sp != split && n_loc > 0)
-            bulk_load_g2s(pbuf + (size_t)sp * LR * kRecvStride, slab0 + ((size_t)sp * 128 + r0) * kRecvStride,
-                          (uint32_t)n_loc * kRowBytes, &bar.xch_full);
-      }
-      const bool got = wait_bar(&bar.xch_full, 0, abort_flag, p.status, ST_TIMEOUT_EPILOGUE);
       const int qg = q0 + row / p.G;
-      if (mine && got && qg < p.Lq && !*abort_flag) {
+      if (mine && qg < p.Lq && !*abort_flag) {
         const int lr = row - r0;
         float M = m_ref;
         for (int sp = 0; sp < ns; ++sp)
@@ -717,11 +681,8 @@ bool attn_tc_supported(int dtype, int Hq, int Hkv, int d) {
   return G >= 1 && G <= 128 && (128 % G) == 0;
 }
 
-size_t attn_tc_workspace_bytes(int B, int Lq, int Hq, int Hkv, int n_keys) {
-  int QT, n_qtiles, n_splits, tps;
-  plan_tc(B, Lq, Hq, Hkv, n_keys, QT, n_qtiles, n_splits, tps);
-  if (n_splits <= 1) return 0;
-  return (size_t)B * Hkv * n_qtiles * n_splits * 128 * kRecvStride * sizeof(float);
+size_t attn_tc_workspace_bytes(int, int, int, int, int) {
+  return 0;   // the key splits merge through distributed shared memory
 }
 
 int launch_attn_tc(const AttnArgs& a, int32_t* status, cudaStream_t s) {
@@ -740,13 +701,6 @@ int launch_attn_tc(const AttnArgs& a, int32_t* status, cudaStream_t s) {
   const float scale = a.scale > 0.f ? a.scale : 1.0f / sqrtf((float)a.d);
   p.scale_log2 = scale * 1.4426950408889634f;
   p.key_pos = a.key_pos;
-  p.xscratch = static_cast<float*>(a.ws);
-  if (p.n_splits > 1) {
-    const size_t need = (size_t)a.B * a.Hkv * p.n_qtiles * p.n_splits * 128 * kRecvStride * sizeof(float);
-    DLLM_REQUIRE(a.ws != nullptr && a.ws_bytes >= need && ((uintptr_t)a.ws % 16) == 0, DLLM_ERR_WORKSPACE,
-                 "attention: split exchange needs %zu bytes of 16-byte aligned workspace (have %zu)", need,
-                 a.ws_bytes);
-  }
   p.out = static_cast<__nv_bfloat16*>(a.out);
   p.status = status;
   p.live = a.live;

@@ -47,6 +47,7 @@ def parse():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--workload", default=UNDERSTANDING.name)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-fp8", action="store_true", help="skip the FP8-checkpoint leg")
     return ap.parse_args()
 
 
@@ -256,34 +257,18 @@ def algorithmic_bytes(w, passes, commit_active):
 
 
 # ---------------------------------------------------------------------------------------------- native arm
-def main():
-    args = parse()
-    w = BY_NAME[args.workload]
-    if args.impl == "reference":
-        run_reference(args, w)
-        return
+def measure(args, w, wt, caches, tokens0, mask0, dev, world, local, e2e):
+    """Time whole blocks of workload w through the library's block graph (see the module docstring); with e2e also
+    the two end-to-end variants through host buffers. Returns the numbers of the bench line."""
     import torch
     import torch.distributed as dist
     from block_diffusion_moe_dllm_b200 import binding as bd
     from block_diffusion_moe_dllm_b200 import kernel_bench as kb
-    from block_diffusion_moe_dllm_b200 import replicas, synth
+    from block_diffusion_moe_dllm_b200 import replicas
     from block_diffusion_moe_dllm_b200.engine import DenoiseEngine
 
-    world, rank, local = dist_env()
-    torch.cuda.set_device(local)
-    dev = f"cuda:{local}"
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    bd.load()
-
-    seed = replicas.replica_seed(w.seed, rank)
-    wt = synth.make_weights(w, dev, seed=seed)
-    caches = synth.make_prefix_cache(w, dev, seed=seed)
-    tokens0, mask0 = synth.make_block_state(w, dev, seed=seed)
     eng = DenoiseEngine(w, wt, caches, dev)
     stream = torch.cuda.current_stream()
-
     # the whole block as the library's block graph: the T_s passes, each inside a conditional node that runs it only
     # while the block has masked positions, and the commit pass; every step resets the block state from a device
     # copy first. Kernels per pass are counted on host-driven calls.
@@ -374,34 +359,85 @@ def main():
         return replicas.aggregate_throughput(w.B * w.L * live * args.steps, t, world)
 
     io = {"h2d_bytes_per_step": h_tok.numel() * 4 + h_mask.numel(), "d2h_bytes_per_step": h_out.numel() * 4}
-    e2e = {"value": e2e_run(False), "unit": "tokens/s", **io,
-           "path": "dllm_denoise_step called from the host for every pass and the commit pass"}
-    e2e_graph = {"value": e2e_run(True), "unit": "tokens/s", **io,
-                 "path": "dllm_block_graph_launch per block (passes after the block finished are skipped)"}
+    e2e_host = e2e_graph = None
+    if e2e:
+        e2e_host = {"value": e2e_run(False), "unit": "tokens/s", **io,
+                    "path": "dllm_denoise_step called from the host for every pass and the commit pass"}
+        e2e_graph = {"value": e2e_run(True), "unit": "tokens/s", **io,
+                     "path": "dllm_block_graph_launch per block (passes after the block finished are skipped)"}
     assert bd.status_check(eng.ws) == bd.OK
     del graph
+    return {"value": value, "ms_per_step": 1000.0 * step_s, "committed": committed,
+            "timed_units": {"n": len(units), "unit_s": units, "steps_per_unit": args.steps},
+            "graph_conditional": graph_cond if graph_cond else f"no: {graph_note}",
+            "passes_per_block": {"live": live, "launched": live if graph_cond else w.T_s,
+                                 "rows_per_live_pass": [p["rows"] for p in passes if p["live"]]},
+            "active": {"mean": statistics.mean(act) if act else 0, "min": min(act) if act else 0,
+                       "max": max(act) if act else 0},
+            "gpu_launches": ((live if graph_cond else w.T_s) * per_pass + per_commit) * args.steps * len(units),
+            "clocks": clk, "e2e": e2e_host, "e2e_graph": e2e_graph, "step_roof": step_roof}
+
+
+def main():
+    args = parse()
+    w = BY_NAME[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+        return
+    import torch
+    import torch.distributed as dist
+    from block_diffusion_moe_dllm_b200 import binding as bd
+    from block_diffusion_moe_dllm_b200 import replicas, synth
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = f"cuda:{local}"
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    bd.load()
+
+    seed = replicas.replica_seed(w.seed, rank)
+    wt = synth.make_weights(w, dev, seed=seed)
+    caches = synth.make_prefix_cache(w, dev, seed=seed)
+    tokens0, mask0 = synth.make_block_state(w, dev, seed=seed)
+    r = measure(args, w, wt, caches, tokens0, mask0, dev, world, local, e2e=True)
+
+    # ---- the same workload from the FP8 checkpoint (E4M3 expert and LM-head weights with per-row scales): its own
+    # routing and passes, since the dequantised weights differ from the bf16 ones
+    fp8 = None
+    w8 = BY_NAME.get(w.name + "-fp8")
+    if w8 is not None and w.wfmt != "fp8" and not args.no_fp8:
+        wt8 = synth.make_weights(w8, dev, seed=seed)
+        r8 = measure(args, w8, wt8, caches, tokens0, mask0, dev, world, local, e2e=False)
+        fp8 = {"workload": w8.name, "value": r8["value"], "unit": "tokens/s", "ms_per_step": r8["ms_per_step"],
+               "committed_tokens_per_s": r8["committed"], "passes_per_block": r8["passes_per_block"],
+               "active_experts_per_layer": r8["active"], "step_roofline": r8["step_roof"],
+               "timed_units": r8["timed_units"], "clocks": r8["clocks"], "gpu_launches": r8["gpu_launches"]}
+        del wt8
+        torch.cuda.empty_cache()
 
     # ---- dominant kernel, timed alone with CUDA events at this workload's shapes
-    roof, kernels = kernel_rooflines(w, wt, dev, stream)
+    roof, kernels = kernel_rooflines(w, wt, dev, torch.cuda.current_stream())
 
     if rank == 0:
-        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-                "warmup": args.warmup, "ms_per_step": 1000.0 * step_s, "higher_is_better": True,
+        line = {"metric": METRIC, "value": r["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": r["ms_per_step"], "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
                 "step": "one block: state reset, then the library's block graph: T_s denoising passes, each in a "
                         "conditional node that runs it only while masked positions are left, and the commit pass",
                 "config": bench_config(w, world),
-                "timed_units": {"n": len(units), "unit_s": units, "steps_per_unit": args.steps},
-                "committed_tokens_per_s": committed,
-                "block_graph_conditional": graph_cond if graph_cond else f"no: {graph_note}",
-                "passes_per_block": {"live": live, "launched": live if graph_cond else w.T_s,
-                                     "rows_per_live_pass": [p["rows"] for p in passes if p["live"]]},
-                "active_experts_per_layer": {"mean": statistics.mean(act) if act else 0,
-                                             "min": min(act) if act else 0, "max": max(act) if act else 0},
-                "gpu_launches": ((live if graph_cond else w.T_s) * per_pass + per_commit) * args.steps * len(units),
-                "clocks": clk,
-                "e2e": e2e, "e2e_graph": e2e_graph, "roofline": roof, "step_roofline": step_roof,
+                "timed_units": r["timed_units"],
+                "committed_tokens_per_s": r["committed"],
+                "block_graph_conditional": r["graph_conditional"],
+                "passes_per_block": r["passes_per_block"],
+                "active_experts_per_layer": r["active"],
+                "gpu_launches": r["gpu_launches"],
+                "clocks": r["clocks"],
+                "e2e": r["e2e"], "e2e_graph": r["e2e_graph"], "roofline": roof, "step_roofline": r["step_roof"],
                 "kernels": kernels}
+        if fp8 is not None:
+            line["fp8_weights"] = fp8
         if not args.no_cpu_baseline and world == 1:
             line["cpu_baseline"] = cpu_baseline(w)
         print(json.dumps(line), flush=True)

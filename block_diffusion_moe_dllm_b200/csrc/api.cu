@@ -806,10 +806,13 @@ int dllm_block_graph_skips_finished_passes(const dllm_block_graph* g) { return g
 
 namespace {
 // Conditional (IF) nodes through the driver API, with the context given explicitly (the node, its handle and the
-// kernels of its body must share one context: the current one).
+// kernels of its body must share one context: the current one). The entry points are requested at the ABI of CUDA
+// 12.3, where cuGraphAddNode takes per-edge data (left null here): the default query returns that version under a
+// 12.x runtime, and calling it with the older five-argument signature is what made the driver refuse the node.
 typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
 typedef CUresult (*CondHandleCreateFn)(CUgraphConditionalHandle*, CUgraph, CUcontext, unsigned int, unsigned int);
-typedef CUresult (*GraphAddNodeFn)(CUgraphNode*, CUgraph, const CUgraphNode*, size_t, CUgraphNodeParams*);
+typedef CUresult (*GraphAddNodeFn)(CUgraphNode*, CUgraph, const CUgraphNode*, const CUgraphEdgeData*, size_t,
+                                   CUgraphNodeParams*);
 
 struct CondApi {
   CtxGetCurrentFn ctx_get = nullptr;
@@ -824,7 +827,8 @@ const CondApi& cond_api() {
     auto get = [](const char* name) -> void* {
       void* p = nullptr;
       cudaDriverEntryPointQueryResult q;
-      if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess)
+      if (cudaGetDriverEntryPointByVersion(name, &p, 12030, cudaEnableDefault, &q) != cudaSuccess ||
+          q != cudaDriverEntryPointSuccess)
         return nullptr;
       return p;
     };
@@ -852,7 +856,8 @@ bool add_if_node(cudaGraph_t graph, cudaGraphConditionalHandle cond, CUcontext c
   np.conditional.ctx = ctx;
   CUgraphNode n = nullptr;
   CUgraphNode dep = reinterpret_cast<CUgraphNode>(prev);
-  const CUresult rc = api.add_node(&n, reinterpret_cast<CUgraph>(graph), prev ? &dep : nullptr, prev ? 1 : 0, &np);
+  const CUresult rc =
+      api.add_node(&n, reinterpret_cast<CUgraph>(graph), prev ? &dep : nullptr, nullptr, prev ? 1 : 0, &np);
   if (rc != CUDA_SUCCESS) {
     snprintf(g_cond_note, sizeof(g_cond_note), "conditional node refused: cuGraphAddNode returned %d", (int)rc);
     return false;
@@ -951,15 +956,36 @@ int dllm_block_graph_create(const dllm_model* m, const dllm_state* st, const dll
       cudaGraphNode_t node = nullptr;
       cudaGraph_t body = nullptr;
       if (!add_if_node(g->graph, cond, ctx, prev, &node, &body)) {
-        dllm_block_graph_destroy(g);
-        dllm_host::set_error("block_graph_create: a conditional node was refused after the first was accepted");
-        return DLLM_ERR_CUDA;
+        r = DLLM_ERR_CUDA;
+        break;
       }
       r = capture_pass(body, nullptr, 0, t, 0, true);
       prev = node;
     }
     if (!r) r = capture_pass(g->graph, &prev, 1, 0, 1, false);
-  } else {
+    if (!r) {
+      e = cudaGraphInstantiate(&g->exec, g->graph, 0);
+      if (e != cudaSuccess) {
+        snprintf(g_cond_note, sizeof(g_cond_note), "conditional graph not instantiated: %s", cudaGetErrorString(e));
+        r = DLLM_ERR_CUDA;
+      }
+    } else if (!g_cond_note[0]) {
+      snprintf(g_cond_note, sizeof(g_cond_note), "conditional body not captured: %s", dllm_last_error());
+    }
+    if (r) {
+      // the conditional build failed part way: start again with one unconditional capture
+      (void)cudaGetLastError();
+      use_cond = false;
+      r = DLLM_OK;
+      if (g->exec) cudaGraphExecDestroy(g->exec);
+      g->exec = nullptr;
+      cudaGraphDestroy(g->graph);
+      g->graph = nullptr;
+      e = cudaGraphCreate(&g->graph, 0);
+      if (e != cudaSuccess) return fail(e, "block_graph_create: cudaGraphCreate");
+    }
+  }
+  if (!use_cond) {
     // one capture of the whole block: the passes and the commit pass in stream order
     e = cudaStreamBeginCaptureToGraph(capture_stream, g->graph, nullptr, nullptr, 0, cudaStreamCaptureModeThreadLocal);
     if (e != cudaSuccess) return fail(e, "block_graph_create: cudaStreamBeginCaptureToGraph");
@@ -978,8 +1004,10 @@ int dllm_block_graph_create(const dllm_model* m, const dllm_state* st, const dll
     dllm_block_graph_destroy(g);
     return r;
   }
-  e = cudaGraphInstantiate(&g->exec, g->graph, 0);
-  if (e != cudaSuccess) return fail(e, "block_graph_create: cudaGraphInstantiate");
+  if (!g->exec) {
+    e = cudaGraphInstantiate(&g->exec, g->graph, 0);
+    if (e != cudaSuccess) return fail(e, "block_graph_create: cudaGraphInstantiate");
+  }
   g->passes = p->T_s;
   g->conditional = use_cond ? 1 : 0;
   // leave the reason for a graph without conditions in the thread's last-error text (the call still succeeds)

@@ -33,7 +33,7 @@ constexpr int STAGE_COLS = 32;         // epilogue column chunk
 constexpr int STAGING_BYTES = 128 * STAGE_COLS * 4;
 constexpr int MAX_GROUPS = 1040;
 constexpr int NUM_THREADS = 192;
-constexpr int NUM_THREADS_F8 = 320;    // FP8 weights: four more warps turn the E4M3 tiles into bf16 operand tiles
+constexpr int NUM_THREADS_F8 = 448;    // FP8 weights: two groups of four more warps convert alternate E4M3 tiles
 constexpr int RAW_BYTES = 128 * BK;    // 8 KB E4M3 weight tile per stage
 constexpr int SMEM_LIMIT = 232448;
 
@@ -391,12 +391,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
   // bf16 weights: STAGES stages of [A weight tile][B activation tile]. FP8 weights: STAGES stages of [E4M3 weight
   // codes][B activation tile] (half the weight bytes, so a deeper ring), and MS A operand slots of 32 columns in
   // tensor memory that the converter warps fill from the codes.
-  constexpr int MS = F8 ? 3 : 0;
+  // The slots fill the tensor memory the two accumulators leave free: a slot is busy from its conversion through
+  // the MMA's completion (a round trip of some 2000 cycles), so three slots held the FP8 kernel to half the HBM
+  // rate at decode shapes.
+  constexpr int MS = F8 ? ((512 - 2 * BN) / 32 < 16 ? (512 - 2 * BN) / 32 : 16) : 0;
   constexpr int MSD = MS > 0 ? MS : 1;        // slot count as a divisor (the bf16 instantiations use no slots)
   constexpr int W_BYTES = F8 ? RAW_BYTES : A_BYTES;
   constexpr int STAGE_BYTES = W_BYTES + B_BYTES;
   constexpr uint32_t W_TX = W_BYTES;                                      // weight bytes a stage's TMA brings
-  constexpr uint32_t TMEM_COLS = F8 ? (2 * BN + MS * 32 <= 256 ? 256 : 512) : 2 * BN;
+  constexpr uint32_t TMEM_COLS = F8 ? 512 : 2 * BN;
+  static_assert(!F8 || 2 * BN + MS * 32 <= 512, "FP8 A slots exceed the tensor memory");
   uint8_t* stages = base;
   float* staging = reinterpret_cast<float*>(base + STAGES * STAGE_BYTES);
   Smem& sm = *reinterpret_cast<Smem*>(reinterpret_cast<uint8_t*>(staging) + STAGING_BYTES);
@@ -604,17 +608,20 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
       tc::mbar_wait(&sm.done, 0, 1u << 20);
     }
   } else if (F8 && warp >= 6) {
-    // ------------------------------------------------------------------ FP8: converter warps 6..9
-    // per k-block, in the MMA's order: once the A slot is free and the stage's codes have landed, each thread writes
-    // its TMEM lane (the warp's quadrant) of the slot from its row of codes, waits for its stores, and arrives on the
-    // slot's conv barrier
+    // ------------------------------------------------------------------ FP8: converter warps 6..13
+    // two groups of four warps (one per TMEM lane quadrant) take alternate k-blocks, so that one group's loads,
+    // conversions and store waits overlap the other's. Per k-block, in the MMA's order: once the A slot is free and
+    // the stage's codes have landed, each thread writes its TMEM lane of the slot from its row of codes, waits for
+    // its stores, and arrives on the slot's conv barrier
     const int row = (warp & 3) * 32 + lane;   // the TMEM lane this warp may access
+    const uint32_t cg = (uint32_t)(warp - 6) >> 2;
     uint32_t it = 0;
     bool ok = true;
     for (int wk = wk_begin; wk < total && ok; wk += wk_step) {
       const int ks = wk - (wk / p.ksplit) * p.ksplit;
       const int kb0 = ks * kblocks / p.ksplit, kb1 = (ks + 1) * kblocks / p.ksplit;
       for (int kb = kb0; kb < kb1; ++kb, ++it) {
+        if ((it & 1u) != cg) continue;   // the other group's k-block
         const int s = it % STAGES, ms = it % MSD;
         if (!wait_bar(&sm.mempty[ms], ((it / MSD) & 1) ^ 1, abort_flag, p.status, ST_TIMEOUT_MMA) ||
             !wait_bar(&sm.full[s], (it / STAGES) & 1, abort_flag, p.status, ST_TIMEOUT_MMA)) { ok = false; break; }

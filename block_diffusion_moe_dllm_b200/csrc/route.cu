@@ -374,63 +374,44 @@ DLLM_DEV void cta_redecide(RedecideSmem<NW>& rs, const float* __restrict__ score
   }
 }
 
-// Tokens [t0, t1) whose fix_thr is not NaN (near-ties flagged by route_topk_kernel) into the CTA's list; past the
-// list's capacity, the token's warp decides it alone. Every warp of the CTA calls this; rs.n_flag starts at 0.
-template <int PER, int NW, typename T>
-DLLM_DEV void collect_flagged(RedecideSmem<NW>& rd, int t0, int t1, const float* __restrict__ fix_thr,
-                              const float* __restrict__ scores, const float* __restrict__ bias, int E, int k,
-                              const T* __restrict__ h, const T* __restrict__ w, int H, int32_t* __restrict__ ids,
-                              float* __restrict__ gates) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int tb = t0 + warp * 32; tb < t1; tb += NW * 32) {
-    const int t = tb + lane;
-    const float th = t < t1 ? fix_thr[t] : __int_as_float(0x7fc00000);
-    const bool fl = !isnan(th);
-    const unsigned bal = __ballot_sync(0xffffffffu, fl);
-    int base = 0;
-    if (lane == 0 && bal) base = atomicAdd(&rd.n_flag, __popc(bal));
-    base = __shfl_sync(0xffffffffu, base, 0);
-    const int f = base + __popc(bal & ((1u << lane) - 1u));
-    if (fl && f < kMaxFlagged) {
-      rd.ftok[f] = t;
-      rd.fthr[f] = th;
-    }
-    unsigned over = __ballot_sync(0xffffffffu, fl && f >= kMaxFlagged);
-    while (over) {
-      const int j = __ffs(over) - 1;
-      over &= over - 1;
-      const int tt = tb + j;
-      int my_id;
-      float my_gate;
-      exact_redecide<PER>(scores + (int64_t)tt * E, bias, E, k, h + (int64_t)tt * H, w, H,
-                          __shfl_sync(0xffffffffu, th, j), lane, my_id, my_gate);
-      if (lane < k) {
-        ids[(int64_t)tt * k + lane] = my_id;
-        gates[(int64_t)tt * k + lane] = my_gate;
-      }
-    }
-  }
-}
-
-// Many tokens: one warp per token, the fp32 selection. A token whose selection is a near-tie (see kRouteGuard) gets
-// fix_thr[t] = its candidate threshold, every other token NaN; the histogram launch decides those tokens again
-// before it counts.
-template <int PER>
-__global__ void route_topk_kernel(float* __restrict__ scores, const float* __restrict__ bias, int Tk, int E, int k,
-                                  int from_logits, int32_t* __restrict__ ids, float* __restrict__ gates,
-                                  float* __restrict__ fix_thr, const int32_t* __restrict__ live) {
+// Many tokens: one warp per token, 8 tokens per CTA, the fp32 selection; the CTA's near-tie tokens (see
+// kRouteGuard) are then decided again exactly by the CTA's 8 warps together (cta_redecide). Near-ties are rare and
+// spread over the CTAs, so the exact dot products run in parallel across the GPU.
+template <int PER, typename T>
+__global__ void __launch_bounds__(256) route_topk_kernel(float* __restrict__ scores, const float* __restrict__ bias,
+                                                         int Tk, int E, int k, int from_logits,
+                                                         const T* __restrict__ h, const T* __restrict__ w, int H,
+                                                         int32_t* __restrict__ ids, float* __restrict__ gates,
+                                                         const int32_t* __restrict__ live) {
   pdl_enter();
   if (live && *live == 0) return;   // a pass with no masked position left does nothing
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-  if (warp >= Tk) return;
-  int my_id;
-  float my_gate, thr;
-  const bool near = warp_topk<PER>(scores + (int64_t)warp * E, bias, E, k, from_logits, lane, my_id, my_gate, thr);
-  if (lane < k) {
-    ids[(int64_t)warp * k + lane] = my_id;
-    gates[(int64_t)warp * k + lane] = my_gate;
+  __shared__ RedecideSmem<8> rd;
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  const int t = blockIdx.x * 8 + wib;
+  if (threadIdx.x == 0) rd.n_flag = 0;
+  __syncthreads();
+  if (t < Tk) {
+    int my_id;
+    float my_gate, thr;
+    const bool near = warp_topk<PER>(scores + (int64_t)t * E, bias, E, k, from_logits, lane, my_id, my_gate, thr);
+    if (lane < k) {
+      ids[(int64_t)t * k + lane] = my_id;
+      gates[(int64_t)t * k + lane] = my_gate;
+    }
+    if (near && lane == 0) {
+      const int f = atomicAdd(&rd.n_flag, 1);   // at most 8 <= kMaxFlagged
+      rd.ftok[f] = t;
+      rd.fthr[f] = thr;
+    }
   }
-  if (lane == 0) fix_thr[warp] = near ? thr : __int_as_float(0x7fc00000);
+  __syncthreads();
+  if (rd.n_flag == 0) return;   // uniform over the CTA
+  cta_redecide<PER, 8>(rd, scores, bias, E, k, h, w, H, [&](int tt, int ln, int id, float g) {
+    if (ln < k) {
+      ids[(int64_t)tt * k + ln] = id;
+      gates[(int64_t)tt * k + ln] = g;
+    }
+  });
 }
 
 // Few tokens (Tk <= 32, Tk * k <= 1024, E <= 256): top-k (with the exact re-decision of near-ties) and the stable
@@ -542,39 +523,20 @@ __global__ void __launch_bounds__(1024) route_small_kernel(float* __restrict__ s
 }
 
 // Stable permutation for many assignments, in three launches over segments of seg_tok consecutive tokens (seg_tok
-// * k assignments, a multiple of 256): per-segment expert histograms (after the segment's near-tie tokens are
-// decided again); one CTA turns them into counts, offsets and every segment's first output position per expert;
+// * k assignments, a multiple of 256): per-segment expert histograms; one CTA turns them into counts, offsets and every segment's first output position per expert;
 // then each segment writes its assignments' positions in order. Positions within an expert follow the assignment
 // index a = t * k + j, so an expert's rows stay sorted by token.
 
-// Exact re-decision of the segment's flagged tokens (a warp per token; fix_thr as written by route_topk_kernel),
-// then seg_hist[s][e] = assignments of expert e in segment s.
-template <int PER, typename T>
-__global__ void __launch_bounds__(256) route_seg_hist_kernel(int32_t* __restrict__ ids, float* __restrict__ gates,
-                                                             const float* __restrict__ scores,
-                                                             const float* __restrict__ bias,
-                                                             const float* __restrict__ fix_thr,
-                                                             const T* __restrict__ h, const T* __restrict__ w, int H,
-                                                             int Tk, int E, int k, int seg_tok,
-                                                             int32_t* __restrict__ seg_hist,
+// seg_hist[s][e] = assignments of expert e in segment s.
+__global__ void __launch_bounds__(256) route_seg_hist_kernel(const int32_t* __restrict__ ids, int Tk, int k,
+                                                             int E, int seg_tok, int32_t* __restrict__ seg_hist,
                                                              const int32_t* __restrict__ live) {
   pdl_enter();
   if (live && *live == 0) return;   // a pass with no masked position left does nothing
   extern __shared__ int sh_hist[];
-  __shared__ RedecideSmem<8> rd;
   for (int i = threadIdx.x; i < E; i += blockDim.x) sh_hist[i] = 0;
-  if (threadIdx.x == 0) rd.n_flag = 0;
   __syncthreads();
   const int t0 = blockIdx.x * seg_tok, t1 = min(Tk, t0 + seg_tok);
-  collect_flagged<PER, 8>(rd, t0, t1, fix_thr, scores, bias, E, k, h, w, H, ids, gates);
-  __syncthreads();
-  cta_redecide<PER, 8>(rd, scores, bias, E, k, h, w, H, [&](int t, int ln, int id, float g) {
-    if (ln < k) {
-      ids[(int64_t)t * k + ln] = id;
-      gates[(int64_t)t * k + ln] = g;
-    }
-  });
-  __syncthreads();   // the re-decided ids (global writes of this CTA) are visible to the whole CTA
   const int a0 = t0 * k, a1 = t1 * k;
   for (int a = a0 + threadIdx.x; a < a1; a += blockDim.x) atomicAdd(&sh_hist[ids[a]], 1);
   __syncthreads();
@@ -699,42 +661,26 @@ __global__ void __launch_bounds__(256) route_seg_scatter_kernel(const int32_t* _
   }
 }
 
-// Mid-size routing (E <= 256, Tk * k <= kPermCtaMax): after route_topk_kernel, one CTA of 1024 threads decides the
-// flagged near-tie tokens again and builds counts, offsets and the stable permutation, in place of the segmented
-// three launches. Warp w takes the assignments [w per, (w + 1) per) (per a multiple of 32); pass 1 counts them per
-// expert (__match_any_sync groups), the 32 warps' counts are prefixed per expert on top of the expert's offset, and
-// pass 2 writes position = warp's running base + rank among the chunk's lanes with the same expert, so positions
-// within an expert follow the assignment index a = t k + j, as in the other permutation kernels.
+// Mid-size routing (Tk * k <= kPermCtaMax): after route_topk_kernel, one CTA of 1024 threads builds counts, offsets
+// and the stable permutation, in place of the segmented three launches. Warp w takes the assignments
+// [w per, (w + 1) per) (per a multiple of 32); pass 1 counts them per expert (__match_any_sync groups), the 32
+// warps' counts are prefixed per expert on top of the expert's offset, and pass 2 writes position = warp's running
+// base + rank among the chunk's lanes with the same expert, so positions within an expert follow the assignment
+// index a = t k + j, as in the other permutation kernels.
 constexpr int kPermCtaMax = 8192;
 
-template <int PER, typename T>
-__global__ void __launch_bounds__(1024) route_perm_cta_kernel(int32_t* __restrict__ ids, float* __restrict__ gates,
-                                                              const float* __restrict__ scores,
-                                                              const float* __restrict__ bias,
-                                                              const float* __restrict__ fix_thr,
-                                                              const T* __restrict__ h, const T* __restrict__ w, int H,
-                                                              int Tk, int E, int k, int32_t* __restrict__ counts,
+__global__ void __launch_bounds__(1024) route_perm_cta_kernel(const int32_t* __restrict__ ids, int Tk, int E, int k,
+                                                              int32_t* __restrict__ counts,
                                                               int32_t* __restrict__ offsets,
                                                               int32_t* __restrict__ perm, int32_t* __restrict__ inv,
                                                               const int32_t* __restrict__ live) {
   pdl_enter();
   if (live && *live == 0) return;   // a pass with no masked position left does nothing
   extern __shared__ int wh[];        // [32][E]
-  __shared__ RedecideSmem<32> rd;
   __shared__ int wtot[32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   for (int i = tid; i < 32 * E; i += blockDim.x) wh[i] = 0;
-  if (tid == 0) rd.n_flag = 0;
   __syncthreads();
-  collect_flagged<PER, 32>(rd, 0, Tk, fix_thr, scores, bias, E, k, h, w, H, ids, gates);
-  __syncthreads();
-  cta_redecide<PER, 32>(rd, scores, bias, E, k, h, w, H, [&](int t, int ln, int id, float g) {
-    if (ln < k) {
-      ids[(int64_t)t * k + ln] = id;
-      gates[(int64_t)t * k + ln] = g;
-    }
-  });
-  __syncthreads();   // the re-decided ids (global writes of this CTA) are visible to the whole CTA
   const int n = Tk * k;
   const int per = ((n + 31) / 32 + 31) & ~31;
   const int a0 = min(n, warp * per), a1 = min(n, a0 + per);
@@ -800,11 +746,10 @@ __global__ void __launch_bounds__(1024) route_perm_cta_kernel(int32_t* __restric
 
 }  // namespace
 
-// Layout of the router scratch: per-segment expert histograms, then one fp32 near-tie threshold per token.
+// Layout of the router scratch: per-segment expert histograms.
 struct RouteScratch {
   int seg_tok, S;
   int32_t* seg_hist;
-  float* fix_thr;
 };
 
 RouteScratch route_scratch(int Tk, int E, int k, void* base) {
@@ -812,8 +757,8 @@ RouteScratch route_scratch(int Tk, int E, int k, void* base) {
   r.seg_tok = route_segment_tokens(Tk, k);
   r.S = std::max(1, (Tk + r.seg_tok - 1) / r.seg_tok);
   const size_t hist = ((size_t)r.S * E * sizeof(int32_t) + 255) & ~size_t(255);
+  (void)hist;
   r.seg_hist = static_cast<int32_t*>(base);
-  r.fix_thr = base ? reinterpret_cast<float*>(static_cast<char*>(base) + hist) : nullptr;
   return r;
 }
 
@@ -837,28 +782,26 @@ int launch_select_per(float* scores, const float* bias, int Tk, int E, int k, in
     }
   }
   const RouteScratch rs = route_scratch(Tk, E, k, scratch);
-  // one warp per token, 4 per CTA: many tokens spread over all the SMs (one thread per token, tried for thousands
+  // one warp per token, 8 per CTA: many tokens spread over all the SMs (one thread per token, tried for thousands
   // of tokens, reads each 1 KB score row with 32 lines in flight per warp instruction and was 2x slower)
-  launch_pdl(route_topk_kernel<PER>, (Tk + 3) / 4, 128, 0, s, scores, bias, Tk, E, k, from_logits, ids, gates,
-             rs.fix_thr, live);
+  launch_pdl(route_topk_kernel<PER, T>, (Tk + 7) / 8, 256, 0, s, scores, bias, Tk, E, k, from_logits, h, w, H, ids,
+             gates, live);
   DLLM_CHECK_LAUNCH("route_topk_kernel");
   const int n = Tk * k, seg = rs.seg_tok * k;
-  if constexpr (PER <= 8) {
-    if (n <= kPermCtaMax) {   // one CTA decides the flagged tokens again and builds the permutation
-      const size_t smem = (size_t)32 * E * sizeof(int);
-      static bool cfg = false;
-      if (!cfg) {
-        cudaFuncSetAttribute(route_perm_cta_kernel<PER, T>, cudaFuncAttributeMaxDynamicSharedMemorySize, 32 * 1024);
-        cfg = true;
-      }
-      launch_pdl(route_perm_cta_kernel<PER, T>, 1, 1024, smem, s, ids, gates, (const float*)scores, bias,
-                 (const float*)rs.fix_thr, h, w, H, Tk, E, k, counts, offsets, perm, inv, live);
-      DLLM_CHECK_LAUNCH("route_perm_cta_kernel");
-      return DLLM_OK;
+  if (n <= kPermCtaMax) {   // one CTA builds the permutation
+    const size_t smem = (size_t)32 * E * sizeof(int);
+    static bool cfg = false;
+    if (!cfg) {
+      cudaFuncSetAttribute(route_perm_cta_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 128 * 1024);
+      cfg = true;
     }
+    launch_pdl(route_perm_cta_kernel, 1, 1024, smem, s, (const int32_t*)ids, Tk, E, k, counts, offsets, perm, inv,
+               live);
+    DLLM_CHECK_LAUNCH("route_perm_cta_kernel");
+    return DLLM_OK;
   }
-  launch_pdl(route_seg_hist_kernel<PER, T>, rs.S, 256, (size_t)E * sizeof(int), s, ids, gates,
-             (const float*)scores, bias, (const float*)rs.fix_thr, h, w, H, Tk, E, k, rs.seg_tok, rs.seg_hist, live);
+  launch_pdl(route_seg_hist_kernel, rs.S, 256, (size_t)E * sizeof(int), s, (const int32_t*)ids, Tk, k, E,
+             rs.seg_tok, rs.seg_hist, live);
   DLLM_CHECK_LAUNCH("route_seg_hist_kernel");
   launch_pdl(route_seg_scan_kernel, 1, 1024, 0, s, rs.seg_hist, rs.S, E, n, counts, offsets, live);
   DLLM_CHECK_LAUNCH("route_seg_scan_kernel");
@@ -897,8 +840,7 @@ int route_segment_tokens(int Tk, int k) {
 
 size_t route_scratch_bytes(int Tk, int E, int k) {
   const RouteScratch r = route_scratch(Tk, E, k, nullptr);
-  const size_t hist = ((size_t)r.S * E * sizeof(int32_t) + 255) & ~size_t(255);
-  return hist + (size_t)std::max(Tk, 1) * sizeof(float);
+  return ((size_t)r.S * E * sizeof(int32_t) + 255) & ~size_t(255);
 }
 
 int launch_route(int dtype, const void* h, const void* w_router, const float* bias, int Tk, int H, int E, int k,

@@ -87,10 +87,29 @@ def _check_pass(w, eng, f, dtype):
     return flag
 
 
+def _score_shift(score, r, c, dz):
+    """First-order bound on how far a position score r (largest probability c) moves when every logit of the row
+    moves by at most dz: dp_v = p_v (dz_v - sum_u p_u dz_u), so |dp_v| <= 2 dz p_v. top_k_margin p1 - p2 moves by
+    at most 2 dz (p1 + p2) <= 4 dz c; neg_entropy sum_v p_v log p_v moves by sum_v |log p_v + 1| |dp_v|
+    <= 2 dz (|r| + 1)."""
+    if score == 1:
+        return 4.0 * dz * c
+    return 2.0 * dz * (abs(r) + 1.0)
+
+
 def _decisions_agree(w, u_or, eng, flag):
     """Compare the unmask decisions where the oracle's choice is not a near-tie (ranking by the workload's score,
-    threshold on the largest probability)."""
+    threshold on the largest probability). For the margin and entropy scores the near-tie band also covers what
+    the observed difference between the two sides' logits (dz, largest over the scored rows; guidance scales it by
+    1 + 2 s) can move the scores by."""
     Bl = w.B // 2 if w.cfg else w.B
+    dz = 0.0
+    if w.score:
+        f = u_or["forward"]
+        n = len(f["row_pos"])
+        dz = float(np.max(np.abs(to64(eng.logits(n)) - f["logits"]))) if n else 0.0
+        if w.cfg:
+            dz *= 1.0 + 2.0 * abs(w.cfg_scale)
     g_mask = eng.mask.cpu().numpy()
     g_nsel = eng.nsel.cpu().numpy()
     clean = True
@@ -98,11 +117,16 @@ def _decisions_agree(w, u_or, eng, flag):
         c = u_or["conf"][b]
         rk = u_or["rank"][b][c > 0]
         row_flag = flag[b * w.L:(b + 1) * w.L].any() or (w.cfg and flag[(b + Bl) * w.L:(b + Bl + 1) * w.L].any())
-        ranked = np.sort(rk)[::-1]
+        order = np.argsort(-rk, kind="stable")
+        ranked, c_ranked = rk[order], c[c > 0][order]
         k = u_or["nsel"][b]
         near = False
         if 0 < k < len(ranked):
-            near = (ranked[k - 1] - ranked[k]) < E2E_CONF_MARGIN * max(abs(ranked[k - 1]), 1e-30)
+            gap = ranked[k - 1] - ranked[k]
+            near = gap < E2E_CONF_MARGIN * max(abs(ranked[k - 1]), 1e-30)
+            if w.score:   # the band a logit difference of up to dz can move the two scores by
+                near |= gap < 2.0 * (_score_shift(w.score, ranked[k - 1], c_ranked[k - 1], dz) +
+                                     _score_shift(w.score, ranked[k], c_ranked[k], dz))
         if w.mode == 1:
             near |= bool(np.any(np.abs(c[c > 0] - w.tau) < E2E_CONF_MARGIN))
         if near or row_flag:

@@ -31,7 +31,8 @@ int launch_combine_norm(int dtype, void* x, const float* y, const float* gates, 
 // router
 int num_sms();
 
-// seg_scratch: route_scratch_bytes(Tk, E, k) bytes, 256-byte aligned (per-segment histograms of the permutation)
+// seg_scratch: route_scratch_bytes(Tk, E, k) bytes, 256-byte aligned (per-segment histograms of the permutation and
+// the near-tie thresholds of the selection)
 int launch_route(int dtype, const void* h, const void* w_router, const float* bias, int Tk, int H, int E, int k,
                  int32_t* ids, float* gates, float* scores, int32_t* counts, int32_t* offsets, int32_t* perm,
                  int32_t* inv, void* seg_scratch, cudaStream_t s, const int32_t* live = nullptr);

@@ -285,6 +285,105 @@ DLLM_DEV void exact_redecide(const float* __restrict__ srow, const float* __rest
   my_gate = (float)(mine / gsum);
 }
 
+// Exact dot-product terms of one 16-byte chunk of a row pair, added in fp64: bf16 products are exact in fp32, fp32
+// products are formed in fp64.
+DLLM_DEV void acc16(const uint4& hv, const uint4& wv, double& s, const __nv_bfloat16*) {
+  float fh[8], fw[8];
+  bf16x8_to_f32(hv, fh);
+  bf16x8_to_f32(wv, fw);
+  double a = 0.0, b = 0.0;
+#pragma unroll
+  for (int u = 0; u < 8; u += 2) {
+    a += (double)(fh[u] * fw[u]);
+    b += (double)(fh[u + 1] * fw[u + 1]);
+  }
+  s += a + b;
+}
+DLLM_DEV void acc16(const uint4& hv, const uint4& wv, double& s, const float*) {
+  s = fma((double)__uint_as_float(hv.x), (double)__uint_as_float(wv.x), s);
+  s = fma((double)__uint_as_float(hv.y), (double)__uint_as_float(wv.y), s);
+  s = fma((double)__uint_as_float(hv.z), (double)__uint_as_float(wv.z), s);
+  s = fma((double)__uint_as_float(hv.w), (double)__uint_as_float(wv.w), s);
+}
+
+// Exact selection of one near-tie token by its own warp. The candidate experts (fp32 biased score at least thr,
+// the (k+1)-th value minus the guard) are compacted into lanes; their exact scores come four candidates at a time,
+// each lane holding its 16-byte chunks of the four weight rows and of the token row at once (eight chunks per lane
+// in flight), so a candidate group costs about one trip to L2 per 2048 bf16 elements instead of one per candidate;
+// then k rounds of a warp arg-max give the slots in order (ties -> lower expert) and the gates (unbiased fp64
+// scores renormalised). More than 32 candidates (only with many equal scores): exact_redecide.
+template <int PER, typename T>
+DLLM_DEV void warp_exact_select(float* __restrict__ srow, const float* __restrict__ bias, int E, int k,
+                                const T* __restrict__ hrow, const T* __restrict__ w, int H, float thr, int lane,
+                                int& my_id, float& my_gate) {
+  __syncwarp();   // the warp's own write-back of the sigmoid scores is visible to every lane
+  constexpr int VE = 16 / sizeof(T);   // elements per 16-byte chunk
+  constexpr int CH = 8;                // chunks per lane per pass over the row
+  int n = 0, ce = 0x7fffffff;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int ex = i * 32 + lane;
+    unsigned bal = __ballot_sync(0xffffffffu, ex < E && srow[ex] + bias[ex] >= thr);
+    while (bal) {
+      const int src = __ffs(bal) - 1;
+      bal &= bal - 1;
+      if (lane == n) ce = i * 32 + src;
+      ++n;
+    }
+  }
+  if (n > 32) {
+    exact_redecide<PER>(srow, bias, E, k, hrow, w, H, thr, lane, my_id, my_gate);
+    return;
+  }
+  double cv = -INFINITY;   // lane j < n: exact biased score of candidate j
+  for (int c0 = 0; c0 < n; c0 += 4) {
+    int eq[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) eq[q] = __shfl_sync(0xffffffffu, ce, min(c0 + q, n - 1));
+    double acc[4] = {0.0, 0.0, 0.0, 0.0};
+    for (int b0 = 0; b0 < H; b0 += 32 * VE * CH) {
+      uint4 hv[CH], wv[4][CH];
+#pragma unroll
+      for (int j = 0; j < CH; ++j) {
+        const int c = b0 + (j * 32 + lane) * VE;
+        const bool in = c < H;
+        hv[j] = in ? *reinterpret_cast<const uint4*>(hrow + c) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          wv[q][j] = in ? *reinterpret_cast<const uint4*>(w + (int64_t)eq[q] * H + c) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int j = 0; j < CH; ++j) acc16(hv[j], wv[q][j], acc[q], hrow);
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const double dot = warp_sum(acc[q]);
+      if (lane == c0 + q && c0 + q < n) cv = 1.0 / (1.0 + exp(-dot)) + (double)bias[eq[q]];
+    }
+  }
+  double v = lane < n ? cv : -INFINITY;
+  const int e = lane < n ? ce : 0x7fffffff;
+  double gsum = 0.0, mine = 0.0;
+  my_id = 0;
+  for (int j = 0; j < k; ++j) {
+    double bv = v;
+    int be = e;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const double ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+      if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
+    }
+    if (e == be) v = -INFINITY;
+    const double sc = bv - (double)bias[be];
+    gsum += sc;
+    if (lane == j) { my_id = be; mine = sc; }
+  }
+  my_gate = (float)(mine / gsum);
+}
+
 // Cooperative exact re-decision of a CTA's near-tie tokens. The warps first list their flagged tokens; then, in
 // rounds of one flagged token per warp, (a) each warp lists its token's candidate experts (those whose fp32 biased
 // score is at least the token's threshold, at most 32 of them), (b) all warps of the CTA compute the candidates'
@@ -374,44 +473,60 @@ DLLM_DEV void cta_redecide(RedecideSmem<NW>& rs, const float* __restrict__ score
   }
 }
 
-// Many tokens: one warp per token, 8 tokens per CTA, the fp32 selection; the CTA's near-tie tokens (see
-// kRouteGuard) are then decided again exactly by the CTA's 8 warps together (cta_redecide). Near-ties are rare and
-// spread over the CTAs, so the exact dot products run in parallel across the GPU.
-template <int PER, typename T>
-__global__ void __launch_bounds__(256) route_topk_kernel(float* __restrict__ scores, const float* __restrict__ bias,
-                                                         int Tk, int E, int k, int from_logits,
-                                                         const T* __restrict__ h, const T* __restrict__ w, int H,
-                                                         int32_t* __restrict__ ids, float* __restrict__ gates,
-                                                         const int32_t* __restrict__ live) {
+// Many tokens: one warp per token, the fp32 selection. A token whose selection is a near-tie (see kRouteGuard) gets
+// fix_thr[t] = its candidate threshold, every other token NaN; route_exact_kernel decides those tokens again.
+template <int PER>
+__global__ void route_topk_kernel(float* __restrict__ scores, const float* __restrict__ bias, int Tk, int E, int k,
+                                  int from_logits, int32_t* __restrict__ ids, float* __restrict__ gates,
+                                  float* __restrict__ fix_thr, const int32_t* __restrict__ live) {
   pdl_enter();
   if (live && *live == 0) return;   // a pass with no masked position left does nothing
-  __shared__ RedecideSmem<8> rd;
-  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-  const int t = blockIdx.x * 8 + wib;
-  if (threadIdx.x == 0) rd.n_flag = 0;
-  __syncthreads();
-  if (t < Tk) {
-    int my_id;
-    float my_gate, thr;
-    const bool near = warp_topk<PER>(scores + (int64_t)t * E, bias, E, k, from_logits, lane, my_id, my_gate, thr);
-    if (lane < k) {
-      ids[(int64_t)t * k + lane] = my_id;
-      gates[(int64_t)t * k + lane] = my_gate;
-    }
-    if (near && lane == 0) {
-      const int f = atomicAdd(&rd.n_flag, 1);   // at most 8 <= kMaxFlagged
-      rd.ftok[f] = t;
-      rd.fthr[f] = thr;
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (warp >= Tk) return;
+  int my_id;
+  float my_gate, thr;
+  const bool near = warp_topk<PER>(scores + (int64_t)warp * E, bias, E, k, from_logits, lane, my_id, my_gate, thr);
+  if (lane < k) {
+    ids[(int64_t)warp * k + lane] = my_id;
+    gates[(int64_t)warp * k + lane] = my_gate;
+  }
+  if (lane == 0) fix_thr[warp] = near ? thr : __int_as_float(0x7fc00000);
+}
+
+// The near-tie tokens flagged by route_topk_kernel, decided again exactly, one warp per token (warp_exact_select):
+// a persistent grid whose warp w takes the tokens w, w + W, w + 2W, ... (W warps in all), reading 32 of their flags
+// at once, so near-ties that cluster in neighbouring tokens still spread over every warp. Kept apart from the top-k
+// kernel, whose register budget it would otherwise set.
+template <int PER, typename T>
+__global__ void __launch_bounds__(256, 1) route_exact_kernel(float* __restrict__ scores,
+                                                             const float* __restrict__ bias, int Tk, int E, int k,
+                                                             const T* __restrict__ h, const T* __restrict__ w,
+                                                             int H, const float* __restrict__ fix_thr,
+                                                             int32_t* __restrict__ ids, float* __restrict__ gates,
+                                                             const int32_t* __restrict__ live) {
+  pdl_enter();
+  if (live && *live == 0) return;   // a pass with no masked position left does nothing
+  const int lane = threadIdx.x & 31;
+  const int gw = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int W = gridDim.x * (blockDim.x >> 5);
+  for (int base = gw; base < Tk; base += 32 * W) {
+    const int t = base + lane * W;
+    const float th = t < Tk ? fix_thr[t] : __int_as_float(0x7fc00000);
+    unsigned bal = __ballot_sync(0xffffffffu, !isnan(th));
+    while (bal) {
+      const int j = __ffs(bal) - 1;
+      bal &= bal - 1;
+      const int tt = base + j * W;
+      int my_id;
+      float my_gate;
+      warp_exact_select<PER>(scores + (int64_t)tt * E, bias, E, k, h + (int64_t)tt * H, w, H,
+                             __shfl_sync(0xffffffffu, th, j), lane, my_id, my_gate);
+      if (lane < k) {
+        ids[(int64_t)tt * k + lane] = my_id;
+        gates[(int64_t)tt * k + lane] = my_gate;
+      }
     }
   }
-  __syncthreads();
-  if (rd.n_flag == 0) return;   // uniform over the CTA
-  cta_redecide<PER, 8>(rd, scores, bias, E, k, h, w, H, [&](int tt, int ln, int id, float g) {
-    if (ln < k) {
-      ids[(int64_t)tt * k + ln] = id;
-      gates[(int64_t)tt * k + ln] = g;
-    }
-  });
 }
 
 // Few tokens (Tk <= 32, Tk * k <= 1024, E <= 256): top-k (with the exact re-decision of near-ties) and the stable
@@ -746,10 +861,11 @@ __global__ void __launch_bounds__(1024) route_perm_cta_kernel(const int32_t* __r
 
 }  // namespace
 
-// Layout of the router scratch: per-segment expert histograms.
+// Layout of the router scratch: per-segment expert histograms, then one fp32 near-tie threshold per token.
 struct RouteScratch {
   int seg_tok, S;
   int32_t* seg_hist;
+  float* fix_thr;
 };
 
 RouteScratch route_scratch(int Tk, int E, int k, void* base) {
@@ -757,8 +873,8 @@ RouteScratch route_scratch(int Tk, int E, int k, void* base) {
   r.seg_tok = route_segment_tokens(Tk, k);
   r.S = std::max(1, (Tk + r.seg_tok - 1) / r.seg_tok);
   const size_t hist = ((size_t)r.S * E * sizeof(int32_t) + 255) & ~size_t(255);
-  (void)hist;
   r.seg_hist = static_cast<int32_t*>(base);
+  r.fix_thr = base ? reinterpret_cast<float*>(static_cast<char*>(base) + hist) : nullptr;
   return r;
 }
 
@@ -782,11 +898,14 @@ int launch_select_per(float* scores, const float* bias, int Tk, int E, int k, in
     }
   }
   const RouteScratch rs = route_scratch(Tk, E, k, scratch);
-  // one warp per token, 8 per CTA: many tokens spread over all the SMs (one thread per token, tried for thousands
+  // one warp per token, 4 per CTA: many tokens spread over all the SMs (one thread per token, tried for thousands
   // of tokens, reads each 1 KB score row with 32 lines in flight per warp instruction and was 2x slower)
-  launch_pdl(route_topk_kernel<PER, T>, (Tk + 7) / 8, 256, 0, s, scores, bias, Tk, E, k, from_logits, h, w, H, ids,
-             gates, live);
+  launch_pdl(route_topk_kernel<PER>, (Tk + 3) / 4, 128, 0, s, scores, bias, Tk, E, k, from_logits, ids, gates,
+             rs.fix_thr, live);
   DLLM_CHECK_LAUNCH("route_topk_kernel");
+  launch_pdl(route_exact_kernel<PER, T>, std::min(num_sms(), (Tk + 7) / 8), 256, 0, s, scores, bias, Tk, E, k, h, w,
+             H, (const float*)rs.fix_thr, ids, gates, live);
+  DLLM_CHECK_LAUNCH("route_exact_kernel");
   const int n = Tk * k, seg = rs.seg_tok * k;
   if (n <= kPermCtaMax) {   // one CTA builds the permutation
     const size_t smem = (size_t)32 * E * sizeof(int);
@@ -840,7 +959,8 @@ int route_segment_tokens(int Tk, int k) {
 
 size_t route_scratch_bytes(int Tk, int E, int k) {
   const RouteScratch r = route_scratch(Tk, E, k, nullptr);
-  return ((size_t)r.S * E * sizeof(int32_t) + 255) & ~size_t(255);
+  const size_t hist = ((size_t)r.S * E * sizeof(int32_t) + 255) & ~size_t(255);
+  return hist + (size_t)std::max(Tk, 1) * sizeof(float);
 }
 
 int launch_route(int dtype, const void* h, const void* w_router, const float* bias, int Tk, int H, int E, int k,

@@ -119,8 +119,8 @@ def test_grouped_gemm_rejects_bad_arguments(lib):
 
 
 def test_route_workspace_covers_scores_and_permutation_segments(lib):
-    """The router's workspace holds the fp32 scores and one expert histogram per permutation segment (segments of
-    whole tokens, a multiple of 256 assignments, at most 128 of them)."""
+    """The router's workspace holds the fp32 scores, one expert histogram per permutation segment (segments of
+    whole tokens, a multiple of 256 assignments, at most 128 of them) and one near-tie threshold per token."""
     import math
     lib.dllm_moe_route_workspace_size.restype = C.c_size_t
     for Tk, E, k in [(32, 256, 8), (512, 256, 8), (32768, 256, 8), (1001, 1000, 3), (5000, 96, 4), (77, 256, 6)]:
@@ -129,7 +129,7 @@ def test_route_workspace_covers_scores_and_permutation_segments(lib):
         assert (seg_tok * k) % 256 == 0
         segments = -(-Tk // seg_tok)
         assert segments <= 128
-        need = Tk * E * 4 + segments * E * 4
+        need = Tk * E * 4 + segments * E * 4 + Tk * 4
         r = bd.RouteDesc(Tk, 2048, E, k, bd.BF16)
         assert lib.dllm_moe_route_workspace_size(C.byref(r)) >= need
 

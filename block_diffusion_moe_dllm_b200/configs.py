@@ -109,7 +109,12 @@ PREFILL = Workload("prefill-1layer-b8-4096", "bf16", 1, 2048, 16, 4, 128, 256, 8
 ONE_LAYER_FP8 = replace(ONE_LAYER, name="moe-dllm-1layer-p1024-b1-fp8", wfmt="fp8")
 UNDERSTANDING_FP8 = replace(UNDERSTANDING, name="understanding-20layer-b16-p2688-thr0.9-fp8", wfmt="fp8")
 
-ALL = [TINY_F32, ONE_LAYER, T2I, THINKING, UNDERSTANDING, PREFILL, ONE_LAYER_FP8, UNDERSTANDING_FP8]
+# one layer of the understanding workload (its batch, prefix and vocabulary): the size a profiler capture of the
+# step's kernels takes (a few GB on the device)
+UNDERSTANDING_1LAYER = replace(UNDERSTANDING, name="understanding-1layer-b16-p2688-thr0.9", n_layers=1)
+
+ALL = [TINY_F32, ONE_LAYER, T2I, THINKING, UNDERSTANDING, PREFILL, ONE_LAYER_FP8, UNDERSTANDING_FP8,
+       UNDERSTANDING_1LAYER]
 BY_NAME = {w.name: w for w in ALL}
 
 

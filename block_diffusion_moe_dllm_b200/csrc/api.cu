@@ -237,6 +237,8 @@ int validate_step(const dllm_model* m, const dllm_state* st, const dllm_step_par
   if (m->weight_format == DLLM_WEIGHTS_FP8) {
     REQ(m->dtype == DLLM_BF16, DLLM_ERR_UNSUPPORTED, "denoise_step: FP8 weights need bf16 storage");
     REQ(m->w_lm_scale, DLLM_ERR_INVALID_ARG, "denoise_step: FP8 weights need w_lm_scale");
+    REQ(m->H % 128 == 0 && m->I % 128 == 0, DLLM_ERR_UNSUPPORTED,
+        "denoise_step: FP8 weights need H and I multiples of 128");
     for (int l = 0; l < m->n_layers; ++l) {
       const dllm_layer& L = m->layers[l];
       REQ(L.w_gu_scale && L.w_down_scale && (!L.w_gu_shared || (L.w_gu_shared_scale && L.w_down_shared_scale)),
@@ -549,6 +551,7 @@ int dllm_moe_experts(const dllm_expert_desc* d, const void* h, const void* w_gu,
   REQ((d->H * esize(d->dtype)) % 16 == 0, DLLM_ERR_SHAPE, "moe_experts: H row bytes must be a multiple of 16");
   if (d->w_fp8) {
     REQ(d->dtype == DLLM_BF16, DLLM_ERR_UNSUPPORTED, "moe_experts: FP8 weights need bf16 storage");
+    REQ(d->H % 128 == 0 && d->I % 128 == 0, DLLM_ERR_UNSUPPORTED, "moe_experts: FP8 weights need H, I multiples of 128");
     REQ(w_gu_scale && w_down_scale && (!w_gu_shared || (w_gu_shared_scale && w_down_shared_scale)),
         DLLM_ERR_INVALID_ARG, "moe_experts: FP8 weights need their row scales");
   }

@@ -34,7 +34,8 @@ constexpr int STAGING_BYTES = 128 * STAGE_COLS * 4;
 constexpr int MAX_GROUPS = 1040;
 constexpr int NUM_THREADS = 192;
 constexpr int NUM_THREADS_F8 = 448;    // FP8 weights: two groups of four more warps convert alternate E4M3 tiles
-constexpr int RAW_BYTES = 128 * BK;    // 8 KB E4M3 weight tile per stage
+constexpr int F8_KS = 2;               // FP8 weights: 64-wide K blocks per stage (one 128-byte row of codes)
+constexpr int RAW_BYTES = 128 * BK * F8_KS;   // 16 KB E4M3 weight tile per stage
 constexpr int SMEM_LIMIT = 232448;
 
 struct Smem {
@@ -347,29 +348,33 @@ __device__ __forceinline__ void epilogue_logits_conf(const KParams& p, const flo
   }
 }
 
-// FP8 weights: row r of one stage's E4M3 tile as 32 columns of bf16 pairs in TMEM lane r, the A operand the MMA
-// reads from tensor memory. The TMA box lands row r at byte r * 64 of the stage with 64-byte swizzling (its four
-// 16-byte pieces XOR-permuted by (r >> 1) & 3), so the eight rows a quarter-warp reads hit eight different bank
-// groups. Every E4M3 value is exact in bf16 (3 mantissa bits, exponents 2^-9 .. 2^8), so the tile holds the codes'
-// values unscaled; the per-row scale is applied to the accumulator.
+// FP8 weights: row r of one stage's E4M3 tile (128 codes) as 64 columns of bf16 pairs in TMEM lane r, the A
+// operand the MMA reads from tensor memory. The TMA box lands row r at byte r * 128 of the stage with 128-byte
+// swizzling (its eight 16-byte pieces XOR-permuted by r & 7), so the eight rows a quarter-warp reads hit eight
+// different bank groups. Every E4M3 value is exact in bf16 (3 mantissa bits, exponents 2^-9 .. 2^8), so the tile
+// holds the codes' values unscaled; the per-row scale is applied to the accumulator.
 __device__ __forceinline__ void convert_e4m3_row_to_tmem(const uint8_t* raw, int row, uint32_t taddr) {
-  uint32_t o[32];
-  const int sw = (row >> 1) & 3;
+  const int sw = row & 7;
 #pragma unroll
-  for (int part = 0; part < 4; ++part) {
-    const uint4 q = *reinterpret_cast<const uint4*>(raw + row * 64 + ((part ^ sw) << 4));
-    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+  for (int half = 0; half < 2; ++half) {
+    uint32_t o[32];
 #pragma unroll
-    for (int h = 0; h < 8; ++h) {
-      const uint16_t pair = (uint16_t)(w[h >> 1] >> ((h & 1) * 16));
-      uint32_t f16x2;
-      asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(f16x2) : "h"(pair));
-      const float2 fv = __half22float2(*reinterpret_cast<const __half2*>(&f16x2));
-      const __nv_bfloat162 bv = __floats2bfloat162_rn(fv.x, fv.y);
-      o[part * 8 + h] = *reinterpret_cast<const uint32_t*>(&bv);
+    for (int pp = 0; pp < 4; ++pp) {
+      const int piece = half * 4 + pp;
+      const uint4 q = *reinterpret_cast<const uint4*>(raw + row * 128 + ((piece ^ sw) << 4));
+      const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+      for (int h = 0; h < 8; ++h) {
+        const uint16_t pair = (uint16_t)(w[h >> 1] >> ((h & 1) * 16));
+        uint32_t f16x2;
+        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(f16x2) : "h"(pair));
+        const float2 fv = __half22float2(*reinterpret_cast<const __half2*>(&f16x2));
+        const __nv_bfloat162 bv = __floats2bfloat162_rn(fv.x, fv.y);
+        o[pp * 8 + h] = *reinterpret_cast<const uint32_t*>(&bv);
+      }
     }
+    tc::tmem_st32(taddr + half * 32, o);
   }
-  tc::tmem_st32(taddr, o);
 }
 
 // Scale of tile row r of tile (g, mt) for FP8 weights: the row of W (or W2 for the extra group) it came from.
@@ -387,20 +392,26 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   constexpr int NT = F8 ? NUM_THREADS_F8 : NUM_THREADS;
-  constexpr int B_BYTES = BN * BK * 2;
+  // a stage covers KS 64-wide K blocks: one for bf16 weights (a 128-byte row of 64 elements), two for FP8 (a
+  // 128-byte row of 128 codes, so that each weight row read from HBM per stage is as long as in bf16)
+  constexpr int KS = F8 ? F8_KS : 1;
+  constexpr int SBK = BK * KS;                // K elements per stage
+  constexpr int B_HALF = BN * BK * 2;         // the activation tile of one 64-wide K block
+  constexpr int B_BYTES = B_HALF * KS;
   // bf16 weights: STAGES stages of [A weight tile][B activation tile]. FP8 weights: STAGES stages of [E4M3 weight
   // codes][B activation tile] (half the weight bytes, so a deeper ring), and MS A operand slots of 32 columns in
   // tensor memory that the converter warps fill from the codes.
   // The slots fill the tensor memory the two accumulators leave free: a slot is busy from its conversion through
   // the MMA's completion (a round trip of some 2000 cycles), so three slots held the FP8 kernel to half the HBM
   // rate at decode shapes.
-  constexpr int MS = F8 ? ((512 - 2 * BN) / 32 < 16 ? (512 - 2 * BN) / 32 : 16) : 0;
+  constexpr int SLOT_COLS = 32 * KS;           // TMEM columns of one A slot (bf16 pairs of a stage's K)
+  constexpr int MS = F8 ? ((512 - 2 * BN) / SLOT_COLS < 16 ? (512 - 2 * BN) / SLOT_COLS : 16) : 0;
   constexpr int MSD = MS > 0 ? MS : 1;        // slot count as a divisor (the bf16 instantiations use no slots)
   constexpr int W_BYTES = F8 ? RAW_BYTES : A_BYTES;
   constexpr int STAGE_BYTES = W_BYTES + B_BYTES;
   constexpr uint32_t W_TX = W_BYTES;                                      // weight bytes a stage's TMA brings
   constexpr uint32_t TMEM_COLS = F8 ? 512 : 2 * BN;
-  static_assert(!F8 || 2 * BN + MS * 32 <= 512, "FP8 A slots exceed the tensor memory");
+  static_assert(!F8 || 2 * BN + MS * SLOT_COLS <= 512, "FP8 A slots exceed the tensor memory");
   uint8_t* stages = base;
   float* staging = reinterpret_cast<float*>(base + STAGES * STAGE_BYTES);
   Smem& sm = *reinterpret_cast<Smem*>(reinterpret_cast<uint8_t*>(staging) + STAGING_BYTES);
@@ -432,7 +443,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
   // Weights are never written by the kernels ahead of this one: the first tile's first weight stages can stream
   // in before the dependency wait (their transaction bytes are expected now; the arrival, with the activation
   // bytes, comes in the producer loop). Every lane of warp 0 derives the same count.
-  const int kblocks = p.K / BK;
+  const int kblocks = p.K / SBK;
   int npf = 0;
   if (p.prefetch_w) {
     const int t0 = p.ksplit > 1 ? (int)blockIdx.y : (int)blockIdx.x;
@@ -444,7 +455,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
       const uint64_t pol_w = tc::policy_evict_first();
       for (int i = 0; i < npf; ++i) {
         tc::mbar_expect_tx(&sm.full[i], W_TX);
-        tc::tma_load_2d(stages + i * STAGE_BYTES, &tmap_w, (kb0 + i) * BK, t0 * 128, &sm.full[i], pol_w);
+        tc::tma_load_2d(stages + i * STAGE_BYTES, &tmap_w, (kb0 + i) * SBK, t0 * 128, &sm.full[i], pol_w);
       }
     }
   }
@@ -525,7 +536,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
         const CUtensorMap* wm = extra ? &tmap_w2 : &tmap_w;
         const int64_t wrow = extra ? 0 : (int64_t)g * p.w_group_stride;
         const int nb = (nval + XBOX_ROWS - 1) / XBOX_ROWS;
-        const uint32_t bytes = W_TX + nb * XBOX_BYTES;
+        const uint32_t bytes = W_TX + KS * nb * XBOX_BYTES;
         const int xrow = sm.grp_off[g] + n0;
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % STAGES;
@@ -538,14 +549,17 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
           } else {
             tc::mbar_arrive_expect_tx(&sm.full[s], bytes);
             if (p.swiglu) {
-              tc::tma_load_2d(a, wm, kb * BK, (int)(wrow + mt * 64), &sm.full[s], pol_w);
-              tc::tma_load_2d(a + W_TX / 2, wm, kb * BK, (int)(wrow + p.M + mt * 64), &sm.full[s], pol_w);
+              tc::tma_load_2d(a, wm, kb * SBK, (int)(wrow + mt * 64), &sm.full[s], pol_w);
+              tc::tma_load_2d(a + W_TX / 2, wm, kb * SBK, (int)(wrow + p.M + mt * 64), &sm.full[s], pol_w);
             } else {
-              tc::tma_load_2d(a, wm, kb * BK, (int)(wrow + mt * 128), &sm.full[s], pol_w);
+              tc::tma_load_2d(a, wm, kb * SBK, (int)(wrow + mt * 128), &sm.full[s], pol_w);
             }
           }
-          for (int j = 0; j < nb; ++j)
-            tc::tma_load_2d(b + j * XBOX_BYTES, &tmap_x, kb * BK, xrow + j * XBOX_ROWS, &sm.full[s], pol_x);
+#pragma unroll
+          for (int hk = 0; hk < KS; ++hk)
+            for (int j = 0; j < nb; ++j)
+              tc::tma_load_2d(b + hk * B_HALF + j * XBOX_BYTES, &tmap_x, kb * SBK + hk * BK, xrow + j * XBOX_ROWS,
+                              &sm.full[s], pol_x);
         }
       }
       if (!ok) {
@@ -587,10 +601,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
             const int ms = it % MSD;
             if (!wait_bar(&sm.conv[ms], (it / MSD) & 1, abort_flag, p.status, ST_TIMEOUT_MMA)) { ok = false; break; }
             tc::fence_after_sync();
-            const uint32_t ta = sm.tmem_base + 2 * BN + ms * 32;
+            const uint32_t ta = sm.tmem_base + 2 * BN + ms * SLOT_COLS;
 #pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk)
-              tc::mma_bf16_tmem_a(d, ta + kk * 8, tc::sdesc_k128(b + kk * 32), idesc, (kb != kb0) || kk != 0);
+            for (int kk = 0; kk < SBK / 16; ++kk)
+              tc::mma_bf16_tmem_a(d, ta + kk * 8, tc::sdesc_k128(b + (kk >> 2) * B_HALF + (kk & 3) * 32), idesc,
+                                  (kb != kb0) || kk != 0);
             tc::mma_commit(&sm.mempty[ms]);
           } else {
             tc::fence_after_sync();
@@ -627,7 +642,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
             !wait_bar(&sm.full[s], (it / STAGES) & 1, abort_flag, p.status, ST_TIMEOUT_MMA)) { ok = false; break; }
         tc::fence_after_sync();
         convert_e4m3_row_to_tmem(stages + s * STAGE_BYTES, row,
-                                 sm.tmem_base + ((uint32_t)((warp & 3) * 32) << 16) + 2 * BN + ms * 32);
+                                 sm.tmem_base + ((uint32_t)((warp & 3) * 32) << 16) + 2 * BN + ms * SLOT_COLS);
         tc::tmem_st_wait();
         tc::fence_before_sync();
         tc::mbar_arrive(&sm.conv[ms]);
@@ -1009,8 +1024,8 @@ EncodeTiledFn get_encode() {
   return fn;
 }
 
-// bf16 [rows, K] with 128-byte swizzled boxes of 64 x box_rows, or (u8) E4M3 codes [rows, K] with 64-byte swizzled
-// boxes of 64 bytes x box_rows (the converter warps read them row by row)
+// bf16 [rows, K] with 128-byte swizzled boxes of 64 x box_rows, or (u8) E4M3 codes [rows, K] with 128-byte swizzled
+// boxes of 128 codes x box_rows (the converter warps read them row by row)
 int make_map(CUtensorMap* m, const void* ptr, int64_t rows, int K, int box_rows, bool u8 = false) {
   EncodeTiledFn enc = get_encode();
   if (!enc) {
@@ -1019,11 +1034,11 @@ int make_map(CUtensorMap* m, const void* ptr, int64_t rows, int K, int box_rows,
   }
   cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)K * (u8 ? 1 : 2)};
-  cuuint32_t box[2] = {(cuuint32_t)BK, (cuuint32_t)box_rows};
+  cuuint32_t box[2] = {(cuuint32_t)(u8 ? BK * F8_KS : BK), (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(m, u8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr),
                    dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   u8 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     dllm_host::set_error("cuTensorMapEncodeTiled failed (%d) rows=%lld K=%d box_rows=%d", (int)r, (long long)rows,
@@ -1041,7 +1056,7 @@ template <int BN, int STAGES, bool F8 = false>
 int launch(const GemmArgs& a, const CUtensorMap& mw, const CUtensorMap& mw2, const CUtensorMap& mx,
            const KParams& kp, cudaStream_t s) {
   // (matches the kernel's layout: stages of [weights (bf16 or E4M3)][activations])
-  constexpr int STAGE_BYTES = (F8 ? RAW_BYTES : A_BYTES) + BN * BK * 2;
+  constexpr int STAGE_BYTES = F8 ? RAW_BYTES + BN * BK * 2 * F8_KS : A_BYTES + BN * BK * 2;
   constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + STAGING_BYTES + (int)sizeof(Smem);
   static_assert(SMEM <= SMEM_LIMIT, "shared memory budget");
   // With programmatic dependent launch a CTA allocates tensor memory before it waits for the kernels ahead of it.
@@ -1197,6 +1212,8 @@ int gemm_bf16_tc(const GemmArgs& a, cudaStream_t s) {
     DLLM_REQUIRE(a.w_scale && (!a.w2 || a.w2_scale), DLLM_ERR_INVALID_ARG, "gemm: FP8 weights need their row scales");
     DLLM_REQUIRE(a.epi.kind == EPI_STORE || a.epi.kind == EPI_SWIGLU, DLLM_ERR_UNSUPPORTED,
                  "gemm: FP8 weights take the store or SwiGLU epilogue");
+    DLLM_REQUIRE(a.K % (BK * F8_KS) == 0, DLLM_ERR_UNSUPPORTED, "gemm: FP8 weights need K=%d a multiple of %d",
+                 a.K, BK * F8_KS);
   }
   CUtensorMap mw, mw2, mx;
   int st = make_map(&mw, a.w, a.w_rows, a.K, box_rows, f8);
@@ -1235,9 +1252,9 @@ int gemm_bf16_tc(const GemmArgs& a, cudaStream_t s) {
   kp.prefetch_w = (!a.swiglu && !a.n_dev && !a.has_extra && a.host_cnt <= (ks > 1 ? 32 : bn)) ? 1 : 0;
   int st2;
   if (f8) {   // single-CTA tiles, no split-K (the weight-streaming shapes FP8 weights serve)
-    if (bn == 32) st2 = launch<32, 16, true>(a, mw, mw2, mx, kp, s);
-    else if (bn == 64) st2 = launch<64, 12, true>(a, mw, mw2, mx, kp, s);
-    else st2 = launch<128, 8, true>(a, mw, mw2, mx, kp, s);
+    if (bn == 32) st2 = launch<32, 8, true>(a, mw, mw2, mx, kp, s);
+    else if (bn == 64) st2 = launch<64, 6, true>(a, mw, mw2, mx, kp, s);
+    else st2 = launch<128, 4, true>(a, mw, mw2, mx, kp, s);
   } else if (gemm_uses_pairs(a)) {
     kp.prefetch_w = 0;
     st2 = launch_pair(mw, mw2, mx, kp, s);

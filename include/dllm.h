@@ -87,7 +87,8 @@ DLLM_API int dllm_selftest_bounded_wait(void* ws, size_t ws_bytes, cudaStream_t 
  * no format): a matrix W [M, K] is stored as M x K E4M3 codes (OCP 8-bit float without infinities, one byte each,
  * row-major) plus one fp32 scale per row, W[m, k] = value(code[m, k]) * scale[m]. Products with FP8 weights are
  * scale[m] * sum_k x[k] value(code[m, k]) accumulated in fp32 (the codes' values are exact in bf16). Only the large
- * matrices take this form: the routed and shared experts and the LM head.
+ * matrices take this form: the routed and shared experts and the LM head. Their K (H, and I for the down
+ * projection) must be a multiple of 128 (one 128-byte row of codes per pipeline stage).
  */
 #define DLLM_WEIGHTS_BF16 0 /* weights in the storage type */
 #define DLLM_WEIGHTS_FP8 1  /* experts and LM head as E4M3 codes with per-row fp32 scales */

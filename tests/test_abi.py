@@ -101,6 +101,9 @@ def test_route_and_experts_reject_bad_arguments(lib):
     e.I, e.w_fp8 = 512, 1                # FP8 expert weights without their row scales
     assert lib.dllm_moe_experts(C.byref(e), *([FAKE] * 5), *no_scales, *([FAKE] * 6), FAKE, 1 << 30,
                                 None) == bd.ERR_INVALID_ARG
+    e.I = 192                            # FP8: K of the down projection not a multiple of 128
+    assert lib.dllm_moe_experts(C.byref(e), *([FAKE] * 5), *([FAKE] * 4), *([FAKE] * 6), FAKE, 1 << 30,
+                                None) == bd.ERR_UNSUPPORTED
 
 
 def test_grouped_gemm_rejects_bad_arguments(lib):

@@ -181,6 +181,7 @@ struct StepPlan {
   void* logits;
   void* partials;
   int conf_parts;   // > 0: the LM head writes this many confidence partials per row (fused epilogue)
+  float2* rope_tab;  // [L][64] RoPE (cos, sin) of the block's positions (tensor-core QKV epilogue)
   void* unmask_extras;   // the other position scores' statistics (null for the largest probability)
   float* retain_raw;
   size_t total;
@@ -301,6 +302,7 @@ void plan_step(const dllm_model* m, const dllm_state* st, const dllm_step_params
                        ? c.take<float>((size_t)std::max(s.Tk, s.halves * s.max_rows) *
                                        std::max(std::max(proj_n, H), s.vlen) * 4)
                        : nullptr;
+  s.rope_tab = m->dtype == DLLM_BF16 ? c.take<float2>((size_t)st->L * 64 * sizeof(float2)) : nullptr;
   s.row_pos = c.take<int32_t>((size_t)s.max_rows * 4);
   s.n_rows = c.take<int32_t>(16);
   s.xf = c.take((size_t)s.halves * s.max_rows * H * es);
@@ -667,14 +669,18 @@ int denoise_step_impl(const dllm_model* m, const dllm_state* st, const dllm_step
   // launches. A commit pass always runs.
   const int32_t* live = p->commit ? nullptr : s.n_rows + 2;
   const bool fuse = fused_rows_ok(dt, H);
+  RopeTable rope;   // the block's RoPE angles, for the tensor-core QKV epilogue
+  rope.tab = s.rope_tab; rope.pos0 = P; rope.L = L; rope.base = m->rope_base;
   if (fuse) {
-    // embedding, layer 0's attention-input norm and (denoising passes) the masked-row list in one launch
+    // embedding, layer 0's attention-input norm, (denoising passes) the masked-row list and the RoPE table in one
+    // launch
     TRY(launch_embed_norm(dt, st->tokens, p->commit ? nullptr : st->mask, m->mask_id, m->embed, s.x, s.h,
                           m->layers[0].attn_norm, s.Tk, H, m->eps, st->mask, s.Bl * L, s.halves,
-                          p->commit ? nullptr : s.row_pos, s.n_rows, stream));
+                          p->commit ? nullptr : s.row_pos, s.n_rows, stream, rope));
   } else {
     if (!p->commit) TRY(launch_masked_rows(st->mask, s.Bl * L, s.halves, s.row_pos, s.n_rows, stream));
     TRY(launch_embed(dt, st->tokens, p->commit ? nullptr : st->mask, m->mask_id, m->embed, s.x, s.Tk, H, stream));
+    TRY(launch_rope_table(rope, stream));
   }
   for (int l = 0; l < m->n_layers; ++l) {
     const dllm_layer& Ly = m->layers[l];
@@ -696,7 +702,7 @@ int denoise_step_impl(const dllm_model* m, const dllm_state* st, const dllm_step
     g.M = (m->Hq + 2 * m->Hkv) * m->d; g.host_cnt = s.Tk; g.max_cnt = s.Tk; g.cnt_bound = s.Tk; g.dtype = dt;
     g.status = status; g.f32_scratch = s.proj_scratch; g.live = live;
     g.epi.kind = EPI_QKV; g.epi.q_out = s.q; g.epi.Hq = m->Hq; g.epi.Hkv = m->Hkv; g.epi.d = m->d; g.epi.L = L;
-    g.epi.pos0 = P; g.epi.rope_base = m->rope_base;
+    g.epi.pos0 = P; g.epi.rope_base = m->rope_base; g.epi.rope_tab = s.rope_tab;
     if (p->sprint) {
       g.epi.k_dst = Ly.k_thin; g.epi.v_dst = Ly.v_thin; g.epi.cap = st->cap_thin; g.epi.slot0 = p->n_keep;
       if (p->commit) { g.epi.k_dst2 = Ly.k_cache; g.epi.v_dst2 = Ly.v_cache; g.epi.cap2 = st->cap; g.epi.slot2 = P; }

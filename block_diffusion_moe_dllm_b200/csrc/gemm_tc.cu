@@ -147,16 +147,6 @@ __device__ __forceinline__ float4 ld_dsmem4(const float* local, uint32_t rank) {
   return v;
 }
 
-// cos and sin of pos * inv_freq: the angle is formed and reduced to [-pi, pi] in fp64, then evaluated in fp32
-// (absolute error ~1e-7 for any position).
-__device__ __forceinline__ void rope_cos_sin(int pos, double inv_freq, float* c, float* s) {
-  const double two_pi = 6.283185307179586476925286766559;
-  const double inv_two_pi = 0.15915494309189533576888376337251;
-  double a = (double)pos * inv_freq;
-  a -= two_pi * rint(a * inv_two_pi);
-  sincosf((float)a, s, c);
-}
-
 // Eight consecutive staging values of token column j from feature m0 (two 16-byte shared-memory loads).
 __device__ __forceinline__ void stage8(const float* stage, int j, int m0, float* v) {
   const float4 a = *reinterpret_cast<const float4*>(stage + j * 128 + m0);
@@ -206,17 +196,19 @@ __device__ void epilogue_chunk(const KParams& p, const float* stage, int g, int 
       const float4 a2 = *reinterpret_cast<const float4*>(stage + j * 128 + 64 + m0);
       const float x1[4] = {a1.x, a1.y, a1.z, a1.w}, x2[4] = {a2.x, a2.y, a2.z, a2.w};
       float y1[4], y2[4];
-      const int pos = e.pos0 + tr % e.L;
+      if (rot) {
+        // (cos, sin) of pairs m0 .. m0 + 3 at the token's position: two 16-byte loads of the block's table
+        const float4* cs = reinterpret_cast<const float4*>(e.rope_tab + (tr % e.L) * 64 + m0);
+        const float4 c01 = cs[0], c23 = cs[1];
+        const float c[4] = {c01.x, c01.z, c23.x, c23.z}, sn[4] = {c01.y, c01.w, c23.y, c23.w};
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        y1[u] = x1[u];
-        y2[u] = x2[u];
-        if (rot) {
-          float c, sn;
-          rope_cos_sin(pos, e.inv_freq[m0 + u], &c, &sn);
-          y1[u] = x1[u] * c - x2[u] * sn;
-          y2[u] = x2[u] * c + x1[u] * sn;
+        for (int u = 0; u < 4; ++u) {
+          y1[u] = x1[u] * c[u] - x2[u] * sn[u];
+          y2[u] = x2[u] * c[u] + x1[u] * sn[u];
         }
+      } else {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) { y1[u] = x1[u]; y2[u] = x2[u]; }
       }
       __nv_bfloat162 t0 = __floats2bfloat162_rn(y1[0], y1[1]), t1 = __floats2bfloat162_rn(y1[2], y1[3]);
       __nv_bfloat162 t2 = __floats2bfloat162_rn(y2[0], y2[1]), t3 = __floats2bfloat162_rn(y2[2], y2[3]);
@@ -1205,7 +1197,8 @@ int gemm_bf16_tc(const GemmArgs& a, cudaStream_t s) {
   DLLM_REQUIRE(((uintptr_t)a.x % 16 == 0) && ((uintptr_t)a.w % 16 == 0) && (!a.w2 || (uintptr_t)a.w2 % 16 == 0),
                DLLM_ERR_ALIGN, "gemm: operands must be 16-byte aligned");
   if (a.epi.kind == EPI_QKV)
-    DLLM_REQUIRE(a.epi.d == 128, DLLM_ERR_UNSUPPORTED, "gemm: QKV epilogue needs head dim 128");
+    DLLM_REQUIRE(a.epi.d == 128 && a.epi.rope_tab != nullptr && ((uintptr_t)a.epi.rope_tab % 16) == 0,
+                 DLLM_ERR_UNSUPPORTED, "gemm: QKV epilogue needs head dim 128 and the block's RoPE table");
   const int box_rows = a.swiglu ? 64 : 128;
   const bool f8 = a.w_fp8 != 0;
   if (f8) {
@@ -1240,8 +1233,6 @@ int gemm_bf16_tc(const GemmArgs& a, cudaStream_t s) {
   kp.w_scale = a.w_scale;
   kp.w2_scale = a.w2_scale;
   kp.epi = a.epi;
-  if (kp.epi.kind == EPI_QKV)
-    for (int m = 0; m < 64; ++m) kp.epi.inv_freq[m] = std::pow((double)kp.epi.rope_base, -2.0 * (double)m / 128.0);
   kp.status = a.status;
   const int bn = gemm_bn(a);
   const int ks = gemm_splitk_factor(a, bn);

@@ -44,8 +44,8 @@ struct EpiParams {
   void* v_dst2 = nullptr;
   int cap = 0, slot0 = 0, cap2 = 0, slot2 = 0;
   int Hq = 0, Hkv = 0, d = 0, L = 1, pos0 = 0;
-  float rope_base = 10000.f;
-  double inv_freq[64] = {};         // rope_base^(-2 m / 128), m < 64 (filled on the host by gemm_bf16_tc)
+  float rope_base = 10000.f;         // fp32 path (the SIMT epilogue evaluates the angles itself)
+  const float2* rope_tab = nullptr;  // [L][64] (cos, sin) of the block's positions (RopeTable), tensor-core path
   // EPI_STORE of bf16 logits: also the confidence partial of every token row over the vocabulary rows this CTA
   // produced, at conf_part[row * conf_nparts + CTA index] (only with gemm_conf_parts(...) == conf_nparts)
   ConfPartial* conf_part = nullptr;

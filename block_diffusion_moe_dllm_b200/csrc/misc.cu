@@ -278,14 +278,35 @@ DLLM_DEV void store_norm_row(const uint4* keep, int nvec, float inv, const T* __
 // CTA t < rows: x[t] = embed[mask[t] ? mask_id : tokens[t]] and h[t] = norm(x[t]) * g. With the masked-row list
 // requested, one extra CTA writes it (the ascending still-masked positions of the first n_pos, their count and
 // count * halves), as masked_rows_kernel does.
+// Entry idx of a block's RoPE table (see RopeTable): the angle and its cosine and sine in fp64, rounded once.
+DLLM_DEV void rope_entry(const RopeTable& r, int idx) {
+  if (!r.tab || idx >= r.L * 64) return;
+  const int i = idx >> 6, m = idx & 63;
+  const double a = (double)(r.pos0 + i) * pow((double)r.base, -2.0 * (double)m / 128.0);
+  double sn, cs;
+  sincos(a, &sn, &cs);
+  r.tab[idx] = make_float2((float)cs, (float)sn);
+}
+
+__global__ void __launch_bounds__(256) rope_table_kernel(RopeTable r) {
+  pdl_enter();
+  rope_entry(r, (int)blockIdx.x * 256 + (int)threadIdx.x);
+}
+
 template <typename T>
 __global__ void __launch_bounds__(256) embed_norm_kernel(const int32_t* __restrict__ tokens,
                                                          const uint8_t* __restrict__ mask, int mask_id,
                                                          const T* __restrict__ table, T* __restrict__ x,
                                                          T* __restrict__ h, const T* __restrict__ g, int rows, int H,
                                                          float eps, const uint8_t* __restrict__ list_mask, int n_pos,
-                                                         int halves, int32_t* row_pos, int32_t* n_out) {
+                                                         int halves, int32_t* row_pos, int32_t* n_out,
+                                                         RopeTable rope) {
   pdl_enter();
+  const int first_rope = rows + (row_pos ? 1 : 0);
+  if ((int)blockIdx.x >= first_rope) {   // the block's RoPE table
+    rope_entry(rope, ((int)blockIdx.x - first_rope) * 256 + (int)threadIdx.x);
+    return;
+  }
   __shared__ float red[8];
   if ((int)blockIdx.x == rows) {
     __shared__ int warp_tot[8];
@@ -342,18 +363,25 @@ __global__ void __launch_bounds__(256) embed_norm_kernel(const int32_t* __restri
   store_norm_row<T>(keep, nvec, 1.0f / sqrtf(ss / (float)H + eps), g, h + (int64_t)t * H);
 }
 
+int launch_rope_table(const RopeTable& r, cudaStream_t s) {
+  if (!r.tab || r.L <= 0) return DLLM_OK;
+  launch_pdl(rope_table_kernel, (r.L * 64 + 255) / 256, 256, 0, s, r);
+  DLLM_CHECK_LAUNCH("rope_table_kernel");
+  return DLLM_OK;
+}
+
 int launch_embed_norm(int dtype, const int32_t* tokens, const uint8_t* mask, int mask_id, const void* table, void* x,
                       void* h, const void* g, int rows, int H, float eps, const uint8_t* list_mask, int n_pos,
-                      int halves, int32_t* row_pos, int32_t* n_out, cudaStream_t s) {
-  if (rows <= 0) return DLLM_OK;
-  const int ctas = rows + (row_pos ? 1 : 0);
+                      int halves, int32_t* row_pos, int32_t* n_out, cudaStream_t s, const RopeTable& rope) {
+  if (rows <= 0) return launch_rope_table(rope, s);
+  const int ctas = rows + (row_pos ? 1 : 0) + (rope.tab ? (rope.L * 64 + 255) / 256 : 0);
   if (dtype == DLLM_BF16)
     launch_pdl(embed_norm_kernel<__nv_bfloat16>, ctas, 256, 0, s, tokens, mask, mask_id,
                (const __nv_bfloat16*)table, (__nv_bfloat16*)x, (__nv_bfloat16*)h, (const __nv_bfloat16*)g, rows, H,
-               eps, list_mask, n_pos, halves, row_pos, n_out);
+               eps, list_mask, n_pos, halves, row_pos, n_out, rope);
   else
     launch_pdl(embed_norm_kernel<float>, ctas, 256, 0, s, tokens, mask, mask_id, (const float*)table, (float*)x,
-               (float*)h, (const float*)g, rows, H, eps, list_mask, n_pos, halves, row_pos, n_out);
+               (float*)h, (const float*)g, rows, H, eps, list_mask, n_pos, halves, row_pos, n_out, rope);
   DLLM_CHECK_LAUNCH("embed_norm_kernel");
   return DLLM_OK;
 }

@@ -21,9 +21,19 @@ int launch_combine(int dtype, void* x, const float* y, const float* gates, const
 // Fused row stages (bf16 rows of up to 8192 elements, fp32 up to 4096: kRowVecs 16-byte vectors per thread).
 constexpr int kRowVecs = 4;
 enum NormMode { NORM_NEXT = 0, NORM_FINAL = 1 };
+// RoPE table of a block (head dim 128): tab[i * 64 + m] = (cos, sin) of (pos0 + i) * base^(-2 m / 128) for i < L,
+// m < 64, evaluated in fp64 and rounded once to fp32 (tab == nullptr: no table).
+struct RopeTable {
+  float2* tab = nullptr;
+  int pos0 = 0, L = 0;
+  float base = 10000.f;
+};
+int launch_rope_table(const RopeTable& r, cudaStream_t s);
+// the embedding kernel also fills the RoPE table (extra CTAs) when rope.tab is set
 int launch_embed_norm(int dtype, const int32_t* tokens, const uint8_t* mask, int mask_id, const void* table, void* x,
                       void* h, const void* g, int rows, int H, float eps, const uint8_t* list_mask, int n_pos,
-                      int halves, int32_t* row_pos, int32_t* n_out, cudaStream_t s);
+                      int halves, int32_t* row_pos, int32_t* n_out, cudaStream_t s,
+                      const RopeTable& rope = RopeTable());
 int launch_combine_norm(int dtype, void* x, const float* y, const float* gates, const int32_t* inv, int k, int Tk,
                         int shared, int H, const void* g, float eps, void* out, int mode, const uint8_t* mask,
                         int n_half_pos, const int32_t* n_dev, cudaStream_t s, const int32_t* live = nullptr);

@@ -340,11 +340,27 @@ __device__ __forceinline__ void epilogue_logits_conf(const KParams& p, const flo
   }
 }
 
+// Two E4M3 codes (bytes 0 and 1, or 2 and 3, of w, as selected by prmt_sel) as a bf16 pair, exactly. The code
+// s.eeee.mmm placed as the bf16 bit pattern s.0000eeee.mmm0000 is value(code) * 2^-120 for every code, the
+// subnormal ones included (both formats scale their subnormals by their fixed minimum exponent), so the pair is
+// formed with integer operations (a byte permute that also replicates each code's sign bit, a shift and a mask)
+// and multiplied by 2^120, exact in bf16 arithmetic (which keeps subnormal inputs). No conversion instruction is
+// needed, so the pairs come from the integer and fused multiply-add pipes. NaN codes are not expected in weights.
+template <uint32_t PRMT_SEL>
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t w) {
+  uint32_t q;
+  asm("prmt.b32 %0, %1, 0, %2;" : "=r"(q) : "r"(w), "n"(PRMT_SEL));
+  const uint32_t bits = (q << 4) & 0x87f087f0u;
+  uint32_t r;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(bits), "r"(0x7b807b80u));   // x 2^120
+  return r;
+}
+
 // FP8 weights: row r of one stage's E4M3 tile (128 codes) as 64 columns of bf16 pairs in TMEM lane r, the A
 // operand the MMA reads from tensor memory. The TMA box lands row r at byte r * 128 of the stage with 128-byte
 // swizzling (its eight 16-byte pieces XOR-permuted by r & 7), so the eight rows a quarter-warp reads hit eight
-// different bank groups. Every E4M3 value is exact in bf16 (3 mantissa bits, exponents 2^-9 .. 2^8), so the tile
-// holds the codes' values unscaled; the per-row scale is applied to the accumulator.
+// different bank groups. The tile holds the codes' values unscaled; the per-row scale is applied to the
+// accumulator.
 __device__ __forceinline__ void convert_e4m3_row_to_tmem(const uint8_t* raw, int row, uint32_t taddr) {
   const int sw = row & 7;
 #pragma unroll
@@ -356,13 +372,10 @@ __device__ __forceinline__ void convert_e4m3_row_to_tmem(const uint8_t* raw, int
       const uint4 q = *reinterpret_cast<const uint4*>(raw + row * 128 + ((piece ^ sw) << 4));
       const uint32_t w[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-      for (int h = 0; h < 8; ++h) {
-        const uint16_t pair = (uint16_t)(w[h >> 1] >> ((h & 1) * 16));
-        uint32_t f16x2;
-        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(f16x2) : "h"(pair));
-        const float2 fv = __half22float2(*reinterpret_cast<const __half2*>(&f16x2));
-        const __nv_bfloat162 bv = __floats2bfloat162_rn(fv.x, fv.y);
-        o[pp * 8 + h] = *reinterpret_cast<const uint32_t*>(&bv);
+      for (int i = 0; i < 4; ++i) {
+        // selectors: bytes (c0, sign(c0), c1, sign(c1)) and (c2, sign(c2), c3, sign(c3))
+        o[pp * 8 + 2 * i] = e4m3x2_to_bf16x2<0x9180u>(w[i]);
+        o[pp * 8 + 2 * i + 1] = e4m3x2_to_bf16x2<0xB3A2u>(w[i]);
       }
     }
     tc::tmem_st32(taddr + half * 32, o);

@@ -294,6 +294,25 @@ def test_gemm_fp8_lm_head_shape(N):
     assert_close(to64(y)[:, cols], want, "bf16", "FP8 LM-head logits")
 
 
+def test_gemm_fp8_every_code_exact():
+    """Every E4M3 code, the subnormal ones included, reaches the tensor cores with its exact value: weight rows
+    hold all 254 non-NaN codes in rotated order (scale 1), the token rows are one-hot, so every output is a single
+    code's value (exact in bf16) and must equal the oracle's E4M3 definition bit for bit."""
+    M, K, N = 256, 128, 128
+    m, k = np.meshgrid(np.arange(M), np.arange(K), indexing="ij")
+    codes = ((m + 3 * k) % 256).astype(np.uint8)
+    codes[(codes & 0x7F) == 0x7F] = 0                       # the two NaN codes -> +0
+    wq = torch.from_numpy(codes).to(DEV)
+    sc = torch.ones(M, dtype=torch.float32, device=DEV)
+    x = torch.zeros((N, K), dtype=torch.bfloat16, device=DEV)
+    x[torch.arange(N), torch.arange(N) % K] = 1.0
+    y = torch.empty((N, M), dtype=torch.bfloat16, device=DEV)
+    bd.gemm(x, wq, y, N, M, K, bd.BF16, w_scale=sc)
+    torch.cuda.synchronize()
+    want = O.e4m3_value(codes).T[np.arange(N) % K]          # y[n, m] = value(code[m, n])
+    assert np.array_equal(to64(y), want)
+
+
 # ------------------------------------------------------------------------------------------------ attention
 def _attn_case(dtype, B, Lq, Hq, Hkv, d, blk, q_pos0, n_keys, cap, key_pos=None, seed=0, nan_tail=False):
     t = _tdt(dtype)

@@ -306,64 +306,108 @@ DLLM_DEV void acc16(const uint4& hv, const uint4& wv, double& s, const float*) {
   s = fma((double)__uint_as_float(hv.w), (double)__uint_as_float(wv.w), s);
 }
 
+// One lane-strided pass of a weight row against the token row chunks hv (CH 16-byte chunks per lane, block b0):
+// loads of the row's chunks into wv.
+template <int CH, typename T>
+DLLM_DEV void load_row_chunks(const T* __restrict__ row, int H, int b0, int lane, uint4 (&wv)[CH]) {
+  constexpr int VE = 16 / sizeof(T);
+#pragma unroll
+  for (int j = 0; j < CH; ++j) {
+    const int c = b0 + (j * 32 + lane) * VE;
+    wv[j] = c < H ? *reinterpret_cast<const uint4*>(row + c) : make_uint4(0, 0, 0, 0);
+  }
+}
+
+// A token's selection decided exactly when there are more than 32 candidates (only with many equal scores):
+// kept out of line, it is never on a hot path.
+template <typename T>
+__device__ __noinline__ void exact_select_many(const float* __restrict__ srow, const float* __restrict__ bias, int E,
+                                               int k, const T* __restrict__ hrow, const T* __restrict__ w, int H,
+                                               float thr, int lane, int* my_id, float* my_gate) {
+  double gsum = 0.0, mine = 0.0;
+  double last = INFINITY;
+  int last_e = -1;
+  *my_id = 0;
+  for (int j = 0; j < k; ++j) {
+    // the best candidate below (last, last_e) in (score desc, expert asc) order, rescoring every candidate
+    double bv = -INFINITY;
+    int be = 0x7fffffff;
+    for (int e0 = 0; e0 < E; e0 += 32) {
+      const int ex = e0 + lane;
+      unsigned bal = __ballot_sync(0xffffffffu, ex < E && srow[ex] + bias[ex] >= thr);
+      while (bal) {
+        const int src = __ffs(bal) - 1;
+        bal &= bal - 1;
+        const int eb = e0 + src;
+        const double v = 1.0 / (1.0 + exp(-warp_dot64<2>(hrow, w + (int64_t)eb * H, H, lane))) + (double)bias[eb];
+        const bool below = v < last || (v == last && eb > last_e);
+        if (below && (v > bv || (v == bv && eb < be))) { bv = v; be = eb; }
+      }
+    }
+    last = bv;
+    last_e = be;
+    const double sc = bv - (double)bias[be];
+    gsum += sc;
+    if (lane == j) { *my_id = be; mine = sc; }
+  }
+  *my_gate = (float)(mine / gsum);
+}
+
 // Exact selection of one near-tie token by its own warp. The candidate experts (fp32 biased score at least thr,
-// the (k+1)-th value minus the guard) are compacted into lanes; their exact scores come four candidates at a time,
-// each lane holding its 16-byte chunks of the four weight rows and of the token row at once (eight chunks per lane
-// in flight), so a candidate group costs about one trip to L2 per 2048 bf16 elements instead of one per candidate;
-// then k rounds of a warp arg-max give the slots in order (ties -> lower expert) and the gates (unbiased fp64
-// scores renormalised). More than 32 candidates (only with many equal scores): exact_redecide.
-template <int PER, typename T>
-DLLM_DEV void warp_exact_select(float* __restrict__ srow, const float* __restrict__ bias, int E, int k,
+// the (k+1)-th value minus the guard) are compacted into lanes; each candidate's exact score is a warp-wide dot
+// product with the token row held in registers, the next candidate's weight row loading while the current one is
+// summed (bf16 products are exact in fp32 and are added in fp64); then k rounds of a warp arg-max give the slots
+// in order (ties -> lower expert) and the gates (unbiased fp64 scores renormalised). Returns false (the fp32
+// decision stands) only when fewer than k experts pass the threshold, which takes non-finite scores.
+template <typename T>
+DLLM_DEV bool warp_exact_select(const float* __restrict__ srow, const float* __restrict__ bias, int E, int k,
                                 const T* __restrict__ hrow, const T* __restrict__ w, int H, float thr, int lane,
                                 int& my_id, float& my_gate) {
-  __syncwarp();   // the warp's own write-back of the sigmoid scores is visible to every lane
   constexpr int VE = 16 / sizeof(T);   // elements per 16-byte chunk
-  constexpr int CH = 8;                // chunks per lane per pass over the row
+  constexpr int CH = 8;                // chunks per lane per block of the row
+  constexpr int BLK = 32 * VE * CH;    // row elements per block
   int n = 0, ce = 0x7fffffff;
-#pragma unroll
-  for (int i = 0; i < PER; ++i) {
-    const int ex = i * 32 + lane;
+  for (int e0 = 0; e0 < E; e0 += 32) {
+    const int ex = e0 + lane;
     unsigned bal = __ballot_sync(0xffffffffu, ex < E && srow[ex] + bias[ex] >= thr);
     while (bal) {
       const int src = __ffs(bal) - 1;
       bal &= bal - 1;
-      if (lane == n) ce = i * 32 + src;
+      if (lane == n) ce = e0 + src;
       ++n;
     }
   }
+  if (n < k) return false;
   if (n > 32) {
-    exact_redecide<PER>(srow, bias, E, k, hrow, w, H, thr, lane, my_id, my_gate);
-    return;
+    exact_select_many<T>(srow, bias, E, k, hrow, w, H, thr, lane, &my_id, &my_gate);
+    return true;
   }
-  double cv = -INFINITY;   // lane j < n: exact biased score of candidate j
-  for (int c0 = 0; c0 < n; c0 += 4) {
-    int eq[4];
+  double dot = 0.0;   // lane j < n: candidate j's dot product
+  for (int b0 = 0; b0 < H; b0 += BLK) {
+    uint4 hv[CH], wa[CH], wb[CH];
+    load_row_chunks<CH>(hrow, H, b0, lane, hv);
+    load_row_chunks<CH>(w + (int64_t)__shfl_sync(0xffffffffu, ce, 0) * H, H, b0, lane, wa);
+#pragma unroll 1
+    for (int c = 0; c < n; c += 2) {
+      const bool two = c + 1 < n;
+      const int e1 = __shfl_sync(0xffffffffu, ce, two ? c + 1 : c);
+      if (two) load_row_chunks<CH>(w + (int64_t)e1 * H, H, b0, lane, wb);
+      double acc = 0.0;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) eq[q] = __shfl_sync(0xffffffffu, ce, min(c0 + q, n - 1));
-    double acc[4] = {0.0, 0.0, 0.0, 0.0};
-    for (int b0 = 0; b0 < H; b0 += 32 * VE * CH) {
-      uint4 hv[CH], wv[4][CH];
+      for (int j = 0; j < CH; ++j) acc16(hv[j], wa[j], acc, hrow);
+      acc = warp_sum(acc);
+      if (lane == c) dot += acc;
+      if (c + 2 < n) load_row_chunks<CH>(w + (int64_t)__shfl_sync(0xffffffffu, ce, c + 2) * H, H, b0, lane, wa);
+      if (two) {
+        double acc1 = 0.0;
 #pragma unroll
-      for (int j = 0; j < CH; ++j) {
-        const int c = b0 + (j * 32 + lane) * VE;
-        const bool in = c < H;
-        hv[j] = in ? *reinterpret_cast<const uint4*>(hrow + c) : make_uint4(0, 0, 0, 0);
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-          wv[q][j] = in ? *reinterpret_cast<const uint4*>(w + (int64_t)eq[q] * H + c) : make_uint4(0, 0, 0, 0);
+        for (int j = 0; j < CH; ++j) acc16(hv[j], wb[j], acc1, hrow);
+        acc1 = warp_sum(acc1);
+        if (lane == c + 1) dot += acc1;
       }
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-#pragma unroll
-        for (int j = 0; j < CH; ++j) acc16(hv[j], wv[q][j], acc[q], hrow);
-    }
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const double dot = warp_sum(acc[q]);
-      if (lane == c0 + q && c0 + q < n) cv = 1.0 / (1.0 + exp(-dot)) + (double)bias[eq[q]];
     }
   }
-  double v = lane < n ? cv : -INFINITY;
+  double v = lane < n ? 1.0 / (1.0 + exp(-dot)) + (double)bias[min(ce, E - 1)] : -INFINITY;
   const int e = lane < n ? ce : 0x7fffffff;
   double gsum = 0.0, mine = 0.0;
   my_id = 0;
@@ -382,6 +426,7 @@ DLLM_DEV void warp_exact_select(float* __restrict__ srow, const float* __restric
     if (lane == j) { my_id = be; mine = sc; }
   }
   my_gate = (float)(mine / gsum);
+  return true;
 }
 
 // Cooperative exact re-decision of a CTA's near-tie tokens. The warps first list their flagged tokens; then, in
@@ -497,13 +542,13 @@ __global__ void route_topk_kernel(float* __restrict__ scores, const float* __res
 // a persistent grid whose warp w takes the tokens w, w + W, w + 2W, ... (W warps in all), reading 32 of their flags
 // at once, so near-ties that cluster in neighbouring tokens still spread over every warp. Kept apart from the top-k
 // kernel, whose register budget it would otherwise set.
-template <int PER, typename T>
-__global__ void __launch_bounds__(256, 1) route_exact_kernel(float* __restrict__ scores,
-                                                             const float* __restrict__ bias, int Tk, int E, int k,
-                                                             const T* __restrict__ h, const T* __restrict__ w,
-                                                             int H, const float* __restrict__ fix_thr,
-                                                             int32_t* __restrict__ ids, float* __restrict__ gates,
-                                                             const int32_t* __restrict__ live) {
+template <typename T>
+__global__ void __launch_bounds__(256) route_exact_kernel(const float* __restrict__ scores,
+                                                         const float* __restrict__ bias, int Tk, int E, int k,
+                                                         const T* __restrict__ h, const T* __restrict__ w, int H,
+                                                         const float* __restrict__ fix_thr,
+                                                         int32_t* __restrict__ ids, float* __restrict__ gates,
+                                                         const int32_t* __restrict__ live) {
   pdl_enter();
   if (live && *live == 0) return;   // a pass with no masked position left does nothing
   const int lane = threadIdx.x & 31;
@@ -517,11 +562,10 @@ __global__ void __launch_bounds__(256, 1) route_exact_kernel(float* __restrict__
       const int j = __ffs(bal) - 1;
       bal &= bal - 1;
       const int tt = base + j * W;
-      int my_id;
-      float my_gate;
-      warp_exact_select<PER>(scores + (int64_t)tt * E, bias, E, k, h + (int64_t)tt * H, w, H,
-                             __shfl_sync(0xffffffffu, th, j), lane, my_id, my_gate);
-      if (lane < k) {
+      int my_id = 0;
+      float my_gate = 0.f;
+      if (warp_exact_select<T>(scores + (int64_t)tt * E, bias, E, k, h + (int64_t)tt * H, w, H,
+                               __shfl_sync(0xffffffffu, th, j), lane, my_id, my_gate) && lane < k) {
         ids[(int64_t)tt * k + lane] = my_id;
         gates[(int64_t)tt * k + lane] = my_gate;
       }
@@ -903,8 +947,8 @@ int launch_select_per(float* scores, const float* bias, int Tk, int E, int k, in
   launch_pdl(route_topk_kernel<PER>, (Tk + 3) / 4, 128, 0, s, scores, bias, Tk, E, k, from_logits, ids, gates,
              rs.fix_thr, live);
   DLLM_CHECK_LAUNCH("route_topk_kernel");
-  launch_pdl(route_exact_kernel<PER, T>, std::min(num_sms(), (Tk + 7) / 8), 256, 0, s, scores, bias, Tk, E, k, h, w,
-             H, (const float*)rs.fix_thr, ids, gates, live);
+  launch_pdl(route_exact_kernel<T>, std::min(num_sms(), (Tk + 7) / 8), 256, 0, s, (const float*)scores, bias, Tk, E,
+             k, h, w, H, (const float*)rs.fix_thr, ids, gates, live);
   DLLM_CHECK_LAUNCH("route_exact_kernel");
   const int n = Tk * k, seg = rs.seg_tok * k;
   if (n <= kPermCtaMax) {   // one CTA builds the permutation

@@ -33,7 +33,8 @@ constexpr int STAGE_COLS = 32;         // epilogue column chunk
 constexpr int STAGING_BYTES = 128 * STAGE_COLS * 4;
 constexpr int MAX_GROUPS = 1040;
 constexpr int NUM_THREADS = 192;
-constexpr int NUM_THREADS_F8 = 448;    // FP8 weights: two groups of four more warps convert alternate E4M3 tiles
+constexpr int NUM_THREADS_F8 = 480;    // FP8 weights: two groups of four warps convert alternate E4M3 tiles, one
+                                       // more warp loads the activation tiles
 constexpr int F8_KS = 2;               // FP8 weights: 64-wide K blocks per stage (one 128-byte row of codes)
 constexpr int RAW_BYTES = 128 * BK * F8_KS;   // 16 KB E4M3 weight tile per stage
 constexpr int SMEM_LIMIT = 232448;
@@ -43,6 +44,8 @@ struct Smem {
   uint64_t empty[16];
   uint64_t conv[16];                // FP8: A slot's 128 TMEM rows written (128 converter arrivals)
   uint64_t mempty[16];              // FP8: A slot free again (MMA commit)
+  uint64_t bfull[8];                // FP8: activation stage landed (TMA)
+  uint64_t bempty[8];               // FP8: activation stage read by the MMAs (MMA commit)
   uint64_t tfull[2];
   uint64_t tempty[2];
   uint64_t done;
@@ -390,7 +393,7 @@ __device__ __forceinline__ float f8_row_scale(const KParams& p, int g, int mt, i
   return sc[wr];
 }
 
-template <int BN, int STAGES, bool F8 = false>
+template <int BN, int STAGES, bool F8 = false, int BST = 1>
 __global__ void __launch_bounds__(F8 ? NUM_THREADS_F8 : NUM_THREADS, 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_w2,
                const __grid_constant__ CUtensorMap tmap_x, const KParams p) {
@@ -403,22 +406,23 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
   constexpr int SBK = BK * KS;                // K elements per stage
   constexpr int B_HALF = BN * BK * 2;         // the activation tile of one 64-wide K block
   constexpr int B_BYTES = B_HALF * KS;
-  // bf16 weights: STAGES stages of [A weight tile][B activation tile]. FP8 weights: STAGES stages of [E4M3 weight
-  // codes][B activation tile] (half the weight bytes, so a deeper ring), and MS A operand slots of 32 columns in
-  // tensor memory that the converter warps fill from the codes.
-  // The slots fill the tensor memory the two accumulators leave free: a slot is busy from its conversion through
-  // the MMA's completion (a round trip of some 2000 cycles), so three slots held the FP8 kernel to half the HBM
-  // rate at decode shapes.
+  // bf16 weights: STAGES stages of [A weight tile][B activation tile]. FP8 weights: a ring of STAGES E4M3 weight
+  // tiles (the HBM stream, released by the converter warps as soon as they have read a tile, so that its depth alone
+  // sets the weight bytes in flight), a ring of BST activation tiles (from L2, released by the MMAs), and MS A
+  // operand slots in tensor memory that the converter warps fill from the codes. The slots fill the tensor memory
+  // the two accumulators leave free: a slot is busy from its conversion through the MMA's completion.
   constexpr int SLOT_COLS = 32 * KS;           // TMEM columns of one A slot (bf16 pairs of a stage's K)
   constexpr int MS = F8 ? ((512 - 2 * BN) / SLOT_COLS < 16 ? (512 - 2 * BN) / SLOT_COLS : 16) : 0;
   constexpr int MSD = MS > 0 ? MS : 1;        // slot count as a divisor (the bf16 instantiations use no slots)
   constexpr int W_BYTES = F8 ? RAW_BYTES : A_BYTES;
-  constexpr int STAGE_BYTES = W_BYTES + B_BYTES;
+  constexpr int STAGE_BYTES = F8 ? W_BYTES : W_BYTES + B_BYTES;
   constexpr uint32_t W_TX = W_BYTES;                                      // weight bytes a stage's TMA brings
   constexpr uint32_t TMEM_COLS = F8 ? 512 : 2 * BN;
   static_assert(!F8 || 2 * BN + MS * SLOT_COLS <= 512, "FP8 A slots exceed the tensor memory");
+  static_assert(!F8 || BST <= 8, "FP8 activation ring");
   uint8_t* stages = base;
-  float* staging = reinterpret_cast<float*>(base + STAGES * STAGE_BYTES);
+  uint8_t* bring = base + STAGES * STAGE_BYTES;                           // FP8 activation ring
+  float* staging = reinterpret_cast<float*>(bring + (F8 ? BST * B_BYTES : 0));
   Smem& sm = *reinterpret_cast<Smem*>(reinterpret_cast<uint8_t*>(staging) + STAGING_BYTES);
 
   const int tid = threadIdx.x;
@@ -430,12 +434,17 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
     sm.abort_flag = 0;
     for (int s = 0; s < STAGES; ++s) {
       tc::mbar_init(&sm.full[s], 1);
-      tc::mbar_init(&sm.empty[s], 1);
+      tc::mbar_init(&sm.empty[s], F8 ? 128 : 1);   // FP8: released by the 128 converter threads that read it
     }
     for (int s = 0; s < MS; ++s) {
       tc::mbar_init(&sm.conv[s], 128);   // the slot's 128 TMEM rows written
       tc::mbar_init(&sm.mempty[s], 1);   // the slot read by the MMAs
     }
+    if (F8)
+      for (int b = 0; b < BST; ++b) {
+        tc::mbar_init(&sm.bfull[b], 1);
+        tc::mbar_init(&sm.bempty[b], 1);
+      }
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(&sm.tfull[b], 1);
       tc::mbar_init(&sm.tempty[b], 128);
@@ -550,9 +559,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
           uint8_t* a = stages + s * STAGE_BYTES;
           uint8_t* b = a + W_BYTES;
           if (it < (uint32_t)npf) {   // weight stage already in flight: arrive with the activation bytes
-            tc::mbar_arrive_expect_tx(&sm.full[s], bytes - W_TX);
+            if (F8) tc::mbar_arrive(&sm.full[s]);
+            else tc::mbar_arrive_expect_tx(&sm.full[s], bytes - W_TX);
           } else {
-            tc::mbar_arrive_expect_tx(&sm.full[s], bytes);
+            tc::mbar_arrive_expect_tx(&sm.full[s], F8 ? W_TX : bytes);
             if (p.swiglu) {
               tc::tma_load_2d(a, wm, kb * SBK, (int)(wrow + mt * 64), &sm.full[s], pol_w);
               tc::tma_load_2d(a + W_TX / 2, wm, kb * SBK, (int)(wrow + p.M + mt * 64), &sm.full[s], pol_w);
@@ -560,11 +570,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
               tc::tma_load_2d(a, wm, kb * SBK, (int)(wrow + mt * 128), &sm.full[s], pol_w);
             }
           }
-#pragma unroll
-          for (int hk = 0; hk < KS; ++hk)
+          if constexpr (!F8)
             for (int j = 0; j < nb; ++j)
-              tc::tma_load_2d(b + hk * B_HALF + j * XBOX_BYTES, &tmap_x, kb * SBK + hk * BK, xrow + j * XBOX_ROWS,
-                              &sm.full[s], pol_x);
+              tc::tma_load_2d(b + j * XBOX_BYTES, &tmap_x, kb * SBK, xrow + j * XBOX_ROWS, &sm.full[s], pol_x);
         }
       }
       if (!ok) {
@@ -577,6 +585,41 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
       for (uint32_t i = it; i < (uint32_t)npf; ++i) {
         tc::mbar_arrive(&sm.full[i]);
         tc::mbar_wait(&sm.full[i], 0, 1u << 16);
+      }
+    }
+  } else if (F8 && warp == 14) {
+    // ------------------------------------------------------------------ FP8: activation producer
+    if (tc::elect_one()) {
+      tc::prefetch_tmap(&tmap_x);
+      const uint64_t pol_x = tc::policy_evict_last();
+      uint32_t it = 0;
+      bool ok = true;
+      for (int wk = wk_begin; wk < total && ok; wk += wk_step) {
+        const int t = wk / p.ksplit, ks = wk - t * p.ksplit;
+        const int kb0 = ks * kblocks / p.ksplit, kb1 = (ks + 1) * kblocks / p.ksplit;
+        int g, mt, n0, nval;
+        decode_tile<BN>(sm, p.m_tiles, t, g, mt, n0, nval);
+        const int nb = (nval + XBOX_ROWS - 1) / XBOX_ROWS;
+        const int xrow = sm.grp_off[g] + n0;
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          const int bb = it % BST;
+          if (!wait_bar(&sm.bempty[bb], ((it / BST) & 1) ^ 1, abort_flag, p.status, ST_TIMEOUT_PRODUCER)) {
+            ok = false;
+            break;
+          }
+          uint8_t* b = bring + bb * B_BYTES;
+          tc::mbar_arrive_expect_tx(&sm.bfull[bb], (uint32_t)(KS * nb * XBOX_BYTES));
+#pragma unroll
+          for (int hk = 0; hk < KS; ++hk)
+            for (int j = 0; j < nb; ++j)
+              tc::tma_load_2d(b + hk * B_HALF + j * XBOX_BYTES, &tmap_x, kb * SBK + hk * BK, xrow + j * XBOX_ROWS,
+                              &sm.bfull[bb], pol_x);
+        }
+      }
+      if (!ok) {
+        // drain: wait (bounded) for the copies of the last issued stages to land before leaving
+        const uint32_t first = it > (uint32_t)BST ? it - BST : 0;
+        for (uint32_t i = first; i < it; ++i) tc::mbar_wait(&sm.bfull[i % BST], (i / BST) & 1, 1u << 16);
       }
     }
   } else if (warp == 1) {
@@ -596,29 +639,32 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
         const uint32_t idesc = tc::idesc_bf16_f32(128, N);
         const uint32_t d = sm.tmem_base + buf * BN;
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
-          const int s = it % STAGES;
-          const uint32_t ph = (it / STAGES) & 1;
-          if (!wait_bar(&sm.full[s], ph, abort_flag, p.status, ST_TIMEOUT_MMA)) { ok = false; break; }
-          const uint32_t a = tc::smem_u32(stages + s * STAGE_BYTES);
-          const uint32_t b = a + W_BYTES;
           if constexpr (F8) {
-            // A from tensor memory: the converted slot of this k-block
-            const int ms = it % MSD;
-            if (!wait_bar(&sm.conv[ms], (it / MSD) & 1, abort_flag, p.status, ST_TIMEOUT_MMA)) { ok = false; break; }
+            // A from tensor memory (the converted slot of this stage), B from the activation ring
+            const int ms = it % MSD, bb = it % BST;
+            if (!wait_bar(&sm.bfull[bb], (it / BST) & 1, abort_flag, p.status, ST_TIMEOUT_MMA) ||
+                !wait_bar(&sm.conv[ms], (it / MSD) & 1, abort_flag, p.status, ST_TIMEOUT_MMA)) { ok = false; break; }
             tc::fence_after_sync();
+            const uint32_t b = tc::smem_u32(bring + bb * B_BYTES);
             const uint32_t ta = sm.tmem_base + 2 * BN + ms * SLOT_COLS;
 #pragma unroll
             for (int kk = 0; kk < SBK / 16; ++kk)
               tc::mma_bf16_tmem_a(d, ta + kk * 8, tc::sdesc_k128(b + (kk >> 2) * B_HALF + (kk & 3) * 32), idesc,
                                   (kb != kb0) || kk != 0);
             tc::mma_commit(&sm.mempty[ms]);
+            tc::mma_commit(&sm.bempty[bb]);
           } else {
+            const int s = it % STAGES;
+            const uint32_t ph = (it / STAGES) & 1;
+            if (!wait_bar(&sm.full[s], ph, abort_flag, p.status, ST_TIMEOUT_MMA)) { ok = false; break; }
+            const uint32_t a = tc::smem_u32(stages + s * STAGE_BYTES);
+            const uint32_t b = a + W_BYTES;
             tc::fence_after_sync();
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk)
               tc::mma_bf16(d, tc::sdesc_k128(a + kk * 32), tc::sdesc_k128(b + kk * 32), idesc, (kb != kb0) || kk != 0);
+            tc::mma_commit(&sm.empty[s]);
           }
-          tc::mma_commit(&sm.empty[s]);
         }
         if (!ok) break;
         tc::mma_commit(&sm.tfull[buf]);
@@ -628,7 +674,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
       tc::mbar_wait(&sm.done, 0, 1u << 20);
     }
   } else if (F8 && warp >= 6) {
-    // ------------------------------------------------------------------ FP8: converter warps 6..13
+    // ------------------------------------------------------------------ FP8: converter warps 6..13 (warp 14 took
+    // the branch above)
     // two groups of four warps (one per TMEM lane quadrant) take alternate k-blocks, so that one group's loads,
     // conversions and store waits overlap the other's. Per k-block, in the MMA's order: once the A slot is free and
     // the stage's codes have landed, each thread writes its TMEM lane of the slot from its row of codes, waits for
@@ -648,6 +695,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
         tc::fence_after_sync();
         convert_e4m3_row_to_tmem(stages + s * STAGE_BYTES, row,
                                  sm.tmem_base + ((uint32_t)((warp & 3) * 32) << 16) + 2 * BN + ms * SLOT_COLS);
+        tc::mbar_arrive(&sm.empty[s]);   // this thread's codes are read (release orders the loads before it)
         tc::tmem_st_wait();
         tc::fence_before_sync();
         tc::mbar_arrive(&sm.conv[ms]);
@@ -1057,12 +1105,12 @@ int make_map(CUtensorMap* m, const void* ptr, int64_t rows, int K, int box_rows,
 int launch_cluster_splitk(const GemmArgs& a, const CUtensorMap& mw, const CUtensorMap& mw2, const CUtensorMap& mx,
                           const KParams& kp, cudaStream_t s);
 
-template <int BN, int STAGES, bool F8 = false>
+template <int BN, int STAGES, bool F8 = false, int BST = 1>
 int launch(const GemmArgs& a, const CUtensorMap& mw, const CUtensorMap& mw2, const CUtensorMap& mx,
            const KParams& kp, cudaStream_t s) {
-  // (matches the kernel's layout: stages of [weights (bf16 or E4M3)][activations])
-  constexpr int STAGE_BYTES = F8 ? RAW_BYTES + BN * BK * 2 * F8_KS : A_BYTES + BN * BK * 2;
-  constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + STAGING_BYTES + (int)sizeof(Smem);
+  // (matches the kernel's layout: bf16 stages of [weights][activations]; FP8 rings of codes and of activations)
+  constexpr int SMEM = F8 ? 1024 + STAGES * RAW_BYTES + BST * BN * BK * 2 * F8_KS + STAGING_BYTES + (int)sizeof(Smem)
+                          : 1024 + STAGES * (A_BYTES + BN * BK * 2) + STAGING_BYTES + (int)sizeof(Smem);
   static_assert(SMEM <= SMEM_LIMIT, "shared memory budget");
   // With programmatic dependent launch a CTA allocates tensor memory before it waits for the kernels ahead of it.
   // More than half an SM's shared memory per CTA keeps two tensor-memory kernels from sharing an SM, so a later
@@ -1070,12 +1118,13 @@ int launch(const GemmArgs& a, const CUtensorMap& mw, const CUtensorMap& mw2, con
   static_assert(SMEM > 233472 / 2, "tensor-memory kernels must not share an SM");
   static bool configured = false;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, STAGES, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         SMEM);
+    cudaError_t e = cudaFuncSetAttribute(gemm_tc_kernel<BN, STAGES, F8, BST>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
     if (e != cudaSuccess) return dllm_host::cuda_status(e, "cudaFuncSetAttribute(gemm_tc)");
     configured = true;
   }
-  launch_pdl((gemm_tc_kernel<BN, STAGES, F8>), num_sms(), F8 ? NUM_THREADS_F8 : NUM_THREADS, SMEM, s, mw, mw2, mx, kp);
+  launch_pdl((gemm_tc_kernel<BN, STAGES, F8, BST>), num_sms(), F8 ? NUM_THREADS_F8 : NUM_THREADS, SMEM, s, mw, mw2,
+             mx, kp);
   DLLM_CHECK_LAUNCH("gemm_tc_kernel");
   return DLLM_OK;
 }
@@ -1256,9 +1305,9 @@ int gemm_bf16_tc(const GemmArgs& a, cudaStream_t s) {
   kp.prefetch_w = (!a.swiglu && !a.n_dev && !a.has_extra && a.host_cnt <= (ks > 1 ? 32 : bn)) ? 1 : 0;
   int st2;
   if (f8) {   // single-CTA tiles, no split-K (the weight-streaming shapes FP8 weights serve)
-    if (bn == 32) st2 = launch<32, 8, true>(a, mw, mw2, mx, kp, s);
-    else if (bn == 64) st2 = launch<64, 6, true>(a, mw, mw2, mx, kp, s);
-    else st2 = launch<128, 4, true>(a, mw, mw2, mx, kp, s);
+    if (bn == 32) st2 = launch<32, 10, true, 3>(a, mw, mw2, mx, kp, s);
+    else if (bn == 64) st2 = launch<64, 9, true, 3>(a, mw, mw2, mx, kp, s);
+    else st2 = launch<128, 8, true, 2>(a, mw, mw2, mx, kp, s);
   } else if (gemm_uses_pairs(a)) {
     kp.prefetch_w = 0;
     st2 = launch_pair(mw, mw2, mx, kp, s);

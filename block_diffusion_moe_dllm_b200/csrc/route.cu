@@ -354,11 +354,15 @@ __device__ __noinline__ void exact_select_many(const float* __restrict__ srow, c
 }
 
 // Exact selection of one near-tie token by its own warp. The candidate experts (fp32 biased score at least thr,
-// the (k+1)-th value minus the guard) are compacted into lanes; each candidate's exact score is a warp-wide dot
-// product with the token row held in registers, the next candidate's weight row loading while the current one is
-// summed (bf16 products are exact in fp32 and are added in fp64); then k rounds of a warp arg-max give the slots
-// in order (ties -> lower expert) and the gates (unbiased fp64 scores renormalised). Returns false (the fp32
-// decision stands) only when fewer than k experts pass the threshold, which takes non-finite scores.
+// the (k+1)-th value minus the guard) are compacted into lanes and sorted by their fp32 biased score (ties -> lower
+// expert). A candidate whose fp32 value is within kRouteGuard of a neighbour in that order is uncertain; only the
+// uncertain ones are scored exactly (a warp-wide dot product of the token row, held in registers, with the
+// expert's row, the next uncertain expert's row loading while the current one is summed: bf16 products are exact
+// in fp32 and are added in fp64). Every fp32 score is within half the guard of its exact value, so a certain
+// candidate's fp32 value orders it against every other candidate exactly as the exact values would; the selection
+// (k rounds of a warp arg-max on exact values where computed, fp32 values elsewhere) therefore equals the exact
+// one, with the gates from the same scores. Returns false (the fp32 decision stands) only when fewer than k
+// experts pass the threshold, which takes non-finite scores.
 template <typename T>
 DLLM_DEV bool warp_exact_select(const float* __restrict__ srow, const float* __restrict__ bias, int E, int k,
                                 const T* __restrict__ hrow, const T* __restrict__ w, int H, float thr, int lane,
@@ -382,33 +386,61 @@ DLLM_DEV bool warp_exact_select(const float* __restrict__ srow, const float* __r
     exact_select_many<T>(srow, bias, E, k, hrow, w, H, thr, lane, &my_id, &my_gate);
     return true;
   }
-  double dot = 0.0;   // lane j < n: candidate j's dot product
-  for (int b0 = 0; b0 < H; b0 += BLK) {
+  // sort the candidates by (fp32 biased value desc, expert asc): bitonic network over the warp
+  float fv = lane < n ? srow[ce] + bias[ce] : -INFINITY;
+  int fe = lane < n ? ce : 0x7fffffff;
+#pragma unroll
+  for (int size = 2; size <= 32; size <<= 1) {
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, fv, stride);
+      const int oe = __shfl_xor_sync(0xffffffffu, fe, stride);
+      const bool other_first = ov > fv || (ov == fv && oe < fe);   // the partner precedes this lane's entry
+      const bool lower = (lane & stride) == 0;                     // this lane takes the earlier position
+      const bool desc = (lane & size) == 0 || size == 32;          // the final merge runs one way
+      if ((lower == desc) == other_first) { fv = ov; fe = oe; }
+    }
+  }
+  const float prv = __shfl_up_sync(0xffffffffu, fv, 1), nxt = __shfl_down_sync(0xffffffffu, fv, 1);
+  const bool unc = lane < n && ((lane > 0 && prv - fv < kRouteGuard) || (lane + 1 < n && fv - nxt < kRouteGuard));
+  const unsigned ubal = __ballot_sync(0xffffffffu, unc);
+  double dot = 0.0;   // uncertain lanes: the candidate's exact dot product
+  const int nu = __popc(ubal);
+  for (int b0 = 0; b0 < H && nu > 0; b0 += BLK) {
     uint4 hv[CH], wa[CH], wb[CH];
+    unsigned rest = ubal;
+    int cur = __ffs(rest) - 1;
+    rest &= rest - 1;
     load_row_chunks<CH>(hrow, H, b0, lane, hv);
-    load_row_chunks<CH>(w + (int64_t)__shfl_sync(0xffffffffu, ce, 0) * H, H, b0, lane, wa);
+    load_row_chunks<CH>(w + (int64_t)__shfl_sync(0xffffffffu, fe, cur) * H, H, b0, lane, wa);
 #pragma unroll 1
-    for (int c = 0; c < n; c += 2) {
-      const bool two = c + 1 < n;
-      const int e1 = __shfl_sync(0xffffffffu, ce, two ? c + 1 : c);
-      if (two) load_row_chunks<CH>(w + (int64_t)e1 * H, H, b0, lane, wb);
+    while (cur >= 0) {
+      const int nx = rest ? __ffs(rest) - 1 : -1;
+      if (rest) rest &= rest - 1;
+      if (nx >= 0) load_row_chunks<CH>(w + (int64_t)__shfl_sync(0xffffffffu, fe, nx) * H, H, b0, lane, wb);
       double acc = 0.0;
 #pragma unroll
       for (int j = 0; j < CH; ++j) acc16(hv[j], wa[j], acc, hrow);
       acc = warp_sum(acc);
-      if (lane == c) dot += acc;
-      if (c + 2 < n) load_row_chunks<CH>(w + (int64_t)__shfl_sync(0xffffffffu, ce, c + 2) * H, H, b0, lane, wa);
-      if (two) {
-        double acc1 = 0.0;
+      if (lane == cur) dot += acc;
+      cur = nx;
+      if (cur < 0) break;
+      const int nx2 = rest ? __ffs(rest) - 1 : -1;
+      if (rest) rest &= rest - 1;
+      if (nx2 >= 0) load_row_chunks<CH>(w + (int64_t)__shfl_sync(0xffffffffu, fe, nx2) * H, H, b0, lane, wa);
+      double acc1 = 0.0;
 #pragma unroll
-        for (int j = 0; j < CH; ++j) acc16(hv[j], wb[j], acc1, hrow);
-        acc1 = warp_sum(acc1);
-        if (lane == c + 1) dot += acc1;
-      }
+      for (int j = 0; j < CH; ++j) acc16(hv[j], wb[j], acc1, hrow);
+      acc1 = warp_sum(acc1);
+      if (lane == cur) dot += acc1;
+      cur = nx2;
     }
   }
-  double v = lane < n ? 1.0 / (1.0 + exp(-dot)) + (double)bias[min(ce, E - 1)] : -INFINITY;
-  const int e = lane < n ? ce : 0x7fffffff;
+  // selection keys: exact biased and unbiased scores where computed, fp32 elsewhere
+  const int eb = lane < n ? fe : 0;
+  const double raw = unc ? 1.0 / (1.0 + exp(-dot)) : (double)srow[eb];
+  double v = lane < n ? (unc ? raw + (double)bias[eb] : (double)fv) : -INFINITY;
+  const int e = lane < n ? fe : 0x7fffffff;
   double gsum = 0.0, mine = 0.0;
   my_id = 0;
   for (int j = 0; j < k; ++j) {
@@ -420,8 +452,8 @@ DLLM_DEV bool warp_exact_select(const float* __restrict__ srow, const float* __r
       const int oe = __shfl_xor_sync(0xffffffffu, be, o);
       if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
     }
+    const double sc = __shfl_sync(0xffffffffu, raw, __ffs(__ballot_sync(0xffffffffu, e == be)) - 1);
     if (e == be) v = -INFINITY;
-    const double sc = bv - (double)bias[be];
     gsum += sc;
     if (lane == j) { my_id = be; mine = sc; }
   }

@@ -1305,9 +1305,11 @@ int gemm_bf16_tc(const GemmArgs& a, cudaStream_t s) {
   kp.prefetch_w = (!a.swiglu && !a.n_dev && !a.has_extra && a.host_cnt <= (ks > 1 ? 32 : bn)) ? 1 : 0;
   int st2;
   if (f8) {   // single-CTA tiles, no split-K (the weight-streaming shapes FP8 weights serve)
-    if (bn == 32) st2 = launch<32, 10, true, 3>(a, mw, mw2, mx, kp, s);
-    else if (bn == 64) st2 = launch<64, 9, true, 3>(a, mw, mw2, mx, kp, s);
-    else st2 = launch<128, 8, true, 2>(a, mw, mw2, mx, kp, s);
+    // (weight-code ring, activation ring): the activation ring also has to cover a load from L2 plus the wait for
+    // the stage's conversion and MMA, so it is not kept minimal
+    if (bn == 32) st2 = launch<32, 9, true, 6>(a, mw, mw2, mx, kp, s);
+    else if (bn == 64) st2 = launch<64, 8, true, 4>(a, mw, mw2, mx, kp, s);
+    else st2 = launch<128, 6, true, 3>(a, mw, mw2, mx, kp, s);
   } else if (gemm_uses_pairs(a)) {
     kp.prefetch_w = 0;
     st2 = launch_pair(mw, mw2, mx, kp, s);

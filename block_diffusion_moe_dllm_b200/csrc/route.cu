@@ -86,10 +86,20 @@ __global__ void __launch_bounds__(256) route_scores_kernel(const T* __restrict__
 // score or above it are re-scored.
 constexpr float kRouteGuard = 1e-5f;
 
+// Order-preserving map of a float to an unsigned key (and back): larger floats get larger keys, -inf the smallest.
+DLLM_DEV uint32_t ord_key(float x) {
+  const uint32_t u = __float_as_uint(x);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+DLLM_DEV float ord_value(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
 // Top-k of one token's expert scores, one warp. Lane l owns experts e = i * 32 + l (i < PER); the selection key is
 // the biased score val = raw + bias (ties to the lower expert), the gate the unbiased raw score, renormalised over
 // the chosen k. Each lane sorts its PER candidates with an insertion network (descending val, ascending e); then
-// k rounds take the warp-wide best head (a 5-step butterfly on (val, e)) and the winning lane pops its head; one
+// k rounds take the warp-wide best head (two warp reductions: the largest val, then the lowest e holding it) and
+// the winning lane pops its head; one
 // more round reads the (k+1)-th value without popping it. With from_logits the raw scores are sigmoid(logit) and
 // are written back over the logits. Returns (warp-uniform) whether two consecutive values among the top k + 1
 // are closer than kRouteGuard; thr is then the (k+1)-th value minus the guard (-inf when k == E).
@@ -141,14 +151,12 @@ DLLM_DEV bool warp_topk(float* __restrict__ srow, const float* __restrict__ bias
   my_gate = 0.f;
   const int rounds = k < E ? k + 1 : k;
   for (int j = 0; j < rounds; ++j) {
-    float bv = v[0];
-    int be = e[0];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
-      if (ov > bv || (ov == bv && oe < be)) { bv = ov; be = oe; }
-    }
+    // the warp's best head: the largest value (an order-preserving unsigned image of the float, one warp
+    // reduction), then the lowest expert among the heads that hold it (a second one)
+    const uint32_t key = ord_key(v[0]);
+    const uint32_t kmax = __reduce_max_sync(0xffffffffu, key);
+    const int be = (int)__reduce_min_sync(0xffffffffu, key == kmax ? (uint32_t)e[0] : 0xffffffffu);
+    const float bv = ord_value(kmax);
     if (j > 0 && prev - bv < kRouteGuard) near = true;
     prev = bv;
     if (j == k) {   // the (k+1)-th value: read, not taken

@@ -88,9 +88,14 @@ void carve_experts(Carver& c, int dtype, int Tk, int H, int k, int I, int shared
   b.scratch = dtype == DLLM_F32 ? c.take<float>(gemm_f32_scratch_bytes(rows, std::max(2 * I, H), 0)) : nullptr;
 }
 
+// N tile of the expert GEMMs (the host cannot see the routed counts): wide enough for four times the average rows
+// per expert and at least 128, since a denoising block's masked positions share most of their routing (the block
+// starts from one mask token), which piles many rows on a few experts; an expert with more rows than the N tile
+// streams its weight tiles once per extra tile (measured: 128 instead of 64 took one understanding layer from 463
+// to 449 us; random routing is unaffected).
 int expert_bn_hint(int Tk, int k, int E) {
   const int avg = (Tk * k + E - 1) / E;
-  return std::min(Tk, std::max(64, 4 * avg));
+  return std::min(Tk, std::max(128, 4 * avg));
 }
 
 // The combine's follow-up RMSNorm, fused into it (PostNorm::g == nullptr: plain combine).

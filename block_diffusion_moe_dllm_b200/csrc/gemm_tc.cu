@@ -739,13 +739,17 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
         tc::fence_before_sync();
         tc::mbar_arrive(&sm.tempty[buf]);
       } else {
-        // cluster split-K (BN == 32, one chunk): this slice's accumulator into this CTA's staging tile
-        float v[STAGE_COLS];
-        const uint32_t taddr = sm.tmem_base + ((uint32_t)(q * 32) << 16) + buf * BN;
-        tc::tmem_ld16(taddr, v);
-        tc::tmem_ld16(taddr + 16, v + 16);
+        // cluster split-K: this slice's accumulator as [column][128 rows] fp32, in the staging tile (N tile 32) or
+        // in the operand ring, idle now (wider N tiles; this CTA's one work item has been consumed)
+        float* accs = BN == 32 ? staging : reinterpret_cast<float*>(stages);
+        for (int c0 = 0; c0 < nval; c0 += STAGE_COLS) {
+          float v[STAGE_COLS];
+          const uint32_t taddr = sm.tmem_base + ((uint32_t)(q * 32) << 16) + buf * BN + c0;
+          tc::tmem_ld16(taddr, v);
+          tc::tmem_ld16(taddr + 16, v + 16);
 #pragma unroll
-        for (int j = 0; j < STAGE_COLS; ++j) staging[j * 128 + row] = v[j];
+          for (int j = 0; j < STAGE_COLS; ++j) accs[(c0 + j) * 128 + row] = v[j];
+        }
         tc::fence_before_sync();
         tc::mbar_arrive(&sm.tempty[buf]);
       }
@@ -779,15 +783,17 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
       decode_tile<BN>(sm, p.m_tiles, t, g, mt, n0, nval);
       const int etid = tid - 64;
       const int cb = rank * nval / p.ksplit, ce = (rank + 1) * nval / p.ksplit;
-      float* red = reinterpret_cast<float*>(stages);   // the operand ring is idle now
+      // every slice's accumulator (see above) and, after it, this rank's sums (the operand ring is idle now)
+      const float* accs = BN == 32 ? staging : reinterpret_cast<const float*>(stages);
+      float* red = reinterpret_cast<float*>(stages) + (BN == 32 ? 0 : 128 * BN);
       const int r8 = (etid & 15) * 8;                   // rows r8 .. r8 + 7
       for (int j = cb + (etid >> 4); j < ce; j += 8) {
         float4 lo[8], hi[8];
 #pragma unroll
         for (int sp = 0; sp < 8; ++sp) {
           const uint32_t rk = sp < p.ksplit ? (uint32_t)sp : 0u;
-          lo[sp] = ld_dsmem4(staging + j * 128 + r8, rk);
-          hi[sp] = ld_dsmem4(staging + j * 128 + r8 + 4, rk);
+          lo[sp] = ld_dsmem4(accs + j * 128 + r8, rk);
+          hi[sp] = ld_dsmem4(accs + j * 128 + r8 + 4, rk);
         }
         float4 a = lo[0], c = hi[0];
 #pragma unroll
@@ -803,7 +809,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
       cluster_arrive();
       arrived = true;
       tc::named_bar_sync(1, 128);
-      if (ce > cb) epilogue_chunk<BN>(p, red, g, mt, n0 + cb, ce - cb, 0, sm.grp_off[g], etid);
+      for (int c = 0; c < ce - cb; c += STAGE_COLS)
+        epilogue_chunk<BN>(p, red + c * 128, g, mt, n0 + cb + c, ce - cb - c, 0, sm.grp_off[g], etid);
     }
     if (!arrived) cluster_arrive();
     cluster_wait();
@@ -1197,6 +1204,78 @@ int launch_cluster_splitk(const GemmArgs& a, const CUtensorMap& mw, const CUtens
   return DLLM_OK;
 }
 
+// ---- wide split-K: dense projections over several N tiles of rows (the 512 rows of a denoising block) whose
+// 128-row tiles would each stream a whole K of weights and tokens on fewer SMs than the GPU has. N tiles of 128 or
+// 256 rows split along K over a thread-block cluster put every SM to work on a slice with less operand traffic per
+// SM; each slice's accumulator goes through the idle operand ring to the cluster's reduction.
+template <int BN, int STAGES>
+constexpr int splitk_smem() {
+  return 1024 + STAGES * (A_BYTES + BN * BK * 2) + STAGING_BYTES + (int)sizeof(Smem);
+}
+
+template <int BN, int STAGES>
+static cudaError_t configure_splitk_t() {
+  static cudaError_t st = cudaFuncSetAttribute(gemm_tc_kernel<BN, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               splitk_smem<BN, STAGES>());
+  return st;
+}
+
+template <int BN, int STAGES>
+static int max_active_clusters_t(int ks) {
+  static int cache[9] = {0};
+  if (ks < 1 || ks > 8) return 0;
+  if (cache[ks] > 0) return cache[ks];
+  int n = 0;
+  if (configure_splitk_t<BN, STAGES>() == cudaSuccess) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(ks, 1, 1);
+    cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = splitk_smem<BN, STAGES>();
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = ks;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel<BN, STAGES>, &cfg) != cudaSuccess) n = 0;
+  }
+  if (n <= 0) {
+    cudaGetLastError();
+    n = num_sms() / (2 * ks);
+  }
+  cache[ks] = std::max(n, 1);
+  return cache[ks];
+}
+
+template <int BN, int STAGES>
+static int launch_wide_splitk(const GemmArgs& a, const CUtensorMap& mw, const CUtensorMap& mw2, const CUtensorMap& mx,
+                              const KParams& kp, cudaStream_t s) {
+  static_assert(splitk_smem<BN, STAGES>() <= SMEM_LIMIT, "shared memory budget");
+  static_assert(STAGES * (A_BYTES + BN * BK * 2) >= 128 * BN * 4 + 128 * (BN / 2) * 4,
+                "the operand ring holds a slice's accumulator and a rank's sums");
+  cudaError_t e = configure_splitk_t<BN, STAGES>();
+  if (e != cudaSuccess) return dllm_host::cuda_status(e, "cudaFuncSetAttribute(gemm_tc wide split-K)");
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(kp.ksplit, (a.M / 128) * ((a.host_cnt + BN - 1) / BN), 1);
+  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = splitk_smem<BN, STAGES>();
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kp.ksplit;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // see pdl_wait
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  e = cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, STAGES>, mw, mw2, mx, kp);
+  if (e != cudaSuccess) return dllm_host::cuda_status(e, "cudaLaunchKernelEx(gemm_tc wide split-K)");
+  DLLM_CHECK_LAUNCH("gemm_tc_kernel (wide split-K)");
+  return DLLM_OK;
+}
+
 static_assert(PAIR_SMEM <= SMEM_LIMIT, "shared memory budget (CTA pairs)");
 static_assert(PAIR_SMEM > 233472 / 2, "tensor-memory kernels must not share an SM");
 
@@ -1296,8 +1375,9 @@ int gemm_bf16_tc(const GemmArgs& a, cudaStream_t s) {
   kp.w2_scale = a.w2_scale;
   kp.epi = a.epi;
   kp.status = a.status;
-  const int bn = gemm_bn(a);
-  const int ks = gemm_splitk_factor(a, bn);
+  const WideSplit wide = wide_splitk_plan(a);
+  const int bn = wide.ks > 1 ? wide.bn : gemm_bn(a);
+  const int ks = wide.ks > 1 ? wide.ks : gemm_splitk_factor(a, bn);
   if (a.epi.conf_part)
     DLLM_REQUIRE(a.epi.conf_nparts > 0 && gemm_conf_parts(a) == a.epi.conf_nparts, DLLM_ERR_UNSUPPORTED,
                  "gemm: fused confidence epilogue unsupported for this shape");
@@ -1313,6 +1393,9 @@ int gemm_bf16_tc(const GemmArgs& a, cudaStream_t s) {
   } else if (gemm_uses_pairs(a)) {
     kp.prefetch_w = 0;
     st2 = launch_pair(mw, mw2, mx, kp, s);
+  } else if (wide.ks > 1) {
+    st2 = wide.bn == 128 ? launch_wide_splitk<128, 6>(a, mw, mw2, mx, kp, s)
+                         : launch_wide_splitk<256, 4>(a, mw, mw2, mx, kp, s);
   } else if (ks > 1) st2 = launch_cluster_splitk(a, mw, mw2, mx, kp, s);
   else if (bn == 32) st2 = launch<32, 9>(a, mw, mw2, mx, kp, s);
   else if (bn == 64) st2 = launch<64, 8>(a, mw, mw2, mx, kp, s);
@@ -1356,6 +1439,32 @@ int gemm_splitk_factor(const GemmArgs& a, int bn) {
   int ks = std::max(1, std::min(std::min(kblocks / 2, 8), num_sms() / tiles));
   while (ks > 1 && tiles > max_active_clusters(ks)) --ks;
   return ks;
+}
+
+// Wide split-K plan (see launch_wide_splitk) for a dense bf16 projection over more than one 32-row tile with a
+// row count fixed on the host: among N tiles of 128 and 256 rows and 2..8 K slices whose clusters all fit in one
+// wave, the one with the least operand traffic per CTA ((128 + N tile) x K / slices), taken when it is at most
+// three quarters of the plain kernel's (one 128 x gemm_bn tile per CTA, or several when tiles outnumber SMs).
+// Measured at 512 rows: QKV 23 -> ... us, output projection 17 -> ... us.
+WideSplit wide_splitk_plan(const GemmArgs& a) {
+  WideSplit best;
+  if (a.dtype != DLLM_BF16 || !dense(a) || a.w_fp8 || a.epi.conf_part || a.cnt_dev || a.host_cnt <= 32) return best;
+  const int kblocks = a.K / BK, mt = a.M / 128, rows = a.host_cnt, sms = num_sms();
+  const int bn0 = gemm_bn(a);
+  const int tiles0 = mt * ((rows + bn0 - 1) / bn0);
+  const double base = (double)(128 + std::min(bn0, rows)) * a.K * ((tiles0 + sms - 1) / sms);
+  double cost = 0.75 * base;
+  for (int bn : {128, 256}) {
+    const int tiles = mt * ((rows + bn - 1) / bn);
+    for (int ks = 2; ks <= 8 && 2 * ks <= kblocks; ++ks) {
+      if (tiles * ks > sms) break;
+      const int act = bn == 128 ? max_active_clusters_t<128, 6>(ks) : max_active_clusters_t<256, 4>(ks);
+      if (tiles > act) continue;
+      const double c = (double)(128 + std::min(bn, rows)) * a.K / ks;
+      if (c < cost) { cost = c; best.bn = bn; best.ks = ks; }
+    }
+  }
+  return best;
 }
 
 bool gemm_uses_pairs(const GemmArgs& a) {

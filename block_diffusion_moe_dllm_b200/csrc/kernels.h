@@ -92,6 +92,12 @@ int gemm_bf16_tc(const GemmArgs& a, cudaStream_t s);
 int bn_for(int max_cnt);
 int gemm_bn(const GemmArgs& a);
 int gemm_splitk_factor(const GemmArgs& a, int bn);
+// N tile and K slices of a dense projection run as wide split-K clusters (ks > 1), or ks = 1 when the plain or the
+// 32-row split-K kernel serves it better.
+struct WideSplit {
+  int bn = 0, ks = 1;
+};
+WideSplit wide_splitk_plan(const GemmArgs& a);
 
 int gemm_f32_simt(const GemmArgs& a, cudaStream_t s);
 size_t gemm_f32_scratch_bytes(int64_t x_rows, int M, int swiglu);

@@ -51,6 +51,23 @@ def test_gemm_bf16_split_k(N, M, K):
     assert_close(to64(y), O.store(to64(y0) + to64(x) @ to64(w).T, "bf16"), "bf16", "split-K gemm")
 
 
+@pytest.mark.parametrize("N,M,K,residual", [(512, 3072, 2048, 0), (512, 2048, 2048, 1), (300, 2048, 1024, 1),
+                                            (384, 1024, 2048, 0)])
+def test_gemm_bf16_wide_split_k(N, M, K, residual):
+    """A block's rows (a few hundred) against a dense projection: N tiles of 128 or 256 rows whose K slices run as
+    one cluster, every slice's accumulator staged in its operand ring and each rank reducing and storing its share
+    of the columns (ragged last N tile at 300 rows)."""
+    x = synth.normal((N, K), 1.0, 12, f"wx{N}{K}", DEV)
+    w = synth.normal((M, K), 0.02, 12, f"ww{M}{K}", DEV)
+    y0 = synth.normal((N, M), 1.0, 12, f"wy{N}{M}", DEV)
+    y = y0.clone()
+    bd.gemm(x, w, y, N, M, K, bd.BF16, residual=residual)
+    torch.cuda.synchronize()
+    acc = to64(x) @ to64(w).T
+    want = O.store(to64(y0) + acc, "bf16") if residual else O.store(acc, "bf16")
+    assert_close(to64(y), want, "bf16", "gemm (wide split-K)")
+
+
 @pytest.mark.parametrize("N,M,K,residual", [(1200, 2048, 256, 0), (4100, 2048, 512, 1), (600, 4096, 128, 0)])
 def test_gemm_bf16_cta_pairs(N, M, K, residual):
     """N tile 256 with enough tiles: CTA pairs share each MMA (M = 256 across two SMs, half of the N tile's rows

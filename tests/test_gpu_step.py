@@ -225,6 +225,14 @@ def test_step_small_bf16_sprint_mixed_modality():
         assert np.all((kp < 64).sum(axis=1) == 32)
 
 
+def test_step_block_rows_full_width_projections():
+    """Sixteen rows of a 32-token block (512 token rows) through full-width projections (hidden 2048, 16 q heads,
+    4 kv heads): the QKV projection with RoPE and cache writes and the output projection with the residual run as
+    wide split-K clusters, whose ranks each write their share of the columns."""
+    w = scaled(ONE_LAYER, name="block-rows-h2048", n_layers=1, E=8, k=2, I=128, V=1024, B=16, P=64, L=32, T_s=4)
+    _one_pass(w, seed=13)
+
+
 def test_step_small_bf16_threshold():
     w = scaled(SMALL, mode=1, tau=0.9, k_max=8, T_s=16, lm_std=1.0)
     _one_pass(w, seed=5)

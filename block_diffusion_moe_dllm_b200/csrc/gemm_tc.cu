@@ -786,25 +786,29 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
       // every slice's accumulator (see above) and, after it, this rank's sums (the operand ring is idle now)
       const float* accs = BN == 32 ? staging : reinterpret_cast<const float*>(stages);
       float* red = reinterpret_cast<float*>(stages) + (BN == 32 ? 0 : 128 * BN);
-      const int r8 = (etid & 15) * 8;                   // rows r8 .. r8 + 7
-      for (int j = cb + (etid >> 4); j < ce; j += 8) {
-        float4 lo[8], hi[8];
+      // the share is columns [cb, ce) of every slice, one contiguous run of 128-row columns: each thread sums
+      // 16-byte vectors of it over the slices in rank order, two vectors at a time with the loads from every
+      // slice issued before the first add (2 x ksplit loads from distributed shared memory in flight per thread)
+      const int n4 = (ce - cb) * 32;   // float4 vectors in the share
+      const float4* src = reinterpret_cast<const float4*>(accs + cb * 128);
+      float4* dst = reinterpret_cast<float4*>(red);
+      for (int i0 = etid; i0 < n4; i0 += 2 * 128) {
+        float4 v[8][2];
 #pragma unroll
-        for (int sp = 0; sp < 8; ++sp) {
-          const uint32_t rk = sp < p.ksplit ? (uint32_t)sp : 0u;
-          lo[sp] = ld_dsmem4(accs + j * 128 + r8, rk);
-          hi[sp] = ld_dsmem4(accs + j * 128 + r8 + 4, rk);
-        }
-        float4 a = lo[0], c = hi[0];
+        for (int sp = 0; sp < 8; ++sp)
 #pragma unroll
-        for (int sp = 1; sp < 8; ++sp) {
-          if (sp < p.ksplit) {
-            a.x += lo[sp].x; a.y += lo[sp].y; a.z += lo[sp].z; a.w += lo[sp].w;
-            c.x += hi[sp].x; c.y += hi[sp].y; c.z += hi[sp].z; c.w += hi[sp].w;
-          }
+          for (int u = 0; u < 2; ++u)
+            v[sp][u] = (sp < p.ksplit && i0 + u * 128 < n4)
+                           ? ld_dsmem4(reinterpret_cast<const float*>(src + i0 + u * 128), (uint32_t)sp)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          float4 a = v[0][u];
+#pragma unroll
+          for (int sp = 1; sp < 8; ++sp)
+            if (sp < p.ksplit) { a.x += v[sp][u].x; a.y += v[sp][u].y; a.z += v[sp][u].z; a.w += v[sp][u].w; }
+          if (i0 + u * 128 < n4) dst[i0 + u * 128] = a;
         }
-        *reinterpret_cast<float4*>(red + (j - cb) * 128 + r8) = a;
-        *reinterpret_cast<float4*>(red + (j - cb) * 128 + r8 + 4) = c;
       }
       cluster_arrive();
       arrived = true;

@@ -1446,13 +1446,16 @@ int gemm_splitk_factor(const GemmArgs& a, int bn) {
 }
 
 // Wide split-K plan (see launch_wide_splitk) for a dense bf16 projection over more than one 32-row tile with a
-// row count fixed on the host: among N tiles of 128 and 256 rows and 2..8 K slices whose clusters all fit in one
-// wave, the one with the least operand traffic per CTA ((128 + N tile) x K / slices), taken when it is at most
-// three quarters of the plain kernel's (one 128 x gemm_bn tile per CTA, or several when tiles outnumber SMs).
-// Measured at 512 rows: QKV 23 -> ... us, output projection 17 -> ... us.
+// row count fixed on the host and at most four 128-row weight tiles (the router's logits): among N tiles of 128
+// and 256 rows and 2..8 K slices whose clusters all fit in one wave, the one with the least operand traffic per CTA
+// ((128 + N tile) x K / slices), taken when it is at most three quarters of the plain kernel's. Measured at 512
+// rows: the router (256 experts x 2048) 32.1 -> 29.4 us for logits, top-k and permutation; the wider QKV and
+// output projections gained nothing (15.9 us both ways) or lost (12.5 -> 15.0 us): their slices' 64-128 KB
+// accumulators cost as much to stage and reduce as the operand traffic saved.
 WideSplit wide_splitk_plan(const GemmArgs& a) {
   WideSplit best;
   if (a.dtype != DLLM_BF16 || !dense(a) || a.w_fp8 || a.epi.conf_part || a.cnt_dev || a.host_cnt <= 32) return best;
+  if (a.M > 512) return best;
   const int kblocks = a.K / BK, mt = a.M / 128, rows = a.host_cnt, sms = num_sms();
   const int bn0 = gemm_bn(a);
   const int tiles0 = mt * ((rows + bn0 - 1) / bn0);

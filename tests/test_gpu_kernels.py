@@ -51,12 +51,13 @@ def test_gemm_bf16_split_k(N, M, K):
     assert_close(to64(y), O.store(to64(y0) + to64(x) @ to64(w).T, "bf16"), "bf16", "split-K gemm")
 
 
-@pytest.mark.parametrize("N,M,K,residual", [(512, 3072, 2048, 0), (512, 2048, 2048, 1), (300, 2048, 1024, 1),
-                                            (384, 1024, 2048, 0)])
+@pytest.mark.parametrize("N,M,K,residual", [(512, 256, 2048, 0), (300, 512, 1024, 1), (384, 384, 2048, 1),
+                                            (1000, 512, 2048, 0)])
 def test_gemm_bf16_wide_split_k(N, M, K, residual):
-    """A block's rows (a few hundred) against a dense projection: N tiles of 128 or 256 rows whose K slices run as
-    one cluster, every slice's accumulator staged in its operand ring and each rank reducing and storing its share
-    of the columns (ragged last N tile at 300 rows)."""
+    """A block's rows (hundreds) against a projection of at most four weight tiles (the router's logits): N tiles
+    of 128 rows (256 at 1000 rows) whose eight K slices run as one cluster, every slice's accumulator staged in its
+    operand ring and each rank reducing and storing its share of the columns (ragged last N tiles at 300 and 1000
+    rows)."""
     x = synth.normal((N, K), 1.0, 12, f"wx{N}{K}", DEV)
     w = synth.normal((M, K), 0.02, 12, f"ww{M}{K}", DEV)
     y0 = synth.normal((N, M), 1.0, 12, f"wy{N}{M}", DEV)

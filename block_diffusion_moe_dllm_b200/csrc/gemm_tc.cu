@@ -70,6 +70,7 @@ struct KParams {
   const int32_t* grp_cnt;
   const int32_t* cnt_dev;
   const int32_t* live;     // nullable: *live == 0 empties every group (a denoising pass with no masked position)
+  unsigned* zero_word;     // nullable: set to 0 by CTA 0 after the dependency wait (the next kernel's ticket)
   const float* w_scale;    // FP8 weights: per weight row of W / W2 (null otherwise)
   const float* w2_scale;
   EpiParams epi;
@@ -476,6 +477,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
   // everything above reads only the weights and on-chip state; the group counts below come from the kernels
   // before this one
   pdl_enter();
+  if (p.zero_word && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *p.zero_word = 0u;
   // ---- group table: counts, offsets and the exclusive prefix of tiles per group
   const bool dead = p.live && *p.live == 0;
   for (int g = tid; g < n_groups; g += NT) {
@@ -880,6 +882,7 @@ gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_con
   __syncthreads();
   cluster_sync();   // both CTAs' barriers exist before any cross-CTA arrive
   pdl_enter();
+  if (p.zero_word && blockIdx.x == 0 && threadIdx.x == 0) *p.zero_word = 0u;
   // ---- group table (tiles counted in m-tile pairs)
   const bool dead = p.live && *p.live == 0;
   for (int g = tid; g < n_groups; g += NUM_THREADS) {
@@ -1375,6 +1378,7 @@ int gemm_bf16_tc(const GemmArgs& a, cudaStream_t s) {
   kp.grp_cnt = a.grp_cnt;
   kp.cnt_dev = a.cnt_dev;
   kp.live = a.live;
+  kp.zero_word = a.zero_word;
   kp.w_scale = a.w_scale;
   kp.w2_scale = a.w2_scale;
   kp.epi = a.epi;

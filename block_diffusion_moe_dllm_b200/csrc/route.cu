@@ -26,8 +26,10 @@ DLLM_DEV void load8(const float* p, float* f) {
 template <typename T>
 __global__ void __launch_bounds__(256) route_scores_kernel(const T* __restrict__ h, const T* __restrict__ w, int Tk,
                                                            int H, int E, float* __restrict__ scores,
-                                                           const int32_t* __restrict__ live) {
+                                                           const int32_t* __restrict__ live,
+                                                           unsigned* __restrict__ zero_word) {
   pdl_enter();
+  if (zero_word && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *zero_word = 0u;   // the next kernel's ticket
   if (live && *live == 0) return;   // a pass with no masked position left does nothing
   extern __shared__ __align__(16) unsigned char hs_raw[];
   T* hs = reinterpret_cast<T*>(hs_raw);  // [TT][H]
@@ -868,34 +870,32 @@ __global__ void __launch_bounds__(256) route_seg_scatter_kernel(const int32_t* _
 // index a = t k + j, as in the other permutation kernels.
 constexpr int kPermCtaMax = 8192;
 
-__global__ void __launch_bounds__(1024) route_perm_cta_kernel(const int32_t* __restrict__ ids, int Tk, int E, int k,
-                                                              int32_t* __restrict__ counts,
-                                                              int32_t* __restrict__ offsets,
-                                                              int32_t* __restrict__ perm, int32_t* __restrict__ inv,
-                                                              const int32_t* __restrict__ live) {
-  pdl_enter();
-  if (live && *live == 0) return;   // a pass with no masked position left does nothing
-  extern __shared__ int wh[];        // [32][E]
-  __shared__ int wtot[32];
+// The stable permutation of n assignments by one CTA of NW warps (E <= 32 NW): counts, offsets and each
+// assignment's position. Warp w takes the assignments [w per, (w + 1) per) (per a multiple of 32); pass 1 counts
+// them per expert (__match_any_sync groups), the warps' counts are prefixed per expert on top of the expert's
+// offset, and pass 2 writes position = warp's running base + rank among the chunk's lanes with the same expert.
+// wh: NW x E ints of shared memory, wtot: 32 ints.
+template <int NW>
+DLLM_DEV void cta_permutation(const int32_t* __restrict__ ids, int n, int E, int32_t* __restrict__ counts,
+                              int32_t* __restrict__ offsets, int32_t* __restrict__ perm, int32_t* __restrict__ inv,
+                              int* wh, int* wtot) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  for (int i = tid; i < 32 * E; i += blockDim.x) wh[i] = 0;
+  for (int i = tid; i < NW * E; i += NW * 32) wh[i] = 0;
   __syncthreads();
-  const int n = Tk * k;
-  const int per = ((n + 31) / 32 + 31) & ~31;
+  const int per = ((n + NW - 1) / NW + 31) & ~31;
   const int a0 = min(n, warp * per), a1 = min(n, a0 + per);
   for (int c = a0; c < a1; c += 32) {
     const int a = c + lane;
-    const int ex = a < a1 ? ids[a] : -1;
+    const int ex = a < a1 ? __ldcg(ids + a) : -1;   // from L2: other CTAs of the launch may have written them
     const unsigned grp = __match_any_sync(0xffffffffu, ex);
     if (a < a1 && lane == __ffs(grp) - 1) wh[warp * E + ex] += __popc(grp);
   }
   __syncthreads();
-  // per expert (one thread each, E <= 1024): prefix over the warps, total count, then the exclusive scan of the
-  // totals over experts
+  // per expert (one thread each): prefix over the warps, total count, then the exclusive scan of the totals
   int cnt = 0;
   if (tid < E) {
 #pragma unroll 8
-    for (int q = 0; q < 32; ++q) {
+    for (int q = 0; q < NW; ++q) {
       const int v = wh[q * E + tid];
       wh[q * E + tid] = cnt;
       cnt += v;
@@ -910,7 +910,7 @@ __global__ void __launch_bounds__(1024) route_perm_cta_kernel(const int32_t* __r
   if (lane == 31) wtot[warp] = inc;
   __syncthreads();
   if (warp == 0) {
-    int x = wtot[lane];
+    int x = lane < NW ? wtot[lane] : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int y = __shfl_up_sync(0xffffffffu, x, o);
@@ -924,13 +924,13 @@ __global__ void __launch_bounds__(1024) route_perm_cta_kernel(const int32_t* __r
     counts[tid] = cnt;
     offsets[tid] = excl;
 #pragma unroll 8
-    for (int q = 0; q < 32; ++q) wh[q * E + tid] += excl;
+    for (int q = 0; q < NW; ++q) wh[q * E + tid] += excl;
   }
   if (tid == 0) offsets[E] = n;
   __syncthreads();
   for (int c = a0; c < a1; c += 32) {
     const int a = c + lane;
-    const int ex = a < a1 ? ids[a] : -1;
+    const int ex = a < a1 ? __ldcg(ids + a) : -1;
     const unsigned grp = __match_any_sync(0xffffffffu, ex);
     if (a < a1) {
       const int pos = wh[warp * E + ex] + __popc(grp & ((1u << lane) - 1u));
@@ -943,13 +943,81 @@ __global__ void __launch_bounds__(1024) route_perm_cta_kernel(const int32_t* __r
   }
 }
 
+// Mid-size routing (Tk * k <= kPermCtaMax) when the fused decode kernel does not apply: after route_topk_kernel
+// (and the exact re-decisions), one CTA of 1024 threads builds counts, offsets and the stable permutation, in place
+// of the segmented three launches.
+__global__ void __launch_bounds__(1024) route_perm_cta_kernel(const int32_t* __restrict__ ids, int Tk, int E, int k,
+                                                              int32_t* __restrict__ counts,
+                                                              int32_t* __restrict__ offsets,
+                                                              int32_t* __restrict__ perm, int32_t* __restrict__ inv,
+                                                              const int32_t* __restrict__ live) {
+  pdl_enter();
+  if (live && *live == 0) return;   // a pass with no masked position left does nothing
+  extern __shared__ int wh[];        // [32][E]
+  __shared__ int wtot[32];
+  cta_permutation<32>(ids, Tk * k, E, counts, offsets, perm, inv, wh, wtot);
+}
+
+// Decode-sized routing (E <= 256, Tk * k <= kPermCtaMax) in one launch after the logits: a warp per token takes the
+// fp32 top-k (warp_topk) and, for a near-tie, decides it again exactly in place (warp_exact_select); the last CTA to
+// finish (a ticket counter, zeroed before the first launch and by that CTA after use) builds the permutation from
+// every CTA's ids (the threadfence / ticket pattern makes them visible to it).
+template <int PER, typename T>
+__global__ void __launch_bounds__(256, 1) route_decode_kernel(float* __restrict__ scores,
+                                                              const float* __restrict__ bias, int Tk, int E, int k,
+                                                              int from_logits, const T* __restrict__ h,
+                                                              const T* __restrict__ w, int H,
+                                                              int32_t* __restrict__ ids, float* __restrict__ gates,
+                                                              int32_t* __restrict__ counts,
+                                                              int32_t* __restrict__ offsets,
+                                                              int32_t* __restrict__ perm, int32_t* __restrict__ inv,
+                                                              unsigned* __restrict__ ticket,
+                                                              const int32_t* __restrict__ live) {
+  pdl_enter();
+  if (live && *live == 0) return;   // a pass with no masked position left does nothing
+  __shared__ int wh[8 * 256];
+  __shared__ int wtot[32];
+  __shared__ bool last;
+  const int lane = threadIdx.x & 31;
+  for (int t = blockIdx.x * 8 + (threadIdx.x >> 5); t < Tk; t += gridDim.x * 8) {
+    int my_id;
+    float my_gate, thr;
+    float* srow = scores + (int64_t)t * E;
+    if (warp_topk<PER>(srow, bias, E, k, from_logits, lane, my_id, my_gate, thr)) {
+      __syncwarp();   // this warp's write-back of the sigmoid scores is visible to all its lanes
+      int eid = my_id;
+      float egate = my_gate;
+      if (warp_exact_select<T>(srow, bias, E, k, h + (int64_t)t * H, w, H, thr, lane, eid, egate)) {
+        my_id = eid;
+        my_gate = egate;
+      }
+    }
+    if (lane < k) {
+      ids[(int64_t)t * k + lane] = my_id;
+      gates[(int64_t)t * k + lane] = my_gate;
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    last = atomicAdd(ticket, 1u) == gridDim.x - 1;
+  }
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  cta_permutation<8>(ids, Tk * k, E, counts, offsets, perm, inv, wh, wtot);
+  if (threadIdx.x == 0) *ticket = 0u;   // ready for the next launch
+}
+
 }  // namespace
 
-// Layout of the router scratch: per-segment expert histograms, then one fp32 near-tie threshold per token.
+// Layout of the router scratch: per-segment expert histograms, one fp32 near-tie threshold per token, and the
+// ticket counter of route_decode_kernel.
 struct RouteScratch {
   int seg_tok, S;
   int32_t* seg_hist;
   float* fix_thr;
+  unsigned* ticket;
 };
 
 RouteScratch route_scratch(int Tk, int E, int k, void* base) {
@@ -957,8 +1025,10 @@ RouteScratch route_scratch(int Tk, int E, int k, void* base) {
   r.seg_tok = route_segment_tokens(Tk, k);
   r.S = std::max(1, (Tk + r.seg_tok - 1) / r.seg_tok);
   const size_t hist = ((size_t)r.S * E * sizeof(int32_t) + 255) & ~size_t(255);
+  const size_t thr = ((size_t)std::max(Tk, 1) * sizeof(float) + 255) & ~size_t(255);
   r.seg_hist = static_cast<int32_t*>(base);
   r.fix_thr = base ? reinterpret_cast<float*>(static_cast<char*>(base) + hist) : nullptr;
+  r.ticket = base ? reinterpret_cast<unsigned*>(static_cast<char*>(base) + hist + thr) : nullptr;
   return r;
 }
 
@@ -982,6 +1052,14 @@ int launch_select_per(float* scores, const float* bias, int Tk, int E, int k, in
     }
   }
   const RouteScratch rs = route_scratch(Tk, E, k, scratch);
+  if constexpr (PER <= 8) {
+    if (Tk * k <= kPermCtaMax) {   // one launch: top-k, exact re-decisions and (last CTA) the permutation
+      launch_pdl(route_decode_kernel<PER, T>, std::min(num_sms(), (Tk + 7) / 8), 256, 0, s, scores, bias, Tk, E, k,
+                 from_logits, h, w, H, ids, gates, counts, offsets, perm, inv, rs.ticket, live);
+      DLLM_CHECK_LAUNCH("route_decode_kernel");
+      return DLLM_OK;
+    }
+  }
   // one warp per token, 4 per CTA: many tokens spread over all the SMs (one thread per token, tried for thousands
   // of tokens, reads each 1 KB score row with 32 lines in flight per warp instruction and was 2x slower)
   launch_pdl(route_topk_kernel<PER>, (Tk + 3) / 4, 128, 0, s, scores, bias, Tk, E, k, from_logits, ids, gates,
@@ -1044,7 +1122,8 @@ int route_segment_tokens(int Tk, int k) {
 size_t route_scratch_bytes(int Tk, int E, int k) {
   const RouteScratch r = route_scratch(Tk, E, k, nullptr);
   const size_t hist = ((size_t)r.S * E * sizeof(int32_t) + 255) & ~size_t(255);
-  return hist + (size_t)std::max(Tk, 1) * sizeof(float);
+  const size_t thr = ((size_t)std::max(Tk, 1) * sizeof(float) + 255) & ~size_t(255);
+  return hist + thr + 256;
 }
 
 int launch_route(int dtype, const void* h, const void* w_router, const float* bias, int Tk, int H, int E, int k,
@@ -1059,6 +1138,7 @@ int launch_route(int dtype, const void* h, const void* w_router, const float* bi
     g.x = h; g.x_rows = Tk; g.w = w_router; g.w_rows = E; g.K = H; g.M = E; g.host_cnt = Tk; g.max_cnt = Tk;
     g.cnt_bound = Tk; g.dtype = DLLM_BF16; g.live = live;
     g.epi.kind = EPI_STORE; g.epi.out = scores; g.epi.ldo = E; g.epi.out_f32 = 1;
+    g.zero_word = route_scratch(Tk, E, k, seg_scratch).ticket;   // route_decode_kernel's ticket
     int st = gemm_bf16_tc(g, s);
     if (st) return st;
     return launch_select(scores, bias, Tk, E, k, 1, (const __nv_bfloat16*)h, (const __nv_bfloat16*)w_router, H, ids,
@@ -1074,14 +1154,15 @@ int launch_route(int dtype, const void* h, const void* w_router, const float* bi
       cfg = true;
     }
     launch_pdl(route_scores_kernel<__nv_bfloat16>, g1, 256, smem, s, (const __nv_bfloat16*)h,
-                                                             (const __nv_bfloat16*)w_router, Tk, H, E, scores, live);
+               (const __nv_bfloat16*)w_router, Tk, H, E, scores, live, route_scratch(Tk, E, k, seg_scratch).ticket);
   } else {
     static bool cfg = false;
     if (!cfg) {
       cudaFuncSetAttribute(route_scores_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
       cfg = true;
     }
-    launch_pdl(route_scores_kernel<float>, g1, 256, smem, s, (const float*)h, (const float*)w_router, Tk, H, E, scores, live);
+    launch_pdl(route_scores_kernel<float>, g1, 256, smem, s, (const float*)h, (const float*)w_router, Tk, H, E, scores,
+               live, route_scratch(Tk, E, k, seg_scratch).ticket);
   }
   DLLM_CHECK_LAUNCH("route_scores_kernel");
   if (dtype == DLLM_BF16)

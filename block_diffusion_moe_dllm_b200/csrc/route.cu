@@ -879,16 +879,26 @@ template <int NW>
 DLLM_DEV void cta_permutation(const int32_t* __restrict__ ids, int n, int E, int32_t* __restrict__ counts,
                               int32_t* __restrict__ offsets, int32_t* __restrict__ perm, int32_t* __restrict__ inv,
                               int* wh, int* wtot) {
+  // every chunk of this warp's assignments is loaded once, up front (n <= kPermCtaMax): the two passes below then
+  // run on registers instead of one dependent trip to L2 per chunk
+  constexpr int MAXC = (kPermCtaMax + NW * 32 - 1) / (NW * 32);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   for (int i = tid; i < NW * E; i += NW * 32) wh[i] = 0;
-  __syncthreads();
   const int per = ((n + NW - 1) / NW + 31) & ~31;
   const int a0 = min(n, warp * per), a1 = min(n, a0 + per);
-  for (int c = a0; c < a1; c += 32) {
-    const int a = c + lane;
-    const int ex = a < a1 ? __ldcg(ids + a) : -1;   // from L2: other CTAs of the launch may have written them
-    const unsigned grp = __match_any_sync(0xffffffffu, ex);
-    if (a < a1 && lane == __ffs(grp) - 1) wh[warp * E + ex] += __popc(grp);
+  int ex[MAXC];
+#pragma unroll
+  for (int c = 0; c < MAXC; ++c) {
+    const int a = a0 + c * 32 + lane;
+    ex[c] = a < a1 ? __ldcg(ids + a) : -1;   // from L2: other CTAs of the launch may have written them
+  }
+  __syncthreads();
+#pragma unroll
+  for (int c = 0; c < MAXC; ++c) {
+    if (a0 + c * 32 >= a1) break;
+    const int a = a0 + c * 32 + lane;
+    const unsigned grp = __match_any_sync(0xffffffffu, ex[c]);
+    if (a < a1 && lane == __ffs(grp) - 1) wh[warp * E + ex[c]] += __popc(grp);
   }
   __syncthreads();
   // per expert (one thread each): prefix over the warps, total count, then the exclusive scan of the totals
@@ -928,17 +938,18 @@ DLLM_DEV void cta_permutation(const int32_t* __restrict__ ids, int n, int E, int
   }
   if (tid == 0) offsets[E] = n;
   __syncthreads();
-  for (int c = a0; c < a1; c += 32) {
-    const int a = c + lane;
-    const int ex = a < a1 ? __ldcg(ids + a) : -1;
-    const unsigned grp = __match_any_sync(0xffffffffu, ex);
+#pragma unroll
+  for (int c = 0; c < MAXC; ++c) {
+    if (a0 + c * 32 >= a1) break;
+    const int a = a0 + c * 32 + lane;
+    const unsigned grp = __match_any_sync(0xffffffffu, ex[c]);
     if (a < a1) {
-      const int pos = wh[warp * E + ex] + __popc(grp & ((1u << lane) - 1u));
+      const int pos = wh[warp * E + ex[c]] + __popc(grp & ((1u << lane) - 1u));
       perm[pos] = a;
       inv[a] = pos;
     }
     __syncwarp();
-    if (a < a1 && lane == __ffs(grp) - 1) wh[warp * E + ex] += __popc(grp);
+    if (a < a1 && lane == __ffs(grp) - 1) wh[warp * E + ex[c]] += __popc(grp);
     __syncwarp();
   }
 }

@@ -820,13 +820,13 @@ int dllm_block_graph_skips_finished_passes(const dllm_block_graph* g) { return g
 
 namespace {
 // Conditional (IF) nodes through the driver API, with the context given explicitly (the node, its handle and the
-// kernels of its body must share one context: the current one). The entry points are requested at the ABI of CUDA
-// 12.3, where cuGraphAddNode takes per-edge data (left null here): the default query returns that version under a
-// 12.x runtime, and calling it with the older five-argument signature is what made the driver refuse the node.
+// kernels of its body must share one context: the current one). cuGraphAddNode is requested at the ABI of CUDA 12.2
+// (no per-edge data): measured on driver 13.0, that entry point adds the IF node, while the 12.3 one with per-edge
+// data (null here) refuses it with CUDA_ERROR_INVALID_VALUE, and so did the default query, which returns the 12.3
+// one under a 12.x runtime.
 typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
 typedef CUresult (*CondHandleCreateFn)(CUgraphConditionalHandle*, CUgraph, CUcontext, unsigned int, unsigned int);
-typedef CUresult (*GraphAddNodeFn)(CUgraphNode*, CUgraph, const CUgraphNode*, const CUgraphEdgeData*, size_t,
-                                   CUgraphNodeParams*);
+typedef CUresult (*GraphAddNodeFn)(CUgraphNode*, CUgraph, const CUgraphNode*, size_t, CUgraphNodeParams*);
 
 struct CondApi {
   CtxGetCurrentFn ctx_get = nullptr;
@@ -838,17 +838,17 @@ const CondApi& cond_api() {
   static CondApi api;
   static std::once_flag once;
   std::call_once(once, [] {
-    auto get = [](const char* name) -> void* {
+    auto get = [](const char* name, unsigned version) -> void* {
       void* p = nullptr;
       cudaDriverEntryPointQueryResult q;
-      if (cudaGetDriverEntryPointByVersion(name, &p, 12030, cudaEnableDefault, &q) != cudaSuccess ||
+      if (cudaGetDriverEntryPointByVersion(name, &p, version, cudaEnableDefault, &q) != cudaSuccess ||
           q != cudaDriverEntryPointSuccess)
         return nullptr;
       return p;
     };
-    api.ctx_get = reinterpret_cast<CtxGetCurrentFn>(get("cuCtxGetCurrent"));
-    api.handle_create = reinterpret_cast<CondHandleCreateFn>(get("cuGraphConditionalHandleCreate"));
-    api.add_node = reinterpret_cast<GraphAddNodeFn>(get("cuGraphAddNode"));
+    api.ctx_get = reinterpret_cast<CtxGetCurrentFn>(get("cuCtxGetCurrent", 12030));
+    api.handle_create = reinterpret_cast<CondHandleCreateFn>(get("cuGraphConditionalHandleCreate", 12030));
+    api.add_node = reinterpret_cast<GraphAddNodeFn>(get("cuGraphAddNode", 12020));
   });
   return api;
 }
@@ -870,8 +870,7 @@ bool add_if_node(cudaGraph_t graph, cudaGraphConditionalHandle cond, CUcontext c
   np.conditional.ctx = ctx;
   CUgraphNode n = nullptr;
   CUgraphNode dep = reinterpret_cast<CUgraphNode>(prev);
-  const CUresult rc =
-      api.add_node(&n, reinterpret_cast<CUgraph>(graph), prev ? &dep : nullptr, nullptr, prev ? 1 : 0, &np);
+  const CUresult rc = api.add_node(&n, reinterpret_cast<CUgraph>(graph), prev ? &dep : nullptr, prev ? 1 : 0, &np);
   if (rc != CUDA_SUCCESS) {
     snprintf(g_cond_note, sizeof(g_cond_note), "conditional node refused: cuGraphAddNode returned %d", (int)rc);
     return false;

@@ -917,37 +917,32 @@ int dllm_block_graph_create(const dllm_model* m, const dllm_state* st, const dll
   if (e != cudaSuccess) return fail(e, "block_graph_create: cudaGraphCreate");
   // conditional passes when the driver offers them (the handle and the nodes on the current context); otherwise
   // the passes follow one another unconditionally and those after an early finish return at entry
+  // A conditional handle serves one node (measured on driver 13.0: a second IF node on the handle of the first is
+  // refused with CUDA_ERROR_INVALID_VALUE, one on a handle of its own is added), so pass t has handle t. Every
+  // handle is reset at each launch of the graph: handle 0 to 1 (the first pass always runs), the others to 0; the
+  // unmask selection of pass t sets handle t + 1 to (masked positions left > 0), so a pass that is skipped leaves
+  // every later one skipped too.
   const CondApi& api = cond_api();
   CUcontext ctx = nullptr;
-  cudaGraphConditionalHandle cond = 0;
+  std::vector<cudaGraphConditionalHandle> conds(p->T_s, cudaGraphConditionalHandle());
   bool use_cond = false;
   g_cond_note[0] = 0;
   if (!(api.ctx_get && api.handle_create && api.add_node)) {
     snprintf(g_cond_note, sizeof(g_cond_note), "conditional nodes: driver entry points unavailable");
   } else {
     const CUresult rc0 = api.ctx_get(&ctx);
-    const CUresult rc1 = (rc0 == CUDA_SUCCESS && ctx)
-                             ? api.handle_create(reinterpret_cast<CUgraphConditionalHandle*>(&cond),
-                                                 reinterpret_cast<CUgraph>(g->graph), ctx, 1,
-                                                 CU_GRAPH_COND_ASSIGN_DEFAULT)
-                             : CUDA_ERROR_INVALID_CONTEXT;
+    CUresult rc1 = (rc0 == CUDA_SUCCESS && ctx) ? CUDA_SUCCESS : CUDA_ERROR_INVALID_CONTEXT;
+    for (int t = 0; t < p->T_s && rc1 == CUDA_SUCCESS; ++t)
+      rc1 = api.handle_create(reinterpret_cast<CUgraphConditionalHandle*>(&conds[t]),
+                              reinterpret_cast<CUgraph>(g->graph), ctx, t == 0 ? 1u : 0u,
+                              CU_GRAPH_COND_ASSIGN_DEFAULT);
     use_cond = rc1 == CUDA_SUCCESS;
     if (!use_cond)
       snprintf(g_cond_note, sizeof(g_cond_note), "conditional handle refused: cuCtxGetCurrent %d, handle %d",
                (int)rc0, (int)rc1);
   }
-  cudaGraphNode_t first = nullptr;
-  cudaGraph_t first_body = nullptr;
-  if (use_cond && !add_if_node(g->graph, cond, ctx, nullptr, &first, &first_body)) {
-    // the conditional node was refused: a fresh graph without conditions (the handle stays unused)
-    use_cond = false;
-    cudaGraphDestroy(g->graph);
-    g->graph = nullptr;
-    e = cudaGraphCreate(&g->graph, 0);
-    if (e != cudaSuccess) return fail(e, "block_graph_create: cudaGraphCreate");
-  }
   auto capture_pass = [&](cudaGraph_t target, const cudaGraphNode_t* deps, size_t n_deps, int t, int commit,
-                          bool set_cond) -> int {
+                          cudaGraphConditionalHandle next, bool set_next) -> int {
     cudaError_t ce = cudaStreamBeginCaptureToGraph(capture_stream, target, deps, nullptr, n_deps,
                                                    cudaStreamCaptureModeThreadLocal);
     if (ce != cudaSuccess) return dllm_host::cuda_status(ce, "block_graph_create: cudaStreamBeginCaptureToGraph");
@@ -955,7 +950,7 @@ int dllm_block_graph_create(const dllm_model* m, const dllm_state* st, const dll
     q.t = commit ? 0 : t;
     q.commit = commit;
     q.retain = !commit && p->sprint && t == 0 ? 1 : 0;
-    int rr = denoise_step_impl(m, st, &q, ws, ws_bytes, capture_stream, cond, set_cond ? 1 : 0);
+    int rr = denoise_step_impl(m, st, &q, ws, ws_bytes, capture_stream, next, set_next ? 1 : 0);
     cudaGraph_t captured = nullptr;
     ce = cudaStreamEndCapture(capture_stream, &captured);
     if (rr) return rr;
@@ -963,19 +958,19 @@ int dllm_block_graph_create(const dllm_model* m, const dllm_state* st, const dll
     return DLLM_OK;
   };
   if (use_cond) {
-    cudaGraphNode_t prev = first;
-    r = capture_pass(first_body, nullptr, 0, 0, 0, true);
-    for (int t = 1; t < p->T_s && !r; ++t) {
+    cudaGraphNode_t prev = nullptr;
+    for (int t = 0; t < p->T_s && !r; ++t) {
       cudaGraphNode_t node = nullptr;
       cudaGraph_t body = nullptr;
-      if (!add_if_node(g->graph, cond, ctx, prev, &node, &body)) {
+      if (!add_if_node(g->graph, conds[t], ctx, prev, &node, &body)) {
         r = DLLM_ERR_CUDA;
         break;
       }
-      r = capture_pass(body, nullptr, 0, t, 0, true);
+      const bool last = t + 1 == p->T_s;
+      r = capture_pass(body, nullptr, 0, t, 0, last ? cudaGraphConditionalHandle() : conds[t + 1], !last);
       prev = node;
     }
-    if (!r) r = capture_pass(g->graph, &prev, 1, 0, 1, false);
+    if (!r) r = capture_pass(g->graph, &prev, 1, 0, 1, cudaGraphConditionalHandle(), false);
     if (!r) {
       e = cudaGraphInstantiate(&g->exec, g->graph, 0);
       if (e != cudaSuccess) {

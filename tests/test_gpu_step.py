@@ -460,6 +460,7 @@ def test_block_graph_matches_host_driven_block(early):
     want = _snapshot(eng, caches)
     want_sel = (eng.sel.clone(), eng.nsel.clone(), eng.remaining.clone())
     g = eng.block_graph()
+    assert g.conditional, g.note
     for _ in range(2):
         for (k, v), (k0, v0) in zip(caches, caches0):
             k.copy_(k0)

@@ -37,6 +37,8 @@ using namespace dllm;
 namespace {
 
 constexpr size_t kStatusBytes = 256;
+// words of the status block past the status word: the expert GEMMs' work counters (own 64-byte lines)
+constexpr int kWorkCtr1 = 16, kWorkCtr2 = 32;
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 inline int esize(int dtype) { return dtype == DLLM_BF16 ? 2 : 4; }
@@ -126,7 +128,10 @@ int run_experts(int dtype, int Tk, int H, int E, int k, int I, const void* h, co
   const int shared = w_gu_s != nullptr;
   const int n_assign = Tk * k;
   const int64_t rows = (int64_t)n_assign + (shared ? Tk : 0);
-  int st = launch_gather_rows(dtype, h, perm, k, Tk, shared, b.xp, H, s, live);
+  // the two GEMMs' work counters sit in the workspace's status block (the status word is its first word)
+  unsigned* ctr1 = reinterpret_cast<unsigned*>(status) + kWorkCtr1;
+  unsigned* ctr2 = reinterpret_cast<unsigned*>(status) + kWorkCtr2;
+  int st = launch_gather_rows(dtype, h, perm, k, Tk, shared, b.xp, H, s, live, ctr1, ctr2);
   if (st) return st;
   GemmArgs g1;
   g1.x = b.xp; g1.x_rows = rows;
@@ -136,7 +141,7 @@ int run_experts(int dtype, int Tk, int H, int E, int k, int I, const void* h, co
   g1.n_dev = E; g1.grp_off = offsets; g1.grp_cnt = counts;
   g1.has_extra = shared; g1.extra_off = n_assign; g1.extra_cnt = Tk;
   g1.max_cnt = expert_bn_hint(Tk, k, E); g1.cnt_bound = Tk;
-  g1.dtype = dtype; g1.status = status; g1.f32_scratch = b.scratch; g1.live = live;
+  g1.dtype = dtype; g1.status = status; g1.f32_scratch = b.scratch; g1.live = live; g1.work_ctr = ctr1;
   g1.w_fp8 = fp8; g1.w_scale = sc.gu; g1.w2_scale = sc.gu_shared;
   g1.epi.kind = EPI_SWIGLU; g1.epi.out = b.act; g1.epi.ldo = I;
   st = run_gemm(g1, s);
@@ -144,7 +149,7 @@ int run_experts(int dtype, int Tk, int H, int E, int k, int I, const void* h, co
   GemmArgs g2 = g1;
   g2.x = b.act; g2.K = I; g2.M = H; g2.swiglu = 0;
   g2.w = w_down; g2.w_rows = (int64_t)E * H; g2.w2 = w_down_s; g2.w2_rows = H; g2.w_group_stride = H;
-  g2.w_scale = sc.down; g2.w2_scale = sc.down_shared;
+  g2.w_scale = sc.down; g2.w2_scale = sc.down_shared; g2.work_ctr = ctr2;
   g2.epi = EpiParams();
   g2.epi.kind = EPI_STORE; g2.epi.out = b.y; g2.epi.ldo = H; g2.epi.out_f32 = 1;
   st = run_gemm(g2, s);

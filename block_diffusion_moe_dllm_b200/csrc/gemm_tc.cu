@@ -33,6 +33,7 @@ constexpr int STAGE_COLS = 32;         // epilogue column chunk
 constexpr int STAGING_BYTES = 128 * STAGE_COLS * 4;
 constexpr int MAX_GROUPS = 1040;
 constexpr int NUM_THREADS = 192;
+constexpr int NUM_THREADS_SPLIT = 224;   // bf16 weights in a ring of their own: warp 6 loads the activations
 constexpr int NUM_THREADS_F8 = 480;    // FP8 weights: two groups of four warps convert alternate E4M3 tiles, one
                                        // more warp loads the activation tiles
 constexpr int F8_KS = 2;               // FP8 weights: 64-wide K blocks per stage (one 128-byte row of codes)
@@ -48,7 +49,10 @@ struct Smem {
   uint64_t bempty[8];               // FP8: activation stage read by the MMAs (MMA commit)
   uint64_t tfull[2];
   uint64_t tempty[2];
+  uint64_t wq_full[4];              // dynamic schedule: work item published by the producer thread
+  uint64_t wq_empty[4];             // dynamic schedule: work item read by every other role
   uint64_t done;
+  int wq_item[4];
   uint32_t tmem_base;
   int abort_flag;
   int drained;                      // CTA pairs: the leader saw every issued stage of both CTAs land
@@ -71,6 +75,7 @@ struct KParams {
   const int32_t* cnt_dev;
   const int32_t* live;     // nullable: *live == 0 empties every group (a denoising pass with no masked position)
   unsigned* zero_word;     // nullable: set to 0 by CTA 0 after the dependency wait (the next kernel's ticket)
+  unsigned* work_ctr;      // nullable: dynamic schedule (see work_produce); zero when the kernel starts
   const float* w_scale;    // FP8 weights: per weight row of W / W2 (null otherwise)
   const float* w2_scale;
   EpiParams epi;
@@ -124,6 +129,62 @@ __device__ __forceinline__ void decode_tile(const Smem& sm, int m_tiles, int t, 
   int nt = local - mt * ntl;
   n0 = nt * BN;
   nval = min(BN, sm.grp_cnt[g] - n0);
+}
+
+// Work items. Static schedule: CTA c takes items c, c + step, ... Dynamic schedule (grouped launches given a work
+// counter, zeroed by the kernel that gathers their rows): warp 0's producer thread takes the next item from the
+// counter when its operand ring has room for it, so a CTA that finished its tiles early takes more, and hands it to
+// the other roles through a ring of WQ entries in shared memory (full: published; empty: read by the MMA thread and
+// one lane of every other consuming warp). The tiles of one expert launch differ widely in cost: an expert with a
+// few rows streams its weight tile from HBM for them, a crowded one re-reads its weight tiles from L2 once per N
+// tile. Item -1 ends the loop; -2 means a wait gave up (the abort flag is set).
+constexpr int WQ = 4;
+
+__device__ __forceinline__ int work_produce(Smem& sm, const KParams& p, uint32_t q, int begin, int step, int total,
+                                            volatile int* abort_flag) {
+  if (!p.work_ctr) {
+    const int w = begin + (int)q * step;
+    return w < total ? w : -1;
+  }
+  const uint32_t s = q % WQ;
+  if (!wait_bar(&sm.wq_empty[s], ((q / WQ) & 1) ^ 1, abort_flag, p.status, ST_TIMEOUT_PRODUCER)) return -2;
+  const unsigned u = atomicAdd(p.work_ctr, 1u);
+  const int w = u < (unsigned)total ? (int)u : -1;
+  sm.wq_item[s] = w;
+  tc::mbar_arrive(&sm.wq_full[s]);   // release: the item is visible to the roles that wait on the barrier
+  return w;
+}
+
+// Consumer side: by one thread (warp_wide false) or by all lanes of a warp together (lane 0 waits, reads, arrives
+// for the warp and broadcasts the item).
+__device__ __forceinline__ int work_consume(Smem& sm, const KParams& p, uint32_t q, int begin, int step, int total,
+                                            volatile int* abort_flag, int code, bool warp_wide) {
+  if (!p.work_ctr) {
+    const int w = begin + (int)q * step;
+    return w < total ? w : -1;
+  }
+  const uint32_t s = q % WQ;
+  int w = -2;
+  if (!warp_wide || (threadIdx.x & 31) == 0) {
+    if (wait_bar(&sm.wq_full[s], (q / WQ) & 1, abort_flag, p.status, code)) {
+      w = *reinterpret_cast<volatile int*>(&sm.wq_item[s]);
+      tc::mbar_arrive(&sm.wq_empty[s]);
+    }
+  }
+  if (warp_wide) w = __shfl_sync(0xffffffffu, w, 0);
+  return w;
+}
+
+// Tile of work item wk (K slice ks of it in cluster split-K mode). The dynamic schedule starts with the extra
+// group (the shared expert: every token's row, the longest run of full tiles) so that it does not form the tail.
+__device__ __forceinline__ int work_tile(const Smem& sm, const KParams& p, int wk, int& ks) {
+  const int t = wk / p.ksplit;
+  ks = wk - t * p.ksplit;
+  if (p.work_ctr && p.has_extra) {
+    const int r = t + sm.tile_prefix[p.n_dev];
+    return r >= sm.total_tiles ? r - sm.total_tiles : r;
+  }
+  return t;
 }
 
 __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }
@@ -395,12 +456,17 @@ __device__ __forceinline__ float f8_row_scale(const KParams& p, int g, int mt, i
 }
 
 template <int BN, int STAGES, bool F8 = false, int BST = 1>
-__global__ void __launch_bounds__(F8 ? NUM_THREADS_F8 : NUM_THREADS, 1)
+__global__ void __launch_bounds__(F8 ? NUM_THREADS_F8 : (BST > 1 ? NUM_THREADS_SPLIT : NUM_THREADS), 1)
 gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_w2,
                const __grid_constant__ CUtensorMap tmap_x, const KParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  constexpr int NT = F8 ? NUM_THREADS_F8 : NUM_THREADS;
+  constexpr int NT = F8 ? NUM_THREADS_F8 : (BST > 1 ? NUM_THREADS_SPLIT : NUM_THREADS);
+  // separate rings of weight tiles and of activation tiles (always for FP8; for bf16 when BST > 1): the weight ring's
+  // depth alone then sets the weight bytes in flight, which bounds a CTA's share of HBM bandwidth when its tiles
+  // stream weights for a few rows each
+  constexpr bool SPLIT = F8 || BST > 1;
+  constexpr int XWARP = F8 ? 14 : 6;          // the activation producer's warp in split mode
   // a stage covers KS 64-wide K blocks: one for bf16 weights (a 128-byte row of 64 elements), two for FP8 (a
   // 128-byte row of 128 codes, so that each weight row read from HBM per stage is as long as in bf16)
   constexpr int KS = F8 ? F8_KS : 1;
@@ -416,14 +482,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
   constexpr int MS = F8 ? ((512 - 2 * BN) / SLOT_COLS < 16 ? (512 - 2 * BN) / SLOT_COLS : 16) : 0;
   constexpr int MSD = MS > 0 ? MS : 1;        // slot count as a divisor (the bf16 instantiations use no slots)
   constexpr int W_BYTES = F8 ? RAW_BYTES : A_BYTES;
-  constexpr int STAGE_BYTES = F8 ? W_BYTES : W_BYTES + B_BYTES;
+  constexpr int STAGE_BYTES = SPLIT ? W_BYTES : W_BYTES + B_BYTES;
   constexpr uint32_t W_TX = W_BYTES;                                      // weight bytes a stage's TMA brings
   constexpr uint32_t TMEM_COLS = F8 ? 512 : 2 * BN;
   static_assert(!F8 || 2 * BN + MS * SLOT_COLS <= 512, "FP8 A slots exceed the tensor memory");
-  static_assert(!F8 || BST <= 8, "FP8 activation ring");
+  static_assert(BST <= 8, "activation ring");
   uint8_t* stages = base;
-  uint8_t* bring = base + STAGES * STAGE_BYTES;                           // FP8 activation ring
-  float* staging = reinterpret_cast<float*>(bring + (F8 ? BST * B_BYTES : 0));
+  uint8_t* bring = base + STAGES * STAGE_BYTES;                           // split mode: activation ring
+  float* staging = reinterpret_cast<float*>(bring + (SPLIT ? BST * B_BYTES : 0));
   Smem& sm = *reinterpret_cast<Smem*>(reinterpret_cast<uint8_t*>(staging) + STAGING_BYTES);
 
   const int tid = threadIdx.x;
@@ -441,7 +507,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
       tc::mbar_init(&sm.conv[s], 128);   // the slot's 128 TMEM rows written
       tc::mbar_init(&sm.mempty[s], 1);   // the slot read by the MMAs
     }
-    if (F8)
+    if (SPLIT)
       for (int b = 0; b < BST; ++b) {
         tc::mbar_init(&sm.bfull[b], 1);
         tc::mbar_init(&sm.bempty[b], 1);
@@ -449,6 +515,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
     for (int b = 0; b < 2; ++b) {
       tc::mbar_init(&sm.tfull[b], 1);
       tc::mbar_init(&sm.tempty[b], 128);
+    }
+    for (int q = 0; q < WQ; ++q) {
+      tc::mbar_init(&sm.wq_full[q], 1);
+      // readers of an item: the MMA thread, the four epilogue warps, in split mode the activation producer thread
+      // and for FP8 the eight converter warps
+      tc::mbar_init(&sm.wq_empty[q], F8 ? 14 : (SPLIT ? 6 : 5));
     }
     tc::mbar_init(&sm.done, 1);
     tc::fence_mbar_init();
@@ -543,8 +615,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
       const uint64_t pol_x = tc::policy_evict_last();
       uint32_t it = 0;
       bool ok = true;
-      for (int wk = wk_begin; wk < total && ok; wk += wk_step) {
-        const int t = wk / p.ksplit, ks = wk - t * p.ksplit;
+      for (uint32_t q = 0; ok; ++q) {
+        const int wk = work_produce(sm, p, q, wk_begin, wk_step, total, abort_flag);
+        if (wk < 0) {
+          ok = wk == -1;
+          break;
+        }
+        int ks;
+        const int t = work_tile(sm, p, wk, ks);
         const int kb0 = ks * kblocks / p.ksplit, kb1 = (ks + 1) * kblocks / p.ksplit;
         int g, mt, n0, nval;
         decode_tile<BN>(sm, p.m_tiles, t, g, mt, n0, nval);
@@ -561,10 +639,10 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
           uint8_t* a = stages + s * STAGE_BYTES;
           uint8_t* b = a + W_BYTES;
           if (it < (uint32_t)npf) {   // weight stage already in flight: arrive with the activation bytes
-            if (F8) tc::mbar_arrive(&sm.full[s]);
+            if (SPLIT) tc::mbar_arrive(&sm.full[s]);
             else tc::mbar_arrive_expect_tx(&sm.full[s], bytes - W_TX);
           } else {
-            tc::mbar_arrive_expect_tx(&sm.full[s], F8 ? W_TX : bytes);
+            tc::mbar_arrive_expect_tx(&sm.full[s], SPLIT ? W_TX : bytes);
             if (p.swiglu) {
               tc::tma_load_2d(a, wm, kb * SBK, (int)(wrow + mt * 64), &sm.full[s], pol_w);
               tc::tma_load_2d(a + W_TX / 2, wm, kb * SBK, (int)(wrow + p.M + mt * 64), &sm.full[s], pol_w);
@@ -572,7 +650,7 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
               tc::tma_load_2d(a, wm, kb * SBK, (int)(wrow + mt * 128), &sm.full[s], pol_w);
             }
           }
-          if constexpr (!F8)
+          if constexpr (!SPLIT)
             for (int j = 0; j < nb; ++j)
               tc::tma_load_2d(b + j * XBOX_BYTES, &tmap_x, kb * SBK, xrow + j * XBOX_ROWS, &sm.full[s], pol_x);
         }
@@ -589,15 +667,21 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
         tc::mbar_wait(&sm.full[i], 0, 1u << 16);
       }
     }
-  } else if (F8 && warp == 14) {
-    // ------------------------------------------------------------------ FP8: activation producer
+  } else if (SPLIT && warp == XWARP) {
+    // ------------------------------------------------------------------ split mode: activation producer
     if (tc::elect_one()) {
       tc::prefetch_tmap(&tmap_x);
       const uint64_t pol_x = tc::policy_evict_last();
       uint32_t it = 0;
       bool ok = true;
-      for (int wk = wk_begin; wk < total && ok; wk += wk_step) {
-        const int t = wk / p.ksplit, ks = wk - t * p.ksplit;
+      for (uint32_t q = 0; ok; ++q) {
+        const int wk = work_consume(sm, p, q, wk_begin, wk_step, total, abort_flag, ST_TIMEOUT_PRODUCER, false);
+        if (wk < 0) {
+          ok = wk == -1;
+          break;
+        }
+        int ks;
+        const int t = work_tile(sm, p, wk, ks);
         const int kb0 = ks * kblocks / p.ksplit, kb1 = (ks + 1) * kblocks / p.ksplit;
         int g, mt, n0, nval;
         decode_tile<BN>(sm, p.m_tiles, t, g, mt, n0, nval);
@@ -629,8 +713,14 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
     if (tc::elect_one()) {
       uint32_t it = 0, tcount = 0;
       bool ok = true;
-      for (int wk = wk_begin; wk < total && ok; wk += wk_step, ++tcount) {
-        const int t = wk / p.ksplit, ks = wk - t * p.ksplit;
+      for (uint32_t q = 0; ok; ++q, ++tcount) {
+        const int wk = work_consume(sm, p, q, wk_begin, wk_step, total, abort_flag, ST_TIMEOUT_MMA, false);
+        if (wk < 0) {
+          ok = wk == -1;
+          break;
+        }
+        int ks;
+        const int t = work_tile(sm, p, wk, ks);
         const int kb0 = ks * kblocks / p.ksplit, kb1 = (ks + 1) * kblocks / p.ksplit;
         int g, mt, n0, nval;
         decode_tile<BN>(sm, p.m_tiles, t, g, mt, n0, nval);
@@ -656,16 +746,21 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
             tc::mma_commit(&sm.mempty[ms]);
             tc::mma_commit(&sm.bempty[bb]);
           } else {
-            const int s = it % STAGES;
+            const int s = it % STAGES, bb = it % BST;
             const uint32_t ph = (it / STAGES) & 1;
-            if (!wait_bar(&sm.full[s], ph, abort_flag, p.status, ST_TIMEOUT_MMA)) { ok = false; break; }
+            if (!wait_bar(&sm.full[s], ph, abort_flag, p.status, ST_TIMEOUT_MMA) ||
+                (SPLIT && !wait_bar(&sm.bfull[bb], (it / BST) & 1, abort_flag, p.status, ST_TIMEOUT_MMA))) {
+              ok = false;
+              break;
+            }
             const uint32_t a = tc::smem_u32(stages + s * STAGE_BYTES);
-            const uint32_t b = a + W_BYTES;
+            const uint32_t b = SPLIT ? tc::smem_u32(bring + bb * B_BYTES) : a + W_BYTES;
             tc::fence_after_sync();
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk)
               tc::mma_bf16(d, tc::sdesc_k128(a + kk * 32), tc::sdesc_k128(b + kk * 32), idesc, (kb != kb0) || kk != 0);
             tc::mma_commit(&sm.empty[s]);
+            if (SPLIT) tc::mma_commit(&sm.bempty[bb]);
           }
         }
         if (!ok) break;
@@ -686,8 +781,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
     const uint32_t cg = (uint32_t)(warp - 6) >> 2;
     uint32_t it = 0;
     bool ok = true;
-    for (int wk = wk_begin; wk < total && ok; wk += wk_step) {
-      const int ks = wk - (wk / p.ksplit) * p.ksplit;
+    for (uint32_t qi = 0; ok; ++qi) {
+      const int wk = work_consume(sm, p, qi, wk_begin, wk_step, total, abort_flag, ST_TIMEOUT_MMA, true);
+      if (wk < 0) break;
+      int ks;
+      (void)work_tile(sm, p, wk, ks);
       const int kb0 = ks * kblocks / p.ksplit, kb1 = (ks + 1) * kblocks / p.ksplit;
       for (int kb = kb0; kb < kb1; ++kb, ++it) {
         if ((it & 1u) != cg) continue;   // the other group's k-block
@@ -712,8 +810,11 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
 #pragma unroll
     for (int i = 0; i < 4; ++i) { run.m[i] = -INFINITY; run.idx[i] = 0x7fffffff; run.s[i] = 0.0; }
     uint32_t tcount = 0;
-    for (int wk = wk_begin; wk < total; wk += wk_step, ++tcount) {
-      const int t = wk / p.ksplit;
+    for (uint32_t qi = 0;; ++qi, ++tcount) {
+      const int wk = work_consume(sm, p, qi, wk_begin, wk_step, total, abort_flag, ST_TIMEOUT_EPILOGUE, true);
+      if (wk < 0) break;
+      int ks;
+      const int t = work_tile(sm, p, wk, ks);
       int g, mt, n0, nval;
       decode_tile<BN>(sm, p.m_tiles, t, g, mt, n0, nval);
       const uint32_t buf = tcount & 1, tph = (tcount >> 1) & 1;
@@ -1122,9 +1223,11 @@ int launch_cluster_splitk(const GemmArgs& a, const CUtensorMap& mw, const CUtens
 template <int BN, int STAGES, bool F8 = false, int BST = 1>
 int launch(const GemmArgs& a, const CUtensorMap& mw, const CUtensorMap& mw2, const CUtensorMap& mx,
            const KParams& kp, cudaStream_t s) {
-  // (matches the kernel's layout: bf16 stages of [weights][activations]; FP8 rings of codes and of activations)
+  // (matches the kernel's layout: bf16 stages of [weights][activations], or with BST > 1 a ring of weight tiles and
+  // one of activation tiles; FP8 rings of codes and of activations)
   constexpr int SMEM = F8 ? 1024 + STAGES * RAW_BYTES + BST * BN * BK * 2 * F8_KS + STAGING_BYTES + (int)sizeof(Smem)
-                          : 1024 + STAGES * (A_BYTES + BN * BK * 2) + STAGING_BYTES + (int)sizeof(Smem);
+                     : BST > 1 ? 1024 + STAGES * A_BYTES + BST * BN * BK * 2 + STAGING_BYTES + (int)sizeof(Smem)
+                               : 1024 + STAGES * (A_BYTES + BN * BK * 2) + STAGING_BYTES + (int)sizeof(Smem);
   static_assert(SMEM <= SMEM_LIMIT, "shared memory budget");
   // With programmatic dependent launch a CTA allocates tensor memory before it waits for the kernels ahead of it.
   // More than half an SM's shared memory per CTA keeps two tensor-memory kernels from sharing an SM, so a later
@@ -1137,8 +1240,8 @@ int launch(const GemmArgs& a, const CUtensorMap& mw, const CUtensorMap& mw2, con
     if (e != cudaSuccess) return dllm_host::cuda_status(e, "cudaFuncSetAttribute(gemm_tc)");
     configured = true;
   }
-  launch_pdl((gemm_tc_kernel<BN, STAGES, F8, BST>), num_sms(), F8 ? NUM_THREADS_F8 : NUM_THREADS, SMEM, s, mw, mw2,
-             mx, kp);
+  launch_pdl((gemm_tc_kernel<BN, STAGES, F8, BST>), num_sms(),
+             F8 ? NUM_THREADS_F8 : (BST > 1 ? NUM_THREADS_SPLIT : NUM_THREADS), SMEM, s, mw, mw2, mx, kp);
   DLLM_CHECK_LAUNCH("gemm_tc_kernel");
   return DLLM_OK;
 }
@@ -1390,6 +1493,9 @@ int gemm_bf16_tc(const GemmArgs& a, cudaStream_t s) {
     DLLM_REQUIRE(a.epi.conf_nparts > 0 && gemm_conf_parts(a) == a.epi.conf_nparts, DLLM_ERR_UNSUPPORTED,
                  "gemm: fused confidence epilogue unsupported for this shape");
   kp.ksplit = ks;
+  // grouped launches of single-CTA tiles take their tiles from the work counter (the CTA pair kernel keeps its
+  // static schedule)
+  kp.work_ctr = ((a.swiglu || a.n_dev || a.has_extra) && ks == 1) ? a.work_ctr : nullptr;
   kp.prefetch_w = (!a.swiglu && !a.n_dev && !a.has_extra && a.host_cnt <= (ks > 1 ? 32 : bn)) ? 1 : 0;
   int st2;
   if (f8) {   // single-CTA tiles, no split-K (the weight-streaming shapes FP8 weights serve)
@@ -1405,7 +1511,13 @@ int gemm_bf16_tc(const GemmArgs& a, cudaStream_t s) {
     st2 = wide.bn == 128 ? launch_wide_splitk<128, 6>(a, mw, mw2, mx, kp, s)
                          : launch_wide_splitk<256, 4>(a, mw, mw2, mx, kp, s);
   } else if (ks > 1) st2 = launch_cluster_splitk(a, mw, mw2, mx, kp, s);
-  else if (bn == 32) st2 = launch<32, 9>(a, mw, mw2, mx, kp, s);
+  else if (kp.work_ctr) {
+    // grouped (expert) launches: weight ring of its own, as deep as shared memory allows
+    if (bn == 32) st2 = launch<32, 11, false, 4>(a, mw, mw2, mx, kp, s);
+    else if (bn == 64) st2 = launch<64, 10, false, 4>(a, mw, mw2, mx, kp, s);
+    else if (bn == 128) st2 = launch<128, 9, false, 3>(a, mw, mw2, mx, kp, s);
+    else st2 = launch<256, 6, false, 2>(a, mw, mw2, mx, kp, s);
+  } else if (bn == 32) st2 = launch<32, 9>(a, mw, mw2, mx, kp, s);
   else if (bn == 64) st2 = launch<64, 8>(a, mw, mw2, mx, kp, s);
   else if (bn == 128) st2 = launch<128, 6>(a, mw, mw2, mx, kp, s);
   else st2 = launch<256, 4>(a, mw, mw2, mx, kp, s);

@@ -79,6 +79,7 @@ struct GemmArgs {
   int dtype = 0;           // DLLM_BF16 / DLLM_F32
   const int32_t* live = nullptr;  // nullable device word: 0 = the pass has nothing left to do (every group empty)
   unsigned* zero_word = nullptr;   // nullable device word the kernel sets to 0 once the kernels before it are done
+  unsigned* work_ctr = nullptr;    // grouped launches: nullable work counter, zero at launch (dynamic tile schedule)
   // FP8 weights: W and W2 hold E4M3 codes (one byte each, same row layout) and w_scale / w2_scale one fp32 scale per
   // weight row (w_scale indexed like the rows of W, w2_scale like those of W2); the output is scale[row] * (X q^T)
   int w_fp8 = 0;

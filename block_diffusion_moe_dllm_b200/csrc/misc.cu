@@ -169,8 +169,14 @@ int launch_masked_rows(const uint8_t* mask, int n_pos, int halves, int32_t* row_
 // Xp[r] = h[perm[r] / k] for r < Tk * k (assignments grouped by expert), Xp[Tk * k + t] = h[t] (shared expert).
 template <typename T>
 __global__ void gather_rows_kernel(const T* __restrict__ h, const int32_t* __restrict__ perm, int k, int n_assign,
-                                   int shared, T* __restrict__ xp, int H, const int32_t* __restrict__ live) {
+                                   int shared, T* __restrict__ xp, int H, const int32_t* __restrict__ live,
+                                   unsigned* __restrict__ ctr_a, unsigned* __restrict__ ctr_b) {
   pdl_enter();
+  // the work counters of the two expert GEMMs that follow (every kernel before this one is done with them)
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    if (ctr_a) *ctr_a = 0u;
+    if (ctr_b) *ctr_b = 0u;
+  }
   if (live && *live == 0) return;   // a pass with no masked position left does nothing
   const int r = blockIdx.x;
   int src;
@@ -184,14 +190,15 @@ __global__ void gather_rows_kernel(const T* __restrict__ h, const int32_t* __res
 }
 
 int launch_gather_rows(int dtype, const void* h, const int32_t* perm, int k, int Tk, int shared, void* xp, int H,
-                       cudaStream_t s, const int32_t* live) {
+                       cudaStream_t s, const int32_t* live, unsigned* ctr_a, unsigned* ctr_b) {
   const int rows = Tk * k + (shared ? Tk : 0);
   if (rows <= 0) return DLLM_OK;
   if (dtype == DLLM_BF16)
     launch_pdl(gather_rows_kernel<__nv_bfloat16>, rows, 128, 0, s, (const __nv_bfloat16*)h, perm, k, Tk * k, shared,
-                                                           (__nv_bfloat16*)xp, H, live);
+               (__nv_bfloat16*)xp, H, live, ctr_a, ctr_b);
   else
-    launch_pdl(gather_rows_kernel<float>, rows, 128, 0, s, (const float*)h, perm, k, Tk * k, shared, (float*)xp, H, live);
+    launch_pdl(gather_rows_kernel<float>, rows, 128, 0, s, (const float*)h, perm, k, Tk * k, shared, (float*)xp, H,
+               live, ctr_a, ctr_b);
   DLLM_CHECK_LAUNCH("gather_rows_kernel");
   return DLLM_OK;
 }

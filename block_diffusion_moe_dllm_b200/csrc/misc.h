@@ -14,8 +14,11 @@ int launch_masked_rows(const uint8_t* mask, int n_pos, int halves, int32_t* row_
                        cudaStream_t s);
 // live (nullable, every launcher below that takes it): device word; 0 = the denoising pass has no masked position
 // left, and the kernel returns at once
+// ctr_a, ctr_b (nullable): device words set to 0 once the kernels before the gather are done (the work counters
+// of the expert GEMMs after it)
 int launch_gather_rows(int dtype, const void* h, const int32_t* perm, int k, int Tk, int shared, void* xp, int H,
-                       cudaStream_t s, const int32_t* live = nullptr);
+                       cudaStream_t s, const int32_t* live = nullptr, unsigned* ctr_a = nullptr,
+                       unsigned* ctr_b = nullptr);
 int launch_combine(int dtype, void* x, const float* y, const float* gates, const int32_t* inv, int k, int Tk,
                    int shared, int H, cudaStream_t s, const int32_t* live = nullptr);
 // Fused row stages (bf16 rows of up to 8192 elements, fp32 up to 4096: kRowVecs 16-byte vectors per thread).

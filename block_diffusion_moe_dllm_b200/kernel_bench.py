@@ -114,7 +114,23 @@ def bench_proj(w: Workload, reps, dev, stream, weights=None):
     return out
 
 
-def bench_experts(w: Workload, reps, dev, stream, weights=None):
+def skewed_routing(w: Workload, rows, dev):
+    """Router outputs (ids, gates, counts, offsets, perm, inv) for synth.skewed_expert_choices: the assignments
+    r * k + j sorted by expert, stably (the order the library's permutation has)."""
+    ids = synth.skewed_expert_choices(rows, w.E, w.k, w.seed)
+    e = ids.flatten().long()
+    perm = torch.sort(e, stable=True).indices.to(torch.int32)
+    inv = torch.empty_like(perm)
+    inv[perm.long()] = torch.arange(perm.numel(), dtype=torch.int32)
+    counts = torch.bincount(e, minlength=w.E).to(torch.int32)
+    offsets = torch.zeros(w.E + 1, dtype=torch.int32)
+    offsets[1:] = torch.cumsum(counts, 0).to(torch.int32)
+    gates = synth.uniform((rows, w.k), 0.1, 1.0, w.seed, "skewed_gates")
+    gates = gates / gates.sum(1, keepdim=True)
+    return tuple(t.to(dev) for t in (ids, gates, counts, offsets, perm, inv))
+
+
+def bench_experts(w: Workload, reps, dev, stream, weights=None, routing="router"):
     rows = w.B * w.L
     lw = weights["layers"][0] if weights else synth.make_weights(
         Workload(**{**w.__dict__, "n_layers": 1, "V": 128}), dev)["layers"][0]
@@ -129,6 +145,8 @@ def bench_experts(w: Workload, reps, dev, stream, weights=None):
     bd.moe_route(h, lw["w_router"], lw["router_bias"], ids, gates, counts, offsets, perm, inv, rows, w.H, w.E, w.k,
                  bd.BF16, ws=ws)
     torch.cuda.synchronize()
+    if routing == "skewed":
+        ids, gates, counts, offsets, perm, inv = skewed_routing(w, rows, dev)
     active = int((counts > 0).sum().item())
     x = torch.zeros((rows, w.H), dtype=torch.bfloat16, device=dev)
     scales = tuple(lw[n + "_scale"] for n in ("w_gu", "w_down", "w_gu_shared", "w_down_shared")) \
@@ -147,7 +165,7 @@ def bench_experts(w: Workload, reps, dev, stream, weights=None):
             _result("moe_route[scores+topk+permute]", troute, rbytes, {"rows": rows})]
 
 
-def bench_expert_gemms(w: Workload, reps, dev, stream, weights=None):
+def bench_expert_gemms(w: Workload, reps, dev, stream, weights=None, routing="router"):
     """The two grouped expert GEMMs alone (dllm_grouped_gemm, the kernels the expert call launches), at the
     workload's routed token rows (router output of random activations) plus the shared expert's rows: gate|up with
     the SwiGLU epilogue, then down with fp32 rows."""
@@ -165,6 +183,8 @@ def bench_expert_gemms(w: Workload, reps, dev, stream, weights=None):
     bd.moe_route(h, lw["w_router"], lw["router_bias"], ids, gates, counts, offsets, perm, inv, rows, w.H, w.E, w.k,
                  bd.BF16, ws=ws)
     torch.cuda.synchronize()
+    if routing == "skewed":
+        _, _, counts, offsets, _, _ = skewed_routing(w, rows, dev)
     active = int((counts > 0).sum().item())
     n = rows * w.k + rows
     hint = min(rows, max(64, 4 * ((rows * w.k + w.E - 1) // w.E)))
@@ -253,11 +273,68 @@ def bench_step(w: Workload, reps, dev, stream):
             "rows": w.B * w.L, "layers": w.n_layers}
 
 
+def bench_block(w: Workload, reps, dev, stream, trace=False):
+    """One whole block (the T_s passes called from the host, then the commit pass) from the block's start state,
+    after one warm-up block, timed with CUDA events. Routing and the rows of each pass are those of a real block,
+    so this is the command the block's ncu launch list is taken with; `launches_before` is the number of the
+    library's launches before the timed blocks (the ncu launch skip)."""
+    from .engine import DenoiseEngine
+    wt = synth.make_weights(w, dev)
+    caches = synth.make_prefix_cache(w, dev)
+    tokens, mask = synth.make_block_state(w, dev)
+    eng = DenoiseEngine(w, wt, caches, dev)
+    eng.set_block(tokens, mask)
+    eng.decode_block()
+    torch.cuda.synchronize()
+    n0 = bd.launch_count()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ts = []
+    for _ in range(reps):
+        eng.set_block(tokens, mask)     # the commit pass rewrites the same cache positions every block
+        a.record(stream)
+        eng.decode_block()
+        b.record(stream)
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b) / 1000.0)
+    t = sorted(ts)[len(ts) // 2]
+    out = {"kernel": "block", "us": t * 1e6, "launches_before": n0,
+           "launches_per_block": (bd.launch_count() - n0) // max(reps, 1), "passes": w.T_s, "layers": w.n_layers}
+    if trace:
+        out["kernels"] = trace_block(eng, tokens, mask)
+    return out
+
+
+def trace_block(eng, tokens, mask):
+    """Device time per kernel over one more block, from the CUDA activity trace (CUPTI through torch.profiler):
+    launches, total us and share per kernel name, largest first. Kernels overlap their neighbours' tails under
+    programmatic dependent launch, so the sum can exceed the block's event-timed duration slightly."""
+    from torch.profiler import profile, ProfilerActivity
+    eng.set_block(tokens, mask)
+    torch.cuda.synchronize()
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        eng.decode_block()
+        torch.cuda.synchronize()
+    rows = {}
+    for ev in prof.events():
+        if ev.device_type.name != "CUDA" or not ev.name or "Memcpy" in ev.name or "Memset" in ev.name:
+            continue
+        r = rows.setdefault(ev.name, [0, 0.0])
+        r[0] += 1
+        r[1] += ev.device_time_total if hasattr(ev, "device_time_total") else ev.cuda_time_total
+    total = sum(v[1] for v in rows.values()) or 1.0
+    return [{"name": k, "launches": v[0], "us": round(v[1], 1), "share": round(v[1] / total, 4)}
+            for k, v in sorted(rows.items(), key=lambda kv: -kv[1][1])]
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--kernel", default="all")
     ap.add_argument("--workload", default=ONE_LAYER.name)
     ap.add_argument("--reps", type=int, default=20)
+    ap.add_argument("--trace", action="store_true", help="block: device time per kernel from the CUDA activity trace")
+    ap.add_argument("--routing", default="router", choices=["router", "skewed"],
+                    help="experts, expert_gemms: the router's choices on random activations, or the skewed choices of "
+                         "a block's own routing (synth.skewed_expert_choices)")
     a = ap.parse_args()
     w = BY_NAME[a.workload]
     dev = "cuda"
@@ -269,15 +346,17 @@ def main():
     if a.kernel in ("proj", "all"):
         out.extend(bench_proj(w, a.reps, dev, stream))
     if a.kernel in ("experts", "route", "all"):
-        out.extend(bench_experts(w, a.reps, dev, stream))
+        out.extend(bench_experts(w, a.reps, dev, stream, routing=a.routing))
     if a.kernel in ("experts", "expert_gemms", "all"):
-        out.extend(bench_expert_gemms(w, a.reps, dev, stream))
+        out.extend(bench_expert_gemms(w, a.reps, dev, stream, routing=a.routing))
     if a.kernel in ("unmask", "all") and w.L <= 32:   # the prefill shape has no unmasking step
         out.append(bench_unmask(w, a.reps, dev, stream))
     if a.kernel in ("attn", "all"):
         out.append(bench_attn(w, a.reps, dev, stream))
     if a.kernel == "step":
         out.append(bench_step(w, a.reps, dev, stream))
+    if a.kernel == "block":
+        out.append(bench_block(w, a.reps, dev, stream, a.trace))
     for r in out:
         print(json.dumps(r), flush=True)
 

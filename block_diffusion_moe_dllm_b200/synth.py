@@ -145,3 +145,27 @@ def make_block_state(w: Workload, device="cpu", seed=None, masked_fraction=1.0):
         tokens[half:] = tokens[:half]
     tokens = torch.where(mask.bool(), torch.full_like(tokens, w.mask_id), tokens)
     return tokens, mask
+
+
+def skewed_expert_choices(rows, E, k, seed, tag="skewed_ids", n_hot=8, n_warm=60, p_hot=0.67):
+    """Expert choices [rows, k] int32 (distinct per row) with the skew a block's own router shows on an untrained
+    backbone, where most block positions hold the same mask token: each slot picks, with probability ``p_hot``, one
+    of ``n_hot`` crowded experts, else one of ``n_warm`` others (both sets drawn at random from the E experts).
+    Measured on the 20-layer understanding workload: about 8 experts with 340-512 rows each and some 60 with a
+    median of 18 rows take the 4096 assignments of 512 rows."""
+    g = _gen(seed, tag, "cpu")
+    experts = torch.randperm(E, generator=g)
+    hot, warm = experts[:n_hot], experts[n_hot:n_hot + n_warm]
+    ids = torch.empty((rows, k), dtype=torch.int32)
+    u = torch.rand((rows, k), generator=g)
+    for r in range(rows):
+        taken = set()
+        for j in range(k):
+            pool = hot if (u[r, j] < p_hot and len(taken & set(hot.tolist())) < n_hot) else warm
+            while True:
+                e = int(pool[int(torch.randint(0, len(pool), (1,), generator=g))])
+                if e not in taken:
+                    break
+            taken.add(e)
+            ids[r, j] = e
+    return ids

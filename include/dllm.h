@@ -21,7 +21,8 @@
  *   - Bf16 tensors read by TMA need 16-byte aligned bases and row strides (DLLM_ERR_ALIGN otherwise).
  *   - A workspace is caller-provided device scratch of at least the size the matching *_workspace_size query
  *     returns, 256-byte aligned. Its first 256 bytes hold a status word that kernels set when a bounded wait
- *     gives up (DLLM_ERR_TIMEOUT through dllm_status_check). Calls that share a workspace must be ordered
+ *     gives up (DLLM_ERR_TIMEOUT through dllm_status_check) and the expert GEMMs' work counters (reset by the
+ *     kernels themselves; the caller never initialises them). Calls that share a workspace must be ordered
  *     (same stream); calls on different workspaces are independent and re-entrant.
  */
 #ifndef DLLM_H_

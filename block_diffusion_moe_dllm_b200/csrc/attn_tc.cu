@@ -148,10 +148,36 @@ __device__ __forceinline__ void cluster_wait() {
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
-// Each lane reads 64 consecutive 32-bit columns of its own TMEM lane.
+// 32 columns without the wait: the registers are valid after tcgen05.wait::ld.
+__device__ __forceinline__ void tmem_ld32_issue(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+
+// Each lane reads 64 consecutive 32-bit columns of its own TMEM lane (two loads in flight, one wait).
 __device__ __forceinline__ void tmem_ld64(uint32_t taddr, float* v) {
-  tmem_ld32(taddr, v);
-  tmem_ld32(taddr + 32, v + 32);
+  uint32_t r[64];
+  tmem_ld32_issue(taddr, r);
+  tmem_ld32_issue(taddr + 32, r + 32);
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 64; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// A whole 128-column row of S: four loads in flight, one wait.
+__device__ __forceinline__ void tmem_ld128(uint32_t taddr, float* v) {
+  uint32_t r[128];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) tmem_ld32_issue(taddr + 32 * c, r + 32 * c);
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 128; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 // Packed fp32 pairs (sm_100 f32x2 instructions) and the hardware base-2 exponential (ex2.approx.ftz: relative
@@ -386,20 +412,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       const short* kbt = bar.kblk[grp][i & 1];
       if (!wait_bar(&bar.s_full[grp], i & 1, abort_flag, p.status, ST_TIMEOUT_EPILOGUE)) ok = false;
       tc::fence_after_sync();
-      // row maximum of the visible scores
+      // the row of S (one TMEM round trip), then the maximum of its visible scores
+      float sv[128];
+      tmem_ld128(tSg, sv);
       float mt = -INFINITY;
+      if (fast) {
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        float v[64];
-        tmem_ld64(tSg + 64 * c, v);
-        if (fast) {
+        for (int u = 0; u < 128; ++u) mt = fmaxf(mt, sv[u]);
+      } else {
 #pragma unroll
-          for (int u = 0; u < 64; ++u) mt = fmaxf(mt, v[u]);
-        } else {
-#pragma unroll
-          for (int u = 0; u < 64; ++u)
-            if (kbt[64 * c + u] <= qrel) mt = fmaxf(mt, v[u]);
-        }
+        for (int u = 0; u < 128; ++u)
+          if (kbt[u] <= qrel) mt = fmaxf(mt, sv[u]);
       }
       mt *= p.scale_log2;
       // the reference maximum moves only when this tile's maximum exceeds it by more than 2^8
@@ -415,8 +438,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
       const bool any = mg != -INFINITY;
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
-        float v[64];
-        tmem_ld64(tSg + 64 * c, v);
+        const float* v = sv + 64 * c;
         uint32_t pk[32];
         if (fast) {     // every key visible: the tile maximum is finite, so mg is too
 #pragma unroll
@@ -441,8 +463,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             rs2 = add2(rs2, pk2(e0, e1));
           }
         }
-        // keys [64c, 64c + 64) -> columns [32c, 32c + 32): S there has been read (c = 0: this chunk's first half;
-        // c = 1: chunk 0)
+        // keys [64c, 64c + 64) -> columns [32c, 32c + 32) (S has been read into registers)
         tc::tmem_st32(tSg + 32 * c, pk);
       }
       // O_g holds the group's previous P V once that phase completes (every phase is waited in order, so the

@@ -110,23 +110,51 @@ DLLM_DEV bool warp_topk(float* __restrict__ srow, const float* __restrict__ bias
                         int lane, int& my_id, float& my_gate, float& thr) {
   float v[PER], r[PER];
   int e[PER];
+  // every load of the row (and of the bias) in flight before the first use: the row was just written by another
+  // kernel, and loads issued one after another behind the write-back of each sigmoid would pay the L2 round trip
+  // PER times
+  float xs[PER], bs[PER];
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int ex = i * 32 + lane;
+    xs[i] = ex < E ? __ldcg(srow + ex) : 0.f;
+    bs[i] = ex < E ? __ldg(bias + ex) : 0.f;
+  }
 #pragma unroll
   for (int i = 0; i < PER; ++i) {
     const int ex = i * 32 + lane;
     const bool in = ex < E;
-    float x = in ? srow[ex] : 0.f;
+    float x = xs[i];
     if (from_logits && in) {
-      x = 1.0f / (1.0f + expf(-x));
+      // intrinsic exponential and approximate divide: within about 1e-6 relative of the rounded sigmoid, an order
+      // below the guard band
+      x = __fdividef(1.0f, 1.0f + __expf(-x));
       srow[ex] = x;
     }
     r[i] = x;
-    v[i] = in ? x + bias[ex] : -INFINITY;
+    v[i] = in ? x + bs[i] : -INFINITY;
     e[i] = in ? ex : 0x7fffffff;
   }
-  // insertion network: after step i, entries [0, i] are sorted (PER <= 8; wider rows keep the unsorted
-  // candidates and the winning lane rescans them, below)
+  // each lane's candidates in order, largest first (ties: lower expert first). Eight: Batcher's odd-even merge
+  // network (19 comparators in 6 layers, so the chain of dependent compares is 6 long); fewer: an insertion
+  // network; more than eight: the lane keeps them unsorted and the winning lane rescans them (below)
+  auto cas = [&](int i, int j) {   // entry i gets the better of entries i and j
+    const bool sw = v[j] > v[i] || (v[j] == v[i] && e[j] < e[i]);
+    const float tv = v[i], tr = r[i];
+    const int te = e[i];
+    v[i] = sw ? v[j] : tv; r[i] = sw ? r[j] : tr; e[i] = sw ? e[j] : te;
+    v[j] = sw ? tv : v[j]; r[j] = sw ? tr : r[j]; e[j] = sw ? te : e[j];
+  };
+  if constexpr (PER == 8) {
+    cas(0, 1); cas(2, 3); cas(4, 5); cas(6, 7);
+    cas(0, 2); cas(1, 3); cas(4, 6); cas(5, 7);
+    cas(1, 2); cas(5, 6);
+    cas(0, 4); cas(1, 5); cas(2, 6); cas(3, 7);
+    cas(2, 4); cas(3, 5);
+    cas(1, 2); cas(3, 4); cas(5, 6);
+  }
 #pragma unroll
-  for (int i = 1; i < (PER <= 8 ? PER : 1); ++i) {
+  for (int i = 1; i < (PER < 8 ? PER : 1); ++i) {
 #pragma unroll
     for (int j = i; j > 0; --j) {
       const bool sw = v[j] > v[j - 1] || (v[j] == v[j - 1] && e[j] < e[j - 1]);

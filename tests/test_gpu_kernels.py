@@ -126,7 +126,8 @@ def test_gemm_f32():
                                             ("bf16", 20, 256, 512, 8), ("f32", 32, 128, 64, 32),
                                             ("bf16", 4096, 512, 256, 8), ("bf16", 1001, 256, 1000, 3),
                                             ("f32", 4100, 64, 32, 2), ("bf16", 5000, 256, 96, 4),
-                                            ("bf16", 1024, 512, 128, 8), ("f32", 4096, 64, 32, 2)])
+                                            ("bf16", 1024, 512, 128, 8), ("f32", 4096, 64, 32, 2),
+                                            ("bf16", 33, 256, 96, 4), ("f32", 1000, 128, 200, 6)])
 def test_route(dtype, Tk, H, E, k):
     t = _tdt(dtype)
     h = synth.normal((Tk, H), 1.0, 5, f"rh{Tk}", DEV, t)

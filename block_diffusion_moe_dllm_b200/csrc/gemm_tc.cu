@@ -1511,18 +1511,15 @@ int gemm_bf16_tc(const GemmArgs& a, cudaStream_t s) {
     st2 = wide.bn == 128 ? launch_wide_splitk<128, 6>(a, mw, mw2, mx, kp, s)
                          : launch_wide_splitk<256, 4>(a, mw, mw2, mx, kp, s);
   } else if (ks > 1) st2 = launch_cluster_splitk(a, mw, mw2, mx, kp, s);
-  else if (kp.work_ctr) {
-    // grouped (expert) launches: a weight ring and an activation ring. Measured on a 20-layer block at N tile 128
-    // (same GPU, weight + activation stages): 8 + 4 took 150.7 ms, 7 + 5 151.3, 6 + 6 151.9, 9 + 3 153.1; a shared
-    // ring of 6 stages 153.9
+  else {
+    // single-CTA tiles: a weight ring and an activation ring. Measured on a 20-layer block at N tile 128 (same
+    // GPU, weight + activation stages of the expert GEMMs): 8 + 4 took 150.7 ms, 7 + 5 151.3, 6 + 6 151.9, 9 + 3
+    // 153.1, a shared ring of 6 stages 153.9; the same split for the dense projections (QKV, output) 150.5 -> 150.1
     if (bn == 32) st2 = launch<32, 11, false, 4>(a, mw, mw2, mx, kp, s);
     else if (bn == 64) st2 = launch<64, 10, false, 4>(a, mw, mw2, mx, kp, s);
     else if (bn == 128) st2 = launch<128, 8, false, 4>(a, mw, mw2, mx, kp, s);
     else st2 = launch<256, 6, false, 2>(a, mw, mw2, mx, kp, s);
-  } else if (bn == 32) st2 = launch<32, 9>(a, mw, mw2, mx, kp, s);
-  else if (bn == 64) st2 = launch<64, 8>(a, mw, mw2, mx, kp, s);
-  else if (bn == 128) st2 = launch<128, 6>(a, mw, mw2, mx, kp, s);
-  else st2 = launch<256, 4>(a, mw, mw2, mx, kp, s);
+  }
   return st2;
 }
 

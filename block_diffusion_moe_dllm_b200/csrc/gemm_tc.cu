@@ -484,7 +484,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
   constexpr int W_BYTES = F8 ? RAW_BYTES : A_BYTES;
   constexpr int STAGE_BYTES = SPLIT ? W_BYTES : W_BYTES + B_BYTES;
   constexpr uint32_t W_TX = W_BYTES;                                      // weight bytes a stage's TMA brings
-  constexpr uint32_t TMEM_COLS = F8 ? 512 : 2 * BN;
+  // two accumulators of BN columns; the allocation is a power of two (N tile 96: 256 columns)
+  constexpr uint32_t TMEM_COLS = F8 ? 512 : (2 * BN <= 64 ? 64 : 2 * BN <= 128 ? 128 : 2 * BN <= 256 ? 256 : 512);
   static_assert(!F8 || 2 * BN + MS * SLOT_COLS <= 512, "FP8 A slots exceed the tensor memory");
   static_assert(BST <= 8, "activation ring");
   uint8_t* stages = base;
@@ -1517,6 +1518,7 @@ int gemm_bf16_tc(const GemmArgs& a, cudaStream_t s) {
     // 153.1, a shared ring of 6 stages 153.9; the same split for the dense projections (QKV, output) 150.5 -> 150.1
     if (bn == 32) st2 = launch<32, 11, false, 4>(a, mw, mw2, mx, kp, s);
     else if (bn == 64) st2 = launch<64, 10, false, 4>(a, mw, mw2, mx, kp, s);
+    else if (bn == 96) st2 = launch<96, 8, false, 5>(a, mw, mw2, mx, kp, s);
     else if (bn == 128) st2 = launch<128, 8, false, 4>(a, mw, mw2, mx, kp, s);
     else st2 = launch<256, 6, false, 2>(a, mw, mw2, mx, kp, s);
   }
@@ -1539,8 +1541,14 @@ static bool dense(const GemmArgs& a) { return !a.swiglu && !a.n_dev && !a.has_ex
 int gemm_bn(const GemmArgs& a) {
   int bn = bn_for(a.max_cnt);
   if (a.w_fp8) return std::min(bn, 128);   // FP8 weights: single-CTA tiles of at most 128 rows
-  if (dense(a))
-    while (bn > 32 && (a.M / 128) * ((a.max_cnt + bn - 1) / bn) < num_sms() / 2) bn /= 2;
+  if (dense(a)) {
+    const int mt = a.M / 128;
+    while (bn > 32 && mt * ((a.max_cnt + bn - 1) / bn) < num_sms() / 2) bn /= 2;
+    // N tile 96 where 128 leaves more than a quarter of the SMs without a tile and 96 still fits one wave (the QKV
+    // projection of 512 rows: 96 -> 144 tiles, each CTA moving 7/8 of the operand bytes)
+    if (bn == 128 && mt * ((a.max_cnt + 127) / 128) < num_sms() * 3 / 4 && mt * ((a.max_cnt + 95) / 96) <= num_sms())
+      bn = 96;
+  }
   return bn;
 }
 

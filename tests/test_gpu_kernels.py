@@ -26,8 +26,11 @@ def _tdt(name):
 
 # ------------------------------------------------------------------------------------------------ GEMM
 @pytest.mark.parametrize("N,M,K", [(1, 128, 64), (5, 256, 128), (32, 384, 2048), (77, 256, 512), (200, 128, 256),
-                                   (300, 256, 192), (513, 128, 64)])
+                                   (300, 256, 192), (513, 128, 64), (512, 3072, 2048), (500, 3072, 512),
+                                   (440, 2816, 1024)])
 def test_gemm_bf16_store(N, M, K):
+    """Dense projections; the last three take the 96-row N tile (one wave of 96-row tiles where 128-row tiles would
+    leave a quarter of the SMs idle), ragged at 500 and 440 rows."""
     x = synth.normal((N, K), 1.0, 1, f"gx{N}", DEV)
     w = synth.normal((M, K), 0.05, 1, f"gw{M}{K}", DEV)
     y = torch.full((N, M), float("nan"), dtype=torch.bfloat16, device=DEV)

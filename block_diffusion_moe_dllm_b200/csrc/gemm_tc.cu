@@ -1509,8 +1509,9 @@ int gemm_bf16_tc(const GemmArgs& a, cudaStream_t s) {
     kp.prefetch_w = 0;
     st2 = launch_pair(mw, mw2, mx, kp, s);
   } else if (wide.ks > 1) {
-    st2 = wide.bn == 128 ? launch_wide_splitk<128, 6>(a, mw, mw2, mx, kp, s)
-                         : launch_wide_splitk<256, 4>(a, mw, mw2, mx, kp, s);
+    st2 = wide.bn == 64 ? launch_wide_splitk<64, 8>(a, mw, mw2, mx, kp, s)
+          : wide.bn == 128 ? launch_wide_splitk<128, 6>(a, mw, mw2, mx, kp, s)
+                           : launch_wide_splitk<256, 4>(a, mw, mw2, mx, kp, s);
   } else if (ks > 1) st2 = launch_cluster_splitk(a, mw, mw2, mx, kp, s);
   else {
     // single-CTA tiles: a weight ring and an activation ring. Measured on a 20-layer block at N tile 128 (same
@@ -1569,12 +1570,13 @@ int gemm_splitk_factor(const GemmArgs& a, int bn) {
 }
 
 // Wide split-K plan (see launch_wide_splitk) for a dense bf16 projection over more than one 32-row tile with a
-// row count fixed on the host and at most four 128-row weight tiles (the router's logits): among N tiles of 128
-// and 256 rows and 2..8 K slices whose clusters all fit in one wave, the one with the least operand traffic per CTA
-// ((128 + N tile) x K / slices), taken when it is at most three quarters of the plain kernel's. Measured at 512
-// rows: the router (256 experts x 2048) 32.1 -> 29.4 us for logits, top-k and permutation; the wider QKV and
-// output projections gained nothing (15.9 us both ways) or lost (12.5 -> 15.0 us): their slices' 64-128 KB
-// accumulators cost as much to stage and reduce as the operand traffic saved.
+// row count fixed on the host and at most four 128-row weight tiles (the router's logits): among N tiles of 64,
+// 128 and 256 rows and 2..8 K slices whose clusters all fit in one wave, the one with the least operand traffic per
+// CTA ((128 + N tile) x K / slices), taken when it is at most three quarters of the plain kernel's. Measured at 512
+// rows: the router (256 experts x 2048) 32.1 -> 29.4 us for logits, top-k and permutation with N tile 128 (64 CTAs),
+// and N tile 64 (128 CTAs) took a 20-layer block from 149.6 to 147.6 ms; the wider QKV and output projections
+// gained nothing (15.9 us both ways) or lost (12.5 -> 15.0 us): their slices' 64-128 KB accumulators cost as much
+// to stage and reduce as the operand traffic saved.
 WideSplit wide_splitk_plan(const GemmArgs& a) {
   WideSplit best;
   if (a.dtype != DLLM_BF16 || !dense(a) || a.w_fp8 || a.epi.conf_part || a.cnt_dev || a.host_cnt <= 32) return best;
@@ -1584,11 +1586,12 @@ WideSplit wide_splitk_plan(const GemmArgs& a) {
   const int tiles0 = mt * ((rows + bn0 - 1) / bn0);
   const double base = (double)(128 + std::min(bn0, rows)) * a.K * ((tiles0 + sms - 1) / sms);
   double cost = 0.75 * base;
-  for (int bn : {128, 256}) {
+  for (int bn : {64, 128, 256}) {
     const int tiles = mt * ((rows + bn - 1) / bn);
     for (int ks = 2; ks <= 8 && 2 * ks <= kblocks; ++ks) {
       if (tiles * ks > sms) break;
-      const int act = bn == 128 ? max_active_clusters_t<128, 6>(ks) : max_active_clusters_t<256, 4>(ks);
+      const int act = bn == 64 ? max_active_clusters_t<64, 8>(ks)
+                      : bn == 128 ? max_active_clusters_t<128, 6>(ks) : max_active_clusters_t<256, 4>(ks);
       if (tiles > act) continue;
       const double c = (double)(128 + std::min(bn, rows)) * a.K / ks;
       if (c < cost) { cost = c; best.bn = bn; best.ks = ks; }

@@ -1316,8 +1316,8 @@ int launch_cluster_splitk(const GemmArgs& a, const CUtensorMap& mw, const CUtens
 }
 
 // ---- wide split-K: dense projections over several N tiles of rows (the 512 rows of a denoising block) whose
-// 128-row tiles would each stream a whole K of weights and tokens on fewer SMs than the GPU has. N tiles of 128 or
-// 256 rows split along K over a thread-block cluster put every SM to work on a slice with less operand traffic per
+// 128-row tiles would each stream a whole K of weights and tokens on fewer SMs than the GPU has. N tiles of 64, 128
+// or 256 rows split along K over a thread-block cluster put every SM to work on a slice with less operand traffic per
 // SM; each slice's accumulator goes through the idle operand ring to the cluster's reduction.
 template <int BN, int STAGES>
 constexpr int splitk_smem() {

@@ -187,7 +187,7 @@ def bench_expert_gemms(w: Workload, reps, dev, stream, weights=None, routing="ro
         _, _, counts, offsets, _, _ = skewed_routing(w, rows, dev)
     active = int((counts > 0).sum().item())
     n = rows * w.k + rows
-    hint = min(rows, max(64, 4 * ((rows * w.k + w.E - 1) // w.E)))
+    hint = min(rows, max(128, 4 * ((rows * w.k + w.E - 1) // w.E)))   # the step's N-tile hint for expert GEMMs
     xp = synth.normal((n, w.H), 1.0, 6, "kb_xp", dev)
     act = torch.empty((n, w.I), dtype=torch.bfloat16, device=dev)
     y = torch.empty((n, w.H), dtype=torch.float32, device=dev)

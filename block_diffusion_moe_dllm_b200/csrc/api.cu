@@ -78,7 +78,7 @@ int run_gemm(GemmArgs& a, cudaStream_t s) {
 struct ExpertBufs {
   void* xp;
   void* act;
-  float* y;
+  void* y;        // expert output rows in the storage type
   float* scratch;
 };
 
@@ -86,7 +86,7 @@ void carve_experts(Carver& c, int dtype, int Tk, int H, int k, int I, int shared
   const int64_t rows = (int64_t)Tk * k + (shared ? Tk : 0);
   b.xp = c.take(rows * H * esize(dtype));
   b.act = c.take(rows * I * esize(dtype));
-  b.y = c.take<float>(rows * H * 4);
+  b.y = c.take(rows * H * esize(dtype));
   b.scratch = dtype == DLLM_F32 ? c.take<float>(gemm_f32_scratch_bytes(rows, std::max(2 * I, H), 0)) : nullptr;
 }
 
@@ -151,7 +151,7 @@ int run_experts(int dtype, int Tk, int H, int E, int k, int I, const void* h, co
   g2.w = w_down; g2.w_rows = (int64_t)E * H; g2.w2 = w_down_s; g2.w2_rows = H; g2.w_group_stride = H;
   g2.w_scale = sc.down; g2.w2_scale = sc.down_shared; g2.work_ctr = ctr2;
   g2.epi = EpiParams();
-  g2.epi.kind = EPI_STORE; g2.epi.out = b.y; g2.epi.ldo = H; g2.epi.out_f32 = 1;
+  g2.epi.kind = EPI_STORE; g2.epi.out = b.y; g2.epi.ldo = H; g2.epi.out_f32 = dtype == DLLM_F32;
   st = run_gemm(g2, s);
   if (st) return st;
   if (pn.g)

@@ -204,9 +204,18 @@ int launch_gather_rows(int dtype, const void* h, const int32_t* perm, int k, int
 }
 
 // ------------------------------------------------------------------------------------------------ combine
+// Four consecutive expert-output values as fp32 (rows in the storage type: bf16 rows are 8-byte loads).
+__device__ __forceinline__ float4 load_y4(const float* y) { return *reinterpret_cast<const float4*>(y); }
+__device__ __forceinline__ float4 load_y4(const __nv_bfloat16* y) {
+  const uint2 u = *reinterpret_cast<const uint2*>(y);
+  const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
+  const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
+  return make_float4(a.x, a.y, b.x, b.y);
+}
+
 // x[t] = x[t] + (y[Tk*k + t] + sum_j gates[t, j] * y[inv[t*k + j]]), summed in fp32 in slot order, rounded once.
 template <typename T>
-__global__ void __launch_bounds__(128) combine_kernel(T* __restrict__ x, const float* __restrict__ y,
+__global__ void __launch_bounds__(128) combine_kernel(T* __restrict__ x, const T* __restrict__ y,
                                                       const float* __restrict__ gates, const int32_t* __restrict__ inv,
                                                       int k, int n_assign, int shared, int H,
                                                       const int32_t* __restrict__ live) {
@@ -216,11 +225,10 @@ __global__ void __launch_bounds__(128) combine_kernel(T* __restrict__ x, const f
   const int t = blockIdx.x;
   const int h0 = (blockIdx.y * blockDim.x + threadIdx.x) * 4;
   if (h0 >= H) return;
-  float4 acc = shared ? *reinterpret_cast<const float4*>(y + (int64_t)(n_assign + t) * H + h0)
-                      : make_float4(0.f, 0.f, 0.f, 0.f);
+  float4 acc = shared ? load_y4(y + (int64_t)(n_assign + t) * H + h0) : make_float4(0.f, 0.f, 0.f, 0.f);
   for (int j = 0; j < k; ++j) {
     const float gj = gates[t * k + j];
-    const float4 v = *reinterpret_cast<const float4*>(y + (int64_t)inv[t * k + j] * H + h0);
+    const float4 v = load_y4(y + (int64_t)inv[t * k + j] * H + h0);
     acc.x += gj * v.x;
     acc.y += gj * v.y;
     acc.z += gj * v.z;
@@ -233,15 +241,16 @@ __global__ void __launch_bounds__(128) combine_kernel(T* __restrict__ x, const f
   xr[3] = from_f32<T>(to_f32(xr[3]) + acc.w);
 }
 
-int launch_combine(int dtype, void* x, const float* y, const float* gates, const int32_t* inv, int k, int Tk,
+int launch_combine(int dtype, void* x, const void* y, const float* gates, const int32_t* inv, int k, int Tk,
                    int shared, int H, cudaStream_t s, const int32_t* live) {
   if (Tk <= 0) return DLLM_OK;
   dim3 grid(Tk, (H / 4 + 127) / 128);
   if (dtype == DLLM_BF16)
-    launch_pdl(combine_kernel<__nv_bfloat16>, grid, 128, 0, s, (__nv_bfloat16*)x, y, gates, inv, k, Tk * k, shared, H,
-               live);
+    launch_pdl(combine_kernel<__nv_bfloat16>, grid, 128, 0, s, (__nv_bfloat16*)x, (const __nv_bfloat16*)y, gates, inv,
+               k, Tk * k, shared, H, live);
   else
-    launch_pdl(combine_kernel<float>, grid, 128, 0, s, (float*)x, y, gates, inv, k, Tk * k, shared, H, live);
+    launch_pdl(combine_kernel<float>, grid, 128, 0, s, (float*)x, (const float*)y, gates, inv, k, Tk * k, shared, H,
+               live);
   DLLM_CHECK_LAUNCH("combine_kernel");
   return DLLM_OK;
 }
@@ -398,7 +407,7 @@ int launch_embed_norm(int dtype, const int32_t* tokens, const uint8_t* mask, int
 // final-norm row of a still-masked position only, at its place in the LM head's row list (rank among the masked
 // positions of its half, plus n for the unconditional half), which is the order masked_rows_kernel produces.
 template <typename T>
-__global__ void __launch_bounds__(256) combine_norm_kernel(T* __restrict__ x, const float* __restrict__ y,
+__global__ void __launch_bounds__(256) combine_norm_kernel(T* __restrict__ x, const T* __restrict__ y,
                                                            const float* __restrict__ gates,
                                                            const int32_t* __restrict__ inv, int k, int n_assign,
                                                            int shared, int H, const T* __restrict__ g, float eps,
@@ -423,16 +432,15 @@ __global__ void __launch_bounds__(256) combine_norm_kernel(T* __restrict__ x, co
       float acc[VE];
 #pragma unroll
       for (int u = 0; u < VE; u += 4) {
-        const float4 v = shared ? *reinterpret_cast<const float4*>(y + (int64_t)(n_assign + t) * H + h0 + u)
-                                : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 v = shared ? load_y4(y + (int64_t)(n_assign + t) * H + h0 + u) : make_float4(0.f, 0.f, 0.f, 0.f);
         acc[u] = v.x; acc[u + 1] = v.y; acc[u + 2] = v.z; acc[u + 3] = v.w;
       }
       for (int j = 0; j < k; ++j) {
         const float gj = gates[t * k + j];
-        const float* yr = y + (int64_t)inv[t * k + j] * H + h0;
+        const T* yr = y + (int64_t)inv[t * k + j] * H + h0;
 #pragma unroll
         for (int u = 0; u < VE; u += 4) {
-          const float4 v = *reinterpret_cast<const float4*>(yr + u);
+          const float4 v = load_y4(yr + u);
           acc[u] += gj * v.x; acc[u + 1] += gj * v.y; acc[u + 2] += gj * v.z; acc[u + 3] += gj * v.w;
         }
       }
@@ -465,15 +473,16 @@ __global__ void __launch_bounds__(256) combine_norm_kernel(T* __restrict__ x, co
   store_norm_row<T>(keep, nvec, 1.0f / sqrtf(ss / (float)H + eps), g, out + (int64_t)row * H);
 }
 
-int launch_combine_norm(int dtype, void* x, const float* y, const float* gates, const int32_t* inv, int k, int Tk,
+int launch_combine_norm(int dtype, void* x, const void* y, const float* gates, const int32_t* inv, int k, int Tk,
                         int shared, int H, const void* g, float eps, void* out, int mode, const uint8_t* mask,
                         int n_half_pos, const int32_t* n_dev, cudaStream_t s, const int32_t* live) {
   if (Tk <= 0) return DLLM_OK;
   if (dtype == DLLM_BF16)
-    launch_pdl(combine_norm_kernel<__nv_bfloat16>, Tk, 256, 0, s, (__nv_bfloat16*)x, y, gates, inv, k, Tk * k, shared,
+    launch_pdl(combine_norm_kernel<__nv_bfloat16>, Tk, 256, 0, s, (__nv_bfloat16*)x, (const __nv_bfloat16*)y, gates,
+               inv, k, Tk * k, shared,
                H, (const __nv_bfloat16*)g, eps, (__nv_bfloat16*)out, mode, mask, n_half_pos, n_dev, live);
   else
-    launch_pdl(combine_norm_kernel<float>, Tk, 256, 0, s, (float*)x, y, gates, inv, k, Tk * k, shared, H,
+    launch_pdl(combine_norm_kernel<float>, Tk, 256, 0, s, (float*)x, (const float*)y, gates, inv, k, Tk * k, shared, H,
                (const float*)g, eps, (float*)out, mode, mask, n_half_pos, n_dev, live);
   DLLM_CHECK_LAUNCH("combine_norm_kernel");
   return DLLM_OK;

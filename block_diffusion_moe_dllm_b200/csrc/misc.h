@@ -19,7 +19,7 @@ int launch_masked_rows(const uint8_t* mask, int n_pos, int halves, int32_t* row_
 int launch_gather_rows(int dtype, const void* h, const int32_t* perm, int k, int Tk, int shared, void* xp, int H,
                        cudaStream_t s, const int32_t* live = nullptr, unsigned* ctr_a = nullptr,
                        unsigned* ctr_b = nullptr);
-int launch_combine(int dtype, void* x, const float* y, const float* gates, const int32_t* inv, int k, int Tk,
+int launch_combine(int dtype, void* x, const void* y, const float* gates, const int32_t* inv, int k, int Tk,
                    int shared, int H, cudaStream_t s, const int32_t* live = nullptr);
 // Fused row stages (bf16 rows of up to 8192 elements, fp32 up to 4096: kRowVecs 16-byte vectors per thread).
 constexpr int kRowVecs = 4;
@@ -37,7 +37,7 @@ int launch_embed_norm(int dtype, const int32_t* tokens, const uint8_t* mask, int
                       void* h, const void* g, int rows, int H, float eps, const uint8_t* list_mask, int n_pos,
                       int halves, int32_t* row_pos, int32_t* n_out, cudaStream_t s,
                       const RopeTable& rope = RopeTable());
-int launch_combine_norm(int dtype, void* x, const float* y, const float* gates, const int32_t* inv, int k, int Tk,
+int launch_combine_norm(int dtype, void* x, const void* y, const float* gates, const int32_t* inv, int k, int Tk,
                         int shared, int H, const void* g, float eps, void* out, int mode, const uint8_t* mask,
                         int n_half_pos, const int32_t* n_dev, cudaStream_t s, const int32_t* live = nullptr);
 

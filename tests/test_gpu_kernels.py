@@ -1,4 +1,5 @@
 """Per-call parity of the CUDA library against the fp64 oracle on seeded inputs (GPU)."""
+import ctypes as C
 import math
 
 import numpy as np
@@ -232,6 +233,42 @@ def test_experts(dtype, Tk, H, E, k, I, shared):
                         to64(sgu) if shared else None, to64(sd) if shared else None, dtype)
     want = O.store(to64(x0) + delta, dtype)
     assert_close(to64(x), want, dtype, "experts")
+
+
+@pytest.mark.parametrize("Tk", [512, 200])
+def test_experts_crowded_routing_with_stale_work_counters(Tk):
+    """The block's own routing piles rows on a few experts (synth.skewed_expert_choices: 8 crowded experts with
+    hundreds of rows, ~60 with a few each): the tiles the expert GEMMs' dynamic schedule balances. The schedule's
+    work counters sit in the workspace's status block and are reset by the row gather at every call, so words left
+    there by anything else (planted here) must not change the result."""
+    dtype, H, E, k, I = "bf16", 2048, 256, 8, 512
+    t = _tdt(dtype)
+    h = synth.normal((Tk, H), 1.0, 16, "ch", DEV, t)
+    x0 = synth.normal((Tk, H), 1.0, 16, "cx", DEV, t)
+    wgu = synth.normal((E, 2 * I, H), 0.02, 16, "cgu", DEV, t)
+    wd = synth.normal((E, H, I), 0.02, 16, "cd", DEV, t)
+    sgu = synth.normal((2 * I, H), 0.02, 16, "csgu", DEV, t)
+    sd = synth.normal((H, I), 0.02, 16, "csd", DEV, t)
+    ids = synth.skewed_expert_choices(Tk, E, k, 16).numpy()
+    g = np.random.default_rng(Tk)
+    gates = g.uniform(0.1, 1.0, (Tk, k)).astype(np.float32)
+    gates = (gates / gates.sum(1, keepdims=True)).astype(np.float32)
+    counts, offsets, perm, inv = assignment_tables(ids, E)
+    assert counts.max() >= 128, "the case must hold experts with more rows than one N tile"
+    cvt = lambda a: torch.from_numpy(a).to(DEV)
+    desc = bd.ExpertDesc(Tk, H, E, k, I, DT[dtype], 0)
+    ws = bd.Workspace(bd.load().dllm_moe_experts_workspace_size(C.byref(desc)), DEV)
+    off = ws.addr - ws.buf.data_ptr()
+    for word in (16, 32):   # the two GEMMs' counters (bytes 64 and 128 of the status block)
+        ws.buf[off + 4 * word: off + 4 * word + 4] = torch.tensor([0x78, 0x56, 0x34, 0x12], dtype=torch.uint8)
+    x = x0.clone()
+    bd.moe_experts(h, wgu, wd, sgu, sd, cvt(counts), cvt(offsets), cvt(perm), cvt(inv), cvt(gates), x, Tk, H, E, k,
+                   I, DT[dtype], ws=ws)
+    torch.cuda.synchronize()
+    assert bd.status_check(ws) == bd.OK
+    delta = O.moe_delta(to64(h), ids, gates.astype(np.float64), to64(wgu), to64(wd), to64(sgu), to64(sd), dtype)
+    want = O.store(to64(x0) + delta, dtype)
+    assert_close(to64(x), want, dtype, "experts, crowded routing")
 
 
 @pytest.mark.parametrize("Tk,E,k,I,H,swiglu", [(512, 256, 8, 512, 2048, 1), (512, 256, 8, 512, 2048, 0),

@@ -41,6 +41,9 @@ Readings where the pages are silent (each also listed in the design notes):
   * threshold rule (formula stripped on the page): k_t = min(m, max(ceil(m / (T_s - t)), min(k_max, #{c > tau}))).
   * CFG: z = z_u + s (z_c - z_u), s = cfg_scale, in fp64; decisions within the float32 rounding bound of that
     formula are flagged as near-ties (cfg_fp32_error_bound).
+  * editing CFG (three rows per position, formula not printed): z = z_u + s_i (z_i - z_u) + s_t (z_c - z_i), with
+    s_t = cfg_text_scale (cfg_scale here) and s_i = cfg_image_scale; rows (b, b + B/3, b + 2B/3) are (instruction
+    and image, image only, unconditional); near-ties by cfg3_fp32_error_bound.
   * confidence c = max softmax at temperature 1 over the scored vocabulary; candidate = lowest argmax.
   * storage rounding: wherever the library stores a tensor in its storage type (bf16 or fp32) the oracle rounds
     its fp64 value to that type (round-to-nearest-even) at the same point; between those points it is fp64.
@@ -293,6 +296,28 @@ def cfg_fp32_error_bound(zc, zu, scale):
     return 1.01 * 2.0 ** -24 * np.max(2.0 * np.abs(d) + np.abs(zu + d), axis=-1)
 
 
+def cfg3_combine(zc, zi, zu, text_scale, image_scale):
+    """Editing guidance with three rows per position (HF-mirror README, note under "SPRINT 加速技术": Editing CFG
+    guides three ways through cfg_text_scale / cfg_image_scale; the formula is not printed on the pages, this is the
+    plain reading): z = z_u + s_i (z_i - z_u) + s_t (z_c - z_i), with z_c the row conditioned on the instruction and
+    the source image, z_i the row conditioned on the image only, z_u the unconditional row; s_t = cfg_text_scale,
+    s_i = cfg_image_scale. In fp64."""
+    zc, zi, zu = f64(zc), f64(zi), f64(zu)
+    return zu + float(image_scale) * (zi - zu) + float(text_scale) * (zc - zi)
+
+
+def cfg3_fp32_error_bound(zc, zi, zu, text_scale, image_scale):
+    """Largest rounding error, per row, of the float32 evaluation a = z_u + s_i (z_i - z_u), z = a + s_t (z_c - z_i)
+    with every operation rounded to nearest: with u = 2^-24, to first order |fl(z) - z| <= u (2 |m_i| + |a| +
+    2 |m_t| + |z|), m_i = s_i (z_i - z_u), m_t = s_t (z_c - z_i) (each difference's error scales with its product);
+    1 % is added for the second-order terms."""
+    zc, zi, zu = f64(zc), f64(zi), f64(zu)
+    mi = float(image_scale) * (zi - zu)
+    mt = float(text_scale) * (zc - zi)
+    a = zu + mi
+    return 1.01 * 2.0 ** -24 * np.max(2.0 * np.abs(mi) + np.abs(a) + 2.0 * np.abs(mt) + np.abs(a + mt), axis=-1)
+
+
 def confidence(z):
     """[R] "SPRINT": c = max_v softmax(z)_v, the candidate token is the lowest argmax.
     z [n, V] -> (cand [n] int64, c [n], lse [n], zmax [n])."""
@@ -358,12 +383,14 @@ def select_positions(conf_row, masked_row, k):
 
 
 def unmask(z_rows, row_pos, tokens, mask, t, T_s, mode=0, tau=0.9, k_max=8, vocab_offset=0,
-           z_uncond=None, cfg_scale=1.0, score="low_confidence"):
+           z_uncond=None, cfg_scale=1.0, score="low_confidence", z_image=None, cfg_image_scale=1.0):
     """One unmasking step over a batch of block rows.
 
     z_rows [n, V]: logits of the still-masked positions, row r belongs to flat position row_pos[r] = b*L + i of
     the conditional rows. With ``z_uncond`` given, the rows are combined by CFG first (fp64), and the selection
-    is written to both halves of the batch (rows b and b + B/2).
+    is written to both halves of the batch (rows b and b + B/2). With ``z_image`` given too (editing guidance), the
+    three rows of a position are combined by cfg3_combine and the selection is written to the three thirds of the
+    batch (rows b, b + B/3, b + 2B/3).
 
     Near-tie flags (decisions a correct implementation may take either way): a confidence margin below 1e-6
     relative between the last chosen and the first unchosen position (tie_rank), a confidence within 1e-6 of tau
@@ -379,8 +406,12 @@ def unmask(z_rows, row_pos, tokens, mask, t, T_s, mode=0, tau=0.9, k_max=8, voca
     tokens = np.array(tokens, dtype=np.int64, copy=True)
     mask = np.array(mask, dtype=np.int64, copy=True)
     B, L = mask.shape
-    Bl = B // 2 if z_uncond is not None else B
-    if z_uncond is not None:
+    groups = 1 if z_uncond is None else (3 if z_image is not None else 2)
+    Bl = B // groups
+    if z_image is not None:
+        z = cfg3_combine(z_rows, z_image, z_uncond, cfg_scale, cfg_image_scale)
+        z_err = cfg3_fp32_error_bound(z_rows, z_image, z_uncond, cfg_scale, cfg_image_scale)
+    elif z_uncond is not None:
         z = cfg_combine(z_rows, z_uncond, cfg_scale)
         z_err = cfg_fp32_error_bound(z_rows, z_uncond, cfg_scale)
     else:
@@ -421,9 +452,9 @@ def unmask(z_rows, row_pos, tokens, mask, t, T_s, mode=0, tau=0.9, k_max=8, voca
         for i in chosen:
             tokens[b, i] = cand[b, i]
             mask[b, i] = 0
-            if z_uncond is not None:
-                tokens[b + Bl, i] = cand[b, i]
-                mask[b + Bl, i] = 0
+            for grp in range(1, groups):   # the guidance rows of the same position take the same token
+                tokens[b + grp * Bl, i] = cand[b, i]
+                mask[b + grp * Bl, i] = 0
         sel.append(chosen)
         nsel[b] = kt
     return dict(tokens=tokens, mask=mask, sel=sel, nsel=nsel, conf=conf, rank=rank, cand=cand,
@@ -492,9 +523,10 @@ def forward_block(w, weights, caches, tokens, mask, keep=None, want_logits=True,
     out["x"] = x.reshape(B, L, H)
     if want_logits:
         xf = store(rmsnorm(x, weights["final_norm"], w.eps), dt)
-        Bl = B // 2 if w.cfg else B
+        groups = 1 + w.cfg   # cfg 1: (cond, uncond) halves; cfg 2 (editing): (cond, image-only, uncond) thirds
+        Bl = B // groups
         row_pos = np.nonzero(np.asarray(mask)[:Bl].reshape(-1))[0]
-        rows = list(row_pos) + ([p + Bl * L for p in row_pos] if w.cfg else [])
+        rows = [p + grp * Bl * L for grp in range(groups) for p in row_pos]
         wl = f64(weights["w_lm"][w.vocab_offset: w.vocab_offset + w.vlen])
         out["logits"] = store(xf[rows] @ wl.T, dt)
         out["row_pos"] = row_pos
@@ -505,9 +537,17 @@ def denoise_step(w, weights, caches, tokens, mask, t, keep=None):
     """One denoising pass at step t: backbone, LM head over the masked rows, confidence, unmasking."""
     f = forward_block(w, weights, caches, tokens, mask, keep=keep)
     n = len(f["row_pos"])
-    zc, zu = (f["logits"][:n], f["logits"][n:]) if w.cfg else (f["logits"], None)
+    z = f["logits"]
+    zi = None
+    if w.cfg == 2:
+        zc, zi, zu = z[:n], z[n:2 * n], z[2 * n:]
+    elif w.cfg:
+        zc, zu = z[:n], z[n:]
+    else:
+        zc, zu = z, None
     u = unmask(zc, f["row_pos"], tokens, mask, t, w.T_s, w.mode, w.tau, w.k_max, w.vocab_offset,
-               z_uncond=zu, cfg_scale=w.cfg_scale, score=SCORES[getattr(w, "score", 0)])
+               z_uncond=zu, cfg_scale=w.cfg_scale, score=SCORES[getattr(w, "score", 0)], z_image=zi,
+               cfg_image_scale=getattr(w, "cfg_image_scale", 1.0))
     u["forward"] = f
     return u
 

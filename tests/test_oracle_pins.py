@@ -403,6 +403,54 @@ def test_unmask_selection_and_writeback():
     assert u["tokens"][1, 2] == 5 and u["mask"][1, 2] == 0
 
 
+def test_cfg3_reduces_to_two_way_guidance():
+    """Editing guidance against the two-way formula and the rows themselves (float32-representable inputs, so every
+    case below is exact in fp64): an image-only row equal to the unconditional one leaves text guidance of the full
+    row; text scale 0 leaves image guidance between the image-only and the unconditional rows; an image-only row
+    equal to the full row leaves two-way guidance with the image scale; both scales 1 give the full row."""
+    zc = rng.standard_normal((3, 40)).astype(np.float32).astype(np.float64)
+    zi = rng.standard_normal((3, 40)).astype(np.float32).astype(np.float64)
+    zu = rng.standard_normal((3, 40)).astype(np.float32).astype(np.float64)
+    assert np.array_equal(O.cfg3_combine(zc, zu, zu, 2.5, 1.5), O.cfg_combine(zc, zu, 2.5))
+    assert np.array_equal(O.cfg3_combine(zc, zi, zu, 0.0, 1.5), O.cfg_combine(zi, zu, 1.5))
+    assert np.array_equal(O.cfg3_combine(zc, zc, zu, 2.5, 1.5), O.cfg_combine(zc, zu, 1.5))
+    assert np.array_equal(O.cfg3_combine(zc, zi, zu, 1.0, 1.0), zc)
+
+
+def test_cfg3_fp32_error_bound_covers_float32_evaluation():
+    """The bound covers a float32 evaluation in the stated order, each operation rounded to nearest, on rows with
+    large and cancelling logits."""
+    g = np.random.default_rng(7)
+    zc = (g.standard_normal((64, 300)) * 20).astype(np.float32)
+    zi = (zc + g.standard_normal((64, 300)).astype(np.float32) * 0.5).astype(np.float32)
+    zu = (g.standard_normal((64, 300)) * 20).astype(np.float32)
+    for st, si in ((4.0, 1.5), (1.0, 1.0), (7.5, 0.25)):
+        st32, si32 = np.float32(st), np.float32(si)
+        a = zu + si32 * (zi - zu)
+        z32 = (a + st32 * (zc - zi)).astype(np.float64)
+        err = np.abs(z32 - O.cfg3_combine(zc, zi, zu, st, si)).max(axis=1)
+        assert np.all(err <= O.cfg3_fp32_error_bound(zc, zi, zu, st, si))
+
+
+def test_unmask_editing_guidance_updates_every_third():
+    """With three rows per position the chosen token is written to the position in all three thirds of the batch,
+    and the choice is that of the guided logits."""
+    B, L, V = 6, 4, 10   # 2 logical rows
+    mask = np.ones((B, L), dtype=np.int64)
+    tokens = np.full((B, L), V - 1, dtype=np.int64)
+    row_pos = np.arange(2 * L)
+    g = np.random.default_rng(3)
+    zc, zi, zu = (g.standard_normal((2 * L, V)) for _ in range(3))
+    u = O.unmask(zc, row_pos, tokens, mask, t=0, T_s=2, mode=0, k_max=8, z_uncond=zu, cfg_scale=3.0, z_image=zi,
+                 cfg_image_scale=1.5)
+    z = O.cfg3_combine(zc, zi, zu, 3.0, 1.5)
+    for b in range(2):
+        for i in u["sel"][b]:
+            want = int(np.argmax(z[b * L + i]))
+            for grp in range(3):
+                assert u["tokens"][b + 2 * grp, i] == want and u["mask"][b + 2 * grp, i] == 0
+
+
 def test_cfg_combine_special_scales():
     zc = rng.standard_normal((3, 50)).astype(np.float32).astype(np.float64)
     zu = rng.standard_normal((3, 50)).astype(np.float32).astype(np.float64)

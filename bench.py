@@ -63,6 +63,7 @@ def bench_config(w, world):
             "weights": "fp8 e4m3 experts + lm head, per-row fp32 scales" if w.wfmt == "fp8" else "bf16",
             "mode": "threshold" if w.mode else "fixed", "tau": w.tau if w.mode else None,
             "k_max": w.k_max if w.mode else None, "cfg": w.cfg_scale if w.cfg else None,
+            **({"cfg_image": w.cfg_image_scale} if w.cfg == 2 else {}),
             "sprint_keep": w.keep_ratio if w.sprint else None,
             "parallelism": f"replicas{world}" if world > 1 else "single",
             "l2": "inputs larger than L2 (weights streamed per pass)"}
@@ -135,7 +136,7 @@ class OracleSample:
         t0 = time.time()
         self.O = O
         self.w = w
-        self.rows = 2 if w.cfg else 1
+        self.rows = 1 + w.cfg
         self.ws = scaled(w, name=w.name + "-sample", n_layers=1, B=self.rows)
         self.wt = synth.make_weights(self.ws, "cpu")
         caches = synth.make_prefix_cache(self.ws, "cpu")
@@ -216,7 +217,7 @@ def block_stats(eng, w, tokens0, mask0):
         return eng.expert_counts(v).cpu()
 
     for t in range(w.T_s):
-        n_masked = int(eng.mask[: (w.B // 2 if w.cfg else w.B)].sum().item())
+        n_masked = int(eng.mask[: w.B // (1 + w.cfg)].sum().item())
         eng.step(t)
         torch.cuda.synchronize()
         live = n_masked > 0
@@ -319,7 +320,7 @@ def measure(args, w, wt, caches, tokens0, mask0, dev, world, local, e2e):
 
     passes, commit_active = block_stats(eng, w, tokens0, mask0)
     live = sum(p["live"] for p in passes)
-    Bl = w.B // 2 if w.cfg else w.B
+    Bl = w.B // (1 + w.cfg)
     value = replicas.aggregate_throughput(w.B * w.L * live * args.steps, elapsed, world)
     committed = replicas.aggregate_throughput(Bl * w.L * args.steps, elapsed, world)
     block_bytes = algorithmic_bytes(w, passes, commit_active)

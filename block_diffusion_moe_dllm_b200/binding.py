@@ -53,7 +53,7 @@ class ExpertDesc(C.Structure):
 class UnmaskDesc(C.Structure):
     _fields_ = [("B", i32), ("L", i32), ("V", i32), ("max_rows", i32), ("t", i32), ("T_s", i32), ("mode", i32),
                 ("tau", f32), ("k_max", i32), ("cfg", i32), ("cfg_scale", f32), ("vocab_offset", i32),
-                ("dtype", i32), ("score", i32)]
+                ("dtype", i32), ("score", i32), ("cfg_image_scale", f32)]
 
 
 class Layer(C.Structure):
@@ -79,7 +79,7 @@ class StepParams(C.Structure):
     _fields_ = [("t", i32), ("T_s", i32), ("mode", i32), ("tau", f32), ("k_max", i32), ("cfg", i32),
                 ("cfg_scale", f32), ("vocab_offset", i32), ("vocab_len", i32), ("sprint", i32), ("n_keep", i32),
                 ("retain", i32), ("commit", i32), ("sel", vp), ("nsel", vp), ("conf", vp), ("remaining", vp),
-                ("score", i32), ("sprint_alpha", f32), ("n_keep_img", i32)]
+                ("score", i32), ("sprint_alpha", f32), ("n_keep_img", i32), ("cfg_image_scale", f32)]
 
 
 class StepViews(C.Structure):
@@ -251,9 +251,10 @@ def moe_experts(h, w_gu, w_down, w_gu_shared, w_down_shared, counts, offsets, pe
 
 def unmask(logits, row_pos, n_rows_dev, tokens, mask, sel, nsel, conf, remaining, B, L, V, max_rows, t, T_s,
            dtype, mode=FIXED, tau=0.9, k_max=8, cfg=0, cfg_scale=1.0, vocab_offset=0, score=SCORE_LOW_CONFIDENCE,
-           ws=None, stream=None):
+           ws=None, stream=None, cfg_image_scale=1.0):
     lib = load()
-    desc = UnmaskDesc(B, L, V, max_rows, t, T_s, mode, tau, k_max, cfg, cfg_scale, vocab_offset, dtype, score)
+    desc = UnmaskDesc(B, L, V, max_rows, t, T_s, mode, tau, k_max, cfg, cfg_scale, vocab_offset, dtype, score,
+                      cfg_image_scale)
     need = lib.dllm_unmask_workspace_size(C.byref(desc))
     ws = (ws or Workspace(need, logits.device)).ensure(need)
     return check(lib.dllm_unmask(C.byref(desc), ptr(logits), ptr(row_pos), ptr(n_rows_dev), ptr(tokens), ptr(mask),

@@ -23,15 +23,16 @@ class Workload:
     k: int                # experts per token
     I: int                # expert intermediate size (routed and shared)
     V: int                # vocabulary rows of the LM head
-    B: int                # batch rows (cond + uncond count as two rows)
+    B: int                # batch rows (each guidance row counts as a row)
     P: int                # cached prefix length before the block
     L: int                # block length
     T_s: int              # denoising steps per block
     mode: int = 0         # 0 = fixed schedule, 1 = threshold acceptance
     tau: float = 0.9
     k_max: int = 8
-    cfg: int = 0          # 1: rows [0, B/2) are conditional, rows [B/2, B) unconditional
-    cfg_scale: float = 2.0
+    cfg: int = 0          # 1: rows [0, B/2) conditional, [B/2, B) unconditional; 2 (editing): rows [0, B/3) on
+                          # instruction and image, [B/3, 2B/3) on the image only, [2B/3, B) unconditional
+    cfg_scale: float = 2.0   # two-way scale, or the text scale of editing guidance
     vocab_offset: int = 0 # first LM-head row scored (image-token slice)
     vocab_len: int = 0    # rows scored; 0 = all V
     sprint: int = 0       # SPRINT prefix retention at the first step of each block
@@ -47,6 +48,13 @@ class Workload:
     sprint_alpha: float = 1.0   # SPRINT importance = alpha * key norm + (1 - alpha) * confidence
     n_img_prefix: int = 0       # > 0: the first n_img_prefix prefix positions are image tokens (modality counts)
     img_keep_ratio: float = 1.0 # with image positions: keep ceil(ratio * n_img) of them, the rest of n_keep text
+    cfg_image_scale: float = 1.0  # editing guidance (cfg 2): the image scale
+
+    def __post_init__(self):
+        # SPRINT serves no guidance and two-way guidance; under editing guidance it falls back to the plain decode on
+        # the full caches (HF-mirror README, note under "SPRINT 加速技术")
+        if self.cfg == 2 and self.sprint:
+            object.__setattr__(self, "sprint", 0)
 
     @property
     def Tk(self) -> int:
@@ -92,6 +100,13 @@ ONE_LAYER = Workload("moe-dllm-1layer-p1024-b1", "bf16", 1, 2048, 16, 4, 128, 25
 T2I = Workload("t2i-20layer-cfg2-b2", "bf16", 20, 2048, 16, 4, 128, 256, 8, 512, 157184, 2, 256 + 2048, 32, 8,
                cfg=1, cfg_scale=2.0, vocab_offset=157184 - 16384, vocab_len=16384)
 
+# image editing: 20 layers, three guidance rows (instruction and image, image only, unconditional), a 512 x 512
+# source image as 256 tokens plus a 64-token instruction in the prefix, the 256 output image tokens in blocks of 32
+# at 8 steps per block with text scale 4.0 (the README's editing example) and image scale 1.0; the middle block
+# (128 output tokens committed) is the representative one
+EDIT = Workload("edit-20layer-cfg3-b3", "bf16", 20, 2048, 16, 4, 128, 256, 8, 512, 157184, 3, 64 + 256 + 128, 32, 8,
+                cfg=2, cfg_scale=4.0, cfg_image_scale=1.0, vocab_offset=157184 - 16384, vocab_len=16384)
+
 # thinking mode: 20 layers, batch 8, 4096-token prefix, SPRINT keeps 50 % of the prefix by key norm,
 # 32 steps per block
 THINKING = Workload("thinking-20layer-b8-p4096-sprint50", "bf16", 20, 2048, 16, 4, 128, 256, 8, 512, 157184, 8,
@@ -113,7 +128,7 @@ UNDERSTANDING_FP8 = replace(UNDERSTANDING, name="understanding-20layer-b16-p2688
 # step's kernels takes (a few GB on the device)
 UNDERSTANDING_1LAYER = replace(UNDERSTANDING, name="understanding-1layer-b16-p2688-thr0.9", n_layers=1)
 
-ALL = [TINY_F32, ONE_LAYER, T2I, THINKING, UNDERSTANDING, PREFILL, ONE_LAYER_FP8, UNDERSTANDING_FP8,
+ALL = [TINY_F32, ONE_LAYER, T2I, EDIT, THINKING, UNDERSTANDING, PREFILL, ONE_LAYER_FP8, UNDERSTANDING_FP8,
        UNDERSTANDING_1LAYER]
 BY_NAME = {w.name: w for w in ALL}
 

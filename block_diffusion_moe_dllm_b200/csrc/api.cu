@@ -217,7 +217,10 @@ int validate_step(const dllm_model* m, const dllm_state* st, const dllm_step_par
   REQ(p->mode == DLLM_UNMASK_FIXED || p->mode == DLLM_UNMASK_THRESHOLD, DLLM_ERR_INVALID_ARG, "bad unmask mode");
   REQ(p->score >= DLLM_SCORE_LOW_CONFIDENCE && p->score <= DLLM_SCORE_NEG_ENTROPY, DLLM_ERR_INVALID_ARG,
       "denoise_step: bad score %d", p->score);
-  REQ(!p->cfg || st->B % 2 == 0, DLLM_ERR_SHAPE, "denoise_step: cfg needs an even number of rows");
+  REQ(p->cfg >= 0 && p->cfg <= 2, DLLM_ERR_INVALID_ARG, "denoise_step: cfg %d (0, 1 or 2)", p->cfg);
+  REQ(st->B % (1 + p->cfg) == 0, DLLM_ERR_SHAPE, "denoise_step: cfg %d needs B a multiple of %d", p->cfg, 1 + p->cfg);
+  REQ(p->cfg != 2 || !p->sprint, DLLM_ERR_UNSUPPORTED,
+      "denoise_step: SPRINT with editing guidance (cfg 2) is not supported; run those blocks on the full caches");
   const int vlen = p->vocab_len ? p->vocab_len : m->V;
   REQ(p->vocab_offset >= 0 && p->vocab_offset + vlen <= m->V, DLLM_ERR_SHAPE, "denoise_step: vocab slice out of range");
   if (p->sprint) {
@@ -277,7 +280,7 @@ void plan_step(const dllm_model* m, const dllm_state* st, const dllm_step_params
   const int es = esize(m->dtype);
   s.B = st->B;
   s.L = st->L;
-  s.halves = p->cfg ? 2 : 1;
+  s.halves = 1 + p->cfg;   // row groups: (cond), (cond, uncond) or (cond, image only, uncond)
   s.Bl = st->B / s.halves;
   s.Tk = st->B * st->L;
   s.vlen = p->vocab_len ? p->vocab_len : m->V;
@@ -607,6 +610,7 @@ int dllm_unmask(const dllm_unmask_desc* d, const void* logits, const int32_t* ro
   REQ(d->mode == DLLM_UNMASK_FIXED || d->k_max >= 1, DLLM_ERR_INVALID_ARG, "unmask: k_max must be >= 1");
   REQ(d->dtype == DLLM_BF16 || d->dtype == DLLM_F32, DLLM_ERR_INVALID_ARG, "unmask: bad dtype");
   REQ(d->vocab_offset >= 0, DLLM_ERR_INVALID_ARG, "unmask: negative vocab_offset");
+  REQ(d->cfg >= 0 && d->cfg <= 2, DLLM_ERR_INVALID_ARG, "unmask: cfg %d (0, 1 or 2)", d->cfg);
   REQ(d->score >= DLLM_SCORE_LOW_CONFIDENCE && d->score <= DLLM_SCORE_NEG_ENTROPY, DLLM_ERR_INVALID_ARG,
       "unmask: bad score %d", d->score);
   int st = check_ws(ws, ws_bytes, dllm_unmask_workspace_size(d));
@@ -615,7 +619,7 @@ int dllm_unmask(const dllm_unmask_desc* d, const void* logits, const int32_t* ro
   UnmaskArgs a;
   a.B = d->B; a.L = d->L; a.V = d->V; a.max_rows = d->max_rows; a.t = d->t; a.T_s = d->T_s; a.mode = d->mode;
   a.k_max = d->k_max; a.cfg = d->cfg; a.vocab_offset = d->vocab_offset; a.dtype = d->dtype; a.tau = d->tau;
-  a.cfg_scale = d->cfg_scale; a.logits = logits; a.row_pos = row_pos; a.n_rows = n_rows_dev; a.tokens = tokens;
+  a.cfg_scale = d->cfg_scale; a.cfg_image_scale = d->cfg_image_scale; a.logits = logits; a.row_pos = row_pos; a.n_rows = n_rows_dev; a.tokens = tokens;
   a.mask = mask; a.sel = sel; a.nsel = nsel; a.conf = conf; a.remaining = remaining;
   a.n_chunks = unmask_chunks(d->max_rows, d->V);
   a.partials = c.take(unmask_partials_bytes(d->max_rows, a.n_chunks));
@@ -757,10 +761,10 @@ int denoise_step_impl(const dllm_model* m, const dllm_state* st, const dllm_step
                     counts, s.offsets, s.perm, s.inv, s.gates, s.x, s.eb, status, stream, pn, live, esc));
   }
   if (p->commit) return DLLM_OK;
-  // final norm on the masked rows (cond, then uncond) unless fused above, LM head, confidence + unmasking
+  // final norm on the masked rows (one group after the other) unless fused above, LM head, confidence + unmasking
   if (!fuse)
     TRY(launch_rmsnorm(dt, s.x, m->final_norm, s.xf, s.halves * s.max_rows, H, m->eps, s.row_pos, s.n_rows,
-                       p->cfg, s.Bl * L, stream));
+                       s.halves, s.Bl * L, stream));
   GemmArgs gl;
   gl.x = s.xf; gl.x_rows = (int64_t)s.halves * s.max_rows;
   const bool lm_fp8 = m->weight_format == DLLM_WEIGHTS_FP8;
@@ -779,7 +783,8 @@ int denoise_step_impl(const dllm_model* m, const dllm_state* st, const dllm_step
   UnmaskArgs ua;
   ua.B = s.Bl; ua.L = L; ua.V = s.vlen; ua.max_rows = s.max_rows; ua.t = p->t; ua.T_s = p->T_s; ua.mode = p->mode;
   ua.k_max = p->k_max; ua.cfg = p->cfg; ua.vocab_offset = p->vocab_offset; ua.dtype = dt; ua.tau = p->tau;
-  ua.cfg_scale = p->cfg_scale; ua.logits = s.logits; ua.row_pos = s.row_pos; ua.n_rows = s.n_rows;
+  ua.cfg_scale = p->cfg_scale; ua.cfg_image_scale = p->cfg_image_scale; ua.logits = s.logits; ua.row_pos = s.row_pos;
+  ua.n_rows = s.n_rows;
   ua.tokens = st->tokens; ua.mask = st->mask; ua.sel = p->sel; ua.nsel = p->nsel; ua.conf = p->conf;
   ua.remaining = p->remaining; ua.partials = s.partials;
   ua.n_chunks = s.conf_parts ? s.conf_parts : s.n_chunks;

@@ -34,20 +34,21 @@ int launch_embed(int dtype, const int32_t* tokens, const uint8_t* mask, int mask
 
 // ------------------------------------------------------------------------------------------------ RMSNorm
 // out[r] = x[src(r)] / sqrt(mean(x^2) + eps) * g, fp32 math. src(r) = r, or through a compacted row list:
-// rows r < n come from row_pos[r], rows n <= r < 2n from row_pos[r - n] + uncond_off (n = *n_dev).
+// row r = g * n + j (n = *n_dev, group g < groups) comes from row_pos[j] + g * group_off.
 template <typename T>
 __global__ void __launch_bounds__(256) rmsnorm_kernel(const T* __restrict__ x, const T* __restrict__ g,
                                                       T* __restrict__ out, int H, float eps,
                                                       const int32_t* __restrict__ row_pos,
-                                                      const int32_t* __restrict__ n_dev, int two_halves,
-                                                      int uncond_off) {
+                                                      const int32_t* __restrict__ n_dev, int groups,
+                                                      int group_off) {
   pdl_enter();
   int r = blockIdx.x;
   int src = r;
   if (row_pos) {
     const int n = *n_dev;
-    if (r >= n * (two_halves ? 2 : 1)) return;
-    src = (r < n) ? row_pos[r] : row_pos[r - n] + uncond_off;
+    if (r >= n * groups) return;
+    const int g = r / n;
+    src = row_pos[r - g * n] + g * group_off;
   }
   const T* xr = x + (int64_t)src * H;
   T* o = out + (int64_t)r * H;
@@ -110,15 +111,15 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const T* __restrict__ x, c
 }
 
 int launch_rmsnorm(int dtype, const void* x, const void* g, void* out, int rows, int H, float eps,
-                   const int32_t* row_pos, const int32_t* n_dev, int two_halves, int uncond_off, cudaStream_t s) {
+                   const int32_t* row_pos, const int32_t* n_dev, int groups, int group_off, cudaStream_t s) {
   if (rows <= 0) return DLLM_OK;
   if (dtype == DLLM_BF16)
     launch_pdl(rmsnorm_kernel<__nv_bfloat16>, rows, 256, 0, s, (const __nv_bfloat16*)x, (const __nv_bfloat16*)g,
-                                                       (__nv_bfloat16*)out, H, eps, row_pos, n_dev, two_halves,
-                                                       uncond_off);
+                                                       (__nv_bfloat16*)out, H, eps, row_pos, n_dev, groups,
+                                                       group_off);
   else
     launch_pdl(rmsnorm_kernel<float>, rows, 256, 0, s, (const float*)x, (const float*)g, (float*)out, H, eps, row_pos,
-                                               n_dev, two_halves, uncond_off);
+                                               n_dev, groups, group_off);
   DLLM_CHECK_LAUNCH("rmsnorm_kernel");
   return DLLM_OK;
 }

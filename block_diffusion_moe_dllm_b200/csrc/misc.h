@@ -9,7 +9,7 @@ namespace dllm {
 int launch_embed(int dtype, const int32_t* tokens, const uint8_t* mask, int mask_id, const void* table, void* x,
                  int rows, int H, cudaStream_t s);
 int launch_rmsnorm(int dtype, const void* x, const void* g, void* out, int rows, int H, float eps,
-                   const int32_t* row_pos, const int32_t* n_dev, int two_halves, int uncond_off, cudaStream_t s);
+                   const int32_t* row_pos, const int32_t* n_dev, int groups, int group_off, cudaStream_t s);
 int launch_masked_rows(const uint8_t* mask, int n_pos, int halves, int32_t* row_pos, int32_t* n_out,
                        cudaStream_t s);
 // live (nullable, every launcher below that takes it): device word; 0 = the denoising pass has no masked position
@@ -74,6 +74,7 @@ struct UnmaskArgs {
   void* extras = nullptr;        // score != 0: max_rows * n_chunks ConfExtra, then B * L floats of ranking scores
   float* conf_hist = nullptr;    // nullable: accepted positions' confidences at conf_hist[row * stride + off + i]
   int conf_hist_stride = 0, conf_hist_off = 0;
+  float cfg_image_scale = 1.f;   // cfg 2: the image scale s_i of the editing guidance (cfg_scale is s_t)
 };
 int unmask_chunks(int max_rows, int V);
 size_t unmask_partials_bytes(int max_rows, int n_chunks);

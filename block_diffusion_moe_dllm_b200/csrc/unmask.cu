@@ -46,6 +46,21 @@ DLLM_DEV float guided(float zc, float zu, float s) {
   return __fadd_rn(zu, __fmul_rn(s, __fsub_rn(zc, zu)));
 }
 
+DLLM_DEV float guided3(float zc, float zi, float zu, float st, float si) {
+  // editing guidance: a = zu + si * (zi - zu), z = a + st * (zc - zi), each operation rounded to fp32 in this order
+  const float a = __fadd_rn(zu, __fmul_rn(si, __fsub_rn(zi, zu)));
+  return __fadd_rn(a, __fmul_rn(st, __fsub_rn(zc, zi)));
+}
+
+// The guided value of one vocabulary entry from the rows of its position: CFG 0 the row itself; CFG 1 the pair
+// (z1 = unconditional) with scale st; CFG 2 the triple (z1 = image only, z2 = unconditional) with scales st, si.
+template <int CFG>
+DLLM_DEV float guide(float zc, float z1, float z2, float st, float si) {
+  if constexpr (CFG == 1) return guided(zc, z1, st);
+  else if constexpr (CFG == 2) return guided3(zc, z1, z2, st, si);
+  else return zc;
+}
+
 // The hardware base-2 exponential (ex2.approx.ftz: relative error about 2^-22, results below 2^-126 flushed to 0,
 // which against a maximum term of 1 is far below fp32 resolution). Sums and scalings of fp32 pairs use the sm_100
 // packed instructions (__fadd2_rn / __fmul2_rn: one issue for two lanes' worth).
@@ -92,17 +107,19 @@ DLLM_DEV void load8f(const float* p, float* f) {
   f[4] = __uint_as_float(b.x); f[5] = __uint_as_float(b.y); f[6] = __uint_as_float(b.z); f[7] = __uint_as_float(b.w);
 }
 
-template <typename T, bool CFG>
+// Rows of the guidance: the position's row r among the n_rows of each group, group g at rows [g * n, (g + 1) * n).
+template <typename T, int CFG>
 __global__ void __launch_bounds__(256) unmask_reduce_kernel(const T* __restrict__ logits,
                                                             const int32_t* __restrict__ n_rows, int max_rows, int V,
-                                                            int chunk, float cfg_scale, Partial* __restrict__ part,
+                                                            int chunk, float st, float si, Partial* __restrict__ part,
                                                             int n_chunks) {
   pdl_enter();
   const int r = blockIdx.x, c = blockIdx.y;
   const int n = min(*n_rows, max_rows);   // the device count never exceeds the rows the buffers hold
   if (r >= n) return;
   const T* zc = logits + (int64_t)r * V;
-  const T* zu = logits + (int64_t)(r + n) * V;
+  const T* z1 = logits + (int64_t)(r + n) * V;
+  const T* z2 = logits + (int64_t)(r + 2 * n) * V;   // read only with CFG 2
   const int v0 = c * chunk, v1 = min(V, v0 + chunk);
   Partial p{-INFINITY, 0x7fffffff, 0.0};
   const int nvec = (v1 - v0) >> 3;
@@ -114,12 +131,23 @@ __global__ void __launch_bounds__(256) unmask_reduce_kernel(const T* __restrict_
       float a[8], b[8];
       load8f(zc + v0 + i * 8, a);
       load8f(zc + v0 + (i + 256) * 8, b);
-      if (CFG) {
+      if constexpr (CFG == 1) {
         float ua[8], ub[8];
-        load8f(zu + v0 + i * 8, ua);
-        load8f(zu + v0 + (i + 256) * 8, ub);
+        load8f(z1 + v0 + i * 8, ua);
+        load8f(z1 + v0 + (i + 256) * 8, ub);
 #pragma unroll
-        for (int u = 0; u < 8; ++u) { a[u] = guided(a[u], ua[u], cfg_scale); b[u] = guided(b[u], ub[u], cfg_scale); }
+        for (int u = 0; u < 8; ++u) { a[u] = guided(a[u], ua[u], st); b[u] = guided(b[u], ub[u], st); }
+      } else if constexpr (CFG == 2) {
+        float ia[8], ib[8], ua[8], ub[8];
+        load8f(z1 + v0 + i * 8, ia);
+        load8f(z1 + v0 + (i + 256) * 8, ib);
+        load8f(z2 + v0 + i * 8, ua);
+        load8f(z2 + v0 + (i + 256) * 8, ub);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          a[u] = guided3(a[u], ia[u], ua[u], st, si);
+          b[u] = guided3(b[u], ib[u], ub[u], st, si);
+        }
       }
       update8(p, a, v0 + i * 8);
       update8(p, b, v0 + (i + 256) * 8);
@@ -127,19 +155,24 @@ __global__ void __launch_bounds__(256) unmask_reduce_kernel(const T* __restrict_
     for (; i < nvec; i += 256) {
       float a[8];
       load8f(zc + v0 + i * 8, a);
-      if (CFG) {
+      if constexpr (CFG == 1) {
         float ua[8];
-        load8f(zu + v0 + i * 8, ua);
+        load8f(z1 + v0 + i * 8, ua);
 #pragma unroll
-        for (int u = 0; u < 8; ++u) a[u] = guided(a[u], ua[u], cfg_scale);
+        for (int u = 0; u < 8; ++u) a[u] = guided(a[u], ua[u], st);
+      } else if constexpr (CFG == 2) {
+        float ia[8], ua[8];
+        load8f(z1 + v0 + i * 8, ia);
+        load8f(z2 + v0 + i * 8, ua);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) a[u] = guided3(a[u], ia[u], ua[u], st, si);
       }
       update8(p, a, v0 + i * 8);
     }
   }
   // scalar part: the whole chunk when vector loads are not possible, else the tail
   for (int v = v0 + (vec_ok ? nvec * 8 : 0) + threadIdx.x; v < v1; v += 256) {
-    float z = to_f32(zc[v]);
-    if (CFG) z = guided(z, to_f32(zu[v]), cfg_scale);
+    const float z = guide<CFG>(to_f32(zc[v]), CFG ? to_f32(z1[v]) : 0.f, CFG == 2 ? to_f32(z2[v]) : 0.f, st, si);
     Partial q{z, v, 1.0};
     merge(p, q);
   }
@@ -227,10 +260,10 @@ DLLM_DEV ExtPartial ext_warp_merge(ExtPartial p) {
 
 // CTA per (row, chunk), any storage type, optional guidance: the extended partial of the chunk, stored as the
 // ConfPartial (m, idx, s) and its ConfExtra (m2, t).
-template <typename T, bool CFG>
+template <typename T, int CFG>
 __global__ void __launch_bounds__(256) unmask_reduce_ext_kernel(const T* __restrict__ logits,
                                                                 const int32_t* __restrict__ n_rows, int max_rows,
-                                                                int V, int chunk, float cfg_scale,
+                                                                int V, int chunk, float st, float si,
                                                                 Partial* __restrict__ part,
                                                                 ConfExtra* __restrict__ extra, int n_chunks) {
   pdl_enter();
@@ -238,12 +271,12 @@ __global__ void __launch_bounds__(256) unmask_reduce_ext_kernel(const T* __restr
   const int n = min(*n_rows, max_rows);
   if (r >= n) return;
   const T* zc = logits + (int64_t)r * V;
-  const T* zu = logits + (int64_t)(r + n) * V;
+  const T* z1 = logits + (int64_t)(r + n) * V;
+  const T* z2 = logits + (int64_t)(r + 2 * n) * V;   // read only with CFG 2
   const int v0 = c * chunk, v1 = min(V, v0 + chunk);
   ExtPartial p = ext_empty();
   for (int v = v0 + threadIdx.x; v < v1; v += 256) {
-    float z = to_f32(zc[v]);
-    if (CFG) z = guided(z, to_f32(zu[v]), cfg_scale);
+    const float z = guide<CFG>(to_f32(zc[v]), CFG ? to_f32(z1[v]) : 0.f, CFG == 2 ? to_f32(z2[v]) : 0.f, st, si);
     ext_add(p, z, v);
   }
   p = ext_warp_merge(p);
@@ -469,13 +502,12 @@ __global__ void __launch_bounds__(1024) unmask_select_kernel(Partial* part, int 
       sel[b * L + rnk] = lane;
       tokens[p] = cand;
       mask[p] = 0;
-      if (cfg) {
-        tokens[p + B * L] = cand;
-        mask[p + B * L] = 0;
+      for (int g = 1; g <= cfg; ++g) {   // the guidance rows of the position take the same token
+        tokens[p + g * B * L] = cand;
+        mask[p + g * B * L] = 0;
       }
       if (conf_hist) {   // the accepted position's confidence, for the importance of later SPRINT selections
-        conf_hist[(int64_t)b * hist_stride + hist_off + lane] = c;
-        if (cfg) conf_hist[(int64_t)(b + B) * hist_stride + hist_off + lane] = c;
+        for (int g = 0; g <= cfg; ++g) conf_hist[(int64_t)(b + g * B) * hist_stride + hist_off + lane] = c;
       }
     }
     if (lane == 0) {
@@ -515,6 +547,24 @@ size_t unmask_extras_bytes(int score, int max_rows, int n_chunks, int B, int L) 
   return ex + (size_t)B * L * sizeof(float);
 }
 
+// The reduction kernels for the guidance mode a.cfg (0 none, 1 two-way, 2 editing).
+template <typename T>
+void launch_reduce(const T* z, const UnmaskArgs& a, dim3 grid, int chunk, Partial* part, cudaStream_t s) {
+  const float st = a.cfg_scale, si = a.cfg_image_scale;
+  if (a.cfg == 2) launch_pdl((unmask_reduce_kernel<T, 2>), grid, 256, 0, s, z, a.n_rows, a.max_rows, a.V, chunk, st, si, part, a.n_chunks);
+  else if (a.cfg == 1) launch_pdl((unmask_reduce_kernel<T, 1>), grid, 256, 0, s, z, a.n_rows, a.max_rows, a.V, chunk, st, si, part, a.n_chunks);
+  else launch_pdl((unmask_reduce_kernel<T, 0>), grid, 256, 0, s, z, a.n_rows, a.max_rows, a.V, chunk, st, si, part, a.n_chunks);
+}
+
+template <typename T>
+void launch_reduce_ext(const T* z, const UnmaskArgs& a, dim3 grid, int chunk, Partial* part, ConfExtra* extra,
+                       cudaStream_t s) {
+  const float st = a.cfg_scale, si = a.cfg_image_scale;
+  if (a.cfg == 2) launch_pdl((unmask_reduce_ext_kernel<T, 2>), grid, 256, 0, s, z, a.n_rows, a.max_rows, a.V, chunk, st, si, part, extra, a.n_chunks);
+  else if (a.cfg == 1) launch_pdl((unmask_reduce_ext_kernel<T, 1>), grid, 256, 0, s, z, a.n_rows, a.max_rows, a.V, chunk, st, si, part, extra, a.n_chunks);
+  else launch_pdl((unmask_reduce_ext_kernel<T, 0>), grid, 256, 0, s, z, a.n_rows, a.max_rows, a.V, chunk, st, si, part, extra, a.n_chunks);
+}
+
 int launch_unmask(const UnmaskArgs& a, cudaStream_t s) {
   const int chunk = ((a.V + a.n_chunks - 1) / a.n_chunks + 7) & ~7;
   const bool ext = a.score != DLLM_SCORE_LOW_CONFIDENCE;
@@ -530,22 +580,15 @@ int launch_unmask(const UnmaskArgs& a, cudaStream_t s) {
   if (a.max_rows > 0 && ext) {
     dim3 grid(a.max_rows, a.n_chunks);
     Partial* part = static_cast<Partial*>(a.partials);
-    if (a.dtype == DLLM_BF16) {
-      const __nv_bfloat16* z = static_cast<const __nv_bfloat16*>(a.logits);
-      if (a.cfg) launch_pdl((unmask_reduce_ext_kernel<__nv_bfloat16, true>), grid, 256, 0, s, z, a.n_rows, a.max_rows, a.V, chunk, a.cfg_scale, part, extra, a.n_chunks);
-      else launch_pdl((unmask_reduce_ext_kernel<__nv_bfloat16, false>), grid, 256, 0, s, z, a.n_rows, a.max_rows, a.V, chunk, a.cfg_scale, part, extra, a.n_chunks);
-    } else {
-      const float* z = static_cast<const float*>(a.logits);
-      if (a.cfg) launch_pdl((unmask_reduce_ext_kernel<float, true>), grid, 256, 0, s, z, a.n_rows, a.max_rows, a.V, chunk, a.cfg_scale, part, extra, a.n_chunks);
-      else launch_pdl((unmask_reduce_ext_kernel<float, false>), grid, 256, 0, s, z, a.n_rows, a.max_rows, a.V, chunk, a.cfg_scale, part, extra, a.n_chunks);
-    }
+    if (a.dtype == DLLM_BF16) launch_reduce_ext(static_cast<const __nv_bfloat16*>(a.logits), a, grid, chunk, part, extra, s);
+    else launch_reduce_ext(static_cast<const float*>(a.logits), a, grid, chunk, part, extra, s);
     DLLM_CHECK_LAUNCH("unmask_reduce_ext_kernel");
   } else if (a.max_rows > 0 && !a.partials_ready) {
     dim3 grid(a.max_rows, a.n_chunks);
     Partial* part = static_cast<Partial*>(a.partials);
     if (a.dtype == DLLM_BF16) {
       const __nv_bfloat16* z = static_cast<const __nv_bfloat16*>(a.logits);
-      if (a.cfg) launch_pdl((unmask_reduce_kernel<__nv_bfloat16, true>), grid, 256, 0, s, z, a.n_rows, a.max_rows, a.V, chunk, a.cfg_scale, part, a.n_chunks);
+      if (a.cfg) launch_reduce(z, a, grid, chunk, part, s);
       else if (a.V % 8 == 0 && chunk <= kRegChunk) {
         // the shallowest register depth that holds a thread's share of the chunk
         const int vpt = (chunk / 8 + 255) / 256;
@@ -555,11 +598,9 @@ int launch_unmask(const UnmaskArgs& a, cudaStream_t s) {
         else if (vpt <= 12) launch_pdl(unmask_reduce_bf16_kernel<12>, g2, 256, 0, s, z, a.n_rows, a.max_rows, a.V, chunk, part, a.n_chunks);
         else launch_pdl(unmask_reduce_bf16_kernel<16>, g2, 256, 0, s, z, a.n_rows, a.max_rows, a.V, chunk, part, a.n_chunks);
       }
-      else launch_pdl((unmask_reduce_kernel<__nv_bfloat16, false>), grid, 256, 0, s, z, a.n_rows, a.max_rows, a.V, chunk, a.cfg_scale, part, a.n_chunks);
+      else launch_reduce(z, a, grid, chunk, part, s);
     } else {
-      const float* z = static_cast<const float*>(a.logits);
-      if (a.cfg) launch_pdl((unmask_reduce_kernel<float, true>), grid, 256, 0, s, z, a.n_rows, a.max_rows, a.V, chunk, a.cfg_scale, part, a.n_chunks);
-      else launch_pdl((unmask_reduce_kernel<float, false>), grid, 256, 0, s, z, a.n_rows, a.max_rows, a.V, chunk, a.cfg_scale, part, a.n_chunks);
+      launch_reduce(static_cast<const float*>(a.logits), a, grid, chunk, part, s);
     }
     DLLM_CHECK_LAUNCH("unmask_reduce_kernel");
   }

@@ -62,6 +62,7 @@ extern "C" int dllm_unmask_noalloc(const dllm_unmask_desc* d, const void* logits
   DLLM_REQUIRE(d->mode == DLLM_UNMASK_FIXED || d->k_max >= 1, DLLM_ERR_INVALID_ARG, "unmask_noalloc: k_max must be >= 1");
   DLLM_REQUIRE(d->dtype == DLLM_BF16 || d->dtype == DLLM_F32, DLLM_ERR_INVALID_ARG, "unmask_noalloc: bad dtype");
   DLLM_REQUIRE(d->vocab_offset >= 0, DLLM_ERR_INVALID_ARG, "unmask_noalloc: negative vocab_offset");
+  DLLM_REQUIRE(d->cfg >= 0 && d->cfg <= 2, DLLM_ERR_INVALID_ARG, "unmask_noalloc: cfg %d (0, 1 or 2)", d->cfg);
   DLLM_REQUIRE(d->score >= DLLM_SCORE_LOW_CONFIDENCE && d->score <= DLLM_SCORE_NEG_ENTROPY, DLLM_ERR_INVALID_ARG,
                "unmask_noalloc: bad score %d", d->score);
   const int n_chunks = unmask_chunks(d->max_rows, d->V);
@@ -76,7 +77,7 @@ extern "C" int dllm_unmask_noalloc(const dllm_unmask_desc* d, const void* logits
   UnmaskArgs a;
   a.B = d->B; a.L = d->L; a.V = d->V; a.max_rows = d->max_rows; a.t = d->t; a.T_s = d->T_s; a.mode = d->mode;
   a.k_max = d->k_max; a.cfg = d->cfg; a.vocab_offset = d->vocab_offset; a.dtype = d->dtype; a.tau = d->tau;
-  a.cfg_scale = d->cfg_scale; a.logits = logits; a.row_pos = row_pos; a.n_rows = n_rows_dev; a.tokens = tokens;
+  a.cfg_scale = d->cfg_scale; a.cfg_image_scale = d->cfg_image_scale; a.logits = logits; a.row_pos = row_pos; a.n_rows = n_rows_dev; a.tokens = tokens;
   a.mask = mask; a.sel = sel; a.nsel = nsel; a.conf = conf; a.remaining = remaining;
   a.partials = scratch;
   a.n_chunks = n_chunks;

@@ -63,7 +63,7 @@ class DenoiseEngine:
             self.prefix_modality[: w.n_img_prefix] = 1
         self.state = bd.State(w.B, w.L, w.P, self.cap, self.cap_thin, bd.ptr(self.tokens), bd.ptr(self.mask),
                               bd.ptr(self.prefix_conf), bd.ptr(self.prefix_modality))
-        Bl = w.B // 2 if w.cfg else w.B
+        Bl = w.B // (1 + w.cfg)
         self.sel = torch.full((Bl, w.L), -1, dtype=torch.int32, device=device)
         self.nsel = torch.zeros(Bl, dtype=torch.int32, device=device)
         self.conf = torch.zeros((Bl, w.L), dtype=torch.float32, device=device)
@@ -84,7 +84,7 @@ class DenoiseEngine:
         return bd.StepParams(t, w.T_s, w.mode, w.tau, w.k_max, w.cfg, w.cfg_scale, w.vocab_offset, w.vocab_len,
                              w.sprint, w.n_keep if w.sprint else 0, int(retain), int(commit), bd.ptr(self.sel),
                              bd.ptr(self.nsel), bd.ptr(self.conf), bd.ptr(self.remaining), w.score, w.sprint_alpha,
-                             w.n_keep_img)
+                             w.n_keep_img, w.cfg_image_scale)
 
     def set_block(self, tokens, mask):
         self.tokens.copy_(tokens)
@@ -139,7 +139,7 @@ class DenoiseEngine:
         """The last pass's logits [rows, vlen] as a tensor view of the workspace."""
         w = self.w
         v = self.views()
-        halves = 2 if w.cfg else 1
+        halves = 1 + w.cfg
         numel = halves * n_rows * w.vlen
         dt = torch_dtype(w.dtype)
         return _device_view(v.logits, numel, dt, self.ws.buf).reshape(halves * n_rows, w.vlen)

@@ -78,7 +78,7 @@ def wbytes(w: Workload):
 
 
 def bench_lm_head(w: Workload, reps, dev, stream, weights=None):
-    rows = (2 if w.cfg else 1) * (w.B // (2 if w.cfg else 1)) * w.L
+    rows = w.B * w.L   # every guidance group's rows
     if weights:
         wl, sc = weights["w_lm"], weights.get("w_lm_scale")
     else:
@@ -207,9 +207,9 @@ def bench_expert_gemms(w: Workload, reps, dev, stream, weights=None, routing="ro
 
 
 def bench_unmask(w: Workload, reps, dev, stream):
-    Bl = w.B // 2 if w.cfg else w.B
+    Bl = w.B // (1 + w.cfg)
     n = Bl * w.L
-    logits = synth.normal(((2 if w.cfg else 1) * n, w.vlen), 3.0, 3, "kb_logits", dev)
+    logits = synth.normal(((1 + w.cfg) * n, w.vlen), 3.0, 3, "kb_logits", dev)
     row_pos = torch.arange(n, dtype=torch.int32, device=dev)
     n_dev = torch.tensor([n], dtype=torch.int32, device=dev)
     tok = torch.zeros((w.B, w.L), dtype=torch.int32, device=dev)
@@ -225,7 +225,7 @@ def bench_unmask(w: Workload, reps, dev, stream):
         msk.copy_(msk0)
         bd.unmask(logits, row_pos, n_dev, tok, msk, sel, nsel, conf, rem, Bl, w.L, w.vlen, n, 0, w.T_s, bd.BF16,
                   mode=w.mode, tau=w.tau, k_max=w.k_max, cfg=w.cfg, cfg_scale=w.cfg_scale,
-                  vocab_offset=w.vocab_offset, ws=ws)
+                  vocab_offset=w.vocab_offset, ws=ws, cfg_image_scale=w.cfg_image_scale)
     t = timed(call, reps, stream)
     nbytes = logits.numel() * 2
     return _result("unmask[reduce+select]", t, nbytes, {"rows": n, "V": w.vlen})

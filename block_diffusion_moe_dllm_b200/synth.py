@@ -131,7 +131,8 @@ def make_prefix_cache(w: Workload, device="cpu", seed=None, cap=None):
 
 
 def make_block_state(w: Workload, device="cpu", seed=None, masked_fraction=1.0):
-    """Block tokens [B, L] int32 and mask [B, L] uint8. In cfg workloads both halves share one pattern."""
+    """Block tokens [B, L] int32 and mask [B, L] uint8. In guided workloads every row group (halves with cfg 1,
+    thirds with cfg 2) shares the first group's pattern."""
     s = w.seed if seed is None else seed
     tokens = randint((w.B, w.L), 0, w.V - 1, s, "block_tokens", device)
     if masked_fraction >= 1.0:
@@ -140,9 +141,10 @@ def make_block_state(w: Workload, device="cpu", seed=None, masked_fraction=1.0):
         u = uniform((w.B, w.L), 0.0, 1.0, s, "block_mask", device)
         mask = (u < masked_fraction).to(torch.uint8)
     if w.cfg:
-        half = w.B // 2
-        mask[half:] = mask[:half]
-        tokens[half:] = tokens[:half]
+        Bl = w.B // (1 + w.cfg)
+        for g in range(1, 1 + w.cfg):
+            mask[g * Bl:(g + 1) * Bl] = mask[:Bl]
+            tokens[g * Bl:(g + 1) * Bl] = tokens[:Bl]
     tokens = torch.where(mask.bool(), torch.full_like(tokens, w.mask_id), tokens)
     return tokens, mask
 

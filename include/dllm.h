@@ -251,11 +251,16 @@ DLLM_API size_t dllm_moe_experts_workspace_size(const dllm_expert_desc* desc);
  * Confidence and unmasking ([R] "SPRINT — 학습 없는 추론 가속": c = max_v p(v | x_t), accept every c > tau, at
  * least ceil(m / (T - t)) per step; [M] "SPRINT 加速技术": k = ceil(remaining / steps_left), batch acceptance).
  * For each still-masked position r (n_rows of them; row r is flat position row_pos[r] = b * L + i of the
- * logical rows): z = logits[r] (with cfg: z = zu + cfg_scale * (zc - zu) in fp32, zc = logits[r],
- * zu = logits[n_rows + r]); candidate = vocab_offset + lowest argmax of z; c = 1 / sum_v exp(z_v - max z).
+ * logical rows): z = logits[r]; with cfg 1 z = zu + cfg_scale * (zc - zu) in fp32, zc = logits[r],
+ * zu = logits[n_rows + r] ([M] text-to-image usage, cfg_scale); with cfg 2, editing guidance ([M] note under
+ * "SPRINT 加速技术": three-way guidance through cfg_text_scale and cfg_image_scale; formula not printed, plain
+ * reading) z = a + cfg_scale * (zc - zi), a = zu + cfg_image_scale * (zi - zu), each operation rounded to fp32 in
+ * that order, zi = logits[n_rows + r] (image only), zu = logits[2 n_rows + r]; candidate = vocab_offset + lowest
+ * argmax of z; c = 1 / sum_v exp(z_v - max z).
  * Per logical row b with m masked positions: k_t positions by the ranking score descending (c itself by default;
  * rounded to fp32; equal values -> lower position) get their
- * candidate written to tokens and their mask cleared; with cfg the uncond row b + B gets the same update.
+ * candidate written to tokens and their mask cleared; with cfg the guidance rows b + g * B (g = 1 .. cfg) get the
+ * same update.
  *   logits [n_rows * (1 + cfg), V] in the storage type; row_pos [>= n_rows] int32: the still-masked flat
  *   positions of the logical rows in increasing order (row r of the logits belongs to the r-th masked position;
  *   every masked position must be listed, otherwise the results for the logical row are undefined);
@@ -276,6 +281,7 @@ typedef struct {
   int32_t vocab_offset;
   int32_t dtype;
   int32_t score;     /* DLLM_SCORE_*: the ranking of the positions */
+  float cfg_image_scale;   /* cfg 2: the image scale of the editing guidance (cfg_scale is the text scale) */
 } dllm_unmask_desc;
 DLLM_API int dllm_unmask(const dllm_unmask_desc* desc, const void* logits, const int32_t* row_pos, const int32_t* n_rows_dev,
                 int32_t* tokens, uint8_t* mask, int32_t* sel, int32_t* nsel, float* conf, int32_t* remaining,
@@ -339,7 +345,8 @@ typedef struct {
 
 /* Decoding state of one block (device pointers except the sizes). */
 typedef struct {
-  int32_t B;         /* batch rows (with cfg: B/2 conditional rows then B/2 unconditional rows) */
+  int32_t B;         /* batch rows (cfg 1: B/2 conditional rows then B/2 unconditional rows; cfg 2: B/3 rows
+                        conditioned on instruction and image, B/3 on the image only, B/3 unconditional) */
   int32_t L;         /* block length (<= 32) */
   int32_t P;         /* clean positions in the cache before this block (the block sits at [P, P + L)) */
   int32_t cap;       /* rows per (row, kv head) of the full caches, >= P + L */
@@ -357,7 +364,8 @@ typedef struct {
   int32_t mode;         /* DLLM_UNMASK_FIXED or DLLM_UNMASK_THRESHOLD */
   float tau;
   int32_t k_max;
-  int32_t cfg;          /* 1: rows pair as (b, b + B/2) = (cond, uncond) */
+  int32_t cfg;          /* 1: rows pair as (b, b + B/2) = (cond, uncond); 2 (editing guidance, no SPRINT): rows
+                           (b, b + B/3, b + 2B/3) = (instruction and image, image only, uncond) */
   float cfg_scale;
   int32_t vocab_offset; /* LM-head rows [vocab_offset, vocab_offset + vocab_len) are scored */
   int32_t vocab_len;    /* 0 = V */
@@ -374,6 +382,7 @@ typedef struct {
   int32_t score;      /* DLLM_SCORE_*: the ranking of the still-masked positions */
   float sprint_alpha;   /* SPRINT importance mix (1: key norm alone; needs state->prefix_conf otherwise) */
   int32_t n_keep_img;   /* with state->prefix_modality: image positions among the n_keep kept */
+  float cfg_image_scale; /* cfg 2: the image scale of the editing guidance (cfg_scale is the text scale) */
 } dllm_step_params;
 
 /*

@@ -75,7 +75,7 @@ def check_unmask(u, conf, nsel, sel, tokens, mask, Bl, cfg):
     """Library unmask outputs (numpy) against the oracle's dict u: confidences within u["conf_rtol"] at masked
     positions; for every logical row whose decision is not a near-tie (u["tie_rank"], u["tie_tau"]) the count,
     the chosen positions in rank order and the mask exactly, and the written tokens exactly except where the
-    candidate itself is a near-tie (u["tie_cand"]); with cfg the unconditional twin rows too."""
+    candidate itself is a near-tie (u["tie_cand"]); with cfg (1 or 2) the guidance rows b + g * Bl too."""
     m_ = u["conf"] > 0
     err = np.abs(conf.astype(np.float64) - u["conf"])
     assert np.all(err[m_] <= u["conf_rtol"][m_] * u["conf"][m_] + 1e-12), "confidences differ"
@@ -87,6 +87,6 @@ def check_unmask(u, conf, nsel, sel, tokens, mask, Bl, cfg):
         assert np.array_equal(mask[b], u["mask"][b]), f"row {b}: mask"
         ok = ~u["tie_cand"][b]
         assert np.array_equal(tokens[b][ok], u["tokens"][b][ok]), f"row {b}: tokens"
-        if cfg:
-            assert np.array_equal(mask[b + Bl], u["mask"][b + Bl])
-            assert np.array_equal(tokens[b + Bl][ok], u["tokens"][b + Bl][ok])
+        for g in range(1, 1 + int(cfg)):
+            assert np.array_equal(mask[b + g * Bl], u["mask"][b + g * Bl]), f"row {b} group {g}: mask"
+            assert np.array_equal(tokens[b + g * Bl][ok], u["tokens"][b + g * Bl][ok]), f"row {b} group {g}: tokens"

@@ -142,6 +142,34 @@ def test_unmask_rejects_bad_arguments(lib):
     assert lib.dllm_unmask(C.byref(u), *([FAKE] * 10), FAKE, 1 << 30, None) == bd.ERR_SHAPE   # L > 32
     u.L, u.max_rows, u.t = 32, 32, 8
     assert lib.dllm_unmask(C.byref(u), *([FAKE] * 10), FAKE, 1 << 30, None) == bd.ERR_INVALID_ARG  # t >= T_s
+    u.t, u.cfg = 0, 3                    # guidance modes are 0, 1 and 2
+    assert lib.dllm_unmask(C.byref(u), *([FAKE] * 10), FAKE, 1 << 30, None) == bd.ERR_INVALID_ARG
+
+
+def test_step_checks_guidance_groups(lib):
+    """Editing guidance (cfg 2) needs a multiple of three rows and runs without SPRINT (the plain decode on the full
+    caches); two-way guidance an even number of rows; other modes are refused. Host-side checks only."""
+    layers = (bd.Layer * 1)()
+    for name in ("attn_norm", "w_qkv", "w_o", "ffn_norm", "w_router", "router_bias", "w_gu", "w_down",
+                 "w_gu_shared", "w_down_shared", "k_cache", "v_cache", "k_thin", "v_thin", "keep_pos"):
+        setattr(layers[0], name, FAKE)
+    m = bd.Model(1, 2048, 16, 4, 128, 256, 8, 512, 157184, bd.BF16, 1e-6, 1e4, 0, FAKE, FAKE, FAKE, layers)
+    st = bd.State(3, 32, 1024, 1056, 544, FAKE, FAKE)
+    p = bd.StepParams(0, 8, 0, 0.9, 8, 2, 4.0, 0, 0, 0, 0, 0, 0, FAKE, FAKE, FAKE, FAKE, 0, 1.0, 0, 1.5)
+    size = lambda: lib.dllm_denoise_step_workspace_size(C.byref(m), C.byref(st), C.byref(p))
+    assert size() > 0
+    st.B = 4
+    assert size() == 0 and lib.dllm_denoise_step(C.byref(m), C.byref(st), C.byref(p), FAKE, 1 << 40, None) == bd.ERR_SHAPE
+    p.cfg = 1
+    assert size() > 0
+    st.B = 3
+    assert size() == 0
+    p.cfg = 3
+    assert lib.dllm_denoise_step(C.byref(m), C.byref(st), C.byref(p), FAKE, 1 << 40, None) == bd.ERR_INVALID_ARG
+    p.cfg, p.sprint, p.n_keep = 2, 1, 512
+    assert lib.dllm_denoise_step(C.byref(m), C.byref(st), C.byref(p), FAKE, 1 << 40, None) == bd.ERR_UNSUPPORTED
+    p.cfg = 0
+    assert size() > 0
 
 
 def test_retain_rejects_bad_arguments(lib):

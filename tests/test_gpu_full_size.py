@@ -15,7 +15,7 @@ import torch
 
 from block_diffusion_moe_dllm_b200 import binding as bd
 from block_diffusion_moe_dllm_b200 import synth
-from block_diffusion_moe_dllm_b200.configs import PREFILL, T2I, THINKING, UNDERSTANDING
+from block_diffusion_moe_dllm_b200.configs import EDIT, PREFILL, T2I, THINKING, UNDERSTANDING
 from block_diffusion_moe_dllm_b200.engine import DenoiseEngine
 from oracle import dllm_oracle as O
 from _util import ROUTE_TIE, assert_close, assignment_tables, check_unmask, random_assignments, same_routing, to64
@@ -168,13 +168,13 @@ def test_full_lm_head_understanding():
 
 
 # ------------------------------------------------------------------------------------------------ unmask
-@pytest.mark.parametrize("w", [T2I, THINKING, UNDERSTANDING], ids=["t2i", "thinking", "understanding"])
+@pytest.mark.parametrize("w", [T2I, EDIT, THINKING, UNDERSTANDING], ids=["t2i", "edit", "thinking", "understanding"])
 def test_full_unmask(w):
-    Bl = w.B // 2 if w.cfg else w.B
+    Bl = w.B // (1 + w.cfg)
     L, V = w.L, w.vlen
     n = Bl * L
     std = 6.0 if w.mode == 1 else 1.0
-    logits = synth.normal(((2 if w.cfg else 1) * n, V), std, 26, "fu_z", DEV)
+    logits = synth.normal(((1 + w.cfg) * n, V), std, 26, "fu_z", DEV)
     mask = np.ones((w.B, L), dtype=np.uint8)
     tokens = np.full((w.B, L), w.mask_id, dtype=np.int32)
     row_pos = np.arange(n, dtype=np.int32)
@@ -185,18 +185,19 @@ def test_full_unmask(w):
     rem = torch.empty(1, dtype=torch.int32, device=DEV)
     bd.unmask(logits, torch.from_numpy(row_pos).to(DEV), torch.tensor([n], dtype=torch.int32, device=DEV), dt, dm,
               sel, nsel, conf, rem, Bl, L, V, n, 0, w.T_s, bd.BF16, mode=w.mode, tau=w.tau, k_max=w.k_max, cfg=w.cfg,
-              cfg_scale=w.cfg_scale, vocab_offset=w.vocab_offset)
+              cfg_scale=w.cfg_scale, vocab_offset=w.vocab_offset, cfg_image_scale=w.cfg_image_scale)
     torch.cuda.synchronize()
     zl = to64(logits)
     u = O.unmask(zl[:n], row_pos, tokens, mask, 0, w.T_s, w.mode, float(np.float32(w.tau)), w.k_max,
-                 w.vocab_offset, z_uncond=zl[n:] if w.cfg else None, cfg_scale=float(np.float32(w.cfg_scale)))
+                 w.vocab_offset, z_uncond=zl[w.cfg * n:] if w.cfg else None, cfg_scale=float(np.float32(w.cfg_scale)),
+                 z_image=zl[n:2 * n] if w.cfg == 2 else None, cfg_image_scale=float(np.float32(w.cfg_image_scale)))
     check_unmask(u, conf.cpu().numpy(), nsel.cpu().numpy(), sel.cpu().numpy(), dt.cpu().numpy(), dm.cpu().numpy(),
                  Bl, w.cfg)
 
 
 # ------------------------------------------------------------------------------------------------ whole pass
 def _check_pass_properties(w, eng, tok0, mask0, t):
-    Bl = w.B // 2 if w.cfg else w.B
+    Bl = w.B // (1 + w.cfg)
     conf = eng.conf.cpu().numpy().astype(np.float64)
     nsel = eng.nsel.cpu().numpy()
     tok = eng.tokens.cpu().numpy()
@@ -223,12 +224,12 @@ def _check_pass_properties(w, eng, tok0, mask0, t):
             assert c[newly].min() >= c[still].max()
         assert np.all((tok[b][newly] >= w.vocab_offset) & (tok[b][newly] < w.vocab_offset + w.vlen))
         assert np.array_equal(tok[b][~newly], t0[b][~newly])
-        if w.cfg:
-            assert np.array_equal(tok[b + Bl], tok[b]) and np.array_equal(msk[b + Bl], msk[b])
+        for g in range(1, 1 + w.cfg):
+            assert np.array_equal(tok[b + g * Bl], tok[b]) and np.array_equal(msk[b + g * Bl], msk[b])
     assert eng.remaining.item() == int(msk[:Bl].sum())
 
 
-@pytest.mark.parametrize("w", [T2I, THINKING, UNDERSTANDING], ids=["t2i", "thinking", "understanding"])
+@pytest.mark.parametrize("w", [T2I, EDIT, THINKING, UNDERSTANDING], ids=["t2i", "edit", "thinking", "understanding"])
 def test_full_denoise_pass_properties(w):
     wt = synth.make_weights(w, DEV)
     caches = synth.make_prefix_cache(w, DEV)
@@ -240,7 +241,7 @@ def test_full_denoise_pass_properties(w):
         eng.step(0)
         torch.cuda.synchronize()
         assert bd.status_check(eng.ws) == bd.OK
-        n = int(mask0[: (w.B // 2 if w.cfg else w.B)].sum().item())
+        n = int(mask0[: w.B // (1 + w.cfg)].sum().item())
         lg = eng.logits(n)
         assert torch.isfinite(lg.float()).all()
         results.append((eng.tokens.clone(), eng.mask.clone(), eng.conf.clone(), lg.clone()))

@@ -511,21 +511,27 @@ def test_prefix_retain_mixed_importance_and_modality(B, P, n_keep, n_img, n_keep
 
 
 # ------------------------------------------------------------------------------------------------ unmask
-def _unmask_case(B, L, V, masked_frac, t, T_s, mode, std, cfg=False, scale=2.0, tau=0.9, k_max=8, voff=0,
-                 dtype="bf16", seed=0, count_excess=None, score=0):
-    """count_excess: the call's row capacity is exactly the masked count n and the device count says
-    n + count_excess; the library must treat it as n (the logits hold n rows per half)."""
+def _unmask_case(B, L, V, masked_frac, t, T_s, mode, std, cfg=0, scale=2.0, tau=0.9, k_max=8, voff=0,
+                 dtype="bf16", seed=0, count_excess=None, score=0, iscale=1.0, zi_near=None):
+    """cfg 0, 1 (two-way) or 2 (editing: rows per position (full, image only, unconditional)). count_excess: the
+    call's row capacity is exactly the masked count n and the device count says n + count_excess; the library must
+    treat it as n (the logits hold n rows per group). zi_near: with cfg 2, the image-only rows are the full rows
+    plus noise of this size (close rows, as a real model's are, so that the text term cancels to a small
+    difference)."""
+    cfg = int(cfg)
     g = np.random.default_rng(seed)
-    Btot = 2 * B if cfg else B
+    Btot = (1 + cfg) * B
     mask = (g.uniform(size=(B, L)) < masked_frac).astype(np.uint8)
     mask[0, 0] = 1
-    if cfg:
-        mask = np.concatenate([mask, mask])
+    mask = np.concatenate([mask] * (1 + cfg))
     tokens = np.where(mask == 1, V - 1, g.integers(0, V, (Btot, L))).astype(np.int32)
     row_pos = np.nonzero(mask[:B].reshape(-1))[0].astype(np.int32)
     n = len(row_pos)
     t_dt = _tdt(dtype)
-    logits = synth.normal(((2 if cfg else 1) * n, V), std, seed, f"ul{V}", DEV, t_dt)
+    logits = synth.normal(((1 + cfg) * n, V), std, seed, f"ul{V}", DEV, t_dt)
+    if cfg == 2 and zi_near is not None:
+        noise = synth.normal((n, V), zi_near, seed, f"ul{V}_zi", DEV, torch.float32)
+        logits[n:2 * n] = (logits[:n].float() + noise).to(t_dt)
     dm = torch.from_numpy(mask).to(DEV)
     dt_ = torch.from_numpy(tokens).to(DEV)
     sel = torch.empty((B, L), dtype=torch.int32, device=DEV)
@@ -536,11 +542,12 @@ def _unmask_case(B, L, V, masked_frac, t, T_s, mode, std, cfg=False, scale=2.0, 
     nd = torch.tensor([n if count_excess is None else n + count_excess], dtype=torch.int32, device=DEV)
     cap = B * L if count_excess is None else n
     bd.unmask(logits, rp, nd, dt_, dm, sel, nsel, conf, rem, B, L, V, cap, t, T_s, DT[dtype], mode=mode, tau=tau,
-              k_max=k_max, cfg=int(cfg), cfg_scale=scale, vocab_offset=voff, score=score)
+              k_max=k_max, cfg=cfg, cfg_scale=scale, vocab_offset=voff, score=score, cfg_image_scale=iscale)
     torch.cuda.synchronize()
     zl = to64(logits)
     u = O.unmask(zl[:n], row_pos, tokens, mask, t, T_s, mode, float(np.float32(tau)), k_max, voff,
-                 z_uncond=zl[n:] if cfg else None, cfg_scale=float(np.float32(scale)), score=O.SCORES[score])
+                 z_uncond=zl[cfg * n:] if cfg else None, cfg_scale=float(np.float32(scale)), score=O.SCORES[score],
+                 z_image=zl[n:2 * n] if cfg == 2 else None, cfg_image_scale=float(np.float32(iscale)))
     check_unmask(u, conf.cpu().numpy(), nsel.cpu().numpy(), sel.cpu().numpy(), dt_.cpu().numpy(), dm.cpu().numpy(),
                  B, cfg)
     assert rem.item() == int(dm[:B].sum().item())
@@ -566,6 +573,26 @@ def test_unmask_cfg_image_slice():
     _unmask_case(1, 32, 16384, 0.7, 2, 8, bd.FIXED, 1.0, cfg=True, scale=2.0, voff=157184 - 16384, seed=13)
 
 
+@pytest.mark.parametrize("scale,iscale,near", [(4.0, 1.0, 0.3), (7.5, 1.5, 0.1), (4.0, 1.0, None)])
+def test_unmask_editing_guidance_image_slice(scale, iscale, near):
+    """Editing guidance (three rows per position) on the image-token slice: confidences, counts, chosen positions
+    and the tokens written to all three row groups against the oracle, at the editing example's text scale 4.0 and
+    a larger pair, with image-only rows close to the full rows and unrelated ones."""
+    _unmask_case(2, 32, 16384, 0.7, 2, 8, bd.FIXED, 1.0, cfg=2, scale=scale, iscale=iscale,
+                 voff=157184 - 16384, seed=17, zi_near=near)
+
+
+@pytest.mark.parametrize("score", [0, 1, 2], ids=["low_confidence", "top_k_margin", "neg_entropy"])
+def test_unmask_editing_guidance_scores_full_vocab(score):
+    """Editing guidance through each ranking's reduction (the largest-probability one and the extended one of the
+    other scores) over the full vocabulary, whose 157184 entries are not a multiple of the vector chunk, with
+    threshold acceptance; fp32 logits check the scalar tail of the same kernels."""
+    _unmask_case(1, 32, 157184, 1.0, 1, 8, 1, 3.0, cfg=2, scale=4.0, iscale=1.25, seed=50 + score, score=score,
+                 zi_near=0.5)
+    _unmask_case(2, 16, 1001, 0.8, 0, 4, bd.FIXED, 1.0, cfg=2, scale=2.0, iscale=0.5, seed=53 + score, score=score,
+                 dtype="f32")
+
+
 def test_unmask_last_step_takes_all():
     u = _unmask_case(3, 32, 4096, 0.3, 7, 8, bd.FIXED, 1.0, seed=14)
     assert np.all(u["mask"] == 0)
@@ -589,7 +616,7 @@ def test_unmask_position_scores_cfg_full_vocab(score):
     _unmask_case(1, 32, 157184, 1.0, 1, 8, 1, 3.0, cfg=True, scale=2.0, seed=45 + score, score=score)
 
 
-@pytest.mark.parametrize("cfg", [False, True])
+@pytest.mark.parametrize("cfg", [0, 1, 2])
 def test_unmask_device_count_above_capacity_is_clamped(cfg):
     """A device row count above the call's max_rows is read as max_rows: no partial or logit row beyond the
     capacity is touched, and the result is that of the true count."""

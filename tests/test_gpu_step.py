@@ -77,12 +77,12 @@ def _check_pass(w, eng, f, dtype):
     assert ok.sum() >= 0.5 * len(ok), "too many routing near-ties for a meaningful comparison"
     assert_close(x[ok], f["x"].reshape(-1, w.H)[ok], dtype, "hidden state after the last layer", ulps=2)
     lg = to64(eng.logits(n))
-    Bl = w.B // 2 if w.cfg else w.B
-    rows = list(f["row_pos"]) + ([p + Bl * w.L for p in f["row_pos"]] if w.cfg else [])
+    groups = 1 + w.cfg
+    Bl = w.B // groups
+    rows = [p + g * Bl * w.L for g in range(groups) for p in f["row_pos"]]
     okr = ~flag[np.asarray(rows, dtype=np.int64)]
-    if w.cfg:  # a guided row needs both of its rows clean
-        okr = okr[:n] & okr[n:]
-        okr = np.concatenate([okr, okr])
+    if w.cfg:  # a guided row needs all of its rows clean
+        okr = np.tile(okr.reshape(groups, n).all(axis=0), groups)
     assert_close(lg[okr], f["logits"][okr], dtype, "logits of the masked rows", ulps=2,
                  scale=max(1.0, w.lm_std / 0.02))
     return flag
@@ -98,26 +98,36 @@ def _score_shift(score, r, c, dz):
     return 2.0 * dz * (abs(r) + 1.0)
 
 
+def _guidance_gain(w):
+    """How much guidance can scale a common difference dz of its rows' logits: z = zu + s (zc - zu) moves by at
+    most (|1 - s| + |s|) dz; z = zu (1 - s_i) + zi (s_i - s_t) + zc s_t by at most (|1 - s_i| + |s_i - s_t| +
+    |s_t|) dz."""
+    if w.cfg == 2:
+        return abs(1.0 - w.cfg_image_scale) + abs(w.cfg_image_scale - w.cfg_scale) + abs(w.cfg_scale)
+    if w.cfg:
+        return abs(1.0 - w.cfg_scale) + abs(w.cfg_scale)
+    return 1.0
+
+
 def _decisions_agree(w, u_or, eng, flag):
     """Compare the unmask decisions where the oracle's choice is not a near-tie (ranking by the workload's score,
     threshold on the largest probability). For the margin and entropy scores the near-tie band also covers what
-    the observed difference between the two sides' logits (dz, largest over the scored rows; guidance scales it by
-    1 + 2 s) can move the scores by."""
-    Bl = w.B // 2 if w.cfg else w.B
+    the observed difference between the two sides' logits (dz, largest over the scored rows, scaled by the
+    guidance) can move the scores by."""
+    Bl = w.B // (1 + w.cfg)
     dz = 0.0
     if w.score:
         f = u_or["forward"]
         n = len(f["row_pos"])
         dz = float(np.max(np.abs(to64(eng.logits(n)) - f["logits"]))) if n else 0.0
-        if w.cfg:
-            dz *= 1.0 + 2.0 * abs(w.cfg_scale)
+        dz *= _guidance_gain(w)
     g_mask = eng.mask.cpu().numpy()
     g_nsel = eng.nsel.cpu().numpy()
     clean = True
     for b in range(Bl):
         c = u_or["conf"][b]
         rk = u_or["rank"][b][c > 0]
-        row_flag = flag[b * w.L:(b + 1) * w.L].any() or (w.cfg and flag[(b + Bl) * w.L:(b + Bl + 1) * w.L].any())
+        row_flag = any(flag[(b + g * Bl) * w.L:(b + g * Bl + 1) * w.L].any() for g in range(1 + w.cfg))
         order = np.argsort(-rk, kind="stable")
         ranked, c_ranked = rk[order], c[c > 0][order]
         k = u_or["nsel"][b]
@@ -140,10 +150,11 @@ def _decisions_agree(w, u_or, eng, flag):
 
 def _check_candidates(w, eng, u_or, f, flag):
     """Candidate tokens written this step agree wherever the oracle's top-2 logit gap is clear."""
-    Bl = w.B // 2 if w.cfg else w.B
     n = len(f["row_pos"])
     z = f["logits"][:n]
-    if w.cfg:
+    if w.cfg == 2:
+        z = O.cfg3_combine(z, f["logits"][n:2 * n], f["logits"][2 * n:], w.cfg_scale, w.cfg_image_scale)
+    elif w.cfg:
         z = O.cfg_combine(z, f["logits"][n:], w.cfg_scale)
     top2 = np.sort(z, axis=1)[:, -2:]
     clear = (top2[:, 1] - top2[:, 0]) > 0.05
@@ -201,6 +212,18 @@ def test_step_small_bf16_partly_masked_mid_block():
 def test_step_small_bf16_cfg_image_slice():
     w = scaled(SMALL, B=2, cfg=1, cfg_scale=2.0, vocab_offset=1024 - 256, vocab_len=256)
     _one_pass(w, seed=3)
+
+
+def test_step_small_bf16_editing_guidance():
+    """Editing guidance: three rows per position (instruction and image, image only, unconditional), the
+    image-token slice of the head, text scale 4 and image scale 1.5; the chosen tokens land in all three groups."""
+    w = scaled(SMALL, name="small-bf16-edit", B=3, cfg=2, cfg_scale=4.0, cfg_image_scale=1.5,
+               vocab_offset=1024 - 256, vocab_len=256)
+    eng, u = _one_pass(w, seed=10)
+    g_tok, g_mask = eng.tokens.cpu().numpy(), eng.mask.cpu().numpy()
+    assert np.array_equal(g_mask[0], g_mask[1]) and np.array_equal(g_mask[0], g_mask[2])
+    assert np.array_equal(g_tok[0], g_tok[1]) and np.array_equal(g_tok[0], g_tok[2])
+    assert int(eng.nsel[0].item()) > 0
 
 
 def test_step_small_bf16_sprint():

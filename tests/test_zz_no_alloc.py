@@ -23,12 +23,11 @@ def _inputs(B, L, V, seed, cfg):
     g = np.random.default_rng(seed)
     mask = (g.uniform(size=(B, L)) < 0.75).astype(np.uint8)
     mask[:, 0] = 1
-    if cfg:
-        mask = np.concatenate([mask, mask])
+    mask = np.concatenate([mask] * (1 + cfg))   # every guidance row group shares the pattern
     tokens = np.where(mask == 1, V - 1, g.integers(0, V, mask.shape)).astype(np.int32)
     row_pos = np.nonzero(mask[:B].reshape(-1))[0].astype(np.int32)
     n = len(row_pos)
-    logits = synth.normal(((2 if cfg else 1) * n, V), 3.0, seed, f"noalloc{V}", DEV)
+    logits = synth.normal(((1 + cfg) * n, V), 3.0, seed, f"noalloc{V}", DEV)
     rp = torch.from_numpy(np.concatenate([row_pos, np.zeros(B * L - n, np.int32)])).to(DEV)
     nd = torch.tensor([n], dtype=torch.int32, device=DEV)
     return logits, rp, nd, torch.from_numpy(tokens).to(DEV), torch.from_numpy(mask).to(DEV)
@@ -40,10 +39,11 @@ def _outputs(B, L):
 
 
 @pytest.mark.parametrize("B,L,V,t,T_s,mode,cfg", [(16, 32, 157184, 0, 32, bd.THRESHOLD, 0),
-                                                  (2, 32, 16384, 1, 8, bd.FIXED, 1)])
+                                                  (2, 32, 16384, 1, 8, bd.FIXED, 1),
+                                                  (2, 32, 16384, 1, 8, bd.FIXED, 2)])
 def test_unmask_noalloc_matches_workspace_version(B, L, V, t, T_s, mode, cfg):
     lib = bd.load()
-    desc = bd.UnmaskDesc(B, L, V, B * L, t, T_s, mode, 0.9, 8, cfg, 2.0, 0, bd.BF16)
+    desc = bd.UnmaskDesc(B, L, V, B * L, t, T_s, mode, 0.9, 8, cfg, 2.0, 0, bd.BF16, 0, 1.5)
     need = lib.dllm_unmask_workspace_size(C.byref(desc))
     ws = bd.Workspace(need, DEV)
     stream = bd.stream_handle()

@@ -225,8 +225,9 @@ DLLM_API size_t dllm_moe_route_workspace_size(const dllm_route_desc* desc);
  * of each expert are the stated layer configuration of this library's workloads). Routed experts plus shared
  * expert, added to the residual:
  *   x[t] <- x[t] + shared(h[t]) + sum_j gates[t, j] * expert_{ids[t, j]}(h[t]),
- * expert_e(v) = W_down[e] (silu(W_gate[e] v) * (W_up[e] v)) (SwiGLU; the SwiGLU activation is stored in the
- * storage type), summed in slot order j = 0..k-1 in fp32 and rounded once.
+ * expert_e(v) = W_down[e] (silu(W_gate[e] v) * (W_up[e] v)) (SwiGLU; the SwiGLU activation and each expert's
+ * output row, accumulated in fp32, are stored in the storage type), the shared row then the gate-weighted rows
+ * summed onto the residual in slot order j = 0..k-1 in fp32 and rounded once.
  *   h [Tk, H]; w_gu [E, 2I, H] (rows [0, I) gate, [I, 2I) up); w_down [E, H, I]; w_gu_shared [2I, H] and
  *   w_down_shared [H, I] (both NULL: no shared expert); counts/offsets/perm/inv/gates as produced by
  *   dllm_moe_route; x_inout [Tk, H].

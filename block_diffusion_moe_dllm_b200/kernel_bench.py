@@ -168,7 +168,7 @@ def bench_experts(w: Workload, reps, dev, stream, weights=None, routing="router"
 def bench_expert_gemms(w: Workload, reps, dev, stream, weights=None, routing="router"):
     """The two grouped expert GEMMs alone (dllm_grouped_gemm, the kernels the expert call launches), at the
     workload's routed token rows (router output of random activations) plus the shared expert's rows: gate|up with
-    the SwiGLU epilogue, then down with fp32 rows."""
+    the SwiGLU epilogue, then down with rows in the storage type (bf16), as the expert call stores them."""
     rows = w.B * w.L
     lw = weights["layers"][0] if weights else synth.make_weights(
         Workload(**{**w.__dict__, "n_layers": 1, "V": 128}), dev)["layers"][0]
@@ -190,17 +190,17 @@ def bench_expert_gemms(w: Workload, reps, dev, stream, weights=None, routing="ro
     hint = min(rows, max(128, 4 * ((rows * w.k + w.E - 1) // w.E)))   # the step's N-tile hint for expert GEMMs
     xp = synth.normal((n, w.H), 1.0, 6, "kb_xp", dev)
     act = torch.empty((n, w.I), dtype=torch.bfloat16, device=dev)
-    y = torch.empty((n, w.H), dtype=torch.float32, device=dev)
+    y = torch.empty((n, w.H), dtype=torch.bfloat16, device=dev)
     f8 = "w_gu_scale" in lw
     sc = (lambda name: lw[name + "_scale"] if f8 else None)
     t1 = timed(lambda: bd.grouped_gemm(xp, lw["w_gu"], lw["w_gu_shared"], counts, offsets, act, w.E, n, w.H, w.I,
                                        bd.BF16, swiglu=1, extra_rows=rows, max_rows_hint=hint, w_scale=sc("w_gu"),
                                        w_extra_scale=sc("w_gu_shared"), ws=ws), reps, stream)
     t2 = timed(lambda: bd.grouped_gemm(act, lw["w_down"], lw["w_down_shared"], counts, offsets, y, w.E, n, w.I, w.H,
-                                       bd.BF16, extra_rows=rows, max_rows_hint=hint, y_f32=1, w_scale=sc("w_down"),
+                                       bd.BF16, extra_rows=rows, max_rows_hint=hint, y_f32=0, w_scale=sc("w_down"),
                                        w_extra_scale=sc("w_down_shared"), ws=ws), reps, stream)
     b1 = (active + 1) * 2 * w.I * w.H * wbytes(w) + n * w.H * 2 + n * w.I * 2
-    b2 = (active + 1) * w.H * w.I * wbytes(w) + n * w.I * 2 + n * w.H * 4
+    b2 = (active + 1) * w.H * w.I * wbytes(w) + n * w.I * 2 + n * w.H * 2
     f1, f2 = 2.0 * n * 2 * w.I * w.H, 2.0 * n * w.H * w.I
     return [_result("gemm_tc_kernel[experts_swiglu]", t1, b1, _flops({"active_experts": active, "rows": n}, f1, t1)),
             _result("gemm_tc_kernel[experts_down]", t2, b2, _flops({"active_experts": active, "rows": n}, f2, t2))]

@@ -530,20 +530,24 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
   __syncthreads();
   // Weights are never written by the kernels ahead of this one: the first tile's first weight stages can stream
   // in before the dependency wait (their transaction bytes are expected now; the arrival, with the activation
-  // bytes, comes in the producer loop). Every lane of warp 0 derives the same count.
+  // bytes, comes in the producer loop). Every lane of warp 0 derives the same count. Dense launches whose row count
+  // is fixed on the host know their first tile's weight tile here (tile t0 -> m-tile t0 / N tiles per weight tile);
+  // measured on a 20-layer understanding block (the 512-row QKV, output and router-logit projections): 141.2 ->
+  // 140.4 ms.
   const int kblocks = p.K / SBK;
   int npf = 0;
   if (p.prefetch_w) {
     const int t0 = p.ksplit > 1 ? (int)blockIdx.y : (int)blockIdx.x;
     const int ks0 = p.ksplit > 1 ? (int)blockIdx.x : 0;
     const int kb0 = ks0 * kblocks / p.ksplit, kb1 = (ks0 + 1) * kblocks / p.ksplit;
-    if (t0 < p.m_tiles) npf = min(STAGES, kb1 - kb0);
+    const int ntl = max(1, (p.host_cnt + BN - 1) / BN);   // N tiles per weight tile (row count fixed on the host)
+    if (t0 < p.m_tiles * ntl) npf = min(STAGES, kb1 - kb0);
     if (warp == 0 && npf > 0 && tc::elect_one()) {
       tc::prefetch_tmap(&tmap_w);
       const uint64_t pol_w = tc::policy_evict_first();
       for (int i = 0; i < npf; ++i) {
         tc::mbar_expect_tx(&sm.full[i], W_TX);
-        tc::tma_load_2d(stages + i * STAGE_BYTES, &tmap_w, (kb0 + i) * SBK, t0 * 128, &sm.full[i], pol_w);
+        tc::tma_load_2d(stages + i * STAGE_BYTES, &tmap_w, (kb0 + i) * SBK, (t0 / ntl) * 128, &sm.full[i], pol_w);
       }
     }
   }
@@ -1497,7 +1501,7 @@ int gemm_bf16_tc(const GemmArgs& a, cudaStream_t s) {
   // grouped launches of single-CTA tiles take their tiles from the work counter (the CTA pair kernel keeps its
   // static schedule)
   kp.work_ctr = ((a.swiglu || a.n_dev || a.has_extra) && ks == 1) ? a.work_ctr : nullptr;
-  kp.prefetch_w = (!a.swiglu && !a.n_dev && !a.has_extra && a.host_cnt <= (ks > 1 ? 32 : bn)) ? 1 : 0;
+  kp.prefetch_w = (!a.swiglu && !a.n_dev && !a.has_extra && (a.host_cnt <= (ks > 1 ? 32 : bn) || !a.cnt_dev)) ? 1 : 0;
   int st2;
   if (f8) {   // single-CTA tiles, no split-K (the weight-streaming shapes FP8 weights serve)
     // (weight-code ring, activation ring): the activation ring also has to cover a load from L2 plus the wait for

@@ -469,12 +469,17 @@ def test_finished_pass_costs_only_its_launches():
     assert dead < 0.5 * live, f"finished pass {dead * 1e3:.0f} us vs live pass {live * 1e3:.0f} us"
 
 
-@pytest.mark.parametrize("early", [False, True], ids=["fixed-schedule", "finishes-at-first-pass"])
-def test_block_graph_matches_host_driven_block(early):
+@pytest.mark.parametrize("early,edit", [(False, False), (True, False), (False, True)],
+                         ids=["fixed-schedule", "finishes-at-first-pass", "editing-guidance"])
+def test_block_graph_matches_host_driven_block(early, edit):
     """dllm_block_graph_create captures a block (T_s passes, each inside a conditional node that runs it only while
     masked positions are left, then the commit pass). Launched from the same start it leaves the same tokens, mask,
-    caches and step outputs as the passes called one by one from the host, launched twice in a row."""
+    caches and step outputs as the passes called one by one from the host, launched twice in a row. With editing
+    guidance the three row groups end with the same tokens."""
     w = scaled(SMALL, name="small-bf16-graph", mode=1, tau=0.0, k_max=32, T_s=6) if early else SMALL
+    if edit:
+        w = scaled(SMALL, name="small-bf16-graph-edit", B=3, cfg=2, cfg_scale=4.0, cfg_image_scale=1.5,
+                   vocab_offset=1024 - 256, vocab_len=256)
     wt, caches, eng, _, _ = _setup(w, seed=43)
     tokens0, mask0 = eng.tokens.clone(), eng.mask.clone()
     caches0 = [(k.clone(), v.clone()) for k, v in caches]
@@ -498,4 +503,6 @@ def test_block_graph_matches_host_driven_block(early):
         if not early:     # with an early finish the graph skips passes whose step outputs the host loop rewrote
             assert torch.equal(eng.sel, want_sel[0]) and torch.equal(eng.nsel, want_sel[1])
         assert int(eng.remaining.item()) == 0 and int(eng.mask.sum().item()) == 0
+        if edit:
+            assert torch.equal(eng.tokens[0], eng.tokens[1]) and torch.equal(eng.tokens[0], eng.tokens[2])
     del g

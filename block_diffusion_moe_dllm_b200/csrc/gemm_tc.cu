@@ -187,6 +187,29 @@ __device__ __forceinline__ int work_tile(const Smem& sm, const KParams& p, int w
   return t;
 }
 
+// Wait for this thread's outstanding tcgen05.ld; the 32 registers are in-out operands, so no use of them can be
+// scheduled before the wait.
+__device__ __forceinline__ void tmem_wait_ld32(uint32_t* r) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]),
+                 "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+                 "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+               :
+               : "memory");
+}
+// 32 columns of this lane without the wait (valid after tmem_wait_ld32 on the same registers).
+__device__ __forceinline__ void tmem_ld32_issue(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+
 __device__ __forceinline__ float silu_f(float g) { return g / (1.0f + expf(-g)); }
 
 // Barrier over every thread of every CTA of the cluster (release / acquire on shared memory).
@@ -946,11 +969,16 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant
 // and accumulator ready (tfull) to the barriers of both CTAs; warps 2-5 of each CTA drain their TMEM half and arrive on the
 // leader's tempty (128 + 128 arrivals). Measured with the peer instead forwarding each landed stage to the leader
 // (a remote arrive after waiting on its own barrier): 2.5x slower, the extra hop stalling every stage.
+// The epilogue bounds this kernel at the prefill shape: with its stores left out (a timing build) the down expert
+// GEMM at 32768 tokens (K = 512, eight k-steps per tile) took 475 us instead of 937. Its chunks therefore run as a
+// pipeline: the next chunk's columns are loaded from TMEM while this one is staged and stored, and the staging
+// area is double-buffered, so a chunk needs one barrier instead of two (5 operand stages make room for it):
+// 937-955 -> 828-830 us for that GEMM, 1221 -> 1195 us for the SwiGLU GEMM, the 512-row LM head unchanged.
 constexpr int PAIR_BN = 256;
-constexpr int PAIR_STAGES = 6;
+constexpr int PAIR_STAGES = 5;
 constexpr int PAIR_B_BYTES = (PAIR_BN / 2) * BK * 2;
 constexpr int PAIR_STAGE_BYTES = A_BYTES + PAIR_B_BYTES;
-constexpr int PAIR_SMEM = 1024 + PAIR_STAGES * PAIR_STAGE_BYTES + STAGING_BYTES + (int)sizeof(Smem);
+constexpr int PAIR_SMEM = 1024 + PAIR_STAGES * PAIR_STAGE_BYTES + 2 * STAGING_BYTES + (int)sizeof(Smem);
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
 gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_w2,
@@ -960,7 +988,7 @@ gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_con
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = base;
   float* staging = reinterpret_cast<float*>(base + STAGES * PAIR_STAGE_BYTES);
-  Smem& sm = *reinterpret_cast<Smem*>(base + STAGES * PAIR_STAGE_BYTES + STAGING_BYTES);
+  Smem& sm = *reinterpret_cast<Smem*>(base + STAGES * PAIR_STAGE_BYTES + 2 * STAGING_BYTES);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -1136,7 +1164,7 @@ gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_con
     const int row = q * 32 + lane;
     const int etid = tid - 64;
     const uint32_t tempty0 = tc::mapa_u32(tc::smem_u32(&sm.tempty[0]), 0);
-    uint32_t tcount = 0;
+    uint32_t tcount = 0, chunk = 0;
     for (int t = pair; t < total; t += n_pairs, ++tcount) {
       int g, mp, n0, nval;
       decode_tile<PAIR_BN>(sm, m_pairs, t, g, mp, n0, nval);
@@ -1144,16 +1172,27 @@ gemm_tc_pair_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_con
       const uint32_t buf = tcount & 1, tph = (tcount >> 1) & 1;
       if (!wait_bar(&sm.tfull[buf], tph, abort_flag, p.status, ST_TIMEOUT_EPILOGUE)) break;
       tc::fence_after_sync();
-      for (int c0 = 0; c0 < nval; c0 += STAGE_COLS) {
-        float v[STAGE_COLS];
-        const uint32_t taddr = sm.tmem_base + ((uint32_t)(q * 32) << 16) + buf * PAIR_BN + c0;
-        tc::tmem_ld16(taddr, v);
-        tc::tmem_ld16(taddr + 16, v + 16);
-        tc::named_bar_sync(1, 128);
+      // the next chunk's columns are in flight while this one is staged and stored
+      const uint32_t tb = sm.tmem_base + ((uint32_t)(q * 32) << 16) + buf * PAIR_BN;
+      const int nch = (nval + STAGE_COLS - 1) / STAGE_COLS;
+      uint32_t ra[STAGE_COLS], rb[STAGE_COLS];
+      auto stage_store = [&](const uint32_t* r, int ci) {
+        float* st = staging + (chunk & 1) * (STAGING_BYTES / 4);
 #pragma unroll
-        for (int j = 0; j < STAGE_COLS; ++j) staging[j * 128 + row] = v[j];
+        for (int j = 0; j < STAGE_COLS; ++j) st[j * 128 + row] = __uint_as_float(r[j]);
         tc::named_bar_sync(1, 128);
-        epilogue_chunk<PAIR_BN>(p, staging, g, mt, n0, nval, c0, sm.grp_off[g], etid);
+        epilogue_chunk<PAIR_BN>(p, st, g, mt, n0, nval, ci * STAGE_COLS, sm.grp_off[g], etid);
+        ++chunk;
+      };
+      tmem_ld32_issue(tb, ra);
+      for (int ci = 0; ci < nch; ci += 2) {
+        tmem_wait_ld32(ra);
+        if (ci + 1 < nch) tmem_ld32_issue(tb + (ci + 1) * STAGE_COLS, rb);
+        stage_store(ra, ci);
+        if (ci + 1 >= nch) break;
+        tmem_wait_ld32(rb);
+        if (ci + 2 < nch) tmem_ld32_issue(tb + (ci + 2) * STAGE_COLS, ra);
+        stage_store(rb, ci + 1);
       }
       tc::fence_before_sync();
       tc::mbar_arrive_cluster(tempty0 + 8u * buf);

@@ -226,6 +226,16 @@ def test_step_small_bf16_editing_guidance():
     assert int(eng.nsel[0].item()) > 0
 
 
+def test_step_small_bf16_editing_guidance_threshold():
+    """Editing guidance with threshold acceptance on logits spread wide enough that confidences cross tau and the
+    cap binds: counts, chosen positions and tokens of all three groups against the oracle."""
+    w = scaled(SMALL, name="small-bf16-edit-thr", B=3, cfg=2, cfg_scale=4.0, cfg_image_scale=1.25, mode=1, tau=0.9,
+               k_max=8, T_s=16, lm_std=1.0)
+    eng, u = _one_pass(w, seed=11)
+    g_mask = eng.mask.cpu().numpy()
+    assert np.array_equal(g_mask[0], g_mask[1]) and np.array_equal(g_mask[0], g_mask[2])
+
+
 def test_step_small_bf16_sprint():
     w = scaled(SMALL, B=3, P=96, sprint=1, keep_ratio=0.5)
     _one_pass(w, seed=4)
